@@ -1,0 +1,407 @@
+"""Pins for the CPU oracle: each test ties one oracle function to something other
+than the oracle itself (a hand-worked example, a closed form, a special case that
+reduces to a library routine, an invariant, or exhaustive enumeration)."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3 encoder (OCP FP8 spec) -- pinned to the spec's fixed points and to
+# torch's own CPU cast.
+# ---------------------------------------------------------------------------
+def test_e4m3_spec_points():
+    pts = {0.0: 0x00, 1.0: 0x38, -2.0: 0xC0, 448.0: 0x7E, -448.0: 0xFE, 2.0 ** -9: 0x01,
+           2.0 ** -6: 0x08, 7 * 2.0 ** -9: 0x07, 1.125: 0x39, 240.0: 0x77, 0.5: 0x30}
+    for x, c in pts.items():
+        assert O.e4m3_encode(np.array([x], np.float32))[0] == c, x
+        assert O.e4m3_decode(np.array([c], np.uint8))[0] == x
+    # satfinite: finite overflow clamps to +-448
+    assert list(O.e4m3_encode(np.array([500.0, 1e30, -1e30, np.inf], np.float32))) == [0x7E, 0x7E, 0xFE, 0x7E]
+
+
+def test_e4m3_roundtrip_all_codes():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    vals = O.e4m3_decode(codes).astype(np.float32)
+    back = O.e4m3_encode(vals)
+    # +0 and -0 are distinct codes that both decode to zero
+    assert np.array_equal(back[codes != 0x80], codes[codes != 0x80])
+
+
+def test_e4m3_matches_torch_cast():
+    rng = np.random.default_rng(0)
+    x = np.concatenate([
+        rng.standard_normal(200000) * s for s in (1e-3, 0.05, 1.0, 30.0, 200.0)
+    ]).astype(np.float32)
+    # every midpoint between adjacent finite codes: exercises ties-to-even
+    pos = np.sort(O.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8)))
+    mids = ((pos[1:] + pos[:-1]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids, pos.astype(np.float32)])
+    x = x[np.abs(x) < 448.0]
+    ours = O.e4m3_encode(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+# ---------------------------------------------------------------------------
+# Decision logits
+# ---------------------------------------------------------------------------
+def test_decide_proj_hand_example():
+    # h = (1,1,1,1): mean square 1, so with eps = 0 the RMSNorm output is gamma.
+    h = np.ones((1, 1, 4))
+    gamma = np.array([1.0, 2.0, 0.0, -1.0])
+    W = np.array([[1.0, 1.0, 1.0, 1.0], [0.0, 0.0, 0.0, 1.0]])
+    a = O.decide_proj(h, gamma, W, None, [5.0, 5.0], scale=100.0, eps=0.0)
+    assert a[0, 0, 0] == 2.0 * 100 - 5      # W0 . gamma = 2
+    assert a[0, 1, 0] == -1.0 * 100 - 5     # W1 . gamma = -1
+    # eps enters under the square root: mean square 1 + eps 3 -> 1/2
+    a = O.decide_proj(h, gamma, W, None, [0.0, 0.0], scale=1.0, eps=3.0)
+    assert a[0, 0, 0] == 1.0 and a[0, 1, 0] == -0.5
+    # hidden (3, 4): mean square 12.5
+    a = O.decide_proj(np.array([[[3.0, 4.0]]]), np.ones(2), np.array([[1.0, 0.0]]), None, [0.0],
+                      scale=1.0, eps=0.0)
+    assert a[0, 0, 0] == pytest.approx(3.0 / math.sqrt(12.5), rel=1e-15)
+
+
+def test_decide_proj_invariants():
+    rng = np.random.default_rng(1)
+    B, T, hid, H = 2, 5, 16, 3
+    h = rng.standard_normal((B, T, hid))
+    g = rng.standard_normal(hid)
+    W = rng.standard_normal((H, hid))
+    off = rng.standard_normal((B, H))
+    a = O.decide_proj(h, g, W, None, off, eps=0.0)
+    # RMSNorm makes the logit invariant to the scale of h (eps = 0)
+    assert np.allclose(O.decide_proj(h * 7.5, g, W, None, off, eps=0.0), a, rtol=1e-12, atol=1e-9)
+    # zero projection (the adapter's initial state): alpha = -offset, gate open
+    z = O.decide_proj(h, g, np.zeros_like(W), None, off)
+    assert np.array_equal(z, np.broadcast_to(-off[:, :, None], z.shape))
+    # a bias adds bias * scale
+    bias = np.array([0.5, -1.0, 2.0])
+    ab = O.decide_proj(h, g, W, bias, off, eps=0.0)
+    assert np.allclose(ab - a, 100.0 * bias[None, :, None], atol=1e-9)
+    # layer granularity: every head takes head 0's logit
+    al = O.decide_proj(h, g, W, None, off, eps=0.0, layer_mode=True)
+    for hd in range(H):
+        assert np.array_equal(al[:, hd], a[:, 0])
+
+
+def test_decide_neuron():
+    rng = np.random.default_rng(2)
+    B, T, Hq, Hkv, D = 2, 4, 8, 2, 8
+    x = rng.standard_normal((B, T, Hq, D))
+    off = np.array([[1.0, 2.0], [3.0, 4.0]])
+    g = Hq // Hkv
+    a, xz = O.decide_neuron(x, g, Hkv, off, scale=100.0)
+    for b in range(B):
+        for hd in range(Hkv):
+            assert np.array_equal(a[b, hd], x[b, :, hd * g, D - 1] * 100.0 - off[b, hd])
+    # the decision neuron of the first query head of each group is zeroed, nothing else
+    diff = xz != x
+    assert np.all(xz[:, :, ::g, D - 1] == 0)
+    assert not diff[:, :, :, : D - 1].any()
+    assert not np.delete(diff[..., D - 1], np.arange(0, Hq, g), axis=2).any()
+    al, _ = O.decide_neuron(x, g, Hkv, off, layer_mode=True)
+    assert np.array_equal(al[:, 1], al[:, 0]) and np.array_equal(al[:, 0], a[:, 0])
+
+
+def test_rope_matches_complex_rotation():
+    # half-split RoPE is multiplication of (x_i + i x_{i+D/2}) by exp(i * angle)
+    rng = np.random.default_rng(3)
+    B, T, H, D = 1, 6, 2, 8
+    x = rng.standard_normal((B, T, H, D))
+    ang = rng.uniform(-3, 3, (10, D // 2))
+    y = O.rope(x, 2, np.cos(ang), np.sin(ang))
+    z = (x[..., : D // 2] + 1j * x[..., D // 2:]) * np.exp(1j * ang[2:2 + T])[None, :, None, :]
+    assert np.allclose(y[..., : D // 2], z.real, atol=1e-14)
+    assert np.allclose(y[..., D // 2:], z.imag, atol=1e-14)
+
+
+def test_rope_relative_position():
+    # with true rotary tables, <R(m) q, R(n) k> depends only on m - n
+    from learned_kv_cache_dms_b200.inputs import rope_tables
+    cos, sin = (t.double().numpy() for t in rope_tables(64, 16, theta=10000.0))
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((1, 1, 1, 16))
+    k = rng.standard_normal((1, 1, 1, 16))
+    d1 = np.sum(O.rope(q, 10, cos, sin) * O.rope(k, 7, cos, sin))
+    d2 = np.sum(O.rope(q, 40, cos, sin) * O.rope(k, 37, cos, sin))
+    assert d1 == pytest.approx(d2, rel=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# Append rule / cache state
+# ---------------------------------------------------------------------------
+def closed_form_state(evict, w):
+    """Parallel characterisation of the append rule (independent of the oracle's
+    sequential replay): a token opens a new slot iff it is in the first window or
+    the token w earlier is kept; a token that does not open a slot inherits the
+    slot of the token w earlier."""
+    T = len(evict)
+    opens = [t < w or not evict[t - w] for t in range(T)]
+    newslot = np.cumsum([0] + opens[:-1]) if T else np.array([])
+    slot = []
+    for t in range(T):
+        r = t
+        while not opens[r]:
+            r -= w
+        slot.append(int(newslot[r]))
+    count = int(sum(opens))
+    slot_pos = [-1] * count
+    for t in range(T):
+        if t >= T - w or not evict[t]:
+            slot_pos[slot[t]] = t
+    return slot, count, slot_pos
+
+
+def oracle_state(evict, w, P, max_pos=None, prealloc=0, pool=None):
+    T = len(evict)
+    max_pos = max_pos or max(T, 1)
+    pool = pool or (max_pos // P + 2)
+    c = O.Cache(1, 1, 1, 4, w, P, max_pos, pool, prealloc, store_values=False)
+    c.prefill(0, np.array(evict, np.uint8).reshape(1, 1, T))
+    return c, c.export(0)
+
+
+def test_append_rule_golden():
+    g = json.load(open(os.path.join(GOLDEN, "append_rule_w3_p2.json")))
+    c, s = oracle_state(g["evict"], g["window"], g["block"], max_pos=12)
+    n = g["count"]
+    assert s["count"][0, 0] == n
+    assert list(s["slot_pos"][0, 0, :n]) == g["slot_pos"]
+    assert list(s["ring_slot"][0, 0]) == g["ring_slot"]
+    assert list(s["ring_evict"][0, 0]) == g["ring_evict"]
+    assert list(s["page_table"][0, 0, :3]) == g["page_table"]
+    # token-by-token slots: replay prefixes
+    for t in range(len(g["evict"])):
+        _, st = oracle_state(g["evict"][: t + 1], g["window"], g["block"], max_pos=12)
+        assert st["slot_pos"][0, 0, g["slot_of_token"][t]] == t
+    # the retained set equals the visible keys of the last query
+    assert sorted(s["slot_pos"][0, 0, :n]) == g["visible_keys_of_query_9"]
+
+
+@pytest.mark.parametrize("T,w", [(1, 1), (5, 2), (7, 3), (12, 4)])
+def test_append_rule_exhaustive(T, w):
+    for bits in range(1 << T):
+        ev = [(bits >> t) & 1 for t in range(T)]
+        slot, count, slot_pos = closed_form_state(ev, w)
+        _, s = oracle_state(ev, w, 2)
+        assert s["count"][0, 0] == count
+        assert list(s["slot_pos"][0, 0, :count]) == slot_pos
+        for t in range(max(0, T - w), T):
+            assert s["ring_slot"][0, 0, t % w] == slot[t]
+            assert s["ring_evict"][0, 0, t % w] == ev[t]
+
+
+def test_append_rule_random_long():
+    rng = np.random.default_rng(5)
+    for T, w, P, keep in [(600, 32, 16, 0.5), (2000, 512, 256, 0.125), (3000, 100, 64, 0.9)]:
+        ev = (rng.random(T) > keep).astype(int).tolist()
+        slot, count, slot_pos = closed_form_state(ev, w)
+        _, s = oracle_state(ev, w, P)
+        assert s["count"][0, 0] == count
+        # the retained count: a full window plus every kept token before it
+        assert count == min(T, w) + sum(1 - e for e in ev[: max(0, T - w)])
+        assert list(s["slot_pos"][0, 0, :count]) == slot_pos
+        assert s["npages"][0, 0] == -(-count // P)
+
+
+def test_all_keep_and_all_evict():
+    T, w, P = 100, 8, 4
+    _, s = oracle_state([0] * T, w, P)
+    assert s["count"][0, 0] == T and list(s["slot_pos"][0, 0, :T]) == list(range(T))
+    assert list(s["page_table"][0, 0, :T // P]) == list(range(T // P))
+    _, s = oracle_state([1] * T, w, P)
+    assert s["count"][0, 0] == w
+    # pure sliding window: slot s holds the last token congruent to s mod w
+    assert list(s["slot_pos"][0, 0, :w]) == [T - w + ((sl - T) % w) for sl in range(w)]
+
+
+def test_prefill_then_appends_equals_longer_prefill():
+    rng = np.random.default_rng(6)
+    B, H, T, n, w, P = 2, 3, 70, 25, 16, 8
+    ev = (rng.random((B, H, T + n)) > 0.4).astype(np.uint8)
+    a = O.Cache(1, B, H, 4, w, P, T + n, 200, 0, store_values=False)
+    a.prefill(0, ev)
+    b = O.Cache(1, B, H, 4, w, P, T + n, 200, 0, store_values=False)
+    b.prefill(0, np.ascontiguousarray(ev[:, :, :T]))
+    for t in range(T, T + n):
+        b.append(0, np.ascontiguousarray(ev[:, :, t]))
+    sa, sb = a.export(0), b.export(0)
+    for key in ("count", "slot_pos", "ring_slot", "ring_evict", "npos"):
+        assert np.array_equal(sa[key], sb[key]), key
+    # page ids differ only in allocation order (prefill grants per (b, h) at
+    # once, appends interleave heads), never in the number of pages per head
+    assert np.array_equal(sa["npages"], sb["npages"])
+
+
+def test_page_ids_prealloc_and_order():
+    # prealloc pages are numbered row-major over (layer, b, h, page); later
+    # grants come from one ascending counter in (b, h) row-major order
+    B, H, w, P = 2, 2, 4, 4
+    L = 2
+    c = O.Cache(L, B, H, 4, w, P, 40, 100, prealloc_tokens=8)
+    T = 20
+    ev = np.zeros((B, H, T), np.uint8)
+    c.prefill(1, ev)
+    s = c.export(1)
+    pre = 2
+    for b in range(B):
+        for h in range(H):
+            base = ((1 * B + b) * H + h) * pre
+            assert list(s["page_table"][b, h, :2]) == [base, base + 1]
+    first_free = L * B * H * pre
+    expect = first_free
+    for b in range(B):
+        for h in range(H):
+            assert list(s["page_table"][b, h, 2:5]) == [expect, expect + 1, expect + 2]
+            expect += 3
+    assert s["next_page"] == expect
+
+
+def test_pool_exhaustion_sets_status():
+    c = O.Cache(1, 1, 1, 4, 4, 2, 64, 3, 0, store_values=False)
+    c.prefill(0, np.zeros((1, 1, 10), np.uint8))
+    assert c.status & 1
+
+
+# ---------------------------------------------------------------------------
+# Attention
+# ---------------------------------------------------------------------------
+def sdpa64(q, k, v, mask):
+    """torch SDPA in fp64 on [B,T,H,D] inputs with GQA expansion; mask [T,T] or None."""
+    Hq, Hkv = q.shape[2], k.shape[2]
+    g = Hq // Hkv
+    qt = torch.from_numpy(q).permute(0, 2, 1, 3)
+    kt = torch.from_numpy(k).permute(0, 2, 1, 3).repeat_interleave(g, dim=1)
+    vt = torch.from_numpy(v).permute(0, 2, 1, 3).repeat_interleave(g, dim=1)
+    if mask is None:
+        o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+    else:
+        o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.from_numpy(mask))
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+def rand_qkv(seed, B, T, Hq, Hkv, D):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, T, Hq, D)), rng.standard_normal((B, T, Hkv, D)),
+            rng.standard_normal((B, T, Hkv, D)))
+
+
+def test_attention_reduces_to_causal():
+    B, T, Hq, Hkv, D = 2, 40, 4, 2, 16
+    q, k, v = rand_qkv(7, B, T, Hq, Hkv, D)
+    ref = sdpa64(q, k, v, None)
+    rng = np.random.default_rng(8)
+    ev = (rng.random((B, Hkv, T)) > 0.5).astype(np.uint8)
+    # window >= sequence length: every causal key is inside the window
+    assert np.allclose(O.prefill_attention(q, k, v, ev, window=T), ref, atol=1e-12)
+    # all keep (or eviction disabled): dense causal attention
+    assert np.allclose(O.prefill_attention(q, k, v, np.zeros_like(ev), window=3), ref, atol=1e-12)
+    assert np.allclose(O.prefill_attention(q, k, v, O.evict_bits(ev, disable_eviction=True), window=3),
+                       ref, atol=1e-12)
+
+
+def test_attention_all_evict_is_sliding_window():
+    B, T, Hq, Hkv, D, w = 1, 50, 4, 1, 8, 7
+    q, k, v = rand_qkv(9, B, T, Hq, Hkv, D)
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    band = (j <= i) & (i - j < w)
+    ref = sdpa64(q, k, v, band)
+    got = O.prefill_attention(q, k, v, np.ones((B, Hkv, T), np.uint8), window=w)
+    assert np.allclose(got, ref, atol=1e-12)
+
+
+def test_attention_single_kept_token():
+    # only token 3 is kept: query i >= 3 + w sees token 3 plus its window
+    B, T, Hq, Hkv, D, w = 1, 30, 2, 1, 8, 5
+    q, k, v = rand_qkv(10, B, T, Hq, Hkv, D)
+    ev = np.ones((B, Hkv, T), np.uint8)
+    ev[0, 0, 3] = 0
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    mask = (j <= i) & ((i - j < w) | (j == 3))
+    assert np.allclose(O.prefill_attention(q, k, v, ev, window=w), sdpa64(q, k, v, mask), atol=1e-12)
+
+
+def test_attention_convex_combination_and_rows():
+    B, T, Hq, Hkv, D, w = 1, 20, 2, 1, 8, 4
+    q, k, _ = rand_qkv(11, B, T, Hq, Hkv, D)
+    v = np.tile(np.arange(D, dtype=np.float64), (B, T, Hkv, 1))
+    ev = (np.random.default_rng(12).random((B, Hkv, T)) > 0.5).astype(np.uint8)
+    o = O.prefill_attention(q, k, v, ev, w)
+    assert np.allclose(o, np.arange(D)[None, None, None, :], atol=1e-12)
+    q, k, v = rand_qkv(13, B, T, Hq, Hkv, D)
+    full = O.prefill_attention(q, k, v, ev, w)
+    rows = [(0, 1, 19), (0, 0, 3), (0, 1, 0)]
+    part = O.prefill_attention(q, k, v, ev, w, rows=rows)
+    for r, (b, hq, i) in enumerate(rows):
+        assert np.array_equal(part[r], full[b, i, hq])
+
+
+def test_decode_attention_equals_prefill_row():
+    # decoding token t over the cache equals row t of the masked prefill
+    B, T, Hq, Hkv, D, w, P = 2, 60, 4, 2, 16, 8, 4
+    q, k, v = rand_qkv(14, B, T, Hq, Hkv, D)
+    ev = (np.random.default_rng(15).random((B, Hkv, T)) > 0.5).astype(np.uint8)
+    full = O.prefill_attention(q, k, v, ev, w)
+    T0 = 40
+    c = O.Cache(1, B, Hkv, D, w, P, T, 100, 0)
+    c.prefill(0, np.ascontiguousarray(ev[:, :, :T0]), k[:, :T0].astype(np.float32), v[:, :T0].astype(np.float32))
+    for t in range(T0, T):
+        c.append(0, np.ascontiguousarray(ev[:, :, t]), np.ascontiguousarray(k[:, t]).astype(np.float32),
+                 np.ascontiguousarray(v[:, t]).astype(np.float32))
+        qt = np.ascontiguousarray(q[:, t])
+        # keys are stored as fp32 in the cache: compare with the fp32-rounded inputs
+        ref = O.prefill_attention(q, k.astype(np.float32), v.astype(np.float32), ev, w,
+                                  rows=[(b, hq, t) for b in range(B) for hq in range(Hq)])
+        got = c.decode_attention(0, qt)
+        assert np.allclose(got.reshape(-1, D), ref, atol=1e-12)
+    assert np.allclose(full[:, T - 1], c.decode_attention(0, np.ascontiguousarray(q[:, T - 1])), atol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# FP8 pages
+# ---------------------------------------------------------------------------
+def test_fp8_prefill_page_scale_and_codes():
+    B, H, D, w, P, T = 1, 1, 8, 2, 4, 6
+    rng = np.random.default_rng(16)
+    k = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    v = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    ev = np.zeros((B, H, T), np.uint8)  # all kept: slot t holds token t
+    c = O.Cache(1, B, H, D, w, P, T, 4, 0, fp8=True)
+    c.prefill(0, ev, k, v)
+    pg = c.pages()
+    for p in range(2):
+        rows = k[0, p * P:(p + 1) * P, 0]
+        s = np.float32(np.max(np.abs(rows))) / np.float32(448.0)
+        assert pg["kscale"][p] == s
+        assert np.array_equal(pg["kcode"][p, :len(rows)], O.e4m3_encode(rows / s))
+
+
+def test_fp8_decode_rescale_rule():
+    # row 0 has amax 1; row 1 has amax 2 -> the page scale doubles and row 0 is
+    # re-encoded from its decoded value
+    D, w, P = 4, 2, 4
+    c = O.Cache(1, 1, 1, D, w, P, 8, 2, 0, fp8=True)
+    r0 = np.array([[1.0, 0.3, -0.7, 0.1]], np.float32)
+    r1 = np.array([[2.0, -1.5, 0.2, 0.9]], np.float32)
+    c.prefill(0, np.zeros((1, 1, 1), np.uint8), r0.reshape(1, 1, 1, D), r0.reshape(1, 1, 1, D))
+    c.append(0, np.zeros((1, 1), np.uint8), r1, r1)
+    pg = c.pages()
+    s0 = np.float32(1.0) / np.float32(448.0)
+    s1 = np.float32(2.0) / np.float32(448.0)
+    assert pg["kscale"][0] == s1
+    c0 = O.e4m3_encode(r0[0] / s0)
+    dq = (O.e4m3_decode(c0).astype(np.float32) * s0).astype(np.float32)
+    assert np.array_equal(pg["kcode"][0, 0], O.e4m3_encode(dq / s1))
+    assert np.array_equal(pg["kcode"][0, 1], O.e4m3_encode(r1[0] / s1))
