@@ -1,0 +1,408 @@
+// Host side of libdms: descriptor checks, the cache's memory plan inside the
+// caller's buffer, the per-layer state machine and the launch sequence of each
+// entry point.  No device memory is ever allocated here.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "dms_internal.cuh"
+
+using namespace dms;
+
+namespace {
+
+constexpr int kMaxPrefillTokens = 1 << 18;
+constexpr int kMaxSmsForWork = 160;  // bound used to size the decode work list
+
+struct Plan {
+  size_t ctrl, pos, count, npages, page_table, slot_pos, ring, kept, kept_count, kept_upto, items, item_off, part_acc,
+      part_ml, k_scale, v_scale, k_pool, v_pool, total;
+  int maxp, cap, pre_pages, items_cap, first_free;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int elem_bytes(int dt) { return dt == DMS_F32 ? 4 : dt == DMS_BF16 ? 2 : 1; }
+
+int check_desc(const dms_cache_desc* d) {
+  if (!d) return DMS_ERR_INVALID;
+  if (d->num_layers <= 0 || d->batch <= 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0) return DMS_ERR_INVALID;
+  if (d->head_dim != 64 && d->head_dim != 128) return DMS_ERR_INVALID;
+  if (d->num_q_heads % d->num_kv_heads) return DMS_ERR_INVALID;
+  if (d->num_q_heads / d->num_kv_heads > 16) return DMS_ERR_INVALID;
+  if (d->block <= 0 || d->block % 16 || d->block > 4096) return DMS_ERR_INVALID;
+  if (d->window <= d->block) return DMS_ERR_INVALID;  // block must be below the window
+  if (d->max_positions <= 0 || d->max_positions > (1 << 20)) return DMS_ERR_INVALID;
+  if (d->prealloc_tokens < 0 || d->pool_pages <= 0) return DMS_ERR_INVALID;
+  if (d->act_dtype != DMS_F32 && d->act_dtype != DMS_BF16) return DMS_ERR_INVALID;
+  if (!(d->kv_dtype == d->act_dtype || (d->kv_dtype == DMS_FP8_E4M3 && d->act_dtype == DMS_BF16)))
+    return DMS_ERR_INVALID;
+  if (d->alpha_per != DMS_ALPHA_PER_HEAD && d->alpha_per != DMS_ALPHA_PER_LAYER) return DMS_ERR_INVALID;
+  if (d->alpha_source < DMS_ALPHA_PROJ || d->alpha_source > DMS_ALPHA_QUERY_NEURON) return DMS_ERR_INVALID;
+  if (d->alpha_source == DMS_ALPHA_PROJ) {
+    if (d->hidden <= 0 || d->hidden % 8) return DMS_ERR_INVALID;
+    if (d->num_kv_heads > 8 || static_cast<long>(d->num_kv_heads) * d->hidden > 40960) return DMS_ERR_INVALID;
+  }
+  if (d->alpha_source != DMS_ALPHA_PROJ && d->num_kv_heads > 32) return DMS_ERR_INVALID;
+  if (!(d->alpha_scale == d->alpha_scale) || !(d->rms_eps >= 0.0f)) return DMS_ERR_INVALID;
+  return DMS_OK;
+}
+
+Plan make_plan(const dms_cache_desc* d) {
+  Plan p{};
+  const size_t L = d->num_layers, B = d->batch, H = d->num_kv_heads, g = d->num_q_heads / d->num_kv_heads;
+  p.maxp = (d->max_positions + d->block - 1) / d->block;
+  p.cap = p.maxp * d->block;
+  p.pre_pages = std::min(p.maxp, (d->prealloc_tokens + d->block - 1) / d->block);
+  p.items_cap = static_cast<int>(std::max<size_t>(B * H * p.maxp, 4 * kMaxSmsForWork) + B * H);
+  p.first_free = static_cast<int>(L * B * H * p.pre_pages);
+  size_t o = 0;
+  auto take = [&](size_t bytes, size_t al) {
+    o = align_up(o, al);
+    size_t r = o;
+    o += bytes;
+    return r;
+  };
+  p.ctrl = take(CTRL_WORDS * 4, 256);
+  p.pos = take(L * B * 4, 256);
+  p.count = take(L * B * H * 4, 256);
+  p.npages = take(L * B * H * 4, 256);
+  p.page_table = take(L * B * H * p.maxp * 4, 256);
+  p.slot_pos = take(L * B * H * p.cap * 4, 256);
+  p.ring = take(L * B * H * d->window * 4, 256);
+  p.kept = take(B * H * d->max_positions * 4, 256);
+  p.kept_count = take(B * H * 4, 256);
+  p.kept_upto = take(B * H * (d->max_positions + 1) * 4, 256);
+  p.items = take(static_cast<size_t>(p.items_cap) * 16, 256);
+  p.item_off = take((B * H + 1) * 4, 256);
+  p.part_acc = take(static_cast<size_t>(p.items_cap) * g * d->head_dim * 4, 256);
+  p.part_ml = take(static_cast<size_t>(p.items_cap) * g * 2 * 4, 256);
+  p.k_scale = take(static_cast<size_t>(d->pool_pages) * 4, 256);
+  p.v_scale = take(static_cast<size_t>(d->pool_pages) * 4, 256);
+  const size_t page_bytes = static_cast<size_t>(d->block) * d->head_dim * elem_bytes(d->kv_dtype);
+  p.k_pool = take(page_bytes * d->pool_pages, 1024);
+  p.v_pool = take(page_bytes * d->pool_pages, 1024);
+  p.total = align_up(o, 256);
+  return p;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// Tensor map over a page pool viewed as a 2-D tensor [pool_pages * P rows, D].
+// Boxes are 16 rows by up to 128 bytes; bf16 tiles use the 128-byte swizzle,
+// FP8 tiles none (they are widened to bf16 in shared memory).
+bool make_pool_map(CUtensorMap* map, void* base, const dms_cache_desc* d) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const int eb = elem_bytes(d->kv_dtype);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d->head_dim),
+                        static_cast<cuuint64_t>(d->pool_pages) * static_cast<cuuint64_t>(d->block)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d->head_dim) * eb};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(std::min(d->head_dim, 128 / eb)), 16u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUtensorMapDataType dt = d->kv_dtype == DMS_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                           : d->kv_dtype == DMS_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                                    : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUtensorMapSwizzle sw = d->kv_dtype == DMS_FP8_E4M3 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUresult r = enc(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+struct dms_cache {
+  dms_cache_desc desc;
+  Plan plan;
+  CacheView view;
+  char* base;
+  size_t bytes;
+  int device;
+  int num_sms;
+  std::vector<int> positions;  // host copy of tokens appended per layer
+  std::vector<char> prefilled;
+  CUtensorMap kmap, vmap;
+  bool has_maps;
+};
+
+extern "C" {
+
+void dms_cache_desc_default(dms_cache_desc* d) {
+  if (!d) return;
+  std::memset(d, 0, sizeof(*d));
+  d->window = 512;
+  d->block = 256;
+  d->prealloc_tokens = 4096;
+  d->act_dtype = DMS_BF16;
+  d->kv_dtype = DMS_BF16;
+  d->alpha_per = DMS_ALPHA_PER_HEAD;
+  d->alpha_source = DMS_ALPHA_PROJ;
+  d->alpha_scale = 100.0f;
+  d->rms_eps = 1e-6f;
+  d->disable_eviction = 0;
+}
+
+int dms_cache_bytes(const dms_cache_desc* desc, size_t* dev_bytes) {
+  int e = check_desc(desc);
+  if (e) return e;
+  if (!dev_bytes) return DMS_ERR_INVALID;
+  Plan p = make_plan(desc);
+  if (static_cast<long long>(desc->pool_pages) < static_cast<long long>(p.first_free)) return DMS_ERR_INVALID;
+  *dev_bytes = p.total;
+  return DMS_OK;
+}
+
+int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, void* stream, dms_cache** out) {
+  if (!out) return DMS_ERR_INVALID;
+  *out = nullptr;
+  int e = check_desc(desc);
+  if (e) return e;
+  Plan p = make_plan(desc);
+  if (desc->pool_pages < p.first_free) return DMS_ERR_INVALID;
+  if (!dev_mem || (reinterpret_cast<uintptr_t>(dev_mem) & 255)) return DMS_ERR_INVALID;
+  if (bytes < p.total) return DMS_ERR_NOMEM;
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, dev_mem) != cudaSuccess || attr.type != cudaMemoryTypeDevice) {
+    cudaGetLastError();
+    return DMS_ERR_INVALID;
+  }
+  dms_cache* c = new (std::nothrow) dms_cache();
+  if (!c) return DMS_ERR_INVALID;
+  c->desc = *desc;
+  c->plan = p;
+  c->base = static_cast<char*>(dev_mem);
+  c->bytes = bytes;
+  c->device = attr.device;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
+    delete c;
+    return DMS_ERR_CUDA;
+  }
+  c->positions.assign(desc->num_layers, 0);
+  c->prefilled.assign(desc->num_layers, 0);
+  CacheView& v = c->view;
+  v.L = desc->num_layers;
+  v.B = desc->batch;
+  v.Hq = desc->num_q_heads;
+  v.Hkv = desc->num_kv_heads;
+  v.D = desc->head_dim;
+  v.hidden = desc->hidden;
+  v.w = desc->window;
+  v.P = desc->block;
+  v.maxp = p.maxp;
+  v.cap = p.cap;
+  v.pool_pages = desc->pool_pages;
+  v.pre_pages = p.pre_pages;
+  v.max_pos = desc->max_positions;
+  v.kv_dtype = desc->kv_dtype;
+  v.act_dtype = desc->act_dtype;
+  v.alpha_per = desc->alpha_per;
+  v.alpha_source = desc->alpha_source;
+  v.disable = desc->disable_eviction ? 1 : 0;
+  v.alpha_scale = desc->alpha_scale;
+  v.rms_eps = desc->rms_eps;
+  v.num_sms = c->num_sms;
+  char* b = c->base;
+  v.ctrl = reinterpret_cast<int*>(b + p.ctrl);
+  v.pos = reinterpret_cast<int*>(b + p.pos);
+  v.count = reinterpret_cast<int*>(b + p.count);
+  v.npages = reinterpret_cast<int*>(b + p.npages);
+  v.page_table = reinterpret_cast<int*>(b + p.page_table);
+  v.slot_pos = reinterpret_cast<int*>(b + p.slot_pos);
+  v.ring = reinterpret_cast<int*>(b + p.ring);
+  v.kept = reinterpret_cast<int*>(b + p.kept);
+  v.kept_count = reinterpret_cast<int*>(b + p.kept_count);
+  v.kept_upto = reinterpret_cast<int*>(b + p.kept_upto);
+  v.items = reinterpret_cast<int4*>(b + p.items);
+  v.item_off = reinterpret_cast<int*>(b + p.item_off);
+  v.part_acc = reinterpret_cast<float*>(b + p.part_acc);
+  v.part_ml = reinterpret_cast<float*>(b + p.part_ml);
+  v.items_cap = p.items_cap;
+  v.k_scale = reinterpret_cast<float*>(b + p.k_scale);
+  v.v_scale = reinterpret_cast<float*>(b + p.v_scale);
+  v.k_pool = b + p.k_pool;
+  v.v_pool = b + p.v_pool;
+  c->has_maps = false;
+  if (desc->kv_dtype != DMS_F32) {
+    int prev = cur;
+    if (prev != c->device) cudaSetDevice(c->device);
+    c->has_maps = make_pool_map(&c->kmap, v.k_pool, desc) && make_pool_map(&c->vmap, v.v_pool, desc);
+    if (prev != c->device) cudaSetDevice(prev);
+    if (!c->has_maps) {
+      delete c;
+      return DMS_ERR_CUDA;
+    }
+  }
+  if (launch_init(v, true, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    delete c;
+    return DMS_ERR_CUDA;
+  }
+  *out = c;
+  return DMS_OK;
+}
+
+int dms_cache_free(dms_cache* c) {
+  delete c;
+  return DMS_OK;
+}
+
+int dms_cache_reset(dms_cache* c, void* stream) {
+  if (!c) return DMS_ERR_INVALID;
+  if (launch_init(c->view, false, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DMS_ERR_CUDA;
+  std::fill(c->positions.begin(), c->positions.end(), 0);
+  std::fill(c->prefilled.begin(), c->prefilled.end(), 0);
+  return DMS_OK;
+}
+
+int dms_cache_get_layout(const dms_cache* c, dms_cache_layout* l) {
+  if (!c || !l) return DMS_ERR_INVALID;
+  const Plan& p = c->plan;
+  l->total_bytes = p.total;
+  l->status = p.ctrl + CTRL_STATUS * 4;
+  l->next_page = p.ctrl + CTRL_NEXT_PAGE * 4;
+  l->pos = p.pos;
+  l->count = p.count;
+  l->npages = p.npages;
+  l->page_table = p.page_table;
+  l->slot_pos = p.slot_pos;
+  l->ring = p.ring;
+  l->k_pool = p.k_pool;
+  l->v_pool = p.v_pool;
+  l->k_scale = p.k_scale;
+  l->v_scale = p.v_scale;
+  l->max_pages_per_head = p.maxp;
+  l->slot_capacity = p.cap;
+  l->prealloc_pages = p.pre_pages;
+  l->first_free_page = p.first_free;
+  return DMS_OK;
+}
+
+int dms_cache_status(dms_cache* c, void* stream, int* status) {
+  if (!c || !status) return DMS_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  if (cudaMemcpyAsync(&h, c->view.ctrl + CTRL_STATUS, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DMS_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DMS_ERR_CUDA;
+  *status = h;
+  return DMS_OK;
+}
+
+int dms_cache_positions(const dms_cache* c, int layer) {
+  if (!c || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
+  return c->positions[layer];
+}
+
+static int check_decide(const dms_cache* c, const dms_decide_params* d) {
+  if (!d || !d->offset) return DMS_ERR_INVALID;
+  if (d->offset_batch_stride != 0 && d->offset_batch_stride != c->desc.num_kv_heads) return DMS_ERR_INVALID;
+  if (c->desc.alpha_source == DMS_ALPHA_PROJ && (!d->hidden || !d->norm_weight || !d->proj_weight))
+    return DMS_ERR_INVALID;
+  return DMS_OK;
+}
+
+static DecideArgs decide_args(const dms_decide_params* d) {
+  DecideArgs a;
+  a.hidden = d->hidden;
+  a.gamma = d->norm_weight;
+  a.W = d->proj_weight;
+  a.bias = d->proj_bias;
+  a.offset = d->offset;
+  a.offset_bstride = d->offset_batch_stride;
+  return a;
+}
+
+int dms_decide(dms_cache* c, int T, const dms_decide_params* d, void* neuron_src, float* alpha, void* stream) {
+  if (!c || !alpha || T <= 0 || T > c->desc.max_positions) return DMS_ERR_INVALID;
+  int e = check_decide(c, d);
+  if (e) return e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t r;
+  if (c->desc.alpha_source == DMS_ALPHA_PROJ) {
+    r = launch_decide_proj(c->view, T, decide_args(d), alpha, s);
+  } else {
+    if (!neuron_src) return DMS_ERR_INVALID;
+    const bool key = c->desc.alpha_source == DMS_ALPHA_KEY_NEURON;
+    r = launch_neuron_rope(c->view, T, 0, key ? nullptr : neuron_src, key ? neuron_src : nullptr, d->offset,
+                           d->offset_batch_stride, true, alpha, nullptr, nullptr, s);
+  }
+  return r == cudaSuccess ? DMS_OK : DMS_ERR_CUDA;
+}
+
+int dms_prefill(dms_cache* c, int layer, const dms_prefill_args* a, void* stream) {
+  if (!c || !a || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
+  const int T = a->seq_len;
+  if (T <= 0 || T > c->desc.max_positions || T > kMaxPrefillTokens) return DMS_ERR_INVALID;
+  if (!a->q || !a->k || !a->v || !a->o || !a->alpha) return DMS_ERR_INVALID;
+  if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
+  if (a->decide) {
+    int e = check_decide(c, a->decide);
+    if (e) return e;
+  }
+  if (c->prefilled[layer]) return DMS_ERR_STATE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const CacheView& v = c->view;
+  const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
+  if (a->decide && !neuron) {
+    if (launch_decide_proj(v, T, decide_args(a->decide), a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
+  }
+  if (neuron || a->rope_cos) {
+    if (launch_neuron_rope(v, T, 0, a->q, a->k, neuron ? a->decide->offset : nullptr,
+                           neuron ? a->decide->offset_batch_stride : 0, neuron, a->alpha, a->rope_cos, a->rope_sin,
+                           s) != cudaSuccess)
+      return DMS_ERR_CUDA;
+  }
+  if (launch_prefill_scan(v, layer, T, a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
+  if (launch_prefill_scatter(v, layer, T, a->k, a->v, s) != cudaSuccess) return DMS_ERR_CUDA;
+  if (launch_prefill_attention(v, T, a->q, a->k, a->v, a->o, s) != cudaSuccess) return DMS_ERR_CUDA;
+  c->prefilled[layer] = 1;
+  c->positions[layer] = T;
+  return DMS_OK;
+}
+
+int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* stream) {
+  if (!c || !a || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
+  if (!a->q || !a->k || !a->v || !a->o || !a->alpha) return DMS_ERR_INVALID;
+  if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
+  if (a->decide) {
+    int e = check_decide(c, a->decide);
+    if (e) return e;
+  }
+  if (!c->prefilled[layer] || c->positions[layer] >= c->desc.max_positions) return DMS_ERR_STATE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const CacheView& v = c->view;
+  const int t = c->positions[layer];
+  const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
+  if (a->decide && !neuron) {
+    if (launch_decide_proj(v, 1, decide_args(a->decide), a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
+  }
+  if (neuron || a->rope_cos) {
+    if (launch_neuron_rope(v, 1, t, a->q, a->k, neuron ? a->decide->offset : nullptr,
+                           neuron ? a->decide->offset_batch_stride : 0, neuron, a->alpha, a->rope_cos, a->rope_sin,
+                           s) != cudaSuccess)
+      return DMS_ERR_CUDA;
+  }
+  if (launch_decode_append(v, layer, t, a->k, a->v, a->alpha, c->num_sms, s) != cudaSuccess) return DMS_ERR_CUDA;
+  if (launch_decode_attention(v, layer, a->q, a->o, c->has_maps ? &c->kmap : nullptr,
+                              c->has_maps ? &c->vmap : nullptr, c->num_sms, s) != cudaSuccess)
+    return DMS_ERR_CUDA;
+  c->positions[layer] = t + 1;
+  return DMS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,260 @@
+// Internal definitions shared by the CUDA translation units of libdms.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dms.h"
+
+namespace dms {
+
+// ---------------------------------------------------------------------------
+// Control words at the start of the cache buffer.
+// ---------------------------------------------------------------------------
+enum Ctrl {
+  CTRL_STATUS = 0,       // sticky DMS_ST_* bits
+  CTRL_NEXT_PAGE = 1,    // next page id the ascending counter hands out
+  CTRL_DONE_SCAN = 2,    // arrival counter of the prefill scan CTAs
+  CTRL_DONE_APPEND = 3,  // arrival counter of the decode append CTAs
+  CTRL_NITEMS = 4,       // decode attention work items of the last step
+  CTRL_CHUNK = 5,        // slots per work item of the last step
+  CTRL_WORDS = 64
+};
+
+// Device view of one cache: sizes and device pointers into the caller buffer.
+struct CacheView {
+  int L, B, Hq, Hkv, D, hidden, w, P, maxp, cap, pool_pages, pre_pages, max_pos;
+  int kv_dtype, act_dtype, alpha_per, alpha_source, disable;
+  float alpha_scale, rms_eps;
+  int num_sms;
+  int* ctrl;
+  int* pos;         // [L,B]
+  int* count;       // [L,B,Hkv]
+  int* npages;      // [L,B,Hkv]
+  int* page_table;  // [L,B,Hkv,maxp]
+  int* slot_pos;    // [L,B,Hkv,cap]
+  int* ring;        // [L,B,Hkv,w]
+  int* kept;        // [B,Hkv,max_pos]   prefill scratch: kept positions, ascending
+  int* kept_count;  // [B,Hkv]
+  int* kept_upto;   // [B,Hkv,max_pos+1] prefill scratch: kept tokens before position t
+  int4* items;      // [items_cap] decode work items: (bh, s0, s1, 0)
+  int* item_off;    // [B*Hkv+1]
+  float* part_acc;  // [items_cap, g, D]
+  float* part_ml;   // [items_cap, g, 2]  (running max, running sum)
+  int items_cap;
+  float* k_scale;   // [pool_pages]
+  float* v_scale;
+  void* k_pool;     // [pool_pages, P, D]
+  void* v_pool;
+};
+
+constexpr unsigned RING_EVICT = 0x80000000u;
+constexpr int RING_SLOT_MASK = 0x7FFFFFFF;
+
+// Bounded spin limit for every device-side wait.
+constexpr long long kSpinLimit = 1ll << 26;
+
+__device__ __forceinline__ void set_status(int* ctrl, int bits) { atomicOr(&ctrl[CTRL_STATUS], bits); }
+
+// ---------------------------------------------------------------------------
+// Element helpers
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Unpack a 16-byte vector into floats (8 bf16 or 4 fp32).
+template <typename T>
+struct Vec16 {
+  static constexpr int N = 16 / sizeof(T);
+};
+
+__device__ __forceinline__ void unpack16(const uint4& u, float* f, const __nv_bfloat16*) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(p[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void unpack16(const uint4& u, float* f, const float*) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+
+// FP8 E4M3 encode with round-to-nearest-even and saturation to +-448.
+__device__ __forceinline__ uint8_t fp8_encode(float x) {
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+__device__ __forceinline__ float fp8_decode(uint8_t c) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024,
+// a multiple of 32).  `tmp` holds 32 ints of shared memory.  Returns the
+// exclusive prefix; *total receives the block sum.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int s = lane < nw ? tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    tmp[lane] = s;  // inclusive prefix of warp sums
+  }
+  __syncthreads();
+  int warp_base = wid ? tmp[wid - 1] : 0;
+  *total = tmp[nw - 1];
+  __syncthreads();
+  return warp_base + x - v;
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers: cp.async, ldmatrix, mma.sync, mbarrier, TMA tile loads.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool valid) {
+  int src_bytes = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                            uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                                  uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D = A * B + D, m16n8k16, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: returns false (and the caller must give up) after kSpinLimit tries.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  for (long long i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// 2-D TMA tile load (no multicast) into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];\n" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (one per translation unit).
+// ---------------------------------------------------------------------------
+struct DecideArgs {
+  const void* hidden;
+  const void* gamma;
+  const void* W;
+  const void* bias;
+  const float* offset;
+  int offset_bstride;
+};
+
+cudaError_t launch_init(const CacheView& c, bool full, cudaStream_t s);
+cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, float* alpha, cudaStream_t s);
+cudaError_t launch_neuron_rope(const CacheView& c, int T, int pos0, void* q, void* k, const float* offset,
+                               int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
+                               const float* sin_t, cudaStream_t s);
+cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T, const float* alpha, cudaStream_t s);
+cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T, const void* k, const void* v,
+                                   cudaStream_t s);
+cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, const void* k, const void* v,
+                                     void* o, cudaStream_t s);
+cudaError_t launch_decode_append(const CacheView& c, int layer, int t, const void* k, const void* v,
+                                 const float* alpha, int num_sms, cudaStream_t s);
+cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q, void* o,
+                                    const CUtensorMap* kmap, const CUtensorMap* vmap, int num_sms,
+                                    cudaStream_t s);
+
+}  // namespace dms

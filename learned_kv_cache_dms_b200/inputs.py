@@ -124,15 +124,17 @@ def calibrate_offsets(raw_logits: np.ndarray, keep) -> tuple[np.ndarray, float]:
     """Offsets [B, H] that keep a `keep` fraction of tokens per (b, h).
 
     raw_logits[B, H, T] are the logits computed with a zero offset; a token is
-    kept when raw <= offset.  The offset sits halfway between the k-th and
-    (k+1)-th smallest raw logits (k = round(keep * T)), so every decision has a
-    margin; the smallest margin is returned too.
+    kept when raw <= offset.  The offset sits in the middle of the widest gap
+    between consecutive sorted raw logits within +-1% of rank k = keep * T, so
+    every decision has a margin that floating-point rounding cannot cross; the
+    smallest margin is returned too.
     """
     raw = np.asarray(raw_logits, np.float64)
     B, H, T = raw.shape
     keep = np.broadcast_to(np.asarray(keep, np.float64), (B, H))
     off = np.empty((B, H), np.float64)
     margin = math.inf
+    win = max(1, T // 100)
     for b in range(B):
         for h in range(H):
             s = np.sort(raw[b, h])
@@ -142,7 +144,9 @@ def calibrate_offsets(raw_logits: np.ndarray, keep) -> tuple[np.ndarray, float]:
             elif k >= T:
                 o = s[-1] + 1.0
             else:
-                o = 0.5 * (s[k - 1] + s[k])
+                lo, hi = max(1, k - win), min(T - 1, k + win)
+                j = lo + int(np.argmax(s[lo:hi + 1] - s[lo - 1:hi]))
+                o = 0.5 * (s[j - 1] + s[j])
             off[b, h] = o
             margin = min(margin, float(np.min(np.abs(raw[b, h] - o))))
     return off.astype(np.float32), margin

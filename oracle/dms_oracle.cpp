@@ -334,6 +334,10 @@ void oracle_decide_neuron(int B, int T, int Hsrc, int D, int group, int Hkv, dou
 // Rotary embedding, half-split form: for i < D/2 the pair (x_i, x_{i+D/2}) is
 // rotated by the angle of (position, i), with cos/sin read from caller tables
 // [max_pos, D/2].  x is [B,T,H,D]; token t sits at position pos0 + t.
+// Computed in fp32 with each product and sum rounded separately
+// (x_i' = fl(fl(x_i c) - fl(x_{i+D/2} s)), x_{i+D/2}' = fl(fl(x_{i+D/2} c) + fl(x_i s))):
+// the rotated keys are stored in the activation dtype and their FP8 codes are
+// integer decisions, so the oracle rounds exactly as the kernel does.
 void oracle_rope(int B, int T, int H, int D, double* x, int pos0, const double* cos_t,
                  const double* sin_t) {
   const int half = D / 2;
@@ -344,9 +348,11 @@ void oracle_rope(int B, int T, int H, int D, double* x, int pos0, const double* 
         const double* c = cos_t + static_cast<size_t>(pos0 + t) * half;
         const double* s = sin_t + static_cast<size_t>(pos0 + t) * half;
         for (int i = 0; i < half; ++i) {
-          double a = e[i], bb = e[i + half];
-          e[i] = a * c[i] - bb * s[i];
-          e[i + half] = bb * c[i] + a * s[i];
+          const float a = static_cast<float>(e[i]), bb = static_cast<float>(e[i + half]);
+          const float cf = static_cast<float>(c[i]), sf = static_cast<float>(s[i]);
+          const float ac = a * cf, bs = bb * sf, bc = bb * cf, as = a * sf;
+          e[i] = static_cast<double>(ac - bs);
+          e[i + half] = static_cast<double>(bc + as);
         }
       }
 }

@@ -1,0 +1,84 @@
+"""GPU parity: libdms (through the C ABI) against the CPU oracle on the same
+seeded inputs.  Sizes are small enough for the oracle to finish in seconds but
+span several tiles, pages and a ragged tail."""
+import numpy as np
+import pytest
+import torch
+
+from harness import Case, build, check_case
+
+CASES = {
+    # the tiny fp32 workload: B1, hidden 256, 4/2 heads, D64, 256 + 16 tokens, w32, P16, keep 1/2
+    "tiny_f32_proj": Case(B=1, T=256, steps=16, Hq=4, Hkv=2, D=64, hidden=256, w=32, P=16, act="f32", kv="f32",
+                          source="proj", keep=0.5, seed=1001),
+    "bf16_d128_input_ragged": Case(B=2, T=600, steps=40, Hq=8, Hkv=2, D=128, w=64, P=32, act="bf16", kv="bf16",
+                                   source="input", keep=0.3, prealloc=64, seed=2),
+    "bf16_d128_proj": Case(B=2, T=515, steps=24, Hq=8, Hkv=4, D=128, hidden=512, w=96, P=32, act="bf16",
+                           kv="bf16", source="proj", keep=(1 / 16, 1 / 4), seed=3),
+    "bf16_d64_proj_layer": Case(B=2, T=333, steps=20, Hq=4, Hkv=4, D=64, hidden=256, w=48, P=16, act="bf16",
+                                kv="bf16", source="proj", per="layer", keep=0.25, seed=4),
+    "fp8_key_rope_head": Case(B=2, T=700, steps=30, Hq=8, Hkv=2, D=64, w=64, P=32, act="bf16", kv="fp8",
+                              source="key", keep=0.125, rope=True, seed=5),
+    "fp8_key_rope_layer": Case(B=2, T=700, steps=30, Hq=8, Hkv=2, D=64, w=64, P=32, act="bf16", kv="fp8",
+                               source="key", per="layer", keep=0.125, rope=True, seed=6),
+    "bf16_query_neuron": Case(B=1, T=400, steps=12, Hq=8, Hkv=2, D=128, w=64, P=32, act="bf16", kv="bf16",
+                              source="query", keep=0.2, seed=7),
+    "fp8_d128_input": Case(B=2, T=500, steps=20, Hq=4, Hkv=2, D=128, w=64, P=32, act="bf16", kv="fp8",
+                           source="input", keep=0.4, seed=8),
+    "f32_rope_input": Case(B=1, T=200, steps=10, Hq=4, Hkv=1, D=128, w=40, P=16, act="f32", kv="f32",
+                           source="input", keep=0.5, rope=True, seed=9),
+    # degenerate decision patterns
+    "all_keep": Case(B=1, T=300, steps=10, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16", source="input",
+                     keep=1.0, seed=10),
+    "all_evict": Case(B=1, T=300, steps=40, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16", source="input",
+                      keep=0.0, seed=11),
+    "disable_eviction": Case(B=1, T=300, steps=10, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16",
+                             source="input", keep=0.1, disable=True, seed=12),
+    # sequences shorter than the window, and a single-token prompt
+    "short_prompt": Case(B=2, T=20, steps=60, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16", source="input",
+                         keep=0.3, seed=13),
+    "one_token_prompt": Case(B=1, T=1, steps=40, Hq=4, Hkv=2, D=128, w=32, P=16, act="bf16", kv="bf16",
+                             source="input", keep=0.5, seed=14),
+    # second layer of a two-layer cache with preallocation
+    "layer1_of_2": Case(B=2, T=260, steps=12, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16",
+                        source="input", keep=0.3, layers=2, layer=1, prealloc=64, seed=15),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_case_inputs_and_oracle(name):
+    """CPU: the case's inputs build, its decision margins clear the bound, and
+    the oracle's own invariants hold (retained count)."""
+    case = CASES[name]
+    ins = build(case)
+    ev = ins["evict"]
+    T, w = case.T, case.w
+    cnt = ins["state_prefill"]["count"]
+    expect = min(T, w) + (1 - ev[:, :, : max(0, T - w)]).sum(-1)
+    if case.per == "layer":
+        expect = np.broadcast_to(expect[:, :1], expect.shape)
+    assert np.array_equal(cnt, expect)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_gpu_parity(name):
+    errs = check_case(CASES[name])
+    print(name, errs)
+
+
+@pytest.mark.gpu
+def test_disable_eviction_is_vanilla_causal():
+    """With eviction disabled the GPU output is plain causal attention (torch SDPA, fp64)."""
+    case = CASES["disable_eviction"]
+    ins = build(case)
+    from harness import run_gpu
+    res = run_gpu(case, ins)
+    T = case.T
+    q = torch.from_numpy(ins["q_stored"][:, :T]).permute(0, 2, 1, 3)
+    k = torch.from_numpy(ins["k_stored"][:, :T]).permute(0, 2, 1, 3).repeat_interleave(case.Hq // case.Hkv, 1)
+    v = torch.from_numpy(ins["v"][:, :T].double().numpy()).permute(0, 2, 1, 3).repeat_interleave(
+        case.Hq // case.Hkv, 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True).permute(0, 2, 1, 3).numpy()
+    assert np.max(np.abs(res["o_prefill"].double().numpy() - ref)) <= 2e-2
+    assert res["state_final"]["count"].min().item() == case.N
