@@ -238,12 +238,35 @@ DMS_API int dms_cache_status(dms_cache* cache, void* stream, int* status);
 DMS_API int dms_decide(dms_cache* cache, int seq_len, const dms_decide_params* decide, void* neuron_src,
                float* alpha, void* stream);
 
-/* Prefill layer `layer` (0 <= layer < L) of an empty cache; see dms_prefill_args. */
+/* Prefill layer `layer` (0 <= layer < L) of an empty cache; see dms_prefill_args.
+ * Equivalent to dms_prefill_compact followed by dms_prefill_attention. */
 DMS_API int dms_prefill(dms_cache* cache, int layer, const dms_prefill_args* args, void* stream);
+
+/* Steps 1-3 of dms_prefill: decision logits, neuron zeroing / rotation, and the
+ * compaction of the prompt into the layer's pages ([FastDMS] prefill kernel).
+ * Leaves the position-sorted list of kept tokens in the cache's scratch for
+ * dms_prefill_attention.  DMS_ERR_STATE if the layer was already filled. */
+DMS_API int dms_prefill_compact(dms_cache* cache, int layer, const dms_prefill_args* args, void* stream);
+
+/* Step 4 of dms_prefill: the DMS-masked attention of the prompt.  Must follow
+ * dms_prefill_compact of the same layer and length (else DMS_ERR_STATE); reads
+ * args->q, k, v (as rotated by the compaction) and writes args->o. */
+DMS_API int dms_prefill_attention(dms_cache* cache, int layer, const dms_prefill_args* args, void* stream);
 
 /* One decode step of layer `layer` after its prefill; DMS_ERR_STATE before the
  * prefill or when max_positions tokens are already held. */
 DMS_API int dms_decode_step(dms_cache* cache, int layer, const dms_decode_args* args, void* stream);
+
+/* First half of dms_decode_step: decision logit, rotation and the append of
+ * the new token ([FastDMS] decode kernel), plus the work list of the attention.
+ * The token's position is read on the device, so the call may be captured in a
+ * CUDA graph; `o` is not used. */
+DMS_API int dms_decode_append(dms_cache* cache, int layer, const dms_decode_args* args, void* stream);
+
+/* Second half of dms_decode_step: split-K grouped attention of q [B,Hq,D] over
+ * each head's retained slots, written to o [B,Hq,D] (act dtype).  Must follow a
+ * dms_decode_append of the same layer (else DMS_ERR_STATE). */
+DMS_API int dms_decode_attention(dms_cache* cache, int layer, const void* q, void* o, void* stream);
 
 /* Tokens appended so far to `layer` (host-side counter, no device access). */
 DMS_API int dms_cache_positions(const dms_cache* cache, int layer);

@@ -80,14 +80,20 @@ _lib.dms_cache_status.argtypes = [_P, _P, C.POINTER(C.c_int)]
 _lib.dms_decide.argtypes = [_P, C.c_int, C.POINTER(dms_decide_params), _P, _P, _P]
 _lib.dms_prefill.argtypes = [_P, C.c_int, C.POINTER(dms_prefill_args), _P]
 _lib.dms_decode_step.argtypes = [_P, C.c_int, C.POINTER(dms_decode_args), _P]
+_lib.dms_prefill_compact.argtypes = [_P, C.c_int, C.POINTER(dms_prefill_args), _P]
+_lib.dms_prefill_attention.argtypes = [_P, C.c_int, C.POINTER(dms_prefill_args), _P]
+_lib.dms_decode_append.argtypes = [_P, C.c_int, C.POINTER(dms_decode_args), _P]
+_lib.dms_decode_attention.argtypes = [_P, C.c_int, _P, _P, _P]
 _lib.dms_cache_positions.argtypes = [_P, C.c_int]
 for _f in ("dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset", "dms_cache_get_layout",
-           "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step", "dms_cache_positions"):
+           "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step", "dms_cache_positions",
+           "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append", "dms_decode_attention"):
     getattr(_lib, _f).restype = C.c_int
 
 EXPORTED = ("dms_cache_desc_default", "dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset",
             "dms_cache_get_layout", "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step",
-            "dms_cache_positions")
+            "dms_cache_positions", "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append",
+            "dms_decode_attention")
 
 
 def _check(code, where):
@@ -162,6 +168,22 @@ def dms_decode_step(handle: int, layer: int, args: dms_decode_args, stream=None)
     _check(_lib.dms_decode_step(handle, layer, C.byref(args), _stream(stream)), "dms_decode_step")
 
 
+def dms_prefill_compact(handle: int, layer: int, args: dms_prefill_args, stream=None) -> None:
+    _check(_lib.dms_prefill_compact(handle, layer, C.byref(args), _stream(stream)), "dms_prefill_compact")
+
+
+def dms_prefill_attention(handle: int, layer: int, args: dms_prefill_args, stream=None) -> None:
+    _check(_lib.dms_prefill_attention(handle, layer, C.byref(args), _stream(stream)), "dms_prefill_attention")
+
+
+def dms_decode_append(handle: int, layer: int, args: dms_decode_args, stream=None) -> None:
+    _check(_lib.dms_decode_append(handle, layer, C.byref(args), _stream(stream)), "dms_decode_append")
+
+
+def dms_decode_attention(handle: int, layer: int, q, o, stream=None) -> None:
+    _check(_lib.dms_decode_attention(handle, layer, _ptr(q), _ptr(o), _stream(stream)), "dms_decode_attention")
+
+
 def dms_cache_positions(handle: int, layer: int) -> int:
     return _check(_lib.dms_cache_positions(handle, layer), "dms_cache_positions")
 
@@ -207,21 +229,29 @@ class Cache:
     def positions(self, layer: int) -> int:
         return dms_cache_positions(self.handle, layer)
 
-    def prefill(self, layer, q, k, v, o, alpha, decide: dms_decide_params | None = None, rope=None, stream=None):
+    @staticmethod
+    def prefill_args(q, k, v, o, alpha, decide: dms_decide_params | None = None, rope=None) -> dms_prefill_args:
         a = dms_prefill_args()
         a.seq_len = q.shape[1]
         a.q, a.k, a.v, a.o, a.alpha = _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(alpha)
         a.decide = C.pointer(decide) if decide is not None else None
         a.rope_cos, a.rope_sin = (_ptr(rope[0]), _ptr(rope[1])) if rope is not None else (None, None)
-        dms_prefill(self.handle, layer, a, stream)
+        return a
 
-    def decode_step(self, layer, q, k, v, o, alpha, decide: dms_decide_params | None = None, rope=None,
-                    stream=None):
+    @staticmethod
+    def decode_args(q, k, v, o, alpha, decide: dms_decide_params | None = None, rope=None) -> dms_decode_args:
         a = dms_decode_args()
         a.q, a.k, a.v, a.o, a.alpha = _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(alpha)
         a.decide = C.pointer(decide) if decide is not None else None
         a.rope_cos, a.rope_sin = (_ptr(rope[0]), _ptr(rope[1])) if rope is not None else (None, None)
-        dms_decode_step(self.handle, layer, a, stream)
+        return a
+
+    def prefill(self, layer, q, k, v, o, alpha, decide: dms_decide_params | None = None, rope=None, stream=None):
+        dms_prefill(self.handle, layer, self.prefill_args(q, k, v, o, alpha, decide, rope), stream)
+
+    def decode_step(self, layer, q, k, v, o, alpha, decide: dms_decide_params | None = None, rope=None,
+                    stream=None):
+        dms_decode_step(self.handle, layer, self.decode_args(q, k, v, o, alpha, decide, rope), stream)
 
     # --- state views (for inspection) ---
     def _view(self, off, n, dtype):

@@ -137,6 +137,9 @@ struct dms_cache {
   std::vector<char> prefilled;
   CUtensorMap kmap, vmap;
   bool has_maps;
+  int compacted_layer = -1;  // layer whose kept list the prefill attention may use
+  int compacted_len = 0;
+  int worklist_layer = -1;   // layer whose decode work list is current
 };
 
 extern "C" {
@@ -266,6 +269,8 @@ int dms_cache_reset(dms_cache* c, void* stream) {
   if (launch_init(c->view, false, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DMS_ERR_CUDA;
   std::fill(c->positions.begin(), c->positions.end(), 0);
   std::fill(c->prefilled.begin(), c->prefilled.end(), 0);
+  c->compacted_layer = -1;
+  c->worklist_layer = -1;
   return DMS_OK;
 }
 
@@ -338,23 +343,27 @@ int dms_decide(dms_cache* c, int T, const dms_decide_params* d, void* neuron_src
   } else {
     if (!neuron_src) return DMS_ERR_INVALID;
     const bool key = c->desc.alpha_source == DMS_ALPHA_KEY_NEURON;
-    r = launch_neuron_rope(c->view, T, 0, key ? nullptr : neuron_src, key ? neuron_src : nullptr, d->offset,
+    r = launch_neuron_rope(c->view, T, nullptr, key ? nullptr : neuron_src, key ? neuron_src : nullptr, d->offset,
                            d->offset_batch_stride, true, alpha, nullptr, nullptr, s);
   }
   return r == cudaSuccess ? DMS_OK : DMS_ERR_CUDA;
 }
 
-int dms_prefill(dms_cache* c, int layer, const dms_prefill_args* a, void* stream) {
+static int check_prefill(const dms_cache* c, int layer, const dms_prefill_args* a) {
   if (!c || !a || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
   const int T = a->seq_len;
   if (T <= 0 || T > c->desc.max_positions || T > kMaxPrefillTokens) return DMS_ERR_INVALID;
   if (!a->q || !a->k || !a->v || !a->o || !a->alpha) return DMS_ERR_INVALID;
   if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
-  if (a->decide) {
-    int e = check_decide(c, a->decide);
-    if (e) return e;
-  }
+  if (a->decide) return check_decide(c, a->decide);
+  return DMS_OK;
+}
+
+int dms_prefill_compact(dms_cache* c, int layer, const dms_prefill_args* a, void* stream) {
+  int e = check_prefill(c, layer, a);
+  if (e) return e;
   if (c->prefilled[layer]) return DMS_ERR_STATE;
+  const int T = a->seq_len;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CacheView& v = c->view;
   const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
@@ -362,22 +371,39 @@ int dms_prefill(dms_cache* c, int layer, const dms_prefill_args* a, void* stream
     if (launch_decide_proj(v, T, decide_args(a->decide), a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
   }
   if (neuron || a->rope_cos) {
-    if (launch_neuron_rope(v, T, 0, a->q, a->k, neuron ? a->decide->offset : nullptr,
+    if (launch_neuron_rope(v, T, nullptr, a->q, a->k, neuron ? a->decide->offset : nullptr,
                            neuron ? a->decide->offset_batch_stride : 0, neuron, a->alpha, a->rope_cos, a->rope_sin,
                            s) != cudaSuccess)
       return DMS_ERR_CUDA;
   }
   if (launch_prefill_scan(v, layer, T, a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
   if (launch_prefill_scatter(v, layer, T, a->k, a->v, s) != cudaSuccess) return DMS_ERR_CUDA;
-  if (launch_prefill_attention(v, T, a->q, a->k, a->v, a->o, s) != cudaSuccess) return DMS_ERR_CUDA;
   c->prefilled[layer] = 1;
   c->positions[layer] = T;
+  c->compacted_layer = layer;
+  c->compacted_len = T;
   return DMS_OK;
 }
 
-int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* stream) {
+int dms_prefill_attention(dms_cache* c, int layer, const dms_prefill_args* a, void* stream) {
+  int e = check_prefill(c, layer, a);
+  if (e) return e;
+  if (c->compacted_layer != layer || c->compacted_len != a->seq_len) return DMS_ERR_STATE;
+  if (launch_prefill_attention(c->view, a->seq_len, a->q, a->k, a->v, a->o, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return DMS_ERR_CUDA;
+  return DMS_OK;
+}
+
+int dms_prefill(dms_cache* c, int layer, const dms_prefill_args* a, void* stream) {
+  int e = dms_prefill_compact(c, layer, a, stream);
+  if (e) return e;
+  return dms_prefill_attention(c, layer, a, stream);
+}
+
+int dms_decode_append(dms_cache* c, int layer, const dms_decode_args* a, void* stream) {
   if (!c || !a || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
-  if (!a->q || !a->k || !a->v || !a->o || !a->alpha) return DMS_ERR_INVALID;
+  if (!a->q || !a->k || !a->v || !a->alpha) return DMS_ERR_INVALID;
   if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
   if (a->decide) {
     int e = check_decide(c, a->decide);
@@ -386,23 +412,37 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   if (!c->prefilled[layer] || c->positions[layer] >= c->desc.max_positions) return DMS_ERR_STATE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CacheView& v = c->view;
-  const int t = c->positions[layer];
   const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
   if (a->decide && !neuron) {
     if (launch_decide_proj(v, 1, decide_args(a->decide), a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
   }
   if (neuron || a->rope_cos) {
-    if (launch_neuron_rope(v, 1, t, a->q, a->k, neuron ? a->decide->offset : nullptr,
-                           neuron ? a->decide->offset_batch_stride : 0, neuron, a->alpha, a->rope_cos, a->rope_sin,
-                           s) != cudaSuccess)
+    // the token's position is read on the device from the layer's position counter
+    if (launch_neuron_rope(v, 1, v.pos + static_cast<long>(layer) * v.B, a->q, a->k,
+                           neuron ? a->decide->offset : nullptr, neuron ? a->decide->offset_batch_stride : 0, neuron,
+                           a->alpha, a->rope_cos, a->rope_sin, s) != cudaSuccess)
       return DMS_ERR_CUDA;
   }
-  if (launch_decode_append(v, layer, t, a->k, a->v, a->alpha, c->num_sms, s) != cudaSuccess) return DMS_ERR_CUDA;
-  if (launch_decode_attention(v, layer, a->q, a->o, c->has_maps ? &c->kmap : nullptr,
-                              c->has_maps ? &c->vmap : nullptr, c->num_sms, s) != cudaSuccess)
-    return DMS_ERR_CUDA;
-  c->positions[layer] = t + 1;
+  if (launch_decode_append(v, layer, a->k, a->v, a->alpha, c->num_sms, s) != cudaSuccess) return DMS_ERR_CUDA;
+  c->positions[layer] += 1;
+  c->worklist_layer = layer;
   return DMS_OK;
+}
+
+int dms_decode_attention(dms_cache* c, int layer, const void* q, void* o, void* stream) {
+  if (!c || !q || !o || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
+  if (c->worklist_layer != layer) return DMS_ERR_STATE;
+  if (launch_decode_attention(c->view, layer, q, o, c->has_maps ? &c->kmap : nullptr, c->has_maps ? &c->vmap : nullptr,
+                              c->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DMS_ERR_CUDA;
+  return DMS_OK;
+}
+
+int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* stream) {
+  if (a && !a->o) return DMS_ERR_INVALID;
+  int e = dms_decode_append(c, layer, a, stream);
+  if (e) return e;
+  return dms_decode_attention(c, layer, a->q, a->o, stream);
 }
 
 }  // extern "C"

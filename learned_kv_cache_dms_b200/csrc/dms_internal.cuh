@@ -243,7 +243,7 @@ struct DecideArgs {
 
 cudaError_t launch_init(const CacheView& c, bool full, cudaStream_t s);
 cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, float* alpha, cudaStream_t s);
-cudaError_t launch_neuron_rope(const CacheView& c, int T, int pos0, void* q, void* k, const float* offset,
+cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
                                int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
                                const float* sin_t, cudaStream_t s);
 cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T, const float* alpha, cudaStream_t s);
@@ -251,7 +251,7 @@ cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T, const v
                                    cudaStream_t s);
 cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, const void* k, const void* v,
                                      void* o, cudaStream_t s);
-cudaError_t launch_decode_append(const CacheView& c, int layer, int t, const void* k, const void* v,
+cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, const void* v,
                                  const float* alpha, int num_sms, cudaStream_t s);
 cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q, void* o,
                                     const CUtensorMap* kmap, const CUtensorMap* vmap, int num_sms,

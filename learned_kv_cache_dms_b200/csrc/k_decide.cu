@@ -224,10 +224,11 @@ cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, f
 //     the query of head h*g; layer granularity takes head 0's value; then the
 //     decision element of every head is set to zero;
 //  2. (tables given) half-split rotation of every query and key row of the
-//     token at position pos0 + t.
+//     token at position t (prefill), or at the sequence's current position
+//     pos_dev[b] (decode, T == 1).
 // ---------------------------------------------------------------------------
 template <typename TA>
-__global__ void k_neuron_rope(CacheView c, int T, int pos0, TA* q, TA* k, const float* offset, int ostride,
+__global__ void k_neuron_rope(CacheView c, int T, const int* pos_dev, TA* q, TA* k, const float* offset, int ostride,
                               int do_alpha, float* alpha, const float* cos_t, const float* sin_t) {
   const int lane = threadIdx.x & 31;
   const long gw = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -252,8 +253,9 @@ __global__ void k_neuron_rope(CacheView c, int T, int pos0, TA* q, TA* k, const 
       __syncwarp();
     }
     if (cos_t) {
-      const float* cs = cos_t + static_cast<long>(pos0 + t) * half;
-      const float* sn = sin_t + static_cast<long>(pos0 + t) * half;
+      const int p = pos_dev ? pos_dev[b] + t : t;
+      const float* cs = cos_t + static_cast<long>(p) * half;
+      const float* sn = sin_t + static_cast<long>(p) * half;
       const int nrow = c.Hq + c.Hkv;
       for (int idx = lane; idx < nrow * half; idx += 32) {
         const int r = idx / half, i = idx % half;
@@ -269,17 +271,17 @@ __global__ void k_neuron_rope(CacheView c, int T, int pos0, TA* q, TA* k, const 
   }
 }
 
-cudaError_t launch_neuron_rope(const CacheView& c, int T, int pos0, void* q, void* k, const float* offset,
+cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
                                int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
                                const float* sin_t, cudaStream_t s) {
   const long ntok = static_cast<long>(c.B) * T;
   const int grid = static_cast<int>(min((ntok + 7) / 8, static_cast<long>(c.num_sms) * 8));
   if (c.act_dtype == DMS_BF16)
-    k_neuron_rope<__nv_bfloat16><<<grid, 256, 0, s>>>(c, T, pos0, static_cast<__nv_bfloat16*>(q),
+    k_neuron_rope<__nv_bfloat16><<<grid, 256, 0, s>>>(c, T, pos_dev, static_cast<__nv_bfloat16*>(q),
                                                        static_cast<__nv_bfloat16*>(k), offset, offset_bstride,
                                                        do_alpha ? 1 : 0, alpha, cos_t, sin_t);
   else
-    k_neuron_rope<float><<<grid, 256, 0, s>>>(c, T, pos0, static_cast<float*>(q), static_cast<float*>(k), offset,
+    k_neuron_rope<float><<<grid, 256, 0, s>>>(c, T, pos_dev, static_cast<float*>(q), static_cast<float*>(k), offset,
                                               offset_bstride, do_alpha ? 1 : 0, alpha, cos_t, sin_t);
   return cudaGetLastError();
 }

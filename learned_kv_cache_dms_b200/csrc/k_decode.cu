@@ -16,7 +16,7 @@ namespace dms {
 // row raises its scale) and builds the work list of the attention kernel.
 // ---------------------------------------------------------------------------
 template <typename TA, bool FP8>
-__global__ void __launch_bounds__(1024) k_decode_append(CacheView c, int layer, int t, const TA* k, const TA* v,
+__global__ void __launch_bounds__(1024) k_decode_append(CacheView c, int layer, const TA* k, const TA* v,
                                                        const float* alpha, int target_items) {
   extern __shared__ int sh[];
   __shared__ int tmp[32];
@@ -34,8 +34,10 @@ __global__ void __launch_bounds__(1024) k_decode_append(CacheView c, int layer, 
     int need = 0, slot = -1, cnt = 0, have = 0;
     bool reuse = false, evict = false;
     const long li = lbase + i;
+    int t = 0;
     if (i < BH) {
       const int b = i / c.Hkv, h = i % c.Hkv;
+      t = c.pos[layer * c.B + b];  // position of the new token
       const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
       evict = !c.disable && alpha[b * c.Hkv + hs] > 0.0f;
       const int ringv = t >= w ? c.ring[li * w + t % w] : 0;
@@ -82,8 +84,8 @@ __global__ void __launch_bounds__(1024) k_decode_append(CacheView c, int layer, 
     next += tot;
   }
   if (tid == 0) c.ctrl[CTRL_NEXT_PAGE] = min(next, c.pool_pages);
-  for (int b = tid; b < c.B; b += bd) c.pos[layer * c.B + b] = t + 1;
-  __syncthreads();
+  __syncthreads();  // every head has read its position
+  for (int b = tid; b < c.B; b += bd) c.pos[layer * c.B + b] += 1;
 
   // Phase 2: K/V rows, one warp per head
   const int lane = tid & 31, wid = tid >> 5, nwarp = bd >> 5;
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(1024) k_decode_append(CacheView c, int layer, 
   }
 }
 
-cudaError_t launch_decode_append(const CacheView& c, int layer, int t, const void* k, const void* v,
+cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, const void* v,
                                  const float* alpha, int num_sms, cudaStream_t s) {
   const int BH = c.B * c.Hkv;
   const int threads = min(1024, max(128, (BH + 31) / 32 * 32));
@@ -184,19 +186,19 @@ cudaError_t launch_decode_append(const CacheView& c, int layer, int t, const voi
     e = cudaFuncSetAttribute(k_decode_append<__nv_bfloat16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    k_decode_append<__nv_bfloat16, true><<<1, threads, smem, s>>>(c, layer, t, static_cast<const __nv_bfloat16*>(k),
+    k_decode_append<__nv_bfloat16, true><<<1, threads, smem, s>>>(c, layer, static_cast<const __nv_bfloat16*>(k),
                                                                   static_cast<const __nv_bfloat16*>(v), alpha, target);
   } else if (c.kv_dtype == DMS_BF16) {
     e = cudaFuncSetAttribute(k_decode_append<__nv_bfloat16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     k_decode_append<__nv_bfloat16, false><<<1, threads, smem, s>>>(
-        c, layer, t, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), alpha, target);
+        c, layer, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), alpha, target);
   } else {
     e = cudaFuncSetAttribute(k_decode_append<float, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    k_decode_append<float, false><<<1, threads, smem, s>>>(c, layer, t, static_cast<const float*>(k),
+    k_decode_append<float, false><<<1, threads, smem, s>>>(c, layer, static_cast<const float*>(k),
                                                            static_cast<const float*>(v), alpha, target);
   }
   return cudaGetLastError();

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
     kept_upto[T] = tot_keep;
     c.count[lbh] = tot_open;
     c.kept_count[bh] = tot_keep;
+    if (h == 0) c.pos[layer * c.B + b] = T;
   }
   // 5. the last CTA to arrive grants the extra pages of every head, in (b, h)
   //    row-major order, from the ascending page counter.
