@@ -56,6 +56,9 @@ extern "C" {
 #define DMS_ERR_STATE (-2)   /* call not allowed in the cache's current state   */
 #define DMS_ERR_CUDA (-3)    /* a CUDA runtime call failed                      */
 #define DMS_ERR_NOMEM (-4)   /* caller buffer smaller than dms_cache_bytes      */
+#define DMS_ERR_SCRATCH_LIMIT (-5) /* the cache's worst-case split-K partials do not
+                                      fit the fixed scratch of
+                                      dms_decode_attention_noalloc              */
 
 /* ---- device status bits (sticky, read by dms_cache_status) ---------------- */
 #define DMS_ST_POOL_EXHAUSTED 1 /* a page was needed and the pool had none     */
@@ -267,6 +270,28 @@ DMS_API int dms_decode_append(dms_cache* cache, int layer, const dms_decode_args
  * each head's retained slots, written to o [B,Hq,D] (act dtype).  Must follow a
  * dms_decode_append of the same layer (else DMS_ERR_STATE). */
 DMS_API int dms_decode_attention(dms_cache* cache, int layer, const void* q, void* o, void* stream);
+
+/* dms_decode_attention without touching any scratch memory of the caller.
+ * The pages have no counterpart of this call: it exists for embedding the
+ * library in callers that cannot set aside device memory for the split-K
+ * partials -- e.g. an engine whose device memory is handed out by its own
+ * fixed pool at start-up and whose decode loop must never reach cudaMalloc
+ * (cudaMalloc can synchronise the device and can fail once the pool owns the
+ * memory).  Same arguments, same result as dms_decode_attention; the partial
+ * results of the splits live instead in one fixed array of device memory that
+ * the library holds (4 MiB per GPU that loads the library, kept until exit).
+ *  - Limit: the cache's worst case of split-K partials,
+ *    items_cap * (Hq/Hkv) * (head_dim + 2) * 4 bytes with
+ *    items_cap = max(B * Hkv * ceil(max_positions / block), 640) + B * Hkv,
+ *    must fit in 4 MiB; otherwise DMS_ERR_SCRATCH_LIMIT and nothing is launched.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current (no allocation); make that first call before any stream
+ *    capture.
+ *  - Every call shares the one array.  Calls that overlap on the GPU (on
+ *    different streams, or on different caches of the same device without
+ *    ordering) race on it and give wrong results; order them.  No part of the
+ *    array needs to start at zero: every partial is written before it is read. */
+DMS_API int dms_decode_attention_noalloc(dms_cache* cache, int layer, const void* q, void* o, void* stream);
 
 /* Tokens appended so far to `layer` (host-side counter, no device access). */
 DMS_API int dms_cache_positions(const dms_cache* cache, int layer);

@@ -22,14 +22,14 @@ if not os.path.exists(LIB_PATH):
 _lib = C.CDLL(LIB_PATH)
 
 # ---- constants (mirror include/dms.h) ---------------------------------------
-DMS_OK, DMS_ERR_INVALID, DMS_ERR_STATE, DMS_ERR_CUDA, DMS_ERR_NOMEM = 0, -1, -2, -3, -4
+DMS_OK, DMS_ERR_INVALID, DMS_ERR_STATE, DMS_ERR_CUDA, DMS_ERR_NOMEM, DMS_ERR_SCRATCH_LIMIT = 0, -1, -2, -3, -4, -5
 DMS_ST_POOL_EXHAUSTED, DMS_ST_CAPACITY, DMS_ST_TIMEOUT = 1, 2, 4
 DMS_F32, DMS_BF16, DMS_FP8_E4M3 = 0, 1, 2
 DMS_ALPHA_PER_HEAD, DMS_ALPHA_PER_LAYER = 0, 1
 DMS_ALPHA_PROJ, DMS_ALPHA_KEY_NEURON, DMS_ALPHA_QUERY_NEURON = 0, 1, 2
 
 _ERRORS = {DMS_ERR_INVALID: "DMS_ERR_INVALID", DMS_ERR_STATE: "DMS_ERR_STATE", DMS_ERR_CUDA: "DMS_ERR_CUDA",
-           DMS_ERR_NOMEM: "DMS_ERR_NOMEM"}
+           DMS_ERR_NOMEM: "DMS_ERR_NOMEM", DMS_ERR_SCRATCH_LIMIT: "DMS_ERR_SCRATCH_LIMIT"}
 
 
 class DMSError(RuntimeError):
@@ -84,16 +84,18 @@ _lib.dms_prefill_compact.argtypes = [_P, C.c_int, C.POINTER(dms_prefill_args), _
 _lib.dms_prefill_attention.argtypes = [_P, C.c_int, C.POINTER(dms_prefill_args), _P]
 _lib.dms_decode_append.argtypes = [_P, C.c_int, C.POINTER(dms_decode_args), _P]
 _lib.dms_decode_attention.argtypes = [_P, C.c_int, _P, _P, _P]
+_lib.dms_decode_attention_noalloc.argtypes = [_P, C.c_int, _P, _P, _P]
 _lib.dms_cache_positions.argtypes = [_P, C.c_int]
 for _f in ("dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset", "dms_cache_get_layout",
            "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step", "dms_cache_positions",
-           "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append", "dms_decode_attention"):
+           "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append", "dms_decode_attention",
+           "dms_decode_attention_noalloc"):
     getattr(_lib, _f).restype = C.c_int
 
 EXPORTED = ("dms_cache_desc_default", "dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset",
             "dms_cache_get_layout", "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step",
             "dms_cache_positions", "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append",
-            "dms_decode_attention")
+            "dms_decode_attention", "dms_decode_attention_noalloc")
 
 
 def _check(code, where):
@@ -182,6 +184,13 @@ def dms_decode_append(handle: int, layer: int, args: dms_decode_args, stream=Non
 
 def dms_decode_attention(handle: int, layer: int, q, o, stream=None) -> None:
     _check(_lib.dms_decode_attention(handle, layer, _ptr(q), _ptr(o), _stream(stream)), "dms_decode_attention")
+
+
+def dms_decode_attention_noalloc(handle: int, layer: int, q, o, stream=None) -> None:
+    """dms_decode_attention with its split-K scratch in the library's fixed
+    device array instead of the cache buffer (see include/dms.h)."""
+    _check(_lib.dms_decode_attention_noalloc(handle, layer, _ptr(q), _ptr(o), _stream(stream)),
+           "dms_decode_attention_noalloc")
 
 
 def dms_cache_positions(handle: int, layer: int) -> int:

@@ -446,3 +446,58 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention with its split-K partials in a fixed device array owned by
+// the library, for callers that cannot provide scratch memory.  Nothing here
+// allocates: the array is a file-scope __device__ variable, and its device
+// address is looked up once per device.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB per device
+static __device__ __align__(256) unsigned char g_split_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_split_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_split_scratch on `device`.  In host code the symbol is
+// only a host-side stand-in; the real address comes from cudaGetSymbolAddress
+// with that device current.
+int split_scratch_address(int device, void** out) {
+  if (device < 0 || device >= kMaxDevices) return DMS_ERR_INVALID;
+  if (!g_split_scratch_addr[device]) {
+    int prev = -1;
+    if (cudaGetDevice(&prev) != cudaSuccess) return DMS_ERR_CUDA;
+    if (prev != device && cudaSetDevice(device) != cudaSuccess) return DMS_ERR_CUDA;
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_split_scratch);
+    if (prev != device) cudaSetDevice(prev);
+    if (e != cudaSuccess || p == nullptr) return DMS_ERR_CUDA;
+    g_split_scratch_addr[device] = p;
+  }
+  *out = g_split_scratch_addr[device];
+  return DMS_OK;
+}
+
+}  // namespace
+
+extern "C" int dms_decode_attention_noalloc(dms_cache* c, int layer, const void* q, void* o, void* stream) {
+  if (!c || !q || !o || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
+  if (c->worklist_layer != layer) return DMS_ERR_STATE;
+  const size_t g = static_cast<size_t>(c->desc.num_q_heads / c->desc.num_kv_heads);
+  const size_t items = static_cast<size_t>(c->plan.items_cap);
+  const size_t acc_bytes = align_up(items * g * c->desc.head_dim * sizeof(float), 256);
+  const size_t ml_bytes = items * g * 2 * sizeof(float);
+  if (acc_bytes + ml_bytes > kNoAllocScratchBytes) return DMS_ERR_SCRATCH_LIMIT;
+  void* base = nullptr;
+  const int e = split_scratch_address(c->device, &base);
+  if (e) return e;
+  CacheView v = c->view;
+  v.part_acc = static_cast<float*>(base);
+  v.part_ml = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + acc_bytes);
+  if (launch_decode_attention(v, layer, q, o, c->has_maps ? &c->kmap : nullptr, c->has_maps ? &c->vmap : nullptr,
+                              c->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DMS_ERR_CUDA;
+  return DMS_OK;
+}
