@@ -1,6 +1,9 @@
 #!/usr/bin/env python
 """Benchmark of the DMS hot path on B200: decode tokens/s and retained-KV GB/s.
 
+Decode steps are replayed from CUDA graphs captured once (append graph and
+attention graph per step).
+
 One bench step = one pass of the whole path over one batch: cache reset,
 prefill of the prompt (decision logits, compaction into pages, DMS-masked
 attention), then every decode step (decision logit, append with delayed
@@ -47,6 +50,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiler runs)")
     return p.parse_args()
 
 
@@ -198,6 +202,27 @@ class Runner:
         self.dargs = [B_.Cache.decode_args(x["qd"][s], x["kd"][s], x["vd"][s], self.od[s], self.ad[s], self.ddec[s])
                       for s in range(wl_.decode_steps)]
         self.flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+        self.graphs = None
+
+    def capture(self):
+        """CUDA graphs of each decode step's append and attention (the decode
+        kernels read the token position from device memory, so a replay
+        advances the cache exactly like an eager call)."""
+        B_, h = self.B_, self.cache.handle
+        self.cache.reset()
+        B_.dms_prefill(h, 0, self.pargs)
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        gs = []
+        for s in range(self.wl.decode_steps):
+            ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ga, stream=side):
+                B_.dms_decode_append(h, 0, self.dargs[s])
+            with torch.cuda.graph(gb, stream=side):
+                B_.dms_decode_attention(h, 0, self.x["qd"][s], self.od[s])
+            gs.append((ga, gb))
+        torch.cuda.synchronize()
+        self.graphs = gs
 
     def step(self, ev=None, counts=None):
         """One bench step.  ev: list of event tuples filled per segment."""
@@ -216,9 +241,15 @@ class Runner:
             self.flush.fill_(s & 0xFF)
             a, b_, c = E(enable_timing=True), E(enable_timing=True), E(enable_timing=True)
             a.record()
-            B_.dms_decode_append(h, 0, self.dargs[s])
+            if self.graphs is not None:
+                self.graphs[s][0].replay()
+            else:
+                B_.dms_decode_append(h, 0, self.dargs[s])
             b_.record()
-            B_.dms_decode_attention(h, 0, self.x["qd"][s], self.od[s])
+            if self.graphs is not None:
+                self.graphs[s][1].replay()
+            else:
+                B_.dms_decode_attention(h, 0, self.x["qd"][s], self.od[s])
             c.record()
             dec.append((a, b_, c))
             if counts is not None:
@@ -229,7 +260,7 @@ class Runner:
 
 def kernel_launches_per_step(wl):
     # reset (1) + compaction (decide, scan, scatter) + prefill attention (1)
-    # + per decode step: decide, append, split-K attention, combine
+    # + per decode step: decide, append (one graph), split-K attention, combine (one graph)
     return 1 + 3 + 1 + 4 * wl.decode_steps
 
 
@@ -257,9 +288,14 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     assert r.cache.status() == 0
     pairs = visible_pairs(r.alpha, wl)
-    for _ in range(max(0, args.warmup - 1)):
+    o_eager = r.od.clone()
+    r.capture()
+    for _ in range(max(1, args.warmup - 1)):
         r.step()
     torch.cuda.synchronize()
+    assert r.cache.status() == 0
+    # the graph replays must reproduce the eager decode outputs exactly
+    assert torch.equal(o_eager, r.od), "graph replay differs from the eager decode"
 
     barrier(world)
     torch.cuda.synchronize()
@@ -306,7 +342,7 @@ def run_ours(args, world, rank, local):
     prefill_tflops = K * prefill_flops / (prefill_attn_ms / 1e3) / 1e12
     clocks = clk.summary()
 
-    e2e = run_e2e(B_, r, args, world)
+    e2e = None if args.no_e2e else run_e2e(B_, r, args, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, args.cpu_seconds)
