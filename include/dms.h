@@ -280,17 +280,20 @@ DMS_API int dms_decode_attention(dms_cache* cache, int layer, const void* q, voi
  * memory).  Same arguments, same result as dms_decode_attention; the partial
  * results of the splits live instead in one fixed array of device memory that
  * the library holds (4 MiB per GPU that loads the library, kept until exit).
- *  - Limit: the cache's worst case of split-K partials,
- *    items_cap * (Hq/Hkv) * (head_dim + 2) * 4 bytes with
+ *  - Limit: the cache's worst case of split-K scratch, one int per (b, h) for
+ *    the per-head arrival counters (rounded up to 256 bytes) plus
+ *    items_cap * (Hq/Hkv) * (head_dim + 2) * 4 bytes of partials with
  *    items_cap = max(B * Hkv * ceil(max_positions / block), 640) + B * Hkv,
  *    must fit in 4 MiB; otherwise DMS_ERR_SCRATCH_LIMIT and nothing is launched.
  *  - The first call on a device looks up the array's device address with that
  *    device current (no allocation); make that first call before any stream
  *    capture.
- *  - Every call shares the one array.  Calls that overlap on the GPU (on
- *    different streams, or on different caches of the same device without
- *    ordering) race on it and give wrong results; order them.  No part of the
- *    array needs to start at zero: every partial is written before it is read. */
+ *  - Every call shares the one array, which keeps the last call's contents.
+ *    Each call clears the per-head counters on `stream` before its kernel (the
+ *    partials need no clearing: each is written before it is read).  Calls
+ *    that overlap on the GPU (on different streams, or on different caches of
+ *    the same device without ordering) race on the array and give wrong
+ *    results; order them. */
 DMS_API int dms_decode_attention_noalloc(dms_cache* cache, int layer, const void* q, void* o, void* stream);
 
 /* Tokens appended so far to `layer` (host-side counter, no device access). */

@@ -13,7 +13,8 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libdms.so")
+# DMS_LIB_PATH selects another build of the same library (e.g. a tracing build)
+LIB_PATH = os.environ.get("DMS_LIB_PATH") or os.path.join(_PKG, "libdms.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libdms.so is not built: run `python -m learned_kv_cache_dms_b200.build` "

@@ -1,0 +1,358 @@
+// Device building blocks shared by the decode attention kernels.
+#pragma once
+
+#include "dms_internal.cuh"
+
+namespace dms {
+
+constexpr int kSub = 64;     // slots per sub-tile
+constexpr int kStages = 3;   // shared-memory stages of the TMA ring
+constexpr int kThreads = 128;
+
+template <int D, bool FP8>
+struct DecodeSmem {
+  static constexpr int HALVES = D / 64;                 // 128-byte column halves of a bf16 row
+  static constexpr int TILE_BF16 = kSub * D * 2;        // bytes of one bf16 K (or V) sub-tile
+  static constexpr int TILE_RAW = FP8 ? kSub * D : TILE_BF16;
+  static constexpr int STAGE = 2 * TILE_RAW;            // K then V, as loaded
+  static constexpr int CONV = FP8 ? 2 * TILE_BF16 : 0;  // widened bf16 K and V (FP8 only)
+};
+
+struct StageMeta {
+  int item;  // work item index
+  int bh;    // (b, h) of the item
+  int s0;    // first slot of the item
+  int sub;   // first slot of the sub-tile, relative to the item start
+  int rows;  // valid slots in the sub-tile
+  int page;  // page id
+  int last;  // 1 if this is the item's last sub-tile
+};
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a tile written
+// by TMA with the 128-byte swizzle (1024-byte aligned tile).
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// Per-CTA work partition of one layer's decode attention, identical in every
+// CTA: chunk C = the largest power-of-two divisor of P (>= 16) giving at least
+// `target` items; item j of head bh covers slots [j*C, min(count, (j+1)*C)),
+// which lie in one page.  s_cnt[BH] and s_off[BH + 1] are shared memory;
+// `red` holds 32 x 4 ints.  Returns C; s_off[BH] is the item count.
+__device__ __forceinline__ int decode_partition(const int* count, int BH, int P, int target, int* s_cnt, int* s_off,
+                                                int (*red)[4]) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int part[4] = {0, 0, 0, 0};
+  for (int i = tid; i < BH; i += kThreads) {
+    const int cnt = count[i];
+    s_cnt[i] = cnt;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) part[k] += (cnt + (P >> k) - 1) / (P >> k);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part[k] += __shfl_xor_sync(0xffffffffu, part[k], o);
+  __syncthreads();
+  if (lane == 0)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) red[warp][k] = part[k];
+  __syncthreads();
+  int C = P;
+  for (int k = 0; k < 4; ++k) {
+    C = P >> k;
+    const int tot = red[0][k] + red[1][k] + red[2][k] + red[3][k];
+    const int next = C / 2;
+    if (tot >= target || next % 16 != 0 || P % next != 0) break;
+  }
+  __syncthreads();
+  int base = 0;
+  for (int i0 = 0; i0 < BH; i0 += kThreads) {
+    const int i = i0 + tid;
+    const int n = i < BH ? (s_cnt[i] + C - 1) / C : 0;
+    int tot;
+    const int off = block_exclusive_scan(n, &red[0][0], &tot);
+    if (i < BH) s_off[i] = base + off;
+    base += tot;
+  }
+  if (tid == 0) s_off[BH] = base;
+  __syncthreads();
+  return C;
+}
+
+// Q fragments (mma.sync A operand) of the g query heads sharing a KV head;
+// rows >= g are zero.
+template <int D>
+__device__ __forceinline__ void load_q_frags(const __nv_bfloat16* qb, int g, uint32_t (&qa)[D / 16][4]) {
+  const int lane = threadIdx.x & 31;
+  const int ra = lane >> 2, rb = ra + 8;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const int col = ks * 16 + 2 * (lane & 3);
+    qa[ks][0] = ra < g ? *reinterpret_cast<const uint32_t*>(qb + static_cast<long>(ra) * D + col) : 0u;
+    qa[ks][1] = rb < g ? *reinterpret_cast<const uint32_t*>(qb + static_cast<long>(rb) * D + col) : 0u;
+    qa[ks][2] = ra < g ? *reinterpret_cast<const uint32_t*>(qb + static_cast<long>(ra) * D + col + 8) : 0u;
+    qa[ks][3] = rb < g ? *reinterpret_cast<const uint32_t*>(qb + static_cast<long>(rb) * D + col + 8) : 0u;
+  }
+}
+
+// One warp's online-softmax update over keys warp*16 .. warp*16+15 of a
+// staged sub-tile (bf16, 128-byte swizzled, column halves of 64 elements).
+// Keys >= rows and key `masked` are excluded.  Scores are in the log2 domain:
+// s = q.k * kscale * log2(e) / sqrt(D).
+template <int D>
+__device__ __forceinline__ void warp_tile(const unsigned char* kt, const unsigned char* vt, int rows, int masked,
+                                          float kscale_l2, const uint32_t (&qa)[D / 16][4], float (&acc)[D / 8][4],
+                                          float (&mrow)[2], float (&lrow)[2]) {
+  constexpr int KS = D / 16, NT = D / 8;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int mi = lane >> 3, rr = lane & 7;
+  float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int n_row = warp * 16 + (mi >> 1) * 8 + rr;
+    const int chunk = 2 * ks + (mi & 1);
+    uint32_t b0, b1, b2, b3;
+    ldmatrix_x4(b0, b1, b2, b3, smem_u32(kt + (chunk / 8) * kSub * 128 + sw128(n_row, chunk % 8)));
+    uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+    mma_bf16_16816(s[0], qa[ks], bb0);
+    mma_bf16_16816(s[1], qa[ks], bb1);
+  }
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = warp * 16 + nt * 8 + 2 * (lane & 3) + (e & 1);
+      const float x = (key < rows && key != masked) ? s[nt][e] * kscale_l2 : -INFINITY;
+      s[nt][e] = x;
+      mx[e >> 1] = fmaxf(mx[e >> 1], x);
+    }
+  float corr[2], mu[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+    const float mn = fmaxf(mrow[r], mx[r]);
+    mu[r] = mn == -INFINITY ? 0.f : mn;
+    corr[r] = exp2f(mrow[r] - mu[r]);
+    mrow[r] = mn;
+  }
+  float rs[2] = {0.f, 0.f};
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float p = exp2f(s[nt][e] - mu[e >> 1]);
+      s[nt][e] = p;
+      rs[e >> 1] += p;
+    }
+  lrow[0] = lrow[0] * corr[0] + rs[0];
+  lrow[1] = lrow[1] * corr[1] + rs[1];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    acc[nt][0] *= corr[0];
+    acc[nt][1] *= corr[0];
+    acc[nt][2] *= corr[1];
+    acc[nt][3] *= corr[1];
+  }
+  uint32_t pa[4];
+  pa[0] = pack_bf16(s[0][0], s[0][1]);
+  pa[1] = pack_bf16(s[0][2], s[0][3]);
+  pa[2] = pack_bf16(s[1][0], s[1][1]);
+  pa[3] = pack_bf16(s[1][2], s[1][3]);
+#pragma unroll
+  for (int dp = 0; dp < NT / 2; ++dp) {
+    const int n_row = warp * 16 + (mi & 1) * 8 + rr;
+    const int chunk = 2 * dp + (mi >> 1);
+    uint32_t b0, b1, b2, b3;
+    ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(vt + (chunk / 8) * kSub * 128 + sw128(n_row, chunk % 8)));
+    uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+    mma_bf16_16816(acc[2 * dp], pa, bb0);
+    mma_bf16_16816(acc[2 * dp + 1], pa, bb1);
+  }
+}
+
+// Store one warp's state (rows < g) into the merge buffer slot `src`:
+// merge[(src * g + r) * (D + 2) + {0..D-1: acc, D: max, D+1: sum}].
+template <int D>
+__device__ __forceinline__ void warp_state_to_smem(float* merge, int src, int g, const float (&acc)[D / 8][4],
+                                                   const float (&mrow)[2], const float (&lrow)[2]) {
+  constexpr int NT = D / 8, MLD = D + 2;
+  const int lane = threadIdx.x & 31;
+  const int ra = lane >> 2, rb = ra + 8;
+  float lsum[2] = {lrow[0], lrow[1]};
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    lsum[r] += __shfl_xor_sync(0xffffffffu, lsum[r], 1);
+    lsum[r] += __shfl_xor_sync(0xffffffffu, lsum[r], 2);
+  }
+  float* mw = merge + src * g * MLD;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int col = nt * 8 + 2 * (lane & 3);
+    if (ra < g) {
+      mw[ra * MLD + col] = acc[nt][0];
+      mw[ra * MLD + col + 1] = acc[nt][1];
+    }
+    if (rb < g) {
+      mw[rb * MLD + col] = acc[nt][2];
+      mw[rb * MLD + col + 1] = acc[nt][3];
+    }
+  }
+  if ((lane & 3) == 0) {
+    if (ra < g) {
+      mw[ra * MLD + D] = mrow[0];
+      mw[ra * MLD + D + 1] = lsum[0];
+    }
+    if (rb < g) {
+      mw[rb * MLD + D] = mrow[1];
+      mw[rb * MLD + D + 1] = lsum[1];
+    }
+  }
+}
+
+// Merge `nsrc` staged states per row and write the item's partial (acc scaled
+// by vscale, running max, running sum) to global memory.
+template <int D>
+__device__ __forceinline__ void merge_to_partial(const float* merge, int nsrc, int g, float vscale, float* part_acc,
+                                                 float* part_ml, long item) {
+  constexpr int MLD = D + 2;
+  for (int idx = threadIdx.x; idx < g * (D + 1); idx += kThreads) {
+    const int r = idx / (D + 1), d = idx % (D + 1);
+    float M = -INFINITY;
+    for (int sv = 0; sv < nsrc; ++sv) M = fmaxf(M, merge[(sv * g + r) * MLD + D]);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float sum = 0.f;
+    for (int sv = 0; sv < nsrc; ++sv) {
+      const float f = exp2f(merge[(sv * g + r) * MLD + D] - Mu);
+      sum += f * merge[(sv * g + r) * MLD + (d < D ? d : D + 1)];
+    }
+    if (d < D) {
+      part_acc[(item * g + r) * D + d] = sum * vscale;
+    } else {
+      part_ml[(item * g + r) * 2] = M;
+      part_ml[(item * g + r) * 2 + 1] = sum;
+    }
+  }
+}
+
+// LSE combine of a head's partials (items i0..i1) by one CTA:
+//   o[r] = sum_i 2^(m_i[r] - M[r]) acc_i[r] / sum_i 2^(m_i[r] - M[r]) l_i[r].
+// The maxima and weights are staged in shared memory (`wbuf`, at least
+// 2 * kCombineChunk + 16 floats), then each thread owns 4 consecutive output
+// columns of one row and issues its 16-byte loads for all items of a chunk
+// before using them, so the merge costs a few L2 round trips.
+constexpr int kCombineChunk = 256;  // (item, row) pairs staged per pass
+
+template <int D>
+__device__ void combine_head(const float* part_acc, const float* part_ml, int g, int i0, int i1,
+                             __nv_bfloat16* out /* [g, D] rows of this head */, float* wbuf) {
+  const int tid = threadIdx.x;
+  float* s_M = wbuf + 2 * kCombineChunk;  // [g <= 16]
+  float* s_L = s_M + 16;                 // [g]  (wbuf holds 2*kCombineChunk + 32 floats)
+  if (tid < g) {
+    s_M[tid] = -INFINITY;
+    s_L[tid] = 0.f;
+  }
+  constexpr int Q = D / 4;                            // float4 columns per row
+  constexpr int OUTS = (16 * Q + kThreads - 1) / kThreads;  // float4 outputs per thread (g <= 16)
+  float4 accv[OUTS];
+#pragma unroll
+  for (int k = 0; k < OUTS; ++k) accv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int per_chunk = max(1, kCombineChunk / g);
+  for (int c0 = i0; c0 < i1; c0 += per_chunk) {
+    const int n = min(i1, c0 + per_chunk) - c0;
+    __syncthreads();
+    for (int idx = tid; idx < n * g; idx += kThreads) {
+      const long e = (static_cast<long>(c0) * g + idx) * 2;
+      wbuf[idx] = __ldcg(&part_ml[e]);
+      wbuf[kCombineChunk + idx] = __ldcg(&part_ml[e + 1]);
+    }
+    __syncthreads();
+    if (tid < g) {
+      float M = s_M[tid];
+      for (int i = 0; i < n; ++i) M = fmaxf(M, wbuf[i * g + tid]);
+      const float Mu = M == -INFINITY ? 0.f : M;
+      const float rescale = exp2f(s_M[tid] - Mu);
+      float L = s_L[tid] * rescale;
+      for (int i = 0; i < n; ++i) {
+        const float wgt = exp2f(wbuf[i * g + tid] - Mu);
+        wbuf[i * g + tid] = wgt;
+        L += wgt * wbuf[kCombineChunk + i * g + tid];
+      }
+      wbuf[kCombineChunk + tid] = rescale;  // the sums are consumed; reuse the slot
+      s_M[tid] = M;
+      s_L[tid] = L;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < OUTS; ++k) {
+      const int idx = tid + kThreads * k;
+      if (idx >= g * Q) break;
+      const int r = idx / Q, d4 = idx % Q;
+      const float sc = wbuf[kCombineChunk + r];
+      float4 a = accv[k];
+      a.x *= sc;
+      a.y *= sc;
+      a.z *= sc;
+      a.w *= sc;
+      const float4* src = reinterpret_cast<const float4*>(part_acc) + (static_cast<long>(c0) * g + r) * Q + d4;
+      const long stride = static_cast<long>(g) * Q;
+      int i = 0;
+      for (; i + 8 <= n; i += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (i + u) * stride);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float wgt = wbuf[(i + u) * g + r];
+          a.x = fmaf(wgt, v[u].x, a.x);
+          a.y = fmaf(wgt, v[u].y, a.y);
+          a.z = fmaf(wgt, v[u].z, a.z);
+          a.w = fmaf(wgt, v[u].w, a.w);
+        }
+      }
+      for (; i < n; ++i) {
+        const float4 v = __ldcg(src + i * stride);
+        const float wgt = wbuf[i * g + r];
+        a.x = fmaf(wgt, v.x, a.x);
+        a.y = fmaf(wgt, v.y, a.y);
+        a.z = fmaf(wgt, v.z, a.z);
+        a.w = fmaf(wgt, v.w, a.w);
+      }
+      accv[k] = a;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < OUTS; ++k) {
+    const int idx = tid + kThreads * k;
+    if (idx >= g * Q) break;
+    const int r = idx / Q, d4 = idx % Q;
+    const float L = s_L[r];
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    uint2 pk;
+    pk.x = pack_bf16(accv[k].x * inv, accv[k].y * inv);
+    pk.y = pack_bf16(accv[k].z * inv, accv[k].w * inv);
+    *reinterpret_cast<uint2*>(out + static_cast<long>(r) * D + d4 * 4) = pk;
+  }
+}
+
+// Slot plan of the next append of head i of `layer` (token position t):
+// reuse the slot of token t - w when it was marked for eviction, else take slot
+// count (a new page when that slot starts one).  plan.x = slot,
+// plan.y = bit 0 reuse | bit 1 new page | bit 2 over capacity.
+// Loads bypass L1: the state may have been written by other CTAs of the same
+// launch (made visible by their fences).
+__device__ __forceinline__ int2 next_plan(const CacheView& c, long li, int t) {
+  const int w = c.w, P = c.P;
+  const int cnt = __ldcg(&c.count[li]), have = __ldcg(&c.npages[li]);
+  const int ringv = t >= w ? __ldcg(&c.ring[li * w + t % w]) : 0;
+  const bool reuse = t >= w && (static_cast<unsigned>(ringv) & RING_EVICT);
+  if (reuse) return make_int2(ringv & RING_SLOT_MASK, 1);
+  if (cnt >= c.cap) return make_int2(-1, 4);
+  return make_int2(cnt, (cnt % P == 0 && cnt / P >= have) ? 2 : 0);
+}
+
+}  // namespace dms

@@ -17,9 +17,10 @@ namespace {
 
 constexpr int kMaxPrefillTokens = 1 << 18;
 constexpr int kMaxSmsForWork = 160;  // bound used to size the decode work list
+constexpr int kFuseDecideHeads = 64;  // decode decisions fused into the append up to B*Hkv heads
 
 struct Plan {
-  size_t ctrl, pos, count, npages, page_table, slot_pos, ring, kept, kept_count, kept_upto, items, item_off, part_acc,
+  size_t ctrl, pos, count, npages, page_table, slot_pos, ring, plan, kept, kept_count, kept_upto, head_done, part_acc,
       part_ml, k_scale, v_scale, k_pool, v_pool, total;
   int maxp, cap, pre_pages, items_cap, first_free;
 };
@@ -74,11 +75,11 @@ Plan make_plan(const dms_cache_desc* d) {
   p.page_table = take(L * B * H * p.maxp * 4, 256);
   p.slot_pos = take(L * B * H * p.cap * 4, 256);
   p.ring = take(L * B * H * d->window * 4, 256);
+  p.plan = take(L * B * H * 8, 256);
   p.kept = take(B * H * d->max_positions * 4, 256);
   p.kept_count = take(B * H * 4, 256);
   p.kept_upto = take(B * H * (d->max_positions + 1) * 4, 256);
-  p.items = take(static_cast<size_t>(p.items_cap) * 16, 256);
-  p.item_off = take((B * H + 1) * 4, 256);
+  p.head_done = take(B * H * 4, 256);
   p.part_acc = take(static_cast<size_t>(p.items_cap) * g * d->head_dim * 4, 256);
   p.part_ml = take(static_cast<size_t>(p.items_cap) * g * 2 * 4, 256);
   p.k_scale = take(static_cast<size_t>(d->pool_pages) * 4, 256);
@@ -228,11 +229,11 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   v.page_table = reinterpret_cast<int*>(b + p.page_table);
   v.slot_pos = reinterpret_cast<int*>(b + p.slot_pos);
   v.ring = reinterpret_cast<int*>(b + p.ring);
+  v.plan = reinterpret_cast<int2*>(b + p.plan);
   v.kept = reinterpret_cast<int*>(b + p.kept);
   v.kept_count = reinterpret_cast<int*>(b + p.kept_count);
   v.kept_upto = reinterpret_cast<int*>(b + p.kept_upto);
-  v.items = reinterpret_cast<int4*>(b + p.items);
-  v.item_off = reinterpret_cast<int*>(b + p.item_off);
+  v.head_done = reinterpret_cast<int*>(b + p.head_done);
   v.part_acc = reinterpret_cast<float*>(b + p.part_acc);
   v.part_ml = reinterpret_cast<float*>(b + p.part_ml);
   v.items_cap = p.items_cap;
@@ -413,8 +414,14 @@ int dms_decode_append(dms_cache* c, int layer, const dms_decode_args* a, void* s
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CacheView& v = c->view;
   const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
+  // The adapter's decision logits are computed inside the append kernel when
+  // the batch has few heads (one warp per dot product); otherwise by their own
+  // kernel with one CTA per (head, sequence).
+  const bool fuse = a->decide && !neuron && c->desc.batch * c->desc.num_kv_heads <= kFuseDecideHeads;
+  DecideArgs da{};
   if (a->decide && !neuron) {
-    if (launch_decide_proj(v, 1, decide_args(a->decide), a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
+    da = decide_args(a->decide);
+    if (!fuse && launch_decide_proj(v, 1, da, a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
   }
   if (neuron || a->rope_cos) {
     // the token's position is read on the device from the layer's position counter
@@ -423,7 +430,8 @@ int dms_decode_append(dms_cache* c, int layer, const dms_decode_args* a, void* s
                            a->alpha, a->rope_cos, a->rope_sin, s) != cudaSuccess)
       return DMS_ERR_CUDA;
   }
-  if (launch_decode_append(v, layer, a->k, a->v, a->alpha, c->num_sms, s) != cudaSuccess) return DMS_ERR_CUDA;
+  if (launch_decode_append(v, layer, a->k, a->v, a->alpha, fuse ? &da : nullptr, c->num_sms, s) != cudaSuccess)
+    return DMS_ERR_CUDA;
   c->positions[layer] += 1;
   c->worklist_layer = layer;
   return DMS_OK;
@@ -439,10 +447,42 @@ int dms_decode_attention(dms_cache* c, int layer, const void* q, void* o, void* 
 }
 
 int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* stream) {
-  if (a && !a->o) return DMS_ERR_INVALID;
-  int e = dms_decode_append(c, layer, a, stream);
-  if (e) return e;
-  return dms_decode_attention(c, layer, a->q, a->o, stream);
+  if (!c || !a || !a->o) return DMS_ERR_INVALID;
+  if (c->desc.kv_dtype != DMS_BF16) {
+    // FP8 pages re-encode a page before the attention may read it, and fp32
+    // pages use the CUDA-core path: append, then attend.
+    int e = dms_decode_append(c, layer, a, stream);
+    if (e) return e;
+    return dms_decode_attention(c, layer, a->q, a->o, stream);
+  }
+  if (layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
+  if (!a->q || !a->k || !a->v || !a->alpha) return DMS_ERR_INVALID;
+  if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
+  if (a->decide) {
+    int e = check_decide(c, a->decide);
+    if (e) return e;
+  }
+  if (!c->prefilled[layer] || c->positions[layer] >= c->desc.max_positions) return DMS_ERR_STATE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const CacheView& v = c->view;
+  const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
+  if (neuron || a->rope_cos) {
+    if (launch_neuron_rope(v, 1, v.pos + static_cast<long>(layer) * v.B, a->q, a->k,
+                           neuron ? a->decide->offset : nullptr, neuron ? a->decide->offset_batch_stride : 0, neuron,
+                           a->alpha, a->rope_cos, a->rope_sin, s) != cudaSuccess)
+      return DMS_ERR_CUDA;
+  }
+  DecideArgs da{};
+  const bool proj = a->decide && !neuron;
+  if (proj) da = decide_args(a->decide);
+  // One launch: attention over the pre-append slots plus the new token, then
+  // the append, with the adapter's decision logits computed inside.
+  if (launch_decode_fused(v, layer, a->q, a->k, a->v, a->o, a->alpha, proj ? &da : nullptr, &c->kmap, &c->vmap,
+                          c->num_sms, s) != cudaSuccess)
+    return DMS_ERR_CUDA;
+  c->positions[layer] += 1;
+  c->worklist_layer = layer;
+  return DMS_OK;
 }
 
 }  // extern "C"
@@ -487,15 +527,21 @@ extern "C" int dms_decode_attention_noalloc(dms_cache* c, int layer, const void*
   if (c->worklist_layer != layer) return DMS_ERR_STATE;
   const size_t g = static_cast<size_t>(c->desc.num_q_heads / c->desc.num_kv_heads);
   const size_t items = static_cast<size_t>(c->plan.items_cap);
+  const size_t heads = static_cast<size_t>(c->desc.batch) * c->desc.num_kv_heads;
+  const size_t cnt_bytes = align_up(heads * sizeof(int), 256);
   const size_t acc_bytes = align_up(items * g * c->desc.head_dim * sizeof(float), 256);
   const size_t ml_bytes = items * g * 2 * sizeof(float);
-  if (acc_bytes + ml_bytes > kNoAllocScratchBytes) return DMS_ERR_SCRATCH_LIMIT;
+  if (cnt_bytes + acc_bytes + ml_bytes > kNoAllocScratchBytes) return DMS_ERR_SCRATCH_LIMIT;
   void* base = nullptr;
   const int e = split_scratch_address(c->device, &base);
   if (e) return e;
+  unsigned char* p = static_cast<unsigned char*>(base);
   CacheView v = c->view;
-  v.part_acc = static_cast<float*>(base);
-  v.part_ml = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + acc_bytes);
+  v.head_done = reinterpret_cast<int*>(p);  // per-head arrival counters: must start at zero
+  v.part_acc = reinterpret_cast<float*>(p + cnt_bytes);
+  v.part_ml = reinterpret_cast<float*>(p + cnt_bytes + acc_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(v.head_done, 0, heads * sizeof(int), st) != cudaSuccess) return DMS_ERR_CUDA;
   if (launch_decode_attention(v, layer, q, o, c->has_maps ? &c->kmap : nullptr, c->has_maps ? &c->vmap : nullptr,
                               c->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DMS_ERR_CUDA;

@@ -18,9 +18,7 @@ enum Ctrl {
   CTRL_STATUS = 0,       // sticky DMS_ST_* bits
   CTRL_NEXT_PAGE = 1,    // next page id the ascending counter hands out
   CTRL_DONE_SCAN = 2,    // arrival counter of the prefill scan CTAs
-  CTRL_DONE_APPEND = 3,  // arrival counter of the decode append CTAs
-  CTRL_NITEMS = 4,       // decode attention work items of the last step
-  CTRL_CHUNK = 5,        // slots per work item of the last step
+  CTRL_GRID_DONE = 3,    // arrival counter of the fused decode CTAs
   CTRL_WORDS = 64
 };
 
@@ -37,12 +35,12 @@ struct CacheView {
   int* page_table;  // [L,B,Hkv,maxp]
   int* slot_pos;    // [L,B,Hkv,cap]
   int* ring;        // [L,B,Hkv,w]
+  int2* plan;       // [L,B,Hkv] slot plan of the next append (see next_plan)
   int* kept;        // [B,Hkv,max_pos]   prefill scratch: kept positions, ascending
   int* kept_count;  // [B,Hkv]
   int* kept_upto;   // [B,Hkv,max_pos+1] prefill scratch: kept tokens before position t
-  int4* items;      // [items_cap] decode work items: (bh, s0, s1, 0)
-  int* item_off;    // [B*Hkv+1]
-  float* part_acc;  // [items_cap, g, D]
+  int* head_done;   // [B*Hkv] arrival counters of the attention CTAs (self-resetting)
+  float* part_acc;  // [items_cap, g, D]   decode split-K partials, indexed by work item
   float* part_ml;   // [items_cap, g, 2]  (running max, running sum)
   int items_cap;
   float* k_scale;   // [pool_pages]
@@ -58,6 +56,25 @@ constexpr int RING_SLOT_MASK = 0x7FFFFFFF;
 constexpr long long kSpinLimit = 1ll << 26;
 
 __device__ __forceinline__ void set_status(int* ctrl, int bits) { atomicOr(&ctrl[CTRL_STATUS], bits); }
+
+// Phase timeline (tracing builds only, compiled with -DDMS_TRACE): thread 0 of
+// each CTA stores %globaltimer for phase `slot` of kernel `kid` into a
+// per-translation-unit device array read back by dms_debug_trace_read.
+#ifdef DMS_TRACE
+constexpr int kTraceCtas = 4096, kTraceSlots = 16;
+#define DMS_TRACE_MARK(kid, slot)                                                                   \
+  do {                                                                                              \
+    if (threadIdx.x == 0 && blockIdx.x < kTraceCtas) {                                              \
+      unsigned long long t_;                                                                        \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                        \
+      g_dms_trace[((kid) * kTraceCtas + blockIdx.x) * kTraceSlots + (slot)] = t_;                   \
+    }                                                                                               \
+  } while (0)
+#else
+#define DMS_TRACE_MARK(kid, slot) \
+  do {                            \
+  } while (0)
+#endif
 
 // ---------------------------------------------------------------------------
 // Element helpers
@@ -251,10 +268,13 @@ cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T, const v
                                    cudaStream_t s);
 cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, const void* k, const void* v,
                                      void* o, cudaStream_t s);
-cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, const void* v,
-                                 const float* alpha, int num_sms, cudaStream_t s);
+cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, const void* v, float* alpha,
+                                 const DecideArgs* fused_decide, int num_sms, cudaStream_t s);
 cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q, void* o,
                                     const CUtensorMap* kmap, const CUtensorMap* vmap, int num_sms,
                                     cudaStream_t s);
+cudaError_t launch_decode_fused(const CacheView& c, int layer, const void* q, const void* k, const void* v, void* o,
+                                float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
+                                const CUtensorMap* vmap, int num_sms, cudaStream_t s);
 
 }  // namespace dms

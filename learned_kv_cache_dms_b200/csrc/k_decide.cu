@@ -22,7 +22,9 @@ __global__ void k_init(CacheView c) {
     if (i < nbh) {
       c.npages[i] = c.pre_pages;
       c.count[i] = 0;
+      c.plan[i] = make_int2(0, 0);
     }
+    if (i < static_cast<long>(c.B) * c.Hkv) c.head_done[i] = 0;
     if (i < static_cast<long>(c.L) * c.B) c.pos[i] = 0;
     if (i < c.pool_pages) {
       c.k_scale[i] = 0.0f;
@@ -150,20 +152,27 @@ __global__ void __launch_bounds__(256) k_decide_proj(CacheView c, int T, DecideA
 }
 
 // Decode-shaped variant (one token per sequence): one CTA per (kv-head, b),
-// the hidden row and W_h read straight from global memory.
+// the hidden row and W_h read straight from global memory as 16-byte vectors.
 template <typename TA>
 __global__ void __launch_bounds__(256) k_decide_proj_row(CacheView c, DecideArgs a, float* alpha) {
   const int h = blockIdx.x, b = blockIdx.y;
   const int src = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
   const int hid = c.hidden;
-  const TA* x = static_cast<const TA*>(a.hidden) + static_cast<long>(b) * hid;
-  const TA* W = static_cast<const TA*>(a.W) + static_cast<long>(src) * hid;
-  const TA* gamma = static_cast<const TA*>(a.gamma);
+  constexpr int V = 16 / sizeof(TA);
+  const uint4* x = reinterpret_cast<const uint4*>(static_cast<const TA*>(a.hidden) + static_cast<long>(b) * hid);
+  const uint4* W = reinterpret_cast<const uint4*>(static_cast<const TA*>(a.W) + static_cast<long>(src) * hid);
+  const uint4* gamma = reinterpret_cast<const uint4*>(a.gamma);
   float ss = 0.f, dot = 0.f;
-  for (int i = threadIdx.x; i < hid; i += blockDim.x) {
-    const float xv = to_f(x[i]);
-    ss = fmaf(xv, xv, ss);
-    dot = fmaf(to_f(W[i]) * to_f(gamma[i]), xv, dot);
+  for (int vi = threadIdx.x; vi < hid / V; vi += blockDim.x) {
+    float xv[V], wv[V], gv[V];
+    unpack16(x[vi], xv, static_cast<const TA*>(nullptr));
+    unpack16(W[vi], wv, static_cast<const TA*>(nullptr));
+    unpack16(gamma[vi], gv, static_cast<const TA*>(nullptr));
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      ss = fmaf(xv[e], xv[e], ss);
+      dot = fmaf(wv[e] * gv[e], xv[e], dot);
+    }
   }
   __shared__ float red[2][32];
 #pragma unroll

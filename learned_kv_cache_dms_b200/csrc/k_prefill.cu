@@ -10,7 +10,7 @@
 //   slot(t)    = newslot(root(t))
 // The final occupants are the last w tokens plus every earlier kept token, so
 // only those are written; count = number of open tokens.
-#include "dms_internal.cuh"
+#include "decode_common.cuh"
 
 namespace dms {
 
@@ -136,6 +136,9 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
     c.ctrl[CTRL_NEXT_PAGE] = min(next, c.pool_pages);
     c.ctrl[CTRL_DONE_SCAN] = 0;
   }
+  // slot plan of the first decode append (token T) of every head
+  __syncthreads();
+  for (int i = tid; i < BH; i += bd) c.plan[static_cast<long>(layer) * BH + i] = next_plan(c, static_cast<long>(layer) * BH + i, T);
 }
 
 cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T, const float* alpha, cudaStream_t s) {

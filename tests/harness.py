@@ -45,6 +45,7 @@ class Case:
     layer: int = 0
     seed: int = 1
     attn_rows: int | None = None  # sample this many prefill rows (None: all)
+    staged: bool = False          # decode through dms_decode_append + dms_decode_attention
 
     @property
     def N(self):
@@ -228,7 +229,12 @@ def run_gpu(case: Case, ins):
                 keep_alive.append(ht)
             else:
                 dd = B_.decide_params(off)
-        cache.decode_step(case.layer, qt, kt, vt, ot, at, decide=dd, rope=rope)
+        if case.staged:
+            args = B_.Cache.decode_args(qt, kt, vt, ot, at, dd, rope)
+            B_.dms_decode_append(cache.handle, case.layer, args)
+            B_.dms_decode_attention(cache.handle, case.layer, qt, ot)
+        else:
+            cache.decode_step(case.layer, qt, kt, vt, ot, at, decide=dd, rope=rope)
         o_dec.append(ot)
         a_dec.append(at)
     torch.cuda.synchronize()

@@ -39,6 +39,14 @@ CASES = {
                          keep=0.3, seed=13),
     "one_token_prompt": Case(B=1, T=1, steps=40, Hq=4, Hkv=2, D=128, w=32, P=16, act="bf16", kv="bf16",
                              source="input", keep=0.5, seed=14),
+    # the staged API (append, then attention) on bf16 pages
+    "bf16_proj_staged": Case(B=2, T=515, steps=24, Hq=8, Hkv=4, D=128, hidden=512, w=96, P=32, act="bf16",
+                             kv="bf16", source="proj", keep=(1 / 16, 1 / 4), seed=3, staged=True),
+    "bf16_d64_key_rope_staged": Case(B=2, T=400, steps=20, Hq=8, Hkv=2, D=64, w=64, P=32, act="bf16", kv="bf16",
+                                     source="key", keep=0.2, rope=True, seed=16, staged=True),
+    # fused decode over many heads (batch 8: decision logits inside the kernel)
+    "bf16_b8_proj": Case(B=8, T=300, steps=40, Hq=16, Hkv=8, D=128, hidden=256, w=64, P=32, act="bf16", kv="bf16",
+                         source="proj", keep=(1 / 16, 1 / 4), prealloc=96, seed=17),
     # second layer of a two-layer cache with preallocation
     "layer1_of_2": Case(B=2, T=260, steps=12, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16",
                         source="input", keep=0.3, layers=2, layer=1, prealloc=64, seed=15),
