@@ -1,8 +1,9 @@
 #!/usr/bin/env python
 """Benchmark of the DMS hot path on B200: decode tokens/s and retained-KV GB/s.
 
-Decode steps are replayed from CUDA graphs captured once (append graph and
-attention graph per step).
+Decode steps are replayed from CUDA graphs captured once, one graph per step
+holding the step's start/end timing events around its kernel(s), as the step
+would run inside a whole-model graph.
 
 One bench step = one pass of the whole path over one batch: cache reset,
 prefill of the prompt (decision logits, compaction into pages, DMS-masked
@@ -215,12 +216,14 @@ class Runner:
         side = torch.cuda.Stream()
         gs = []
         for s in range(self.wl.decode_steps):
-            ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            ga = torch.cuda.CUDAGraph()
+            ev = (torch.cuda.Event(enable_timing=True, external=True),
+                  torch.cuda.Event(enable_timing=True, external=True))
             with torch.cuda.graph(ga, stream=side):
-                B_.dms_decode_append(h, 0, self.dargs[s])
-            with torch.cuda.graph(gb, stream=side):
-                B_.dms_decode_attention(h, 0, self.x["qd"][s], self.od[s])
-            gs.append((ga, gb))
+                ev[0].record()
+                B_.dms_decode_step(h, 0, self.dargs[s])
+                ev[1].record()
+            gs.append((ga, ev))
         torch.cuda.synchronize()
         self.graphs = gs
 
@@ -239,29 +242,29 @@ class Runner:
         dec = []
         for s in range(self.wl.decode_steps):
             self.flush.fill_(s & 0xFF)
-            a, b_, c = E(enable_timing=True), E(enable_timing=True), E(enable_timing=True)
-            a.record()
             if self.graphs is not None:
+                # the step's graph records its own start/end events around the kernel
                 self.graphs[s][0].replay()
             else:
-                B_.dms_decode_append(h, 0, self.dargs[s])
-            b_.record()
-            if self.graphs is not None:
-                self.graphs[s][1].replay()
-            else:
-                B_.dms_decode_attention(h, 0, self.x["qd"][s], self.od[s])
-            c.record()
-            dec.append((a, b_, c))
+                a, c = E(enable_timing=True), E(enable_timing=True)
+                a.record()
+                B_.dms_decode_step(h, 0, self.dargs[s])
+                c.record()
+                dec.append((a, c))
             if counts is not None:
                 counts.append(self.cache.state(0)["count"].sum().item())
         if ev is not None:
-            ev.append(((e0, e1, e2), dec))
+            # graph events are re-recorded by the next replay: read them now
+            torch.cuda.synchronize()
+            dec_ms = sum(g[1][0].elapsed_time(g[1][1]) for g in self.graphs) if self.graphs else \
+                sum(a.elapsed_time(c) for a, c in dec)
+            ev.append(((e0, e1, e2), dec_ms))
 
 
 def kernel_launches_per_step(wl):
     # reset (1) + compaction (decide, scan, scatter) + prefill attention (1)
-    # + per decode step: decide, append (one graph), split-K attention, combine (one graph)
-    return 1 + 3 + 1 + 4 * wl.decode_steps
+    # + per decode step: one fused kernel (decision logit, attention, combine, append)
+    return 1 + 3 + 1 + 1 * wl.decode_steps
 
 
 def visible_pairs(alpha, wl):
@@ -284,6 +287,9 @@ def run_ours(args, world, rank, local):
     r = Runner(B_, wl, seed=WL.seed + rank)
     # untimed pass: retained counts after each append (identical in every step)
     counts = []
+    r.cache.reset()
+    B_.dms_prefill(r.cache.handle, 0, r.pargs)
+    counts_prefill = r.cache.state(0)["count"].sum().item()
     r.step(counts=counts)
     torch.cuda.synchronize()
     assert r.cache.status() == 0
@@ -311,15 +317,12 @@ def run_ours(args, world, rank, local):
     barrier(world)
     region_ms = t0.elapsed_time(t1)
 
-    compact_ms = prefill_attn_ms = append_ms = attn_ms = 0.0
-    for (e0, e1, e2), dec in evs:
+    compact_ms = prefill_attn_ms = decode_ms = 0.0
+    for (e0, e1, e2), dec_ms in evs:
         compact_ms += e0.elapsed_time(e1)
         prefill_attn_ms += e1.elapsed_time(e2)
-        for a, b_, c in dec:
-            append_ms += a.elapsed_time(b_)
-            attn_ms += b_.elapsed_time(c)
+        decode_ms += dec_ms
     K, S, B = args.steps, wl.decode_steps, wl.batch
-    decode_ms = append_ms + attn_ms
     prefill_ms = compact_ms + prefill_attn_ms
     hot_ms_per_step = (decode_ms + prefill_ms) / K
     # max over ranks of the device times
@@ -330,14 +333,21 @@ def run_ours(args, world, rank, local):
     value = dec_tokens / (decode_ms_max / 1e3)
     prefill_tps = K * B * wl.prompt * world / (prefill_ms_max / 1e3)
 
-    # algorithmic bytes of the decode attention (per launch: retained K/V, q, o, page table entries)
+    # algorithmic bytes of one fused decode step (one launch): the retained K/V
+    # the attention reads (before the append, plus the new row), q and o, the
+    # new K/V row written, the hidden row and W of the decision logits, and the
+    # page-table entries
     D, elem = wl.head_dim, 2
-    qo = 2 * B * wl.q_heads * D * elem
-    kv_bytes = [c * D * 2 * elem for c in counts]
-    pt = [-(-c // wl.block) * 4 for c in counts]  # upper bound folded per head below
-    attn_bytes = sum(kv + qo for kv in kv_bytes) + sum(pt)
-    attn_gbs = K * attn_bytes / (attn_ms / 1e3) / 1e9
+    BH = B * wl.kv_heads
+    per_step_fixed = (2 * B * wl.q_heads * D * elem            # q, o
+                      + 2 * BH * D * elem                      # new K/V rows read
+                      + 2 * BH * D * elem                      # new K/V rows written
+                      + B * wl.hidden * elem + wl.kv_heads * wl.hidden * elem + wl.hidden * elem)  # h, W, gamma
+    pre_counts = [counts_prefill] + counts[:-1]
+    step_bytes = [cp * D * 2 * elem + (-(-cp // wl.block)) * 4 + per_step_fixed for cp in pre_counts]
+    attn_bytes = sum(step_bytes)
     decode_gbs = K * attn_bytes / (decode_ms / 1e3) / 1e9
+    attn_gbs = decode_gbs
     prefill_flops = 4.0 * D * wl.gqa * pairs
     prefill_tflops = K * prefill_flops / (prefill_attn_ms / 1e3) / 1e12
     clocks = clk.summary()
@@ -348,7 +358,7 @@ def run_ours(args, world, rank, local):
         cpu = cpu_baseline(wl, args.cpu_seconds)
     roof = {"bound": "hbm", "achieved": round(attn_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(attn_gbs / pk["hbm_gbs"], 4), "traffic": None,
-            "kernel": "decode attention (split-K k_decode_attn + combine)",
+            "kernel": "fused decode step k_decode_attn<128,bf16,fused> (split-K attention, combine, append)",
             "algorithmic_bytes_per_launch": int(attn_bytes / S), "peak_source": pk_kind}
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -362,8 +372,6 @@ def run_ours(args, world, rank, local):
         "retained_kv_gbps": round(decode_gbs, 1),
         "retained_kv_frac_of_peak": round(decode_gbs / pk["hbm_gbs"], 4),
         "decode_ms_per_token_step": round(decode_ms / (K * S), 5),
-        "decode_attention_ms": round(attn_ms / (K * S), 5),
-        "decode_append_ms": round(append_ms / (K * S), 5),
         "prefill_tok_s": round(prefill_tps, 1),
         "prefill_ms": round(prefill_ms / K, 4),
         "prefill_compact_ms": round(compact_ms / K, 4),

@@ -34,6 +34,54 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Issue the TMA loads of one sub-tile (`rows` slots starting at pool row
+// `row0`, all inside one page) into a stage: K then V, 16-row boxes; bf16 rows
+// as 128-byte column halves with the 128-byte swizzle, FP8 rows unswizzled.
+// Called by one thread; completes on `bar` with the exact byte count.
+template <int D, bool FP8>
+__device__ __forceinline__ void issue_subtile(unsigned char* dst, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                              int row0, int rows, uint64_t* bar) {
+  using S = DecodeSmem<D, FP8>;
+  const int nbox = (rows + 15) / 16;
+  const uint32_t bytes = static_cast<uint32_t>(nbox * 16 * (FP8 ? D : 128) * (FP8 ? 1 : S::HALVES) * 2);
+  mbar_expect_tx(bar, bytes);
+  for (int bx = 0; bx < nbox; ++bx) {
+    if (FP8) {
+      tma_load_2d(dst + bx * 16 * D, kmap, 0, row0 + bx * 16, bar);
+      tma_load_2d(dst + S::TILE_RAW + bx * 16 * D, vmap, 0, row0 + bx * 16, bar);
+    } else {
+      for (int hf = 0; hf < S::HALVES; ++hf) {
+        tma_load_2d(dst + hf * kSub * 128 + bx * 16 * 128, kmap, hf * 64, row0 + bx * 16, bar);
+        tma_load_2d(dst + S::TILE_RAW + hf * kSub * 128 + bx * 16 * 128, vmap, hf * 64, row0 + bx * 16, bar);
+      }
+    }
+  }
+}
+
+// Widen a staged FP8 sub-tile (K then V, unswizzled rows of D codes) to bf16
+// codes (exact) in the 128-byte swizzled layout of `conv` (K then V).
+template <int D>
+__device__ __forceinline__ void widen_fp8_subtile(const unsigned char* raw, unsigned char* conv) {
+  constexpr int TILE_RAW = kSub * D, TILE_BF16 = kSub * D * 2, CH = D / 16;
+  for (int idx = threadIdx.x; idx < 2 * kSub * CH; idx += kThreads) {
+    const int which = idx / (kSub * CH);
+    const int rem = idx % (kSub * CH);
+    const int r = rem / CH, ch = rem % CH;  // 16 codes
+    const uint4 u = *reinterpret_cast<const uint4*>(raw + which * TILE_RAW + r * D + ch * 16);
+    const uint8_t* cb = reinterpret_cast<const uint8_t*>(&u);
+    uint32_t wds[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) wds[e] = pack_bf16(fp8_decode(cb[2 * e]), fp8_decode(cb[2 * e + 1]));
+    unsigned char* dstt = conv + which * TILE_BF16;
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      const int chunk = 2 * ch + hc;
+      *reinterpret_cast<uint4*>(dstt + (chunk / 8) * kSub * 128 + sw128(r, chunk % 8)) =
+          make_uint4(wds[4 * hc], wds[4 * hc + 1], wds[4 * hc + 2], wds[4 * hc + 3]);
+    }
+  }
+}
+
 // Per-CTA work partition of one layer's decode attention, identical in every
 // CTA: chunk C = the largest power-of-two divisor of P (>= 16) giving at least
 // `target` items; item j of head bh covers slots [j*C, min(count, (j+1)*C)),
@@ -99,11 +147,13 @@ __device__ __forceinline__ void load_q_frags(const __nv_bfloat16* qb, int g, uin
 // One warp's online-softmax update over keys warp*16 .. warp*16+15 of a
 // staged sub-tile (bf16, 128-byte swizzled, column halves of 64 elements).
 // Keys >= rows and key `masked` are excluded.  Scores are in the log2 domain:
-// s = q.k * kscale * log2(e) / sqrt(D).
+// s = q.k * kscale * log2(e) / sqrt(D).  The probabilities entering PV are
+// multiplied by `vscale` (the FP8 page scale of V; 1 for bf16 pages), the row
+// sums are not.
 template <int D>
 __device__ __forceinline__ void warp_tile(const unsigned char* kt, const unsigned char* vt, int rows, int masked,
-                                          float kscale_l2, const uint32_t (&qa)[D / 16][4], float (&acc)[D / 8][4],
-                                          float (&mrow)[2], float (&lrow)[2]) {
+                                          float kscale_l2, float vscale, const uint32_t (&qa)[D / 16][4],
+                                          float (&acc)[D / 8][4], float (&mrow)[2], float (&lrow)[2]) {
   constexpr int KS = D / 16, NT = D / 8;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int mi = lane >> 3, rr = lane & 7;
@@ -157,10 +207,10 @@ __device__ __forceinline__ void warp_tile(const unsigned char* kt, const unsigne
     acc[nt][3] *= corr[1];
   }
   uint32_t pa[4];
-  pa[0] = pack_bf16(s[0][0], s[0][1]);
-  pa[1] = pack_bf16(s[0][2], s[0][3]);
-  pa[2] = pack_bf16(s[1][0], s[1][1]);
-  pa[3] = pack_bf16(s[1][2], s[1][3]);
+  pa[0] = pack_bf16(s[0][0] * vscale, s[0][1] * vscale);
+  pa[1] = pack_bf16(s[0][2] * vscale, s[0][3] * vscale);
+  pa[2] = pack_bf16(s[1][0] * vscale, s[1][1] * vscale);
+  pa[3] = pack_bf16(s[1][2] * vscale, s[1][3] * vscale);
 #pragma unroll
   for (int dp = 0; dp < NT / 2; ++dp) {
     const int n_row = warp * 16 + (mi & 1) * 8 + rr;
@@ -212,11 +262,11 @@ __device__ __forceinline__ void warp_state_to_smem(float* merge, int src, int g,
   }
 }
 
-// Merge `nsrc` staged states per row and write the item's partial (acc scaled
-// by vscale, running max, running sum) to global memory.
-template <int D>
-__device__ __forceinline__ void merge_to_partial(const float* merge, int nsrc, int g, float vscale, float* part_acc,
-                                                 float* part_ml, long item) {
+// Merge `nsrc` staged states per row into (acc scaled by vscale, running max,
+// running sum) and hand each value to store(r, d, value) with d in [0, D + 1]
+// (d == D: the max, d == D + 1: the sum).
+template <int D, typename Store>
+__device__ __forceinline__ void merge_sources(const float* merge, int nsrc, int g, float vscale, Store store) {
   constexpr int MLD = D + 2;
   for (int idx = threadIdx.x; idx < g * (D + 1); idx += kThreads) {
     const int r = idx / (D + 1), d = idx % (D + 1);
@@ -229,12 +279,24 @@ __device__ __forceinline__ void merge_to_partial(const float* merge, int nsrc, i
       sum += f * merge[(sv * g + r) * MLD + (d < D ? d : D + 1)];
     }
     if (d < D) {
-      part_acc[(item * g + r) * D + d] = sum * vscale;
+      store(r, d, sum * vscale);
     } else {
-      part_ml[(item * g + r) * 2] = M;
-      part_ml[(item * g + r) * 2 + 1] = sum;
+      store(r, D, M);
+      store(r, D + 1, sum);
     }
   }
+}
+
+// ... into an item's partial in global scratch.
+template <int D>
+__device__ __forceinline__ void merge_to_global(const float* merge, int nsrc, int g, float vscale, float* part_acc,
+                                                float* part_ml, long item) {
+  merge_sources<D>(merge, nsrc, g, vscale, [&](int r, int d, float v) {
+    if (d < D)
+      part_acc[(item * g + r) * D + d] = v;
+    else
+      part_ml[(item * g + r) * 2 + (d - D)] = v;
+  });
 }
 
 // LSE combine of a head's partials (items i0..i1) by one CTA:
@@ -337,6 +399,86 @@ __device__ void combine_head(const float* part_acc, const float* part_ml, int g,
     pk.y = pack_bf16(accv[k].z * inv, accv[k].w * inv);
     *reinterpret_cast<uint2*>(out + static_cast<long>(r) * D + d4 * 4) = pk;
   }
+}
+
+// Adapter decision logit of the new token of sequence b for head `src`, by one
+// CTA of kThreads (all loads of a thread issued before use; bf16 operands).
+// `red` holds 8 floats.  Returns the value in thread 0.
+template <int VPT>
+__device__ __forceinline__ float decide_cta(const CacheView& c, const DecideArgs& a, int b, int src, float* red) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int hid = c.hidden, nvec = hid / 8;
+  const uint4* xr =
+      reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.hidden) + static_cast<long>(b) * hid);
+  const uint4* wr =
+      reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.W) + static_cast<long>(src) * hid);
+  const uint4* gr = reinterpret_cast<const uint4*>(a.gamma);
+  float ss = 0.f, dot = 0.f;
+  for (int v0 = 0; v0 < nvec; v0 += kThreads * VPT) {
+    uint4 xu[VPT], wu[VPT], gu[VPT];
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      const int vi = v0 + u * kThreads + tid;
+      const bool ok = vi < nvec;
+      xu[u] = ok ? xr[vi] : make_uint4(0, 0, 0, 0);
+      wu[u] = ok ? wr[vi] : make_uint4(0, 0, 0, 0);
+      gu[u] = ok ? gr[vi] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      float x[8], wv[8], gv[8];
+      unpack16(xu[u], x, static_cast<const __nv_bfloat16*>(nullptr));
+      unpack16(wu[u], wv, static_cast<const __nv_bfloat16*>(nullptr));
+      unpack16(gu[u], gv, static_cast<const __nv_bfloat16*>(nullptr));
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        ss = fmaf(x[e], x[e], ss);
+        dot = fmaf(wv[e] * gv[e], x[e], dot);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  }
+  __syncthreads();
+  if (lane == 0) {
+    red[wid] = ss;
+    red[4 + wid] = dot;
+  }
+  __syncthreads();
+  float alpha = 0.f;
+  if (tid == 0) {
+    const float s2 = red[0] + red[1] + red[2] + red[3];
+    const float d2 = red[4] + red[5] + red[6] + red[7];
+    const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+    const float inv = 1.0f / sqrtf(s2 / static_cast<float>(hid) + c.rms_eps);
+    const float z = d2 * inv + (bias ? __bfloat162float(bias[src]) : 0.f);
+    alpha = z * c.alpha_scale - a.offset[b * a.offset_bstride + src];
+  }
+  return alpha;
+}
+
+// Distributed shared memory (thread-block clusters).
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+// Address of `p` (this CTA's shared memory) in the shared memory of cluster rank `rank`.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 // Slot plan of the next append of head i of `layer` (token position t):

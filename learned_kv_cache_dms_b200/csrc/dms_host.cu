@@ -75,7 +75,7 @@ Plan make_plan(const dms_cache_desc* d) {
   p.page_table = take(L * B * H * p.maxp * 4, 256);
   p.slot_pos = take(L * B * H * p.cap * 4, 256);
   p.ring = take(L * B * H * d->window * 4, 256);
-  p.plan = take(L * B * H * 8, 256);
+  p.plan = take(2 * L * B * H * 8, 256);
   p.kept = take(B * H * d->max_positions * 4, 256);
   p.kept_count = take(B * H * 4, 256);
   p.kept_upto = take(B * H * (d->max_positions + 1) * 4, 256);
@@ -448,12 +448,20 @@ int dms_decode_attention(dms_cache* c, int layer, const void* q, void* o, void* 
 
 int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* stream) {
   if (!c || !a || !a->o) return DMS_ERR_INVALID;
-  if (c->desc.kv_dtype != DMS_BF16) {
-    // FP8 pages re-encode a page before the attention may read it, and fp32
-    // pages use the CUDA-core path: append, then attend.
+  if (c->desc.kv_dtype == DMS_F32) {
     int e = dms_decode_append(c, layer, a, stream);
     if (e) return e;
     return dms_decode_attention(c, layer, a->q, a->o, stream);
+  }
+  if (c->desc.kv_dtype == DMS_FP8_E4M3) {
+    // FP8 pages may be re-encoded by the append, so the attention follows it:
+    // the append kernel, then the cluster attention over the updated pages.
+    int e = dms_decode_append(c, layer, a, stream);
+    if (e) return e;
+    return launch_decode_cluster(c->view, layer, a->q, a->o, false, nullptr, nullptr, nullptr, nullptr, &c->kmap,
+                                 &c->vmap, c->num_sms, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? DMS_OK
+               : DMS_ERR_CUDA;
   }
   if (layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
   if (!a->q || !a->k || !a->v || !a->alpha) return DMS_ERR_INVALID;
@@ -475,10 +483,10 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   DecideArgs da{};
   const bool proj = a->decide && !neuron;
   if (proj) da = decide_args(a->decide);
-  // One launch: attention over the pre-append slots plus the new token, then
-  // the append, with the adapter's decision logits computed inside.
-  if (launch_decode_fused(v, layer, a->q, a->k, a->v, a->o, a->alpha, proj ? &da : nullptr, &c->kmap, &c->vmap,
-                          c->num_sms, s) != cudaSuccess)
+  // bf16 pages: one launch -- attention over the pre-append slots plus the new
+  // token, then the append, with the adapter's decision logits computed inside.
+  if (launch_decode_cluster(v, layer, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, &c->kmap,
+                            &c->vmap, c->num_sms, s) != cudaSuccess)
     return DMS_ERR_CUDA;
   c->positions[layer] += 1;
   c->worklist_layer = layer;

@@ -19,6 +19,7 @@ enum Ctrl {
   CTRL_NEXT_PAGE = 1,    // next page id the ascending counter hands out
   CTRL_DONE_SCAN = 2,    // arrival counter of the prefill scan CTAs
   CTRL_GRID_DONE = 3,    // arrival counter of the fused decode CTAs
+  CTRL_STEP_PAGES = 4,   // pages granted by the running fused decode step
   CTRL_WORDS = 64
 };
 
@@ -35,7 +36,7 @@ struct CacheView {
   int* page_table;  // [L,B,Hkv,maxp]
   int* slot_pos;    // [L,B,Hkv,cap]
   int* ring;        // [L,B,Hkv,w]
-  int2* plan;       // [L,B,Hkv] slot plan of the next append (see next_plan)
+  int2* plan;       // [2][L,B,Hkv] slot plan of the next append, by parity of its position (next_plan)
   int* kept;        // [B,Hkv,max_pos]   prefill scratch: kept positions, ascending
   int* kept_count;  // [B,Hkv]
   int* kept_upto;   // [B,Hkv,max_pos+1] prefill scratch: kept tokens before position t
@@ -56,6 +57,13 @@ constexpr int RING_SLOT_MASK = 0x7FFFFFFF;
 constexpr long long kSpinLimit = 1ll << 26;
 
 __device__ __forceinline__ void set_status(int* ctrl, int bits) { atomicOr(&ctrl[CTRL_STATUS], bits); }
+
+// Plan entry of head li for the append of the token at position t (the plan is
+// double-buffered by the parity of t so one decode step can read its own plan
+// while writing the next one).
+__device__ __forceinline__ int2* plan_at(const CacheView& c, long li, int t) {
+  return c.plan + static_cast<long>(t & 1) * c.L * c.B * c.Hkv + li;
+}
 
 // Phase timeline (tracing builds only, compiled with -DDMS_TRACE): thread 0 of
 // each CTA stores %globaltimer for phase `slot` of kernel `kid` into a
@@ -273,8 +281,8 @@ cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, c
 cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q, void* o,
                                     const CUtensorMap* kmap, const CUtensorMap* vmap, int num_sms,
                                     cudaStream_t s);
-cudaError_t launch_decode_fused(const CacheView& c, int layer, const void* q, const void* k, const void* v, void* o,
-                                float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
-                                const CUtensorMap* vmap, int num_sms, cudaStream_t s);
+cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
+                                  const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
+                                  const CUtensorMap* vmap, int num_sms, cudaStream_t s);
 
 }  // namespace dms

@@ -23,6 +23,7 @@ __global__ void k_init(CacheView c) {
       c.npages[i] = c.pre_pages;
       c.count[i] = 0;
       c.plan[i] = make_int2(0, 0);
+      c.plan[nbh + i] = make_int2(0, 0);
     }
     if (i < static_cast<long>(c.B) * c.Hkv) c.head_done[i] = 0;
     if (i < static_cast<long>(c.L) * c.B) c.pos[i] = 0;

@@ -138,7 +138,10 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
   }
   // slot plan of the first decode append (token T) of every head
   __syncthreads();
-  for (int i = tid; i < BH; i += bd) c.plan[static_cast<long>(layer) * BH + i] = next_plan(c, static_cast<long>(layer) * BH + i, T);
+  for (int i = tid; i < BH; i += bd) {
+    const long li = static_cast<long>(layer) * BH + i;
+    *plan_at(c, li, T) = next_plan(c, li, T);
+  }
 }
 
 cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T, const float* alpha, cudaStream_t s) {
