@@ -110,32 +110,25 @@ __global__ void __launch_bounds__(128) k_attn_prefill_bf16(CacheView c, int T, c
   }
   cp_async_commit();
 
+  // Two threads per key row: the row's position is read once, then each thread
+  // issues its half of the row's 16-byte copies.
   auto load_tile = [&](int tile, int buf) {
-    // key positions of this tile
-    for (int n = tid; n < kBN; n += 128) {
-      int j;
-      if (tile < n_kept_tiles) {
-        const int idx = tile * kBN + n;
-        j = idx < nk ? kept[idx] : -1;
-      } else {
-        const int jj = jlo + (tile - n_kept_tiles) * kBN + n;
-        j = jj <= jhi ? jj : -1;
-      }
-      sm.kpos[buf][n] = j;
+    const int n = tid >> 1, part = tid & 1;
+    int j;
+    if (tile < n_kept_tiles) {
+      const int kidx = tile * kBN + n;
+      j = kidx < nk ? kept[kidx] : -1;
+    } else {
+      const int jj = jlo + (tile - n_kept_tiles) * kBN + n;
+      j = jj <= jhi ? jj : -1;
     }
-    for (int idx = tid; idx < kBN * CPR; idx += 128) {
-      const int n = idx / CPR, ch = idx % CPR;
-      int j;
-      if (tile < n_kept_tiles) {
-        const int kidx = tile * kBN + n;
-        j = kidx < nk ? kept[kidx] : -1;
-      } else {
-        const int jj = jlo + (tile - n_kept_tiles) * kBN + n;
-        j = jj <= jhi ? jj : -1;
-      }
-      const long off = static_cast<long>(max(j, 0)) * kv_row_stride + ch * 8;
-      cp_async16_zfill(&sm.k[buf][n * LD + ch * 8], kbase + off, j >= 0);
-      cp_async16_zfill(&sm.v[buf][n * LD + ch * 8], vbase + off, j >= 0);
+    if (part == 0) sm.kpos[buf][n] = j;
+    const long off = static_cast<long>(max(j, 0)) * kv_row_stride;
+#pragma unroll
+    for (int cc = 0; cc < CPR / 2; ++cc) {
+      const int ch = part * (CPR / 2) + cc;
+      cp_async16_zfill(&sm.k[buf][n * LD + ch * 8], kbase + off + ch * 8, j >= 0);
+      cp_async16_zfill(&sm.v[buf][n * LD + ch * 8], vbase + off + ch * 8, j >= 0);
     }
     cp_async_commit();
   };
@@ -308,6 +301,10 @@ cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, c
                                             static_cast<const float*>(v), static_cast<float*>(o));
     return cudaGetLastError();
   }
+  // bf16: the tcgen05 kernel; shapes it does not cover (g not a power of two
+  // up to 16) take the mma.sync kernel
+  const cudaError_t e = launch_prefill_attention_tc(c, T, q, k, v, o, s);
+  if (e != cudaErrorNotSupported) return e;
   return c.D == 64 ? launch_bf16<64>(c, T, q, k, v, o, s) : launch_bf16<128>(c, T, q, k, v, o, s);
 }
 
