@@ -20,7 +20,7 @@ constexpr int kMaxSmsForWork = 160;  // bound used to size the decode work list
 constexpr int kFuseDecideHeads = 64;  // decode decisions fused into the append up to B*Hkv heads
 
 struct Plan {
-  size_t ctrl, pos, count, npages, page_table, slot_pos, ring, plan, kept, kept_count, kept_upto, head_done, part_acc,
+  size_t ctrl, pos, count, npages, page_table, slot_pos, ring, plan, kept, kept_count, kept_upto, kept_k, kept_v, head_done, part_acc,
       part_ml, k_scale, v_scale, k_pool, v_pool, total;
   int maxp, cap, pre_pages, items_cap, first_free;
 };
@@ -79,6 +79,9 @@ Plan make_plan(const dms_cache_desc* d) {
   p.kept = take(B * H * d->max_positions * 4, 256);
   p.kept_count = take(B * H * 4, 256);
   p.kept_upto = take(B * H * (d->max_positions + 1) * 4, 256);
+  const size_t kept_rows_bytes = d->act_dtype == DMS_BF16 ? B * H * d->max_positions * d->head_dim * 2 : 0;
+  p.kept_k = take(kept_rows_bytes, 1024);
+  p.kept_v = take(kept_rows_bytes, 1024);
   p.head_done = take(B * H * 4, 256);
   p.part_acc = take(static_cast<size_t>(p.items_cap) * g * d->head_dim * 4, 256);
   p.part_ml = take(static_cast<size_t>(p.items_cap) * g * 2 * 4, 256);
@@ -124,6 +127,19 @@ bool make_pool_map(CUtensorMap* map, void* base, const dms_cache_desc* d) {
   return r == CUDA_SUCCESS;
 }
 
+// Generic bf16 tensor map with the 128-byte swizzle: dims/strides innermost
+// first (strides in bytes for dims 1..rank-1).
+bool make_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                   const cuuint32_t* box) {
+  auto enc = tensor_map_encoder();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 struct dms_cache {
@@ -138,6 +154,8 @@ struct dms_cache {
   std::vector<char> prefilled;
   CUtensorMap kmap, vmap;
   bool has_maps;
+  CUtensorMap kept_kmap, kept_vmap;  // tcgen05 prefill: kept copies
+  bool has_kept_maps = false;
   int compacted_layer = -1;  // layer whose kept list the prefill attention may use
   int compacted_len = 0;
   int worklist_layer = -1;   // layer whose decode work list is current
@@ -233,6 +251,8 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   v.kept = reinterpret_cast<int*>(b + p.kept);
   v.kept_count = reinterpret_cast<int*>(b + p.kept_count);
   v.kept_upto = reinterpret_cast<int*>(b + p.kept_upto);
+  v.kept_k = desc->act_dtype == DMS_BF16 ? b + p.kept_k : nullptr;
+  v.kept_v = desc->act_dtype == DMS_BF16 ? b + p.kept_v : nullptr;
   v.head_done = reinterpret_cast<int*>(b + p.head_done);
   v.part_acc = reinterpret_cast<float*>(b + p.part_acc);
   v.part_ml = reinterpret_cast<float*>(b + p.part_ml);
@@ -251,6 +271,15 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
       delete c;
       return DMS_ERR_CUDA;
     }
+  }
+  if (desc->act_dtype == DMS_BF16) {
+    const int D = desc->head_dim;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D),
+                                static_cast<cuuint64_t>(desc->batch) * desc->num_kv_heads * desc->max_positions};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    const cuuint32_t box[2] = {64u, 128u};
+    c->has_kept_maps = make_bf16_map(&c->kept_kmap, v.kept_k, 2, dims, strides, box) &&
+                       make_bf16_map(&c->kept_vmap, v.kept_v, 2, dims, strides, box);
   }
   if (launch_init(v, true, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     delete c;
@@ -390,7 +419,25 @@ int dms_prefill_attention(dms_cache* c, int layer, const dms_prefill_args* a, vo
   int e = check_prefill(c, layer, a);
   if (e) return e;
   if (c->compacted_layer != layer || c->compacted_len != a->seq_len) return DMS_ERR_STATE;
-  if (launch_prefill_attention(c->view, a->seq_len, a->q, a->k, a->v, a->o, static_cast<cudaStream_t>(stream)) !=
+  // tensor maps of this call's q, k, v for the tcgen05 kernel
+  PrefillMaps maps{};
+  maps.valid = false;
+  const int g = c->desc.num_q_heads / c->desc.num_kv_heads;
+  if (c->has_kept_maps && g <= 16 && (g & (g - 1)) == 0) {
+    const int D = c->desc.head_dim, T = a->seq_len;
+    const cuuint64_t bt = static_cast<cuuint64_t>(c->desc.batch) * T;
+    const cuuint64_t qd[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(c->desc.num_q_heads), bt};
+    const cuuint64_t qs[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(c->desc.num_q_heads) * D * 2};
+    const cuuint32_t qb[3] = {64u, static_cast<cuuint32_t>(g), static_cast<cuuint32_t>(128 / g)};
+    const cuuint64_t kd[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(c->desc.num_kv_heads), bt};
+    const cuuint64_t ks[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(c->desc.num_kv_heads) * D * 2};
+    const cuuint32_t kbx[3] = {64u, 1u, 128u};
+    maps.valid = make_bf16_map(&maps.q, a->q, 3, qd, qs, qb) && make_bf16_map(&maps.k, a->k, 3, kd, ks, kbx) &&
+                 make_bf16_map(&maps.v, a->v, 3, kd, ks, kbx);
+    maps.kept_k = c->kept_kmap;
+    maps.kept_v = c->kept_vmap;
+  }
+  if (launch_prefill_attention(c->view, a->seq_len, a->q, a->k, a->v, a->o, &maps, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return DMS_ERR_CUDA;
   return DMS_OK;

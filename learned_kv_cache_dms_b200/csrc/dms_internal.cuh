@@ -40,6 +40,8 @@ struct CacheView {
   int* kept;        // [B,Hkv,max_pos]   prefill scratch: kept positions, ascending
   int* kept_count;  // [B,Hkv]
   int* kept_upto;   // [B,Hkv,max_pos+1] prefill scratch: kept tokens before position t
+  void* kept_k;     // [B*Hkv, max_pos, D] prefill scratch (bf16 activations): kept keys in list order
+  void* kept_v;     //                      and values
   int* head_done;   // [B*Hkv] arrival counters of the attention CTAs (self-resetting)
   float* part_acc;  // [items_cap, g, D]   decode split-K partials, indexed by work item
   float* part_ml;   // [items_cap, g, 2]  (running max, running sum)
@@ -347,12 +349,16 @@ cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, vo
 cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T, const float* alpha, cudaStream_t s);
 cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T, const void* k, const void* v,
                                    cudaStream_t s);
+// Tensor maps of the tcgen05 prefill attention: q [B*T, Hq, D] (box 64 x g x 128/g),
+// k and v [B*T, Hkv, D] (box 64 x 1 x 128), kept copies [B*Hkv*max_pos, D] (box 64 x 128),
+// all bf16 with the 128-byte swizzle.  `valid` is false when the shape is not covered.
+struct PrefillMaps {
+  CUtensorMap q, k, v, kept_k, kept_v;
+  bool valid;
+};
 cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, const void* k, const void* v,
-                                     void* o, cudaStream_t s);
-// tcgen05 version (bf16, g = Hq/Hkv a power of two <= 16); returns
-// cudaErrorNotSupported for shapes it does not cover.
-cudaError_t launch_prefill_attention_tc(const CacheView& c, int T, const void* q, const void* k, const void* v,
-                                        void* o, cudaStream_t s);
+                                     void* o, const PrefillMaps* maps, cudaStream_t s);
+cudaError_t launch_prefill_attention_tc(const CacheView& c, int T, void* o, const PrefillMaps& maps, cudaStream_t s);
 cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, const void* v, float* alpha,
                                  const DecideArgs* fused_decide, int num_sms, cudaStream_t s);
 cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q, void* o,

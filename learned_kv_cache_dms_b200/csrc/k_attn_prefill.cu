@@ -293,7 +293,7 @@ static cudaError_t launch_bf16(const CacheView& c, int T, const void* q, const v
 }
 
 cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, const void* k, const void* v,
-                                     void* o, cudaStream_t s) {
+                                     void* o, const PrefillMaps* maps, cudaStream_t s) {
   if (c.act_dtype == DMS_F32) {
     const long nrows = static_cast<long>(c.B) * T * c.Hq;
     const int grid = static_cast<int>((nrows * 32 + 255) / 256);
@@ -302,9 +302,8 @@ cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, c
     return cudaGetLastError();
   }
   // bf16: the tcgen05 kernel; shapes it does not cover (g not a power of two
-  // up to 16) take the mma.sync kernel
-  const cudaError_t e = launch_prefill_attention_tc(c, T, q, k, v, o, s);
-  if (e != cudaErrorNotSupported) return e;
+  // up to 16, or inputs not 16-byte aligned for TMA) take the mma.sync kernel
+  if (maps && maps->valid) return launch_prefill_attention_tc(c, T, o, *maps, s);
   return c.D == 64 ? launch_bf16<64>(c, T, q, k, v, o, s) : launch_bf16<128>(c, T, q, k, v, o, s);
 }
 

@@ -19,8 +19,10 @@
 //               O is rescaled rarely (the final O / l is exact either way).
 //   O += P V  : P (bf16, K-major) written to shared memory by the softmax
 //               threads, V staged as MN-major B, O in TMEM columns [128, 128+D)
-// K/V tiles are double-buffered with cp.async (row gathers for the kept list);
-// the next tile's loads overlap the softmax and the P V product.
+// Tiles arrive by TMA (no multicast): band keys/values straight from the input
+// rows, kept ones from the position-sorted kept copy written by the
+// compaction.  Two K/V stages and two S buffers let S(t+1) run on the tensor
+// cores while the softmax of tile t runs; mbarriers order loads, S, and P V.
 #include "dms_internal.cuh"
 
 namespace dms {
@@ -47,7 +49,7 @@ struct TcSmem {
   static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;  // 2 stages
   static constexpr int OFF_P = OFF_V + 2 * KV_BYTES;
   static constexpr int BYTES = OFF_P + P_BYTES;
-  static constexpr uint32_t TMEM_COLS = 256;  // S: 128 columns, O: D columns
+  static constexpr uint32_t TMEM_COLS = 512;  // S double buffer: 2 x 128 columns, O: D columns at 256
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
@@ -73,10 +75,21 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
+// 3-D TMA tile load (no multicast).
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];\n" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    k_attn_prefill_tc(CacheView c, int T, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                      __nv_bfloat16* o) {
+    k_attn_prefill_tc(CacheView c, int T, __nv_bfloat16* o, const __grid_constant__ CUtensorMap qmap,
+                      const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                      const __grid_constant__ CUtensorMap kkmap, const __grid_constant__ CUtensorMap kvmap) {
   using L = TcSmem<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sb = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -87,7 +100,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ float s_lpart[kTcRows];
   __shared__ float s_lsum[kTcRows];
   __shared__ uint32_t tmem_base;
-  __shared__ __align__(8) uint64_t bar_mma;
+  __shared__ __align__(8) uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_pv;
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -99,32 +112,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int h = blockIdx.y, b = blockIdx.z, w = c.w;
   const int i0 = qb * NP, i1 = min(T, i0 + NP);
   const int bh = b * c.Hkv + h;
-  const long kv_row = static_cast<long>(c.Hkv) * D;  // elements between consecutive positions
-  const __nv_bfloat16* kb = k + static_cast<long>(b) * T * kv_row + static_cast<long>(h) * D;
-  const __nv_bfloat16* vb = v + static_cast<long>(b) * T * kv_row + static_cast<long>(h) * D;
   const int* kept = c.kept + static_cast<long>(bh) * c.max_pos;
   const int nk = (i1 - w > 0) ? c.kept_upto[static_cast<long>(bh) * (c.max_pos + 1) + (i1 - w)] : 0;
   const int jlo = max(0, i0 - w + 1), jhi = i1 - 1;
   const int n_kept_tiles = (nk + kTcBN - 1) / kTcBN;
   const int ntiles = n_kept_tiles + (jhi - jlo + kTcBN) / kTcBN;
-
   const int i_row = i0 + row / g, r_row = row % g;
-
-  if (tid == 0) {
-    mbar_init(&bar_mma, 1);
-    fence_mbar_init();
-    s_abort = 0;
-  }
-  if (warp == 0) tmem_alloc(&tmem_base, L::TMEM_COLS);
-
-  // Q rows: 128 x D, K-major, 128-byte swizzle per 64-element half
-  constexpr int CPR = D / 8;  // 16-byte chunks per row
-  for (int idx = tid; idx < kTcRows * CPR; idx += kTcThreads) {
-    const int t = idx / CPR, ch = idx % CPR;
-    const int i = i0 + t / g, hq = h * g + t % g;
-    const __nv_bfloat16* src = q + ((static_cast<long>(b) * T + min(i, T - 1)) * c.Hq + hq) * D + ch * 8;
-    cp_async16_zfill(sQ + (ch / 8) * (kTcRows * 128) + swz(t, ch % 8), src, i < T);
-  }
 
   // position of key row `row` of a tile (-1: absent)
   auto key_pos = [&](int tile) -> int {
@@ -135,76 +128,99 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int jj = jlo + (tile - n_kept_tiles) * kTcBN + row;
     return jj <= jhi ? jj : -1;
   };
-  // Two threads per key row (one per half of its 16-byte chunks).
-  auto load_tile = [&](int st, int j) {
-    unsigned char* sK = sb + L::OFF_K + st * L::KV_BYTES;
-    unsigned char* sV = sb + L::OFF_V + st * L::KV_BYTES;
-    if (half == 0) kpos[st][row] = j;
-    const __nv_bfloat16* ks = kb + static_cast<long>(max(j, 0)) * kv_row;
-    const __nv_bfloat16* vs = vb + static_cast<long>(max(j, 0)) * kv_row;
-#pragma unroll
-    for (int cc = 0; cc < CPR / 2; ++cc) {
-      const int ch = half * (CPR / 2) + cc;
-      const uint32_t dst = (ch / 8) * (kTcBN * 128) + swz(row, ch % 8);
-      cp_async16_zfill(sK + dst, ks + ch * 8, j >= 0);
-      cp_async16_zfill(sV + dst, vs + ch * 8, j >= 0);
+  // TMA loads of a tile's keys or values into stage `st` (thread 0): band
+  // tiles straight from the input rows, kept tiles from the kept copy
+  auto load_kv = [&](int tile, int st, bool is_v) {
+    unsigned char* dst = sb + (is_v ? L::OFF_V : L::OFF_K) + st * L::KV_BYTES;
+    uint64_t* bar = is_v ? &bar_v[st] : &bar_k[st];
+    mbar_expect_tx(bar, L::KV_BYTES);
+    for (int hf = 0; hf < L::HALVES; ++hf) {
+      if (tile < n_kept_tiles)
+        tma_load_2d(dst + hf * (kTcBN * 128), is_v ? &kvmap : &kkmap, hf * 64, bh * c.max_pos + tile * kTcBN, bar);
+      else
+        tma_load_3d(dst + hf * (kTcBN * 128), is_v ? &vmap : &kmap, hf * 64, h,
+                    b * T + jlo + (tile - n_kept_tiles) * kTcBN, bar);
     }
-    cp_async_commit();
   };
 
-  load_tile(0, key_pos(0));
+  if (tid == 0) {
+    mbar_init(&bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_k[i], 1);
+      mbar_init(&bar_v[i], 1);
+      mbar_init(&bar_s[i], 1);
+    }
+    mbar_init(&bar_pv, 1);
+    fence_mbar_init();
+    s_abort = 0;
+    mbar_expect_tx(&bar_q, L::Q_BYTES);
+    for (int hf = 0; hf < L::HALVES; ++hf) tma_load_3d(sQ + hf * (kTcRows * 128), &qmap, hf * 64, h * g, b * T + i0, &bar_q);
+    load_kv(0, 0, false);
+    load_kv(0, 0, true);
+    if (ntiles > 1) {
+      load_kv(1, 1, false);
+      load_kv(1, 1, true);
+    }
+  }
+  if (warp == 0) tmem_alloc(&tmem_base, L::TMEM_COLS);
+  if (half == 0) kpos[0][row] = key_pos(0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
   const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const uint32_t tmem_s = tmem + lane_off + half * 64;               // this thread's 64 score columns
-  const uint32_t tmem_o = tmem + lane_off + kTcBN + half * (D / 2);  // this thread's D/2 output columns
+  const uint32_t tmem_o = tmem + lane_off + 256 + half * (D / 2);  // this thread's D/2 output columns
   constexpr uint32_t IDESC_S = umma_idesc_bf16(128, kTcBN, 0);
   constexpr uint32_t IDESC_O = umma_idesc_bf16(128, D, 1);
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
   float m_ref = -INFINITY, l_part = 0.f;
-  uint32_t phase = 0;
+
+  // S(t) = Q K(t)^T into TMEM buffer t & 1 (thread 0)
+  auto issue_s = [&](int tile) -> bool {
+    const int st = tile & 1;
+    if (!mbar_wait_bounded(&bar_k[st], (tile >> 1) & 1)) return false;
+    tc_fence_after();
+    const uint32_t qa = smem_u32(sQ), ka = smem_u32(sb + L::OFF_K + st * L::KV_BYTES);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t off = (ks / 4) * (kTcRows * 128) + (ks % 4) * 32;
+      const uint32_t koff = (ks / 4) * (kTcBN * 128) + (ks % 4) * 32;
+      umma_bf16(tmem + st * kTcBN, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(ka + koff, 16, 1024),
+                IDESC_S, ks > 0 ? 1u : 0u);
+    }
+    umma_commit(&bar_s[st]);
+    return true;
+  };
+  if (tid == 0) {
+    if (!mbar_wait_bounded(&bar_q, 0) || !issue_s(0)) {
+      set_status(c.ctrl, DMS_ST_TIMEOUT);
+      s_abort = 1;
+    }
+  }
 
   for (int tile = 0; tile < ntiles; ++tile) {
     const int st = tile & 1;
     const bool kept_tile = tile < n_kept_tiles;
-    // position of this thread's key row in the next tile: read now, used after the S wait
-    const int j_next = tile + 1 < ntiles ? key_pos(tile + 1) : -1;
+    const int j_next = tile + 1 < ntiles ? key_pos(tile + 1) : -1;  // read now, stored after the softmax
     TC_MARK(tile, 0);
-    cp_async_wait<0>();
-    fence_proxy_async();  // make the staged tiles visible to the tensor cores
-    __syncthreads();
-    TC_MARK(tile, 1);
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t qa = smem_u32(sQ), ka = smem_u32(sb + L::OFF_K + st * L::KV_BYTES);
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t off = (ks / 4) * (kTcRows * 128) + (ks % 4) * 32;
-        const uint32_t koff = (ks / 4) * (kTcBN * 128) + (ks % 4) * 32;
-        umma_bf16(tmem, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(ka + koff, 16, 1024), IDESC_S,
-                  ks > 0 ? 1u : 0u);
-      }
-      umma_commit(&bar_mma);  // also covers the previous tile's P V
+    // next S on the tensor cores while this tile's softmax runs
+    if (tid == 0 && !s_abort && tile + 1 < ntiles && !issue_s(tile + 1)) {
+      set_status(c.ctrl, DMS_ST_TIMEOUT);
+      s_abort = 1;
     }
-    if (!mbar_wait_bounded(&bar_mma, phase)) {
+    if (!mbar_wait_bounded(&bar_s[st], (tile >> 1) & 1)) {
       if (tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
       s_abort = 1;
     }
-    phase ^= 1;
-    __syncthreads();
-    if (s_abort) break;
     tc_fence_after();
     TC_MARK(tile, 2);
-    // the other stage is free (its S and P V are complete): prefetch the next tile
-    if (tile + 1 < ntiles) load_tile(st ^ 1, j_next);
-    TC_MARK(tile, 5);
+    // K stage st is free (S(tile) complete): fetch the keys of tile + 2
+    if (tid == 0 && tile + 2 < ntiles) load_kv(tile + 2, st, false);
 
     // ---- softmax: this thread's 64 scores of row `row` ----
     uint32_t sr[64];
-    tmem_ld32_nowait(tmem_s, sr);
-    tmem_ld32_nowait(tmem_s + 32, sr + 32);
+    tmem_ld32_nowait(tmem + lane_off + st * kTcBN + half * 64, sr);
+    tmem_ld32_nowait(tmem + lane_off + st * kTcBN + half * 64 + 32, sr + 32);
     tmem_wait_ld();
     TC_MARK(tile, 6);
     // visible: lo <= j <= hi (kept tile: 0 <= j <= i - w; band: i - w < j <= i); absent keys are -1
@@ -225,6 +241,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     s_tmax[half][row] = tmax;
     __syncthreads();
+    if (s_abort) break;
     tmax = fmaxf(s_tmax[0][row], s_tmax[1][row]);
     TC_MARK(tile, 7);
     // raise the reference only when this tile exceeds it by more than 2^8
@@ -236,20 +253,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       l_part *= factor;
     }
     const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a fully masked row so far: all p = 0
+    uint32_t pk[32];
     float psum = 0.f;
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      uint32_t pk[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float p0 = ex2_approx(x[ch * 8 + 2 * e] - m_use);
-        const float p1 = ex2_approx(x[ch * 8 + 2 * e + 1] - m_use);
-        psum += p0 + p1;
-        pk[e] = pack_bf16(p0, p1);
-      }
-      *reinterpret_cast<uint4*>(sP + half * (kTcRows * 128) + swz(row, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    for (int e = 0; e < 32; ++e) {
+      const float p0 = ex2_approx(x[2 * e] - m_use);
+      const float p1 = ex2_approx(x[2 * e + 1] - m_use);
+      psum += p0 + p1;
+      pk[e] = pack_bf16(p0, p1);
     }
     l_part += psum;
+    // P(tile - 1) V has finished with the P buffer, with O and with V stage st ^ 1
+    if (tile > 0 && !mbar_wait_bounded(&bar_pv, (tile - 1) & 1)) {
+      if (tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
+      s_abort = 1;
+    }
+    tc_fence_after();
+    if (tid == 0 && tile >= 1 && tile + 1 < ntiles) load_kv(tile + 1, st ^ 1, true);
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch)
+      *reinterpret_cast<uint4*>(sP + half * (kTcRows * 128) + swz(row, ch)) =
+          make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
     TC_MARK(tile, 8);
     // rescale this thread's half of O in tensor memory where the reference moved
     if (tile > 0 && __any_sync(0xffffffffu, raise && factor != 1.0f)) {
@@ -262,31 +286,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_st32(tmem_o + c0, ov);
       }
     }
+    if (half == 0) kpos[st ^ 1][row] = j_next;  // the next tile's key positions
     TC_MARK(tile, 3);
     fence_proxy_async();  // P visible to the tensor cores
     tc_fence_before();
     __syncthreads();
+    if (s_abort) break;
     if (tid == 0) {
-      tc_fence_after();
-      const uint32_t pa = smem_u32(sP), va = smem_u32(sb + L::OFF_V + st * L::KV_BYTES);
+      if (!mbar_wait_bounded(&bar_v[st], (tile >> 1) & 1)) {
+        set_status(c.ctrl, DMS_ST_TIMEOUT);
+        s_abort = 1;
+      } else {
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sP), va = smem_u32(sb + L::OFF_V + st * L::KV_BYTES);
 #pragma unroll
-      for (int ks = 0; ks < kTcBN / 16; ++ks) {
-        const uint32_t poff = (ks / 4) * (kTcRows * 128) + (ks % 4) * 32;
-        umma_bf16(tmem + kTcBN, umma_desc_sw128(pa + poff, 16, 1024),
-                  umma_desc_sw128(va + ks * 16 * 128, kTcBN * 128, 1024), IDESC_O, (tile > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kTcBN / 16; ++ks) {
+          const uint32_t poff = (ks / 4) * (kTcRows * 128) + (ks % 4) * 32;
+          umma_bf16(tmem + 256, umma_desc_sw128(pa + poff, 16, 1024),
+                    umma_desc_sw128(va + ks * 16 * 128, kTcBN * 128, 1024), IDESC_O, (tile > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(&bar_pv);
       }
     }
     TC_MARK(tile, 4);
   }
 
   // wait for the last P V, then write O / l (l = the two halves' partial sums)
-  if (tid == 0 && !s_abort) umma_commit(&bar_mma);
   if (half == 1) s_lpart[row] = l_part;
   __syncthreads();
   if (half == 0) s_lsum[row] = l_part + s_lpart[row];
   __syncthreads();
   if (!s_abort && ntiles > 0) {
-    if (!mbar_wait_bounded(&bar_mma, phase) && tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
+    if (!mbar_wait_bounded(&bar_pv, (ntiles - 1) & 1) && tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
     tc_fence_after();
     const float inv = s_lsum[row] > 0.f ? 1.f / s_lsum[row] : 0.f;
     __nv_bfloat16* orow = o + ((static_cast<long>(b) * T + i_row) * c.Hq + h * g + r_row) * D + half * (D / 2);
@@ -297,12 +328,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (i_row < T) {
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
-          uint4 pk;
-          pk.x = pack_bf16(ov[e] * inv, ov[e + 1] * inv);
-          pk.y = pack_bf16(ov[e + 2] * inv, ov[e + 3] * inv);
-          pk.z = pack_bf16(ov[e + 4] * inv, ov[e + 5] * inv);
-          pk.w = pack_bf16(ov[e + 6] * inv, ov[e + 7] * inv);
-          *reinterpret_cast<uint4*>(orow + c0 + e) = pk;
+          uint4 pkk;
+          pkk.x = pack_bf16(ov[e] * inv, ov[e + 1] * inv);
+          pkk.y = pack_bf16(ov[e + 2] * inv, ov[e + 3] * inv);
+          pkk.z = pack_bf16(ov[e + 4] * inv, ov[e + 5] * inv);
+          pkk.w = pack_bf16(ov[e + 6] * inv, ov[e + 7] * inv);
+          *reinterpret_cast<uint4*>(orow + c0 + e) = pkk;
         }
       }
     }
@@ -313,25 +344,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 template <int D>
-static cudaError_t launch_tc(const CacheView& c, int T, const void* q, const void* k, const void* v, void* o,
-                             cudaStream_t s) {
+static cudaError_t launch_tc(const CacheView& c, int T, void* o, const PrefillMaps& m, cudaStream_t s) {
   const size_t smem = TcSmem<D>::BYTES + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_attn_prefill_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int g = c.Hq / c.Hkv, NP = kTcRows / g;
   dim3 grid((T + NP - 1) / NP, c.Hkv, c.B);
-  k_attn_prefill_tc<D><<<grid, kTcThreads, smem, s>>>(c, T, static_cast<const __nv_bfloat16*>(q),
-                                                      static_cast<const __nv_bfloat16*>(k),
-                                                      static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o));
+  k_attn_prefill_tc<D><<<grid, kTcThreads, smem, s>>>(c, T, static_cast<__nv_bfloat16*>(o), m.q, m.k, m.v, m.kept_k,
+                                                      m.kept_v);
   return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_attention_tc(const CacheView& c, int T, const void* q, const void* k, const void* v,
-                                        void* o, cudaStream_t s) {
-  const int g = c.Hq / c.Hkv;
-  if (c.act_dtype != DMS_BF16 || g > 16 || (g & (g - 1)) != 0) return cudaErrorNotSupported;
-  return c.D == 64 ? launch_tc<64>(c, T, q, k, v, o, s) : launch_tc<128>(c, T, q, k, v, o, s);
+cudaError_t launch_prefill_attention_tc(const CacheView& c, int T, void* o, const PrefillMaps& maps, cudaStream_t s) {
+  return c.D == 64 ? launch_tc<64>(c, T, o, maps, s) : launch_tc<128>(c, T, o, maps, s);
 }
 
 }  // namespace dms

@@ -43,6 +43,10 @@ cudaError_t launch_init(const CacheView& c, bool full, cudaStream_t s) {
     const size_t pool_bytes = static_cast<size_t>(c.pool_pages) * c.P * c.D * eb;
     cudaError_t e = cudaMemsetAsync(c.k_pool, 0, pool_bytes, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(c.v_pool, 0, pool_bytes, s);
+    // the kept copies too: tiles read (and mask) rows past the kept count
+    const size_t kept_bytes = static_cast<size_t>(c.B) * c.Hkv * c.max_pos * c.D * 2;
+    if (e == cudaSuccess && c.kept_k) e = cudaMemsetAsync(c.kept_k, 0, kept_bytes, s);
+    if (e == cudaSuccess && c.kept_v) e = cudaMemsetAsync(c.kept_v, 0, kept_bytes, s);
     if (e != cudaSuccess) return e;
   }
   const long nbh = static_cast<long>(c.L) * c.B * c.Hkv;

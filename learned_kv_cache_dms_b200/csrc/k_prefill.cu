@@ -176,11 +176,22 @@ __global__ void __launch_bounds__(256) k_prefill_scatter(CacheView c, int layer,
   const int cpr = c.D / V;  // 16-byte chunks per row
   TA* kp = static_cast<TA*>(c.k_pool) + static_cast<long>(id) * c.P * c.D;
   TA* vp = static_cast<TA*>(c.v_pool) + static_cast<long>(id) * c.P * c.D;
+  const int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
   for (int idx = threadIdx.x; idx < rows * cpr; idx += blockDim.x) {
     const int r = idx / cpr, ch = idx % cpr;
-    const long src = ((static_cast<long>(b) * T + slot_pos[r]) * c.Hkv + h) * c.D;
-    reinterpret_cast<uint4*>(kp + static_cast<long>(r) * c.D)[ch] = reinterpret_cast<const uint4*>(k + src)[ch];
-    reinterpret_cast<uint4*>(vp + static_cast<long>(r) * c.D)[ch] = reinterpret_cast<const uint4*>(v + src)[ch];
+    const int t = slot_pos[r];
+    const long src = ((static_cast<long>(b) * T + t) * c.Hkv + h) * c.D;
+    const uint4 kq = reinterpret_cast<const uint4*>(k + src)[ch];
+    const uint4 vq = reinterpret_cast<const uint4*>(v + src)[ch];
+    reinterpret_cast<uint4*>(kp + static_cast<long>(r) * c.D)[ch] = kq;
+    reinterpret_cast<uint4*>(vp + static_cast<long>(r) * c.D)[ch] = vq;
+    if (sizeof(TA) == 2 && c.kept_k && t < T - c.w) {
+      // a kept token before the last window: also into the position-sorted
+      // kept copy read by the tcgen05 prefill attention
+      const long kr = (static_cast<long>(bh) * c.max_pos + kept_upto[t]) * c.D;
+      reinterpret_cast<uint4*>(static_cast<TA*>(c.kept_k) + kr)[ch] = kq;
+      reinterpret_cast<uint4*>(static_cast<TA*>(c.kept_v) + kr)[ch] = vq;
+    }
   }
 }
 
@@ -209,6 +220,19 @@ __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int la
   const int rows = min(c.P, cnt - p * c.P);
   const int* slot_pos = c.slot_pos + lbh * c.cap + static_cast<long>(p) * c.P;
   const int cpr = c.D / 8;  // 8 bf16 per 16-byte input chunk
+  if (c.kept_k) {
+    // kept tokens before the last window: into the position-sorted kept copy
+    const int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
+    for (int idx = threadIdx.x; idx < rows * cpr; idx += blockDim.x) {
+      const int r = idx / cpr, ch = idx % cpr;
+      const int t = slot_pos[r];
+      if (t >= T - c.w) continue;
+      const long src = ((static_cast<long>(b) * T + t) * c.Hkv + h) * c.D;
+      const long kr = (static_cast<long>(bh) * c.max_pos + kept_upto[t]) * c.D;
+      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.kept_k) + kr)[ch] = reinterpret_cast<const uint4*>(k + src)[ch];
+      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.kept_v) + kr)[ch] = reinterpret_cast<const uint4*>(v + src)[ch];
+    }
+  }
   for (int which = 0; which < 2; ++which) {
     const __nv_bfloat16* x = which ? v : k;
     float amax = 0.f;
