@@ -7,18 +7,23 @@ would run inside a whole-model graph.
 
 One bench step = one pass of the whole path over one batch: cache reset,
 prefill of the prompt (decision logits, compaction into pages, DMS-masked
-attention), then every decode step (decision logit, append with delayed
-eviction, split-K attention over the retained pages).  Workload: one Qwen3-8B
-attention layer (hidden 4096, 32 q / 8 kv heads, head_dim 128), batch 1,
-prompt 8192 + 128 decode steps, window 512, block 256, adapter decisions
-calibrated to keep 1/8 of the tokens outside the window; synthetic seeded bf16
-inputs resident in HBM.
+attention) in every layer, then every decode step (decision logit, append with
+delayed eviction, split-K attention over the retained pages) through the
+layer stack.  Default workload: one Qwen3-8B attention layer (hidden 4096,
+32 q / 8 kv heads, head_dim 128), batch 1, prompt 8192 + 128 decode steps,
+window 512, block 256, adapter decisions calibrated to keep 1/8 of the tokens
+outside the window; synthetic seeded bf16 inputs resident in HBM.  --workload
+selects the batch-8 Qwen3-8B layer, the FP8 Llama-3.2-1B layer (32K context,
+key-neuron decisions, rotary tables) or the 36-layer batch-32 stack.
 
-L2: the decode working set (~6 MB) fits in the 126 MB L2, so a 512 MB buffer
-is written before every decode step (outside the timed segments) and the KV
-bytes come from DRAM.  Times are CUDA events on the launching stream.
+L2: a single layer's decode working set (6-60 MB) fits in the 126 MB L2, so a
+512 MB buffer is written before every decode step (outside the timed
+segments) and the KV bytes come from DRAM; the 36-layer stack reads gigabytes
+per step and runs its steps back to back.  Times are CUDA events on the
+launching stream.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--decode-steps N]
 Multi-GPU (torchrun): every rank runs its own replica (independent sequences,
 weak scaling, no collective on the data path); rank 0 prints one JSON line.
 """
@@ -38,7 +43,6 @@ import torch  # noqa: E402
 
 from learned_kv_cache_dms_b200 import inputs as I  # noqa: E402
 
-WL = I.WORKLOADS["qwen8b"]
 METRIC = "DMS decode tok/s and retained-KV HBM GB/s (% of B200 peak), Qwen3-8B shape"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -52,6 +56,12 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiler runs)")
+    p.add_argument("--workload", choices=BENCH_WORKLOADS, default="qwen8b",
+                   help="qwen8b (default): one Qwen3-8B layer, batch 1; qwen8b_c8: batch 8; llama1b(_layer): "
+                        "FP8 pages, key-neuron decisions, 32K context; reason36: 36 layers, batch 32")
+    p.add_argument("--decode-steps", type=int, default=None, help="decode only the first N steps")
+    p.add_argument("--decode-kernel", choices=["auto", "cluster", "flat"], default="auto",
+                   help="decode attention kernel (auto: by the number of heads)")
     return p.parse_args()
 
 
@@ -145,126 +155,232 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------
-def make_desc(B_, wl):
+BENCH_WORKLOADS = ("qwen8b", "qwen8b_c8", "llama1b", "llama1b_layer", "reason36")
+STEP_POOL = 64  # distinct decode-token inputs per layer of a multi-layer stack (cycled)
+
+
+def workload_label(wl, n_dec):
+    if wl.name == "qwen8b" and n_dec == wl.decode_steps:
+        return "qwen8b_layer_b1_ctx8192_dec128"
+    return "%s_L%d_b%d_ctx%d_dec%d_%s" % (wl.name, wl.layers, wl.batch, wl.prompt, n_dec, wl.kv_dtype)
+
+
+def make_desc(B_, wl, kernel="auto"):
     d = B_.dms_cache_desc_default()
+    d.decode_kernel = {"auto": B_.DMS_DECODE_AUTO, "cluster": B_.DMS_DECODE_CLUSTER,
+                       "flat": B_.DMS_DECODE_FLAT}[kernel]
     d.num_layers, d.batch, d.num_q_heads, d.num_kv_heads = wl.layers, wl.batch, wl.q_heads, wl.kv_heads
     d.head_dim, d.hidden, d.window, d.block = wl.head_dim, wl.hidden, wl.window, wl.block
     d.max_positions, d.prealloc_tokens = wl.max_positions, wl.prealloc_tokens
     maxp = -(-wl.max_positions // wl.block)
-    d.pool_pages = wl.layers * wl.batch * wl.kv_heads * maxp
+    pre = min(maxp, -(-wl.prealloc_tokens // wl.block))
+    # pages one head can need: the window, the kept tokens at the largest keep
+    # fraction with 25% slack, one partly filled page
+    hi = wl.keep_range[1] if wl.keep_range else wl.keep
+    need = -(-int(wl.window + 1.25 * hi * wl.max_positions + wl.block) // wl.block)
+    d.pool_pages = wl.layers * wl.batch * wl.kv_heads * min(maxp, max(pre, need))
     d.act_dtype = B_.DMS_BF16
-    d.kv_dtype = B_.DMS_BF16
+    d.kv_dtype = {"bf16": B_.DMS_BF16, "fp8": B_.DMS_FP8_E4M3}[wl.kv_dtype]
+    d.alpha_source = {"proj": B_.DMS_ALPHA_PROJ, "key": B_.DMS_ALPHA_KEY_NEURON}[wl.alpha_source]
+    d.alpha_per = B_.DMS_ALPHA_PER_LAYER if wl.alpha_per == "layer" else B_.DMS_ALPHA_PER_HEAD
     return d
 
 
-def gpu_inputs(wl, seed):
-    g = torch.Generator(device="cuda")
-    g.manual_seed(seed)
-    B, T, S = wl.batch, wl.prompt, wl.decode_steps
-    bf = torch.bfloat16
-
-    def rn(*shape, std=1.0):
-        return (torch.randn(*shape, generator=g, device="cuda", dtype=torch.float32) * std).to(bf)
-
-    x = dict(q=rn(B, T, wl.q_heads, wl.head_dim), k=rn(B, T, wl.kv_heads, wl.head_dim),
-             v=rn(B, T, wl.kv_heads, wl.head_dim), h=rn(B, T, wl.hidden),
-             qd=rn(S, B, wl.q_heads, wl.head_dim), kd=rn(S, B, wl.kv_heads, wl.head_dim),
-             vd=rn(S, B, wl.kv_heads, wl.head_dim), hd=rn(S, B, wl.hidden),
-             gamma=rn(wl.hidden), W=rn(wl.kv_heads, wl.hidden, std=wl.hidden ** -0.5))
-    return x
+def decode_launches_per_step(wl):
+    """Kernels one dms_decode_step launches per layer."""
+    pre = 1 if (wl.alpha_source != "proj" or wl.rope) else 0  # decision neuron / rotary pass
+    if wl.kv_dtype == "fp8":
+        return pre + 2  # append (re-encodes pages), then the cluster attention
+    return pre + 1      # one fused kernel: decision, attention, combine, append
 
 
-def calibrate(B_, cache, wl, x):
-    """Offsets that keep a 1/8 fraction per head, from the library's own logits."""
-    zero = torch.zeros(wl.batch, wl.kv_heads, dtype=torch.float32, device="cuda")
-    raw = torch.empty(wl.batch, wl.kv_heads, wl.prompt, dtype=torch.float32, device="cuda")
-    p = B_.decide_params(zero, hidden=x["h"], norm_weight=x["gamma"], proj_weight=x["W"])
-    B_.dms_decide(cache.handle, wl.prompt, p, None, raw)
-    s, _ = torch.sort(raw, dim=-1)
-    k = int(round(wl.keep * wl.prompt))
-    return (0.5 * (s[..., k - 1] + s[..., k])).contiguous()
+def kernel_launches_per_step(wl, n_dec):
+    # reset (1) + per layer: compaction (decide or neuron/rotary pass, scan,
+    # scatter) + prefill attention (1) + the decode steps
+    return 1 + wl.layers * (3 + 1) + wl.layers * n_dec * decode_launches_per_step(wl)
 
 
 class Runner:
-    def __init__(self, B_, wl, seed):
+    """One workload on one GPU: per-layer seeded inputs in HBM, a cache, and
+    the decode steps captured as CUDA graphs."""
+
+    def __init__(self, B_, wl, seed, n_dec=None, kernel="auto"):
         self.B_, self.wl = B_, wl
-        self.cache = B_.Cache(make_desc(B_, wl))
-        self.x = gpu_inputs(wl, seed)
-        self.off = calibrate(B_, self.cache, wl, self.x)
-        x, wl_ = self.x, wl
-        self.o = torch.empty_like(x["q"])
-        self.alpha = torch.empty(wl_.batch, wl_.kv_heads, wl_.prompt, dtype=torch.float32, device="cuda")
-        self.od = torch.empty_like(x["qd"])
-        self.ad = torch.empty(wl_.decode_steps, wl_.batch, wl_.kv_heads, dtype=torch.float32, device="cuda")
-        self.pdec = B_.decide_params(self.off, hidden=x["h"], norm_weight=x["gamma"], proj_weight=x["W"])
-        self.pargs = B_.Cache.prefill_args(x["q"], x["k"], x["v"], self.o, self.alpha, self.pdec)
-        self.ddec = [B_.decide_params(self.off, hidden=x["hd"][s], norm_weight=x["gamma"], proj_weight=x["W"])
-                     for s in range(wl_.decode_steps)]
-        self.dargs = [B_.Cache.decode_args(x["qd"][s], x["kd"][s], x["vd"][s], self.od[s], self.ad[s], self.ddec[s])
-                      for s in range(wl_.decode_steps)]
+        self.S = n_dec or wl.decode_steps
+        self.L = wl.layers
+        # a single layer draws every decode token; a deep stack cycles a pool
+        self.pool = self.S if self.L == 1 else min(self.S, STEP_POOL)
+        self.desc = make_desc(B_, wl, kernel)
+        self.cache = B_.Cache(self.desc)
+        self.neuron = wl.alpha_source != "proj"
+        # the compaction and the decode step rewrite q and k in place (neuron
+        # zeroing, rotary): pristine copies are restored outside the timed segments
+        self.inplace = self.neuron or wl.rope
+        if self.inplace and self.L > 1:
+            raise NotImplementedError("in-place inputs on a multi-layer stack")
+        self.rope = None
+        if wl.rope:
+            cos, sin = I.rope_tables(wl.max_positions, wl.head_dim)
+            self.rope = (cos.cuda(), sin.cuda())
+        B, T, Hq, D = wl.batch, wl.prompt, wl.q_heads, wl.head_dim
+        # layers do not feed each other: one output buffer serves them all
+        self.o = torch.empty(B, T, Hq, D, dtype=torch.bfloat16, device="cuda")
+        self.od = torch.empty(self.pool, B, Hq, D, dtype=torch.bfloat16, device="cuda")
+        self.lay = [self._layer(l, seed) for l in range(self.L)]
         self.flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+        self.clean = torch.zeros(64 << 20, dtype=torch.float32, device="cuda")
         self.graphs = None
+        self.cycled = self.pool < self.S
+
+    def _layer(self, l, seed):
+        B_, wl = self.B_, self.wl
+        g = torch.Generator(device="cuda")
+        g.manual_seed(seed * 4099 + l)
+        bf = torch.bfloat16
+        B, T, P, Hq, H, D = wl.batch, wl.prompt, self.pool, wl.q_heads, wl.kv_heads, wl.head_dim
+
+        def rn(*shape, std=1.0):
+            return (torch.randn(*shape, generator=g, device="cuda", dtype=torch.float32) * std).to(bf)
+
+        x = dict(q=rn(B, T, Hq, D), k=rn(B, T, H, D), v=rn(B, T, H, D),
+                 qd=rn(P, B, Hq, D), kd=rn(P, B, H, D), vd=rn(P, B, H, D))
+        if not self.neuron:
+            x.update(h=rn(B, T, wl.hidden), hd=rn(P, B, wl.hidden), gamma=rn(wl.hidden),
+                     W=rn(H, wl.hidden, std=wl.hidden ** -0.5))
+        # offsets that keep the workload's fraction of tokens per (b, h)
+        keep = I.keep_fractions(wl, seed)
+        if self.neuron:
+            raw = (x["k"][..., -1].float() * self.desc.alpha_scale).permute(0, 2, 1)
+        else:
+            zero = torch.zeros(B, H, dtype=torch.float32, device="cuda")
+            raw = torch.empty(B, H, T, dtype=torch.float32, device="cuda")
+            p = B_.decide_params(zero, hidden=x["h"], norm_weight=x["gamma"], proj_weight=x["W"])
+            B_.dms_decide(self.cache.handle, T, p, None, raw)
+        raw = raw.cpu().numpy()
+        if wl.alpha_per == "layer":  # every head follows head 0's logit
+            raw = np.broadcast_to(raw[:, :1], raw.shape)
+            keep = np.broadcast_to(keep[:, :1], keep.shape)
+        off, _ = I.calibrate_offsets(raw, keep)
+        x["off"] = torch.from_numpy(off).cuda()
+        if self.inplace:
+            for k_ in ("q", "k", "qd", "kd"):
+                x[k_ + "0"] = x[k_].clone()
+        x["alpha"] = torch.empty(B, H, T, dtype=torch.float32, device="cuda")
+        x["ad"] = torch.empty(P, B, H, dtype=torch.float32, device="cuda")
+        if self.neuron:
+            x["pdec"] = B_.decide_params(x["off"])
+            x["ddec"] = [x["pdec"]] * P
+        else:
+            x["pdec"] = B_.decide_params(x["off"], hidden=x["h"], norm_weight=x["gamma"], proj_weight=x["W"])
+            x["ddec"] = [B_.decide_params(x["off"], hidden=x["hd"][i], norm_weight=x["gamma"], proj_weight=x["W"])
+                         for i in range(P)]
+        x["pargs"] = B_.Cache.prefill_args(x["q"], x["k"], x["v"], self.o, x["alpha"], x["pdec"], self.rope)
+        x["dargs"] = [B_.Cache.decode_args(x["qd"][i], x["kd"][i], x["vd"][i], self.od[i], x["ad"][i],
+                                           x["ddec"][i], self.rope) for i in range(P)]
+        return x
+
+    def l2_flush(self, s):
+        """Evict L2: write a 512 MB buffer, then read a 256 MB one, so that the
+        lines left in L2 are clean and the next step pays no write-back of
+        the flush itself."""
+        self.flush.fill_(s & 0xFF)
+        self._sink = self.clean.sum()
+
+    # restores of inputs the library rewrites in place (outside the timed segments)
+    def restore_prompt(self):
+        if self.inplace:
+            for x in self.lay:
+                x["q"].copy_(x["q0"])
+                x["k"].copy_(x["k0"])
+
+    def restore_token(self, i):
+        if self.inplace:
+            for x in self.lay:
+                x["qd"][i].copy_(x["qd0"][i])
+                x["kd"][i].copy_(x["kd0"][i])
+
+    def prefill_all(self):
+        for l, x in enumerate(self.lay):
+            self.B_.dms_prefill(self.cache.handle, l, x["pargs"])
 
     def capture(self):
-        """CUDA graphs of each decode step's append and attention (the decode
+        """CUDA graphs of the decode steps, one per distinct token input, each
+        holding the step's start/end events around its kernels (the decode
         kernels read the token position from device memory, so a replay
         advances the cache exactly like an eager call)."""
         B_, h = self.B_, self.cache.handle
         self.cache.reset()
-        B_.dms_prefill(h, 0, self.pargs)
+        self.restore_prompt()
+        self.prefill_all()
         torch.cuda.synchronize()
         side = torch.cuda.Stream()
         gs = []
-        for s in range(self.wl.decode_steps):
+        for i in range(self.pool):
+            self.restore_token(i)
+            torch.cuda.synchronize()
             ga = torch.cuda.CUDAGraph()
             ev = (torch.cuda.Event(enable_timing=True, external=True),
                   torch.cuda.Event(enable_timing=True, external=True))
             with torch.cuda.graph(ga, stream=side):
                 ev[0].record()
-                B_.dms_decode_step(h, 0, self.dargs[s])
+                for l, x in enumerate(self.lay):
+                    B_.dms_decode_step(h, l, x["dargs"][i])
                 ev[1].record()
             gs.append((ga, ev))
         torch.cuda.synchronize()
         self.graphs = gs
 
     def step(self, ev=None, counts=None):
-        """One bench step.  ev: list of event tuples filled per segment."""
+        """One bench step: reset, prefill of every layer, every decode step.
+        ev: list that receives (prefill segments, decode ms) of this step."""
         B_, h = self.B_, self.cache.handle
-        self.cache.reset()
-        self.flush.fill_(1)
         E = torch.cuda.Event
-        e0, e1, e2 = E(enable_timing=True), E(enable_timing=True), E(enable_timing=True)
-        e0.record()
-        B_.dms_prefill_compact(h, 0, self.pargs)
-        e1.record()
-        B_.dms_prefill_attention(h, 0, self.pargs)
-        e2.record()
+        self.cache.reset()
+        self.restore_prompt()
+        if not self.cycled:
+            self.l2_flush(1)
+        seg = []
+        for l, x in enumerate(self.lay):
+            e0, e1, e2 = E(enable_timing=True), E(enable_timing=True), E(enable_timing=True)
+            e0.record()
+            B_.dms_prefill_compact(h, l, x["pargs"])
+            e1.record()
+            B_.dms_prefill_attention(h, l, x["pargs"])
+            e2.record()
+            seg.append((e0, e1, e2))
+        if counts is not None:
+            counts.append(self.cache.counts().sum(dtype=torch.int64))
         dec = []
-        for s in range(self.wl.decode_steps):
-            self.flush.fill_(s & 0xFF)
+        d0, d1 = E(enable_timing=True), E(enable_timing=True)
+        d0.record()
+        for s in range(self.S):
+            i = s % self.pool
+            if not self.cycled:
+                # the decode working set fits in L2: evict it before every step
+                self.restore_token(i)
+                self.l2_flush(s)
             if self.graphs is not None:
-                # the step's graph records its own start/end events around the kernel
-                self.graphs[s][0].replay()
+                self.graphs[i][0].replay()
             else:
                 a, c = E(enable_timing=True), E(enable_timing=True)
                 a.record()
-                B_.dms_decode_step(h, 0, self.dargs[s])
+                for l, x in enumerate(self.lay):
+                    B_.dms_decode_step(h, l, x["dargs"][i])
                 c.record()
                 dec.append((a, c))
             if counts is not None:
-                counts.append(self.cache.state(0)["count"].sum().item())
+                counts.append(self.cache.counts().sum(dtype=torch.int64))
+        d1.record()
         if ev is not None:
-            # graph events are re-recorded by the next replay: read them now
             torch.cuda.synchronize()
-            dec_ms = sum(g[1][0].elapsed_time(g[1][1]) for g in self.graphs) if self.graphs else \
-                sum(a.elapsed_time(c) for a, c in dec)
-            ev.append(((e0, e1, e2), dec_ms))
-
-
-def kernel_launches_per_step(wl):
-    # reset (1) + compaction (decide, scan, scatter) + prefill attention (1)
-    # + per decode step: one fused kernel (decision logit, attention, combine, append)
-    return 1 + 3 + 1 + 1 * wl.decode_steps
+            if self.cycled:
+                # steps run back to back: the stack's working set is many times L2
+                dec_ms = d0.elapsed_time(d1)
+            elif self.graphs is not None:
+                dec_ms = sum(g[1][0].elapsed_time(g[1][1]) for g in self.graphs)
+            else:
+                dec_ms = sum(a.elapsed_time(c) for a, c in dec)
+            ev.append((seg, dec_ms))
 
 
 def visible_pairs(alpha, wl):
@@ -280,28 +396,44 @@ def visible_pairs(alpha, wl):
     return int((band[None, None, :] + cum[:, :, upto]).sum())
 
 
+def decode_step_bytes(wl, retained):
+    """Algorithmic HBM bytes of one decode step over the stack, given the
+    retained slots summed over (layer, b, h) before the append: the retained
+    K/V read, page-table entries (and FP8 page scales), q and o, the new K/V
+    row read and written, and the decision inputs (hidden row, W, gamma)."""
+    D, B, L = wl.head_dim, wl.batch, wl.layers
+    elem = 1 if wl.kv_dtype == "fp8" else 2
+    BH = B * wl.kv_heads
+    pages = -(-retained // wl.block)  # a lower bound on pages touched
+    per_page = 4 + (8 if wl.kv_dtype == "fp8" else 0)
+    fixed = L * (2 * B * wl.q_heads * D * 2 + 2 * BH * D * 2 + 2 * BH * D * elem)
+    if wl.alpha_source == "proj":
+        fixed += L * (B * wl.hidden * 2 + wl.kv_heads * wl.hidden * 2 + wl.hidden * 2)
+    return retained * D * 2 * elem + pages * per_page + fixed
+
+
 def run_ours(args, world, rank, local):
     from learned_kv_cache_dms_b200 import binding as B_
-    wl = WL
+    wl = I.WORKLOADS[args.workload]
     pk, pk_kind = peaks()
-    r = Runner(B_, wl, seed=WL.seed + rank)
-    # untimed pass: retained counts after each append (identical in every step)
+    r = Runner(B_, wl, seed=wl.seed + rank, n_dec=args.decode_steps, kernel=args.decode_kernel)
+    S, L = r.S, r.L
+    # untimed pass: retained counts after the prefill and after each append
     counts = []
-    r.cache.reset()
-    B_.dms_prefill(r.cache.handle, 0, r.pargs)
-    counts_prefill = r.cache.state(0)["count"].sum().item()
     r.step(counts=counts)
     torch.cuda.synchronize()
-    assert r.cache.status() == 0
-    pairs = visible_pairs(r.alpha, wl)
+    counts = [int(c.item()) for c in torch.stack(counts).cpu()]
+    assert r.cache.status() == 0, "cache status %d" % r.cache.status()
+    pairs = sum(visible_pairs(x["alpha"], wl) for x in r.lay)
     o_eager = r.od.clone()
     r.capture()
     for _ in range(max(1, args.warmup - 1)):
         r.step()
     torch.cuda.synchronize()
     assert r.cache.status() == 0
-    # the graph replays must reproduce the eager decode outputs exactly
-    assert torch.equal(o_eager, r.od), "graph replay differs from the eager decode"
+    if not r.cycled:
+        # the graph replays must reproduce the eager decode outputs exactly
+        assert torch.equal(o_eager, r.od), "graph replay differs from the eager decode"
 
     barrier(world)
     torch.cuda.synchronize()
@@ -318,11 +450,12 @@ def run_ours(args, world, rank, local):
     region_ms = t0.elapsed_time(t1)
 
     compact_ms = prefill_attn_ms = decode_ms = 0.0
-    for (e0, e1, e2), dec_ms in evs:
-        compact_ms += e0.elapsed_time(e1)
-        prefill_attn_ms += e1.elapsed_time(e2)
+    for seg, dec_ms in evs:
+        for e0, e1, e2 in seg:
+            compact_ms += e0.elapsed_time(e1)
+            prefill_attn_ms += e1.elapsed_time(e2)
         decode_ms += dec_ms
-    K, S, B = args.steps, wl.decode_steps, wl.batch
+    K, B = args.steps, wl.batch
     prefill_ms = compact_ms + prefill_attn_ms
     hot_ms_per_step = (decode_ms + prefill_ms) / K
     # max over ranks of the device times
@@ -333,22 +466,10 @@ def run_ours(args, world, rank, local):
     value = dec_tokens / (decode_ms_max / 1e3)
     prefill_tps = K * B * wl.prompt * world / (prefill_ms_max / 1e3)
 
-    # algorithmic bytes of one fused decode step (one launch): the retained K/V
-    # the attention reads (before the append, plus the new row), q and o, the
-    # new K/V row written, the hidden row and W of the decision logits, and the
-    # page-table entries
-    D, elem = wl.head_dim, 2
-    BH = B * wl.kv_heads
-    per_step_fixed = (2 * B * wl.q_heads * D * elem            # q, o
-                      + 2 * BH * D * elem                      # new K/V rows read
-                      + 2 * BH * D * elem                      # new K/V rows written
-                      + B * wl.hidden * elem + wl.kv_heads * wl.hidden * elem + wl.hidden * elem)  # h, W, gamma
-    pre_counts = [counts_prefill] + counts[:-1]
-    step_bytes = [cp * D * 2 * elem + (-(-cp // wl.block)) * 4 + per_step_fixed for cp in pre_counts]
+    step_bytes = [decode_step_bytes(wl, c) for c in counts[:-1]]
     attn_bytes = sum(step_bytes)
     decode_gbs = K * attn_bytes / (decode_ms / 1e3) / 1e9
-    attn_gbs = decode_gbs
-    prefill_flops = 4.0 * D * wl.gqa * pairs
+    prefill_flops = 4.0 * wl.head_dim * wl.gqa * pairs
     prefill_tflops = K * prefill_flops / (prefill_attn_ms / 1e3) / 1e12
     clocks = clk.summary()
 
@@ -356,21 +477,32 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, args.cpu_seconds)
-    roof = {"bound": "hbm", "achieved": round(attn_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": round(attn_gbs / pk["hbm_gbs"], 4), "traffic": None,
-            "kernel": "fused decode step k_decode_attn<128,bf16,fused> (split-K attention, combine, append)",
-            "algorithmic_bytes_per_launch": int(attn_bytes / S), "peak_source": pk_kind}
+    kname = ("decode step: k_decode_cluster<%d,%s> (split-K attention, on-chip combine%s)%s"
+             % (wl.head_dim, wl.kv_dtype, ", append, decision logit" if wl.kv_dtype == "bf16" else "",
+                " after k_decode_append" if wl.kv_dtype == "fp8" else ""))
+    roof = {"bound": "hbm", "achieved": round(decode_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(decode_gbs / pk["hbm_gbs"], 4), "traffic": None, "kernel": kname,
+            "algorithmic_bytes_per_launch": int(attn_bytes / (S * L)), "peak_source": pk_kind}
+    retained_first = counts[0] / (L * B * wl.kv_heads)
+    retained_last = counts[-1] / (L * B * wl.kv_heads)
+    cfg = {"workload": workload_label(wl, S), "layers": L, "batch": B, "prompt": wl.prompt, "decode_steps": S,
+           "hidden": wl.hidden, "q_heads": wl.q_heads, "kv_heads": wl.kv_heads, "head_dim": wl.head_dim,
+           "window": wl.window, "block": wl.block, "kv_dtype": wl.kv_dtype, "alpha_source": wl.alpha_source,
+           "alpha_per": wl.alpha_per, "keep": list(wl.keep_range) if wl.keep_range else wl.keep,
+           "l2": ("decode steps back to back; the stack's retained KV (%.2f GB per step) is many times L2"
+                  % (step_bytes[0] / 1e9)) if r.cycled else
+                 "512 MB buffer written, then a 256 MB buffer read, before every decode step (untimed)",
+           "parallelism": "dp%d replicas" % world, "decode_kernel": args.decode_kernel}
+    if r.cycled:
+        cfg["decode_inputs"] = "%d distinct token inputs per layer, cycled" % r.pool
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(hot_max, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "qwen8b_layer_b1_ctx8192_dec128", "batch": B, "prompt": wl.prompt,
-                   "decode_steps": S, "hidden": wl.hidden, "q_heads": wl.q_heads, "kv_heads": wl.kv_heads,
-                   "head_dim": D, "window": wl.window, "block": wl.block, "keep": wl.keep,
-                   "l2": "512 MB buffer written before every decode step (untimed)",
-                   "parallelism": "dp%d replicas" % world},
+        "vs_baseline": None, "dtype": "bf16" if wl.kv_dtype == "bf16" else "bf16+fp8kv", "data": "synthetic",
+        "config": cfg,
         "retained_kv_gbps": round(decode_gbs, 1),
         "retained_kv_frac_of_peak": round(decode_gbs / pk["hbm_gbs"], 4),
+        "retained_per_head": [round(retained_first, 1), round(retained_last, 1)],
         "decode_ms_per_token_step": round(decode_ms / (K * S), 5),
         "prefill_tok_s": round(prefill_tps, 1),
         "prefill_ms": round(prefill_ms / K, 4),
@@ -379,10 +511,10 @@ def run_ours(args, world, rank, local):
         "prefill_attention": {"bound": "tensor", "achieved": round(prefill_tflops, 2),
                               "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                               "frac": round(prefill_tflops / pk["bf16_tflops"], 4),
-                              "flops_per_launch": prefill_flops, "visible_pairs": pairs},
-        "achieved_cr": round(wl.max_positions / (counts[-1] / (B * wl.kv_heads)), 3),
+                              "flops_per_launch": prefill_flops / L, "visible_pairs": pairs},
+        "achieved_cr": round(wl.max_positions / retained_last, 3) if S == wl.decode_steps else None,
         "region_ms_per_step_incl_l2_flush": round(region_ms / K, 3),
-        "roofline": roof, "e2e": e2e, "gpu_launches": kernel_launches_per_step(wl) * K,
+        "roofline": roof, "e2e": e2e, "gpu_launches": kernel_launches_per_step(wl, S) * K,
         "clocks": clocks, "cpu_baseline": cpu,
     }
     return line
@@ -396,60 +528,79 @@ def _op(name):
 def run_e2e(B_, r, args, world):
     """Same workload through the public API with host (pinned) buffers: the
     prompt and every decode token are copied host->device and every output
-    device->host inside the timed segments."""
-    wl, x = r.wl, r.x
-    host = {k: v.cpu().pin_memory() for k, v in x.items() if k in ("q", "k", "v", "h", "qd", "kd", "vd", "hd")}
+    device->host inside the timed segments.  A multi-layer stack is sampled
+    over its first E2E_STEPS_STACK decode steps."""
+    wl = r.wl
+    S = r.S if r.L == 1 else min(r.S, E2E_STEPS_STACK)
+    names_p = ("q", "k", "v") + (() if r.neuron else ("h",))
+    names_d = ("qd", "kd", "vd") + (() if r.neuron else ("hd",))
+    src = [{k: (x[k + "0"] if r.inplace and (k + "0") in x else x[k]) for k in names_p + names_d} for x in r.lay]
+    host = [{k: t.cpu().pin_memory() for k, t in s_.items()} for s_ in src]
+    dev = [{k: torch.empty_like(t) for k, t in s_.items()} for s_ in src]
     o_host = torch.empty(tuple(r.o.shape), dtype=r.o.dtype).pin_memory()
     od_host = torch.empty(tuple(r.od.shape), dtype=r.od.dtype).pin_memory()
-    dev = {k: torch.empty_like(x[k]) for k in host}
-    pdec = B_.decide_params(r.off, hidden=dev["h"], norm_weight=x["gamma"], proj_weight=x["W"])
-    pargs = B_.Cache.prefill_args(dev["q"], dev["k"], dev["v"], r.o, r.alpha, pdec)
-    ddec = [B_.decide_params(r.off, hidden=dev["hd"][s], norm_weight=x["gamma"], proj_weight=x["W"])
-            for s in range(wl.decode_steps)]
-    dargs = [B_.Cache.decode_args(dev["qd"][s], dev["kd"][s], dev["vd"][s], r.od[s], r.ad[s], ddec[s])
-             for s in range(wl.decode_steps)]
+    pargs, dargs = [], []
+    for x, d in zip(r.lay, dev):
+        if r.neuron:
+            pd = B_.decide_params(x["off"])
+            dd = [pd] * r.pool
+        else:
+            pd = B_.decide_params(x["off"], hidden=d["h"], norm_weight=x["gamma"], proj_weight=x["W"])
+            dd = [B_.decide_params(x["off"], hidden=d["hd"][i], norm_weight=x["gamma"], proj_weight=x["W"])
+                  for i in range(r.pool)]
+        x["_e2e_keep"] = (pd, dd)
+        pargs.append(B_.Cache.prefill_args(d["q"], d["k"], d["v"], r.o, x["alpha"], pd, r.rope))
+        dargs.append([B_.Cache.decode_args(d["qd"][i], d["kd"][i], d["vd"][i], r.od[i], x["ad"][i], dd[i], r.rope)
+                      for i in range(r.pool)])
     E = torch.cuda.Event
     dec_ms = 0.0
-    h2d = d2h = 0
     for it in range(args.steps + 1):
         r.cache.reset()
-        r.flush.fill_(3)
-        e0, e1 = E(enable_timing=True), E(enable_timing=True)
-        e0.record()
-        for k in ("q", "k", "v", "h"):
-            dev[k].copy_(host[k], non_blocking=True)
-        B_.dms_prefill(r.cache.handle, 0, pargs)
+        r.l2_flush(3)
+        for l in range(r.L):
+            for k in names_p:
+                dev[l][k].copy_(host[l][k], non_blocking=True)
+            B_.dms_prefill(r.cache.handle, l, pargs[l])
         o_host.copy_(r.o, non_blocking=True)
-        e1.record()
         evs = []
-        for s in range(wl.decode_steps):
-            r.flush.fill_(s & 0xFF)
+        for s in range(S):
+            i = s % r.pool
+            if not r.cycled:
+                r.l2_flush(s)
             a, c = E(enable_timing=True), E(enable_timing=True)
             a.record()
-            for k in ("qd", "kd", "vd", "hd"):
-                dev[k][s].copy_(host[k][s], non_blocking=True)
-            B_.dms_decode_step(r.cache.handle, 0, dargs[s])
-            od_host[s].copy_(r.od[s], non_blocking=True)
+            for l in range(r.L):
+                for k in names_d:
+                    dev[l][k][i].copy_(host[l][k][i], non_blocking=True)
+                B_.dms_decode_step(r.cache.handle, l, dargs[l][i])
+            od_host[i].copy_(r.od[i], non_blocking=True)
             c.record()
             evs.append((a, c))
         torch.cuda.synchronize()
         if it == 0:
             continue  # warm-up
         dec_ms += sum(a.elapsed_time(c) for a, c in evs)
-    bpe = 2
-    h2d = (sum(host[k].numel() for k in ("q", "k", "v", "h")) + sum(host[k].numel() for k in ("qd", "kd", "vd", "hd"))) * bpe
-    d2h = (o_host.numel() + od_host.numel()) * bpe
+    h2d = sum(host[l][k].numel() * 2 for l in range(r.L) for k in names_p)
+    h2d += S * sum(host[l][k][0].numel() * 2 for l in range(r.L) for k in names_d)
+    d2h = o_host.numel() * 2 + S * od_host[0].numel() * 2
     dec_ms_max = allreduce(dec_ms, _op("max"), world)
-    val = args.steps * wl.decode_steps * wl.batch * world / (dec_ms_max / 1e3)
-    return {"value": round(val, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    val = args.steps * S * wl.batch * world / (dec_ms_max / 1e3)
+    out = {"value": round(val, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    if S < r.S:
+        out["sample"] = "first %d decode steps" % S
+    return out
+
+
+E2E_STEPS_STACK = 256
 
 
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline arm)
 # ---------------------------------------------------------------------------
 def oracle_decode_sample(wl, seconds, n_steps_max=None):
-    """Time the oracle's decode steps (append + decode attention) on the host
-    cores after an untimed prefill replay.  Returns (tok/s, cores, steps, secs)."""
+    """Time the oracle's decode steps (append + decode attention) of one layer
+    on the host cores after an untimed prefill replay.  Returns (tok/s over
+    the workload's layer stack, cores, steps, secs)."""
     from oracle import oracle as O
     cores = O.set_threads(os.cpu_count() or 1)
     B, T, S = wl.batch, wl.prompt, wl.decode_steps
@@ -457,11 +608,11 @@ def oracle_decode_sample(wl, seconds, n_steps_max=None):
     k = I.normal(s, (0, 2), (B, T + S, wl.kv_heads, wl.head_dim), "bf16").float().numpy()
     v = I.normal(s, (0, 3), (B, T + S, wl.kv_heads, wl.head_dim), "bf16").float().numpy()
     q = I.normal(s, (0, 1), (B, S, wl.q_heads, wl.head_dim), "bf16").double().numpy()
-    alpha = I.synthetic_alpha(s, (0, 5), B, wl.kv_heads, T + S, wl.keep).numpy()
+    alpha = I.synthetic_alpha(s, (0, 5), B, wl.kv_heads, T + S, I.keep_fractions(wl)).numpy()
     ev = (alpha > 0).astype(np.uint8)
     maxp = -(-wl.max_positions // wl.block)
     c = O.Cache(1, B, wl.kv_heads, wl.head_dim, wl.window, wl.block, wl.max_positions,
-                B * wl.kv_heads * maxp, wl.prealloc_tokens)
+                B * wl.kv_heads * maxp, wl.prealloc_tokens, fp8=wl.kv_dtype == "fp8")
     c.prefill(0, np.ascontiguousarray(ev[:, :, :T]), np.ascontiguousarray(k[:, :T]), np.ascontiguousarray(v[:, :T]))
     n = 0
     t0 = time.perf_counter()
@@ -472,20 +623,22 @@ def oracle_decode_sample(wl, seconds, n_steps_max=None):
         c.decode_attention(0, np.ascontiguousarray(q[:, n]))
         n += 1
     dt = time.perf_counter() - t0
-    return n * B / dt, cores, n, dt
+    return n * B / (dt * wl.layers), cores, n, dt
 
 
 def cpu_baseline(wl, seconds):
     tps, cores, n, dt = oracle_decode_sample(wl, seconds)
     return {"value": round(tps, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": "first %d of %d decode steps (append + fp64 decode attention over the retained slots) after "
-                      "an untimed prefill replay of the 8192-token prompt, %.1f s" % (n, wl.decode_steps, dt)}
+            "sample": "first %d of %d decode steps of one layer (append + fp64 decode attention over the retained "
+                      "slots) after an untimed prefill replay of the %d-token prompt, %.1f s%s"
+                      % (n, wl.decode_steps, wl.prompt, dt,
+                         "; scaled to the %d-layer stack" % wl.layers if wl.layers > 1 else "")}
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return None
-    wl = WL
+    wl = I.WORKLOADS[args.workload]
     per_step = 4  # decode steps of the oracle per bench step (bounded sample)
     for _ in range(args.warmup):
         oracle_decode_sample(wl, 1e9, n_steps_max=1)
@@ -493,14 +646,14 @@ def run_reference(args, world, rank):
     cores = 1
     for _ in range(args.steps):
         tps, cores, n, dt = oracle_decode_sample(wl, 1e9, n_steps_max=per_step)
-        tot_tok += n * wl.batch
+        tot_tok += n * wl.batch / wl.layers
         tot_s += dt
     val = tot_tok / tot_s
     return {"impl": "reference", "metric": METRIC, "value": round(val, 2), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "qwen8b_layer_b1_ctx8192_dec128", "batch": wl.batch, "prompt": wl.prompt,
-                       "decode_steps": wl.decode_steps},
+            "config": {"workload": workload_label(wl, args.decode_steps or wl.decode_steps), "batch": wl.batch,
+                       "prompt": wl.prompt, "decode_steps": wl.decode_steps},
             "cpu_baseline": {"value": round(val, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": "%d decode steps per bench step after an untimed prefill replay" % per_step},
             "e2e": {"value": round(val, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

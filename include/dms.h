@@ -64,6 +64,10 @@ extern "C" {
 #define DMS_ST_POOL_EXHAUSTED 1 /* a page was needed and the pool had none     */
 #define DMS_ST_CAPACITY 2       /* a slot index exceeded the per-head capacity */
 #define DMS_ST_TIMEOUT 4        /* a bounded device wait gave up               */
+#define DMS_ST_SPLIT_LIMIT 8    /* FLAT decode: a CTA's share of the slots met
+                                   more heads than its table holds (thousands
+                                   of heads of very different lengths); use
+                                   DMS_DECODE_CLUSTER for such a cache         */
 
 /* ---- enumerations ------------------------------------------------------------ */
 enum dms_dtype { DMS_F32 = 0, DMS_BF16 = 1, DMS_FP8_E4M3 = 2 };
@@ -73,6 +77,14 @@ enum dms_alpha_per { DMS_ALPHA_PER_HEAD = 0, DMS_ALPHA_PER_LAYER = 1 };
  * pre-attention hidden state, dms_separate_alpha=True), or the last neuron of
  * each key / of the first query head of each GQA group (separate_alpha=False). */
 enum dms_alpha_source { DMS_ALPHA_PROJ = 0, DMS_ALPHA_KEY_NEURON = 1, DMS_ALPHA_QUERY_NEURON = 2 };
+
+/* Decode attention kernels.  CLUSTER: one thread-block cluster per (b, h),
+ * partials combined on chip (lowest latency when B * Hkv is small).  FLAT: one
+ * CTA per SM over a balanced list of every head's slots, partials combined by
+ * the last CTA to finish a head (keeps HBM busy at any batch).  AUTO picks
+ * CLUSTER when B * Hkv * 8 <= 2 * SMs (every head gets a full cluster of 8),
+ * else FLAT; FLAT falls back to CLUSTER for shapes it does not stage. */
+enum dms_decode_kernel { DMS_DECODE_AUTO = 0, DMS_DECODE_CLUSTER = 1, DMS_DECODE_FLAT = 2 };
 
 /* ---- cache descriptor ---------------------------------------------------------
  * Mirrors the DMS configuration record ([DMS-Qwen3], Qwen3ConfigDMS table):
@@ -103,6 +115,8 @@ typedef struct dms_cache_desc {
   float alpha_scale;    /* multiplies the raw logit (100)                       */
   float rms_eps;        /* RMSNorm epsilon of the adapter (1e-6)                */
   int disable_eviction; /* nonzero: every decision is "keep" (vanilla model)    */
+  int decode_kernel;    /* enum dms_decode_kernel: how a decode step splits the
+                           attention over the SMs (0: chosen from the shape)  */
 } dms_cache_desc;
 
 /* Fill `desc` with the defaults of the DMS configuration record: window 512,

@@ -24,10 +24,11 @@ _lib = C.CDLL(LIB_PATH)
 
 # ---- constants (mirror include/dms.h) ---------------------------------------
 DMS_OK, DMS_ERR_INVALID, DMS_ERR_STATE, DMS_ERR_CUDA, DMS_ERR_NOMEM, DMS_ERR_SCRATCH_LIMIT = 0, -1, -2, -3, -4, -5
-DMS_ST_POOL_EXHAUSTED, DMS_ST_CAPACITY, DMS_ST_TIMEOUT = 1, 2, 4
+DMS_ST_POOL_EXHAUSTED, DMS_ST_CAPACITY, DMS_ST_TIMEOUT, DMS_ST_SPLIT_LIMIT = 1, 2, 4, 8
 DMS_F32, DMS_BF16, DMS_FP8_E4M3 = 0, 1, 2
 DMS_ALPHA_PER_HEAD, DMS_ALPHA_PER_LAYER = 0, 1
 DMS_ALPHA_PROJ, DMS_ALPHA_KEY_NEURON, DMS_ALPHA_QUERY_NEURON = 0, 1, 2
+DMS_DECODE_AUTO, DMS_DECODE_CLUSTER, DMS_DECODE_FLAT = 0, 1, 2
 
 _ERRORS = {DMS_ERR_INVALID: "DMS_ERR_INVALID", DMS_ERR_STATE: "DMS_ERR_STATE", DMS_ERR_CUDA: "DMS_ERR_CUDA",
            DMS_ERR_NOMEM: "DMS_ERR_NOMEM", DMS_ERR_SCRATCH_LIMIT: "DMS_ERR_SCRATCH_LIMIT"}
@@ -43,7 +44,8 @@ class dms_cache_desc(C.Structure):
     _fields_ = [(n, C.c_int) for n in ("num_layers", "batch", "num_q_heads", "num_kv_heads", "head_dim", "hidden",
                                        "window", "block", "max_positions", "prealloc_tokens", "pool_pages",
                                        "act_dtype", "kv_dtype", "alpha_per", "alpha_source")] + \
-              [("alpha_scale", C.c_float), ("rms_eps", C.c_float), ("disable_eviction", C.c_int)]
+              [("alpha_scale", C.c_float), ("rms_eps", C.c_float), ("disable_eviction", C.c_int),
+               ("decode_kernel", C.c_int)]
 
 
 class dms_cache_layout(C.Structure):
@@ -286,6 +288,12 @@ class Cache:
             next_page=self._view(l.next_page, 1, i32),
             status=self._view(l.status, 1, i32),
         )
+
+    def counts(self):
+        """Retained lengths of every layer, [L, B, Hkv] int32 (a view of the cache)."""
+        d, l = self.desc, self.layout
+        nb = d.num_layers * d.batch * d.num_kv_heads
+        return self._view(l.count, nb, torch.int32).view(d.num_layers, d.batch, d.num_kv_heads)
 
     def pages(self):
         d, l = self.desc, self.layout

@@ -484,17 +484,19 @@ __device__ __forceinline__ float ld_dsmem(uint32_t addr) {
 // Slot plan of the next append of head i of `layer` (token position t):
 // reuse the slot of token t - w when it was marked for eviction, else take slot
 // count (a new page when that slot starts one).  plan.x = slot,
-// plan.y = bit 0 reuse | bit 1 new page | bit 2 over capacity.
+// plan.y = bit 0 reuse | bit 1 new page | bit 2 over capacity; plan.z, plan.w =
+// the head's retained count and pages before the append.
 // Loads bypass L1: the state may have been written by other CTAs of the same
 // launch (made visible by their fences).
-__device__ __forceinline__ int2 next_plan(const CacheView& c, long li, int t) {
-  const int w = c.w, P = c.P;
+__device__ __forceinline__ int4 make_plan(int ringv, int t, int cnt, int have, const CacheView& c) {
+  if (t >= c.w && (static_cast<unsigned>(ringv) & RING_EVICT)) return make_int4(ringv & RING_SLOT_MASK, 1, cnt, have);
+  if (cnt >= c.cap) return make_int4(-1, 4, cnt, have);
+  return make_int4(cnt, (cnt % c.P == 0 && cnt / c.P >= have) ? 2 : 0, cnt, have);
+}
+__device__ __forceinline__ int4 next_plan(const CacheView& c, long li, int t) {
   const int cnt = __ldcg(&c.count[li]), have = __ldcg(&c.npages[li]);
-  const int ringv = t >= w ? __ldcg(&c.ring[li * w + t % w]) : 0;
-  const bool reuse = t >= w && (static_cast<unsigned>(ringv) & RING_EVICT);
-  if (reuse) return make_int2(ringv & RING_SLOT_MASK, 1);
-  if (cnt >= c.cap) return make_int2(-1, 4);
-  return make_int2(cnt, (cnt % P == 0 && cnt / P >= have) ? 2 : 0);
+  const int ringv = t >= c.w ? __ldcg(&c.ring[li * c.w + t % c.w]) : 0;
+  return make_plan(ringv, t, cnt, have, c);
 }
 
 }  // namespace dms

@@ -50,6 +50,7 @@ int check_desc(const dms_cache_desc* d) {
   }
   if (d->alpha_source != DMS_ALPHA_PROJ && d->num_kv_heads > 32) return DMS_ERR_INVALID;
   if (!(d->alpha_scale == d->alpha_scale) || !(d->rms_eps >= 0.0f)) return DMS_ERR_INVALID;
+  if (d->decode_kernel < DMS_DECODE_AUTO || d->decode_kernel > DMS_DECODE_FLAT) return DMS_ERR_INVALID;
   return DMS_OK;
 }
 
@@ -75,7 +76,7 @@ Plan make_plan(const dms_cache_desc* d) {
   p.page_table = take(L * B * H * p.maxp * 4, 256);
   p.slot_pos = take(L * B * H * p.cap * 4, 256);
   p.ring = take(L * B * H * d->window * 4, 256);
-  p.plan = take(2 * L * B * H * 8, 256);
+  p.plan = take(2 * L * B * H * 16, 256);
   p.kept = take(B * H * d->max_positions * 4, 256);
   p.kept_count = take(B * H * 4, 256);
   p.kept_upto = take(B * H * (d->max_positions + 1) * 4, 256);
@@ -107,16 +108,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Tensor map over a page pool viewed as a 2-D tensor [pool_pages * P rows, D].
-// Boxes are 16 rows by up to 128 bytes; bf16 tiles use the 128-byte swizzle,
-// FP8 tiles none (they are widened to bf16 in shared memory).
-bool make_pool_map(CUtensorMap* map, void* base, const dms_cache_desc* d) {
+// Boxes are `rows` rows by up to 128 bytes; bf16 tiles use the 128-byte
+// swizzle, FP8 tiles none (they are widened to bf16 in shared memory).
+bool make_pool_map(CUtensorMap* map, void* base, const dms_cache_desc* d, int rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const int eb = elem_bytes(d->kv_dtype);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(d->head_dim),
                         static_cast<cuuint64_t>(d->pool_pages) * static_cast<cuuint64_t>(d->block)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(d->head_dim) * eb};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(std::min(d->head_dim, 128 / eb)), 16u};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(std::min(d->head_dim, 128 / eb)), static_cast<cuuint32_t>(rows)};
   cuuint32_t estr[2] = {1u, 1u};
   CUtensorMapDataType dt = d->kv_dtype == DMS_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                            : d->kv_dtype == DMS_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
@@ -152,7 +153,8 @@ struct dms_cache {
   int num_sms;
   std::vector<int> positions;  // host copy of tokens appended per layer
   std::vector<char> prefilled;
-  CUtensorMap kmap, vmap;
+  CUtensorMap kmap, vmap;      // pool pages, 16-row boxes
+  CUtensorMap kmap64, vmap64;  // pool pages, 64-row boxes (flat decode kernel)
   bool has_maps;
   CUtensorMap kept_kmap, kept_vmap;  // tcgen05 prefill: kept copies
   bool has_kept_maps = false;
@@ -236,6 +238,7 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   v.alpha_per = desc->alpha_per;
   v.alpha_source = desc->alpha_source;
   v.disable = desc->disable_eviction ? 1 : 0;
+  v.decode_kernel = desc->decode_kernel;
   v.alpha_scale = desc->alpha_scale;
   v.rms_eps = desc->rms_eps;
   v.num_sms = c->num_sms;
@@ -247,7 +250,7 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   v.page_table = reinterpret_cast<int*>(b + p.page_table);
   v.slot_pos = reinterpret_cast<int*>(b + p.slot_pos);
   v.ring = reinterpret_cast<int*>(b + p.ring);
-  v.plan = reinterpret_cast<int2*>(b + p.plan);
+  v.plan = reinterpret_cast<int4*>(b + p.plan);
   v.kept = reinterpret_cast<int*>(b + p.kept);
   v.kept_count = reinterpret_cast<int*>(b + p.kept_count);
   v.kept_upto = reinterpret_cast<int*>(b + p.kept_upto);
@@ -265,7 +268,8 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   if (desc->kv_dtype != DMS_F32) {
     int prev = cur;
     if (prev != c->device) cudaSetDevice(c->device);
-    c->has_maps = make_pool_map(&c->kmap, v.k_pool, desc) && make_pool_map(&c->vmap, v.v_pool, desc);
+    c->has_maps = make_pool_map(&c->kmap, v.k_pool, desc, 16) && make_pool_map(&c->vmap, v.v_pool, desc, 16) &&
+                  make_pool_map(&c->kmap64, v.k_pool, desc, 64) && make_pool_map(&c->vmap64, v.v_pool, desc, 64);
     if (prev != c->device) cudaSetDevice(prev);
     if (!c->has_maps) {
       delete c;
@@ -484,9 +488,41 @@ int dms_decode_append(dms_cache* c, int layer, const dms_decode_args* a, void* s
   return DMS_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Decode attention over a layer's pages (fused: the whole decode step) with
+// the kernel the descriptor selects; the flat kernel hands shapes it does not
+// stage to the cluster kernel.
+int run_decode_kernel(dms_cache* c, int layer, const void* q, void* o, bool fused, const void* k, const void* v,
+                      float* alpha, const DecideArgs* da, cudaStream_t s) {
+  const CacheView& cv = c->view;
+  int mode = c->desc.decode_kernel;
+  if (mode == DMS_DECODE_AUTO)
+    mode = static_cast<long>(cv.B) * cv.Hkv * 8 <= 2L * c->num_sms ? DMS_DECODE_CLUSTER : DMS_DECODE_FLAT;
+  if (mode == DMS_DECODE_FLAT) {
+    bool taken = false;
+    if (launch_decode_flat(cv, layer, q, o, fused, k, v, alpha, da, &c->kmap64, &c->vmap64, s, &taken) != cudaSuccess)
+      return DMS_ERR_CUDA;
+    if (taken) return DMS_OK;
+  }
+  return launch_decode_cluster(cv, layer, q, o, fused, k, v, alpha, da, &c->kmap, &c->vmap, c->num_sms, s) ==
+                 cudaSuccess
+             ? DMS_OK
+             : DMS_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
 int dms_decode_attention(dms_cache* c, int layer, const void* q, void* o, void* stream) {
   if (!c || !q || !o || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
   if (c->worklist_layer != layer) return DMS_ERR_STATE;
+  if (c->has_maps && c->desc.kv_dtype != DMS_F32)
+    return run_decode_kernel(c, layer, q, o, false, nullptr, nullptr, nullptr, nullptr,
+                             static_cast<cudaStream_t>(stream));
   if (launch_decode_attention(c->view, layer, q, o, c->has_maps ? &c->kmap : nullptr, c->has_maps ? &c->vmap : nullptr,
                               c->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DMS_ERR_CUDA;
@@ -505,10 +541,8 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
     // the append kernel, then the cluster attention over the updated pages.
     int e = dms_decode_append(c, layer, a, stream);
     if (e) return e;
-    return launch_decode_cluster(c->view, layer, a->q, a->o, false, nullptr, nullptr, nullptr, nullptr, &c->kmap,
-                                 &c->vmap, c->num_sms, static_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? DMS_OK
-               : DMS_ERR_CUDA;
+    return run_decode_kernel(c, layer, a->q, a->o, false, nullptr, nullptr, nullptr, nullptr,
+                             static_cast<cudaStream_t>(stream));
   }
   if (layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
   if (!a->q || !a->k || !a->v || !a->alpha) return DMS_ERR_INVALID;
@@ -532,9 +566,7 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   if (proj) da = decide_args(a->decide);
   // bf16 pages: one launch -- attention over the pre-append slots plus the new
   // token, then the append, with the adapter's decision logits computed inside.
-  if (launch_decode_cluster(v, layer, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, &c->kmap,
-                            &c->vmap, c->num_sms, s) != cudaSuccess)
-    return DMS_ERR_CUDA;
+  if (int e = run_decode_kernel(c, layer, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, s)) return e;
   c->positions[layer] += 1;
   c->worklist_layer = layer;
   return DMS_OK;

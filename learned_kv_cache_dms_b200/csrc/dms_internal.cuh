@@ -26,7 +26,7 @@ enum Ctrl {
 // Device view of one cache: sizes and device pointers into the caller buffer.
 struct CacheView {
   int L, B, Hq, Hkv, D, hidden, w, P, maxp, cap, pool_pages, pre_pages, max_pos;
-  int kv_dtype, act_dtype, alpha_per, alpha_source, disable;
+  int kv_dtype, act_dtype, alpha_per, alpha_source, disable, decode_kernel;
   float alpha_scale, rms_eps;
   int num_sms;
   int* ctrl;
@@ -36,7 +36,7 @@ struct CacheView {
   int* page_table;  // [L,B,Hkv,maxp]
   int* slot_pos;    // [L,B,Hkv,cap]
   int* ring;        // [L,B,Hkv,w]
-  int2* plan;       // [2][L,B,Hkv] slot plan of the next append, by parity of its position (next_plan)
+  int4* plan;       // [2][L,B,Hkv] plan of the next append, by parity of its position (next_plan)
   int* kept;        // [B,Hkv,max_pos]   prefill scratch: kept positions, ascending
   int* kept_count;  // [B,Hkv]
   int* kept_upto;   // [B,Hkv,max_pos+1] prefill scratch: kept tokens before position t
@@ -62,8 +62,10 @@ __device__ __forceinline__ void set_status(int* ctrl, int bits) { atomicOr(&ctrl
 
 // Plan entry of head li for the append of the token at position t (the plan is
 // double-buffered by the parity of t so one decode step can read its own plan
-// while writing the next one).
-__device__ __forceinline__ int2* plan_at(const CacheView& c, long li, int t) {
+// while writing the next one).  It also snapshots the head's retained count
+// and page count before that append: a decode launch that appends reads every
+// head's count from here, never from the live count its own CTAs update.
+__device__ __forceinline__ int4* plan_at(const CacheView& c, long li, int t) {
   return c.plan + static_cast<long>(t & 1) * c.L * c.B * c.Hkv + li;
 }
 
@@ -364,6 +366,11 @@ cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, c
 cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q, void* o,
                                     const CUtensorMap* kmap, const CUtensorMap* vmap, int num_sms,
                                     cudaStream_t s);
+// Persistent split-K decode over all SMs; *taken is false (nothing launched)
+// when the shape is outside what the kernel stages in shared memory.
+cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
+                               const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
+                               const CUtensorMap* vmap, cudaStream_t s, bool* taken);
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s);

@@ -22,8 +22,8 @@ __global__ void k_init(CacheView c) {
     if (i < nbh) {
       c.npages[i] = c.pre_pages;
       c.count[i] = 0;
-      c.plan[i] = make_int2(0, 0);
-      c.plan[nbh + i] = make_int2(0, 0);
+      c.plan[i] = make_int4(0, 0, 0, 0);
+      c.plan[nbh + i] = make_int4(0, 0, 0, 0);
     }
     if (i < static_cast<long>(c.B) * c.Hkv) c.head_done[i] = 0;
     if (i < static_cast<long>(c.L) * c.B) c.pos[i] = 0;

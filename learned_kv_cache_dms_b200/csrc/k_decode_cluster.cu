@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   for (int i = tid; i < min(c.maxp, kPtCache); i += kThreads) s_pt[i] = c.page_table[li * c.maxp + i];
   const int cnt = c.count[li];
   const int t = FUSED ? c.pos[layer * c.B + b] : 0;
-  const int2 pl = FUSED ? *plan_at(c, li, t) : make_int2(0, 0);
+  const int4 pl = FUSED ? *plan_at(c, li, t) : make_int4(0, 0, 0, 0);
   const int masked_slot = (FUSED && (pl.y & 1)) ? pl.x : -1;
   const int next_page0 = FUSED ? c.ctrl[CTRL_NEXT_PAGE] : 0;
   const int per = ((cnt + cs - 1) / cs + 15) / 16 * 16;
@@ -313,15 +313,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
       }
       if (tid == 0) {
         // plan of the next append (token t + 1), from the values just written
-        const int tn = t + 1;
-        int2 nx;
-        if (tn >= c.w && (static_cast<unsigned>(s_ring_next) & RING_EVICT))
-          nx = make_int2(s_ring_next & RING_SLOT_MASK, 1);
-        else if (cnt_new >= c.cap)
-          nx = make_int2(-1, 4);
-        else
-          nx = make_int2(cnt_new, (cnt_new % c.P == 0 && cnt_new / c.P >= np_new) ? 2 : 0);
-        *plan_at(c, li, tn) = nx;
+        *plan_at(c, li, t + 1) = make_plan(s_ring_next, t + 1, cnt_new, np_new, c);
       }
     }
   }

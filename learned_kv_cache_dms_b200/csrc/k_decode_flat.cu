@@ -1,0 +1,958 @@
+// Decode attention as one persistent split-K pass over every head's retained
+// slots, balanced across all SMs, and the fused decode step built on it.
+//
+// Work: the retained slots of all (b, h) of a layer, cut into units of 16 * 2^k
+// slots (every head gets at least one unit; k is the smallest leaving each CTA
+// at most 62 units), laid end to end; CTA i of the G CTAs (one per SM) takes
+// units [i*U/G, (i+1)*U/G).  Its range covers the tail of one head, whole
+// heads, and the start of another ("segments").  A producer warp streams the
+// range through a ring of shared-memory stages with TMA, one 64-slot sub-tile
+// per stage (never crossing a page; one box per 128-byte column half of K and
+// of V, plus the head's query rows).  Sub-tile n is consumed by consumer warp
+// n mod 4 from one of that warp's own stages (stage w + 4 * (n/4 mod m), m
+// stages per warp, so every use of a stage is ordered by the one warp that
+// waits on it and no mbarrier is ever waited on two phases ahead), and the
+// warp runs the whole online-softmax update of its 64 keys with the
+// g query heads of the KV head as the M dimension of mma.sync tiles; the four
+// warps' states are merged at the end of each segment ([FastDMS], attention
+// scoring: split-K grouped decode attention over variable-length per-head
+// spans; the balanced flat split keeps every SM streaming whatever the batch
+// and the retained lengths).
+//
+// A head held by one CTA is finished there.  A head shared by n CTAs leaves n
+// partials (acc, running max, running sum; log2 domain) in global scratch;
+// the CTA whose arrival completes the head's counter merges them (LSE
+// combine) and writes the output rows.
+//
+// FUSED (bf16 pages): the whole decode step in this launch, as in the cluster
+// kernel.  The attention covers the slots as they were before this step's
+// append, with the slot this token reuses excluded, plus the new token's
+// key/value taken from the input as one more key, merged in by the finishing
+// CTA -- the same visible set as after the append ([DMS-Qwen3], inference
+// mode).  Every count the partition uses is the snapshot in the append plan,
+// which no CTA of this launch rewrites.  The CTA holding a head's first unit
+// computes the head's decision logit while its first tiles land; the
+// finishing CTA appends the token at the slot planned by the previous step,
+// updates the head's count, grants a page when the slot starts one (ids: the
+// page counter at launch plus the head's rank among the heads needing one,
+// (b, h) row-major) and writes the plan of the next append.  The grid's last
+// CTA advances the page counter and the positions.
+#include <algorithm>
+
+#include "decode_common.cuh"
+
+namespace dms {
+
+#ifdef DMS_TRACE
+__device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
+// mark by any one thread (the producer's lane 0)
+#define FLAT_MARK_ANY(slot)                                                            \
+  do {                                                                                 \
+    unsigned long long t_;                                                             \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                             \
+    if (blockIdx.x < kTraceCtas) g_dms_trace[blockIdx.x * kTraceSlots + (slot)] = t_; \
+  } while (0)
+#else
+#define FLAT_MARK_ANY(slot) \
+  do {                      \
+  } while (0)
+#endif
+
+constexpr int kFlatConsumers = 4;                        // warps computing
+constexpr int kFlatProducer = kFlatConsumers;            // warp issuing the TMA loads
+constexpr int kFlatAux = kFlatConsumers + 1;             // warp preparing the append
+constexpr int kFlatThreads = (kFlatConsumers + 2) * 32;
+constexpr int kFlatPrefetch = 8;                         // segments whose new K/V rows are staged
+constexpr int kFlatUnit = 16;                            // slots per work unit (smallest)
+constexpr int kFlatSegMax = 64;                          // head segments per CTA
+constexpr int kFlatPtMax = 512;                          // page ids staged per CTA
+constexpr int kFlatMaxStages = 16;
+constexpr int kFlatRows = 64;                            // slots per sub-tile = rows per TMA box
+
+struct FlatSeg {
+  int bh;           // head, b * Hkv + h
+  int s0, s1;       // this CTA's slots of the head
+  int n0, n1;       // this CTA's sub-tiles [n0, n1) holding them
+  int nparts;       // CTAs sharing the head
+  int first_cta;    // the first of them
+  int first_pslot;  // partial slot of the first of them
+  int pslot;        // this CTA's partial slot
+  int unit0;        // first unit of the head
+  int pt0;          // first page id of [s0, s1) in s_pt, -1: read from the page table
+  int decide;       // 1: this CTA computes the head's decision logit
+  int t;            // position of the token appended by this step
+  int plx, ply;     // plan of the append: slot, flags (1 reuse, 2 new page, 4 over capacity)
+  int cnt, npages;  // the head's retained slots and pages before the append
+  int grant;        // rank of the head among those taking a new page this step
+  int sp_idx;       // index in s_pt of the page of a reused slot, -1: none staged
+  int ring_idx;     // index in s_ring of the ring entry of position t + 1 - w, -1: none
+};
+
+// Stage and use count of sub-tile n: consumer warp n % 4 owns stages
+// w, w + 4, ..., w + 4 (m - 1) and takes them in turn.
+__device__ __forceinline__ void flat_stage(int n, int m, int* st, int* use) {
+  const int j = n / kFlatConsumers;
+  *st = n % kFlatConsumers + kFlatConsumers * (j % m);
+  *use = j / m;
+}
+
+struct FlatMeta {
+  int slot;  // first slot of the sub-tile
+  int rows;  // slots in the sub-tile (0: an empty segment)
+  float ks;  // FP8 page scales
+  float vs;
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+// Contiguous global -> shared copy completing on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+// Barrier of the four consumer warps only (the producer warp never joins).
+__device__ __forceinline__ void consumers_sync() { asm volatile("barrier.sync 1, 128;\n" ::: "memory"); }
+
+// Adapter decision logit of the new token of sequence b for head `src`, by
+// one warp (eight 16-byte vectors of each operand in flight per lane).
+__device__ __forceinline__ float decide_warp(const CacheView& c, const DecideArgs& a, int b, int src) {
+  const int lane = threadIdx.x & 31;
+  const int hid = c.hidden, nvec = hid / 8;
+  const uint4* xr =
+      reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.hidden) + static_cast<long>(b) * hid);
+  const uint4* wr =
+      reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.W) + static_cast<long>(src) * hid);
+  const uint4* gr = reinterpret_cast<const uint4*>(a.gamma);
+  constexpr int VPT = 8;
+  float ss = 0.f, dot = 0.f;
+  for (int v0 = 0; v0 < nvec; v0 += 32 * VPT) {
+    uint4 xu[VPT], wu[VPT], gu[VPT];
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      const int vi = v0 + u * 32 + lane;
+      const bool ok = vi < nvec;
+      xu[u] = ok ? xr[vi] : make_uint4(0, 0, 0, 0);
+      wu[u] = ok ? wr[vi] : make_uint4(0, 0, 0, 0);
+      gu[u] = ok ? gr[vi] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      float x[8], wv[8], gv[8];
+      unpack16(xu[u], x, static_cast<const __nv_bfloat16*>(nullptr));
+      unpack16(wu[u], wv, static_cast<const __nv_bfloat16*>(nullptr));
+      unpack16(gu[u], gv, static_cast<const __nv_bfloat16*>(nullptr));
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        ss = fmaf(x[e], x[e], ss);
+        dot = fmaf(wv[e] * gv[e], x[e], dot);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  }
+  const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+  const float inv = 1.0f / sqrtf(ss / static_cast<float>(hid) + c.rms_eps);
+  const float z = dot * inv + (bias ? __bfloat162float(bias[src]) : 0.f);
+  return z * c.alpha_scale - a.offset[b * a.offset_bstride + src];
+}
+
+// One warp's online-softmax update over KEYS consecutive keys of a staged tile
+// (bf16, 128-byte swizzled, column halves of TROWS rows of 128 bytes; K and V
+// alike), keys numbered from 0 at the tile's first row.  Keys >= rows and key
+// `masked` are excluded.  Scores are in the log2 domain: s = q.k * kscale *
+// log2(e) / sqrt(D).  The probabilities entering PV are multiplied by `vscale`
+// (the FP8 page scale of V; 1 for bf16 pages), the row sums are not.  The
+// QK^T products of the KEYS/16 key pairs and the PV products of the D/16
+// column pairs are independent mma chains, so one warp keeps the tensor pipe
+// busy on its own.
+template <int D, int KEYS, int TROWS>
+__device__ __forceinline__ void warp_tile_keys(const unsigned char* kt, const unsigned char* vt, int rows, int masked,
+                                               float kscale_l2, float vscale, const uint32_t (&qa)[D / 16][4],
+                                               float (&acc)[D / 8][4], float (&mrow)[2], float (&lrow)[2]) {
+  constexpr int KS = D / 16, NT = D / 8, KP = KEYS / 16;
+  const int lane = threadIdx.x & 31;
+  const int mi = lane >> 3, rr = lane & 7;
+  float s[KP][2][4];
+#pragma unroll
+  for (int kp = 0; kp < KP; ++kp)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) s[kp][nt][0] = s[kp][nt][1] = s[kp][nt][2] = s[kp][nt][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int chunk = 2 * ks + (mi & 1);
+#pragma unroll
+    for (int kp = 0; kp < KP; ++kp) {
+      const int n_row = kp * 16 + (mi >> 1) * 8 + rr;
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4(b0, b1, b2, b3, smem_u32(kt + (chunk / 8) * TROWS * 128 + sw128(n_row, chunk % 8)));
+      uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+      mma_bf16_16816(s[kp][0], qa[ks], bb0);
+      mma_bf16_16816(s[kp][1], qa[ks], bb1);
+    }
+  }
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int kp = 0; kp < KP; ++kp)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = kp * 16 + nt * 8 + 2 * (lane & 3) + (e & 1);
+        const float x = (key < rows && key != masked) ? s[kp][nt][e] * kscale_l2 : -INFINITY;
+        s[kp][nt][e] = x;
+        mx[e >> 1] = fmaxf(mx[e >> 1], x);
+      }
+  float corr[2], mu[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+    const float mn = fmaxf(mrow[r], mx[r]);
+    mu[r] = mn == -INFINITY ? 0.f : mn;
+    corr[r] = exp2f(mrow[r] - mu[r]);
+    mrow[r] = mn;
+  }
+  float rs[2] = {0.f, 0.f};
+#pragma unroll
+  for (int kp = 0; kp < KP; ++kp)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float p = exp2f(s[kp][nt][e] - mu[e >> 1]);
+        s[kp][nt][e] = p;
+        rs[e >> 1] += p;
+      }
+  lrow[0] = lrow[0] * corr[0] + rs[0];
+  lrow[1] = lrow[1] * corr[1] + rs[1];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    acc[nt][0] *= corr[0];
+    acc[nt][1] *= corr[0];
+    acc[nt][2] *= corr[1];
+    acc[nt][3] *= corr[1];
+  }
+#pragma unroll
+  for (int kp = 0; kp < KP; ++kp) {
+    uint32_t pa[4];
+    pa[0] = pack_bf16(s[kp][0][0] * vscale, s[kp][0][1] * vscale);
+    pa[1] = pack_bf16(s[kp][0][2] * vscale, s[kp][0][3] * vscale);
+    pa[2] = pack_bf16(s[kp][1][0] * vscale, s[kp][1][1] * vscale);
+    pa[3] = pack_bf16(s[kp][1][2] * vscale, s[kp][1][3] * vscale);
+    const int n_row = kp * 16 + (mi & 1) * 8 + rr;
+#pragma unroll
+    for (int dp = 0; dp < NT / 2; ++dp) {
+      const int chunk = 2 * dp + (mi >> 1);
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(vt + (chunk / 8) * TROWS * 128 + sw128(n_row, chunk % 8)));
+      uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+      mma_bf16_16816(acc[2 * dp], pa, bb0);
+      mma_bf16_16816(acc[2 * dp + 1], pa, bb1);
+    }
+  }
+}
+
+// Widen rows [r0, r0 + CROWS) of a staged FP8 sub-tile (K then V, unswizzled
+// rows of D codes) to bf16 (exact) in the 128-byte swizzled layout of a
+// CROWS-row tile pair at `conv` (K then V), by one warp.
+template <int D, int CROWS>
+__device__ __forceinline__ void widen_fp8_rows(const unsigned char* raw, unsigned char* conv, int r0) {
+  constexpr int TILE_RAW = kFlatRows * D, CTILE = CROWS * D * 2, CH = D / 16;
+  const int lane = threadIdx.x & 31;
+  for (int idx = lane; idx < 2 * CROWS * CH; idx += 32) {
+    const int which = idx / (CROWS * CH);
+    const int rem = idx % (CROWS * CH);
+    const int r = rem / CH, ch = rem % CH;  // 16 codes of row r0 + r
+    const uint4 u = *reinterpret_cast<const uint4*>(raw + which * TILE_RAW + (r0 + r) * D + ch * 16);
+    const uint32_t wsrc[4] = {u.x, u.y, u.z, u.w};
+    uint32_t wds[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __half2_raw lo =
+          __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(wsrc[e] & 0xFFFFu), __NV_E4M3);
+      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(wsrc[e] >> 16), __NV_E4M3);
+      const float2 fl = __half22float2(__half2(lo)), fh = __half22float2(__half2(hi));
+      wds[2 * e] = pack_bf16(fl.x, fl.y);
+      wds[2 * e + 1] = pack_bf16(fh.x, fh.y);
+    }
+    unsigned char* dstt = conv + which * CTILE;
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      const int chunk = 2 * ch + hc;
+      *reinterpret_cast<uint4*>(dstt + (chunk / 8) * CROWS * 128 + sw128(r, chunk % 8)) =
+          make_uint4(wds[4 * hc], wds[4 * hc + 1], wds[4 * hc + 2], wds[4 * hc + 3]);
+    }
+  }
+}
+
+template <int D, bool FP8>
+struct FlatSmem {
+  static constexpr int HALVES = D / 64;
+  static constexpr int TILE = FP8 ? kFlatRows * D : HALVES * kFlatRows * 128;  // K (or V) of one sub-tile
+  static constexpr int CROWS = D == 64 ? 64 : 32;                              // FP8 rows widened at a time
+  static constexpr int CONV_WARP = FP8 ? 2 * CROWS * D * 2 : 0;                // K + V widened, per warp
+  static constexpr int MLD = D + 2;
+  __host__ __device__ static size_t stage_stride(int g) {
+    return (static_cast<size_t>(2 * TILE) + g * D * 2 + 1023) / 1024 * 1024;
+  }
+  // everything but the stage ring
+  __host__ __device__ static size_t fixed(int g) {
+    return 1024 + static_cast<size_t>(kFlatConsumers) * CONV_WARP + (4 * g + g) * MLD * sizeof(float);
+  }
+};
+
+template <int D, bool FP8, bool FUSED>
+__global__ void __launch_bounds__(kFlatThreads, 1)
+    k_decode_flat(CacheView c, int layer, const __nv_bfloat16* q, __nv_bfloat16* o, int nst,
+                  const __nv_bfloat16* k_new, const __nv_bfloat16* v_new, float* alpha, DecideArgs da, int fuse_decide,
+                  const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
+  using F = FlatSmem<D, FP8>;
+  constexpr int KS = D / 16, NT = D / 8, MLD = D + 2;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sbase =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int g = c.Hq / c.Hkv;
+  const size_t stride = F::stage_stride(g);
+  unsigned char* conv_buf = sbase + nst * stride;                                     // [warp][K, V] (FP8)
+  float* merge = reinterpret_cast<float*>(conv_buf + kFlatConsumers * F::CONV_WARP);  // [4 warps][g][MLD]
+  float* cpart = merge + 4 * g * MLD;                                                 // [g][MLD] merged segment
+  __shared__ uint64_t full_bar[kFlatMaxStages], empty_bar[kFlatMaxStages];
+  __shared__ FlatMeta meta[kFlatMaxStages];
+  __shared__ FlatSeg segs[kFlatSegMax];
+  __shared__ int s_pt[kFlatPtMax];
+  __shared__ long s_ptsrc[kFlatPtMax];
+  __shared__ float s_ks[FP8 ? kFlatPtMax : 1], s_vs[FP8 ? kFlatPtMax : 1];
+  __shared__ int s_ring[kFlatSegMax];
+  __shared__ long s_ringsrc[kFlatSegMax];
+  __shared__ float s_x[FUSED ? kFlatSegMax : 1][16];  // new token's scores per segment
+  __shared__ float s_alpha[FUSED ? kFlatSegMax : 1];   // new token's decision logit per segment
+  __shared__ __align__(16) __nv_bfloat16 s_kvnew[FUSED ? kFlatPrefetch : 1][2][D];  // new K, V rows
+  __shared__ __align__(8) uint64_t aux_bar;
+  __shared__ int s_red[32], s_part[kFlatThreads / 32][8];
+  __shared__ int s_nseg, s_nsub, s_npt, s_nring, s_last, s_next_page0, s_unit;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int BH = c.B * c.Hkv;
+  const long lbase = static_cast<long>(layer) * BH;
+  const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+  DMS_TRACE_MARK(0, 0);
+
+  // ---- setup: every CTA derives the same partition ------------------------
+  // (scratch arrays live in the stage ring, unused until the producer starts)
+  int* s_cnt = reinterpret_cast<int*>(sbase);
+  int* s_off = s_cnt + BH;     // [BH + 1] unit offsets
+  int* s_gr = s_off + BH + 1;  // [BH] new-page ranks
+  int* s_plx = s_gr + BH;      // [BH] plan slot
+  int* s_ply = s_plx + BH;     // [BH] plan flags
+  int* s_npg = s_ply + BH;     // [BH] pages before the append
+  if (tid == 0) {
+    for (int i = 0; i < nst; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    mbar_init(&aux_bar, 1);
+    fence_mbar_init();
+    s_next_page0 = FUSED ? c.ctrl[CTRL_NEXT_PAGE] : 0;
+  }
+  {
+    int part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int i = tid; i < BH; i += kFlatThreads) {
+      int cnt;
+      if (FUSED) {
+        // both parities and the position in one round trip; the plan of
+        // position t holds the count before this step's append
+        const int4 p0 = c.plan[lbase + i];
+        const int4 p1 = c.plan[static_cast<long>(c.L) * BH + lbase + i];
+        const int t = c.pos[layer * c.B + i / c.Hkv];
+        const int4 pl = (t & 1) ? p1 : p0;
+        cnt = pl.z;
+        s_plx[i] = pl.x;
+        s_ply[i] = pl.y;
+        s_npg[i] = pl.w;
+      } else {
+        cnt = c.count[lbase + i];  // nothing in this launch changes it
+      }
+      s_cnt[i] = cnt;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) part[k] += max(1, (cnt + (kFlatUnit << k) - 1) / (kFlatUnit << k));
+    }
+    // unit size: the smallest 16 * 2^k slots leaving at most kFlatSegMax - 2
+    // units per CTA, so a CTA's range meets at most that many heads
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) part[k] += __shfl_xor_sync(0xffffffffu, part[k], o2);
+    if (lane == 0)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) s_part[warp][k] = part[k];
+    __syncthreads();
+    if (tid == 0) {
+      int k = 0;
+      for (;; ++k) {
+        long tot = 0;
+        for (int wv = 0; wv < kFlatThreads / 32; ++wv) tot += s_part[wv][k];
+        if (k == 7 || (tot + G - 1) / G <= kFlatSegMax - 2) break;
+      }
+      s_unit = kFlatUnit << k;
+    }
+    __syncthreads();
+  }
+  const int unit = s_unit;
+  {
+    int base = 0, gbase = 0;
+    for (int i0 = 0; i0 < BH; i0 += kFlatThreads) {
+      const int i = i0 + tid;
+      const int n = i < BH ? max(1, (s_cnt[i] + unit - 1) / unit) : 0;
+      int tot;
+      const int off = block_exclusive_scan(n, s_red, &tot);
+      if (i < BH) s_off[i] = base + off;
+      base += tot;
+      if (FUSED) {
+        const int np = (i < BH && (s_ply[i] & 2)) ? 1 : 0;
+        const int goff = block_exclusive_scan(np, s_red, &tot);
+        if (i < BH) s_gr[i] = gbase + goff;
+        gbase += tot;
+      }
+    }
+    if (tid == 0) s_off[BH] = base;
+  }
+  __syncthreads();
+  const long U = s_off[BH];
+  const long u0 = static_cast<long>(cta) * U / G, u1 = static_cast<long>(cta + 1) * U / G;
+  auto cta_of = [&](long u) { return static_cast<int>(((u + 1) * G - 1) / U); };
+  if (tid == 0) {
+    int nseg = 0, nsub = 0, npt = 0, nring = 0;
+    if (u0 < u1) {
+      int lo = 0, hi = BH - 1;  // last head starting at or before u0
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= u0) lo = mid; else hi = mid - 1;
+      }
+      for (int h = lo; h < BH && s_off[h] < u1; ++h) {
+        if (nseg == kFlatSegMax) {
+          set_status(c.ctrl, DMS_ST_SPLIT_LIMIT);
+          break;
+        }
+        FlatSeg sg;
+        const int cnt = s_cnt[h];
+        const long li = lbase + h;
+        sg.bh = h;
+        sg.cnt = cnt;
+        sg.s0 = static_cast<int>(max(0L, u0 - s_off[h]) * unit);
+        sg.s1 = static_cast<int>(min(static_cast<long>(cnt), (u1 - s_off[h]) * unit));
+        if (sg.s0 > sg.s1) sg.s0 = sg.s1;  // an empty head's only unit
+        const int fc = cta_of(s_off[h]), lc = cta_of(s_off[h + 1] - 1);
+        sg.first_cta = fc;
+        // with fewer units than CTAs most CTAs are empty: the head's parts are
+        // then the CTAs of its units, one unit each
+        sg.nparts = min(lc - fc + 1, s_off[h + 1] - s_off[h]);
+        sg.unit0 = s_off[h];
+        const long fu0 = static_cast<long>(fc) * U / G;
+        sg.first_pslot = 2 * fc + (s_off[h] != fu0 ? 1 : 0);
+        sg.pslot = cta == fc ? sg.first_pslot : 2 * cta;
+        sg.decide = (FUSED && fuse_decide && s_off[h] >= u0) ? 1 : 0;
+        sg.t = FUSED ? c.pos[layer * c.B + h / c.Hkv] : 0;
+        sg.plx = FUSED ? s_plx[h] : 0;
+        sg.ply = FUSED ? s_ply[h] : 0;
+        sg.npages = FUSED ? s_npg[h] : 0;
+        sg.grant = FUSED ? s_gr[h] : 0;
+        sg.pt0 = -1;
+        sg.n0 = nsub;
+        if (sg.s1 > sg.s0) {
+          const int p0 = sg.s0 / c.P, p1 = (sg.s1 - 1) / c.P;
+          if (npt + (p1 - p0 + 1) <= kFlatPtMax) {
+            sg.pt0 = npt;
+            for (int p = p0; p <= p1; ++p) s_ptsrc[npt++] = li * c.maxp + p;
+          }
+          for (int s = sg.s0; s < sg.s1;) {
+            s += min(min(kFlatRows, sg.s1 - s), c.P - s % c.P);
+            ++nsub;
+          }
+        } else {
+          ++nsub;  // one empty sub-tile carries the segment's end
+        }
+        sg.n1 = nsub;
+        // what the finishing CTA of the head needs, fetched with the page ids
+        sg.sp_idx = -1;
+        sg.ring_idx = -1;
+        if (FUSED) {
+          if ((sg.ply & 1) && npt < kFlatPtMax) {
+            sg.sp_idx = npt;
+            s_ptsrc[npt++] = li * c.maxp + sg.plx / c.P;
+          }
+          if (sg.t + 1 >= c.w) {
+            sg.ring_idx = nring;
+            s_ringsrc[nring++] = li * c.w + (sg.t + 1) % c.w;
+          }
+        }
+        segs[nseg++] = sg;
+      }
+    }
+    s_nseg = nseg;
+    s_nsub = nsub;
+    s_npt = npt;
+    s_nring = nring;
+  }
+  __syncthreads();
+  const int nseg = s_nseg, nsub = s_nsub;
+  for (int i = tid; i < s_npt; i += kFlatThreads) s_pt[i] = c.page_table[s_ptsrc[i]];
+  if (FUSED)
+    for (int i = tid; i < s_nring; i += kFlatThreads) s_ring[i] = c.ring[s_ringsrc[i]];
+  if (FP8) {
+    __syncthreads();
+    for (int i = tid; i < s_npt; i += kFlatThreads) {
+      s_ks[i] = c.k_scale[s_pt[i]];
+      s_vs[i] = c.v_scale[s_pt[i]];
+    }
+  }
+  __syncthreads();
+  DMS_TRACE_MARK(0, 1);
+
+  if (warp == kFlatAux) {
+    // ---- aux: what the append of each head needs, while the tiles stream --
+    // (the new token's scores and K/V rows, its decision logit), then a
+    // release of aux_bar that the consumers acquire before any head is handed
+    // over or finished
+    if (FUSED) {
+      for (int k = 0; k < nseg; ++k) {
+        const FlatSeg& sg = segs[k];
+        const int bh = sg.bh, b = bh / c.Hkv, h = bh % c.Hkv;
+        const __nv_bfloat16* qrow = q + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D;
+        const __nv_bfloat16* kn = k_new + static_cast<long>(bh) * D;
+        const __nv_bfloat16* vn = v_new + static_cast<long>(bh) * D;
+        float kv[D / 32];
+        __nv_bfloat16 kb[D / 32], vb[D / 32];
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          kb[j] = kn[lane + 32 * j];
+          vb[j] = vn[lane + 32 * j];
+          kv[j] = __bfloat162float(kb[j]);
+        }
+        if (k < kFlatPrefetch) {
+#pragma unroll
+          for (int j = 0; j < D / 32; ++j) {
+            s_kvnew[k][0][lane + 32 * j] = kb[j];
+            s_kvnew[k][1][lane + 32 * j] = vb[j];
+          }
+        }
+        for (int r = 0; r < g; ++r) {
+          float sdot = 0.f;
+#pragma unroll
+          for (int j = 0; j < D / 32; ++j)
+            sdot = fmaf(__bfloat162float(qrow[static_cast<long>(r) * D + lane + 32 * j]), kv[j], sdot);
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, o2);
+          if (lane == 0) s_x[k][r] = sdot * sl2;
+        }
+        float a = 0.f;
+        if (sg.decide) {
+          // decision logit of a head whose first unit is here (layer
+          // granularity: head 0's logit for every head)
+          a = decide_warp(c, da, b, c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h);
+          if (lane == 0) alpha[b * c.Hkv + h] = a;
+        } else if (!fuse_decide) {
+          // written by the neuron pass before this launch
+          a = __ldcg(&alpha[b * c.Hkv + (c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h)]);
+        } else {
+          a = NAN;  // computed by another CTA: read when finishing
+        }
+        if (lane == 0) s_alpha[k] = a;
+      }
+      __threadfence();  // the logits written here are visible before any hand-over
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&aux_bar);
+    DMS_TRACE_MARK(0, 2);
+  } else if (warp == kFlatProducer) {
+    // ---- producer: one thread issues every TMA load of this CTA -----------
+    if (lane == 0) {
+      int n = 0;
+      bool timed_out = false;
+      for (int k = 0; k < nseg; ++k) {
+        const FlatSeg sg = segs[k];
+        const long li = lbase + sg.bh;
+        const int b = sg.bh / c.Hkv, h = sg.bh % c.Hkv;
+        const __nv_bfloat16* qrow = q + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D;
+        int s = sg.s0;
+        do {
+          const int rows = s < sg.s1 ? min(min(kFlatRows, sg.s1 - s), c.P - s % c.P) : 0;
+          int st, use;
+          flat_stage(n, nst / kFlatConsumers, &st, &use);
+          if (use > 0 && !mbar_wait_bounded(&empty_bar[st], (use - 1) & 1)) timed_out = true;
+          FlatMeta m;
+          m.slot = s;
+          m.rows = rows;
+          m.ks = m.vs = 1.0f;
+          int page = 0;
+          if (rows > 0) {
+            const int pi = s / c.P;
+            if (sg.pt0 >= 0) {
+              const int e = sg.pt0 + pi - sg.s0 / c.P;
+              page = s_pt[e];
+              if (FP8) {
+                m.ks = s_ks[e];
+                m.vs = s_vs[e];
+              }
+            } else {
+              page = c.page_table[li * c.maxp + pi];
+              if (FP8) {
+                m.ks = c.k_scale[page];
+                m.vs = c.v_scale[page];
+              }
+            }
+          }
+          meta[st] = m;
+          unsigned char* dst = sbase + st * stride;
+          const uint32_t bytes = (rows > 0 ? 2u * F::TILE : 0u) + static_cast<uint32_t>(g * D * 2);
+          mbar_expect_tx(&full_bar[st], bytes);
+          if (rows > 0) {
+            const int row0 = page * c.P + s % c.P;
+            if (FP8) {
+              tma_load_2d(dst, &kmap, 0, row0, &full_bar[st]);
+              tma_load_2d(dst + F::TILE, &vmap, 0, row0, &full_bar[st]);
+            } else {
+#pragma unroll
+              for (int hf = 0; hf < F::HALVES; ++hf) {
+                tma_load_2d(dst + hf * kFlatRows * 128, &kmap, hf * 64, row0, &full_bar[st]);
+                tma_load_2d(dst + F::TILE + hf * kFlatRows * 128, &vmap, hf * 64, row0, &full_bar[st]);
+              }
+            }
+          }
+          bulk_load(dst + 2 * F::TILE, qrow, static_cast<uint32_t>(g * D * 2), &full_bar[st]);
+          s += rows;
+          ++n;
+          if (n == 1) FLAT_MARK_ANY(10);
+          if (n == nst) FLAT_MARK_ANY(11);
+        } while (s < sg.s1);
+      }
+      // nothing may still be landing in shared memory when the CTA exits
+      for (int j = max(0, n - nst); j < n; ++j) {
+        int st, use;
+        flat_stage(j, nst / kFlatConsumers, &st, &use);
+        if (!mbar_wait_bounded(&full_bar[st], use & 1)) timed_out = true;
+      }
+      FLAT_MARK_ANY(12);
+      if (timed_out) set_status(c.ctrl, DMS_ST_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ---- consumers ---------------------------------------------------------
+    uint32_t qa[KS][4];
+    float acc[NT][4];
+    float mrow[2], lrow[2];
+    bool timed_out = false;
+    for (int k = 0; k < nseg; ++k) {
+      const FlatSeg& sg = segs[k];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+      mrow[0] = mrow[1] = -INFINITY;
+      lrow[0] = lrow[1] = 0.f;
+      bool have_q = false;
+      const int masked_slot = (FUSED && (sg.ply & 1)) ? sg.plx : -1;
+      // this warp's sub-tiles of the segment: n = warp (mod 4)
+      for (int n = sg.n0 + ((warp - sg.n0) % kFlatConsumers + kFlatConsumers) % kFlatConsumers; n < sg.n1;
+           n += kFlatConsumers) {
+        int st, use;
+        flat_stage(n, nst / kFlatConsumers, &st, &use);
+        const bool ok = mbar_wait_bounded(&full_bar[st], use & 1);
+        if (!ok) timed_out = true;
+        if (n == 0) DMS_TRACE_MARK(0, 3);
+        if (n == nsub / 2) DMS_TRACE_MARK(0, 4);
+        const FlatMeta m = meta[st];
+        const unsigned char* stage = sbase + st * stride;
+        if (!have_q) {
+          load_q_frags<D>(reinterpret_cast<const __nv_bfloat16*>(stage + 2 * F::TILE), g, qa);
+          have_q = true;
+        }
+        if (ok && m.rows > 0) {
+          const int masked = masked_slot >= 0 ? masked_slot - m.slot : -1;
+          if (FP8) {
+            unsigned char* cv = conv_buf + warp * F::CONV_WARP;
+#pragma unroll
+            for (int cb = 0; cb < kFlatRows; cb += F::CROWS) {
+              if (cb >= m.rows) break;
+              widen_fp8_rows<D, F::CROWS>(stage, cv, cb);
+              __syncwarp();
+              warp_tile_keys<D, F::CROWS, F::CROWS>(cv, cv + F::CROWS * D * 2, m.rows - cb,
+                                                    masked >= 0 ? masked - cb : -1, m.ks * sl2, m.vs, qa, acc, mrow,
+                                                    lrow);
+              __syncwarp();
+            }
+          } else {
+            warp_tile_keys<D, kFlatRows, kFlatRows>(stage, stage + F::TILE, m.rows, masked, sl2, 1.0f, qa, acc,
+                                                    mrow, lrow);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[st]);
+      }
+
+      // ---- end of a segment: merge the warps, finish or hand over the head --
+      if (k == 0) DMS_TRACE_MARK(0, 5);
+      const int bh = sg.bh, b = bh / c.Hkv, h = bh % c.Hkv;
+      const long li = lbase + bh;
+      warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
+      if (k == 0 && !mbar_wait_bounded(&aux_bar, 0)) timed_out = true;
+      consumers_sync();
+      merge_sources<D>(merge, kFlatConsumers, g, 1.0f, [&](int r, int d, float v) { cpart[r * MLD + d] = v; });
+      consumers_sync();
+      bool finish = sg.nparts == 1;
+      if (!finish) {
+        for (int idx = tid; idx < g * (D + 2); idx += 128) {
+          const int r = idx / (D + 2), d = idx % (D + 2);
+          if (d < D)
+            c.part_acc[(static_cast<long>(sg.pslot) * g + r) * D + d] = cpart[r * MLD + d];
+          else
+            c.part_ml[(static_cast<long>(sg.pslot) * g + r) * 2 + (d - D)] = cpart[r * MLD + d];
+        }
+        __threadfence();
+        consumers_sync();
+        if (tid == 0) {
+          const int old = atomicAdd(&c.head_done[bh], 1);
+          s_last = old == sg.nparts - 1;
+          if (s_last) c.head_done[bh] = 0;
+        }
+        consumers_sync();
+        finish = s_last;
+        if (finish) __threadfence();
+      }
+      if (finish) {
+        // sources: the head's partials (this CTA's in shared memory when it
+        // holds the whole head) and, fused, the new token
+        const int np = sg.nparts;
+        auto pslot_of = [&](int p) {
+          const int cp = U < G ? cta_of(sg.unit0 + p) : sg.first_cta + p;
+          return static_cast<long>(p == 0 ? sg.first_pslot : 2 * cp);
+        };
+        // online LSE merge of the sources, one thread per (row, 4 columns)
+        constexpr int Q4 = D / 4;
+        for (int idx = tid; idx < g * Q4; idx += 128) {
+          const int r = idx / Q4, d4 = idx % Q4;
+          float M = -INFINITY, L = 0.f;
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+          auto add = [&](float m, float l, float4 v) {
+            if (m == -INFINITY) return;  // a source without visible keys
+            if (m > M) {
+              const float f = exp2f(M - m);
+              a.x *= f;
+              a.y *= f;
+              a.z *= f;
+              a.w *= f;
+              L *= f;
+              M = m;
+            }
+            const float wgt = exp2f(m - M);
+            L = fmaf(wgt, l, L);
+            a.x = fmaf(wgt, v.x, a.x);
+            a.y = fmaf(wgt, v.y, a.y);
+            a.z = fmaf(wgt, v.z, a.z);
+            a.w = fmaf(wgt, v.w, a.w);
+          };
+          uint2 vv = make_uint2(0u, 0u);
+          if (FUSED)
+            vv = k < kFlatPrefetch ? *reinterpret_cast<const uint2*>(&s_kvnew[k][1][4 * d4])
+                                   : *reinterpret_cast<const uint2*>(v_new + static_cast<long>(bh) * D + 4 * d4);
+          if (np == 1) {
+            const float* cp = cpart + r * MLD;
+            add(cp[D], cp[D + 1], make_float4(cp[4 * d4], cp[4 * d4 + 1], cp[4 * d4 + 2], cp[4 * d4 + 3]));
+          } else {
+            int p = 0;
+            for (; p + 4 <= np; p += 4) {
+              float4 v[4];
+              float2 ml[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const long ps = pslot_of(p + u);
+                v[u] = __ldcg(reinterpret_cast<const float4*>(c.part_acc + (ps * g + r) * D) + d4);
+                ml[u] = __ldcg(reinterpret_cast<const float2*>(c.part_ml + (ps * g + r) * 2));
+              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u) add(ml[u].x, ml[u].y, v[u]);
+            }
+            for (; p < np; ++p) {
+              const long ps = pslot_of(p);
+              const float2 ml = __ldcg(reinterpret_cast<const float2*>(c.part_ml + (ps * g + r) * 2));
+              add(ml.x, ml.y, __ldcg(reinterpret_cast<const float4*>(c.part_acc + (ps * g + r) * D) + d4));
+            }
+          }
+          if (FUSED) {
+            const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv.x));
+            const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv.y));
+            add(s_x[k][r], 1.0f, make_float4(v01.x, v01.y, v23.x, v23.y));
+          }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          uint2 pk;
+          pk.x = pack_bf16(a.x * inv, a.y * inv);
+          pk.y = pack_bf16(a.z * inv, a.w * inv);
+          *reinterpret_cast<uint2*>(o + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g + r) * D + 4 * d4) =
+              pk;
+        }
+
+        if (FUSED) {
+          // append of the token at the planned slot: every CTA reading this
+          // head has arrived, so its pages are no longer read in this launch
+          const int flags = sg.ply, slot = sg.plx, t = sg.t, cnt = sg.cnt;
+          bool okp = !(flags & 4);
+          int id = -1;
+          const int np_old = sg.npages;
+          if (okp && (flags & 2)) {
+            id = s_next_page0 + sg.grant;
+            if (id >= c.pool_pages || np_old >= c.maxp) okp = false;
+          } else if (okp) {
+            id = sg.sp_idx >= 0 ? s_pt[sg.sp_idx] : c.page_table[li * c.maxp + slot / c.P];
+          }
+          int cnt_new = cnt, np_new = np_old;
+          if (okp) {
+            const long row = static_cast<long>(id) * c.P + slot % c.P;
+            if (tid < D / 8) {
+              const uint4* ksrc = k < kFlatPrefetch ? reinterpret_cast<const uint4*>(s_kvnew[k][0])
+                                                    : reinterpret_cast<const uint4*>(k_new + static_cast<long>(bh) * D);
+              const uint4* vsrc = k < kFlatPrefetch ? reinterpret_cast<const uint4*>(s_kvnew[k][1])
+                                                    : reinterpret_cast<const uint4*>(v_new + static_cast<long>(bh) * D);
+              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.k_pool) + row * D)[tid] = ksrc[tid];
+              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.v_pool) + row * D)[tid] = vsrc[tid];
+            }
+            if (!(flags & 1)) cnt_new = cnt + 1;
+            if (flags & 2) np_new += 1;
+          }
+          if (tid == 0) {
+            if (okp) {
+              if (flags & 2) {
+                c.page_table[li * c.maxp + np_new - 1] = id;
+                c.npages[li] = np_new;
+                atomicAdd(&c.ctrl[CTRL_STEP_PAGES], 1);
+              }
+              const int hs = (fuse_decide || c.alpha_per != DMS_ALPHA_PER_LAYER) ? h : 0;
+              const float av = s_alpha[k] == s_alpha[k] ? s_alpha[k] : __ldcg(&alpha[b * c.Hkv + hs]);
+              const bool evict = !c.disable && av > 0.0f;
+              c.slot_pos[li * c.cap + slot] = t;
+              c.ring[li * c.w + t % c.w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
+              if (!(flags & 1)) c.count[li] = cnt_new;
+            } else {
+              set_status(c.ctrl, (flags & 4) ? DMS_ST_CAPACITY : DMS_ST_POOL_EXHAUSTED);
+            }
+            // plan of the next append (token t + 1), with its count snapshot
+            const int tn = t + 1;
+            const int rn = sg.ring_idx >= 0 ? s_ring[sg.ring_idx] : 0;
+            *plan_at(c, li, tn) = make_plan(rn, tn, cnt_new, np_new, c);
+          }
+        }
+      }
+      consumers_sync();  // merge buffers are reused by the next segment
+      if (k == 0) DMS_TRACE_MARK(0, finish ? 7 : 6);
+      if (finish) DMS_TRACE_MARK(0, 13);
+    }
+    DMS_TRACE_MARK(0, 8);
+    if (timed_out && lane == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
+  }
+
+  if (FUSED) {
+    // the grid's last CTA advances the page counter and the positions
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      s_last = (atomicAdd(&c.ctrl[CTRL_GRID_DONE], 1) == G - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      if (tid == 0) {
+        const int granted = __ldcg(&c.ctrl[CTRL_STEP_PAGES]);
+        c.ctrl[CTRL_NEXT_PAGE] = min(__ldcg(&c.ctrl[CTRL_NEXT_PAGE]) + granted, c.pool_pages);
+        c.ctrl[CTRL_STEP_PAGES] = 0;
+        c.ctrl[CTRL_GRID_DONE] = 0;
+      }
+      for (int bb = tid; bb < c.B; bb += kFlatThreads) c.pos[layer * c.B + bb] += 1;
+    }
+  }
+  DMS_TRACE_MARK(0, 9);
+}
+
+// Launch geometry of the flat kernel, or false when the shape is outside what
+// it stages in shared memory (the caller then takes the cluster kernel).
+template <int D, bool FP8, bool FUSED>
+static bool flat_geometry(const CacheView& c, int* grid, int* nst, size_t* smem) {
+  using F = FlatSmem<D, FP8>;
+  static int budget = -1;  // dynamic shared memory a block may take beside its static arrays
+  if (budget < 0) {
+    int dev = 0, optin = 0;
+    cudaFuncAttributes fa{};
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, k_decode_flat<D, FP8, FUSED>) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    budget = optin - static_cast<int>(fa.sharedSizeBytes);
+  }
+  const int g = c.Hq / c.Hkv, BH = c.B * c.Hkv;
+  const int G = std::min(c.num_sms, c.items_cap / 2);
+  if (G <= 0) return false;
+  // the largest unit (2048 slots) must leave every CTA at most kFlatSegMax - 2 units
+  if ((BH + G - 1) / G > kFlatSegMax - 2) return false;
+  const size_t fixed = F::fixed(g), stride = F::stage_stride(g);
+  if (budget <= 0 || fixed + kFlatConsumers * stride > static_cast<size_t>(budget)) return false;
+  // a whole number of stages per consumer warp
+  const int n = static_cast<int>(std::min<size_t>(kFlatMaxStages, (budget - fixed) / stride)) / kFlatConsumers *
+                kFlatConsumers;
+  if (n < kFlatConsumers) return false;
+  // the partition scratch (6 ints per head) lives in the stage ring
+  if (static_cast<size_t>(6 * BH + 8) * sizeof(int) > n * stride) return false;
+  *grid = G;
+  *nst = n;
+  *smem = fixed + n * stride;
+  return true;
+}
+
+template <int D, bool FP8, bool FUSED>
+static cudaError_t launch_flat_t(const CacheView& c, int layer, const void* q, void* o, const void* k, const void* v,
+                                 float* alpha, const DecideArgs* da, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                 cudaStream_t s, bool* taken) {
+  int grid = 0, nst = 0;
+  size_t smem = 0;
+  *taken = (reinterpret_cast<uintptr_t>(q) & 15) == 0 && flat_geometry<D, FP8, FUSED>(c, &grid, &nst, &smem);
+  if (!*taken) return cudaSuccess;
+  auto kern = k_decode_flat<D, FP8, FUSED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  DecideArgs none{};
+  kern<<<grid, kFlatThreads, smem, s>>>(c, layer, static_cast<const __nv_bfloat16*>(q),
+                                        static_cast<__nv_bfloat16*>(o), nst, static_cast<const __nv_bfloat16*>(k),
+                                        static_cast<const __nv_bfloat16*>(v), alpha, da ? *da : none, da ? 1 : 0,
+                                        *kmap, *vmap);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
+                               const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
+                               const CUtensorMap* vmap, cudaStream_t s, bool* taken) {
+  *taken = false;
+  if (!kmap || !vmap || c.kv_dtype == DMS_F32) return cudaErrorInvalidValue;
+  if (fused) {
+    if (c.kv_dtype != DMS_BF16) return cudaErrorInvalidValue;
+    return c.D == 64 ? launch_flat_t<64, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, s, taken)
+                     : launch_flat_t<128, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, s, taken);
+  }
+  if (c.kv_dtype == DMS_FP8_E4M3)
+    return c.D == 64 ? launch_flat_t<64, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, taken)
+                     : launch_flat_t<128, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, taken);
+  return c.D == 64 ? launch_flat_t<64, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, taken)
+                   : launch_flat_t<128, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, taken);
+}
+
+}  // namespace dms
+
+#ifdef DMS_TRACE
+// Copy the flat kernel's phase timeline to the host (tracing builds only).
+extern "C" __attribute__((visibility("default"))) int dms_debug_trace_read_flat(void* host, size_t bytes) {
+  const size_t n = sizeof(dms::g_dms_trace) < bytes ? sizeof(dms::g_dms_trace) : bytes;
+  return cudaMemcpyFromSymbol(host, dms::g_dms_trace, n) == cudaSuccess ? 0 : -3;
+}
+#endif

@@ -46,6 +46,7 @@ class Case:
     seed: int = 1
     attn_rows: int | None = None  # sample this many prefill rows (None: all)
     staged: bool = False          # decode through dms_decode_append + dms_decode_attention
+    kernel: str = "auto"          # decode attention kernel: auto | cluster | flat
 
     @property
     def N(self):
@@ -171,6 +172,8 @@ def make_desc(B_, case: Case):
         d.hidden = max(d.hidden, 8)
     d.alpha_scale, d.rms_eps = ALPHA_SCALE, RMS_EPS
     d.disable_eviction = int(case.disable)
+    d.decode_kernel = {"auto": B_.DMS_DECODE_AUTO, "cluster": B_.DMS_DECODE_CLUSTER,
+                       "flat": B_.DMS_DECODE_FLAT}[case.kernel]
     return d
 
 

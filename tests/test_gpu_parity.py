@@ -1,6 +1,8 @@
 """GPU parity: libdms (through the C ABI) against the CPU oracle on the same
 seeded inputs.  Sizes are small enough for the oracle to finish in seconds but
 span several tiles, pages and a ragged tail."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -69,10 +71,14 @@ def test_case_inputs_and_oracle(name):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("kernel", ["cluster", "flat"])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_gpu_parity(name):
-    errs = check_case(CASES[name])
-    print(name, errs)
+def test_gpu_parity(name, kernel):
+    """Every case through both decode attention kernels (one cluster per head;
+    one CTA per SM over the flat slot list)."""
+    case = dataclasses.replace(CASES[name], kernel=kernel)
+    errs = check_case(case)
+    print(name, kernel, errs)
 
 
 @pytest.mark.gpu
