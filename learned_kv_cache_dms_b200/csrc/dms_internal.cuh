@@ -73,7 +73,7 @@ __device__ __forceinline__ int4* plan_at(const CacheView& c, long li, int t) {
 // each CTA stores %globaltimer for phase `slot` of kernel `kid` into a
 // per-translation-unit device array read back by dms_debug_trace_read.
 #ifdef DMS_TRACE
-constexpr int kTraceCtas = 4096, kTraceSlots = 16;
+constexpr int kTraceCtas = 4096, kTraceSlots = 32;
 #define DMS_TRACE_MARK(kid, slot)                                                                   \
   do {                                                                                              \
     if (threadIdx.x == 0 && blockIdx.x < kTraceCtas) {                                              \

@@ -22,7 +22,10 @@
 // A head held by one CTA is finished there.  A head shared by n CTAs leaves n
 // partials (acc, running max, running sum; log2 domain) in global scratch;
 // the CTA whose arrival completes the head's counter merges them (LSE
-// combine) and writes the output rows.
+// combine) and writes the output rows.  The consumers only merge their four
+// warp states at a segment's end and hand the result to an aux warp through a
+// two-deep ring; the aux warp writes partials, counts arrivals and finishes
+// heads while the consumers stream on.
 //
 // FUSED (bf16 pages): the whole decode step in this launch, as in the cluster
 // kernel.  The attention covers the slots as they were before this step's
@@ -66,6 +69,7 @@ constexpr int kFlatPrefetch = 8;                         // segments whose new K
 constexpr int kFlatUnit = 16;                            // slots per work unit (smallest)
 constexpr int kFlatSegMax = 64;                          // head segments per CTA
 constexpr int kFlatPtMax = 512;                          // page ids staged per CTA
+constexpr int kFlatSubMax = 256;                         // sub-tile descriptors staged per CTA
 constexpr int kFlatMaxStages = 16;
 constexpr int kFlatRows = 64;                            // slots per sub-tile = rows per TMA box
 
@@ -86,6 +90,7 @@ struct FlatSeg {
   int grant;        // rank of the head among those taking a new page this step
   int sp_idx;       // index in s_pt of the page of a reused slot, -1: none staged
   int ring_idx;     // index in s_ring of the ring entry of position t + 1 - w, -1: none
+  int qoff;         // element offset of the head's query rows in q
 };
 
 // Stage and use count of sub-tile n: consumer warp n % 4 owns stages
@@ -303,7 +308,7 @@ struct FlatSmem {
   }
   // everything but the stage ring
   __host__ __device__ static size_t fixed(int g) {
-    return 1024 + static_cast<size_t>(kFlatConsumers) * CONV_WARP + (4 * g + g) * MLD * sizeof(float);
+    return 1024 + static_cast<size_t>(kFlatConsumers) * CONV_WARP + (4 * g + 2 * g) * MLD * sizeof(float);
   }
 };
 
@@ -321,19 +326,23 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
   const size_t stride = F::stage_stride(g);
   unsigned char* conv_buf = sbase + nst * stride;                                     // [warp][K, V] (FP8)
   float* merge = reinterpret_cast<float*>(conv_buf + kFlatConsumers * F::CONV_WARP);  // [4 warps][g][MLD]
-  float* cpart = merge + 4 * g * MLD;                                                 // [g][MLD] merged segment
+  float* cpart = merge + 4 * g * MLD;  // [2][g][MLD] merged segments handed to the aux warp
   __shared__ uint64_t full_bar[kFlatMaxStages], empty_bar[kFlatMaxStages];
   __shared__ FlatMeta meta[kFlatMaxStages];
   __shared__ FlatSeg segs[kFlatSegMax];
   __shared__ int s_pt[kFlatPtMax];
   __shared__ long s_ptsrc[kFlatPtMax];
-  __shared__ float s_ks[FP8 ? kFlatPtMax : 1], s_vs[FP8 ? kFlatPtMax : 1];
+  __shared__ int4 s_sub[kFlatSubMax];                               // sub-tile descriptors
+  __shared__ int s_n0[kFlatSegMax];                                 // first sub-tile of each segment
+  __shared__ float s_ks[FP8 ? kFlatSubMax : 1], s_vs[FP8 ? kFlatSubMax : 1];  // FP8 scales per sub-tile
   __shared__ int s_ring[kFlatSegMax];
   __shared__ long s_ringsrc[kFlatSegMax];
   __shared__ float s_x[FUSED ? kFlatSegMax : 1][16];  // new token's scores per segment
   __shared__ float s_alpha[FUSED ? kFlatSegMax : 1];   // new token's decision logit per segment
   __shared__ __align__(16) __nv_bfloat16 s_kvnew[FUSED ? kFlatPrefetch : 1][2][D];  // new K, V rows
-  __shared__ __align__(8) uint64_t aux_bar;
+  __shared__ __align__(8) uint64_t hq_full[2], hq_empty[2];  // merged-segment hand-over ring
+  __shared__ __align__(8) uint64_t aux_done;                 // every hand-over processed
+  __shared__ int s_fin[kFlatSegMax], s_nfin;                 // heads the consumers finish
   __shared__ int s_red[32], s_part[kFlatThreads / 32][8];
   __shared__ int s_nseg, s_nsub, s_npt, s_nring, s_last, s_next_page0, s_unit;
 
@@ -352,12 +361,23 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
   int* s_plx = s_gr + BH;      // [BH] plan slot
   int* s_ply = s_plx + BH;     // [BH] plan flags
   int* s_npg = s_ply + BH;     // [BH] pages before the append
+  int* s_tpos = s_npg + BH;    // [BH] position of the appended token
+  if (warp == kFlatProducer && lane == 0) {
+    // the TMA descriptors, fetched while the partition is worked out
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
+  }
   if (tid == 0) {
     for (int i = 0; i < nst; ++i) {
       mbar_init(&full_bar[i], 1);
       mbar_init(&empty_bar[i], 1);
     }
-    mbar_init(&aux_bar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&hq_full[i], 1);
+      mbar_init(&hq_empty[i], 1);
+    }
+    mbar_init(&aux_done, 1);
+    s_nfin = 0;
     fence_mbar_init();
     s_next_page0 = FUSED ? c.ctrl[CTRL_NEXT_PAGE] : 0;
   }
@@ -376,6 +396,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
         s_plx[i] = pl.x;
         s_ply[i] = pl.y;
         s_npg[i] = pl.w;
+        s_tpos[i] = t;
       } else {
         cnt = c.count[lbase + i];  // nothing in this launch changes it
       }
@@ -404,7 +425,11 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     }
     __syncthreads();
   }
+  DMS_TRACE_MARK(0, 16);
   const int unit = s_unit;
+  // sub-tile chunk: the largest of 64, 32, 16 slots dividing the page size,
+  // so chunks never cross a page
+  const int chunk = c.P % kFlatRows == 0 ? kFlatRows : c.P % 32 == 0 ? 32 : 16;
   {
     int base = 0, gbase = 0;
     for (int i0 = 0; i0 < BH; i0 += kFlatThreads) {
@@ -424,102 +449,290 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     if (tid == 0) s_off[BH] = base;
   }
   __syncthreads();
+  DMS_TRACE_MARK(0, 17);
   const long U = s_off[BH];
   const long u0 = static_cast<long>(cta) * U / G, u1 = static_cast<long>(cta + 1) * U / G;
   auto cta_of = [&](long u) { return static_cast<int>(((u + 1) * G - 1) / U); };
-  if (tid == 0) {
-    int nseg = 0, nsub = 0, npt = 0, nring = 0;
-    if (u0 < u1) {
-      int lo = 0, hi = BH - 1;  // last head starting at or before u0
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_off[mid] <= u0) lo = mid; else hi = mid - 1;
-      }
-      for (int h = lo; h < BH && s_off[h] < u1; ++h) {
-        if (nseg == kFlatSegMax) {
-          set_status(c.ctrl, DMS_ST_SPLIT_LIMIT);
-          break;
-        }
-        FlatSeg sg;
-        const int cnt = s_cnt[h];
-        const long li = lbase + h;
-        sg.bh = h;
-        sg.cnt = cnt;
-        sg.s0 = static_cast<int>(max(0L, u0 - s_off[h]) * unit);
-        sg.s1 = static_cast<int>(min(static_cast<long>(cnt), (u1 - s_off[h]) * unit));
-        if (sg.s0 > sg.s1) sg.s0 = sg.s1;  // an empty head's only unit
-        const int fc = cta_of(s_off[h]), lc = cta_of(s_off[h + 1] - 1);
-        sg.first_cta = fc;
-        // with fewer units than CTAs most CTAs are empty: the head's parts are
-        // then the CTAs of its units, one unit each
-        sg.nparts = min(lc - fc + 1, s_off[h + 1] - s_off[h]);
-        sg.unit0 = s_off[h];
-        const long fu0 = static_cast<long>(fc) * U / G;
-        sg.first_pslot = 2 * fc + (s_off[h] != fu0 ? 1 : 0);
-        sg.pslot = cta == fc ? sg.first_pslot : 2 * cta;
-        sg.decide = (FUSED && fuse_decide && s_off[h] >= u0) ? 1 : 0;
-        sg.t = FUSED ? c.pos[layer * c.B + h / c.Hkv] : 0;
-        sg.plx = FUSED ? s_plx[h] : 0;
-        sg.ply = FUSED ? s_ply[h] : 0;
-        sg.npages = FUSED ? s_npg[h] : 0;
-        sg.grant = FUSED ? s_gr[h] : 0;
-        sg.pt0 = -1;
-        sg.n0 = nsub;
-        if (sg.s1 > sg.s0) {
-          const int p0 = sg.s0 / c.P, p1 = (sg.s1 - 1) / c.P;
-          if (npt + (p1 - p0 + 1) <= kFlatPtMax) {
-            sg.pt0 = npt;
-            for (int p = p0; p <= p1; ++p) s_ptsrc[npt++] = li * c.maxp + p;
-          }
-          for (int s = sg.s0; s < sg.s1;) {
-            s += min(min(kFlatRows, sg.s1 - s), c.P - s % c.P);
-            ++nsub;
-          }
-        } else {
-          ++nsub;  // one empty sub-tile carries the segment's end
-        }
-        sg.n1 = nsub;
-        // what the finishing CTA of the head needs, fetched with the page ids
-        sg.sp_idx = -1;
-        sg.ring_idx = -1;
-        if (FUSED) {
-          if ((sg.ply & 1) && npt < kFlatPtMax) {
-            sg.sp_idx = npt;
-            s_ptsrc[npt++] = li * c.maxp + sg.plx / c.P;
-          }
-          if (sg.t + 1 >= c.w) {
-            sg.ring_idx = nring;
-            s_ringsrc[nring++] = li * c.w + (sg.t + 1) % c.w;
-          }
-        }
-        segs[nseg++] = sg;
-      }
+  // heads [h_lo, h_hi] meet this CTA's units (binary searches in every thread)
+  int h_lo = 0, h_hi = -1;
+  if (u0 < u1) {
+    int lo = 0, hi = BH - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= u0) lo = mid; else hi = mid - 1;
     }
+    h_lo = lo;
+    hi = BH - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] < u1) lo = mid; else hi = mid - 1;
+    }
+    h_hi = lo;
+  }
+  int nseg = h_hi - h_lo + 1;
+  if (nseg > kFlatSegMax) {
+    if (tid == 0) set_status(c.ctrl, DMS_ST_SPLIT_LIMIT);
+    nseg = kFlatSegMax;
+  }
+  // one thread per segment: its slots and parts, and how many sub-tiles, page
+  // ids and ring entries it needs (offsets by block scans)
+  FlatSeg sg{};
+  int my_sub = 0, my_pt = 0, my_ring = 0, p0 = 0, p1 = -1;
+  long li = 0;
+  if (tid < nseg) {
+    const int h = h_lo + tid;
+    const int cnt = s_cnt[h];
+    li = lbase + h;
+    sg.bh = h;
+    sg.cnt = cnt;
+    sg.s0 = static_cast<int>(max(0L, u0 - s_off[h]) * unit);
+    sg.s1 = static_cast<int>(min(static_cast<long>(cnt), (u1 - s_off[h]) * unit));
+    if (sg.s0 > sg.s1) sg.s0 = sg.s1;  // an empty head's only unit
+    sg.unit0 = s_off[h];
+    if (s_off[h] >= u0 && s_off[h + 1] <= u1) {
+      sg.nparts = 1;  // the whole head is here
+      sg.first_cta = cta;
+      sg.first_pslot = sg.pslot = 2 * cta;
+    } else {
+      const int fc = cta_of(s_off[h]), lc = cta_of(s_off[h + 1] - 1);
+      sg.first_cta = fc;
+      // with fewer units than CTAs most CTAs are empty: the head's parts are
+      // then the CTAs of its units, one unit each
+      sg.nparts = min(lc - fc + 1, s_off[h + 1] - s_off[h]);
+      const long fu0 = static_cast<long>(fc) * U / G;
+      sg.first_pslot = 2 * fc + (s_off[h] != fu0 ? 1 : 0);
+      sg.pslot = cta == fc ? sg.first_pslot : 2 * cta;
+    }
+    sg.decide = (FUSED && fuse_decide && s_off[h] >= u0) ? 1 : 0;
+    const int b = h / c.Hkv;
+    sg.t = FUSED ? s_tpos[h] : 0;
+    sg.plx = FUSED ? s_plx[h] : 0;
+    sg.ply = FUSED ? s_ply[h] : 0;
+    sg.npages = FUSED ? s_npg[h] : 0;
+    sg.grant = FUSED ? s_gr[h] : 0;
+    sg.qoff = (b * c.Hq + (h % c.Hkv) * g) * D;
+    if (sg.s1 > sg.s0) {
+      p0 = sg.s0 / c.P;
+      p1 = (sg.s1 - 1) / c.P;
+      my_sub = (sg.s1 - 1) / chunk - sg.s0 / chunk + 1;
+      my_pt = p1 - p0 + 1;
+    } else {
+      my_sub = 1;  // one empty sub-tile carries the segment's end
+    }
+    if (FUSED && (sg.ply & 1)) ++my_pt;  // page of the reused slot
+    my_ring = (FUSED && sg.t + 1 >= c.w) ? 1 : 0;
+  }
+  int tot_sub, tot_pt, tot_ring;
+  const int sub0 = block_exclusive_scan(my_sub, s_red, &tot_sub);
+  const int pt0 = block_exclusive_scan(my_pt, s_red, &tot_pt);
+  const int ring0 = block_exclusive_scan(my_ring, s_red, &tot_ring);
+  const bool pt_ok = tot_pt <= kFlatPtMax, table = tot_sub <= kFlatSubMax;
+  if (tid < nseg) {
+    sg.n0 = sub0;
+    sg.n1 = sub0 + my_sub;
+    sg.pt0 = (pt_ok && sg.s1 > sg.s0) ? pt0 : -1;
+    sg.sp_idx = (pt_ok && FUSED && (sg.ply & 1)) ? pt0 + my_pt - 1 : -1;
+    sg.ring_idx = my_ring ? ring0 : -1;
+    if (pt_ok) {
+      for (int p = p0; p <= p1; ++p) s_ptsrc[pt0 + p - p0] = li * c.maxp + p;
+      if (sg.sp_idx >= 0) s_ptsrc[sg.sp_idx] = li * c.maxp + sg.plx / c.P;
+    }
+    if (my_ring) s_ringsrc[ring0] = li * c.w + (sg.t + 1) % c.w;
+    segs[tid] = sg;
+    s_n0[tid] = sub0;
+  }
+  if (tid == 0) {
     s_nseg = nseg;
-    s_nsub = nsub;
-    s_npt = npt;
-    s_nring = nring;
+    s_nsub = tot_sub;
+    s_npt = pt_ok ? tot_pt : 0;
+    s_nring = tot_ring;
   }
   __syncthreads();
-  const int nseg = s_nseg, nsub = s_nsub;
+  DMS_TRACE_MARK(0, 18);
+  nseg = s_nseg;
+  const int nsub = s_nsub;
+  // page ids and ring entries in one round trip, and meanwhile the sub-tile
+  // descriptors, one thread per sub-tile: chunk i of a segment covers slots
+  // [max(s0, (s0/C + i) C), min(s1, (s0/C + i + 1) C)), C the chunk size
   for (int i = tid; i < s_npt; i += kFlatThreads) s_pt[i] = c.page_table[s_ptsrc[i]];
   if (FUSED)
     for (int i = tid; i < s_nring; i += kFlatThreads) s_ring[i] = c.ring[s_ringsrc[i]];
-  if (FP8) {
-    __syncthreads();
-    for (int i = tid; i < s_npt; i += kFlatThreads) {
-      s_ks[i] = c.k_scale[s_pt[i]];
-      s_vs[i] = c.v_scale[s_pt[i]];
+  int4 dsc[(kFlatSubMax + kFlatThreads - 1) / kFlatThreads];
+  if (table) {
+#pragma unroll
+    for (int e = 0; e < (kFlatSubMax + kFlatThreads - 1) / kFlatThreads; ++e) {
+      const int n = tid + e * kFlatThreads;
+      if (n >= nsub) break;
+      int lo = 0, hi = nseg - 1;  // the segment holding sub-tile n
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_n0[mid] <= n) lo = mid; else hi = mid - 1;
+      }
+      const FlatSeg& gs = segs[lo];
+      int slot = gs.s0, rows = 0;
+      if (gs.s1 > gs.s0) {
+        const int cs = gs.s0 / chunk + (n - s_n0[lo]);
+        slot = max(gs.s0, cs * chunk);
+        rows = min(gs.s1, cs * chunk + chunk) - slot;
+      }
+      const int pte = gs.pt0 >= 0 && rows > 0 ? gs.pt0 + slot / c.P - gs.s0 / c.P : -1;
+      dsc[e] = make_int4(slot, rows | (lo << 8), 0, pte);
+    }
+  }
+  __syncthreads();
+  if (table) {
+    // pool rows of the sub-tiles (and FP8 page scales)
+#pragma unroll
+    for (int e = 0; e < (kFlatSubMax + kFlatThreads - 1) / kFlatThreads; ++e) {
+      const int n = tid + e * kFlatThreads;
+      if (n >= nsub) break;
+      int4 d = dsc[e];
+      if ((d.y & 255) > 0) {
+        const FlatSeg& gs = segs[d.y >> 8];
+        const int page = d.w >= 0 ? s_pt[d.w] : c.page_table[(lbase + gs.bh) * c.maxp + d.x / c.P];
+        d.z = page * c.P + d.x % c.P;
+        if (FP8) {
+          s_ks[n] = c.k_scale[page];
+          s_vs[n] = c.v_scale[page];
+        }
+      }
+      s_sub[n] = d;
     }
   }
   __syncthreads();
   DMS_TRACE_MARK(0, 1);
 
+  // Finish head segs[k]: LSE merge of its sources (the CTA's merged state
+  // `cp` when it holds the whole head, else the partials in global scratch)
+  // and, fused, the new token; output rows; append.  Threads tix of nth.
+  auto finish_head = [&](int k, const float* cp, int tix, int nth) {
+        const FlatSeg& sg = segs[k];
+        const int bh = sg.bh, b = bh / c.Hkv, h = bh % c.Hkv;
+        const long li = lbase + bh;
+        const int np = sg.nparts;
+        auto pslot_of = [&](int p) {
+          const int cpi = U < G ? cta_of(sg.unit0 + p) : sg.first_cta + p;
+          return static_cast<long>(p == 0 ? sg.first_pslot : 2 * cpi);
+        };
+        // online LSE merge of the sources, one lane per (row, 4 columns)
+        constexpr int Q4 = D / 4;
+        for (int idx = tix; idx < g * Q4; idx += nth) {
+          const int r = idx / Q4, d4 = idx % Q4;
+          float M = -INFINITY, L = 0.f;
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+          auto add = [&](float m, float l, float4 v) {
+            if (m == -INFINITY) return;  // a source without visible keys
+            if (m > M) {
+              const float f = exp2f(M - m);
+              a.x *= f;
+              a.y *= f;
+              a.z *= f;
+              a.w *= f;
+              L *= f;
+              M = m;
+            }
+            const float wgt = exp2f(m - M);
+            L = fmaf(wgt, l, L);
+            a.x = fmaf(wgt, v.x, a.x);
+            a.y = fmaf(wgt, v.y, a.y);
+            a.z = fmaf(wgt, v.z, a.z);
+            a.w = fmaf(wgt, v.w, a.w);
+          };
+          uint2 vv = make_uint2(0u, 0u);
+          if (FUSED)
+            vv = k < kFlatPrefetch ? *reinterpret_cast<const uint2*>(&s_kvnew[k][1][4 * d4])
+                                   : *reinterpret_cast<const uint2*>(v_new + static_cast<long>(bh) * D + 4 * d4);
+          if (np == 1) {
+            const float* cr = cp + r * MLD;
+            add(cr[D], cr[D + 1], make_float4(cr[4 * d4], cr[4 * d4 + 1], cr[4 * d4 + 2], cr[4 * d4 + 3]));
+          } else {
+            int p = 0;
+            for (; p + 4 <= np; p += 4) {
+              float4 v[4];
+              float2 ml[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const long ps = pslot_of(p + u);
+                v[u] = __ldcg(reinterpret_cast<const float4*>(c.part_acc + (ps * g + r) * D) + d4);
+                ml[u] = __ldcg(reinterpret_cast<const float2*>(c.part_ml + (ps * g + r) * 2));
+              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u) add(ml[u].x, ml[u].y, v[u]);
+            }
+            for (; p < np; ++p) {
+              const long ps = pslot_of(p);
+              const float2 ml = __ldcg(reinterpret_cast<const float2*>(c.part_ml + (ps * g + r) * 2));
+              add(ml.x, ml.y, __ldcg(reinterpret_cast<const float4*>(c.part_acc + (ps * g + r) * D) + d4));
+            }
+          }
+          if (FUSED) {
+            const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv.x));
+            const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv.y));
+            add(s_x[k][r], 1.0f, make_float4(v01.x, v01.y, v23.x, v23.y));
+          }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          uint2 pk;
+          pk.x = pack_bf16(a.x * inv, a.y * inv);
+          pk.y = pack_bf16(a.z * inv, a.w * inv);
+          *reinterpret_cast<uint2*>(o + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g + r) * D + 4 * d4) =
+              pk;
+        }
+        if (tix == 0) FLAT_MARK_ANY(13);
+        if (FUSED) {
+          // append of the token at the planned slot: every CTA reading this
+          // head has arrived, so its pages are no longer read in this launch
+          const int flags = sg.ply, slot = sg.plx, t = sg.t, cnt = sg.cnt;
+          bool okp = !(flags & 4);
+          int id = -1;
+          const int np_old = sg.npages;
+          if (okp && (flags & 2)) {
+            id = s_next_page0 + sg.grant;
+            if (id >= c.pool_pages || np_old >= c.maxp) okp = false;
+          } else if (okp) {
+            id = sg.sp_idx >= 0 ? s_pt[sg.sp_idx] : c.page_table[li * c.maxp + slot / c.P];
+          }
+          int cnt_new = cnt, np_new = np_old;
+          if (okp) {
+            const long row = static_cast<long>(id) * c.P + slot % c.P;
+            for (int e = tix; e < D / 8; e += nth) {
+              const uint4* ksrc = k < kFlatPrefetch ? reinterpret_cast<const uint4*>(s_kvnew[k][0])
+                                                    : reinterpret_cast<const uint4*>(k_new + static_cast<long>(bh) * D);
+              const uint4* vsrc = k < kFlatPrefetch ? reinterpret_cast<const uint4*>(s_kvnew[k][1])
+                                                    : reinterpret_cast<const uint4*>(v_new + static_cast<long>(bh) * D);
+              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.k_pool) + row * D)[e] = ksrc[e];
+              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.v_pool) + row * D)[e] = vsrc[e];
+            }
+            if (!(flags & 1)) cnt_new = cnt + 1;
+            if (flags & 2) np_new += 1;
+          }
+          if (tix == 0) {
+            if (okp) {
+              if (flags & 2) {
+                c.page_table[li * c.maxp + np_new - 1] = id;
+                c.npages[li] = np_new;
+                atomicAdd(&c.ctrl[CTRL_STEP_PAGES], 1);
+              }
+              const int hs = (fuse_decide || c.alpha_per != DMS_ALPHA_PER_LAYER) ? h : 0;
+              const float av = s_alpha[k] == s_alpha[k] ? s_alpha[k] : __ldcg(&alpha[b * c.Hkv + hs]);
+              const bool evict = !c.disable && av > 0.0f;
+              c.slot_pos[li * c.cap + slot] = t;
+              c.ring[li * c.w + t % c.w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
+              if (!(flags & 1)) c.count[li] = cnt_new;
+            } else {
+              set_status(c.ctrl, (flags & 4) ? DMS_ST_CAPACITY : DMS_ST_POOL_EXHAUSTED);
+            }
+            // plan of the next append (token t + 1), with its count snapshot
+            const int tn = t + 1;
+            const int rn = sg.ring_idx >= 0 ? s_ring[sg.ring_idx] : 0;
+            *plan_at(c, li, tn) = make_plan(rn, tn, cnt_new, np_new, c);
+            FLAT_MARK_ANY(15);
+          }
+        }
+      };
+
   if (warp == kFlatAux) {
-    // ---- aux: what the append of each head needs, while the tiles stream --
-    // (the new token's scores and K/V rows, its decision logit), then a
-    // release of aux_bar that the consumers acquire before any head is handed
-    // over or finished
+    // ---- aux: first what the append of each head needs, while the tiles
+    // stream (the new token's scores and K/V rows, its decision logit) ------
     if (FUSED) {
       for (int k = 0; k < nseg; ++k) {
         const FlatSeg& sg = segs[k];
@@ -568,74 +781,122 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
       __threadfence();  // the logits written here are visible before any hand-over
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&aux_bar);
-    DMS_TRACE_MARK(0, 2);
+    if (lane == 0) FLAT_MARK_ANY(2);
+    // ---- hand-overs, in segment order: the consumers' merged state of
+    // segment k arrives in cpart[k & 1].  A head held here alone is finished
+    // here from it; a head shared with other CTAs leaves its partial and
+    // counts its arrival, and its last arrival is queued for the consumers
+    // (a merge over global partials wants more than one warp)
+    bool aux_timed_out = false;
+    for (int k = 0; k < nseg; ++k) {
+      const int j = k & 1;
+      if (!mbar_wait_bounded(&hq_full[j], (k >> 1) & 1)) aux_timed_out = true;
+      const FlatSeg& sg = segs[k];
+      const float* cp = cpart + j * g * MLD;
+      const int bh = sg.bh;
+      bool finish = sg.nparts == 1;
+      if (!finish) {
+        for (int idx = lane; idx < g * (D + 2); idx += 32) {
+          const int r = idx / (D + 2), d = idx % (D + 2);
+          if (d < D)
+            c.part_acc[(static_cast<long>(sg.pslot) * g + r) * D + d] = cp[r * MLD + d];
+          else
+            c.part_ml[(static_cast<long>(sg.pslot) * g + r) * 2 + (d - D)] = cp[r * MLD + d];
+        }
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          last = atomicAdd(&c.head_done[bh], 1) == sg.nparts - 1;
+          if (last) c.head_done[bh] = 0;
+        }
+        finish = __shfl_sync(0xffffffffu, last, 0) != 0;
+        if (finish) __threadfence();
+        if (k == 0 && lane == 0) FLAT_MARK_ANY(finish ? 4 : 6);
+      }
+      if (finish && sg.nparts == 1) {
+        finish_head(k, cp, lane, 32);  // held here alone: sources in shared memory
+      } else if (finish && lane == 0) {
+        s_fin[s_nfin++] = k;  // the head's last part: finished by the consumers
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&hq_empty[j]);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&aux_done);  // releases s_fin
+    if (aux_timed_out && lane == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
   } else if (warp == kFlatProducer) {
     // ---- producer: one thread issues every TMA load of this CTA -----------
     if (lane == 0) {
-      int n = 0;
       bool timed_out = false;
-      for (int k = 0; k < nseg; ++k) {
-        const FlatSeg sg = segs[k];
-        const long li = lbase + sg.bh;
-        const int b = sg.bh / c.Hkv, h = sg.bh % c.Hkv;
-        const __nv_bfloat16* qrow = q + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D;
-        int s = sg.s0;
-        do {
-          const int rows = s < sg.s1 ? min(min(kFlatRows, sg.s1 - s), c.P - s % c.P) : 0;
-          int st, use;
-          flat_stage(n, nst / kFlatConsumers, &st, &use);
-          if (use > 0 && !mbar_wait_bounded(&empty_bar[st], (use - 1) & 1)) timed_out = true;
-          FlatMeta m;
-          m.slot = s;
-          m.rows = rows;
-          m.ks = m.vs = 1.0f;
-          int page = 0;
-          if (rows > 0) {
-            const int pi = s / c.P;
-            if (sg.pt0 >= 0) {
-              const int e = sg.pt0 + pi - sg.s0 / c.P;
-              page = s_pt[e];
-              if (FP8) {
-                m.ks = s_ks[e];
-                m.vs = s_vs[e];
-              }
-            } else {
-              page = c.page_table[li * c.maxp + pi];
-              if (FP8) {
-                m.ks = c.k_scale[page];
-                m.vs = c.v_scale[page];
-              }
-            }
-          }
-          meta[st] = m;
-          unsigned char* dst = sbase + st * stride;
-          const uint32_t bytes = (rows > 0 ? 2u * F::TILE : 0u) + static_cast<uint32_t>(g * D * 2);
-          mbar_expect_tx(&full_bar[st], bytes);
-          if (rows > 0) {
-            const int row0 = page * c.P + s % c.P;
-            if (FP8) {
-              tma_load_2d(dst, &kmap, 0, row0, &full_bar[st]);
-              tma_load_2d(dst + F::TILE, &vmap, 0, row0, &full_bar[st]);
-            } else {
+      const int mper = nst / kFlatConsumers;
+      // sub-tile n into its stage once the stage's previous use is released:
+      // K and V boxes and the head's query rows
+      auto issue = [&](int n, int slot, int rows, int row0, float ks, float vs, int qoff) {
+        int st, use;
+        flat_stage(n, mper, &st, &use);
+        if (use > 0 && !mbar_wait_bounded(&empty_bar[st], (use - 1) & 1)) timed_out = true;
+        FlatMeta m;
+        m.slot = slot;
+        m.rows = rows;
+        m.ks = ks;
+        m.vs = vs;
+        meta[st] = m;
+        unsigned char* dst = sbase + st * stride;
+        const uint32_t bytes = (rows > 0 ? 2u * F::TILE : 0u) + static_cast<uint32_t>(g * D * 2);
+        mbar_expect_tx(&full_bar[st], bytes);
+        if (rows > 0) {
+          if (FP8) {
+            tma_load_2d(dst, &kmap, 0, row0, &full_bar[st]);
+            tma_load_2d(dst + F::TILE, &vmap, 0, row0, &full_bar[st]);
+          } else {
 #pragma unroll
-              for (int hf = 0; hf < F::HALVES; ++hf) {
-                tma_load_2d(dst + hf * kFlatRows * 128, &kmap, hf * 64, row0, &full_bar[st]);
-                tma_load_2d(dst + F::TILE + hf * kFlatRows * 128, &vmap, hf * 64, row0, &full_bar[st]);
-              }
+            for (int hf = 0; hf < F::HALVES; ++hf) {
+              tma_load_2d(dst + hf * kFlatRows * 128, &kmap, hf * 64, row0, &full_bar[st]);
+              tma_load_2d(dst + F::TILE + hf * kFlatRows * 128, &vmap, hf * 64, row0, &full_bar[st]);
             }
           }
-          bulk_load(dst + 2 * F::TILE, qrow, static_cast<uint32_t>(g * D * 2), &full_bar[st]);
-          s += rows;
-          ++n;
-          if (n == 1) FLAT_MARK_ANY(10);
-          if (n == nst) FLAT_MARK_ANY(11);
-        } while (s < sg.s1);
+        }
+        bulk_load(dst + 2 * F::TILE, q + qoff, static_cast<uint32_t>(g * D * 2), &full_bar[st]);
+        if (n == 0) FLAT_MARK_ANY(10);
+        if (n == 1) FLAT_MARK_ANY(14);
+        if (n == nst - 1) FLAT_MARK_ANY(11);
+      };
+      if (table) {
+        for (int n = 0; n < nsub; ++n) {
+          const int4 d = s_sub[n];
+          issue(n, d.x, d.y & 255, d.z, FP8 ? s_ks[n] : 1.0f, FP8 ? s_vs[n] : 1.0f, segs[d.y >> 8].qoff);
+        }
+      } else {
+        // more sub-tiles than the descriptor table holds: worked out on the way
+        int n = 0;
+        for (int k = 0; k < nseg; ++k) {
+          const FlatSeg sg = segs[k];
+          const long lh = lbase + sg.bh;
+          int s = sg.s0;
+          do {
+            const int rows = s < sg.s1 ? min(sg.s1, (s / chunk + 1) * chunk) - s : 0;
+            int row0 = 0;
+            float ks = 1.0f, vs = 1.0f;
+            if (rows > 0) {
+              const int pi = s / c.P;
+              const int page = sg.pt0 >= 0 ? s_pt[sg.pt0 + pi - sg.s0 / c.P] : c.page_table[lh * c.maxp + pi];
+              row0 = page * c.P + s % c.P;
+              if (FP8) {
+                ks = c.k_scale[page];
+                vs = c.v_scale[page];
+              }
+            }
+            issue(n, s, rows, row0, ks, vs, sg.qoff);
+            s += rows;
+            ++n;
+          } while (s < sg.s1);
+        }
       }
       // nothing may still be landing in shared memory when the CTA exits
-      for (int j = max(0, n - nst); j < n; ++j) {
+      for (int j = max(0, nsub - nst); j < nsub; ++j) {
         int st, use;
-        flat_stage(j, nst / kFlatConsumers, &st, &use);
+        flat_stage(j, mper, &st, &use);
         if (!mbar_wait_bounded(&full_bar[st], use & 1)) timed_out = true;
       }
       FLAT_MARK_ANY(12);
@@ -664,7 +925,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
         const bool ok = mbar_wait_bounded(&full_bar[st], use & 1);
         if (!ok) timed_out = true;
         if (n == 0) DMS_TRACE_MARK(0, 3);
-        if (n == nsub / 2) DMS_TRACE_MARK(0, 4);
         const FlatMeta m = meta[st];
         const unsigned char* stage = sbase + st * stride;
         if (!have_q) {
@@ -694,162 +954,22 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
         if (lane == 0) mbar_arrive(&empty_bar[st]);
       }
 
-      // ---- end of a segment: merge the warps, finish or hand over the head --
+      // ---- end of a segment: merge the four warps' states into cpart[k & 1]
+      // (once the aux warp has released it) and hand it over -----------------
       if (k == 0) DMS_TRACE_MARK(0, 5);
-      const int bh = sg.bh, b = bh / c.Hkv, h = bh % c.Hkv;
-      const long li = lbase + bh;
+      const int j = k & 1;
       warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
-      if (k == 0 && !mbar_wait_bounded(&aux_bar, 0)) timed_out = true;
+      if (k >= 2 && !mbar_wait_bounded(&hq_empty[j], ((k >> 1) - 1) & 1)) timed_out = true;
       consumers_sync();
-      merge_sources<D>(merge, kFlatConsumers, g, 1.0f, [&](int r, int d, float v) { cpart[r * MLD + d] = v; });
+      float* cpj = cpart + j * g * MLD;
+      merge_sources<D>(merge, kFlatConsumers, g, 1.0f, [&](int r, int d, float v) { cpj[r * MLD + d] = v; });
       consumers_sync();
-      bool finish = sg.nparts == 1;
-      if (!finish) {
-        for (int idx = tid; idx < g * (D + 2); idx += 128) {
-          const int r = idx / (D + 2), d = idx % (D + 2);
-          if (d < D)
-            c.part_acc[(static_cast<long>(sg.pslot) * g + r) * D + d] = cpart[r * MLD + d];
-          else
-            c.part_ml[(static_cast<long>(sg.pslot) * g + r) * 2 + (d - D)] = cpart[r * MLD + d];
-        }
-        __threadfence();
-        consumers_sync();
-        if (tid == 0) {
-          const int old = atomicAdd(&c.head_done[bh], 1);
-          s_last = old == sg.nparts - 1;
-          if (s_last) c.head_done[bh] = 0;
-        }
-        consumers_sync();
-        finish = s_last;
-        if (finish) __threadfence();
-      }
-      if (finish) {
-        // sources: the head's partials (this CTA's in shared memory when it
-        // holds the whole head) and, fused, the new token
-        const int np = sg.nparts;
-        auto pslot_of = [&](int p) {
-          const int cp = U < G ? cta_of(sg.unit0 + p) : sg.first_cta + p;
-          return static_cast<long>(p == 0 ? sg.first_pslot : 2 * cp);
-        };
-        // online LSE merge of the sources, one thread per (row, 4 columns)
-        constexpr int Q4 = D / 4;
-        for (int idx = tid; idx < g * Q4; idx += 128) {
-          const int r = idx / Q4, d4 = idx % Q4;
-          float M = -INFINITY, L = 0.f;
-          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-          auto add = [&](float m, float l, float4 v) {
-            if (m == -INFINITY) return;  // a source without visible keys
-            if (m > M) {
-              const float f = exp2f(M - m);
-              a.x *= f;
-              a.y *= f;
-              a.z *= f;
-              a.w *= f;
-              L *= f;
-              M = m;
-            }
-            const float wgt = exp2f(m - M);
-            L = fmaf(wgt, l, L);
-            a.x = fmaf(wgt, v.x, a.x);
-            a.y = fmaf(wgt, v.y, a.y);
-            a.z = fmaf(wgt, v.z, a.z);
-            a.w = fmaf(wgt, v.w, a.w);
-          };
-          uint2 vv = make_uint2(0u, 0u);
-          if (FUSED)
-            vv = k < kFlatPrefetch ? *reinterpret_cast<const uint2*>(&s_kvnew[k][1][4 * d4])
-                                   : *reinterpret_cast<const uint2*>(v_new + static_cast<long>(bh) * D + 4 * d4);
-          if (np == 1) {
-            const float* cp = cpart + r * MLD;
-            add(cp[D], cp[D + 1], make_float4(cp[4 * d4], cp[4 * d4 + 1], cp[4 * d4 + 2], cp[4 * d4 + 3]));
-          } else {
-            int p = 0;
-            for (; p + 4 <= np; p += 4) {
-              float4 v[4];
-              float2 ml[4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const long ps = pslot_of(p + u);
-                v[u] = __ldcg(reinterpret_cast<const float4*>(c.part_acc + (ps * g + r) * D) + d4);
-                ml[u] = __ldcg(reinterpret_cast<const float2*>(c.part_ml + (ps * g + r) * 2));
-              }
-#pragma unroll
-              for (int u = 0; u < 4; ++u) add(ml[u].x, ml[u].y, v[u]);
-            }
-            for (; p < np; ++p) {
-              const long ps = pslot_of(p);
-              const float2 ml = __ldcg(reinterpret_cast<const float2*>(c.part_ml + (ps * g + r) * 2));
-              add(ml.x, ml.y, __ldcg(reinterpret_cast<const float4*>(c.part_acc + (ps * g + r) * D) + d4));
-            }
-          }
-          if (FUSED) {
-            const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv.x));
-            const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv.y));
-            add(s_x[k][r], 1.0f, make_float4(v01.x, v01.y, v23.x, v23.y));
-          }
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          uint2 pk;
-          pk.x = pack_bf16(a.x * inv, a.y * inv);
-          pk.y = pack_bf16(a.z * inv, a.w * inv);
-          *reinterpret_cast<uint2*>(o + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g + r) * D + 4 * d4) =
-              pk;
-        }
-
-        if (FUSED) {
-          // append of the token at the planned slot: every CTA reading this
-          // head has arrived, so its pages are no longer read in this launch
-          const int flags = sg.ply, slot = sg.plx, t = sg.t, cnt = sg.cnt;
-          bool okp = !(flags & 4);
-          int id = -1;
-          const int np_old = sg.npages;
-          if (okp && (flags & 2)) {
-            id = s_next_page0 + sg.grant;
-            if (id >= c.pool_pages || np_old >= c.maxp) okp = false;
-          } else if (okp) {
-            id = sg.sp_idx >= 0 ? s_pt[sg.sp_idx] : c.page_table[li * c.maxp + slot / c.P];
-          }
-          int cnt_new = cnt, np_new = np_old;
-          if (okp) {
-            const long row = static_cast<long>(id) * c.P + slot % c.P;
-            if (tid < D / 8) {
-              const uint4* ksrc = k < kFlatPrefetch ? reinterpret_cast<const uint4*>(s_kvnew[k][0])
-                                                    : reinterpret_cast<const uint4*>(k_new + static_cast<long>(bh) * D);
-              const uint4* vsrc = k < kFlatPrefetch ? reinterpret_cast<const uint4*>(s_kvnew[k][1])
-                                                    : reinterpret_cast<const uint4*>(v_new + static_cast<long>(bh) * D);
-              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.k_pool) + row * D)[tid] = ksrc[tid];
-              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.v_pool) + row * D)[tid] = vsrc[tid];
-            }
-            if (!(flags & 1)) cnt_new = cnt + 1;
-            if (flags & 2) np_new += 1;
-          }
-          if (tid == 0) {
-            if (okp) {
-              if (flags & 2) {
-                c.page_table[li * c.maxp + np_new - 1] = id;
-                c.npages[li] = np_new;
-                atomicAdd(&c.ctrl[CTRL_STEP_PAGES], 1);
-              }
-              const int hs = (fuse_decide || c.alpha_per != DMS_ALPHA_PER_LAYER) ? h : 0;
-              const float av = s_alpha[k] == s_alpha[k] ? s_alpha[k] : __ldcg(&alpha[b * c.Hkv + hs]);
-              const bool evict = !c.disable && av > 0.0f;
-              c.slot_pos[li * c.cap + slot] = t;
-              c.ring[li * c.w + t % c.w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
-              if (!(flags & 1)) c.count[li] = cnt_new;
-            } else {
-              set_status(c.ctrl, (flags & 4) ? DMS_ST_CAPACITY : DMS_ST_POOL_EXHAUSTED);
-            }
-            // plan of the next append (token t + 1), with its count snapshot
-            const int tn = t + 1;
-            const int rn = sg.ring_idx >= 0 ? s_ring[sg.ring_idx] : 0;
-            *plan_at(c, li, tn) = make_plan(rn, tn, cnt_new, np_new, c);
-          }
-        }
-      }
-      consumers_sync();  // merge buffers are reused by the next segment
-      if (k == 0) DMS_TRACE_MARK(0, finish ? 7 : 6);
-      if (finish) DMS_TRACE_MARK(0, 13);
+      if (tid == 0) mbar_arrive(&hq_full[j]);
     }
     DMS_TRACE_MARK(0, 8);
+    // the heads whose last part arrived here, once every hand-over is done
+    if (!mbar_wait_bounded(&aux_done, 0)) timed_out = true;
+    for (int f = 0; f < s_nfin; ++f) finish_head(s_fin[f], nullptr, tid, 128);
     if (timed_out && lane == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
   }
 
@@ -903,8 +1023,8 @@ static bool flat_geometry(const CacheView& c, int* grid, int* nst, size_t* smem)
   const int n = static_cast<int>(std::min<size_t>(kFlatMaxStages, (budget - fixed) / stride)) / kFlatConsumers *
                 kFlatConsumers;
   if (n < kFlatConsumers) return false;
-  // the partition scratch (6 ints per head) lives in the stage ring
-  if (static_cast<size_t>(6 * BH + 8) * sizeof(int) > n * stride) return false;
+  // the partition scratch (7 ints per head) lives in the stage ring
+  if (static_cast<size_t>(7 * BH + 8) * sizeof(int) > n * stride) return false;
   *grid = G;
   *nst = n;
   *smem = fixed + n * stride;
