@@ -6,7 +6,10 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
+#include <unordered_map>
+#include <utility>
 #include <vector>
 
 #include "dms_internal.cuh"
@@ -141,6 +144,29 @@ bool make_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_
   return r == CUDA_SUCCESS;
 }
 
+}  // namespace
+
+// The last (cache, layer) this library enqueued work for on each stream
+// (layer -1: every layer, e.g. a reset).  A decode kernel may read its
+// layer's state before the previous kernel of the stream completes only when
+// that kernel was for another (cache, layer).
+namespace {
+std::mutex g_track_mu;
+std::unordered_map<cudaStream_t, std::pair<const void*, int>> g_last_launch;
+
+bool track_launch(const void* cache, int layer, cudaStream_t s) {
+  std::lock_guard<std::mutex> lk(g_track_mu);
+  auto it = g_last_launch.find(s);
+  const bool other = it == g_last_launch.end() ||
+                     !(it->second.first == cache && (it->second.second == layer || it->second.second < 0 || layer < 0));
+  g_last_launch[s] = std::make_pair(cache, layer);
+  return other;
+}
+void forget_cache(const void* cache) {
+  std::lock_guard<std::mutex> lk(g_track_mu);
+  for (auto it = g_last_launch.begin(); it != g_last_launch.end();)
+    it = it->second.first == cache ? g_last_launch.erase(it) : std::next(it);
+}
 }  // namespace
 
 struct dms_cache {
@@ -289,17 +315,20 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
     delete c;
     return DMS_ERR_CUDA;
   }
+  track_launch(c, -1, static_cast<cudaStream_t>(stream));
   *out = c;
   return DMS_OK;
 }
 
 int dms_cache_free(dms_cache* c) {
+  forget_cache(c);
   delete c;
   return DMS_OK;
 }
 
 int dms_cache_reset(dms_cache* c, void* stream) {
   if (!c) return DMS_ERR_INVALID;
+  track_launch(c, -1, static_cast<cudaStream_t>(stream));
   if (launch_init(c->view, false, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DMS_ERR_CUDA;
   std::fill(c->positions.begin(), c->positions.end(), 0);
   std::fill(c->prefilled.begin(), c->prefilled.end(), 0);
@@ -399,6 +428,7 @@ int dms_prefill_compact(dms_cache* c, int layer, const dms_prefill_args* a, void
   if (c->prefilled[layer]) return DMS_ERR_STATE;
   const int T = a->seq_len;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  track_launch(c, layer, s);
   const CacheView& v = c->view;
   const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
   if (a->decide && !neuron) {
@@ -423,6 +453,7 @@ int dms_prefill_attention(dms_cache* c, int layer, const dms_prefill_args* a, vo
   int e = check_prefill(c, layer, a);
   if (e) return e;
   if (c->compacted_layer != layer || c->compacted_len != a->seq_len) return DMS_ERR_STATE;
+  track_launch(c, layer, static_cast<cudaStream_t>(stream));
   // tensor maps of this call's q, k, v for the tcgen05 kernel
   PrefillMaps maps{};
   maps.valid = false;
@@ -463,6 +494,7 @@ int dms_decode_append(dms_cache* c, int layer, const dms_decode_args* a, void* s
   }
   if (!c->prefilled[layer] || c->positions[layer] >= c->desc.max_positions) return DMS_ERR_STATE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  track_launch(c, layer, s);
   const CacheView& v = c->view;
   const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
   // The adapter's decision logits are computed inside the append kernel when
@@ -498,12 +530,14 @@ namespace {
 int run_decode_kernel(dms_cache* c, int layer, const void* q, void* o, bool fused, const void* k, const void* v,
                       float* alpha, const DecideArgs* da, cudaStream_t s) {
   const CacheView& cv = c->view;
+  const bool early = track_launch(c, layer, s);
   int mode = c->desc.decode_kernel;
   if (mode == DMS_DECODE_AUTO)
     mode = static_cast<long>(cv.B) * cv.Hkv * 8 <= 2L * c->num_sms ? DMS_DECODE_CLUSTER : DMS_DECODE_FLAT;
   if (mode == DMS_DECODE_FLAT) {
     bool taken = false;
-    if (launch_decode_flat(cv, layer, q, o, fused, k, v, alpha, da, &c->kmap64, &c->vmap64, s, &taken) != cudaSuccess)
+    if (launch_decode_flat(cv, layer, q, o, fused, k, v, alpha, da, &c->kmap64, &c->vmap64, s, early, &taken) !=
+        cudaSuccess)
       return DMS_ERR_CUDA;
     if (taken) return DMS_OK;
   }
@@ -523,6 +557,7 @@ int dms_decode_attention(dms_cache* c, int layer, const void* q, void* o, void* 
   if (c->has_maps && c->desc.kv_dtype != DMS_F32)
     return run_decode_kernel(c, layer, q, o, false, nullptr, nullptr, nullptr, nullptr,
                              static_cast<cudaStream_t>(stream));
+  track_launch(c, layer, static_cast<cudaStream_t>(stream));
   if (launch_decode_attention(c->view, layer, q, o, c->has_maps ? &c->kmap : nullptr, c->has_maps ? &c->vmap : nullptr,
                               c->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DMS_ERR_CUDA;
@@ -556,6 +591,7 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   const CacheView& v = c->view;
   const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
   if (neuron || a->rope_cos) {
+    track_launch(c, layer, s);
     if (launch_neuron_rope(v, 1, v.pos + static_cast<long>(layer) * v.B, a->q, a->k,
                            neuron ? a->decide->offset : nullptr, neuron ? a->decide->offset_batch_stride : 0, neuron,
                            a->alpha, a->rope_cos, a->rope_sin, s) != cudaSuccess)

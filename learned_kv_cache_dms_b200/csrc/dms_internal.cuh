@@ -367,10 +367,13 @@ cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q
                                     const CUtensorMap* kmap, const CUtensorMap* vmap, int num_sms,
                                     cudaStream_t s);
 // Persistent split-K decode over all SMs; *taken is false (nothing launched)
-// when the shape is outside what the kernel stages in shared memory.
+// when the shape is outside what the kernel stages in shared memory.  `early`:
+// the previous launch of this library on the stream was for another (cache,
+// layer), so the kernel may read this layer's state before the previous
+// kernels complete (programmatic dependent launch).
 cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
-                               const CUtensorMap* vmap, cudaStream_t s, bool* taken);
+                               const CUtensorMap* vmap, cudaStream_t s, bool early, bool* taken);
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s);

@@ -118,6 +118,17 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+// Programmatic dependent launch: let the next kernel of the stream start its
+// prologue, and wait until every kernel this one depends on has completed.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 // Barrier of the four consumer warps only (the producer warp never joins).
 __device__ __forceinline__ void consumers_sync() { asm volatile("barrier.sync 1, 128;\n" ::: "memory"); }
 
@@ -314,7 +325,7 @@ struct FlatSmem {
 
 template <int D, bool FP8, bool FUSED>
 __global__ void __launch_bounds__(kFlatThreads, 1)
-    k_decode_flat(CacheView c, int layer, const __nv_bfloat16* q, __nv_bfloat16* o, int nst,
+    k_decode_flat(CacheView c, int layer, int early, const __nv_bfloat16* q, __nv_bfloat16* o, int nst,
                   const __nv_bfloat16* k_new, const __nv_bfloat16* v_new, float* alpha, DecideArgs da, int fuse_decide,
                   const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
   using F = FlatSmem<D, FP8>;
@@ -352,6 +363,17 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
   const long lbase = static_cast<long>(layer) * BH;
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
   DMS_TRACE_MARK(0, 0);
+  // Programmatic dependent launch.  With `early` (the previous launch of this
+  // library on the stream was for another layer or cache) the partition below
+  // reads only this layer's state before waiting for the previous kernel:
+  // only that kernel may still run (each kernel lets its dependents start
+  // only once its own wait has returned), and it does not write this state.
+  // The page counter, the arrival counters, the partial scratch and the
+  // inputs are touched only after the wait.
+  if (!early) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
 
   // ---- setup: every CTA derives the same partition ------------------------
   // (scratch arrays live in the stage ring, unused until the producer starts)
@@ -379,7 +401,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     mbar_init(&aux_done, 1);
     s_nfin = 0;
     fence_mbar_init();
-    s_next_page0 = FUSED ? c.ctrl[CTRL_NEXT_PAGE] : 0;
   }
   {
     int part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -599,6 +620,11 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
       s_sub[n] = d;
     }
   }
+  if (early) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
+  if (FUSED && tid == 0) s_next_page0 = c.ctrl[CTRL_NEXT_PAGE];
   __syncthreads();
   DMS_TRACE_MARK(0, 1);
 
@@ -803,15 +829,15 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
           else
             c.part_ml[(static_cast<long>(sg.pslot) * g + r) * 2 + (d - D)] = cp[r * MLD + d];
         }
-        __threadfence();
-        __syncwarp();
+        __syncwarp();  // the lanes' partial stores precede lane 0's release
         int last = 0;
         if (lane == 0) {
-          last = atomicAdd(&c.head_done[bh], 1) == sg.nparts - 1;
+          // release: this partial is visible to whoever sees the count;
+          // acquire: the last arrival sees every other part's partial
+          last = atom_add_acq_rel(&c.head_done[bh], 1) == sg.nparts - 1;
           if (last) c.head_done[bh] = 0;
         }
         finish = __shfl_sync(0xffffffffu, last, 0) != 0;
-        if (finish) __threadfence();
         if (k == 0 && lane == 0) FLAT_MARK_ANY(finish ? 4 : 6);
       }
       if (finish && sg.nparts == 1) {
@@ -1034,7 +1060,7 @@ static bool flat_geometry(const CacheView& c, int* grid, int* nst, size_t* smem)
 template <int D, bool FP8, bool FUSED>
 static cudaError_t launch_flat_t(const CacheView& c, int layer, const void* q, void* o, const void* k, const void* v,
                                  float* alpha, const DecideArgs* da, const CUtensorMap* kmap, const CUtensorMap* vmap,
-                                 cudaStream_t s, bool* taken) {
+                                 cudaStream_t s, bool early, bool* taken) {
   int grid = 0, nst = 0;
   size_t smem = 0;
   *taken = (reinterpret_cast<uintptr_t>(q) & 15) == 0 && flat_geometry<D, FP8, FUSED>(c, &grid, &nst, &smem);
@@ -1043,28 +1069,36 @@ static cudaError_t launch_flat_t(const CacheView& c, int layer, const void* q, v
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   DecideArgs none{};
-  kern<<<grid, kFlatThreads, smem, s>>>(c, layer, static_cast<const __nv_bfloat16*>(q),
-                                        static_cast<__nv_bfloat16*>(o), nst, static_cast<const __nv_bfloat16*>(k),
-                                        static_cast<const __nv_bfloat16*>(v), alpha, da ? *da : none, da ? 1 : 0,
-                                        *kmap, *vmap);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kFlatThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, c, layer, early ? 1 : 0, static_cast<const __nv_bfloat16*>(q),
+                            static_cast<__nv_bfloat16*>(o), nst, static_cast<const __nv_bfloat16*>(k),
+                            static_cast<const __nv_bfloat16*>(v), alpha, da ? *da : none, da ? 1 : 0, *kmap, *vmap);
 }
 
 cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
-                               const CUtensorMap* vmap, cudaStream_t s, bool* taken) {
+                               const CUtensorMap* vmap, cudaStream_t s, bool early, bool* taken) {
   *taken = false;
   if (!kmap || !vmap || c.kv_dtype == DMS_F32) return cudaErrorInvalidValue;
   if (fused) {
     if (c.kv_dtype != DMS_BF16) return cudaErrorInvalidValue;
-    return c.D == 64 ? launch_flat_t<64, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, s, taken)
-                     : launch_flat_t<128, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, s, taken);
+    return c.D == 64 ? launch_flat_t<64, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, s, early, taken)
+                     : launch_flat_t<128, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, s, early, taken);
   }
   if (c.kv_dtype == DMS_FP8_E4M3)
-    return c.D == 64 ? launch_flat_t<64, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, taken)
-                     : launch_flat_t<128, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, taken);
-  return c.D == 64 ? launch_flat_t<64, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, taken)
-                   : launch_flat_t<128, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, taken);
+    return c.D == 64 ? launch_flat_t<64, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken)
+                     : launch_flat_t<128, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken);
+  return c.D == 64 ? launch_flat_t<64, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken)
+                   : launch_flat_t<128, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken);
 }
 
 }  // namespace dms
