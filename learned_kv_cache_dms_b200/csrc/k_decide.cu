@@ -233,10 +233,12 @@ cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, f
 }
 
 // ---------------------------------------------------------------------------
-// Neuron decisions and rotary embedding, one warp per token, in place:
+// Neuron decisions and rotary embedding, one thread per (token, row, i <
+// D/2) element pair, in place:
 //  1. (neuron source) alpha = x[D-1] * scale - offset for the key of head h or
-//     the query of head h*g; layer granularity takes head 0's value; then the
-//     decision element of every head is set to zero;
+//     the query of head h*g, read by the thread of pair i = D/2 - 1 of that
+//     row; layer granularity takes head 0's value; then the decision element
+//     of every head is set to zero;
 //  2. (tables given) half-split rotation of every query and key row of the
 //     token at position t (prefill), or at the sequence's current position
 //     pos_dev[b] (decode, T == 1).
@@ -244,43 +246,47 @@ cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, f
 template <typename TA>
 __global__ void k_neuron_rope(CacheView c, int T, const int* pos_dev, TA* q, TA* k, const float* offset, int ostride,
                               int do_alpha, float* alpha, const float* cos_t, const float* sin_t) {
-  const int lane = threadIdx.x & 31;
-  const long gw = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
-  const long ntok = static_cast<long>(c.B) * T;
   const int D = c.D, half = D / 2, g = c.Hq / c.Hkv;
   const bool key = c.alpha_source == DMS_ALPHA_KEY_NEURON;
-  for (long tok = gw; tok < ntok; tok += nwarps) {
+  // with rotary tables every (token, row, i < D/2) pair, else only the
+  // decision neuron of each head (its pair i = D/2 - 1)
+  const int nrow = cos_t ? c.Hq + c.Hkv : c.Hkv;
+  const int npair = cos_t ? half : 1;
+  const long total = static_cast<long>(c.B) * T * nrow * npair;
+  for (long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<long>(gridDim.x) * blockDim.x) {
+    const int i = cos_t ? static_cast<int>(idx % half) : half - 1;
+    const long rt = idx / npair;
+    int r = static_cast<int>(rt % nrow);
+    const long tok = rt / nrow;
+    if (!cos_t) r = key ? c.Hq + r : r * g;  // the neuron rows only
     const int b = static_cast<int>(tok / T), t = static_cast<int>(tok % T);
-    if (do_alpha) {
-      TA* src = key ? k + tok * c.Hkv * D : q + tok * c.Hq * D;
-      const int stride_h = key ? D : g * D;
-      // Hkv <= 32: lane h handles head h
-      const int h = lane;
-      float a = 0.f;
-      if (h < c.Hkv) a = fmaf(to_f(src[h * stride_h + D - 1]), c.alpha_scale, -offset[b * ostride + h]);
-      const float a_head0 = __shfl_sync(0xffffffffu, a, 0);
-      if (c.alpha_per == DMS_ALPHA_PER_LAYER) a = a_head0;
-      if (h < c.Hkv) alpha[(static_cast<long>(b) * c.Hkv + h) * T + t] = a;
-      __syncwarp();
-      for (int h = lane; h < c.Hkv; h += 32) src[h * stride_h + D - 1] = from_f<TA>(0.f);
-      __syncwarp();
+    TA* row = r < c.Hq ? q + (tok * c.Hq + r) * D : k + (tok * c.Hkv + (r - c.Hq)) * D;
+    float x0 = to_f(row[i]), x1 = to_f(row[i + half]);
+    // the decision neuron (the last element of each key, or of the first query
+    // head of each group) is read, then zeroed, before the rotation
+    const bool neuron_row = key ? r >= c.Hq : (r < c.Hq && r % g == 0);
+    if (do_alpha && neuron_row && i == half - 1) {
+      const int h = key ? r - c.Hq : r / g;
+      if (c.alpha_per == DMS_ALPHA_PER_LAYER) {
+        if (h == 0) {
+          const float a = fmaf(x1, c.alpha_scale, -offset[b * ostride]);
+          for (int hh = 0; hh < c.Hkv; ++hh) alpha[(static_cast<long>(b) * c.Hkv + hh) * T + t] = a;
+        }
+      } else {
+        alpha[(static_cast<long>(b) * c.Hkv + h) * T + t] = fmaf(x1, c.alpha_scale, -offset[b * ostride + h]);
+      }
+      x1 = 0.f;
     }
     if (cos_t) {
       const int p = pos_dev ? pos_dev[b] + t : t;
-      const float* cs = cos_t + static_cast<long>(p) * half;
-      const float* sn = sin_t + static_cast<long>(p) * half;
-      const int nrow = c.Hq + c.Hkv;
-      for (int idx = lane; idx < nrow * half; idx += 32) {
-        const int r = idx / half, i = idx % half;
-        TA* row = r < c.Hq ? q + (tok * c.Hq + r) * D : k + (tok * c.Hkv + (r - c.Hq)) * D;
-        const float x0 = to_f(row[i]), x1 = to_f(row[i + half]);
-        const float cv = cs[i], sv = sn[i];
-        // each product and sum rounded separately (no fused multiply-add), so
-        // the stored value does not depend on contraction choices
-        row[i] = from_f<TA>(__fsub_rn(__fmul_rn(x0, cv), __fmul_rn(x1, sv)));
-        row[i + half] = from_f<TA>(__fadd_rn(__fmul_rn(x1, cv), __fmul_rn(x0, sv)));
-      }
+      const float cv = cos_t[static_cast<long>(p) * half + i], sv = sin_t[static_cast<long>(p) * half + i];
+      // each product and sum rounded separately (no fused multiply-add), so
+      // the stored value does not depend on contraction choices
+      row[i] = from_f<TA>(__fsub_rn(__fmul_rn(x0, cv), __fmul_rn(x1, sv)));
+      row[i + half] = from_f<TA>(__fadd_rn(__fmul_rn(x1, cv), __fmul_rn(x0, sv)));
+    } else {
+      row[i + half] = from_f<TA>(x1);
     }
   }
 }
@@ -288,8 +294,8 @@ __global__ void k_neuron_rope(CacheView c, int T, const int* pos_dev, TA* q, TA*
 cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
                                int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
                                const float* sin_t, cudaStream_t s) {
-  const long ntok = static_cast<long>(c.B) * T;
-  const int grid = static_cast<int>(min((ntok + 7) / 8, static_cast<long>(c.num_sms) * 8));
+  const long total = static_cast<long>(c.B) * T * (cos_t ? (c.Hq + c.Hkv) * (c.D / 2) : c.Hkv);
+  const int grid = static_cast<int>(max(1L, min((total + 255) / 256, static_cast<long>(c.num_sms) * 16)));
   if (c.act_dtype == DMS_BF16)
     k_neuron_rope<__nv_bfloat16><<<grid, 256, 0, s>>>(c, T, pos_dev, static_cast<__nv_bfloat16*>(q),
                                                        static_cast<__nv_bfloat16*>(k), offset, offset_bstride,

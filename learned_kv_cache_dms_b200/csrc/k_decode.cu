@@ -181,10 +181,26 @@ __global__ void __launch_bounds__(1024) k_decode_append(CacheView c, int layer, 
         const float s_old = *scale_p;
         float scale = s_old;
         if (s_new > s_old) {
-          // re-encode the page's rows at the larger scale from their decoded values
-          for (int idx = lane; idx < rows * D; idx += 32) {
-            const float dq = __fmul_rn(fp8_decode(page[idx]), s_old);
-            page[idx] = fp8_encode(__fdiv_rn(dq, s_new));
+          // re-encode the page's rows at the larger scale from their decoded
+          // values, 16 codes per lane and four vectors in flight
+          uint4* pv = reinterpret_cast<uint4*>(page);
+          const int nvec = rows * D / 16;
+          for (int v0 = 0; v0 < nvec; v0 += 4 * 32) {
+            uint4 u[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int vi = v0 + e * 32 + lane;
+              if (vi < nvec) u[e] = pv[vi];
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int vi = v0 + e * 32 + lane;
+              if (vi >= nvec) continue;
+              uint8_t* cb = reinterpret_cast<uint8_t*>(&u[e]);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) cb[j] = fp8_encode(__fdiv_rn(__fmul_rn(fp8_decode(cb[j]), s_old), s_new));
+              pv[vi] = u[e];
+            }
           }
           scale = s_new;
           __syncwarp();
@@ -223,7 +239,9 @@ cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, c
                                  const DecideArgs* fused_decide, int num_sms, cudaStream_t s) {
   const int BH = c.B * c.Hkv;
   (void)num_sms;
-  const int threads = min(1024, max(256, (BH + 31) / 32 * 32));
+  // one warp per head for the K/V rows (an FP8 page re-encode is a few
+  // round trips of its own), up to 32 warps
+  const int threads = min(1024, max(256, 32 * BH));
   const size_t smem = static_cast<size_t>(BH) * 3 * sizeof(int);
   if (c.kv_dtype == DMS_FP8_E4M3)
     return launch_append_t<__nv_bfloat16, true>(c, layer, k, v, alpha, fused_decide, threads, smem, s);
