@@ -97,7 +97,9 @@ def build(case: Case):
         W = I.normal(s, (case.layer, 11), (case.Hkv, case.hidden), case.act, std=case.hidden ** -0.5)
         raw = O.decide_proj(_f64(h), _f64(gamma), _f64(W), None, np.zeros((B, case.Hkv)), ALPHA_SCALE, RMS_EPS,
                             layer_mode)
-        off, _ = I.calibrate_offsets(raw[:, :, :T], keep)
+        # offsets from every token's raw logit (prompt and decode), so that no
+        # decision sits within the comparison margin
+        off, _ = I.calibrate_offsets(raw, keep)
         if layer_mode:
             off[:] = off[:, :1]
         alpha_o = O.decide_proj(_f64(h), _f64(gamma), _f64(W), None, off, ALPHA_SCALE, RMS_EPS, layer_mode)
@@ -107,7 +109,7 @@ def build(case: Case):
         src = k if case.source == "key" else q
         group = 1 if case.source == "key" else case.Hq // case.Hkv
         raw, _ = O.decide_neuron(_f64(src), group, case.Hkv, np.zeros((B, case.Hkv)), ALPHA_SCALE, layer_mode)
-        off, _ = I.calibrate_offsets(raw[:, :, :T], keep)
+        off, _ = I.calibrate_offsets(raw, keep)
         if layer_mode:
             off[:] = off[:, :1]
         alpha_o, zeroed = O.decide_neuron(_f64(src), group, case.Hkv, off, ALPHA_SCALE, layer_mode)
