@@ -48,16 +48,25 @@ namespace dms {
 
 #ifdef DMS_TRACE
 __device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
-// mark by any one thread (the producer's lane 0)
-#define FLAT_MARK_ANY(slot)                                                            \
-  do {                                                                                 \
-    unsigned long long t_;                                                             \
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                             \
-    if (blockIdx.x < kTraceCtas) g_dms_trace[blockIdx.x * kTraceSlots + (slot)] = t_; \
+// phase marks of the kernel of layer l (27 layers kept, 148 CTAs each), by
+// thread 0 or by any one thread (the producer's or the aux warp's lane 0)
+#define FLAT_TRACE_ROW (((layer) % 27) * 148 + blockIdx.x)
+#define FLAT_MARK_ANY(slot)                                                                            \
+  do {                                                                                                 \
+    unsigned long long t_;                                                                             \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                             \
+    if (blockIdx.x < 148) g_dms_trace[static_cast<long>(FLAT_TRACE_ROW) * kTraceSlots + (slot)] = t_; \
+  } while (0)
+#define FLAT_MARK(slot)                   \
+  do {                                    \
+    if (threadIdx.x == 0) FLAT_MARK_ANY(slot); \
   } while (0)
 #else
 #define FLAT_MARK_ANY(slot) \
   do {                      \
+  } while (0)
+#define FLAT_MARK(slot) \
+  do {                  \
   } while (0)
 #endif
 
@@ -118,6 +127,24 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// 2-D TMA tile load (no multicast) with an L2 cache policy: the KV pages are
+// read once per step, so they are marked first to evict, which keeps the
+// small per-layer state (plans, page tables, ring) resident in L2 between
+// the steps of a deep layer stack.
+__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, int c0, int c1,
+                                                 uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+      "%3}], [%4], %5;\n" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
   int old;
   asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
@@ -354,15 +381,17 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
   __shared__ __align__(8) uint64_t hq_full[2], hq_empty[2];  // merged-segment hand-over ring
   __shared__ __align__(8) uint64_t aux_done;                 // every hand-over processed
   __shared__ int s_fin[kFlatSegMax], s_nfin;                 // heads the consumers finish
-  __shared__ int s_red[32], s_part[kFlatThreads / 32][8];
-  __shared__ int s_nseg, s_nsub, s_npt, s_nring, s_last, s_next_page0, s_unit;
+  __shared__ int s_part[kFlatThreads / 32][8];  // per-warp candidate unit sums
+  __shared__ int s_ctot[kFlatThreads / 32][2];  // per-warp chunk totals (units, new pages)
+  __shared__ int s_stot[2][3];                  // per-warp segment totals (sub-tiles, page ids, ring entries)
+  __shared__ int s_nseg, s_nsub, s_npt, s_nring, s_last, s_next_page0;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const int BH = c.B * c.Hkv;
   const long lbase = static_cast<long>(layer) * BH;
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-  DMS_TRACE_MARK(0, 0);
+  FLAT_MARK(0);
   // Programmatic dependent launch.  With `early` (the previous launch of this
   // library on the stream was for another layer or cache) the partition below
   // reads only this layer's state before waiting for the previous kernel:
@@ -402,31 +431,53 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     s_nfin = 0;
     fence_mbar_init();
   }
+  // Heads are split into one contiguous chunk per warp.  Each warp loads its
+  // chunk's plans (both parities and the position in one round trip); warp
+  // shuffles then do the reductions and scans, with one exchange of chunk
+  // totals between the warps.
+  constexpr int NW = kFlatThreads / 32;
+  const int hchunk = (BH + NW - 1) / NW;
+  const int hb = min(BH, warp * hchunk), he = min(BH, hb + hchunk);
   {
     int part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int i = tid; i < BH; i += kFlatThreads) {
-      int cnt;
-      if (FUSED) {
-        // both parities and the position in one round trip; the plan of
-        // position t holds the count before this step's append
-        const int4 p0 = c.plan[lbase + i];
-        const int4 p1 = c.plan[static_cast<long>(c.L) * BH + lbase + i];
-        const int t = c.pos[layer * c.B + i / c.Hkv];
-        const int4 pl = (t & 1) ? p1 : p0;
-        cnt = pl.z;
-        s_plx[i] = pl.x;
-        s_ply[i] = pl.y;
-        s_npg[i] = pl.w;
-        s_tpos[i] = t;
-      } else {
-        cnt = c.count[lbase + i];  // nothing in this launch changes it
-      }
-      s_cnt[i] = cnt;
+    constexpr int LB = 4;  // heads per lane whose loads are in flight together
+    for (int i0 = hb; i0 < he; i0 += 32 * LB) {
+      int4 pa[LB], pb[LB];
+      int tt[LB], cc[LB];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) part[k] += max(1, (cnt + (kFlatUnit << k) - 1) / (kFlatUnit << k));
+      for (int u = 0; u < LB; ++u) {
+        const int i = i0 + u * 32 + lane;
+        if (i < he) {
+          if (FUSED) {
+            pa[u] = c.plan[lbase + i];
+            pb[u] = c.plan[static_cast<long>(c.L) * BH + lbase + i];
+            tt[u] = c.pos[layer * c.B + i / c.Hkv];
+          } else {
+            cc[u] = c.count[lbase + i];  // nothing in this launch changes it
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < LB; ++u) {
+        const int i = i0 + u * 32 + lane;
+        if (i >= he) continue;
+        int cnt;
+        if (FUSED) {
+          // the plan of position t holds the count before this step's append
+          const int4 pl = (tt[u] & 1) ? pb[u] : pa[u];
+          cnt = pl.z;
+          s_plx[i] = pl.x;
+          s_ply[i] = pl.y;
+          s_npg[i] = pl.w;
+          s_tpos[i] = tt[u];
+        } else {
+          cnt = cc[u];
+        }
+        s_cnt[i] = cnt;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) part[k] += max(1, (cnt + (kFlatUnit << k) - 1) / (kFlatUnit << k));
+      }
     }
-    // unit size: the smallest 16 * 2^k slots leaving at most kFlatSegMax - 2
-    // units per CTA, so a CTA's range meets at most that many heads
 #pragma unroll
     for (int k = 0; k < 8; ++k)
 #pragma unroll
@@ -434,46 +485,74 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     if (lane == 0)
 #pragma unroll
       for (int k = 0; k < 8; ++k) s_part[warp][k] = part[k];
-    __syncthreads();
-    if (tid == 0) {
-      int k = 0;
-      for (;; ++k) {
-        long tot = 0;
-        for (int wv = 0; wv < kFlatThreads / 32; ++wv) tot += s_part[wv][k];
-        if (k == 7 || (tot + G - 1) / G <= kFlatSegMax - 2) break;
-      }
-      s_unit = kFlatUnit << k;
-    }
-    __syncthreads();
-  }
-  DMS_TRACE_MARK(0, 16);
-  const int unit = s_unit;
-  // sub-tile chunk: the largest of 64, 32, 16 slots dividing the page size,
-  // so chunks never cross a page
-  const int chunk = c.P % kFlatRows == 0 ? kFlatRows : c.P % 32 == 0 ? 32 : 16;
-  {
-    int base = 0, gbase = 0;
-    for (int i0 = 0; i0 < BH; i0 += kFlatThreads) {
-      const int i = i0 + tid;
-      const int n = i < BH ? max(1, (s_cnt[i] + unit - 1) / unit) : 0;
-      int tot;
-      const int off = block_exclusive_scan(n, s_red, &tot);
-      if (i < BH) s_off[i] = base + off;
-      base += tot;
-      if (FUSED) {
-        const int np = (i < BH && (s_ply[i] & 2)) ? 1 : 0;
-        const int goff = block_exclusive_scan(np, s_red, &tot);
-        if (i < BH) s_gr[i] = gbase + goff;
-        gbase += tot;
-      }
-    }
-    if (tid == 0) s_off[BH] = base;
   }
   __syncthreads();
-  DMS_TRACE_MARK(0, 17);
+  // unit size (every thread alike): the smallest 16 * 2^k slots leaving at
+  // most kFlatSegMax - 2 units per CTA, so a CTA's range meets at most that
+  // many heads
+  int unit = kFlatUnit;
+  for (int k = 0;; ++k) {
+    long tot = 0;
+#pragma unroll
+    for (int wv = 0; wv < NW; ++wv) tot += s_part[wv][k];
+    unit = kFlatUnit << k;
+    if (k == 7 || (tot + G - 1) / G <= kFlatSegMax - 2) break;
+  }
+  // unit offsets and new-page ranks: scans within each warp's chunk
+  {
+    int carry = 0, gcarry = 0;
+    for (int i0 = hb; i0 < he; i0 += 32) {
+      const int i = i0 + lane;
+      const int n = i < he ? max(1, (s_cnt[i] + unit - 1) / unit) : 0;
+      const int np = (FUSED && i < he && (s_ply[i] & 2)) ? 1 : 0;
+      int x = n, y = np;
+#pragma unroll
+      for (int o2 = 1; o2 < 32; o2 <<= 1) {
+        const int xa = __shfl_up_sync(0xffffffffu, x, o2), ya = __shfl_up_sync(0xffffffffu, y, o2);
+        if (lane >= o2) {
+          x += xa;
+          y += ya;
+        }
+      }
+      if (i < he) {
+        s_off[i] = carry + x - n;
+        if (FUSED) s_gr[i] = gcarry + y - np;
+      }
+      carry += __shfl_sync(0xffffffffu, x, 31);
+      gcarry += __shfl_sync(0xffffffffu, y, 31);
+    }
+    if (lane == 0) {
+      s_ctot[warp][0] = carry;
+      s_ctot[warp][1] = gcarry;
+    }
+  }
+  FLAT_MARK(16);
+  __syncthreads();
+  {
+    int base = 0, gbase = 0, total = 0;
+#pragma unroll
+    for (int wv = 0; wv < NW; ++wv) {
+      if (wv < warp) {
+        base += s_ctot[wv][0];
+        gbase += s_ctot[wv][1];
+      }
+      total += s_ctot[wv][0];
+    }
+    for (int i = hb + lane; i < he; i += 32) {
+      s_off[i] += base;
+      if (FUSED) s_gr[i] += gbase;
+    }
+    if (tid == 0) s_off[BH] = total;
+  }
+  __syncthreads();
+  FLAT_MARK(17);
   const long U = s_off[BH];
   const long u0 = static_cast<long>(cta) * U / G, u1 = static_cast<long>(cta + 1) * U / G;
-  auto cta_of = [&](long u) { return static_cast<int>(((u + 1) * G - 1) / U); };
+  auto cta_of = [&](long u) {
+    const unsigned long long a = static_cast<unsigned long long>(u + 1) * G - 1;
+    return static_cast<int>((a >> 32) == 0 && (U >> 32) == 0 ? static_cast<unsigned>(a) / static_cast<unsigned>(U)
+                                                              : a / static_cast<unsigned long long>(U));
+  };
   // heads [h_lo, h_hi] meet this CTA's units (binary searches in every thread)
   int h_lo = 0, h_hi = -1;
   if (u0 < u1) {
@@ -495,83 +574,111 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     if (tid == 0) set_status(c.ctrl, DMS_ST_SPLIT_LIMIT);
     nseg = kFlatSegMax;
   }
-  // one thread per segment: its slots and parts, and how many sub-tiles, page
-  // ids and ring entries it needs (offsets by block scans)
+  const int chunk = c.P % kFlatRows == 0 ? kFlatRows : c.P % 32 == 0 ? 32 : 16;
+  // segments: warps 0 and 1, one lane per segment (kFlatSegMax = 64); their
+  // sub-tile, page-id and ring-entry counts are scanned with shuffles
   FlatSeg sg{};
   int my_sub = 0, my_pt = 0, my_ring = 0, p0 = 0, p1 = -1;
+  int xs = 0, xp = 0, xr = 0;  // inclusive scans within the warp
   long li = 0;
-  if (tid < nseg) {
-    const int h = h_lo + tid;
-    const int cnt = s_cnt[h];
-    li = lbase + h;
-    sg.bh = h;
-    sg.cnt = cnt;
-    sg.s0 = static_cast<int>(max(0L, u0 - s_off[h]) * unit);
-    sg.s1 = static_cast<int>(min(static_cast<long>(cnt), (u1 - s_off[h]) * unit));
-    if (sg.s0 > sg.s1) sg.s0 = sg.s1;  // an empty head's only unit
-    sg.unit0 = s_off[h];
-    if (s_off[h] >= u0 && s_off[h + 1] <= u1) {
-      sg.nparts = 1;  // the whole head is here
-      sg.first_cta = cta;
-      sg.first_pslot = sg.pslot = 2 * cta;
-    } else {
-      const int fc = cta_of(s_off[h]), lc = cta_of(s_off[h + 1] - 1);
-      sg.first_cta = fc;
-      // with fewer units than CTAs most CTAs are empty: the head's parts are
-      // then the CTAs of its units, one unit each
-      sg.nparts = min(lc - fc + 1, s_off[h + 1] - s_off[h]);
-      const long fu0 = static_cast<long>(fc) * U / G;
-      sg.first_pslot = 2 * fc + (s_off[h] != fu0 ? 1 : 0);
-      sg.pslot = cta == fc ? sg.first_pslot : 2 * cta;
+  const int ks = warp * 32 + lane;
+  if (warp < 2) {
+    if (ks < nseg) {
+      const int h = h_lo + ks;
+      const int cnt = s_cnt[h];
+      li = lbase + h;
+      sg.bh = h;
+      sg.cnt = cnt;
+      sg.s0 = static_cast<int>(max(0L, u0 - s_off[h]) * unit);
+      sg.s1 = static_cast<int>(min(static_cast<long>(cnt), (u1 - s_off[h]) * unit));
+      if (sg.s0 > sg.s1) sg.s0 = sg.s1;  // an empty head's only unit
+      sg.unit0 = s_off[h];
+      if (s_off[h] >= u0 && s_off[h + 1] <= u1) {
+        sg.nparts = 1;  // the whole head is here
+        sg.first_cta = cta;
+        sg.first_pslot = sg.pslot = 2 * cta;
+      } else {
+        const int fc = cta_of(s_off[h]), lc = cta_of(s_off[h + 1] - 1);
+        sg.first_cta = fc;
+        // with fewer units than CTAs most CTAs are empty: the head's parts are
+        // then the CTAs of its units, one unit each
+        sg.nparts = min(lc - fc + 1, s_off[h + 1] - s_off[h]);
+        const long fu0 = static_cast<long>(fc) * U / G;
+        sg.first_pslot = 2 * fc + (s_off[h] != fu0 ? 1 : 0);
+        sg.pslot = cta == fc ? sg.first_pslot : 2 * cta;
+      }
+      sg.decide = (FUSED && fuse_decide && s_off[h] >= u0) ? 1 : 0;
+      const int b = h / c.Hkv;
+      sg.t = FUSED ? s_tpos[h] : 0;
+      sg.plx = FUSED ? s_plx[h] : 0;
+      sg.ply = FUSED ? s_ply[h] : 0;
+      sg.npages = FUSED ? s_npg[h] : 0;
+      sg.grant = FUSED ? s_gr[h] : 0;
+      sg.qoff = (b * c.Hq + (h % c.Hkv) * g) * D;
+      if (sg.s1 > sg.s0) {
+        p0 = sg.s0 / c.P;
+        p1 = (sg.s1 - 1) / c.P;
+        my_sub = (sg.s1 - 1) / chunk - sg.s0 / chunk + 1;
+        my_pt = p1 - p0 + 1;
+      } else {
+        my_sub = 1;  // one empty sub-tile carries the segment's end
+      }
+      if (FUSED && (sg.ply & 1)) ++my_pt;  // page of the reused slot
+      my_ring = (FUSED && sg.t + 1 >= c.w) ? 1 : 0;
     }
-    sg.decide = (FUSED && fuse_decide && s_off[h] >= u0) ? 1 : 0;
-    const int b = h / c.Hkv;
-    sg.t = FUSED ? s_tpos[h] : 0;
-    sg.plx = FUSED ? s_plx[h] : 0;
-    sg.ply = FUSED ? s_ply[h] : 0;
-    sg.npages = FUSED ? s_npg[h] : 0;
-    sg.grant = FUSED ? s_gr[h] : 0;
-    sg.qoff = (b * c.Hq + (h % c.Hkv) * g) * D;
-    if (sg.s1 > sg.s0) {
-      p0 = sg.s0 / c.P;
-      p1 = (sg.s1 - 1) / c.P;
-      my_sub = (sg.s1 - 1) / chunk - sg.s0 / chunk + 1;
-      my_pt = p1 - p0 + 1;
-    } else {
-      my_sub = 1;  // one empty sub-tile carries the segment's end
+    xs = my_sub;
+    xp = my_pt;
+    xr = my_ring;
+#pragma unroll
+    for (int o2 = 1; o2 < 32; o2 <<= 1) {
+      const int a1 = __shfl_up_sync(0xffffffffu, xs, o2), a2 = __shfl_up_sync(0xffffffffu, xp, o2),
+                a3 = __shfl_up_sync(0xffffffffu, xr, o2);
+      if (lane >= o2) {
+        xs += a1;
+        xp += a2;
+        xr += a3;
+      }
     }
-    if (FUSED && (sg.ply & 1)) ++my_pt;  // page of the reused slot
-    my_ring = (FUSED && sg.t + 1 >= c.w) ? 1 : 0;
-  }
-  int tot_sub, tot_pt, tot_ring;
-  const int sub0 = block_exclusive_scan(my_sub, s_red, &tot_sub);
-  const int pt0 = block_exclusive_scan(my_pt, s_red, &tot_pt);
-  const int ring0 = block_exclusive_scan(my_ring, s_red, &tot_ring);
-  const bool pt_ok = tot_pt <= kFlatPtMax, table = tot_sub <= kFlatSubMax;
-  if (tid < nseg) {
-    sg.n0 = sub0;
-    sg.n1 = sub0 + my_sub;
-    sg.pt0 = (pt_ok && sg.s1 > sg.s0) ? pt0 : -1;
-    sg.sp_idx = (pt_ok && FUSED && (sg.ply & 1)) ? pt0 + my_pt - 1 : -1;
-    sg.ring_idx = my_ring ? ring0 : -1;
-    if (pt_ok) {
-      for (int p = p0; p <= p1; ++p) s_ptsrc[pt0 + p - p0] = li * c.maxp + p;
-      if (sg.sp_idx >= 0) s_ptsrc[sg.sp_idx] = li * c.maxp + sg.plx / c.P;
+    if (lane == 31) {
+      s_stot[warp][0] = xs;
+      s_stot[warp][1] = xp;
+      s_stot[warp][2] = xr;
     }
-    if (my_ring) s_ringsrc[ring0] = li * c.w + (sg.t + 1) % c.w;
-    segs[tid] = sg;
-    s_n0[tid] = sub0;
-  }
-  if (tid == 0) {
-    s_nseg = nseg;
-    s_nsub = tot_sub;
-    s_npt = pt_ok ? tot_pt : 0;
-    s_nring = tot_ring;
   }
   __syncthreads();
-  DMS_TRACE_MARK(0, 18);
+  if (warp < 2) {
+    const int tot_sub = s_stot[0][0] + s_stot[1][0], tot_pt = s_stot[0][1] + s_stot[1][1];
+    const int tot_ring = s_stot[0][2] + s_stot[1][2];
+    const int sub0 = xs - my_sub + (warp ? s_stot[0][0] : 0);
+    const int pt0 = xp - my_pt + (warp ? s_stot[0][1] : 0);
+    const int ring0 = xr - my_ring + (warp ? s_stot[0][2] : 0);
+    const bool pt_ok = tot_pt <= kFlatPtMax;
+    if (ks < nseg) {
+      sg.n0 = sub0;
+      sg.n1 = sub0 + my_sub;
+      sg.pt0 = (pt_ok && sg.s1 > sg.s0) ? pt0 : -1;
+      sg.sp_idx = (pt_ok && FUSED && (sg.ply & 1)) ? pt0 + my_pt - 1 : -1;
+      sg.ring_idx = my_ring ? ring0 : -1;
+      if (pt_ok) {
+        for (int p = p0; p <= p1; ++p) s_ptsrc[pt0 + p - p0] = li * c.maxp + p;
+        if (sg.sp_idx >= 0) s_ptsrc[sg.sp_idx] = li * c.maxp + sg.plx / c.P;
+      }
+      if (my_ring) s_ringsrc[ring0] = li * c.w + (sg.t + 1) % c.w;
+      segs[ks] = sg;
+      s_n0[ks] = sub0;
+    }
+    if (tid == 0) {
+      s_nseg = nseg;
+      s_nsub = tot_sub;
+      s_npt = pt_ok ? tot_pt : 0;
+      s_nring = tot_ring;
+    }
+  }
+  __syncthreads();
+  FLAT_MARK(18);
   nseg = s_nseg;
   const int nsub = s_nsub;
+  const bool table = nsub <= kFlatSubMax;
   // page ids and ring entries in one round trip, and meanwhile the sub-tile
   // descriptors, one thread per sub-tile: chunk i of a segment covers slots
   // [max(s0, (s0/C + i) C), min(s1, (s0/C + i + 1) C)), C the chunk size
@@ -620,13 +727,12 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
       s_sub[n] = d;
     }
   }
-  if (early) {
-    griddep_wait();
-    griddep_launch_dependents();
-  }
-  if (FUSED && tid == 0) s_next_page0 = c.ctrl[CTRL_NEXT_PAGE];
   __syncthreads();
-  DMS_TRACE_MARK(0, 1);
+  FLAT_MARK(1);
+  // Early: the producer starts the first ring of K/V loads (this layer's
+  // pages) before waiting; the aux warp waits before reading the inputs and
+  // the shared counters; the consumers see only what those two publish.
+  // The other warps of the CTA do not wait themselves.
 
   // Finish head segs[k]: LSE merge of its sources (the CTA's merged state
   // `cp` when it holds the whole head, else the partials in global scratch)
@@ -759,6 +865,12 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
   if (warp == kFlatAux) {
     // ---- aux: first what the append of each head needs, while the tiles
     // stream (the new token's scores and K/V rows, its decision logit) ------
+    if (early) {
+      griddep_wait();
+      griddep_launch_dependents();
+    }
+    if (FUSED && lane == 0) s_next_page0 = c.ctrl[CTRL_NEXT_PAGE];  // read by finishes after aux_done
+    __syncwarp();
     if (FUSED) {
       for (int k = 0; k < nseg; ++k) {
         const FlatSeg& sg = segs[k];
@@ -856,9 +968,11 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     if (lane == 0) {
       bool timed_out = false;
       const int mper = nst / kFlatConsumers;
+      const uint64_t kv_policy = l2_evict_first_policy();
       // sub-tile n into its stage once the stage's previous use is released:
-      // K and V boxes and the head's query rows
-      auto issue = [&](int n, int slot, int rows, int row0, float ks, float vs, int qoff) {
+      // K and V boxes, then (issue_q) the head's query rows, one mbarrier
+      // transaction for both
+      auto issue_kv = [&](int n, int slot, int rows, int row0, float ks, float vs) -> unsigned char* {
         int st, use;
         flat_stage(n, mper, &st, &use);
         if (use > 0 && !mbar_wait_bounded(&empty_bar[st], (use - 1) & 1)) timed_out = true;
@@ -873,23 +987,48 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
         mbar_expect_tx(&full_bar[st], bytes);
         if (rows > 0) {
           if (FP8) {
-            tma_load_2d(dst, &kmap, 0, row0, &full_bar[st]);
-            tma_load_2d(dst + F::TILE, &vmap, 0, row0, &full_bar[st]);
+            tma_load_2d_hint(dst, &kmap, 0, row0, &full_bar[st], kv_policy);
+            tma_load_2d_hint(dst + F::TILE, &vmap, 0, row0, &full_bar[st], kv_policy);
           } else {
 #pragma unroll
             for (int hf = 0; hf < F::HALVES; ++hf) {
-              tma_load_2d(dst + hf * kFlatRows * 128, &kmap, hf * 64, row0, &full_bar[st]);
-              tma_load_2d(dst + F::TILE + hf * kFlatRows * 128, &vmap, hf * 64, row0, &full_bar[st]);
+              tma_load_2d_hint(dst + hf * kFlatRows * 128, &kmap, hf * 64, row0, &full_bar[st], kv_policy);
+              tma_load_2d_hint(dst + F::TILE + hf * kFlatRows * 128, &vmap, hf * 64, row0, &full_bar[st],
+                               kv_policy);
             }
           }
         }
-        bulk_load(dst + 2 * F::TILE, q + qoff, static_cast<uint32_t>(g * D * 2), &full_bar[st]);
         if (n == 0) FLAT_MARK_ANY(10);
         if (n == 1) FLAT_MARK_ANY(14);
         if (n == nst - 1) FLAT_MARK_ANY(11);
+        return dst;
       };
+      auto issue_q = [&](int n, int qoff) {
+        int st, use;
+        flat_stage(n, mper, &st, &use);
+        bulk_load(sbase + st * stride + 2 * F::TILE, q + qoff, static_cast<uint32_t>(g * D * 2), &full_bar[st]);
+      };
+      auto issue = [&](int n, int slot, int rows, int row0, float ks, float vs, int qoff) {
+        issue_kv(n, slot, rows, row0, ks, vs);
+        issue_q(n, qoff);
+      };
+      int n_early = 0;
+      if (early && table) {
+        // the first ring of K/V while the previous kernel may still run
+        n_early = min(nsub, nst);
+        for (int n = 0; n < n_early; ++n) {
+          const int4 d = s_sub[n];
+          issue_kv(n, d.x, d.y & 255, d.z, FP8 ? s_ks[n] : 1.0f, FP8 ? s_vs[n] : 1.0f);
+        }
+      }
+      if (early) {
+        griddep_wait();
+        griddep_launch_dependents();
+      }
+      FLAT_MARK_ANY(21);
+      for (int n = 0; n < n_early; ++n) issue_q(n, segs[s_sub[n].y >> 8].qoff);
       if (table) {
-        for (int n = 0; n < nsub; ++n) {
+        for (int n = n_early; n < nsub; ++n) {
           const int4 d = s_sub[n];
           issue(n, d.x, d.y & 255, d.z, FP8 ? s_ks[n] : 1.0f, FP8 ? s_vs[n] : 1.0f, segs[d.y >> 8].qoff);
         }
@@ -950,7 +1089,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
         flat_stage(n, nst / kFlatConsumers, &st, &use);
         const bool ok = mbar_wait_bounded(&full_bar[st], use & 1);
         if (!ok) timed_out = true;
-        if (n == 0) DMS_TRACE_MARK(0, 3);
+        if (n == 0) FLAT_MARK(3);
         const FlatMeta m = meta[st];
         const unsigned char* stage = sbase + st * stride;
         if (!have_q) {
@@ -982,7 +1121,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
 
       // ---- end of a segment: merge the four warps' states into cpart[k & 1]
       // (once the aux warp has released it) and hand it over -----------------
-      if (k == 0) DMS_TRACE_MARK(0, 5);
+      if (k == 0) FLAT_MARK(5);
       const int j = k & 1;
       warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
       if (k >= 2 && !mbar_wait_bounded(&hq_empty[j], ((k >> 1) - 1) & 1)) timed_out = true;
@@ -992,7 +1131,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
       consumers_sync();
       if (tid == 0) mbar_arrive(&hq_full[j]);
     }
-    DMS_TRACE_MARK(0, 8);
+    FLAT_MARK(8);
     // the heads whose last part arrived here, once every hand-over is done
     if (!mbar_wait_bounded(&aux_done, 0)) timed_out = true;
     for (int f = 0; f < s_nfin; ++f) finish_head(s_fin[f], nullptr, tid, 128);
@@ -1018,7 +1157,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
       for (int bb = tid; bb < c.B; bb += kFlatThreads) c.pos[layer * c.B + bb] += 1;
     }
   }
-  DMS_TRACE_MARK(0, 9);
+  FLAT_MARK(9);
 }
 
 // Launch geometry of the flat kernel, or false when the shape is outside what
