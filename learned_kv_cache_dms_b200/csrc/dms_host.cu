@@ -307,7 +307,7 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D),
                                 static_cast<cuuint64_t>(desc->batch) * desc->num_kv_heads * desc->max_positions};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-    const cuuint32_t box[2] = {64u, 128u};
+    const cuuint32_t box[2] = {64u, 64u};  // 64-key tiles of the prefill attention
     c->has_kept_maps = make_bf16_map(&c->kept_kmap, v.kept_k, 2, dims, strides, box) &&
                        make_bf16_map(&c->kept_vmap, v.kept_v, 2, dims, strides, box);
   }
@@ -466,7 +466,7 @@ int dms_prefill_attention(dms_cache* c, int layer, const dms_prefill_args* a, vo
     const cuuint32_t qb[3] = {64u, static_cast<cuuint32_t>(g), static_cast<cuuint32_t>(128 / g)};
     const cuuint64_t kd[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(c->desc.num_kv_heads), bt};
     const cuuint64_t ks[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(c->desc.num_kv_heads) * D * 2};
-    const cuuint32_t kbx[3] = {64u, 1u, 128u};
+    const cuuint32_t kbx[3] = {64u, 1u, 64u};
     maps.valid = make_bf16_map(&maps.q, a->q, 3, qd, qs, qb) && make_bf16_map(&maps.k, a->k, 3, kd, ks, kbx) &&
                  make_bf16_map(&maps.v, a->v, 3, kd, ks, kbx);
     maps.kept_k = c->kept_kmap;

@@ -6,23 +6,29 @@
 //   V_i = { j <= i : i - j < w  or  alpha_j <= 0 }
 // = band (i - w < j <= i)  U  kept prefix (j <= i - w, alpha_j <= 0).
 //
-// A CTA owns 128 query rows = NP = 128/g positions x the g query heads that
-// share one KV head (row t = p * g + r), so every K/V tile feeds all g heads.
-// Key tiles of 128 come from the contiguous band [i0 - w + 1, i1 - 1] and from
+// A CTA owns two Q tiles of 128 rows; a Q tile is NP = 128/g consecutive
+// positions x the g query heads that share one KV head (row t = p * g + r),
+// so every K/V tile feeds 2 x 128 rows.  Key tiles of 64 come from the
+// contiguous band [i0 - w + 1, i1 - 1] of the CTA's 2 NP positions and from
 // the position-sorted kept list; evicted keys outside the window are never
-// loaded.
-//   S = Q K^T : tcgen05.mma M=128, N=128, K=16 x D/16, Q and K K-major in
-//               128-byte-swizzled shared memory, S in TMEM columns [0, 128)
-//   softmax   : 8 warps; row t is TMEM lane t, its 128 scores split between
-//               two threads (columns 0-63 and 64-127).  The exponent reference
-//               of a row is raised only when a tile's max exceeds it by 2^8, so
-//               O is rescaled rarely (the final O / l is exact either way).
-//   O += P V  : P (bf16, K-major) written to shared memory by the softmax
-//               threads, V staged as MN-major B, O in TMEM columns [128, 128+D)
-// Tiles arrive by TMA (no multicast): band keys/values straight from the input
-// rows, kept ones from the position-sorted kept copy written by the
-// compaction.  Two K/V stages and two S buffers let S(t+1) run on the tensor
-// cores while the softmax of tile t runs; mbarriers order loads, S, and P V.
+// loaded.  Warp roles:
+//   load warp  : TMA (no multicast) of the Q tiles, then K and V of every key
+//                tile into a ring of stages (band tiles straight from the
+//                input rows, kept tiles from the kept copy written by the
+//                compaction), with the tile's key positions and, per Q tile,
+//                whether every row sees every key (no mask needed);
+//   MMA warp   : S_w = Q_w K^T (tcgen05.mma M=128, N=64, K=16 x D/16, both
+//                K-major in 128-byte-swizzled shared memory, S_w in TMEM) and
+//                O_w += P_w V (P_w K-major from shared memory, V MN-major,
+//                O_w in TMEM), in the order S0(t+1), S1(t+1), PV0(t), PV1(t):
+//                each Q tile's next scores run on the tensor cores while its
+//                softmax of tile t runs, and the two softmax groups interleave;
+//   softmax    : one warpgroup per Q tile, one thread per row; the exponent
+//                reference of a row is raised only when a tile's max exceeds
+//                it by 2^8, so O is rescaled rarely (O / l is exact either
+//                way).
+// mbarriers order every hand-off (loads, S ready / S read, P ready, P V done,
+// stage free); every wait is bounded.
 #include "dms_internal.cuh"
 
 namespace dms {
@@ -30,26 +36,29 @@ namespace dms {
 #ifdef DMS_TRACE
 __device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
 #endif
-// phases of tile 1 (tracing builds)
-#define TC_MARK(tile, ph) \
-  if ((tile) == 1) DMS_TRACE_MARK(0, (ph))
 
-constexpr int kTcBN = 128;       // keys per tile
-constexpr int kTcRows = 128;     // query rows per CTA (TMEM lanes)
-constexpr int kTcThreads = 256;  // two threads per row
+constexpr int kPfRows = 128;     // query rows per Q tile (TMEM lanes)
+constexpr int kPfQT = 2;         // Q tiles per CTA
+constexpr int kPfBN = 64;        // keys per K/V tile
+constexpr int kPfMmaWarp = 8;    // warps 0-3: softmax of Q tile 0, 4-7: Q tile 1
+constexpr int kPfLoadWarp = 9;
+constexpr int kPfThreads = 320;
 
 template <int D>
-struct TcSmem {
+struct PfSmem {
   static constexpr int HALVES = D / 64;
-  static constexpr int Q_BYTES = HALVES * kTcRows * 128;        // [half][128 rows][128 B]
-  static constexpr int KV_BYTES = HALVES * kTcBN * 128;         // [half][128 keys][128 B]
-  static constexpr int P_BYTES = (kTcBN / 64) * kTcRows * 128;  // [key half][128 rows][128 B]
+  static constexpr int Q_BYTES = HALVES * kPfRows * 128;  // one Q tile: [half][128 rows][128 B]
+  static constexpr int KV_BYTES = HALVES * kPfBN * 128;   // K (or V) of one key tile: [half][64 keys][128 B]
+  static constexpr int P_BYTES = kPfRows * 128;           // one P tile: [128 rows][64 keys x 2 B]
+  static constexpr int ST = D == 64 ? 4 : 3;              // K/V stages
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;       // 2 stages
-  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;  // 2 stages
-  static constexpr int OFF_P = OFF_V + 2 * KV_BYTES;
-  static constexpr int BYTES = OFF_P + P_BYTES;
-  static constexpr uint32_t TMEM_COLS = 512;  // S double buffer: 2 x 128 columns, O: D columns at 256
+  static constexpr int OFF_P = OFF_Q + kPfQT * Q_BYTES;
+  static constexpr int OFF_K = OFF_P + kPfQT * P_BYTES;
+  static constexpr int OFF_V = OFF_K + ST * KV_BYTES;
+  static constexpr int BYTES = OFF_V + ST * KV_BYTES;
+  // tensor memory: S0, S1 (64 columns each), O0, O1 (D columns each)
+  static constexpr uint32_t COL_O = 2 * kPfBN;
+  static constexpr uint32_t TMEM_COLS = COL_O + 2 * D <= 256 ? 256 : 512;
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
@@ -86,272 +95,310 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
 }
 
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kPfThreads, 1)
     k_attn_prefill_tc(CacheView c, int T, __nv_bfloat16* o, const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                       const __grid_constant__ CUtensorMap kkmap, const __grid_constant__ CUtensorMap kvmap) {
-  using L = TcSmem<D>;
+  using L = PfSmem<D>;
+  constexpr int ST = L::ST;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sb = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sQ = sb + L::OFF_Q;
-  unsigned char* sP = sb + L::OFF_P;
-  __shared__ __align__(16) int kpos[2][kTcBN];
-  __shared__ float s_tmax[2][kTcRows];
-  __shared__ float s_lpart[kTcRows];
-  __shared__ float s_lsum[kTcRows];
+  __shared__ __align__(16) int kpos[ST][kPfBN];  // key positions of the tile in each stage (-1: absent)
+  __shared__ int tfull[ST][kPfQT];              // 1: every row of that Q tile sees every key of the tile
   __shared__ uint32_t tmem_base;
-  __shared__ __align__(8) uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_pv;
+  __shared__ __align__(8) uint64_t bar_q, k_full[ST], v_full[ST], kv_empty[ST];
+  __shared__ __align__(8) uint64_t s_full[kPfQT], s_free[kPfQT], p_full[kPfQT], pv_done[kPfQT];
   __shared__ int s_abort;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int row = tid & (kTcRows - 1);  // TMEM lane / query row
-  const int half = tid >> 7;            // which 64 key columns (and D/2 output columns)
-  const int g = c.Hq / c.Hkv, NP = kTcRows / g;
-  const int nqb = (T + NP - 1) / NP;
-  const int qb = nqb - 1 - static_cast<int>(blockIdx.x);  // heavy (late) blocks first
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = c.Hq / c.Hkv, NP = kPfRows / g;
+  const int nblk = (T + kPfQT * NP - 1) / (kPfQT * NP);
+  const int blk = nblk - 1 - static_cast<int>(blockIdx.x);  // heavy (late) blocks first
   const int h = blockIdx.y, b = blockIdx.z, w = c.w;
-  const int i0 = qb * NP, i1 = min(T, i0 + NP);
+  const int i0 = blk * kPfQT * NP, i1 = min(T, i0 + kPfQT * NP);
   const int bh = b * c.Hkv + h;
   const int* kept = c.kept + static_cast<long>(bh) * c.max_pos;
   const int nk = (i1 - w > 0) ? c.kept_upto[static_cast<long>(bh) * (c.max_pos + 1) + (i1 - w)] : 0;
   const int jlo = max(0, i0 - w + 1), jhi = i1 - 1;
-  const int n_kept_tiles = (nk + kTcBN - 1) / kTcBN;
-  const int ntiles = n_kept_tiles + (jhi - jlo + kTcBN) / kTcBN;
-  const int i_row = i0 + row / g, r_row = row % g;
-
-  // position of key row `row` of a tile (-1: absent)
-  auto key_pos = [&](int tile) -> int {
-    if (tile < n_kept_tiles) {
-      const int kidx = tile * kTcBN + row;
-      return kidx < nk ? kept[kidx] : -1;
-    }
-    const int jj = jlo + (tile - n_kept_tiles) * kTcBN + row;
-    return jj <= jhi ? jj : -1;
-  };
-  // TMA loads of a tile's keys or values into stage `st` (thread 0): band
-  // tiles straight from the input rows, kept tiles from the kept copy
-  auto load_kv = [&](int tile, int st, bool is_v) {
-    unsigned char* dst = sb + (is_v ? L::OFF_V : L::OFF_K) + st * L::KV_BYTES;
-    uint64_t* bar = is_v ? &bar_v[st] : &bar_k[st];
-    mbar_expect_tx(bar, L::KV_BYTES);
-    for (int hf = 0; hf < L::HALVES; ++hf) {
-      if (tile < n_kept_tiles)
-        tma_load_2d(dst + hf * (kTcBN * 128), is_v ? &kvmap : &kkmap, hf * 64, bh * c.max_pos + tile * kTcBN, bar);
-      else
-        tma_load_3d(dst + hf * (kTcBN * 128), is_v ? &vmap : &kmap, hf * 64, h,
-                    b * T + jlo + (tile - n_kept_tiles) * kTcBN, bar);
-    }
-  };
+  const int nkt = (nk + kPfBN - 1) / kPfBN;  // kept tiles
+  const int ntiles = nkt + (jhi - jlo + kPfBN) / kPfBN;
 
   if (tid == 0) {
     mbar_init(&bar_q, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_k[i], 1);
-      mbar_init(&bar_v[i], 1);
-      mbar_init(&bar_s[i], 1);
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(&bar_pv, 1);
+    for (int i = 0; i < kPfQT; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kPfRows);
+      mbar_init(&p_full[i], kPfRows);
+      mbar_init(&pv_done[i], 1);
+    }
     fence_mbar_init();
     s_abort = 0;
-    mbar_expect_tx(&bar_q, L::Q_BYTES);
-    for (int hf = 0; hf < L::HALVES; ++hf) tma_load_3d(sQ + hf * (kTcRows * 128), &qmap, hf * 64, h * g, b * T + i0, &bar_q);
-    load_kv(0, 0, false);
-    load_kv(0, 0, true);
-    if (ntiles > 1) {
-      load_kv(1, 1, false);
-      load_kv(1, 1, true);
-    }
   }
-  if (warp == 0) tmem_alloc(&tmem_base, L::TMEM_COLS);
-  if (half == 0) kpos[0][row] = key_pos(0);
+  if (warp == kPfMmaWarp) tmem_alloc(&tmem_base, L::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const uint32_t tmem_o = tmem + lane_off + 256 + half * (D / 2);  // this thread's D/2 output columns
-  constexpr uint32_t IDESC_S = umma_idesc_bf16(128, kTcBN, 0);
-  constexpr uint32_t IDESC_O = umma_idesc_bf16(128, D, 1);
-  const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-  float m_ref = -INFINITY, l_part = 0.f;
-
-  // S(t) = Q K(t)^T into TMEM buffer t & 1 (thread 0)
-  auto issue_s = [&](int tile) -> bool {
-    const int st = tile & 1;
-    if (!mbar_wait_bounded(&bar_k[st], (tile >> 1) & 1)) return false;
-    tc_fence_after();
-    const uint32_t qa = smem_u32(sQ), ka = smem_u32(sb + L::OFF_K + st * L::KV_BYTES);
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const uint32_t off = (ks / 4) * (kTcRows * 128) + (ks % 4) * 32;
-      const uint32_t koff = (ks / 4) * (kTcBN * 128) + (ks % 4) * 32;
-      umma_bf16(tmem + st * kTcBN, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(ka + koff, 16, 1024),
-                IDESC_S, ks > 0 ? 1u : 0u);
-    }
-    umma_commit(&bar_s[st]);
-    return true;
+  auto give_up = [&]() {
+    set_status(c.ctrl, DMS_ST_TIMEOUT);
+    s_abort = 1;
   };
-  if (tid == 0) {
-    if (!mbar_wait_bounded(&bar_q, 0) || !issue_s(0)) {
-      set_status(c.ctrl, DMS_ST_TIMEOUT);
-      s_abort = 1;
-    }
-  }
 
-  for (int tile = 0; tile < ntiles; ++tile) {
-    const int st = tile & 1;
-    const bool kept_tile = tile < n_kept_tiles;
-    const int j_next = tile + 1 < ntiles ? key_pos(tile + 1) : -1;  // read now, stored after the softmax
-    TC_MARK(tile, 0);
-    // next S on the tensor cores while this tile's softmax runs
-    if (tid == 0 && !s_abort && tile + 1 < ntiles && !issue_s(tile + 1)) {
-      set_status(c.ctrl, DMS_ST_TIMEOUT);
-      s_abort = 1;
+  if (warp == kPfLoadWarp) {
+    // ---- loads ---------------------------------------------------------
+    if (lane == 0) {
+      mbar_expect_tx(&bar_q, kPfQT * L::Q_BYTES);
+      for (int qt = 0; qt < kPfQT; ++qt)
+        for (int hf = 0; hf < L::HALVES; ++hf)
+          tma_load_3d(sb + L::OFF_Q + qt * L::Q_BYTES + hf * (kPfRows * 128), &qmap, hf * 64, h * g,
+                      b * T + i0 + qt * NP, &bar_q);
     }
-    if (!mbar_wait_bounded(&bar_s[st], (tile >> 1) & 1)) {
-      if (tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
-      s_abort = 1;
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j % ST, use = j / ST;
+      if (use > 0) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_bounded(&kv_empty[st], (use - 1) & 1);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          if (lane == 0) give_up();
+          break;
+        }
+      }
+      // key positions: two per lane
+      const bool kt = j < nkt;
+      const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int kk = lane + 32 * e;
+        int p;
+        if (kt) {
+          p = jb + kk < nk ? kept[jb + kk] : -1;
+        } else {
+          p = jb + kk <= jhi ? jb + kk : -1;
+        }
+        kpos[st][kk] = p;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        // mask-free for Q tile qt: every key present and visible to all of
+        // its rows [qmin, qmax] (kept: j <= i - w; band: i - w < j <= i)
+        for (int qt = 0; qt < kPfQT; ++qt) {
+          const int qmin = i0 + qt * NP, qmax = min(T, qmin + NP) - 1;
+          int full;
+          if (kt)
+            full = (jb + kPfBN <= nk) && kpos[st][kPfBN - 1] <= qmin - w;
+          else
+            full = (jb + kPfBN - 1 <= jhi) && jb > qmax - w && jb + kPfBN - 1 <= qmin;
+          tfull[st][qt] = full;
+        }
+        mbar_expect_tx(&k_full[st], L::KV_BYTES);
+        for (int hf = 0; hf < L::HALVES; ++hf) {
+          unsigned char* dk = sb + L::OFF_K + st * L::KV_BYTES + hf * (kPfBN * 128);
+          if (kt)
+            tma_load_2d(dk, &kkmap, hf * 64, bh * c.max_pos + jb, &k_full[st]);
+          else
+            tma_load_3d(dk, &kmap, hf * 64, h, b * T + jb, &k_full[st]);
+        }
+        mbar_expect_tx(&v_full[st], L::KV_BYTES);
+        for (int hf = 0; hf < L::HALVES; ++hf) {
+          unsigned char* dv = sb + L::OFF_V + st * L::KV_BYTES + hf * (kPfBN * 128);
+          if (kt)
+            tma_load_2d(dv, &kvmap, hf * 64, bh * c.max_pos + jb, &v_full[st]);
+          else
+            tma_load_3d(dv, &vmap, hf * 64, h, b * T + jb, &v_full[st]);
+        }
+      }
+      __syncwarp();
+      if (s_abort) break;
     }
-    tc_fence_after();
-    TC_MARK(tile, 2);
-    // K stage st is free (S(tile) complete): fetch the keys of tile + 2
-    if (tid == 0 && tile + 2 < ntiles) load_kv(tile + 2, st, false);
-
-    // ---- softmax: this thread's 64 scores of row `row` ----
-    uint32_t sr[64];
-    tmem_ld32_nowait(tmem + lane_off + st * kTcBN + half * 64, sr);
-    tmem_ld32_nowait(tmem + lane_off + st * kTcBN + half * 64 + 32, sr + 32);
-    tmem_wait_ld();
-    TC_MARK(tile, 6);
-    // visible: lo <= j <= hi (kept tile: 0 <= j <= i - w; band: i - w < j <= i); absent keys are -1
-    const int lo = kept_tile ? 0 : max(0, i_row - w + 1);
-    const int hi = kept_tile ? i_row - w : i_row;
-    float x[64];
-    float tmax = -INFINITY;
+  } else if (warp == kPfMmaWarp) {
+    // ---- tensor-core issue (one thread) ------------------------------------
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = umma_idesc_bf16(kPfRows, kPfBN, 0);
+      constexpr uint32_t IDESC_O = umma_idesc_bf16(kPfRows, D, 1);
+      auto issue_s = [&](int qt, int j) -> bool {
+        const int st = j % ST;
+        if (!mbar_wait_bounded(&k_full[st], (j / ST) & 1)) return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sb + L::OFF_Q + qt * L::Q_BYTES);
+        const uint32_t ka = smem_u32(sb + L::OFF_K + st * L::KV_BYTES);
 #pragma unroll
-    for (int n4 = 0; n4 < 16; ++n4) {
-      const int4 jv = reinterpret_cast<const int4*>(kpos[st] + half * 64)[n4];
-      const int js[4] = {jv.x, jv.y, jv.z, jv.w};
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t qoff = (ks / 4) * (kPfRows * 128) + (ks % 4) * 32;
+          const uint32_t koff = (ks / 4) * (kPfBN * 128) + (ks % 4) * 32;
+          umma_bf16(tmem + qt * kPfBN, umma_desc_sw128(qa + qoff, 16, 1024), umma_desc_sw128(ka + koff, 16, 1024),
+                    IDESC_S, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[qt]);
+        return true;
+      };
+      auto issue_pv = [&](int qt, int j) -> bool {
+        const int st = j % ST;
+        if (!mbar_wait_bounded(&v_full[st], (j / ST) & 1)) return false;
+        if (!mbar_wait_bounded(&p_full[qt], j & 1)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sb + L::OFF_P + qt * L::P_BYTES);
+        const uint32_t va = smem_u32(sb + L::OFF_V + st * L::KV_BYTES);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int n = n4 * 4 + e;
-        x[n] = (js[e] >= lo && js[e] <= hi) ? __uint_as_float(sr[n]) * sl2 : -INFINITY;
-        tmax = fmaxf(tmax, x[n]);
+        for (int ks = 0; ks < kPfBN / 16; ++ks)
+          umma_bf16(tmem + L::COL_O + qt * D, umma_desc_sw128(pa + ks * 32, 16, 1024),
+                    umma_desc_sw128(va + ks * 16 * 128, kPfBN * 128, 1024), IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(&pv_done[qt]);
+        return true;
+      };
+      bool ok = mbar_wait_bounded(&bar_q, 0);
+      if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (j + 1 < ntiles) {
+          // the next scores of each Q tile once its softmax has read S(j)
+          ok = mbar_wait_bounded(&s_free[0], j & 1) && issue_s(0, j + 1);
+          ok = ok && mbar_wait_bounded(&s_free[1], j & 1) && issue_s(1, j + 1);
+        }
+        ok = ok && issue_pv(0, j) && issue_pv(1, j);
+        if (ok) umma_commit(&kv_empty[j % ST]);
+        if (s_abort) break;
+      }
+      if (!ok) give_up();
+    }
+  } else {
+    // ---- softmax: warpgroup qt, one thread per row ---------------------------
+    const int qt = warp >> 2, row = tid & (kPfRows - 1);
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tmem_s = tmem + lane_off + qt * kPfBN;
+    const uint32_t tmem_o = tmem + lane_off + L::COL_O + qt * D;
+    unsigned char* sP = sb + L::OFF_P + qt * L::P_BYTES;
+    const int i_row = i0 + qt * NP + row / g, r_row = row % g;
+    const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+    float m_ref = -INFINITY, l_row = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j % ST;
+      const bool kt = j < nkt;
+      // the tile's key positions (published with the loads) and its scores
+      ok = mbar_wait_bounded(&k_full[st], (j / ST) & 1) && mbar_wait_bounded(&s_full[qt], j & 1);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[kPfBN];
+      tmem_ld32_nowait(tmem_s, sr);
+      tmem_ld32_nowait(tmem_s + 32, sr + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&s_free[qt]);  // S may be overwritten by the next tile's scores
+      float x[kPfBN];
+      float tmax = -INFINITY;
+      if (tfull[st][qt]) {
+#pragma unroll
+        for (int n = 0; n < kPfBN; ++n) {
+          x[n] = __uint_as_float(sr[n]) * sl2;
+          tmax = fmaxf(tmax, x[n]);
+        }
+      } else {
+        // visible: lo <= j <= hi (kept: 0 <= j <= i - w; band: i - w < j <= i); absent keys are -1
+        const int lo = kt ? 0 : max(0, i_row - w + 1);
+        const int hi = kt ? i_row - w : i_row;
+#pragma unroll
+        for (int n4 = 0; n4 < kPfBN / 4; ++n4) {
+          const int4 jv = reinterpret_cast<const int4*>(kpos[st])[n4];
+          const int js[4] = {jv.x, jv.y, jv.z, jv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int n = n4 * 4 + e;
+            x[n] = (js[e] >= lo && js[e] <= hi) ? __uint_as_float(sr[n]) * sl2 : -INFINITY;
+            tmax = fmaxf(tmax, x[n]);
+          }
+        }
+      }
+      // raise the reference only when this tile exceeds it by more than 2^8
+      const bool raise = tmax > m_ref + 8.0f;
+      float factor = 1.0f;
+      if (raise) {
+        factor = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - tmax);
+        m_ref = tmax;
+        l_row *= factor;
+      }
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a fully masked row so far: all p = 0
+      uint32_t pk[kPfBN / 2];
+      float psum = 0.f;
+#pragma unroll
+      for (int e = 0; e < kPfBN / 2; ++e) {
+        const float p0 = ex2_approx(x[2 * e] - m_use);
+        const float p1 = ex2_approx(x[2 * e + 1] - m_use);
+        psum += p0 + p1;
+        pk[e] = pack_bf16(p0, p1);
+      }
+      l_row += psum;
+      // P V of the previous tile has finished with P and with O
+      if (j > 0 && !mbar_wait_bounded(&pv_done[qt], (j - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (j > 0 && __any_sync(0xffffffffu, raise && factor != 1.0f)) {
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float ov[32];
+          tmem_ld32(tmem_o + c0, ov);
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) ov[jj] *= factor;
+          tmem_st32(tmem_o + c0, ov);
+        }
+      }
+#pragma unroll
+      for (int ch = 0; ch < kPfBN / 8; ++ch)
+        *reinterpret_cast<uint4*>(sP + swz(row, ch)) =
+            make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+      fence_proxy_async();  // P visible to the tensor cores
+      tc_fence_before();
+      mbar_arrive(&p_full[qt]);
+      if (s_abort) {
+        ok = false;
+        break;
       }
     }
-    s_tmax[half][row] = tmax;
-    __syncthreads();
-    if (s_abort) break;
-    tmax = fmaxf(s_tmax[0][row], s_tmax[1][row]);
-    TC_MARK(tile, 7);
-    // raise the reference only when this tile exceeds it by more than 2^8
-    const bool raise = tmax > m_ref + 8.0f;
-    float factor = 1.0f;
-    if (raise) {
-      factor = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - tmax);
-      m_ref = tmax;
-      l_part *= factor;
-    }
-    const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a fully masked row so far: all p = 0
-    uint32_t pk[32];
-    float psum = 0.f;
+    // the last P V, then O / l
+    if (ok && ntiles > 0) ok = mbar_wait_bounded(&pv_done[qt], (ntiles - 1) & 1);
+    if (!ok) {
+      if ((tid & (kPfRows - 1)) == 0) give_up();
+    } else {
+      tc_fence_after();
+      const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+      __nv_bfloat16* orow = o + ((static_cast<long>(b) * T + i_row) * c.Hq + h * g + r_row) * D;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float p0 = ex2_approx(x[2 * e] - m_use);
-      const float p1 = ex2_approx(x[2 * e + 1] - m_use);
-      psum += p0 + p1;
-      pk[e] = pack_bf16(p0, p1);
-    }
-    l_part += psum;
-    // P(tile - 1) V has finished with the P buffer, with O and with V stage st ^ 1
-    if (tile > 0 && !mbar_wait_bounded(&bar_pv, (tile - 1) & 1)) {
-      if (tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
-      s_abort = 1;
-    }
-    tc_fence_after();
-    if (tid == 0 && tile >= 1 && tile + 1 < ntiles) load_kv(tile + 1, st ^ 1, true);
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-      *reinterpret_cast<uint4*>(sP + half * (kTcRows * 128) + swz(row, ch)) =
-          make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-    TC_MARK(tile, 8);
-    // rescale this thread's half of O in tensor memory where the reference moved
-    if (tile > 0 && __any_sync(0xffffffffu, raise && factor != 1.0f)) {
-#pragma unroll
-      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+      for (int c0 = 0; c0 < D; c0 += 32) {
         float ov[32];
         tmem_ld32(tmem_o + c0, ov);
+        if (i_row < T) {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) ov[jj] *= factor;
-        tmem_st32(tmem_o + c0, ov);
-      }
-    }
-    if (half == 0) kpos[st ^ 1][row] = j_next;  // the next tile's key positions
-    TC_MARK(tile, 3);
-    fence_proxy_async();  // P visible to the tensor cores
-    tc_fence_before();
-    __syncthreads();
-    if (s_abort) break;
-    if (tid == 0) {
-      if (!mbar_wait_bounded(&bar_v[st], (tile >> 1) & 1)) {
-        set_status(c.ctrl, DMS_ST_TIMEOUT);
-        s_abort = 1;
-      } else {
-        tc_fence_after();
-        const uint32_t pa = smem_u32(sP), va = smem_u32(sb + L::OFF_V + st * L::KV_BYTES);
-#pragma unroll
-        for (int ks = 0; ks < kTcBN / 16; ++ks) {
-          const uint32_t poff = (ks / 4) * (kTcRows * 128) + (ks % 4) * 32;
-          umma_bf16(tmem + 256, umma_desc_sw128(pa + poff, 16, 1024),
-                    umma_desc_sw128(va + ks * 16 * 128, kTcBN * 128, 1024), IDESC_O, (tile > 0 || ks > 0) ? 1u : 0u);
-        }
-        umma_commit(&bar_pv);
-      }
-    }
-    TC_MARK(tile, 4);
-  }
-
-  // wait for the last P V, then write O / l (l = the two halves' partial sums)
-  if (half == 1) s_lpart[row] = l_part;
-  __syncthreads();
-  if (half == 0) s_lsum[row] = l_part + s_lpart[row];
-  __syncthreads();
-  if (!s_abort && ntiles > 0) {
-    if (!mbar_wait_bounded(&bar_pv, (ntiles - 1) & 1) && tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
-    tc_fence_after();
-    const float inv = s_lsum[row] > 0.f ? 1.f / s_lsum[row] : 0.f;
-    __nv_bfloat16* orow = o + ((static_cast<long>(b) * T + i_row) * c.Hq + h * g + r_row) * D + half * (D / 2);
-#pragma unroll
-    for (int c0 = 0; c0 < D / 2; c0 += 32) {
-      float ov[32];
-      tmem_ld32(tmem_o + c0, ov);
-      if (i_row < T) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 pkk;
-          pkk.x = pack_bf16(ov[e] * inv, ov[e + 1] * inv);
-          pkk.y = pack_bf16(ov[e + 2] * inv, ov[e + 3] * inv);
-          pkk.z = pack_bf16(ov[e + 4] * inv, ov[e + 5] * inv);
-          pkk.w = pack_bf16(ov[e + 6] * inv, ov[e + 7] * inv);
-          *reinterpret_cast<uint4*>(orow + c0 + e) = pkk;
+          for (int e = 0; e < 32; e += 8) {
+            uint4 pkk;
+            pkk.x = pack_bf16(ov[e] * inv, ov[e + 1] * inv);
+            pkk.y = pack_bf16(ov[e + 2] * inv, ov[e + 3] * inv);
+            pkk.z = pack_bf16(ov[e + 4] * inv, ov[e + 5] * inv);
+            pkk.w = pack_bf16(ov[e + 6] * inv, ov[e + 7] * inv);
+            *reinterpret_cast<uint4*>(orow + c0 + e) = pkk;
+          }
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
+  if (warp == kPfMmaWarp) tmem_dealloc(tmem, L::TMEM_COLS);
 }
 
 template <int D>
 static cudaError_t launch_tc(const CacheView& c, int T, void* o, const PrefillMaps& m, cudaStream_t s) {
-  const size_t smem = TcSmem<D>::BYTES + 1024;
+  const size_t smem = PfSmem<D>::BYTES + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_attn_prefill_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int g = c.Hq / c.Hkv, NP = kTcRows / g;
-  dim3 grid((T + NP - 1) / NP, c.Hkv, c.B);
-  k_attn_prefill_tc<D><<<grid, kTcThreads, smem, s>>>(c, T, static_cast<__nv_bfloat16*>(o), m.q, m.k, m.v, m.kept_k,
+  const int g = c.Hq / c.Hkv, NP = kPfRows / g;
+  dim3 grid((T + kPfQT * NP - 1) / (kPfQT * NP), c.Hkv, c.B);
+  k_attn_prefill_tc<D><<<grid, kPfThreads, smem, s>>>(c, T, static_cast<__nv_bfloat16*>(o), m.q, m.k, m.v, m.kept_k,
                                                       m.kept_v);
   return cudaGetLastError();
 }
