@@ -17,12 +17,12 @@
 //                input rows, kept tiles from the kept copy written by the
 //                compaction), with the tile's key positions and, per Q tile,
 //                whether every row sees every key (no mask needed);
-//   MMA warp   : S_w = Q_w K^T (tcgen05.mma M=128, N=64, K=16 x D/16, both
-//                K-major in 128-byte-swizzled shared memory, S_w in TMEM) and
-//                O_w += P_w V (P_w K-major from shared memory, V MN-major,
-//                O_w in TMEM), in the order S0(t+1), S1(t+1), PV0(t), PV1(t):
-//                each Q tile's next scores run on the tensor cores while its
-//                softmax of tile t runs, and the two softmax groups interleave;
+//   MMA warps  : one per Q tile w: S_w = Q_w K^T (tcgen05.mma M=128, N=64,
+//                K=16 x D/16, both K-major in 128-byte-swizzled shared memory,
+//                S_w in TMEM) and O_w += P_w V (P_w K-major from shared memory,
+//                V MN-major, O_w in TMEM), in the order S_w(t+1), PV_w(t): each
+//                Q tile's next scores run on the tensor cores while its softmax
+//                of tile t runs, and the two Q tiles proceed independently;
 //   softmax    : one warpgroup per Q tile, one thread per row; the exponent
 //                reference of a row is raised only when a tile's max exceeds
 //                it by 2^8, so O is rescaled rarely (O / l is exact either
@@ -40,9 +40,10 @@ __device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
 constexpr int kPfRows = 128;     // query rows per Q tile (TMEM lanes)
 constexpr int kPfQT = 2;         // Q tiles per CTA
 constexpr int kPfBN = 64;        // keys per K/V tile
-constexpr int kPfMmaWarp = 8;    // warps 0-3: softmax of Q tile 0, 4-7: Q tile 1
-constexpr int kPfLoadWarp = 9;
-constexpr int kPfThreads = 320;
+constexpr int kPfMmaWarp = 8;    // warps 0-3: softmax of Q tile 0, 4-7: Q tile 1; 8, 9: MMA issue for
+                                 // Q tile 0, 1
+constexpr int kPfLoadWarp = 10;
+constexpr int kPfThreads = 352;
 
 template <int D>
 struct PfSmem {
@@ -128,12 +129,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int i = 0; i < ST; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], kPfQT);  // both Q tiles' P V done with the stage
     }
     for (int i = 0; i < kPfQT; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kPfRows);
-      mbar_init(&p_full[i], kPfRows);
+      mbar_init(&s_free[i], 4);  // one arrival per softmax warp
+      mbar_init(&p_full[i], 4);
       mbar_init(&pv_done[i], 1);
     }
     fence_mbar_init();
@@ -215,12 +216,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       __syncwarp();
       if (s_abort) break;
     }
-  } else if (warp == kPfMmaWarp) {
-    // ---- tensor-core issue (one thread) ------------------------------------
+  } else if (warp == kPfMmaWarp || warp == kPfMmaWarp + 1) {
+    // ---- tensor-core issue for Q tile qt (one thread) ----------------------
+    const int qt = warp - kPfMmaWarp;
     if (lane == 0) {
       constexpr uint32_t IDESC_S = umma_idesc_bf16(kPfRows, kPfBN, 0);
       constexpr uint32_t IDESC_O = umma_idesc_bf16(kPfRows, D, 1);
-      auto issue_s = [&](int qt, int j) -> bool {
+      auto issue_s = [&](int j) -> bool {
         const int st = j % ST;
         if (!mbar_wait_bounded(&k_full[st], (j / ST) & 1)) return false;
         tc_fence_after();
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         umma_commit(&s_full[qt]);
         return true;
       };
-      auto issue_pv = [&](int qt, int j) -> bool {
+      auto issue_pv = [&](int j) -> bool {
         const int st = j % ST;
         if (!mbar_wait_bounded(&v_full[st], (j / ST) & 1)) return false;
         if (!mbar_wait_bounded(&p_full[qt], j & 1)) return false;
@@ -248,18 +250,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           umma_bf16(tmem + L::COL_O + qt * D, umma_desc_sw128(pa + ks * 32, 16, 1024),
                     umma_desc_sw128(va + ks * 16 * 128, kPfBN * 128, 1024), IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
         umma_commit(&pv_done[qt]);
+        umma_commit(&kv_empty[st]);  // this Q tile is done with the stage
         return true;
       };
-      bool ok = mbar_wait_bounded(&bar_q, 0);
-      if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
+      bool ok = mbar_wait_bounded(&bar_q, 0) && issue_s(0);
       for (int j = 0; ok && j < ntiles; ++j) {
-        if (j + 1 < ntiles) {
-          // the next scores of each Q tile once its softmax has read S(j)
-          ok = mbar_wait_bounded(&s_free[0], j & 1) && issue_s(0, j + 1);
-          ok = ok && mbar_wait_bounded(&s_free[1], j & 1) && issue_s(1, j + 1);
-        }
-        ok = ok && issue_pv(0, j) && issue_pv(1, j);
-        if (ok) umma_commit(&kv_empty[j % ST]);
+        // the next scores once the softmax has read S(j), then P(j) V(j)
+        if (j + 1 < ntiles) ok = mbar_wait_bounded(&s_free[qt], j & 1) && issue_s(j + 1);
+        ok = ok && issue_pv(j);
         if (s_abort) break;
       }
       if (!ok) give_up();
@@ -287,7 +285,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tmem_ld32_nowait(tmem_s + 32, sr + 32);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&s_free[qt]);  // S may be overwritten by the next tile's scores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[qt]);  // S may be overwritten by the next tile's scores
       float x[kPfBN];
       float tmax = -INFINITY;
       if (tfull[st][qt]) {
@@ -353,7 +352,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
       fence_proxy_async();  // P visible to the tensor cores
       tc_fence_before();
-      mbar_arrive(&p_full[qt]);
+      __syncwarp();  // the warp's P rows and O rescale precede lane 0's release
+      if (lane == 0) mbar_arrive(&p_full[qt]);
       if (s_abort) {
         ok = false;
         break;
