@@ -244,6 +244,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Bounded wait that parks the warp: each try may suspend the thread for up to
+// 20 us until the phase completes, so waiting warps leave their issue slots to
+// the others; gives up (returns false) after about 2.6 s.
+__device__ __forceinline__ bool mbar_wait_parked(uint64_t* bar, uint32_t parity) {
+  for (int i = 0; i < (1 << 17); ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
 // Bounded wait: returns false (and the caller must give up) after kSpinLimit tries.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
   for (long long i = 0; i < kSpinLimit; ++i)

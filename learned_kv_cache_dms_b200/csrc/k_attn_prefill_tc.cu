@@ -35,6 +35,19 @@ namespace dms {
 
 #ifdef DMS_TRACE
 __device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
+// per-tile marks of the first CTA of the grid (row = tile), by one thread
+#define PF_MARK(tile, slot)                                                                          \
+  do {                                                                                               \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (tile) < kTraceCtas) {              \
+      unsigned long long t_;                                                                         \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                         \
+      g_dms_trace[static_cast<long>(tile) * kTraceSlots + (slot)] = t_;                              \
+    }                                                                                                \
+  } while (0)
+#else
+#define PF_MARK(tile, slot) \
+  do {                      \
+  } while (0)
 #endif
 
 constexpr int kPfRows = 128;     // query rows per Q tile (TMEM lanes)
@@ -66,9 +79,20 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Named barriers among the two softmax warpgroups (ids 1, 2; 0 is
+// __syncthreads): arrive without waiting, or wait for `count` arrivals.
+template <int ID>
+__device__ __forceinline__ void named_arrive() {
+  asm volatile("bar.arrive %0, %1;\n" ::"n"(ID), "n"(2 * kPfRows) : "memory");
+}
+template <int ID>
+__device__ __forceinline__ void named_sync() {
+  asm volatile("bar.sync %0, %1;\n" ::"n"(ID), "n"(2 * kPfRows) : "memory");
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
-  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));  // stays between the turn barriers
   return y;
 }
 
@@ -110,6 +134,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   __shared__ __align__(8) uint64_t bar_q, k_full[ST], v_full[ST], kv_empty[ST];
   __shared__ __align__(8) uint64_t s_full[kPfQT], s_free[kPfQT], p_full[kPfQT], pv_done[kPfQT];
   __shared__ int s_abort;
+  // anchors of the exponentials' turn: a zero read after the turn begins and
+  // every row's sum written before it ends (a barrier orders memory accesses
+  // only, so the exponentials are tied to it through these)
+  __shared__ float s_turn_zero;
+  __shared__ float s_turn_sum[kPfQT][kPfRows];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = c.Hq / c.Hkv, NP = kPfRows / g;
@@ -139,6 +168,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     fence_mbar_init();
     s_abort = 0;
+    s_turn_zero = 0.f;
   }
   if (warp == kPfMmaWarp) tmem_alloc(&tmem_base, L::TMEM_COLS);
   tc_fence_before();
@@ -163,7 +193,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int st = j % ST, use = j / ST;
       if (use > 0) {
         bool ok = true;
-        if (lane == 0) ok = mbar_wait_bounded(&kv_empty[st], (use - 1) & 1);
+        if (lane == 0) ok = mbar_wait_parked(&kv_empty[st], (use - 1) & 1);
         if (!__shfl_sync(0xffffffffu, ok, 0)) {
           if (lane == 0) give_up();
           break;
@@ -224,7 +254,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       constexpr uint32_t IDESC_O = umma_idesc_bf16(kPfRows, D, 1);
       auto issue_s = [&](int j) -> bool {
         const int st = j % ST;
+        PF_MARK(j, 16 * qt + 8);
         if (!mbar_wait_bounded(&k_full[st], (j / ST) & 1)) return false;
+        PF_MARK(j, 16 * qt + 9);
         tc_fence_after();
         const uint32_t qa = smem_u32(sb + L::OFF_Q + qt * L::Q_BYTES);
         const uint32_t ka = smem_u32(sb + L::OFF_K + st * L::KV_BYTES);
@@ -241,7 +273,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       auto issue_pv = [&](int j) -> bool {
         const int st = j % ST;
         if (!mbar_wait_bounded(&v_full[st], (j / ST) & 1)) return false;
+        PF_MARK(j, 16 * qt + 10);
         if (!mbar_wait_bounded(&p_full[qt], j & 1)) return false;
+        PF_MARK(j, 16 * qt + 11);
         tc_fence_after();
         const uint32_t pa = smem_u32(sb + L::OFF_P + qt * L::P_BYTES);
         const uint32_t va = smem_u32(sb + L::OFF_V + st * L::KV_BYTES);
@@ -273,28 +307,37 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
     float m_ref = -INFINITY, l_row = 0.f;
     bool ok = true;
+    // The two warpgroups take turns for the exponentials (named barrier 1:
+    // WG1 may start, 2: WG0 may start; bar.arrive by the group that finishes,
+    // bar.sync by the one that waits), so one group's exponentials overlap the
+    // other group's tensor-core work and bookkeeping.  Every barrier step runs
+    // even after a failed wait, so neither group can be left waiting.
     for (int j = 0; j < ntiles; ++j) {
       const int st = j % ST;
       const bool kt = j < nkt;
+      if (row == 0) PF_MARK(j, 16 * qt + 0);
       // the tile's key positions (published with the loads) and its scores
-      ok = mbar_wait_bounded(&k_full[st], (j / ST) & 1) && mbar_wait_bounded(&s_full[qt], j & 1);
-      if (!ok) break;
+      ok = ok && mbar_wait_bounded(&k_full[st], (j / ST) & 1) && mbar_wait_bounded(&s_full[qt], j & 1);
+      if (row == 0) PF_MARK(j, 16 * qt + 1);
       tc_fence_after();
       uint32_t sr[kPfBN];
-      tmem_ld32_nowait(tmem_s, sr);
-      tmem_ld32_nowait(tmem_s + 32, sr + 32);
-      tmem_wait_ld();
+      if (ok) {
+        tmem_ld32_nowait(tmem_s, sr);
+        tmem_ld32_nowait(tmem_s + 32, sr + 32);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int n = 0; n < kPfBN; ++n) sr[n] = 0u;
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[qt]);  // S may be overwritten by the next tile's scores
-      float x[kPfBN];
-      float tmax = -INFINITY;
+      if (ok && lane == 0) mbar_arrive(&s_free[qt]);  // S may be overwritten by the next tile's scores
+      if (row == 0) PF_MARK(j, 16 * qt + 2);
+      // raw scores with the invisible ones at -inf; row max over 4 chains
+      float sv[kPfBN];
       if (tfull[st][qt]) {
 #pragma unroll
-        for (int n = 0; n < kPfBN; ++n) {
-          x[n] = __uint_as_float(sr[n]) * sl2;
-          tmax = fmaxf(tmax, x[n]);
-        }
+        for (int n = 0; n < kPfBN; ++n) sv[n] = __uint_as_float(sr[n]);
       } else {
         // visible: lo <= j <= hi (kept: 0 <= j <= i - w; band: i - w < j <= i); absent keys are -1
         const int lo = kt ? 0 : max(0, i_row - w + 1);
@@ -304,13 +347,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const int4 jv = reinterpret_cast<const int4*>(kpos[st])[n4];
           const int js[4] = {jv.x, jv.y, jv.z, jv.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int n = n4 * 4 + e;
-            x[n] = (js[e] >= lo && js[e] <= hi) ? __uint_as_float(sr[n]) * sl2 : -INFINITY;
-            tmax = fmaxf(tmax, x[n]);
-          }
+          for (int e = 0; e < 4; ++e)
+            sv[n4 * 4 + e] = (js[e] >= lo && js[e] <= hi) ? __uint_as_float(sr[n4 * 4 + e]) : -INFINITY;
         }
       }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int n = 0; n < kPfBN; ++n) mx4[n & 3] = fmaxf(mx4[n & 3], sv[n]);
+      const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
       // raise the reference only when this tile exceeds it by more than 2^8
       const bool raise = tmax > m_ref + 8.0f;
       float factor = 1.0f;
@@ -320,23 +364,41 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         l_row *= factor;
       }
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a fully masked row so far: all p = 0
+      if (row == 0) PF_MARK(j, 16 * qt + 6);
+      if (qt == 0) {
+        if (j > 0) named_sync<2>();
+      } else {
+        named_sync<1>();
+      }
+      if (row == 0) PF_MARK(j, 16 * qt + 7);
+      const float neg_m = *reinterpret_cast<volatile float*>(&s_turn_zero) - m_use;
       uint32_t pk[kPfBN / 2];
-      float psum = 0.f;
+      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < kPfBN / 2; ++e) {
-        const float p0 = ex2_approx(x[2 * e] - m_use);
-        const float p1 = ex2_approx(x[2 * e + 1] - m_use);
-        psum += p0 + p1;
+        const float p0 = ex2_approx(fmaf(sv[2 * e], sl2, neg_m));
+        const float p1 = ex2_approx(fmaf(sv[2 * e + 1], sl2, neg_m));
+        ps4[e & 3] += p0 + p1;
         pk[e] = pack_bf16(p0, p1);
       }
-      l_row += psum;
-      // P V of the previous tile has finished with P and with O
-      if (j > 0 && !mbar_wait_bounded(&pv_done[qt], (j - 1) & 1)) {
-        ok = false;
-        break;
+      const float psum = (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+      *reinterpret_cast<volatile float*>(&s_turn_sum[qt][row]) = psum;
+      // the turn ends once every exponential is done: the arrive is control
+      // dependent on their sum (the condition always holds: psum is a sum of
+      // non-negative terms, never this negative NaN pattern)
+      if (__float_as_uint(psum) != 0xFFFFFFFFu) {
+        if (qt == 0)
+          named_arrive<1>();
+        else
+          named_arrive<2>();
       }
+      l_row += psum;
+      if (row == 0) PF_MARK(j, 16 * qt + 3);
+      // P V of the previous tile has finished with P and with O
+      if (j > 0) ok = ok && mbar_wait_bounded(&pv_done[qt], (j - 1) & 1);
       tc_fence_after();
-      if (j > 0 && __any_sync(0xffffffffu, raise && factor != 1.0f)) {
+      if (row == 0) PF_MARK(j, 16 * qt + 4);
+      if (ok && j > 0 && __any_sync(0xffffffffu, raise && factor != 1.0f)) {
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           float ov[32];
@@ -353,12 +415,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       fence_proxy_async();  // P visible to the tensor cores
       tc_fence_before();
       __syncwarp();  // the warp's P rows and O rescale precede lane 0's release
-      if (lane == 0) mbar_arrive(&p_full[qt]);
-      if (s_abort) {
-        ok = false;
-        break;
-      }
+      if (ok && lane == 0) mbar_arrive(&p_full[qt]);
+      if (row == 0) PF_MARK(j, 16 * qt + 5);
+      if (s_abort) ok = false;
     }
+    if (qt == 0 && ntiles > 0) named_sync<2>();  // WG1's last hand-back
     // the last P V, then O / l
     if (ok && ntiles > 0) ok = mbar_wait_bounded(&pv_done[qt], (ntiles - 1) & 1);
     if (!ok) {
