@@ -12,17 +12,21 @@
 // contiguous band [i0 - w + 1, i1 - 1] of the CTA's 2 NP positions and from
 // the position-sorted kept list; evicted keys outside the window are never
 // loaded.  Warp roles:
-//   load warp  : TMA (no multicast) of the Q tiles, then K and V of every key
-//                tile into a ring of stages (band tiles straight from the
-//                input rows, kept tiles from the kept copy written by the
+//   K loader   : TMA (no multicast) of the Q tiles, then K of every key tile
+//                into a ring of stages (band tiles straight from the input
+//                rows, kept tiles from the kept copy written by the
 //                compaction), with the tile's key positions and, per Q tile,
-//                whether every row sees every key (no mask needed);
+//                whether every row sees every key (no mask needed); a K stage
+//                is free again once both Q tiles' scores are computed;
+//   V loader   : V of every key tile into its own ring, free again once both
+//                Q tiles' P V are done;
 //   MMA warps  : one per Q tile w: S_w = Q_w K^T (tcgen05.mma M=128, N=64,
 //                K=16 x D/16, both K-major in 128-byte-swizzled shared memory,
-//                S_w in TMEM) and O_w += P_w V (P_w K-major from shared memory,
-//                V MN-major, O_w in TMEM), in the order S_w(t+1), PV_w(t): each
-//                Q tile's next scores run on the tensor cores while its softmax
-//                of tile t runs, and the two Q tiles proceed independently;
+//                S_w in TMEM) and O_w += P_w V (P_w in TMEM as bf16, V
+//                MN-major in shared memory, O_w in TMEM), in the order
+//                S_w(t+1), PV_w(t): each Q tile's next scores run on the tensor
+//                cores while its softmax of tile t runs, and the two Q tiles
+//                proceed independently;
 //   softmax    : one warpgroup per Q tile, one thread per row; the exponent
 //                reference of a row is raised only when a tile's max exceeds
 //                it by 2^8, so O is rescaled rarely (O / l is exact either
@@ -55,29 +59,26 @@ constexpr int kPfQT = 2;         // Q tiles per CTA
 constexpr int kPfBN = 64;        // keys per K/V tile
 constexpr int kPfMmaWarp = 8;    // warps 0-3: softmax of Q tile 0, 4-7: Q tile 1; 8, 9: MMA issue for
                                  // Q tile 0, 1
-constexpr int kPfLoadWarp = 10;
-constexpr int kPfThreads = 352;
+constexpr int kPfLoadWarp = 10;  // 10: Q and K loads, 11: V loads
+constexpr int kPfThreads = 384;
 
 template <int D>
 struct PfSmem {
   static constexpr int HALVES = D / 64;
   static constexpr int Q_BYTES = HALVES * kPfRows * 128;  // one Q tile: [half][128 rows][128 B]
   static constexpr int KV_BYTES = HALVES * kPfBN * 128;   // K (or V) of one key tile: [half][64 keys][128 B]
-  static constexpr int P_BYTES = kPfRows * 128;           // one P tile: [128 rows][64 keys x 2 B]
-  static constexpr int ST = D == 64 ? 4 : 3;              // K/V stages
+  static constexpr int ST = D == 64 ? 8 : 4;              // K stages, V stages
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_P = OFF_Q + kPfQT * Q_BYTES;
-  static constexpr int OFF_K = OFF_P + kPfQT * P_BYTES;
+  static constexpr int OFF_K = OFF_Q + kPfQT * Q_BYTES;
   static constexpr int OFF_V = OFF_K + ST * KV_BYTES;
   static constexpr int BYTES = OFF_V + ST * KV_BYTES;
-  // tensor memory: S0, S1 (64 columns each), O0, O1 (D columns each)
+  // tensor memory: S0, S1 (64 fp32 columns each), O0, O1 (D columns each),
+  // P0, P1 (64 bf16 = 32 columns each)
   static constexpr uint32_t COL_O = 2 * kPfBN;
-  static constexpr uint32_t TMEM_COLS = COL_O + 2 * D <= 256 ? 256 : 512;
+  static constexpr uint32_t COL_P = COL_O + 2 * D;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(COL_P + kPfQT * kPfBN / 2 <= TMEM_COLS, "tensor memory columns");
 };
-
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
 
 // Named barriers among the two softmax warpgroups (ids 1, 2; 0 is
 // __syncthreads): arrive without waiting, or wait for `count` arrivals.
@@ -128,10 +129,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   constexpr int ST = L::ST;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sb = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(16) int kpos[ST][kPfBN];  // key positions of the tile in each stage (-1: absent)
-  __shared__ int tfull[ST][kPfQT];              // 1: every row of that Q tile sees every key of the tile
+  // key positions of tile t (-1: absent) and, per Q tile, 1 when every row
+  // sees every key; slot t % 2ST, published by kp_full (a K stage is reused
+  // while the softmax may still read the positions of its previous tile)
+  __shared__ __align__(16) int kpos[2 * ST][kPfBN];
+  __shared__ int tfull[2 * ST][kPfQT];
   __shared__ uint32_t tmem_base;
-  __shared__ __align__(8) uint64_t bar_q, k_full[ST], v_full[ST], kv_empty[ST];
+  __shared__ __align__(8) uint64_t bar_q, k_full[ST], v_full[ST], k_empty[ST], v_empty[ST], kp_full[2 * ST];
   __shared__ __align__(8) uint64_t s_full[kPfQT], s_free[kPfQT], p_full[kPfQT], pv_done[kPfQT];
   __shared__ int s_abort;
   // anchors of the exponentials' turn: a zero read after the turn begins and
@@ -158,8 +162,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int i = 0; i < ST; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], kPfQT);  // both Q tiles' P V done with the stage
+      mbar_init(&k_empty[i], kPfQT);  // both Q tiles' scores done with the K stage
+      mbar_init(&v_empty[i], kPfQT);  // both Q tiles' P V done with the V stage
     }
+    for (int i = 0; i < 2 * ST; ++i) mbar_init(&kp_full[i], 1);
     for (int i = 0; i < kPfQT; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);  // one arrival per softmax warp
@@ -181,7 +187,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   };
 
   if (warp == kPfLoadWarp) {
-    // ---- loads ---------------------------------------------------------
+    // ---- Q, then K of every key tile with its positions ------------------
     if (lane == 0) {
       mbar_expect_tx(&bar_q, kPfQT * L::Q_BYTES);
       for (int qt = 0; qt < kPfQT; ++qt)
@@ -190,42 +196,32 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                       b * T + i0 + qt * NP, &bar_q);
     }
     for (int j = 0; j < ntiles; ++j) {
-      const int st = j % ST, use = j / ST;
+      const int st = j % ST, use = j / ST, kp = j % (2 * ST);
+      // key positions, two per lane (the kept-list reads overlap the wait)
+      const bool kt = j < nkt;
+      const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
+      int p[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int kk = lane + 32 * e;
+        if (kt)
+          p[e] = jb + kk < nk ? kept[jb + kk] : -1;
+        else
+          p[e] = jb + kk <= jhi ? jb + kk : -1;
+      }
       if (use > 0) {
         bool ok = true;
-        if (lane == 0) ok = mbar_wait_parked(&kv_empty[st], (use - 1) & 1);
+        if (lane == 0) ok = mbar_wait_parked(&k_empty[st], (use - 1) & 1);
         if (!__shfl_sync(0xffffffffu, ok, 0)) {
           if (lane == 0) give_up();
           break;
         }
       }
-      // key positions: two per lane
-      const bool kt = j < nkt;
-      const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int kk = lane + 32 * e;
-        int p;
-        if (kt) {
-          p = jb + kk < nk ? kept[jb + kk] : -1;
-        } else {
-          p = jb + kk <= jhi ? jb + kk : -1;
-        }
-        kpos[st][kk] = p;
-      }
+      if (lane == 0) PF_MARK(j, 12);
+      kpos[kp][lane] = p[0];
+      kpos[kp][lane + 32] = p[1];
       __syncwarp();
       if (lane == 0) {
-        // mask-free for Q tile qt: every key present and visible to all of
-        // its rows [qmin, qmax] (kept: j <= i - w; band: i - w < j <= i)
-        for (int qt = 0; qt < kPfQT; ++qt) {
-          const int qmin = i0 + qt * NP, qmax = min(T, qmin + NP) - 1;
-          int full;
-          if (kt)
-            full = (jb + kPfBN <= nk) && kpos[st][kPfBN - 1] <= qmin - w;
-          else
-            full = (jb + kPfBN - 1 <= jhi) && jb > qmax - w && jb + kPfBN - 1 <= qmin;
-          tfull[st][qt] = full;
-        }
         mbar_expect_tx(&k_full[st], L::KV_BYTES);
         for (int hf = 0; hf < L::HALVES; ++hf) {
           unsigned char* dk = sb + L::OFF_K + st * L::KV_BYTES + hf * (kPfBN * 128);
@@ -234,13 +230,41 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           else
             tma_load_3d(dk, &kmap, hf * 64, h, b * T + jb, &k_full[st]);
         }
-        mbar_expect_tx(&v_full[st], L::KV_BYTES);
-        for (int hf = 0; hf < L::HALVES; ++hf) {
-          unsigned char* dv = sb + L::OFF_V + st * L::KV_BYTES + hf * (kPfBN * 128);
+        // mask-free for Q tile qt: every key present and visible to all of
+        // its rows [qmin, qmax] (kept: j <= i - w; band: i - w < j <= i)
+        for (int qt = 0; qt < kPfQT; ++qt) {
+          const int qmin = i0 + qt * NP, qmax = min(T, qmin + NP) - 1;
+          int full;
           if (kt)
-            tma_load_2d(dv, &kvmap, hf * 64, bh * c.max_pos + jb, &v_full[st]);
+            full = (jb + kPfBN <= nk) && kpos[kp][kPfBN - 1] <= qmin - w;
           else
-            tma_load_3d(dv, &vmap, hf * 64, h, b * T + jb, &v_full[st]);
+            full = (jb + kPfBN - 1 <= jhi) && jb > qmax - w && jb + kPfBN - 1 <= qmin;
+          tfull[kp][qt] = full;
+        }
+        mbar_arrive(&kp_full[kp]);
+        PF_MARK(j, 13);
+      }
+      __syncwarp();
+      if (s_abort) break;
+    }
+  } else if (warp == kPfLoadWarp + 1) {
+    // ---- V of every key tile -------------------------------------------
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j % ST, use = j / ST;
+      if (lane == 0) {
+        if (use > 0 && !mbar_wait_parked(&v_empty[st], (use - 1) & 1)) {
+          give_up();
+        } else {
+          const bool kt = j < nkt;
+          const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
+          mbar_expect_tx(&v_full[st], L::KV_BYTES);
+          for (int hf = 0; hf < L::HALVES; ++hf) {
+            unsigned char* dv = sb + L::OFF_V + st * L::KV_BYTES + hf * (kPfBN * 128);
+            if (kt)
+              tma_load_2d(dv, &kvmap, hf * 64, bh * c.max_pos + jb, &v_full[st]);
+            else
+              tma_load_3d(dv, &vmap, hf * 64, h, b * T + jb, &v_full[st]);
+          }
         }
       }
       __syncwarp();
@@ -268,6 +292,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     IDESC_S, ks > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[qt]);
+        umma_commit(&k_empty[st]);  // this Q tile is done with the K stage
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
@@ -277,14 +302,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!mbar_wait_bounded(&p_full[qt], j & 1)) return false;
         PF_MARK(j, 16 * qt + 11);
         tc_fence_after();
-        const uint32_t pa = smem_u32(sb + L::OFF_P + qt * L::P_BYTES);
         const uint32_t va = smem_u32(sb + L::OFF_V + st * L::KV_BYTES);
 #pragma unroll
         for (int ks = 0; ks < kPfBN / 16; ++ks)
-          umma_bf16(tmem + L::COL_O + qt * D, umma_desc_sw128(pa + ks * 32, 16, 1024),
-                    umma_desc_sw128(va + ks * 16 * 128, kPfBN * 128, 1024), IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + L::COL_O + qt * D, tmem + L::COL_P + qt * (kPfBN / 2) + ks * 8,
+                       umma_desc_sw128(va + ks * 16 * 128, kPfBN * 128, 1024), IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
         umma_commit(&pv_done[qt]);
-        umma_commit(&kv_empty[st]);  // this Q tile is done with the stage
+        umma_commit(&v_empty[st]);  // this Q tile is done with the V stage
         return true;
       };
       bool ok = mbar_wait_bounded(&bar_q, 0) && issue_s(0);
@@ -302,7 +326,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tmem_s = tmem + lane_off + qt * kPfBN;
     const uint32_t tmem_o = tmem + lane_off + L::COL_O + qt * D;
-    unsigned char* sP = sb + L::OFF_P + qt * L::P_BYTES;
+    const uint32_t tmem_p = tmem + lane_off + L::COL_P + qt * (kPfBN / 2);
     const int i_row = i0 + qt * NP + row / g, r_row = row % g;
     const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
     float m_ref = -INFINITY, l_row = 0.f;
@@ -313,11 +337,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // other group's tensor-core work and bookkeeping.  Every barrier step runs
     // even after a failed wait, so neither group can be left waiting.
     for (int j = 0; j < ntiles; ++j) {
-      const int st = j % ST;
+      const int kp = j % (2 * ST);
       const bool kt = j < nkt;
       if (row == 0) PF_MARK(j, 16 * qt + 0);
-      // the tile's key positions (published with the loads) and its scores
-      ok = ok && mbar_wait_bounded(&k_full[st], (j / ST) & 1) && mbar_wait_bounded(&s_full[qt], j & 1);
+      // the tile's key positions and its scores
+      ok = ok && mbar_wait_bounded(&kp_full[kp], (j / (2 * ST)) & 1) && mbar_wait_bounded(&s_full[qt], j & 1);
       if (row == 0) PF_MARK(j, 16 * qt + 1);
       tc_fence_after();
       uint32_t sr[kPfBN];
@@ -335,7 +359,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (row == 0) PF_MARK(j, 16 * qt + 2);
       // raw scores with the invisible ones at -inf; row max over 4 chains
       float sv[kPfBN];
-      if (tfull[st][qt]) {
+      if (tfull[kp][qt]) {
 #pragma unroll
         for (int n = 0; n < kPfBN; ++n) sv[n] = __uint_as_float(sr[n]);
       } else {
@@ -344,7 +368,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int hi = kt ? i_row - w : i_row;
 #pragma unroll
         for (int n4 = 0; n4 < kPfBN / 4; ++n4) {
-          const int4 jv = reinterpret_cast<const int4*>(kpos[st])[n4];
+          const int4 jv = reinterpret_cast<const int4*>(kpos[kp])[n4];
           const int js[4] = {jv.x, jv.y, jv.z, jv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e)
@@ -408,11 +432,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tmem_st32(tmem_o + c0, ov);
         }
       }
-#pragma unroll
-      for (int ch = 0; ch < kPfBN / 8; ++ch)
-        *reinterpret_cast<uint4*>(sP + swz(row, ch)) =
-            make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-      fence_proxy_async();  // P visible to the tensor cores
+      tmem_st32_nowait(tmem_p, pk);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();  // the warp's P rows and O rescale precede lane 0's release
       if (ok && lane == 0) mbar_arrive(&p_full[qt]);
