@@ -15,9 +15,8 @@
 //   K loader   : TMA (no multicast) of the Q tiles, then K of every key tile
 //                into a ring of stages (band tiles straight from the input
 //                rows, kept tiles from the kept copy written by the
-//                compaction), with the tile's key positions and, per Q tile,
-//                whether every row sees every key (no mask needed); a K stage
-//                is free again once both Q tiles' scores are computed;
+//                compaction); a K stage is free again once both Q tiles'
+//                scores are computed;
 //   V loader   : V of every key tile into its own ring, free again once both
 //                Q tiles' P V are done;
 //   MMA warps  : one per Q tile w: S_w = Q_w K^T (tcgen05.mma M=128, N=64,
@@ -27,7 +26,11 @@
 //                S_w(t+1), PV_w(t): each Q tile's next scores run on the tensor
 //                cores while its softmax of tile t runs, and the two Q tiles
 //                proceed independently;
-//   softmax    : one warpgroup per Q tile, one thread per row; the exponent
+//   softmax    : one warpgroup per Q tile, one thread per row; a row's
+//                visible keys in a tile are one column range (the band is
+//                contiguous in position; the kept list is position-sorted, so
+//                the keys at or before i - w are its first kept_upto(i-w+1)
+//                entries), applied as a bit mask; the exponent
 //                reference of a row is raised only when a tile's max exceeds
 //                it by 2^8, so O is rescaled rarely (O / l is exact either
 //                way).
@@ -97,6 +100,58 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+#ifndef DMS_PF_POLY_PAIRS
+#define DMS_PF_POLY_PAIRS 0  // of every 8 pairs of exponentials, how many run on the FMA pipe
+#endif
+#ifndef DMS_PF_PACK_INT
+#define DMS_PF_PACK_INT 0
+#endif
+
+// 2^x on the FMA pipe: x = j + f with j = round(x), |f| <= 1/2 (the 1.5 * 2^23
+// shifter leaves j in the low mantissa bits), 2^f from a cubic fitted to it on
+// [-1/2, 1/2] (relative error 7.5e-5, below P's bf16 rounding), 2^j added to
+// the exponent field.  x is clamped to -125 so the result stays a normal
+// float (invisible scores, -inf, give 2^-125, below anything a visible key
+// contributes to a row sum of at least 1).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
+  const float p = fmaf(fmaf(fmaf(0.0551716611f, f, 0.24261114f), f, 0.693260968f), f, 0.999928057f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// two non-negative finite floats to bf16 (round half away from zero) with
+// integer operations: a's high half in the low 16 bits, b's in the high
+__device__ __forceinline__ uint32_t pack_bf16_pos(float a, float b) {
+  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
+}
+
+// paired fp32 arithmetic (one instruction for two lanes of a 64-bit pair)
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 32 consecutive fp32 columns of this thread's TMEM lane, without waiting.
 __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t* r) {
   asm volatile(
@@ -129,13 +184,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   constexpr int ST = L::ST;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sb = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // key positions of tile t (-1: absent) and, per Q tile, 1 when every row
-  // sees every key; slot t % 2ST, published by kp_full (a K stage is reused
-  // while the softmax may still read the positions of its previous tile)
-  __shared__ __align__(16) int kpos[2 * ST][kPfBN];
-  __shared__ int tfull[2 * ST][kPfQT];
   __shared__ uint32_t tmem_base;
-  __shared__ __align__(8) uint64_t bar_q, k_full[ST], v_full[ST], k_empty[ST], v_empty[ST], kp_full[2 * ST];
+  __shared__ __align__(8) uint64_t bar_q, k_full[ST], v_full[ST], k_empty[ST], v_empty[ST];
   __shared__ __align__(8) uint64_t s_full[kPfQT], s_free[kPfQT], p_full[kPfQT], pv_done[kPfQT];
   __shared__ int s_abort;
   // anchors of the exponentials' turn: a zero read after the turn begins and
@@ -151,7 +201,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int h = blockIdx.y, b = blockIdx.z, w = c.w;
   const int i0 = blk * kPfQT * NP, i1 = min(T, i0 + kPfQT * NP);
   const int bh = b * c.Hkv + h;
-  const int* kept = c.kept + static_cast<long>(bh) * c.max_pos;
   const int nk = (i1 - w > 0) ? c.kept_upto[static_cast<long>(bh) * (c.max_pos + 1) + (i1 - w)] : 0;
   const int jlo = max(0, i0 - w + 1), jhi = i1 - 1;
   const int nkt = (nk + kPfBN - 1) / kPfBN;  // kept tiles
@@ -165,7 +214,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&k_empty[i], kPfQT);  // both Q tiles' scores done with the K stage
       mbar_init(&v_empty[i], kPfQT);  // both Q tiles' P V done with the V stage
     }
-    for (int i = 0; i < 2 * ST; ++i) mbar_init(&kp_full[i], 1);
     for (int i = 0; i < kPfQT; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);  // one arrival per softmax warp
@@ -196,53 +244,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                       b * T + i0 + qt * NP, &bar_q);
     }
     for (int j = 0; j < ntiles; ++j) {
-      const int st = j % ST, use = j / ST, kp = j % (2 * ST);
-      // key positions, two per lane (the kept-list reads overlap the wait)
-      const bool kt = j < nkt;
-      const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
-      int p[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int kk = lane + 32 * e;
-        if (kt)
-          p[e] = jb + kk < nk ? kept[jb + kk] : -1;
-        else
-          p[e] = jb + kk <= jhi ? jb + kk : -1;
-      }
-      if (use > 0) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait_parked(&k_empty[st], (use - 1) & 1);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) {
-          if (lane == 0) give_up();
-          break;
-        }
-      }
-      if (lane == 0) PF_MARK(j, 12);
-      kpos[kp][lane] = p[0];
-      kpos[kp][lane + 32] = p[1];
-      __syncwarp();
+      const int st = j % ST, use = j / ST;
       if (lane == 0) {
-        mbar_expect_tx(&k_full[st], L::KV_BYTES);
-        for (int hf = 0; hf < L::HALVES; ++hf) {
-          unsigned char* dk = sb + L::OFF_K + st * L::KV_BYTES + hf * (kPfBN * 128);
-          if (kt)
-            tma_load_2d(dk, &kkmap, hf * 64, bh * c.max_pos + jb, &k_full[st]);
-          else
-            tma_load_3d(dk, &kmap, hf * 64, h, b * T + jb, &k_full[st]);
+        if (use > 0 && !mbar_wait_parked(&k_empty[st], (use - 1) & 1)) {
+          give_up();
+        } else {
+          PF_MARK(j, 12);
+          const bool kt = j < nkt;
+          const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
+          mbar_expect_tx(&k_full[st], L::KV_BYTES);
+          for (int hf = 0; hf < L::HALVES; ++hf) {
+            unsigned char* dk = sb + L::OFF_K + st * L::KV_BYTES + hf * (kPfBN * 128);
+            if (kt)
+              tma_load_2d(dk, &kkmap, hf * 64, bh * c.max_pos + jb, &k_full[st]);
+            else
+              tma_load_3d(dk, &kmap, hf * 64, h, b * T + jb, &k_full[st]);
+          }
+          PF_MARK(j, 13);
         }
-        // mask-free for Q tile qt: every key present and visible to all of
-        // its rows [qmin, qmax] (kept: j <= i - w; band: i - w < j <= i)
-        for (int qt = 0; qt < kPfQT; ++qt) {
-          const int qmin = i0 + qt * NP, qmax = min(T, qmin + NP) - 1;
-          int full;
-          if (kt)
-            full = (jb + kPfBN <= nk) && kpos[kp][kPfBN - 1] <= qmin - w;
-          else
-            full = (jb + kPfBN - 1 <= jhi) && jb > qmax - w && jb + kPfBN - 1 <= qmin;
-          tfull[kp][qt] = full;
-        }
-        mbar_arrive(&kp_full[kp]);
-        PF_MARK(j, 13);
       }
       __syncwarp();
       if (s_abort) break;
@@ -329,6 +348,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t tmem_p = tmem + lane_off + L::COL_P + qt * (kPfBN / 2);
     const int i_row = i0 + qt * NP + row / g, r_row = row % g;
     const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    // the row's visible keys: kept-list entries [0, ck) (positions <= i - w)
+    // and band positions [blo, bhi]
+    const int ck_at = min(i_row - w + 1, T);
+    const int ck = ck_at > 0 ? c.kept_upto[static_cast<long>(bh) * (c.max_pos + 1) + ck_at] : 0;
+    const int blo = max(0, i_row - w + 1), bhi = min(i_row, jhi);
     float m_ref = -INFINITY, l_row = 0.f;
     bool ok = true;
     // The two warpgroups take turns for the exponentials (named barrier 1:
@@ -337,11 +362,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // other group's tensor-core work and bookkeeping.  Every barrier step runs
     // even after a failed wait, so neither group can be left waiting.
     for (int j = 0; j < ntiles; ++j) {
-      const int kp = j % (2 * ST);
+      // visible columns [c_lo, c_hi] of this tile for the row
       const bool kt = j < nkt;
+      const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
+      const int c_lo = max(kt ? 0 : blo - jb, 0), c_hi = min(kt ? ck - 1 - jb : bhi - jb, kPfBN - 1);
+      const bool row_full = c_lo == 0 && c_hi == kPfBN - 1;
       if (row == 0) PF_MARK(j, 16 * qt + 0);
-      // the tile's key positions and its scores
-      ok = ok && mbar_wait_bounded(&kp_full[kp], (j / (2 * ST)) & 1) && mbar_wait_bounded(&s_full[qt], j & 1);
+      ok = ok && mbar_wait_bounded(&s_full[qt], j & 1);
       if (row == 0) PF_MARK(j, 16 * qt + 1);
       tc_fence_after();
       uint32_t sr[kPfBN];
@@ -359,25 +386,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (row == 0) PF_MARK(j, 16 * qt + 2);
       // raw scores with the invisible ones at -inf; row max over 4 chains
       float sv[kPfBN];
-      if (tfull[kp][qt]) {
+      if (__all_sync(0xffffffffu, row_full)) {
 #pragma unroll
         for (int n = 0; n < kPfBN; ++n) sv[n] = __uint_as_float(sr[n]);
       } else {
-        // visible: lo <= j <= hi (kept: 0 <= j <= i - w; band: i - w < j <= i); absent keys are -1
-        const int lo = kt ? 0 : max(0, i_row - w + 1);
-        const int hi = kt ? i_row - w : i_row;
-#pragma unroll
-        for (int n4 = 0; n4 < kPfBN / 4; ++n4) {
-          const int4 jv = reinterpret_cast<const int4*>(kpos[kp])[n4];
-          const int js[4] = {jv.x, jv.y, jv.z, jv.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            sv[n4 * 4 + e] = (js[e] >= lo && js[e] <= hi) ? __uint_as_float(sr[n4 * 4 + e]) : -INFINITY;
+        // bits c_lo..c_hi (none when the range is empty)
+        uint32_t m0 = 0u, m1 = 0u;
+        if (c_lo <= c_hi) {
+          const unsigned long long m = (~0ull >> (kPfBN - 1 - (c_hi - c_lo))) << c_lo;
+          m0 = static_cast<uint32_t>(m);
+          m1 = static_cast<uint32_t>(m >> 32);
         }
+#pragma unroll
+        for (int n = 0; n < kPfBN; ++n)
+          sv[n] = (((n < 32 ? m0 : m1) >> (n & 31)) & 1u) ? __uint_as_float(sr[n]) : -INFINITY;
       }
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int n = 0; n < kPfBN; ++n) mx4[n & 3] = fmaxf(mx4[n & 3], sv[n]);
+      for (int n = 0; n < kPfBN; n += 2) mx4[(n >> 1) & 3] = fmax3(mx4[(n >> 1) & 3], sv[n], sv[n + 1]);
       const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
       // raise the reference only when this tile exceeds it by more than 2^8
       const bool raise = tmax > m_ref + 8.0f;
@@ -396,16 +422,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       if (row == 0) PF_MARK(j, 16 * qt + 7);
       const float neg_m = *reinterpret_cast<volatile float*>(&s_turn_zero) - m_use;
+      const uint64_t nm2 = f2_pack(neg_m, neg_m);
       uint32_t pk[kPfBN / 2];
-      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t ps4[4] = {0ull, 0ull, 0ull, 0ull};  // pairs of +0.0f
 #pragma unroll
       for (int e = 0; e < kPfBN / 2; ++e) {
-        const float p0 = ex2_approx(fmaf(sv[2 * e], sl2, neg_m));
-        const float p1 = ex2_approx(fmaf(sv[2 * e + 1], sl2, neg_m));
-        ps4[e & 3] += p0 + p1;
-        pk[e] = pack_bf16(p0, p1);
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), sl2x2, nm2), x0, x1);
+        float p0, p1;
+        if ((e & 7) < DMS_PF_POLY_PAIRS) {
+          p0 = ex2_poly(x0);
+          p1 = ex2_poly(x1);
+        } else {
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
+        }
+        ps4[e & 3] = f2_add(ps4[e & 3], f2_pack(p0, p1));
+        pk[e] = DMS_PF_PACK_INT ? pack_bf16_pos(p0, p1) : pack_bf16(p0, p1);
       }
-      const float psum = (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+      float s_even, s_odd;
+      f2_unpack(f2_add(f2_add(ps4[0], ps4[1]), f2_add(ps4[2], ps4[3])), s_even, s_odd);
+      const float psum = s_even + s_odd;
       *reinterpret_cast<volatile float*>(&s_turn_sum[qt][row]) = psum;
       // the turn ends once every exponential is done: the arrive is control
       // dependent on their sum (the condition always holds: psum is a sum of
