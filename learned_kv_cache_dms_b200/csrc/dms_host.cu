@@ -137,7 +137,7 @@ bool make_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_
                    const cuuint32_t* box) {
   auto enc = tensor_map_encoder();
   if (!enc || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
-  cuuint32_t estr[3] = {1u, 1u, 1u};
+  cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -467,8 +467,13 @@ int dms_prefill_attention(dms_cache* c, int layer, const dms_prefill_args* a, vo
     const cuuint64_t kd[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(c->desc.num_kv_heads), bt};
     const cuuint64_t ks[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(c->desc.num_kv_heads) * D * 2};
     const cuuint32_t kbx[3] = {64u, 1u, 64u};
+    // o as [B][T][Hq][D] (rank 4, so rows at or past T are clipped from stores)
+    const cuuint64_t od[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(c->desc.num_q_heads),
+                              static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(c->desc.batch)};
+    const cuuint64_t os[3] = {qs[0], qs[1], qs[1] * T};
+    const cuuint32_t ob[4] = {64u, static_cast<cuuint32_t>(g), static_cast<cuuint32_t>(128 / g), 1u};
     maps.valid = make_bf16_map(&maps.q, a->q, 3, qd, qs, qb) && make_bf16_map(&maps.k, a->k, 3, kd, ks, kbx) &&
-                 make_bf16_map(&maps.v, a->v, 3, kd, ks, kbx);
+                 make_bf16_map(&maps.v, a->v, 3, kd, ks, kbx) && make_bf16_map(&maps.o, a->o, 4, od, os, ob);
     maps.kept_k = c->kept_kmap;
     maps.kept_v = c->kept_vmap;
   }

@@ -399,7 +399,7 @@ cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T, const v
 // k and v [B*T, Hkv, D] (box 64 x 1 x 128), kept copies [B*Hkv*max_pos, D] (box 64 x 128),
 // all bf16 with the 128-byte swizzle.  `valid` is false when the shape is not covered.
 struct PrefillMaps {
-  CUtensorMap q, k, v, kept_k, kept_v;
+  CUtensorMap q, k, v, o, kept_k, kept_v;
   bool valid;
 };
 cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, const void* k, const void* v,

@@ -70,11 +70,13 @@ struct PfSmem {
   static constexpr int HALVES = D / 64;
   static constexpr int Q_BYTES = HALVES * kPfRows * 128;  // one Q tile: [half][128 rows][128 B]
   static constexpr int KV_BYTES = HALVES * kPfBN * 128;   // K (or V) of one key tile: [half][64 keys][128 B]
-  static constexpr int ST = D == 64 ? 8 : 4;              // K stages, V stages
+  static constexpr int ST = D == 64 ? 8 : 3;              // K stages, V stages
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + kPfQT * Q_BYTES;
   static constexpr int OFF_V = OFF_K + ST * KV_BYTES;
-  static constexpr int BYTES = OFF_V + ST * KV_BYTES;
+  static constexpr int O_BYTES = HALVES * kPfRows * 128;  // per Q tile: O / l (bf16), staged for the TMA stores
+  static constexpr int OFF_O = OFF_V + ST * KV_BYTES;
+  static constexpr int BYTES = OFF_O + kPfQT * O_BYTES;
   // tensor memory: S0, S1 (64 fp32 columns each), O0, O1 (D columns each),
   // P0, P1 (64 bf16 = 32 columns each)
   static constexpr uint32_t COL_O = 2 * kPfBN;
@@ -82,6 +84,10 @@ struct PfSmem {
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(COL_P + kPfQT * kPfBN / 2 <= TMEM_COLS, "tensor memory columns");
 };
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
 
 // Named barriers among the two softmax warpgroups (ids 1, 2; 0 is
 // __syncthreads): arrive without waiting, or wait for `count` arrivals.
@@ -93,6 +99,27 @@ template <int ID>
 __device__ __forceinline__ void named_sync() {
   asm volatile("bar.sync %0, %1;\n" ::"n"(ID), "n"(2 * kPfRows) : "memory");
 }
+
+// the 128 threads of softmax warpgroup qt (ids 3, 4)
+__device__ __forceinline__ void wg_sync(int qt) {
+  if (qt == 0)
+    asm volatile("bar.sync 3, %0;\n" ::"n"(kPfRows) : "memory");
+  else
+    asm volatile("bar.sync 4, %0;\n" ::"n"(kPfRows) : "memory");
+}
+
+// 4-D TMA tile store from shared memory (bulk group), its commit and waits
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* smem_src, int c0, int c1, int c2,
+                                             int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];\n" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(smem_src))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -152,6 +179,22 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// ex2_poly on a pair with paired arithmetic
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& p0, float& p1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t sh = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(x, sh);
+  const uint64_t f = f2_fma(f2_add(t, f2_pack(-12582912.f, -12582912.f)), f2_pack(-1.f, -1.f), x);
+  const uint64_t q = f2_fma(f2_fma(f2_fma(f2_pack(0.0551716611f, 0.0551716611f), f, f2_pack(0.24261114f, 0.24261114f)), f,
+                                   f2_pack(0.693260968f, 0.693260968f)),
+                            f, f2_pack(0.999928057f, 0.999928057f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 // 32 consecutive fp32 columns of this thread's TMEM lane, without waiting.
 __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t* r) {
   asm volatile(
@@ -175,39 +218,101 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// One work item: a block of kPfQT * NP query positions of one (batch, KV head).
+struct PfItem {
+  int h, b, bh, i0, i1, nk, jlo, jhi, nkt, ntiles;
+  bool valid;
+};
+
+// The k-th item of CTA `cta` of G: items are numbered heaviest (latest
+// block) first and dealt in snake order, one per CTA per round, so the
+// rounds' decreasing weights even out across CTAs.
+__device__ __forceinline__ int pf_item_index(int k, int G, int cta) {
+  return k * G + ((k & 1) ? (G - 1 - cta) : cta);
+}
+
+// The item's geometry; nk (kept keys before i1 - w, a table read) is passed in
+// so that callers can fetch it one item ahead.
+__device__ __forceinline__ PfItem pf_item(const CacheView& c, int T, int NP, int nblk, int nitems, int u, int nk) {
+  PfItem it{};
+  it.valid = u < nitems;
+  if (!it.valid) return it;
+  const int per = c.Hkv * c.B, blk = nblk - 1 - u / per, rem = u % per;
+  it.h = rem % c.Hkv;
+  it.b = rem / c.Hkv;
+  it.bh = it.b * c.Hkv + it.h;
+  it.i0 = blk * kPfQT * NP;
+  it.i1 = min(T, it.i0 + kPfQT * NP);
+  it.nk = nk;
+  it.jlo = max(0, it.i0 - c.w + 1);
+  it.jhi = it.i1 - 1;
+  it.nkt = (it.nk + kPfBN - 1) / kPfBN;  // kept tiles
+  it.ntiles = it.nkt + (it.jhi - it.jlo + kPfBN) / kPfBN;
+  return it;
+}
+
+// A table read issued where it is written (the asm keeps the compiler from
+// sinking it to its use, an item later), and the point from which its value
+// may be used (keeps the compiler from consuming it early, which would make
+// the warp wait for the read right after issuing it).
+__device__ __forceinline__ int ld_early_i32(const int* p) {
+  int v;
+  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ int use_late(int v) {
+  int r;
+  asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+  return r;
+}
+
+// kept_upto(bh, x) of item u's (batch, KV head) at position x = i0 + dx
+// (0 when x <= 0 or the item does not exist; x is clamped to T)
+__device__ __forceinline__ int pf_kept_upto(const CacheView& c, int T, int NP, int nblk, int nitems, int u, int dx) {
+  if (u >= nitems) return 0;
+  const int per = c.Hkv * c.B, blk = nblk - 1 - u / per, rem = u % per;
+  const int x = min(blk * kPfQT * NP + dx, T);
+  return x > 0 ? ld_early_i32(c.kept_upto + static_cast<long>((rem / c.Hkv) * c.Hkv + rem % c.Hkv) * (c.max_pos + 1) + x)
+               : 0;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
     k_attn_prefill_tc(CacheView c, int T, __nv_bfloat16* o, const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-                      const __grid_constant__ CUtensorMap kkmap, const __grid_constant__ CUtensorMap kvmap) {
+                      const __grid_constant__ CUtensorMap kkmap, const __grid_constant__ CUtensorMap kvmap,
+                      const __grid_constant__ CUtensorMap omap) {
   using L = PfSmem<D>;
   constexpr int ST = L::ST;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sb = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint32_t tmem_base;
-  __shared__ __align__(8) uint64_t bar_q, k_full[ST], v_full[ST], k_empty[ST], v_empty[ST];
-  __shared__ __align__(8) uint64_t s_full[kPfQT], s_free[kPfQT], p_full[kPfQT], pv_done[kPfQT];
+  __shared__ __align__(8) uint64_t bar_q, q_empty, k_full[ST], v_full[ST], k_empty[ST], v_empty[ST];
+  __shared__ __align__(8) uint64_t s_full[kPfQT], s_free[kPfQT], p_full[kPfQT], pv_done[kPfQT], o_free[kPfQT];
   __shared__ int s_abort;
   // anchors of the exponentials' turn: a zero read after the turn begins and
-  // every row's sum written before it ends (a barrier orders memory accesses
-  // only, so the exponentials are tied to it through these)
+  // every row's sum written (to one word per group) before it ends (a barrier
+  // orders memory accesses only, so the exponentials are tied to it through
+  // these)
   __shared__ float s_turn_zero;
-  __shared__ float s_turn_sum[kPfQT][kPfRows];
+  __shared__ float s_turn_sink[kPfQT];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = c.Hq / c.Hkv, NP = kPfRows / g;
+  const int g = c.Hq / c.Hkv, NP = kPfRows / g, w = c.w;
   const int nblk = (T + kPfQT * NP - 1) / (kPfQT * NP);
-  const int blk = nblk - 1 - static_cast<int>(blockIdx.x);  // heavy (late) blocks first
-  const int h = blockIdx.y, b = blockIdx.z, w = c.w;
-  const int i0 = blk * kPfQT * NP, i1 = min(T, i0 + kPfQT * NP);
-  const int bh = b * c.Hkv + h;
-  const int nk = (i1 - w > 0) ? c.kept_upto[static_cast<long>(bh) * (c.max_pos + 1) + (i1 - w)] : 0;
-  const int jlo = max(0, i0 - w + 1), jhi = i1 - 1;
-  const int nkt = (nk + kPfBN - 1) / kPfBN;  // kept tiles
-  const int ntiles = nkt + (jhi - jlo + kPfBN) / kPfBN;
+  const int nitems = nblk * c.Hkv * c.B, G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+  // item k of this CTA, and its nk (kept keys before i1 - w)
+  auto item_nk = [&](int k) {
+    const int u = pf_item_index(k, G, cta);
+    if (u >= nitems) return 0;
+    const int i0 = (nblk - 1 - u / (c.Hkv * c.B)) * kPfQT * NP, i1 = min(T, i0 + kPfQT * NP);
+    return pf_kept_upto(c, T, NP, nblk, nitems, u, i1 - i0 - w);
+  };
+  auto item = [&](int k, int nk) { return pf_item(c, T, NP, nblk, nitems, pf_item_index(k, G, cta), nk); };
 
   if (tid == 0) {
     mbar_init(&bar_q, 1);
+    mbar_init(&q_empty, kPfQT);  // both Q tiles' last scores of the item done
     for (int i = 0; i < ST; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
@@ -219,6 +324,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&s_free[i], 4);  // one arrival per softmax warp
       mbar_init(&p_full[i], 4);
       mbar_init(&pv_done[i], 1);
+      mbar_init(&o_free[i], 4);  // O of the item read out: the next item may start a fresh sum
     }
     fence_mbar_init();
     s_abort = 0;
@@ -235,59 +341,70 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   };
 
   if (warp == kPfLoadWarp) {
-    // ---- Q, then K of every key tile with its positions ------------------
+    // ---- per item: Q (once the previous item's scores are done), then K of
+    // every key tile -----------------------------------------------------------
     if (lane == 0) {
-      mbar_expect_tx(&bar_q, kPfQT * L::Q_BYTES);
-      for (int qt = 0; qt < kPfQT; ++qt)
-        for (int hf = 0; hf < L::HALVES; ++hf)
-          tma_load_3d(sb + L::OFF_Q + qt * L::Q_BYTES + hf * (kPfRows * 128), &qmap, hf * 64, h * g,
-                      b * T + i0 + qt * NP, &bar_q);
-    }
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = j % ST, use = j / ST;
-      if (lane == 0) {
-        if (use > 0 && !mbar_wait_parked(&k_empty[st], (use - 1) & 1)) {
+      int t = 0;  // tiles loaded so far (ring position)
+      PfItem it = item(0, item_nk(0));
+      for (int k = 0; it.valid && !s_abort; ++k) {
+        const int nk_next = item_nk(k + 1);
+        if (k > 0 && !mbar_wait_parked(&q_empty, (k - 1) & 1)) {
           give_up();
-        } else {
-          PF_MARK(j, 12);
-          const bool kt = j < nkt;
-          const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
+          break;
+        }
+        mbar_expect_tx(&bar_q, kPfQT * L::Q_BYTES);
+        for (int qt = 0; qt < kPfQT; ++qt)
+          for (int hf = 0; hf < L::HALVES; ++hf)
+            tma_load_3d(sb + L::OFF_Q + qt * L::Q_BYTES + hf * (kPfRows * 128), &qmap, hf * 64, it.h * g,
+                        it.b * T + it.i0 + qt * NP, &bar_q);
+        for (int j = 0; j < it.ntiles; ++j, ++t) {
+          const int st = t % ST, use = t / ST;
+          if (use > 0 && !mbar_wait_parked(&k_empty[st], (use - 1) & 1)) {
+            give_up();
+            break;
+          }
+          PF_MARK(t, 12);
+          const bool kt = j < it.nkt;
+          const int jb = kt ? j * kPfBN : it.jlo + (j - it.nkt) * kPfBN;
           mbar_expect_tx(&k_full[st], L::KV_BYTES);
           for (int hf = 0; hf < L::HALVES; ++hf) {
             unsigned char* dk = sb + L::OFF_K + st * L::KV_BYTES + hf * (kPfBN * 128);
             if (kt)
-              tma_load_2d(dk, &kkmap, hf * 64, bh * c.max_pos + jb, &k_full[st]);
+              tma_load_2d(dk, &kkmap, hf * 64, it.bh * c.max_pos + jb, &k_full[st]);
             else
-              tma_load_3d(dk, &kmap, hf * 64, h, b * T + jb, &k_full[st]);
+              tma_load_3d(dk, &kmap, hf * 64, it.h, it.b * T + jb, &k_full[st]);
           }
-          PF_MARK(j, 13);
+          PF_MARK(t, 13);
         }
+        it = item(k + 1, use_late(nk_next));
       }
-      __syncwarp();
-      if (s_abort) break;
     }
   } else if (warp == kPfLoadWarp + 1) {
-    // ---- V of every key tile -------------------------------------------
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = j % ST, use = j / ST;
-      if (lane == 0) {
-        if (use > 0 && !mbar_wait_parked(&v_empty[st], (use - 1) & 1)) {
-          give_up();
-        } else {
-          const bool kt = j < nkt;
-          const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
+    // ---- V of every key tile of every item ------------------------------
+    if (lane == 0) {
+      int t = 0;
+      PfItem it = item(0, item_nk(0));
+      for (int k = 0; it.valid && !s_abort; ++k) {
+        const int nk_next = item_nk(k + 1);
+        for (int j = 0; j < it.ntiles; ++j, ++t) {
+          const int st = t % ST, use = t / ST;
+          if (use > 0 && !mbar_wait_parked(&v_empty[st], (use - 1) & 1)) {
+            give_up();
+            break;
+          }
+          const bool kt = j < it.nkt;
+          const int jb = kt ? j * kPfBN : it.jlo + (j - it.nkt) * kPfBN;
           mbar_expect_tx(&v_full[st], L::KV_BYTES);
           for (int hf = 0; hf < L::HALVES; ++hf) {
             unsigned char* dv = sb + L::OFF_V + st * L::KV_BYTES + hf * (kPfBN * 128);
             if (kt)
-              tma_load_2d(dv, &kvmap, hf * 64, bh * c.max_pos + jb, &v_full[st]);
+              tma_load_2d(dv, &kvmap, hf * 64, it.bh * c.max_pos + jb, &v_full[st]);
             else
-              tma_load_3d(dv, &vmap, hf * 64, h, b * T + jb, &v_full[st]);
+              tma_load_3d(dv, &vmap, hf * 64, it.h, it.b * T + jb, &v_full[st]);
           }
         }
+        it = item(k + 1, use_late(nk_next));
       }
-      __syncwarp();
-      if (s_abort) break;
     }
   } else if (warp == kPfMmaWarp || warp == kPfMmaWarp + 1) {
     // ---- tensor-core issue for Q tile qt (one thread) ----------------------
@@ -295,11 +412,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = umma_idesc_bf16(kPfRows, kPfBN, 0);
       constexpr uint32_t IDESC_O = umma_idesc_bf16(kPfRows, D, 1);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % ST;
-        PF_MARK(j, 16 * qt + 8);
-        if (!mbar_wait_bounded(&k_full[st], (j / ST) & 1)) return false;
-        PF_MARK(j, 16 * qt + 9);
+      // S(t) = Q K(t)^T; after the item's last scores Q may be replaced
+      auto issue_s = [&](int t, bool last_of_item) -> bool {
+        const int st = t % ST;
+        PF_MARK(t, 16 * qt + 8);
+        if (!mbar_wait_bounded(&k_full[st], (t / ST) & 1)) return false;
+        PF_MARK(t, 16 * qt + 9);
         tc_fence_after();
         const uint32_t qa = smem_u32(sb + L::OFF_Q + qt * L::Q_BYTES);
         const uint32_t ka = smem_u32(sb + L::OFF_K + st * L::KV_BYTES);
@@ -312,14 +430,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         umma_commit(&s_full[qt]);
         umma_commit(&k_empty[st]);  // this Q tile is done with the K stage
+        if (last_of_item) umma_commit(&q_empty);
         return true;
       };
-      auto issue_pv = [&](int j) -> bool {
-        const int st = j % ST;
-        if (!mbar_wait_bounded(&v_full[st], (j / ST) & 1)) return false;
-        PF_MARK(j, 16 * qt + 10);
-        if (!mbar_wait_bounded(&p_full[qt], j & 1)) return false;
-        PF_MARK(j, 16 * qt + 11);
+      // O += P(t) V(t); the item's first product starts a fresh sum once the
+      // previous item's O has been read out
+      auto issue_pv = [&](int t, int j, int k) -> bool {
+        const int st = t % ST;
+        if (!mbar_wait_bounded(&v_full[st], (t / ST) & 1)) return false;
+        PF_MARK(t, 16 * qt + 10);
+        if (!mbar_wait_bounded(&p_full[qt], t & 1)) return false;
+        if (j == 0 && k > 0 && !mbar_wait_bounded(&o_free[qt], (k - 1) & 1)) return false;
+        PF_MARK(t, 16 * qt + 11);
         tc_fence_after();
         const uint32_t va = smem_u32(sb + L::OFF_V + st * L::KV_BYTES);
 #pragma unroll
@@ -330,12 +452,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         umma_commit(&v_empty[st]);  // this Q tile is done with the V stage
         return true;
       };
-      bool ok = mbar_wait_bounded(&bar_q, 0) && issue_s(0);
-      for (int j = 0; ok && j < ntiles; ++j) {
-        // the next scores once the softmax has read S(j), then P(j) V(j)
-        if (j + 1 < ntiles) ok = mbar_wait_bounded(&s_free[qt], j & 1) && issue_s(j + 1);
-        ok = ok && issue_pv(j);
-        if (s_abort) break;
+      int t = 0;
+      PfItem it = item(0, item_nk(0));
+      bool ok = !it.valid || (mbar_wait_bounded(&bar_q, 0) && issue_s(0, it.ntiles == 1));
+      for (int k = 0; ok && it.valid; ++k) {
+        const PfItem nx = item(k + 1, item_nk(k + 1));  // (used at the item's last tile)
+        for (int j = 0; ok && j < it.ntiles; ++j, ++t) {
+          // within the item: the next scores once the softmax has read S(t),
+          // then P(t) V(t); at its last tile P V first (the epilogue waits for
+          // it), then the next item's first scores
+          if (j + 1 < it.ntiles) {
+            ok = mbar_wait_bounded(&s_free[qt], t & 1) && issue_s(t + 1, j + 2 == it.ntiles);
+            ok = ok && issue_pv(t, j, k);
+          } else {
+            ok = issue_pv(t, j, k);
+            if (nx.valid)
+              ok = ok && mbar_wait_bounded(&s_free[qt], t & 1) && mbar_wait_bounded(&bar_q, (k + 1) & 1) &&
+                   issue_s(t + 1, nx.ntiles == 1);
+          }
+          if (s_abort) ok = false;
+        }
+        it = nx;
       }
       if (!ok) give_up();
     }
@@ -346,163 +483,196 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t tmem_s = tmem + lane_off + qt * kPfBN;
     const uint32_t tmem_o = tmem + lane_off + L::COL_O + qt * D;
     const uint32_t tmem_p = tmem + lane_off + L::COL_P + qt * (kPfBN / 2);
-    const int i_row = i0 + qt * NP + row / g, r_row = row % g;
+    const int p_row = qt * NP + row / g;  // the row's position within the item
     const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
-    // the row's visible keys: kept-list entries [0, ck) (positions <= i - w)
-    // and band positions [blo, bhi]
-    const int ck_at = min(i_row - w + 1, T);
-    const int ck = ck_at > 0 ? c.kept_upto[static_cast<long>(bh) * (c.max_pos + 1) + ck_at] : 0;
-    const int blo = max(0, i_row - w + 1), bhi = min(i_row, jhi);
-    float m_ref = -INFINITY, l_row = 0.f;
+    // the row's count of visible kept keys: kept-list entries [0, ck) are the
+    // positions <= i - w
+    auto kept_visible = [&](int k) {
+      return pf_kept_upto(c, T, NP, nblk, nitems, pf_item_index(k, G, cta), p_row - w + 1);
+    };
     bool ok = true;
+    int t = 0;
+    PfItem it = item(0, item_nk(0));
+    int ck = kept_visible(0);
     // The two warpgroups take turns for the exponentials (named barrier 1:
     // WG1 may start, 2: WG0 may start; bar.arrive by the group that finishes,
     // bar.sync by the one that waits), so one group's exponentials overlap the
-    // other group's tensor-core work and bookkeeping.  Every barrier step runs
-    // even after a failed wait, so neither group can be left waiting.
-    for (int j = 0; j < ntiles; ++j) {
-      // visible columns [c_lo, c_hi] of this tile for the row
-      const bool kt = j < nkt;
-      const int jb = kt ? j * kPfBN : jlo + (j - nkt) * kPfBN;
-      const int c_lo = max(kt ? 0 : blo - jb, 0), c_hi = min(kt ? ck - 1 - jb : bhi - jb, kPfBN - 1);
-      const bool row_full = c_lo == 0 && c_hi == kPfBN - 1;
-      if (row == 0) PF_MARK(j, 16 * qt + 0);
-      ok = ok && mbar_wait_bounded(&s_full[qt], j & 1);
-      if (row == 0) PF_MARK(j, 16 * qt + 1);
-      tc_fence_after();
-      uint32_t sr[kPfBN];
-      if (ok) {
-        tmem_ld32_nowait(tmem_s, sr);
-        tmem_ld32_nowait(tmem_s + 32, sr + 32);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int n = 0; n < kPfBN; ++n) sr[n] = 0u;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (ok && lane == 0) mbar_arrive(&s_free[qt]);  // S may be overwritten by the next tile's scores
-      if (row == 0) PF_MARK(j, 16 * qt + 2);
-      // raw scores with the invisible ones at -inf; row max over 4 chains
-      float sv[kPfBN];
-      if (__all_sync(0xffffffffu, row_full)) {
-#pragma unroll
-        for (int n = 0; n < kPfBN; ++n) sv[n] = __uint_as_float(sr[n]);
-      } else {
-        // bits c_lo..c_hi (none when the range is empty)
-        uint32_t m0 = 0u, m1 = 0u;
-        if (c_lo <= c_hi) {
-          const unsigned long long m = (~0ull >> (kPfBN - 1 - (c_hi - c_lo))) << c_lo;
-          m0 = static_cast<uint32_t>(m);
-          m1 = static_cast<uint32_t>(m >> 32);
-        }
-#pragma unroll
-        for (int n = 0; n < kPfBN; ++n)
-          sv[n] = (((n < 32 ? m0 : m1) >> (n & 31)) & 1u) ? __uint_as_float(sr[n]) : -INFINITY;
-      }
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int n = 0; n < kPfBN; n += 2) mx4[(n >> 1) & 3] = fmax3(mx4[(n >> 1) & 3], sv[n], sv[n + 1]);
-      const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
-      // raise the reference only when this tile exceeds it by more than 2^8
-      const bool raise = tmax > m_ref + 8.0f;
-      float factor = 1.0f;
-      if (raise) {
-        factor = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - tmax);
-        m_ref = tmax;
-        l_row *= factor;
-      }
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a fully masked row so far: all p = 0
-      if (row == 0) PF_MARK(j, 16 * qt + 6);
-      if (qt == 0) {
-        if (j > 0) named_sync<2>();
-      } else {
-        named_sync<1>();
-      }
-      if (row == 0) PF_MARK(j, 16 * qt + 7);
-      const float neg_m = *reinterpret_cast<volatile float*>(&s_turn_zero) - m_use;
-      const uint64_t nm2 = f2_pack(neg_m, neg_m);
-      uint32_t pk[kPfBN / 2];
-      uint64_t ps4[4] = {0ull, 0ull, 0ull, 0ull};  // pairs of +0.0f
-#pragma unroll
-      for (int e = 0; e < kPfBN / 2; ++e) {
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), sl2x2, nm2), x0, x1);
-        float p0, p1;
-        if ((e & 7) < DMS_PF_POLY_PAIRS) {
-          p0 = ex2_poly(x0);
-          p1 = ex2_poly(x1);
+    // other group's tensor-core work and bookkeeping.  Both groups walk the
+    // same items and tiles, and every barrier step runs even after a failed
+    // wait, so neither group can be left waiting.
+    for (int k = 0; it.valid; ++k) {
+      const int nk_next = item_nk(k + 1), ck_next = kept_visible(k + 1);
+      const int i_row = it.i0 + p_row;
+      const int blo = max(0, i_row - w + 1), bhi = min(i_row, it.jhi);  // band positions of the row
+      float m_ref = -INFINITY, l_row = 0.f;
+      for (int j = 0; j < it.ntiles; ++j, ++t) {
+        // visible columns [c_lo, c_hi] of this tile for the row
+        const bool kt = j < it.nkt;
+        const int jb = kt ? j * kPfBN : it.jlo + (j - it.nkt) * kPfBN;
+        const int c_lo = max(kt ? 0 : blo - jb, 0), c_hi = min(kt ? ck - 1 - jb : bhi - jb, kPfBN - 1);
+        const bool row_full = c_lo == 0 && c_hi == kPfBN - 1;
+        if (row == 0) PF_MARK(t, 16 * qt + 0);
+        ok = ok && mbar_wait_bounded(&s_full[qt], t & 1);
+        if (row == 0) PF_MARK(t, 16 * qt + 1);
+        tc_fence_after();
+        uint32_t sr[kPfBN];
+        if (ok) {
+          tmem_ld32_nowait(tmem_s, sr);
+          tmem_ld32_nowait(tmem_s + 32, sr + 32);
+          tmem_wait_ld();
         } else {
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
-        }
-        ps4[e & 3] = f2_add(ps4[e & 3], f2_pack(p0, p1));
-        pk[e] = DMS_PF_PACK_INT ? pack_bf16_pos(p0, p1) : pack_bf16(p0, p1);
-      }
-      float s_even, s_odd;
-      f2_unpack(f2_add(f2_add(ps4[0], ps4[1]), f2_add(ps4[2], ps4[3])), s_even, s_odd);
-      const float psum = s_even + s_odd;
-      *reinterpret_cast<volatile float*>(&s_turn_sum[qt][row]) = psum;
-      // the turn ends once every exponential is done: the arrive is control
-      // dependent on their sum (the condition always holds: psum is a sum of
-      // non-negative terms, never this negative NaN pattern)
-      if (__float_as_uint(psum) != 0xFFFFFFFFu) {
-        if (qt == 0)
-          named_arrive<1>();
-        else
-          named_arrive<2>();
-      }
-      l_row += psum;
-      if (row == 0) PF_MARK(j, 16 * qt + 3);
-      // P V of the previous tile has finished with P and with O
-      if (j > 0) ok = ok && mbar_wait_bounded(&pv_done[qt], (j - 1) & 1);
-      tc_fence_after();
-      if (row == 0) PF_MARK(j, 16 * qt + 4);
-      if (ok && j > 0 && __any_sync(0xffffffffu, raise && factor != 1.0f)) {
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float ov[32];
-          tmem_ld32(tmem_o + c0, ov);
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) ov[jj] *= factor;
-          tmem_st32(tmem_o + c0, ov);
+          for (int n = 0; n < kPfBN; ++n) sr[n] = 0u;
         }
+        tc_fence_before();
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(&s_free[qt]);  // S may be overwritten by the next tile's scores
+        if (row == 0) PF_MARK(t, 16 * qt + 2);
+        // raw scores with the invisible ones at -inf; row max over 4 chains
+        float sv[kPfBN];
+        if (__all_sync(0xffffffffu, row_full)) {
+#pragma unroll
+          for (int n = 0; n < kPfBN; ++n) sv[n] = __uint_as_float(sr[n]);
+        } else {
+          // bits c_lo..c_hi (none when the range is empty)
+          uint32_t m0 = 0u, m1 = 0u;
+          if (c_lo <= c_hi) {
+            const unsigned long long m = (~0ull >> (kPfBN - 1 - (c_hi - c_lo))) << c_lo;
+            m0 = static_cast<uint32_t>(m);
+            m1 = static_cast<uint32_t>(m >> 32);
+          }
+#pragma unroll
+          for (int n = 0; n < kPfBN; ++n)
+            sv[n] = (((n < 32 ? m0 : m1) >> (n & 31)) & 1u) ? __uint_as_float(sr[n]) : -INFINITY;
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int n = 0; n < kPfBN; n += 2) mx4[(n >> 1) & 3] = fmax3(mx4[(n >> 1) & 3], sv[n], sv[n + 1]);
+        const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+        // raise the reference only when this tile exceeds it by more than 2^8
+        const bool raise = tmax > m_ref + 8.0f;
+        float factor = 1.0f;
+        if (raise) {
+          factor = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - tmax);
+          m_ref = tmax;
+          l_row *= factor;
+        }
+        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a fully masked row so far: all p = 0
+        if (row == 0) PF_MARK(t, 16 * qt + 6);
+        if (qt == 0) {
+          if (t > 0) named_sync<2>();
+        } else {
+          named_sync<1>();
+        }
+        if (row == 0) PF_MARK(t, 16 * qt + 7);
+        const float neg_m = *reinterpret_cast<volatile float*>(&s_turn_zero) - m_use;
+        const uint64_t nm2 = f2_pack(neg_m, neg_m);
+        uint32_t pk[kPfBN / 2];
+        uint64_t ps4[4] = {0ull, 0ull, 0ull, 0ull};  // pairs of +0.0f
+#pragma unroll
+        for (int e = 0; e < kPfBN / 2; ++e) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), sl2x2, nm2), x0, x1);
+          float p0, p1;
+          if ((e & 7) < DMS_PF_POLY_PAIRS) {
+            ex2_poly2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          ps4[e & 3] = f2_add(ps4[e & 3], f2_pack(p0, p1));
+          pk[e] = DMS_PF_PACK_INT ? pack_bf16_pos(p0, p1) : pack_bf16(p0, p1);
+        }
+        float s_even, s_odd;
+        f2_unpack(f2_add(f2_add(ps4[0], ps4[1]), f2_add(ps4[2], ps4[3])), s_even, s_odd);
+        const float psum = s_even + s_odd;
+        *reinterpret_cast<volatile float*>(&s_turn_sink[qt]) = psum;
+        // the turn ends once every exponential is done: the arrive is control
+        // dependent on their sum (the condition always holds: psum is a sum of
+        // non-negative terms, never this negative NaN pattern)
+        if (__float_as_uint(psum) != 0xFFFFFFFFu) {
+          if (qt == 0)
+            named_arrive<1>();
+          else
+            named_arrive<2>();
+        }
+        l_row += psum;
+        if (row == 0) PF_MARK(t, 16 * qt + 3);
+        // P V of the previous tile has finished with P and with O (for the
+        // item's first tile the previous item's epilogue waited for it)
+        if (j > 0) ok = ok && mbar_wait_bounded(&pv_done[qt], (t - 1) & 1);
+        tc_fence_after();
+        if (row == 0) PF_MARK(t, 16 * qt + 4);
+        if (ok && j > 0 && __any_sync(0xffffffffu, raise && factor != 1.0f)) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float ov[32];
+            tmem_ld32(tmem_o + c0, ov);
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) ov[jj] *= factor;
+            tmem_st32(tmem_o + c0, ov);
+          }
+        }
+        tmem_st32_nowait(tmem_p, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();  // the warp's P rows and O rescale precede lane 0's release
+        if (ok && lane == 0) mbar_arrive(&p_full[qt]);
+        if (row == 0) PF_MARK(t, 16 * qt + 5);
+        if (s_abort) ok = false;
       }
-      tmem_st32_nowait(tmem_p, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();  // the warp's P rows and O rescale precede lane 0's release
-      if (ok && lane == 0) mbar_arrive(&p_full[qt]);
-      if (row == 0) PF_MARK(j, 16 * qt + 5);
-      if (s_abort) ok = false;
-    }
-    if (qt == 0 && ntiles > 0) named_sync<2>();  // WG1's last hand-back
-    // the last P V, then O / l
-    if (ok && ntiles > 0) ok = mbar_wait_bounded(&pv_done[qt], (ntiles - 1) & 1);
-    if (!ok) {
-      if ((tid & (kPfRows - 1)) == 0) give_up();
-    } else {
+      // the item's last P V, then O / l; O is released to the next item as
+      // soon as it is in registers
+      ok = ok && mbar_wait_bounded(&pv_done[qt], (t - 1) & 1);
+      if (row == 0) PF_MARK(t - 1, 16 * qt + 14);
       tc_fence_after();
+      // read O, release it, write O / l (bf16, 64-column boxes) to this
+      // group's staging tile once the previous item's TMA stores have read
+      // it, and store it with the TMA (rows at or past T are clipped by the
+      // map)
       const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
-      __nv_bfloat16* orow = o + ((static_cast<long>(b) * T + i_row) * c.Hq + h * g + r_row) * D;
-#pragma unroll
+      unsigned char* stg = sb + L::OFF_O + qt * L::O_BYTES;
+      const bool store = ok && it.i0 + qt * NP < T;
+      if (store) {
+        if (row == 0) bulk_wait_read0();  // the previous item's stores have read the staging tile
+        wg_sync(qt);
+      }
+#pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         float ov[32];
-        tmem_ld32(tmem_o + c0, ov);
-        if (i_row < T) {
+        if (ok) tmem_ld32(tmem_o + c0, ov);
+        if (store) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 pkk;
-            pkk.x = pack_bf16(ov[e] * inv, ov[e + 1] * inv);
-            pkk.y = pack_bf16(ov[e + 2] * inv, ov[e + 3] * inv);
-            pkk.z = pack_bf16(ov[e + 4] * inv, ov[e + 5] * inv);
-            pkk.w = pack_bf16(ov[e + 6] * inv, ov[e + 7] * inv);
-            *reinterpret_cast<uint4*>(orow + c0 + e) = pkk;
+          for (int ch = 0; ch < 4; ++ch) {
+            const int e = ch * 8;
+            *reinterpret_cast<uint4*>(stg + (c0 / 64) * (kPfRows * 128) + swz(row, (c0 % 64) / 8 + ch)) =
+                make_uint4(pack_bf16(ov[e] * inv, ov[e + 1] * inv), pack_bf16(ov[e + 2] * inv, ov[e + 3] * inv),
+                           pack_bf16(ov[e + 4] * inv, ov[e + 5] * inv), pack_bf16(ov[e + 6] * inv, ov[e + 7] * inv));
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (row == 0) PF_MARK(t - 1, 16 * qt + 15);
+      if (ok && lane == 0) mbar_arrive(&o_free[qt]);
+      if (store) {
+        fence_proxy_async();  // the tile visible to the TMA
+        wg_sync(qt);
+        if (row == 0) {
+          for (int hf = 0; hf < L::HALVES; ++hf)
+            tma_store_4d(&omap, stg + hf * (kPfRows * 128), hf * 64, it.h * g, it.i0 + qt * NP, it.b);
+          bulk_commit();
+        }
+      }
+      if (row == 0) PF_MARK(t, 16 * qt + 14);
+      it = item(k + 1, use_late(nk_next));
+      ck = use_late(ck_next);
+      if (row == 0) PF_MARK(t, 16 * qt + 15);
     }
+    if (qt == 0 && t > 0) named_sync<2>();  // WG1's last hand-back
+    if (row == 0) bulk_wait0();                 // this group's stores complete before the CTA ends
+    if (!ok && row == 0) give_up();
   }
   tc_fence_before();
   __syncthreads();
@@ -516,9 +686,10 @@ static cudaError_t launch_tc(const CacheView& c, int T, void* o, const PrefillMa
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int g = c.Hq / c.Hkv, NP = kPfRows / g;
-  dim3 grid((T + kPfQT * NP - 1) / (kPfQT * NP), c.Hkv, c.B);
+  const long nitems = static_cast<long>((T + kPfQT * NP - 1) / (kPfQT * NP)) * c.Hkv * c.B;
+  const int grid = static_cast<int>(min(nitems, static_cast<long>(c.num_sms)));  // persistent: one CTA per SM
   k_attn_prefill_tc<D><<<grid, kPfThreads, smem, s>>>(c, T, static_cast<__nv_bfloat16*>(o), m.q, m.k, m.v, m.kept_k,
-                                                      m.kept_v);
+                                                      m.kept_v, m.o);
   return cudaGetLastError();
 }
 
