@@ -5,18 +5,20 @@
 // about two CTAs per SM) covers one (b, h): CTA r attends a contiguous range of
 // the head's retained slots, staged by TMA in sub-tiles of at most 64 slots
 // that never cross a page, with the g query heads as the M dimension of
-// mma.sync tiles.  Each CTA leaves its merged partial (acc, running max,
-// running sum, log2 domain) in its own shared memory; after a cluster barrier
-// rank 0 reads the cs partials through distributed shared memory and writes
-// the head's output rows ([FastDMS], attention scoring: split-K grouped compact
-// decode attention over variable-length per-head live spans -- here the split
-// never leaves the chip).
+// mma.sync tiles.  Each CTA merges its warps into one partial (acc, running
+// max, running sum, log2 domain) and writes it with st.async into the shared
+// memory of the cluster's last rank (the owner), completing bytes on an
+// mbarrier there; the owner, whose share of the slots is the smallest, merges
+// the cs partials from its own shared memory and writes the head's output
+// rows ([FastDMS], attention scoring: split-K grouped compact decode
+// attention over variable-length per-head live spans -- here the split never
+// leaves the chip).  The other ranks leave as soon as their partial is sent.
 //
 // FUSED (bf16 pages): the whole decode step in one launch.  The attention runs
 // over the slots as they were before this step's append, with the slot this
 // token reuses masked out and the new token's key/value taken from the input
 // as one more key of rank 0 -- the same visible set as after the append.  Rank
-// 0 then appends the token at the slot fixed by the plan of the previous step
+// 0 (the owner) then appends the token at the slot fixed by the plan of the previous step
 // ([DMS-Qwen3], inference mode: a token overwrites the slot of the token
 // leaving the window when that one was marked, else takes the next slot; a new
 // page when that slot starts one), updates the head's count and writes the
@@ -39,9 +41,15 @@ template <int D, bool FP8>
 struct ClusterSmem {
   using S = DecodeSmem<D, FP8>;
   static constexpr int MLD = D + 2;
-  static size_t bytes(int g) {
-    return 1024 + kStages * S::STAGE + S::CONV + (5 * g + g) * MLD * sizeof(float) +
-           (3 * kMaxCluster * 16 + 16) * sizeof(float);
+  static constexpr int IMLD = D + 4;  // inbox row: D values, max, sum, 2 pad (16-byte rows)
+  // floats of the merge buffer [5 sources][g][MLD], rounded up so the inbox
+  // after it starts on 16 bytes
+  __host__ __device__ static int merge_floats(int g) { return (5 * g * MLD + 3) / 4 * 4; }
+  // stages, conversion tile, merge buffer, the owner's inbox [cs][g][IMLD],
+  // weights [max(cs, 5)][g], row maxima and sums [2][16]
+  static size_t bytes(int g, int cs) {
+    return 1024 + kStages * S::STAGE + S::CONV + (merge_floats(g) + cs * g * IMLD) * sizeof(float) +
+           (kMaxCluster * 16 + 32) * sizeof(float);
   }
 };
 
@@ -59,7 +67,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
                                                             const __grid_constant__ CUtensorMap kmap,
                                                             const __grid_constant__ CUtensorMap vmap) {
   using S = DecodeSmem<D, FP8>;
-  constexpr int KS = D / 16, NT = D / 8, MLD = D + 2;
+  constexpr int KS = D / 16, NT = D / 8, MLD = D + 2, IMLD = ClusterSmem<D, FP8>::IMLD;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sbase =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -67,12 +75,11 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   unsigned char* conv_buf = sbase + kStages * S::STAGE;
   const int g = c.Hq / c.Hkv;
   float* merge = reinterpret_cast<float*>(conv_buf + S::CONV);  // [5 sources][g][MLD]
-  float* cpart = merge + 5 * g * MLD;                           // [g][MLD] this CTA's partial
-  float* sm_m = cpart + g * MLD;                                // [cs][g] maxima of the cluster's partials
-  float* sm_l = sm_m + kMaxCluster * 16;                        // [cs][g] sums, then weights
-  float* sm_w = sm_l + kMaxCluster * 16;                        // [cs][g] weights
+  float* inbox = merge + ClusterSmem<D, FP8>::merge_floats(g);  // [cs][g][IMLD] partials, on the owner (16-byte aligned)
+  float* sm_w = inbox + cs * g * IMLD;                          // [sources][g] weights
   float* sm_L = sm_w + kMaxCluster * 16;                        // [g]
   __shared__ uint64_t full_bar[kStages];
+  __shared__ uint64_t inbox_bar;  // the owner: every rank's partial has landed
   __shared__ SubMeta meta[kStages];
   __shared__ int s_abort, s_have, s_last, s_red[32], s_ring_next;
   __shared__ float s_fred[8], s_alpha, s_xscore[16];
@@ -89,6 +96,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   DMS_TRACE_MARK(0, 0);
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&full_bar[i], 1);
+    mbar_init(&inbox_bar, 1);
     fence_mbar_init();
     s_abort = 0;
   }
@@ -102,9 +110,14 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   const int4 pl = FUSED ? *plan_at(c, li, t) : make_int4(0, 0, 0, 0);
   const int masked_slot = (FUSED && (pl.y & 1)) ? pl.x : -1;
   const int next_page0 = FUSED ? c.ctrl[CTRL_NEXT_PAGE] : 0;
-  const int per = ((cnt + cs - 1) / cs + 15) / 16 * 16;
-  const int s_begin = min(cnt, rank * per), s_end = min(cnt, s_begin + per);
+  // ranks 0 .. cs-2 take `per` slots each, the owner the rest: a quarter share
+  // when it also computes the decision logit, half a share otherwise (it
+  // merges the partials and appends)
+  const int oq = (FUSED && fuse_decide) ? 1 : 2;
+  const int per = cs == 1 ? cnt : ((4 * cnt + 4 * (cs - 1) + oq - 1) / (4 * (cs - 1) + oq) + 15) / 16 * 16;
+  const int s_begin = min(cnt, rank * per), s_end = rank == owner ? cnt : min(cnt, s_begin + per);
   __syncthreads();
+  cluster_arrive_relaxed();  // this CTA's barriers are initialised (waited before the first remote store)
 
   int p_s = s_begin;
   auto produce = [&](int stage) -> bool {
@@ -194,8 +207,8 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   }
 
   DMS_TRACE_MARK(0, 3);
-  // merge the warps (and, for rank 0 of a fused step, the new token) into this
-  // CTA's partial
+  // merge the warps (and, for the owner of a fused step, the new token) into
+  // this CTA's partial, written into slot `rank` of the owner's inbox
   warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
   int nsrc = 4;
   if (FUSED && rank == owner) {
@@ -208,61 +221,85 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     nsrc = 5;
   }
   __syncthreads();
-  merge_sources<D>(merge, nsrc, g, 1.0f, [&](int r, int d, float v) { cpart[r * MLD + d] = v; });
-  cluster_sync();  // every partial of the cluster is in place
+  // per row: the sources' weights 2^(m_s - M) and the merged (M, L)
+  if (tid < g) {
+    float M = -INFINITY;
+    for (int sv = 0; sv < nsrc; ++sv) M = fmaxf(M, merge[(sv * g + tid) * MLD + D]);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float L = 0.f;
+    for (int sv = 0; sv < nsrc; ++sv) {
+      const float wgt = exp2f(merge[(sv * g + tid) * MLD + D] - Mu);
+      sm_w[sv * g + tid] = wgt;
+      L = fmaf(wgt, merge[(sv * g + tid) * MLD + D + 1], L);
+    }
+    sm_L[tid] = M;
+    sm_L[16 + tid] = L;
+  }
+  __syncthreads();
+  cluster_wait();  // every CTA's barriers are initialised
+  // this CTA's partial row r: acc (4 values per thread and pass), then (M, L);
+  // written into slot `rank` of the owner's inbox (st.async to another rank)
+  const uint32_t dst = dsmem_addr(inbox + rank * g * IMLD, owner), rbar = dsmem_addr(&inbox_bar, owner);
+  for (int e4 = tid; e4 < g * (D / 4); e4 += kThreads) {
+    const int r = e4 / (D / 4), d = 4 * (e4 % (D / 4));
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sv = 0; sv < nsrc; ++sv) {
+      const float wgt = sm_w[sv * g + r];
+      const float* src = merge + (sv * g + r) * MLD + d;
+      v.x = fmaf(wgt, src[0], v.x);
+      v.y = fmaf(wgt, src[1], v.y);
+      v.z = fmaf(wgt, src[2], v.z);
+      v.w = fmaf(wgt, src[3], v.w);
+    }
+    if (rank != owner)
+      st_async_v4(dst + 4u * static_cast<uint32_t>(r * IMLD + d), v, rbar);
+    else
+      *reinterpret_cast<float4*>(inbox + (owner * g + r) * IMLD + d) = v;
+  }
+  if (tid < g) {
+    if (rank != owner)
+      st_async_v2(dst + 4u * static_cast<uint32_t>(tid * IMLD + D), sm_L[tid], sm_L[16 + tid], rbar);
+    else {
+      inbox[(owner * g + tid) * IMLD + D] = sm_L[tid];
+      inbox[(owner * g + tid) * IMLD + D + 1] = sm_L[16 + tid];
+    }
+  }
+  if (rank != owner) {
+    DMS_TRACE_MARK(0, 4);
+    DMS_TRACE_MARK(0, 6);
+    return;  // nothing reads this CTA's shared memory
+  }
+  if (tid == 0) mbar_expect_tx(&inbox_bar, static_cast<uint32_t>((cs - 1) * g * (D + 2) * 4));
+  bool landed = true;
+  if (cs > 1 && !mbar_wait_bounded(&inbox_bar, 0)) {
+    landed = false;
+    if (tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
+  }
+  __syncthreads();  // the owner's own partial is in place too
   DMS_TRACE_MARK(0, 4);
 
-  // Combine the cs partials through distributed shared memory: CTA `rank`
-  // merges output elements [rank * per_cta, (rank + 1) * per_cta) of the head's
-  // g x D block, with every remote load of a thread issued before use.
-  {
-    const int total = g * D;
-    const int per_cta = (total + cs - 1) / cs;
-    const int e0 = rank * per_cta, e1 = min(total, e0 + per_cta);
-    const int r0 = e0 / D, r1 = e1 > e0 ? (e1 - 1) / D : r0 - 1;  // rows touched
-    const int nrows = r1 - r0 + 1;
-    for (int idx = tid; idx < cs * nrows; idx += kThreads) {
-      const int k = idx / nrows, r = r0 + idx % nrows;
-      sm_m[idx] = ld_dsmem(dsmem_addr(&cpart[r * MLD + D], k));
-      sm_l[idx] = ld_dsmem(dsmem_addr(&cpart[r * MLD + D + 1], k));
-    }
-    __syncthreads();
-    if (tid < nrows) {
+  // the head's output rows: weights of the cs partials per row, then O / L
+  if (landed) {
+    if (tid < g) {
       float M = -INFINITY;
-      for (int k = 0; k < cs; ++k) M = fmaxf(M, sm_m[k * nrows + tid]);
+      for (int k = 0; k < cs; ++k) M = fmaxf(M, inbox[(k * g + tid) * IMLD + D]);
       const float Mu = M == -INFINITY ? 0.f : M;
       float L = 0.f;
       for (int k = 0; k < cs; ++k) {
-        const float wgt = exp2f(sm_m[k * nrows + tid] - Mu);
-        sm_w[k * nrows + tid] = wgt;
-        L += wgt * sm_l[k * nrows + tid];
+        const float wgt = exp2f(inbox[(k * g + tid) * IMLD + D] - Mu);
+        sm_w[k * g + tid] = wgt;
+        L = fmaf(wgt, inbox[(k * g + tid) * IMLD + D + 1], L);
       }
       sm_L[tid] = L;
     }
     __syncthreads();
     __nv_bfloat16* ob = o + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D;
-    constexpr int EPT = 4;  // output elements per thread per pass
-    for (int base = e0; base < e1; base += kThreads * EPT) {
-      float v[EPT][kPickCluster];
-#pragma unroll
-      for (int j = 0; j < EPT; ++j) {
-        const int e = base + j * kThreads + tid;
-#pragma unroll
-        for (int k = 0; k < kPickCluster; ++k)
-          v[j][k] = (e < e1 && k < cs) ? ld_dsmem(dsmem_addr(&cpart[(e / D) * MLD + e % D], k)) : 0.f;
-      }
-#pragma unroll
-      for (int j = 0; j < EPT; ++j) {
-        const int e = base + j * kThreads + tid;
-        if (e >= e1) continue;
-        const int rl = e / D - r0;
-        float a = 0.f;
-#pragma unroll
-        for (int k = 0; k < kPickCluster; ++k)
-          if (k < cs) a = fmaf(sm_w[k * nrows + rl], v[j][k], a);
-        const float L = sm_L[rl];
-        ob[e] = __float2bfloat16_rn(L > 0.f ? a / L : 0.f);
-      }
+    for (int e = tid; e < g * D; e += kThreads) {
+      const int r = e / D, d = e % D;
+      float a = 0.f;
+      for (int k = 0; k < cs; ++k) a = fmaf(sm_w[k * g + r], inbox[(k * g + r) * IMLD + d], a);
+      const float L = sm_L[r];
+      ob[e] = __float2bfloat16_rn(L > 0.f ? a / L : 0.f);
     }
   }
 
@@ -280,11 +317,12 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
         int before;
         block_exclusive_scan(n_before, s_red, &before);
         id = next_page0 + before;
-        if (id >= c.pool_pages || c.npages[li] >= c.maxp) ok = false;
+        if (id >= c.pool_pages || pl.w >= c.maxp) ok = false;
       } else if (ok) {
-        id = c.page_table[li * c.maxp + slot / c.P];
+        const int pi = slot / c.P;
+        id = pi < kPtCache ? s_pt[pi] : c.page_table[li * c.maxp + pi];
       }
-      int cnt_new = cnt, np_new = c.npages[li];
+      int cnt_new = cnt, np_new = pl.w;  // pages before the append (plan snapshot)
       if (ok) {
         const long row = static_cast<long>(id) * c.P + slot % c.P;
         if (tid < D / 8) {
@@ -318,13 +356,12 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     }
   }
   DMS_TRACE_MARK(0, 5);
-  cluster_sync();  // rank 0 is done reading the cluster's shared memory
 
   if (FUSED) {
-    // the grid's last CTA advances the page counter and the positions
+    // the grid's last owner advances the page counter and the positions
     if (tid == 0) {
       __threadfence();
-      s_last = (atomicAdd(&c.ctrl[CTRL_GRID_DONE], 1) == static_cast<int>(gridDim.x) - 1) ? 1 : 0;
+      s_last = (atomicAdd(&c.ctrl[CTRL_GRID_DONE], 1) == static_cast<int>(gridDim.x) / cs - 1) ? 1 : 0;
     }
     __syncthreads();
     if (s_last) {
@@ -342,13 +379,25 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
 }
 
 // Cluster size: the largest power of two <= 8 with cs * B * Hkv <= 2 * SMs
-// (about two CTAs per SM) that the device can co-schedule.
+// (about two CTAs per SM) whose shared memory fits and which the device can
+// co-schedule.
 template <int D, bool FP8, bool FUSED>
-static int pick_cluster(int heads, int num_sms, size_t smem) {
-  static int max_cs = 0;
-  if (max_cs == 0) {
-    max_cs = 1;
+static int pick_cluster(int heads, int g, int num_sms) {
+  static int max_cs[17] = {0};  // by g (<= 16)
+  int& m = max_cs[g < 16 ? g : 16];
+  if (m == 0) {
+    m = 1;
+    int dev = 0, optin = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     for (int cs = kPickCluster; cs > 1; cs >>= 1) {
+      const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs);
+      if (smem + 4096 > static_cast<size_t>(optin)) continue;  // static shared memory on top
+      if (cudaFuncSetAttribute(k_decode_cluster<D, FP8, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -362,14 +411,14 @@ static int pick_cluster(int heads, int num_sms, size_t smem) {
       cfg.numAttrs = 1;
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, k_decode_cluster<D, FP8, FUSED>, &cfg) == cudaSuccess && n > 0) {
-        max_cs = cs;
+        m = cs;
         break;
       }
       cudaGetLastError();
     }
   }
   int cs = 1;
-  while (cs * 2 <= max_cs && static_cast<long>(cs) * 2 * heads <= 2L * num_sms) cs *= 2;
+  while (cs * 2 <= m && static_cast<long>(cs) * 2 * heads <= 2L * num_sms) cs *= 2;
   return cs;
 }
 
@@ -378,13 +427,14 @@ static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q
                                    const void* v, float* alpha, const DecideArgs* da, const CUtensorMap* kmap,
                                    const CUtensorMap* vmap, int num_sms, cudaStream_t s) {
   const int g = c.Hq / c.Hkv;
-  const size_t smem = ClusterSmem<D, FP8>::bytes(g);
   auto kern = k_decode_cluster<D, FP8, FUSED>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
   const int heads = c.B * c.Hkv;
-  const int cs = pick_cluster<D, FP8, FUSED>(heads, num_sms, smem);
+  const int cs = pick_cluster<D, FP8, FUSED>(heads, g, num_sms);
+  const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
