@@ -460,6 +460,13 @@ __device__ __forceinline__ float decide_cta(const CacheView& c, const DecideArgs
   return alpha;
 }
 
+// Programmatic dependent launch: let the next kernel of the stream start its
+// prologue, and wait until every kernel this one depends on has completed.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 // Distributed shared memory (thread-block clusters).
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;

@@ -546,7 +546,7 @@ int run_decode_kernel(dms_cache* c, int layer, const void* q, void* o, bool fuse
       return DMS_ERR_CUDA;
     if (taken) return DMS_OK;
   }
-  return launch_decode_cluster(cv, layer, q, o, fused, k, v, alpha, da, &c->kmap, &c->vmap, c->num_sms, s) ==
+  return launch_decode_cluster(cv, layer, q, o, fused, k, v, alpha, da, &c->kmap, &c->vmap, c->num_sms, s, early) ==
                  cudaSuccess
              ? DMS_OK
              : DMS_ERR_CUDA;

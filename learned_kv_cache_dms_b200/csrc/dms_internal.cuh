@@ -420,6 +420,6 @@ cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, voi
                                const CUtensorMap* vmap, cudaStream_t s, bool early, bool* taken);
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
-                                  const CUtensorMap* vmap, int num_sms, cudaStream_t s);
+                                  const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early);
 
 }  // namespace dms

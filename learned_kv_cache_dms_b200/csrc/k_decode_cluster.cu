@@ -60,7 +60,7 @@ struct SubMeta {
 };
 
 template <int D, bool FP8, bool FUSED>
-__global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int layer, const __nv_bfloat16* q,
+__global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int layer, int early, const __nv_bfloat16* q,
                                                             __nv_bfloat16* o, int cs, const __nv_bfloat16* k_new,
                                                             const __nv_bfloat16* v_new, float* alpha, DecideArgs da,
                                                             int fuse_decide,
@@ -94,6 +94,17 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   const int b = bh / c.Hkv, h = bh % c.Hkv;
   const long li = static_cast<long>(layer) * c.B * c.Hkv + bh;
   DMS_TRACE_MARK(0, 0);
+  // Programmatic dependent launch.  With `early` (the previous launch of this
+  // library on the stream was for another layer or cache) this layer's state
+  // is read and the first tiles are requested before waiting for the previous
+  // kernel: only that kernel may still run (each kernel lets its dependents
+  // start only once its own wait has returned), and it does not write this
+  // state.  The page counter, the inputs and the outputs are touched only
+  // after the wait.
+  if (!early) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&full_bar[i], 1);
     mbar_init(&inbox_bar, 1);
@@ -109,7 +120,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   const int t = FUSED ? c.pos[layer * c.B + b] : 0;
   const int4 pl = FUSED ? *plan_at(c, li, t) : make_int4(0, 0, 0, 0);
   const int masked_slot = (FUSED && (pl.y & 1)) ? pl.x : -1;
-  const int next_page0 = FUSED ? c.ctrl[CTRL_NEXT_PAGE] : 0;
   // ranks 0 .. cs-2 take `per` slots each, the owner the rest: a quarter share
   // when it also computes the decision logit, half a share otherwise (it
   // merges the partials and appends)
@@ -137,6 +147,11 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     for (int st = 0; st < kStages; ++st)
       if (produce(st)) ++produced;
 
+  if (early) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
+  const int next_page0 = FUSED ? c.ctrl[CTRL_NEXT_PAGE] : 0;
   uint32_t qa[KS][4];
   const __nv_bfloat16* qb = q + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D;
   load_q_frags<D>(qb, g, qa);
@@ -425,7 +440,7 @@ static int pick_cluster(int heads, int g, int num_sms) {
 template <int D, bool FP8, bool FUSED>
 static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q, void* o, const void* k,
                                    const void* v, float* alpha, const DecideArgs* da, const CUtensorMap* kmap,
-                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s) {
+                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early) {
   const int g = c.Hq / c.Hkv;
   auto kern = k_decode_cluster<D, FP8, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -436,37 +451,39 @@ static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(cs * heads, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   DecideArgs none{};
-  return cudaLaunchKernelEx(&cfg, kern, c, layer, static_cast<const __nv_bfloat16*>(q),
+  return cudaLaunchKernelEx(&cfg, kern, c, layer, early ? 1 : 0, static_cast<const __nv_bfloat16*>(q),
                             static_cast<__nv_bfloat16*>(o), cs, static_cast<const __nv_bfloat16*>(k),
                             static_cast<const __nv_bfloat16*>(v), alpha, da ? *da : none, da ? 1 : 0, *kmap, *vmap);
 }
 
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
-                                  const CUtensorMap* vmap, int num_sms, cudaStream_t s) {
+                                  const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early) {
   if (!kmap || !vmap || c.kv_dtype == DMS_F32) return cudaErrorInvalidValue;
   if (fused) {
     if (c.kv_dtype != DMS_BF16) return cudaErrorInvalidValue;
-    return c.D == 64 ? launch_cluster_t<64, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s)
-                     : launch_cluster_t<128, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s);
+    return c.D == 64 ? launch_cluster_t<64, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s, early)
+                     : launch_cluster_t<128, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s, early);
   }
   if (c.kv_dtype == DMS_FP8_E4M3)
-    return c.D == 64 ? launch_cluster_t<64, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s)
-                     : launch_cluster_t<128, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s);
-  return c.D == 64 ? launch_cluster_t<64, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s)
-                   : launch_cluster_t<128, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s);
+    return c.D == 64 ? launch_cluster_t<64, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early)
+                     : launch_cluster_t<128, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early);
+  return c.D == 64 ? launch_cluster_t<64, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early)
+                   : launch_cluster_t<128, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early);
 }
 
 }  // namespace dms

@@ -147,12 +147,6 @@ __device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
   asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
 }
-// Programmatic dependent launch: let the next kernel of the stream start its
-// prologue, and wait until every kernel this one depends on has completed.
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-}
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 // Barrier of the four consumer warps only (the producer warp never joins).
 __device__ __forceinline__ void consumers_sync() { asm volatile("barrier.sync 1, 128;\n" ::: "memory"); }
 
