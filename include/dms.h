@@ -160,6 +160,8 @@ typedef struct dms_cache_layout {
  *   [DMS-Qwen3] "Gumbel 噪声与可微门控": at inference a token is evicted iff
  *   alpha > 0 (alpha == 0 keeps), and never when disable_eviction is set. */
 typedef struct dms_decide_params {
+  /* PROJ: hidden, norm_weight and proj_weight are read as 16-byte vectors and
+   * must be 16-byte aligned (DMS_ERR_INVALID otherwise). */
   const void* hidden;      /* device [B,T,hidden] (decode: [B,hidden]), act dtype; PROJ only */
   const void* norm_weight; /* device gamma [hidden], act dtype; PROJ only                 */
   const void* proj_weight; /* device W [Hkv,hidden], act dtype; PROJ only                 */

@@ -144,6 +144,16 @@ bool make_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map of the adapter's hidden rows [B*T, hidden] for the tensor-core
+// decision kernel (bf16 only); false when it cannot be built.
+bool make_hidden_map(CUtensorMap* map, const dms_cache_desc* d, const void* hidden, int T) {
+  if (d->act_dtype != DMS_BF16 || !hidden) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d->hidden), static_cast<cuuint64_t>(d->batch) * T};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d->hidden) * 2};
+  const cuuint32_t box[2] = {64u, 64u};  // 64 hidden elements x 64 tokens
+  return make_bf16_map(map, hidden, 2, dims, strides, box);
+}
+
 }  // namespace
 
 // The last (cache, layer) this library enqueued work for on each stream
@@ -379,8 +389,12 @@ int dms_cache_positions(const dms_cache* c, int layer) {
 static int check_decide(const dms_cache* c, const dms_decide_params* d) {
   if (!d || !d->offset) return DMS_ERR_INVALID;
   if (d->offset_batch_stride != 0 && d->offset_batch_stride != c->desc.num_kv_heads) return DMS_ERR_INVALID;
-  if (c->desc.alpha_source == DMS_ALPHA_PROJ && (!d->hidden || !d->norm_weight || !d->proj_weight))
-    return DMS_ERR_INVALID;
+  if (c->desc.alpha_source == DMS_ALPHA_PROJ) {
+    if (!d->hidden || !d->norm_weight || !d->proj_weight) return DMS_ERR_INVALID;
+    const uintptr_t any = reinterpret_cast<uintptr_t>(d->hidden) | reinterpret_cast<uintptr_t>(d->norm_weight) |
+                          reinterpret_cast<uintptr_t>(d->proj_weight);
+    if (any & 15) return DMS_ERR_INVALID;  // read as 16-byte vectors
+  }
   return DMS_OK;
 }
 
@@ -402,7 +416,9 @@ int dms_decide(dms_cache* c, int T, const dms_decide_params* d, void* neuron_src
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t r;
   if (c->desc.alpha_source == DMS_ALPHA_PROJ) {
-    r = launch_decide_proj(c->view, T, decide_args(d), alpha, s);
+    CUtensorMap hm;
+    const bool have = make_hidden_map(&hm, &c->desc, d->hidden, T);
+    r = launch_decide_proj(c->view, T, decide_args(d), alpha, have ? &hm : nullptr, s);
   } else {
     if (!neuron_src) return DMS_ERR_INVALID;
     const bool key = c->desc.alpha_source == DMS_ALPHA_KEY_NEURON;
@@ -432,7 +448,10 @@ int dms_prefill_compact(dms_cache* c, int layer, const dms_prefill_args* a, void
   const CacheView& v = c->view;
   const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
   if (a->decide && !neuron) {
-    if (launch_decide_proj(v, T, decide_args(a->decide), a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
+    CUtensorMap hm;
+    const bool have = make_hidden_map(&hm, &c->desc, a->decide->hidden, T);
+    if (launch_decide_proj(v, T, decide_args(a->decide), a->alpha, have ? &hm : nullptr, s) != cudaSuccess)
+      return DMS_ERR_CUDA;
   }
   if (neuron || a->rope_cos) {
     if (launch_neuron_rope(v, T, nullptr, a->q, a->k, neuron ? a->decide->offset : nullptr,
@@ -509,7 +528,7 @@ int dms_decode_append(dms_cache* c, int layer, const dms_decode_args* a, void* s
   DecideArgs da{};
   if (a->decide && !neuron) {
     da = decide_args(a->decide);
-    if (!fuse && launch_decide_proj(v, 1, da, a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
+    if (!fuse && launch_decide_proj(v, 1, da, a->alpha, nullptr, s) != cudaSuccess) return DMS_ERR_CUDA;
   }
   if (neuron || a->rope_cos) {
     // the token's position is read on the device from the layer's position counter

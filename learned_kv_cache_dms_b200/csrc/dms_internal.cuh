@@ -388,7 +388,10 @@ struct DecideArgs {
 };
 
 cudaError_t launch_init(const CacheView& c, bool full, cudaStream_t s);
-cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, float* alpha, cudaStream_t s);
+// hmap: tensor map of the hidden rows [B*T, hidden] (bf16, 128-byte swizzle,
+// box 64 x 64), or null (CUDA-core kernel).
+cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, float* alpha, const CUtensorMap* hmap,
+                               cudaStream_t s);
 cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
                                int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
                                const float* sin_t, cudaStream_t s);

@@ -62,9 +62,12 @@ cudaError_t launch_init(const CacheView& c, bool full, cudaStream_t s) {
 // 1/rms factor is applied after the dot product:
 //   W_h . (x * inv * gamma) = inv * ((W_h * gamma) . x).
 // Each warp handles kTok tokens at once so each W element read from shared
-// memory serves kTok tokens.  Supports Hkv <= 8.
+// memory serves kTok tokens, and requests the hidden rows kUnroll 16-byte
+// vectors ahead per lane so enough bytes are in flight to stream them at HBM
+// speed.  The folded table is filled with 16-byte loads.  Supports Hkv <= 8.
 // ---------------------------------------------------------------------------
 constexpr int kTok = 4;
+constexpr int kUnroll = 4;
 
 template <typename TA>
 __global__ void __launch_bounds__(256) k_decide_proj(CacheView c, int T, DecideArgs a, float* alpha) {
@@ -74,16 +77,23 @@ __global__ void __launch_bounds__(256) k_decide_proj(CacheView c, int T, DecideA
   const TA* gamma = static_cast<const TA*>(a.gamma);
   const TA* hs = static_cast<const TA*>(a.hidden);
   const TA* bias = static_cast<const TA*>(a.bias);
-  for (int i = threadIdx.x; i < H * hid; i += blockDim.x) wg[i] = to_f(W[i]) * to_f(gamma[i % hid]);
+  constexpr int V = 16 / sizeof(TA);
+  const int nvec = hid / V;
+#pragma unroll 8
+  for (int i = threadIdx.x; i < H * nvec; i += blockDim.x) {
+    float wv[V], gv[V];
+    unpack16(reinterpret_cast<const uint4*>(W)[i], wv, static_cast<const TA*>(nullptr));
+    unpack16(reinterpret_cast<const uint4*>(gamma)[i % nvec], gv, static_cast<const TA*>(nullptr));
+#pragma unroll
+    for (int e = 0; e < V; ++e) wg[i * V + e] = wv[e] * gv[e];
+  }
   __syncthreads();
 
-  constexpr int V = 16 / sizeof(TA);
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   const long gw = static_cast<long>(blockIdx.x) * warps + (threadIdx.x >> 5);
   const long nwarps = static_cast<long>(gridDim.x) * warps;
   const long ntok = static_cast<long>(c.B) * T;
-  const int nvec = hid / V;
   const bool layer_mode = c.alpha_per == DMS_ALPHA_PER_LAYER;
 
   for (long tok0 = gw * kTok; tok0 < ntok; tok0 += nwarps * kTok) {
@@ -95,30 +105,40 @@ __global__ void __launch_bounds__(256) k_decide_proj(CacheView c, int T, DecideA
 #pragma unroll
       for (int j = 0; j < 8; ++j) dot[u][j] = 0.f;
     }
-    for (int vi = lane; vi < nvec; vi += 32) {
-      float x[kTok][V];
+    for (int vb = 0; vb < nvec; vb += 32 * kUnroll) {
+      // every load of the block first, then the arithmetic
+      uint4 raw[kUnroll][kTok];
 #pragma unroll
-      for (int u = 0; u < kTok; ++u) {
-        const long tok = tok0 + u;
-        if (tok < ntok) {
-          uint4 raw = reinterpret_cast<const uint4*>(hs + tok * hid)[vi];
-          unpack16(raw, x[u], static_cast<const TA*>(nullptr));
-        } else {
+      for (int k = 0; k < kUnroll; ++k) {
+        const int vi = vb + k * 32 + lane;
 #pragma unroll
-          for (int e = 0; e < V; ++e) x[u][e] = 0.f;
+        for (int u = 0; u < kTok; ++u) {
+          const long tok = tok0 + u;
+          raw[k][u] = (vi < nvec && tok < ntok) ? reinterpret_cast<const uint4*>(hs + tok * hid)[vi]
+                                                 : make_uint4(0u, 0u, 0u, 0u);
         }
-#pragma unroll
-        for (int e = 0; e < V; ++e) ss[u] = fmaf(x[u][e], x[u][e], ss[u]);
       }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < H) {
-          const float* wp = wg + j * hid + vi * V;
+      for (int k = 0; k < kUnroll; ++k) {
+        const int vi = vb + k * 32 + lane;
+        if (vi >= nvec) continue;
+        float x[kTok][V];
 #pragma unroll
-          for (int e = 0; e < V; ++e) {
-            const float wv = wp[e];
+        for (int u = 0; u < kTok; ++u) {
+          unpack16(raw[k][u], x[u], static_cast<const TA*>(nullptr));
 #pragma unroll
-            for (int u = 0; u < kTok; ++u) dot[u][j] = fmaf(wv, x[u][e], dot[u][j]);
+          for (int e = 0; e < V; ++e) ss[u] = fmaf(x[u][e], x[u][e], ss[u]);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < H) {
+            const float* wp = wg + j * hid + vi * V;
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+              const float wv = wp[e];
+#pragma unroll
+              for (int u = 0; u < kTok; ++u) dot[u][j] = fmaf(wv, x[u][e], dot[u][j]);
+            }
           }
         }
       }
@@ -204,7 +224,180 @@ __global__ void __launch_bounds__(256) k_decide_proj_row(CacheView c, DecideArgs
   }
 }
 
-cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, float* alpha, cudaStream_t s) {
+// ---------------------------------------------------------------------------
+// The same logits for bf16 activations on the tensor cores: a product of the
+// hidden rows [B*T, hidden] with the folded weights (W_h * gamma)^T
+// [hidden, Hkv <= 8], N padded to 8.  W * gamma (exact in 16 bits) is held in
+// shared memory as a bf16 pair hi + lo, so two mma.sync per k-step give the
+// product with fp32 accumulation; the rows' sums of squares come from the A
+// fragments already in registers.  Hidden tiles (64 tokens x 64 elements)
+// stream through an 8-stage TMA ring (no multicast) fed by a producer warp; a
+// persistent grid walks the 64-token tiles.  Consumer warp w takes tokens
+// [16 (w % 4), +16) of the even (w < 4) or odd chunks of the hidden size; the
+// two halves are added through shared memory at the end of the tile.
+// ---------------------------------------------------------------------------
+constexpr int kDpTok = 64, kDpK = 64, kDpStages = 8, kDpWarps = 8;
+constexpr int kDpThreads = (kDpWarps + 1) * 32;
+
+__host__ __device__ inline int dp_wrow(int hid) { return hid + 8; }  // table row (bf16), 16-byte pad
+// byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled TMA tile
+__device__ __forceinline__ uint32_t dp_sw128(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+__host__ __device__ inline size_t dp_smem(int hid) {
+  return 1024 + static_cast<size_t>(kDpStages) * kDpTok * 128 + 2ull * 8 * dp_wrow(hid) * 2;
+}
+
+__global__ void __launch_bounds__(kDpThreads, 1)
+    k_decide_proj_tc(CacheView c, int T, DecideArgs a, float* alpha, const __grid_constant__ CUtensorMap hmap) {
+  extern __shared__ __align__(1024) unsigned char dp_raw[];
+  unsigned char* sb = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dp_raw) + 1023) & ~uintptr_t(1023));
+  __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(sb + kDpStages * kDpTok * 128);  // [2][8][wrow]
+  __shared__ __align__(8) uint64_t full[kDpStages], empty[kDpStages];
+  __shared__ float red[4][6][32];  // odd-chunk halves: acc[4], ss[2] per lane of warps 4..7
+  const int H = c.Hkv, hid = c.hidden, wrow = dp_wrow(hid);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long ntok = static_cast<long>(c.B) * T;
+  const int ntiles = static_cast<int>((ntok + kDpTok - 1) / kDpTok), nk = (hid + kDpK - 1) / kDpK;
+  if (tid == 0) {
+    for (int i = 0; i < kDpStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kDpWarps / 2);  // the four warps of the chunk's parity
+    }
+    fence_mbar_init();
+  }
+  // folded table hi / lo (rows >= H and the pad are zero)
+  const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(a.W);
+  const __nv_bfloat16* gamma = static_cast<const __nv_bfloat16*>(a.gamma);
+  const int nvec = hid / 8;
+#pragma unroll 4
+  for (int i = tid; i < 8 * (wrow / 8); i += kDpThreads) {
+    const int n = i / (wrow / 8), v = i % (wrow / 8);
+    uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+    if (n < H && v < nvec) {
+      float wv[8], gv[8];
+      unpack16(reinterpret_cast<const uint4*>(W + static_cast<long>(n) * hid)[v], wv, static_cast<const __nv_bfloat16*>(nullptr));
+      unpack16(reinterpret_cast<const uint4*>(gamma)[v], gv, static_cast<const __nv_bfloat16*>(nullptr));
+      uint32_t h4[4], l4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float p0 = wv[2 * e] * gv[2 * e], p1 = wv[2 * e + 1] * gv[2 * e + 1];
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+        const float2 hf = __bfloat1622float2(hv);
+        h4[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        l4[e] = pack_bf16(p0 - hf.x, p1 - hf.y);
+      }
+      hi = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+      lo = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+    }
+    reinterpret_cast<uint4*>(wt + static_cast<long>(n) * wrow)[v] = hi;
+    reinterpret_cast<uint4*>(wt + static_cast<long>(8 + n) * wrow)[v] = lo;
+  }
+  __syncthreads();
+
+  if (warp == kDpWarps) {
+    // ---- producer: hidden tiles of this CTA's token tiles ----------------
+    if (lane == 0) {
+      int q = 0;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x)
+        for (int kc = 0; kc < nk; ++kc, ++q) {
+          const int st = q % kDpStages, use = q / kDpStages;
+          if (use > 0 && !mbar_wait_bounded(&empty[st], (use - 1) & 1)) {
+            set_status(c.ctrl, DMS_ST_TIMEOUT);
+            return;
+          }
+          mbar_expect_tx(&full[st], kDpTok * 128);
+          tma_load_2d(sb + st * kDpTok * 128, &hmap, kc * kDpK, tile * kDpTok, &full[st]);
+        }
+    }
+    return;
+  }
+  // ---- consumers ----------------------------------------------------------
+  const bool layer_mode = c.alpha_per == DMS_ALPHA_PER_LAYER;
+  const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+  const int mt = warp & 3, par = warp >> 2;  // token group, chunk parity
+  const int mi = lane >> 3, rr = lane & 7;
+  // ldmatrix row addresses: A rows of this warp; B = table rows n (hi: matrices 0, 1; lo: 2, 3)
+  const int arow = mt * 16 + (mi & 1) * 8 + rr;
+  const uint32_t wbase = smem_u32(wt + static_cast<long>((mi >> 1) * 8 + rr) * wrow + (mi & 1) * 8);
+  int qbase = 0;  // chunks of the CTA's earlier tiles
+  bool ok = true;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, qbase += nk) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float ss[2] = {0.f, 0.f};
+    for (int kc = par; kc < nk; kc += 2) {
+      const int q = qbase + kc, st = q % kDpStages;
+      if (ok && !mbar_wait_bounded(&full[st], (q / kDpStages) & 1)) {
+        ok = false;
+        if (lane == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
+      }
+      if (ok) {
+        const uint32_t xs = smem_u32(sb + st * kDpTok * 128);
+#pragma unroll
+        for (int ks = 0; ks < kDpK / 16; ++ks) {
+          uint32_t af[4], bf[4];
+          ldmatrix_x4(af[0], af[1], af[2], af[3], xs + dp_sw128(arow, 2 * ks + (mi >> 1)));
+          ldmatrix_x4(bf[0], bf[1], bf[2], bf[3], wbase + 2u * static_cast<uint32_t>(kc * kDpK + ks * 16));
+          mma_bf16_16816(acc, af, bf);
+          mma_bf16_16816(acc, af, bf + 2);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&af[r]));
+            ss[r & 1] = fmaf(xv.x, xv.x, fmaf(xv.y, xv.y, ss[r & 1]));
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    // add the odd-chunk half (warp mt + 4) into warp mt
+    if (par == 1) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) red[mt][e][lane] = acc[e];
+      red[mt][4][lane] = ss[0];
+      red[mt][5][lane] = ss[1];
+    }
+    asm volatile("bar.sync 1, %0;\n" ::"n"(kDpWarps * 32) : "memory");
+    if (par == 0) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] += red[mt][e][lane];
+      ss[0] += red[mt][4][lane];
+      ss[1] += red[mt][5][lane];
+      // rows lane/4 and lane/4 + 8 of the group: sums over the 4 lanes of a row
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], 1);
+        ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], 2);
+      }
+      // layer granularity: every head takes head 0's logit (column 0, lane 4 * row)
+      float h0[2];
+      h0[0] = __shfl_sync(0xffffffffu, acc[0], lane & ~3);
+      h0[1] = __shfl_sync(0xffffffffu, acc[2], lane & ~3);
+      if (ok) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const long tok = static_cast<long>(tile) * kDpTok + mt * 16 + (lane >> 2) + 8 * r;
+          if (tok >= ntok) continue;
+          const int b = static_cast<int>(tok / T), t = static_cast<int>(tok % T);
+          const float inv = 1.0f / sqrtf(ss[r] / static_cast<float>(hid) + c.rms_eps);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = 2 * (lane & 3) + e;
+            if (j >= H) continue;
+            const int src = layer_mode ? 0 : j;
+            const float dot = layer_mode ? h0[r] : acc[2 * r + e];
+            const float z = dot * inv + (bias ? __bfloat162float(bias[src]) : 0.f);
+            alpha[(static_cast<long>(b) * H + j) * T + t] = z * c.alpha_scale - a.offset[b * a.offset_bstride + src];
+          }
+        }
+      }
+    }
+    asm volatile("bar.sync 1, %0;\n" ::"n"(kDpWarps * 32) : "memory");  // red is free again
+  }
+}
+
+cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, float* alpha, const CUtensorMap* hmap,
+                               cudaStream_t s) {
   if (T == 1) {
     dim3 grid(c.Hkv, c.B);
     if (c.act_dtype == DMS_BF16)
@@ -213,11 +406,25 @@ cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, f
       k_decide_proj_row<float><<<grid, 256, 0, s>>>(c, a, alpha);
     return cudaGetLastError();
   }
-  const size_t smem = static_cast<size_t>(c.Hkv) * c.hidden * sizeof(float);
   const long ntok = static_cast<long>(c.B) * T;
+  cudaError_t e;
+  if (c.act_dtype == DMS_BF16 && hmap && c.Hkv <= 8) {
+    int dev = 0, optin = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    const size_t smem = dp_smem(c.hidden);
+    if (smem + 1024 <= static_cast<size_t>(optin)) {
+      e = cudaFuncSetAttribute(k_decide_proj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      const long tiles = (ntok + kDpTok - 1) / kDpTok;
+      const int grid = static_cast<int>(min(tiles, static_cast<long>(c.num_sms)));
+      k_decide_proj_tc<<<grid, kDpThreads, smem, s>>>(c, T, a, alpha, *hmap);
+      return cudaGetLastError();
+    }
+  }
+  const size_t smem = static_cast<size_t>(c.Hkv) * c.hidden * sizeof(float);
   const long want = (ntok + 8 * kTok - 1) / (8 * kTok);
   const int grid = static_cast<int>(min(want, static_cast<long>(c.num_sms)));
-  cudaError_t e;
   if (c.act_dtype == DMS_BF16) {
     e = cudaFuncSetAttribute(k_decide_proj<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
