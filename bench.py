@@ -28,6 +28,7 @@ Multi-GPU (torchrun): every rank runs its own replica (independent sequences,
 weak scaling, no collective on the data path); rank 0 prints one JSON line.
 """
 import argparse
+import hashlib
 import json
 import os
 import subprocess
@@ -62,6 +63,9 @@ def parse():
     p.add_argument("--decode-steps", type=int, default=None, help="decode only the first N steps")
     p.add_argument("--decode-kernel", choices=["auto", "cluster", "flat"], default="auto",
                    help="decode attention kernel (auto: by the number of heads)")
+    p.add_argument("--replicas", type=int, default=None,
+                   help="cache replicas per step (default: enough that each step's KV is >= 4x L2; 1 gives a "
+                        "small case for profiler captures, whose numbers are then not L2-cold)")
     return p.parse_args()
 
 
@@ -198,6 +202,46 @@ def kernel_launches_per_step(wl, n_dec):
     # reset (1) + per layer: compaction (decide or neuron/rotary pass, scan,
     # scatter) + prefill attention (1) + the decode steps
     return 1 + wl.layers * (3 + 1) + wl.layers * n_dec * decode_launches_per_step(wl)
+
+
+def decode_kernel_name(wl, choice, num_sms):
+    """The decode kernel the library runs for this workload (its AUTO rule:
+    the cluster kernel while batch * Hkv * 8 <= 2 * SMs)."""
+    if choice == "auto":
+        choice = "cluster" if wl.batch * wl.kv_heads * 8 <= 2 * num_sms else "flat"
+    return "k_decode_" + choice
+
+
+# Sources of each kernel whose DRAM traffic is recorded in profiles/traffic.txt
+TRAFFIC_SOURCES = {
+    "k_decode_cluster": ["k_decode_cluster.cu", "decode_common.cuh"],
+    "k_decode_flat": ["k_decode_flat.cu", "decode_common.cuh"],
+    "k_attn_prefill_tc": ["k_attn_prefill_tc.cu"],
+}
+
+
+def source_digest(kernel):
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "learned_kv_cache_dms_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
+    ncu capture summarised in profiles/, or None when there is none or the
+    kernel's sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if kernel not in TRAFFIC_SOURCES or not os.path.exists(path):
+        return None
+    digest = source_digest(kernel)
+    with open(path) as f:
+        for line in f:
+            fields = line.split()
+            if len(fields) >= 4 and not line.startswith("#") and fields[0] == kernel and fields[1] == workload:
+                return int(fields[2]) if fields[3] == digest else None
+    return None
 
 
 def replicas_for(wl, l2_bytes):
@@ -435,7 +479,7 @@ def run_ours(args, world, rank, local):
     from learned_kv_cache_dms_b200 import binding as B_
     wl = I.WORKLOADS[args.workload]
     pk, pk_kind = peaks()
-    r = Runner(B_, wl, seed=wl.seed + rank, n_dec=args.decode_steps, kernel=args.decode_kernel)
+    r = Runner(B_, wl, seed=wl.seed + rank, n_dec=args.decode_steps, kernel=args.decode_kernel, replicas=args.replicas)
     S, L = r.S, r.L
     # untimed pass: retained counts after the prefill and after each append
     counts = []
@@ -496,11 +540,15 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, args.cpu_seconds)
-    kname = ("decode step: k_decode_cluster<%d,%s> (split-K attention, on-chip combine%s)%s"
-             % (wl.head_dim, wl.kv_dtype, ", append, decision logit" if wl.kv_dtype == "bf16" else "",
+    kern = decode_kernel_name(wl, args.decode_kernel, torch.cuda.get_device_properties(0).multi_processor_count)
+    kname = ("decode step: %s<%d,%s> (split-K attention, %s%s)%s"
+             % (kern, wl.head_dim, wl.kv_dtype,
+                "on-chip combine" if kern == "k_decode_cluster" else "partials merged by the last CTA of a head",
+                ", append, decision logit" if wl.kv_dtype == "bf16" else "",
                 " after k_decode_append" if wl.kv_dtype == "fp8" else ""))
+    traffic = recorded_traffic(kern, workload_label(wl, S)) if args.replicas is None else None
     roof = {"bound": "hbm", "achieved": round(decode_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": round(decode_gbs / pk["hbm_gbs"], 4), "traffic": None, "kernel": kname,
+            "frac": round(decode_gbs / pk["hbm_gbs"], 4), "traffic": traffic, "kernel": kname,
             "algorithmic_bytes_per_launch": int(attn_bytes / (S * L)), "peak_source": pk_kind}
     retained_first = counts[0] / (L * B * wl.kv_heads)
     retained_last = counts[-1] / (L * B * wl.kv_heads)
@@ -625,8 +673,10 @@ E2E_STEPS_STACK = 256
 # ---------------------------------------------------------------------------
 def oracle_decode_sample(wl, seconds, n_steps_max=None):
     """Time the oracle's decode steps (append + decode attention) of one layer
-    on the host cores after an untimed prefill replay.  Returns (tok/s over
-    the workload's layer stack, cores, steps, secs)."""
+    on the host cores after an untimed prefill replay; when the workload's
+    steps take less than `seconds`, further passes over them start from a copy
+    of the prefilled cache (copied outside the timed region).  Returns (tok/s
+    over the workload's layer stack, cores, steps, secs, passes)."""
     from oracle import oracle as O
     cores = O.set_threads(os.cpu_count() or 1)
     B, T, S = wl.batch, wl.prompt, wl.decode_steps
@@ -640,24 +690,31 @@ def oracle_decode_sample(wl, seconds, n_steps_max=None):
     c = O.Cache(1, B, wl.kv_heads, wl.head_dim, wl.window, wl.block, wl.max_positions,
                 B * wl.kv_heads * maxp, wl.prealloc_tokens, fp8=wl.kv_dtype == "fp8")
     c.prefill(0, np.ascontiguousarray(ev[:, :, :T]), np.ascontiguousarray(k[:, :T]), np.ascontiguousarray(v[:, :T]))
-    n = 0
-    t0 = time.perf_counter()
     limit = n_steps_max or S
-    while n < limit and (time.perf_counter() - t0) < seconds:
-        t = T + n
-        c.append(0, np.ascontiguousarray(ev[:, :, t]), np.ascontiguousarray(k[:, t]), np.ascontiguousarray(v[:, t]))
-        c.decode_attention(0, np.ascontiguousarray(q[:, n]))
-        n += 1
-    dt = time.perf_counter() - t0
-    return n * B / (dt * wl.layers), cores, n, dt
+    n = passes = 0
+    dt = 0.0
+    while dt < seconds and (passes == 0 or n_steps_max is None):
+        cc = c.clone() if n_steps_max is None else c
+        t0 = time.perf_counter()
+        i = 0
+        while i < limit and dt + (time.perf_counter() - t0) < seconds:
+            t = T + i
+            cc.append(0, np.ascontiguousarray(ev[:, :, t]), np.ascontiguousarray(k[:, t]), np.ascontiguousarray(v[:, t]))
+            cc.decode_attention(0, np.ascontiguousarray(q[:, i]))
+            i += 1
+        dt += time.perf_counter() - t0
+        n += i
+        passes += 1
+    return n * B / (dt * wl.layers), cores, n, dt, passes
 
 
 def cpu_baseline(wl, seconds):
-    tps, cores, n, dt = oracle_decode_sample(wl, seconds)
+    tps, cores, n, dt, passes = oracle_decode_sample(wl, seconds)
     return {"value": round(tps, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": "first %d of %d decode steps of one layer (append + fp64 decode attention over the retained "
-                      "slots) after an untimed prefill replay of the %d-token prompt, %.1f s%s"
-                      % (n, wl.decode_steps, wl.prompt, dt,
+            "sample": "%d decode steps of one layer (append + fp64 decode attention over the retained slots) in %d "
+                      "pass(es) over the workload's %d steps, each from the cache after an untimed prefill replay of "
+                      "the %d-token prompt, %.1f s timed%s"
+                      % (n, passes, wl.decode_steps, wl.prompt, dt,
                          "; scaled to the %d-layer stack" % wl.layers if wl.layers > 1 else "")}
 
 
@@ -667,11 +724,11 @@ def run_reference(args, world, rank):
     wl = I.WORKLOADS[args.workload]
     per_step = 4  # decode steps of the oracle per bench step (bounded sample)
     for _ in range(args.warmup):
-        oracle_decode_sample(wl, 1e9, n_steps_max=1)
+        oracle_decode_sample(wl, 1e9, n_steps_max=1)[:4]
     tot_tok = tot_s = 0.0
     cores = 1
     for _ in range(args.steps):
-        tps, cores, n, dt = oracle_decode_sample(wl, 1e9, n_steps_max=per_step)
+        tps, cores, n, dt, _ = oracle_decode_sample(wl, 1e9, n_steps_max=per_step)
         tot_tok += n * wl.batch / wl.layers
         tot_s += dt
     val = tot_tok / tot_s

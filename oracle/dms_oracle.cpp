@@ -449,6 +449,8 @@ void* oracle_cache_new(int L, int B, int Hkv, int D, int w, int P, int max_pos, 
 }
 
 void oracle_cache_delete(void* h) { delete static_cast<Cache*>(h); }
+// An independent copy of the whole simulated cache (state and pages).
+void* oracle_cache_clone(void* h) { return new Cache(*static_cast<const Cache*>(h)); }
 
 int oracle_cache_status(void* h) { return static_cast<Cache*>(h)->status; }
 

@@ -34,6 +34,8 @@ def lib():
         L.oracle_cache_new.argtypes = [C.c_int] * 11
         L.oracle_cache_new.restype = C.c_void_p
         L.oracle_cache_delete.argtypes = [C.c_void_p]
+        L.oracle_cache_clone.argtypes = [C.c_void_p]
+        L.oracle_cache_clone.restype = C.c_void_p
         L.oracle_cache_status.argtypes = [C.c_void_p]
         L.oracle_cache_status.restype = C.c_int
         L.oracle_cache_prefill.argtypes = [C.c_void_p, C.c_int, C.c_int, up, fp, fp]
@@ -163,6 +165,13 @@ class Cache:
         self.store_values = bool(store_values)
         self._h = lib().oracle_cache_new(L, B, Hkv, D, window, block, max_pos, pool_pages,
                                          prealloc_tokens, int(self.fp8), int(self.store_values))
+
+    def clone(self):
+        """An independent copy (state and pages) of this cache."""
+        c = Cache.__new__(Cache)
+        c.__dict__.update({k: v for k, v in self.__dict__.items() if k != "_h"})
+        c._h = lib().oracle_cache_clone(self._h)
+        return c
 
     def __del__(self):
         if getattr(self, "_h", None):

@@ -369,6 +369,29 @@ def test_decode_attention_equals_prefill_row():
     assert np.allclose(full[:, T - 1], c.decode_attention(0, np.ascontiguousarray(q[:, T - 1])), atol=1e-6)
 
 
+def test_cache_clone_is_independent():
+    # a clone continues exactly like the original, and appending to one leaves the other unchanged
+    B, T, Hq, Hkv, D, w, P = 1, 30, 2, 1, 8, 4, 4
+    q, k, v = rand_qkv(16, B, T, Hq, Hkv, D)
+    ev = (np.random.default_rng(17).random((B, Hkv, T)) > 0.5).astype(np.uint8)
+    c = O.Cache(1, B, Hkv, D, w, P, T, 40, 0)
+    c.prefill(0, np.ascontiguousarray(ev[:, :, :20]), k[:, :20].astype(np.float32), v[:, :20].astype(np.float32))
+    d = c.clone()
+    q20 = np.ascontiguousarray(q[:, 20])
+    before = c.decode_attention(0, q20)
+    for t in range(20, 25):
+        d.append(0, np.ascontiguousarray(ev[:, :, t]), np.ascontiguousarray(k[:, t]).astype(np.float32),
+                 np.ascontiguousarray(v[:, t]).astype(np.float32))
+    assert np.array_equal(c.decode_attention(0, q20), before)
+    for t in range(20, 25):
+        c.append(0, np.ascontiguousarray(ev[:, :, t]), np.ascontiguousarray(k[:, t]).astype(np.float32),
+                 np.ascontiguousarray(v[:, t]).astype(np.float32))
+    q25 = np.ascontiguousarray(q[:, 24])
+    assert np.array_equal(c.decode_attention(0, q25), d.decode_attention(0, q25))
+    del c
+    assert np.isfinite(d.decode_attention(0, q25)).all()
+
+
 # ---------------------------------------------------------------------------
 # FP8 pages
 # ---------------------------------------------------------------------------
