@@ -467,6 +467,13 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 }
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
+// Atomic add with acquire-release semantics at GPU scope (returns the old value).
+__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // Distributed shared memory (thread-block clusters).
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;

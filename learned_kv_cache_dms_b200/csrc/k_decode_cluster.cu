@@ -37,6 +37,12 @@ __device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
 constexpr int kMaxCluster = 16;  // shared-memory staging bound
 constexpr int kPickCluster = 8;  // largest cluster launched: every cluster of the grid co-resident
 
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int D, bool FP8>
 struct ClusterSmem {
   using S = DecodeSmem<D, FP8>;
@@ -81,7 +87,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   __shared__ uint64_t full_bar[kStages];
   __shared__ uint64_t inbox_bar;  // the owner: every rank's partial has landed
   __shared__ SubMeta meta[kStages];
-  __shared__ int s_abort, s_have, s_last, s_red[32], s_ring_next;
+  __shared__ int s_abort, s_have, s_red[32], s_ring_next;
   __shared__ float s_fred[8], s_alpha, s_xscore[16];
   __shared__ __align__(16) __nv_bfloat16 s_knew[D], s_vnew[D];
   constexpr int kPtCache = 256;  // page-table entries of the head kept in shared memory
@@ -285,111 +291,143 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     return;  // nothing reads this CTA's shared memory
   }
   if (tid == 0) mbar_expect_tx(&inbox_bar, static_cast<uint32_t>((cs - 1) * g * (D + 2) * 4));
-  bool landed = true;
-  if (cs > 1 && !mbar_wait_bounded(&inbox_bar, 0)) {
-    landed = false;
-    if (tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
-  }
-  __syncthreads();  // the owner's own partial is in place too
+  bool landed = cs == 1 || mbar_wait_bounded(&inbox_bar, 0);
+  landed = __syncthreads_and(landed);  // (one answer for the block); the owner's own partial is in place too
+  if (!landed && tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
   DMS_TRACE_MARK(0, 4);
 
-  // the head's output rows: weights of the cs partials per row, then O / L
-  if (landed) {
-    if (tid < g) {
-      float M = -INFINITY;
-      for (int k = 0; k < cs; ++k) M = fmaxf(M, inbox[(k * g + tid) * IMLD + D]);
-      const float Mu = M == -INFINITY ? 0.f : M;
-      float L = 0.f;
-      for (int k = 0; k < cs; ++k) {
-        const float wgt = exp2f(inbox[(k * g + tid) * IMLD + D] - Mu);
-        sm_w[k * g + tid] = wgt;
-        L = fmaf(wgt, inbox[(k * g + tid) * IMLD + D + 1], L);
-      }
-      sm_L[tid] = L;
-    }
-    __syncthreads();
-    __nv_bfloat16* ob = o + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D;
-    for (int e = tid; e < g * D; e += kThreads) {
-      const int r = e / D, d = e % D;
-      float a = 0.f;
-      for (int k = 0; k < cs; ++k) a = fmaf(sm_w[k * g + r], inbox[(k * g + r) * IMLD + d], a);
-      const float L = sm_L[r];
-      ob[e] = __float2bfloat16_rn(L > 0.f ? a / L : 0.f);
-    }
-  }
-
-  if (rank == owner) {
-    if (FUSED) {
-      // append of this head's token at the planned slot (every CTA of the
-      // cluster has finished reading the pages: cluster barrier above)
-      const int flags = pl.y, slot = pl.x;
-      int id = -1;
-      bool ok = !(flags & 4);
-      if (ok && (flags & 2)) {
-        int n_before = 0;
-        for (int i = tid; i < bh; i += kThreads)
-          n_before += (plan_at(c, static_cast<long>(layer) * c.B * c.Hkv + i, t)->y & 2) ? 1 : 0;
-        int before;
-        block_exclusive_scan(n_before, s_red, &before);
-        id = next_page0 + before;
-        if (id >= c.pool_pages || pl.w >= c.maxp) ok = false;
-      } else if (ok) {
-        const int pi = slot / c.P;
-        id = pi < kPtCache ? s_pt[pi] : c.page_table[li * c.maxp + pi];
-      }
-      int cnt_new = cnt, np_new = pl.w;  // pages before the append (plan snapshot)
-      if (ok) {
-        const long row = static_cast<long>(id) * c.P + slot % c.P;
-        if (tid < D / 8) {
-          reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.k_pool) + row * D)[tid] =
-              reinterpret_cast<const uint4*>(s_knew)[tid];
-          reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.v_pool) + row * D)[tid] =
-              reinterpret_cast<const uint4*>(s_vnew)[tid];
-        }
-        if (!(flags & 1)) cnt_new = cnt + 1;
-        if (flags & 2) np_new += 1;
-        if (tid == 0) {
-          if (flags & 2) {
-            c.page_table[li * c.maxp + np_new - 1] = id;
-            c.npages[li] = np_new;
-            atomicAdd(&c.ctrl[CTRL_STEP_PAGES], 1);
-          }
-          const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
-          const float a = fuse_decide ? s_alpha : __ldcg(&alpha[b * c.Hkv + hs]);
-          const bool evict = !c.disable && a > 0.0f;
-          c.slot_pos[li * c.cap + slot] = t;
-          c.ring[li * c.w + t % c.w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
-          if (!(flags & 1)) c.count[li] = cnt_new;
-        }
-      } else if (tid == 0) {
-        set_status(c.ctrl, (flags & 4) ? DMS_ST_CAPACITY : DMS_ST_POOL_EXHAUSTED);
-      }
-      if (tid == 0) {
-        // plan of the next append (token t + 1), from the values just written
-        *plan_at(c, li, t + 1) = make_plan(s_ring_next, t + 1, cnt_new, np_new, c);
-      }
-    }
-  }
-  DMS_TRACE_MARK(0, 5);
-
   if (FUSED) {
-    // the grid's last owner advances the page counter and the positions
-    if (tid == 0) {
-      __threadfence();
-      s_last = (atomicAdd(&c.ctrl[CTRL_GRID_DONE], 1) == static_cast<int>(gridDim.x) / cs - 1) ? 1 : 0;
+    // append of this head's token at the planned slot (every CTA of the
+    // cluster has finished reading the pages: their partials have landed)
+    const int flags = pl.y, slot = pl.x;
+    int id = -1;
+    bool ok = !(flags & 4);
+    if (ok && (flags & 2)) {
+      int n_before = 0;
+      for (int i = tid; i < bh; i += kThreads)
+        n_before += (plan_at(c, static_cast<long>(layer) * c.B * c.Hkv + i, t)->y & 2) ? 1 : 0;
+      int before;
+      block_exclusive_scan(n_before, s_red, &before);
+      id = next_page0 + before;
+      if (id >= c.pool_pages || pl.w >= c.maxp) ok = false;
+    } else if (ok) {
+      const int pi = slot / c.P;
+      id = pi < kPtCache ? s_pt[pi] : c.page_table[li * c.maxp + pi];
     }
-    __syncthreads();
-    if (s_last) {
-      __threadfence();
+    int cnt_new = cnt, np_new = pl.w;  // pages before the append (plan snapshot)
+    if (ok) {
+      const long row = static_cast<long>(id) * c.P + slot % c.P;
+      if (tid < D / 8) {
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.k_pool) + row * D)[tid] =
+            reinterpret_cast<const uint4*>(s_knew)[tid];
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.v_pool) + row * D)[tid] =
+            reinterpret_cast<const uint4*>(s_vnew)[tid];
+      }
+      if (!(flags & 1)) cnt_new = cnt + 1;
+      if (flags & 2) np_new += 1;
       if (tid == 0) {
+        if (flags & 2) {
+          c.page_table[li * c.maxp + np_new - 1] = id;
+          c.npages[li] = np_new;
+          atomicAdd(&c.ctrl[CTRL_STEP_PAGES], 1);
+        }
+        const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
+        const float a = fuse_decide ? s_alpha : __ldcg(&alpha[b * c.Hkv + hs]);
+        const bool evict = !c.disable && a > 0.0f;
+        c.slot_pos[li * c.cap + slot] = t;
+        c.ring[li * c.w + t % c.w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
+        if (!(flags & 1)) c.count[li] = cnt_new;
+      }
+    } else if (tid == 0) {
+      set_status(c.ctrl, (flags & 4) ? DMS_ST_CAPACITY : DMS_ST_POOL_EXHAUSTED);
+    }
+    if (tid == 0) {
+      // plan of the next append (token t + 1), from the values just written
+      *plan_at(c, li, t + 1) = make_plan(s_ring_next, t + 1, cnt_new, np_new, c);
+    }
+    __syncthreads();  // the append (thread 0's page grant included) precedes warp 3's release below
+  }
+  DMS_TRACE_MARK(0, 8);
+
+  if (FUSED && warp == 3) {
+    // warp 3, while warps 0-2 merge: count this owner (the fence releases the
+    // page grant ordered before it by the barrier above); the grid's last
+    // owner advances the page counter and the positions
+    int last = 0;
+    if (lane == 0) {
+      __threadfence();
+      last = atomicAdd(&c.ctrl[CTRL_GRID_DONE], 1) == static_cast<int>(gridDim.x) / cs - 1;
+      if (last) {
+        __threadfence();  // every owner's grant, released before its count, is visible
         const int granted = __ldcg(&c.ctrl[CTRL_STEP_PAGES]);
         c.ctrl[CTRL_NEXT_PAGE] = min(__ldcg(&c.ctrl[CTRL_NEXT_PAGE]) + granted, c.pool_pages);
         c.ctrl[CTRL_STEP_PAGES] = 0;
         c.ctrl[CTRL_GRID_DONE] = 0;
       }
-      for (int bb = tid; bb < c.B; bb += kThreads) c.pos[layer * c.B + bb] += 1;
+    }
+    if (__shfl_sync(0xffffffffu, last, 0))
+      for (int bb = lane; bb < c.B; bb += 32) c.pos[layer * c.B + bb] += 1;
+    DMS_TRACE_MARK(0, 6);
+    return;
+  }
+
+  // the head's output rows: weights of the cs partials per row, then O / L
+  if (landed) {
+    if (tid < g) {
+      float mk[kPickCluster], M = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kPickCluster; ++k) {
+        mk[k] = k < cs ? inbox[(k * g + tid) * IMLD + D] : -INFINITY;
+        M = fmaxf(M, mk[k]);
+      }
+      const float Mu = M == -INFINITY ? 0.f : M;
+      float L = 0.f;
+#pragma unroll
+      for (int k = 0; k < kPickCluster; ++k) {
+        if (k < cs) {
+          const float wgt = ex2_fast(mk[k] - Mu);
+          sm_w[k * g + tid] = wgt;
+          L = fmaf(wgt, inbox[(k * g + tid) * IMLD + D + 1], L);
+        }
+      }
+      sm_L[tid] = L;
+    }
+    // the merging threads: warps 0-2 in a fused step (warp 3 counts the step), else all
+    constexpr int kMergeThreads = FUSED ? kThreads - 32 : kThreads;
+    asm volatile("bar.sync 1, %0;\n" ::"n"(kMergeThreads) : "memory");
+    // four consecutive elements of one row per thread and pass
+    __nv_bfloat16* ob = o + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D;
+    const bool vec_out = (reinterpret_cast<uintptr_t>(ob) & 7) == 0;
+    for (int e4 = tid; e4 < g * (D / 4); e4 += kMergeThreads) {
+      const int r = e4 / (D / 4), d = 4 * (e4 % (D / 4));
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < kPickCluster; ++k) {
+        if (k < cs) {
+          const float wgt = sm_w[k * g + r];
+          const float4 v = *reinterpret_cast<const float4*>(inbox + (k * g + r) * IMLD + d);
+          a.x = fmaf(wgt, v.x, a.x);
+          a.y = fmaf(wgt, v.y, a.y);
+          a.z = fmaf(wgt, v.z, a.z);
+          a.w = fmaf(wgt, v.w, a.w);
+        }
+      }
+      const float L = sm_L[r], inv = L > 0.f ? 1.f / L : 0.f;
+      const uint32_t lo = pack_bf16(a.x * inv, a.y * inv), hi = pack_bf16(a.z * inv, a.w * inv);
+      if (vec_out) {
+        *reinterpret_cast<uint2*>(ob + r * D + d) = make_uint2(lo, hi);
+      } else {
+        const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(&lo);
+        const __nv_bfloat16* ph = reinterpret_cast<const __nv_bfloat16*>(&hi);
+        ob[r * D + d] = pb[0];
+        ob[r * D + d + 1] = pb[1];
+        ob[r * D + d + 2] = ph[0];
+        ob[r * D + d + 3] = ph[1];
+      }
     }
   }
+  DMS_TRACE_MARK(0, 7);
+  DMS_TRACE_MARK(0, 5);
   DMS_TRACE_MARK(0, 6);
 }
 

@@ -142,11 +142,6 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return p;
 }
 
-__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
 // Barrier of the four consumer warps only (the producer warp never joins).
 __device__ __forceinline__ void consumers_sync() { asm volatile("barrier.sync 1, 128;\n" ::: "memory"); }
 
