@@ -9,192 +9,150 @@ __device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
 #endif
 
 // ---------------------------------------------------------------------------
-// Append of token t for every (b, h) of one layer, in one CTA so that page
-// grants follow (b, h) row-major order without inter-CTA ordering:
+// Append of token t for every (b, h) of one layer, one CTA per (b, h):
 //   if t >= w and the token t - w (ring[t % w]) was marked for eviction, the new
 //   token overwrites its slot in place; else it takes slot count++, and a page
 //   is granted from the ascending counter when that slot starts a page
 //   ([DMS-Qwen3], inference mode with the paged KV cache; [FastDMS], decode
 //   kernel: per-step keep/evict, sliding retention window, compact append).
-// The same CTA then writes the K/V rows (FP8: re-encodes the page when the new
-// row raises its scale).
-// With `fuse_decide` the CTA first computes the adapter's decision logits of
-// the new tokens (RMSNorm over the hidden row, one dot product per head, one
-// warp per dot product) and writes them to `alpha`.
+// The decision is the head's plan for position t (slot, flags, count and pages
+// before the append, written by the step before); new pages are numbered from
+// the counter plus the head's rank among the heads needing one, i.e. in (b, h)
+// row-major order (every sequence is at the same position).  The CTA writes the
+// K/V row (FP8: re-encodes the page when the new row raises its scale, every
+// thread of the CTA taking part), the head's state and the plan of position
+// t + 1; the grid's last CTA advances the page counter and the positions.
+// With `fuse_decide` the CTA first computes its head's adapter decision logit
+// (RMSNorm over the hidden row, one dot product) and writes it to `alpha`.
 // ---------------------------------------------------------------------------
-template <typename TA, bool FP8>
-__global__ void __launch_bounds__(1024) k_decode_append(CacheView c, int layer, const TA* k, const TA* v,
-                                                       float* alpha, DecideArgs da, int fuse_decide) {
-  extern __shared__ int sh[];
-  __shared__ int tmp[32];
-  const int BH = c.B * c.Hkv;
-  int* s_slot = sh;          // slot written by head i (-1: dropped)
-  int* s_id = sh + BH;       // page id holding that slot
-  int* s_rows = sh + 2 * BH; // rows in use in that page after the append
-  const long lbase = static_cast<long>(layer) * BH;
-  const int tid = threadIdx.x, bd = blockDim.x, w = c.w, P = c.P;
-  const int lane = tid & 31, wid = tid >> 5, nwarp = bd >> 5;
-  int next = c.ctrl[CTRL_NEXT_PAGE];
-  DMS_TRACE_MARK(1, 0);
+constexpr int kAppendThreads = 128;
 
-  // Phase 0 (optional): decision logits of the new tokens, one warp per
-  // (b, h): the mean square of the hidden row and the dot product with
-  // W_h * gamma in one pass, four 16-byte vectors of each operand in flight.
+template <typename TA, bool FP8>
+__global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, int layer, const TA* k, const TA* v,
+                                                                  float* alpha, DecideArgs da, int fuse_decide) {
+  __shared__ int s_red[32];
+  __shared__ float s_f[2][kAppendThreads / 32];
+  __shared__ int s_last;
+  const int BH = c.B * c.Hkv, bh = blockIdx.x;
+  const int b = bh / c.Hkv, h = bh % c.Hkv;
+  const long lbase = static_cast<long>(layer) * BH, li = lbase + bh;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, w = c.w, P = c.P, D = c.D;
+  DMS_TRACE_MARK(1, 0);
+  // every read of this CTA's state first (one round trip; the plan needs t)
+  const int t = c.pos[layer * c.B + b];
+  const int next_page0 = c.ctrl[CTRL_NEXT_PAGE];
+  const int ring_next = (t + 1 >= w) ? c.ring[li * w + (t + 1) % w] : 0;
+  const int4 pl = *plan_at(c, li, t);
+  const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
+
+  // decision logit of this head (layer granularity: head 0's row of W)
+  float a_dec = 0.f;
   if (fuse_decide) {
     constexpr int V = 16 / sizeof(TA);
     const int hid = c.hidden, nvec = hid / V;
-    const TA* hs = static_cast<const TA*>(da.hidden);
-    const TA* Wt = static_cast<const TA*>(da.W);
-    const TA* gm = static_cast<const TA*>(da.gamma);
-    const TA* bias = static_cast<const TA*>(da.bias);
-    const bool layer_mode = c.alpha_per == DMS_ALPHA_PER_LAYER;
-    const int nh = layer_mode ? 1 : c.Hkv;
-    for (int idx = wid; idx < c.B * nh; idx += nwarp) {
-      const int b = idx / nh, h = idx % nh;
-      const uint4* xr = reinterpret_cast<const uint4*>(hs + static_cast<long>(b) * hid);
-      const uint4* wr = reinterpret_cast<const uint4*>(Wt + static_cast<long>(h) * hid);
-      const uint4* gr = reinterpret_cast<const uint4*>(gm);
-      float ss = 0.f, dot = 0.f;
+    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const TA*>(da.hidden) + static_cast<long>(b) * hid);
+    const uint4* wr = reinterpret_cast<const uint4*>(static_cast<const TA*>(da.W) + static_cast<long>(hs) * hid);
+    const uint4* gr = reinterpret_cast<const uint4*>(da.gamma);
+    float ss = 0.f, dot = 0.f;
 #pragma unroll 4
-      for (int vi = lane; vi < nvec; vi += 32) {
-        const uint4 xu = xr[vi], wu = wr[vi], gu = gr[vi];
-        float x[V], wv[V], gv[V];
-        unpack16(xu, x, static_cast<const TA*>(nullptr));
-        unpack16(wu, wv, static_cast<const TA*>(nullptr));
-        unpack16(gu, gv, static_cast<const TA*>(nullptr));
+    for (int vi = tid; vi < nvec; vi += kAppendThreads) {
+      const uint4 xu = xr[vi], wu = wr[vi], gu = gr[vi];
+      float x[V], wv[V], gv[V];
+      unpack16(xu, x, static_cast<const TA*>(nullptr));
+      unpack16(wu, wv, static_cast<const TA*>(nullptr));
+      unpack16(gu, gv, static_cast<const TA*>(nullptr));
 #pragma unroll
-        for (int e = 0; e < V; ++e) {
-          ss = fmaf(x[e], x[e], ss);
-          dot = fmaf(wv[e] * gv[e], x[e], dot);
-        }
+      for (int e = 0; e < V; ++e) {
+        ss = fmaf(x[e], x[e], ss);
+        dot = fmaf(wv[e] * gv[e], x[e], dot);
       }
+    }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    }
+    if (lane == 0) {
+      s_f[0][wid] = ss;
+      s_f[1][wid] = dot;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      float s2 = 0.f, d2 = 0.f;
+      for (int i = 0; i < kAppendThreads / 32; ++i) {
+        s2 += s_f[0][i];
+        d2 += s_f[1][i];
       }
-      if (lane == 0) {
-        const float inv = 1.0f / sqrtf(ss / static_cast<float>(hid) + c.rms_eps);
-        const float z = dot * inv + (bias ? to_f(bias[h]) : 0.f);
-        const float a = z * c.alpha_scale - da.offset[b * da.offset_bstride + h];
-        if (layer_mode)
-          for (int hh = 0; hh < c.Hkv; ++hh) alpha[b * c.Hkv + hh] = a;
-        else
-          alpha[b * c.Hkv + h] = a;
-      }
+      const TA* bias = static_cast<const TA*>(da.bias);
+      const float inv = 1.0f / sqrtf(s2 / static_cast<float>(hid) + c.rms_eps);
+      const float z = d2 * inv + (bias ? to_f(bias[hs]) : 0.f);
+      a_dec = z * c.alpha_scale - da.offset[b * da.offset_bstride + hs];
+      alpha[b * c.Hkv + h] = a_dec;
     }
     __syncthreads();
   }
   DMS_TRACE_MARK(1, 1);
-  // Phase 1: slots and page grants
-  for (int i0 = 0; i0 < BH; i0 += bd) {
-    const int i = i0 + tid;
-    int need = 0, slot = -1, cnt = 0, have = 0;
-    bool reuse = false, evict = false;
-    const long li = lbase + i;
-    int t = 0;
-    if (i < BH) {
-      const int b = i / c.Hkv, h = i % c.Hkv;
-      t = c.pos[layer * c.B + b];  // position of the new token
-      const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
-      evict = !c.disable && alpha[b * c.Hkv + hs] > 0.0f;
-      const int ringv = t >= w ? c.ring[li * w + t % w] : 0;
-      reuse = t >= w && (static_cast<unsigned>(ringv) & RING_EVICT);
-      cnt = c.count[li];
-      have = c.npages[li];
-      if (reuse) {
-        slot = ringv & RING_SLOT_MASK;
-      } else if (cnt >= c.cap) {
-        set_status(c.ctrl, DMS_ST_CAPACITY);
-      } else {
-        slot = cnt;
-        need = (cnt % P == 0 && cnt / P >= have) ? 1 : 0;
-      }
-    }
-    int tot;
-    const int off = block_exclusive_scan(need, tmp, &tot);
-    if (i < BH) {
-      int id = -1;
-      bool ok = slot >= 0;
-      if (ok && need) {
-        id = next + off;
-        if (id < c.pool_pages && have < c.maxp) {
-          c.page_table[li * c.maxp + have] = id;
-          c.npages[li] = have + 1;
-        } else {
-          set_status(c.ctrl, DMS_ST_POOL_EXHAUSTED);
-          ok = false;
-        }
-      }
-      if (ok) {
-        const int newcnt = reuse ? cnt : cnt + 1;
-        if (!reuse) c.count[li] = newcnt;
-        const int p = slot / P;
-        s_slot[i] = slot;
-        s_id[i] = need ? id : c.page_table[li * c.maxp + p];
-        s_rows[i] = min(P, newcnt - p * P);
-        c.slot_pos[li * c.cap + slot] = t;
-        c.ring[li * w + t % w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
-      } else {
-        s_slot[i] = -1;
-      }
-    }
-    next += tot;
-  }
-  if (tid == 0) c.ctrl[CTRL_NEXT_PAGE] = min(next, c.pool_pages);
-  __syncthreads();  // every head has read its position
-  for (int b = tid; b < c.B; b += bd) c.pos[layer * c.B + b] += 1;
 
-  DMS_TRACE_MARK(1, 2);
-  // Phase 2: K/V rows, one warp per head
-  const int D = c.D;
-  for (int i = wid; i < BH; i += nwarp) {
-    const int slot = s_slot[i];
-    if (slot < 0) continue;
-    const int id = s_id[i];
+  // rank among the lower heads needing a new page (their plans for t)
+  const int flags = pl.y, slot = pl.x, cnt = pl.z, have = pl.w;
+  int id = -1;
+  bool ok = !(flags & 4);
+  if (ok && (flags & 2)) {
+    int n_before = 0;
+    for (int i = tid; i < bh; i += kAppendThreads) n_before += (plan_at(c, lbase + i, t)->y & 2) ? 1 : 0;
+    int tot;  // lower heads needing a page
+    block_exclusive_scan(n_before, s_red, &tot);
+    id = next_page0 + tot;
+    if (id >= c.pool_pages || have >= c.maxp) ok = false;
+  } else if (ok) {
+    id = c.page_table[li * c.maxp + slot / P];
+  }
+  const int cnt_new = (ok && !(flags & 1)) ? cnt + 1 : cnt, np_new = (ok && (flags & 2)) ? have + 1 : have;
+
+  if (ok) {
     const long dst_row = static_cast<long>(id) * P + slot % P;
-    const TA* ksrc = k + static_cast<long>(i) * D;
-    const TA* vsrc = v + static_cast<long>(i) * D;
+    const TA* ksrc = k + static_cast<long>(bh) * D;
+    const TA* vsrc = v + static_cast<long>(bh) * D;
     if (!FP8) {
       const int cpr = D * static_cast<int>(sizeof(TA)) / 16;
-      if (lane < cpr) {
-        reinterpret_cast<uint4*>(static_cast<TA*>(c.k_pool) + dst_row * D)[lane] =
-            reinterpret_cast<const uint4*>(ksrc)[lane];
-        reinterpret_cast<uint4*>(static_cast<TA*>(c.v_pool) + dst_row * D)[lane] =
-            reinterpret_cast<const uint4*>(vsrc)[lane];
+      if (tid < cpr) {
+        reinterpret_cast<uint4*>(static_cast<TA*>(c.k_pool) + dst_row * D)[tid] =
+            reinterpret_cast<const uint4*>(ksrc)[tid];
+        reinterpret_cast<uint4*>(static_cast<TA*>(c.v_pool) + dst_row * D)[tid] =
+            reinterpret_cast<const uint4*>(vsrc)[tid];
       }
     } else {
-      const int rows = s_rows[i];
+      const int rows = min(P, cnt_new - (slot / P) * P);  // rows in use in that page after the append
       for (int which = 0; which < 2; ++which) {
         const TA* x = which ? vsrc : ksrc;
         float* scale_p = (which ? c.v_scale : c.k_scale) + id;
         uint8_t* page = static_cast<uint8_t*>(which ? c.v_pool : c.k_pool) + static_cast<long>(id) * P * D;
-        float xv[4];
-        float amax = 0.f;
-        for (int e = 0; e < D / 32; ++e) {
-          xv[e] = to_f(x[lane + 32 * e]);
-          amax = fmaxf(amax, fabsf(xv[e]));
-        }
+        const float xv = tid < D ? to_f(x[tid]) : 0.f;
+        float amax = fabsf(xv);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0) s_f[0][wid] = amax;
+        __syncthreads();
+        amax = 0.f;
+        for (int i = 0; i < kAppendThreads / 32; ++i) amax = fmaxf(amax, s_f[0][i]);
         const float s_new = __fdiv_rn(amax, 448.0f);
         const float s_old = *scale_p;
         float scale = s_old;
         if (s_new > s_old) {
           // re-encode the page's rows at the larger scale from their decoded
-          // values, 16 codes per lane and four vectors in flight
+          // values, 16 codes per thread and vector, four vectors in flight
           uint4* pv = reinterpret_cast<uint4*>(page);
           const int nvec = rows * D / 16;
-          for (int v0 = 0; v0 < nvec; v0 += 4 * 32) {
+          for (int v0 = 0; v0 < nvec; v0 += 4 * kAppendThreads) {
             uint4 u[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int vi = v0 + e * 32 + lane;
+              const int vi = v0 + e * kAppendThreads + tid;
               if (vi < nvec) u[e] = pv[vi];
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int vi = v0 + e * 32 + lane;
+              const int vi = v0 + e * kAppendThreads + tid;
               if (vi >= nvec) continue;
               uint8_t* cb = reinterpret_cast<uint8_t*>(&u[e]);
 #pragma unroll
@@ -203,51 +161,66 @@ __global__ void __launch_bounds__(1024) k_decode_append(CacheView c, int layer, 
             }
           }
           scale = s_new;
-          __syncwarp();
-          if (lane == 0) *scale_p = s_new;
+          __syncthreads();  // every code re-encoded before the row and the scale
+          if (tid == 0) *scale_p = s_new;
         }
-        for (int e = 0; e < D / 32; ++e)
-          page[static_cast<long>(slot % P) * D + lane + 32 * e] = scale > 0.f ? fp8_encode(__fdiv_rn(xv[e], scale)) : 0;
+        if (tid < D) page[static_cast<long>(slot % P) * D + tid] = scale > 0.f ? fp8_encode(__fdiv_rn(xv, scale)) : 0;
+        __syncthreads();  // s_f reused
       }
     }
   }
-
-  // Phase 3: slot plan of the next append of every head (read by the fused
-  // decode kernel).
+  if (tid == 0) {
+    if (ok) {
+      if (flags & 2) {
+        c.page_table[li * c.maxp + have] = id;
+        c.npages[li] = np_new;
+        atomicAdd(&c.ctrl[CTRL_STEP_PAGES], 1);
+      }
+      if (!(flags & 1)) c.count[li] = cnt_new;
+      const float a = fuse_decide ? a_dec : alpha[b * c.Hkv + hs];
+      const bool evict = !c.disable && a > 0.0f;
+      c.slot_pos[li * c.cap + slot] = t;
+      c.ring[li * w + t % w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
+    } else {
+      set_status(c.ctrl, (flags & 4) ? DMS_ST_CAPACITY : DMS_ST_POOL_EXHAUSTED);
+    }
+    // the plan of position t + 1 from the values just written
+    *plan_at(c, li, t + 1) = make_plan(ring_next, t + 1, cnt_new, np_new, c);
+    // the grid's last CTA advances the page counter and the positions (every
+    // CTA has read them by the time it counts itself)
+    __threadfence();
+    s_last = atomicAdd(&c.ctrl[CTRL_GRID_DONE], 1) == BH - 1;
+  }
   __syncthreads();
-  for (int i = tid; i < BH; i += bd) {
-    const int b = i / c.Hkv;
-    const int tn = c.pos[layer * c.B + b];
-    *plan_at(c, lbase + i, tn) = next_plan(c, lbase + i, tn);
+  if (s_last) {
+    if (tid == 0) {
+      __threadfence();
+      const int granted = __ldcg(&c.ctrl[CTRL_STEP_PAGES]);
+      c.ctrl[CTRL_NEXT_PAGE] = min(__ldcg(&c.ctrl[CTRL_NEXT_PAGE]) + granted, c.pool_pages);
+      c.ctrl[CTRL_STEP_PAGES] = 0;
+      c.ctrl[CTRL_GRID_DONE] = 0;
+    }
+    for (int bb = tid; bb < c.B; bb += kAppendThreads) c.pos[layer * c.B + bb] += 1;
   }
   DMS_TRACE_MARK(1, 3);
 }
 
 template <typename TA, bool FP8>
 static cudaError_t launch_append_t(const CacheView& c, int layer, const void* k, const void* v, float* alpha,
-                                   const DecideArgs* da, int threads, size_t smem, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(k_decode_append<TA, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+                                   const DecideArgs* da, cudaStream_t s) {
   DecideArgs none{};
-  k_decode_append<TA, FP8><<<1, threads, smem, s>>>(c, layer, static_cast<const TA*>(k), static_cast<const TA*>(v),
-                                                    alpha, da ? *da : none, da ? 1 : 0);
+  k_decode_append<TA, FP8><<<c.B * c.Hkv, kAppendThreads, 0, s>>>(c, layer, static_cast<const TA*>(k),
+                                                                  static_cast<const TA*>(v), alpha, da ? *da : none,
+                                                                  da ? 1 : 0);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, const void* v, float* alpha,
                                  const DecideArgs* fused_decide, int num_sms, cudaStream_t s) {
-  const int BH = c.B * c.Hkv;
   (void)num_sms;
-  // one warp per head for the K/V rows (an FP8 page re-encode is a few
-  // round trips of its own), up to 32 warps
-  const int threads = min(1024, max(256, 32 * BH));
-  const size_t smem = static_cast<size_t>(BH) * 3 * sizeof(int);
-  if (c.kv_dtype == DMS_FP8_E4M3)
-    return launch_append_t<__nv_bfloat16, true>(c, layer, k, v, alpha, fused_decide, threads, smem, s);
-  if (c.kv_dtype == DMS_BF16)
-    return launch_append_t<__nv_bfloat16, false>(c, layer, k, v, alpha, fused_decide, threads, smem, s);
-  return launch_append_t<float, false>(c, layer, k, v, alpha, fused_decide, threads, smem, s);
+  if (c.kv_dtype == DMS_FP8_E4M3) return launch_append_t<__nv_bfloat16, true>(c, layer, k, v, alpha, fused_decide, s);
+  if (c.kv_dtype == DMS_BF16) return launch_append_t<__nv_bfloat16, false>(c, layer, k, v, alpha, fused_decide, s);
+  return launch_append_t<float, false>(c, layer, k, v, alpha, fused_decide, s);
 }
 
 // ---------------------------------------------------------------------------
