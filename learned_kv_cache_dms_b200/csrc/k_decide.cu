@@ -498,9 +498,105 @@ __global__ void k_neuron_rope(CacheView c, int T, const int* pos_dev, TA* q, TA*
   }
 }
 
+// Four consecutive pairs (i .. i+3 < D/2) of one row per thread and step: the
+// same arithmetic as above with 8- or 16-byte accesses (rotary tables given;
+// rows and tables 16-byte aligned).
+template <typename TA>
+__device__ __forceinline__ void ld4(const TA* p, float* f);
+template <>
+__device__ __forceinline__ void ld4<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  f[0] = a.x;
+  f[1] = a.y;
+  f[2] = b.x;
+  f[3] = b.y;
+}
+template <>
+__device__ __forceinline__ void ld4<float>(const float* p, float* f) {
+  const float4 u = *reinterpret_cast<const float4*>(p);
+  f[0] = u.x;
+  f[1] = u.y;
+  f[2] = u.z;
+  f[3] = u.w;
+}
+template <typename TA>
+__device__ __forceinline__ void st4(TA* p, const float* f);
+template <>
+__device__ __forceinline__ void st4<__nv_bfloat16>(__nv_bfloat16* p, const float* f) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+}
+template <>
+__device__ __forceinline__ void st4<float>(float* p, const float* f) {
+  *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+}
+
+template <typename TA>
+__global__ void k_neuron_rope4(CacheView c, int T, const int* pos_dev, TA* q, TA* k, const float* offset, int ostride,
+                               int do_alpha, float* alpha, const float* cos_t, const float* sin_t) {
+  const int D = c.D, half = D / 2, nq = half / 4, g = c.Hq / c.Hkv;
+  const bool key = c.alpha_source == DMS_ALPHA_KEY_NEURON;
+  const int nrow = c.Hq + c.Hkv;
+  const long total = static_cast<long>(c.B) * T * nrow * nq;
+  for (long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<long>(gridDim.x) * blockDim.x) {
+    const int i = static_cast<int>(idx % nq) * 4;
+    const long rt = idx / nq;
+    const int r = static_cast<int>(rt % nrow);
+    const long tok = rt / nrow;
+    const int b = static_cast<int>(tok / T), t = static_cast<int>(tok % T);
+    TA* row = r < c.Hq ? q + (tok * c.Hq + r) * D : k + (tok * c.Hkv + (r - c.Hq)) * D;
+    float x0[4], x1[4], cv[4], sv[4];
+    ld4<TA>(row + i, x0);
+    ld4<TA>(row + i + half, x1);
+    const int p = pos_dev ? pos_dev[b] + t : t;
+    ld4<float>(cos_t + static_cast<long>(p) * half + i, cv);
+    ld4<float>(sin_t + static_cast<long>(p) * half + i, sv);
+    // the decision neuron (pair half - 1: the last element of the row) is
+    // read, then zeroed, before the rotation
+    const bool neuron_row = key ? r >= c.Hq : (r < c.Hq && r % g == 0);
+    if (do_alpha && neuron_row && i + 3 == half - 1) {
+      const int h = key ? r - c.Hq : r / g;
+      if (c.alpha_per == DMS_ALPHA_PER_LAYER) {
+        if (h == 0) {
+          const float a = fmaf(x1[3], c.alpha_scale, -offset[b * ostride]);
+          for (int hh = 0; hh < c.Hkv; ++hh) alpha[(static_cast<long>(b) * c.Hkv + hh) * T + t] = a;
+        }
+      } else {
+        alpha[(static_cast<long>(b) * c.Hkv + h) * T + t] = fmaf(x1[3], c.alpha_scale, -offset[b * ostride + h]);
+      }
+      x1[3] = 0.f;
+    }
+    float y0[4], y1[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      // each product and sum rounded separately (no fused multiply-add)
+      y0[e] = __fsub_rn(__fmul_rn(x0[e], cv[e]), __fmul_rn(x1[e], sv[e]));
+      y1[e] = __fadd_rn(__fmul_rn(x1[e], cv[e]), __fmul_rn(x0[e], sv[e]));
+    }
+    st4<TA>(row + i, y0);
+    st4<TA>(row + i + half, y1);
+  }
+}
+
 cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
                                int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
                                const float* sin_t, cudaStream_t s) {
+  const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                       reinterpret_cast<uintptr_t>(cos_t) | reinterpret_cast<uintptr_t>(sin_t);
+  if (cos_t && (al & 15) == 0 && (c.D / 2) % 4 == 0) {
+    const long total4 = static_cast<long>(c.B) * T * (c.Hq + c.Hkv) * (c.D / 8);
+    const int grid4 = static_cast<int>(max(1L, min((total4 + 255) / 256, static_cast<long>(c.num_sms) * 16)));
+    if (c.act_dtype == DMS_BF16)
+      k_neuron_rope4<__nv_bfloat16><<<grid4, 256, 0, s>>>(c, T, pos_dev, static_cast<__nv_bfloat16*>(q),
+                                                           static_cast<__nv_bfloat16*>(k), offset, offset_bstride,
+                                                           do_alpha ? 1 : 0, alpha, cos_t, sin_t);
+    else
+      k_neuron_rope4<float><<<grid4, 256, 0, s>>>(c, T, pos_dev, static_cast<float*>(q), static_cast<float*>(k),
+                                                  offset, offset_bstride, do_alpha ? 1 : 0, alpha, cos_t, sin_t);
+    return cudaGetLastError();
+  }
   const long total = static_cast<long>(c.B) * T * (cos_t ? (c.Hq + c.Hkv) * (c.D / 2) : c.Hkv);
   const int grid = static_cast<int>(max(1L, min((total + 255) / 256, static_cast<long>(c.num_sms) * 16)));
   if (c.act_dtype == DMS_BF16)
