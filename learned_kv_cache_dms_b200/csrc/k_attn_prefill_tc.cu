@@ -127,33 +127,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-#ifndef DMS_PF_POLY_PAIRS
-#define DMS_PF_POLY_PAIRS 0  // of every 8 pairs of exponentials, how many run on the FMA pipe
-#endif
-#ifndef DMS_PF_PACK_INT
-#define DMS_PF_PACK_INT 0
-#endif
-
-// 2^x on the FMA pipe: x = j + f with j = round(x), |f| <= 1/2 (the 1.5 * 2^23
-// shifter leaves j in the low mantissa bits), 2^f from a cubic fitted to it on
-// [-1/2, 1/2] (relative error 7.5e-5, below P's bf16 rounding), 2^j added to
-// the exponent field.  x is clamped to -125 so the result stays a normal
-// float (invisible scores, -inf, give 2^-125, below anything a visible key
-// contributes to a row sum of at least 1).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = __fadd_rn(x, 12582912.f);
-  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
-  const float p = fmaf(fmaf(fmaf(0.0551716611f, f, 0.24261114f), f, 0.693260968f), f, 0.999928057f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// two non-negative finite floats to bf16 (round half away from zero) with
-// integer operations: a's high half in the low 16 bits, b's in the high
-__device__ __forceinline__ uint32_t pack_bf16_pos(float a, float b) {
-  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
-}
-
 // paired fp32 arithmetic (one instruction for two lanes of a 64-bit pair)
 __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
   uint64_t r;
@@ -177,22 +150,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// ex2_poly on a pair with paired arithmetic
-__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& p0, float& p1) {
-  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t sh = f2_pack(12582912.f, 12582912.f);
-  const uint64_t t = f2_add(x, sh);
-  const uint64_t f = f2_fma(f2_add(t, f2_pack(-12582912.f, -12582912.f)), f2_pack(-1.f, -1.f), x);
-  const uint64_t q = f2_fma(f2_fma(f2_fma(f2_pack(0.0551716611f, 0.0551716611f), f, f2_pack(0.24261114f, 0.24261114f)), f,
-                                   f2_pack(0.693260968f, 0.693260968f)),
-                            f, f2_pack(0.999928057f, 0.999928057f));
-  float q0, q1, t0, t1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(t, t0, t1);
-  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane, without waiting.
@@ -574,15 +531,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int e = 0; e < kPfBN / 2; ++e) {
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), sl2x2, nm2), x0, x1);
-          float p0, p1;
-          if ((e & 7) < DMS_PF_POLY_PAIRS) {
-            ex2_poly2(x0, x1, p0, p1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           ps4[e & 3] = f2_add(ps4[e & 3], f2_pack(p0, p1));
-          pk[e] = DMS_PF_PACK_INT ? pack_bf16_pos(p0, p1) : pack_bf16(p0, p1);
+          pk[e] = pack_bf16(p0, p1);
         }
         float s_even, s_odd;
         f2_unpack(f2_add(f2_add(ps4[0], ps4[1]), f2_add(ps4[2], ps4[3])), s_even, s_odd);
