@@ -236,23 +236,26 @@ __global__ void __launch_bounds__(256) k_decide_proj_row(CacheView c, DecideArgs
 // [16 (w % 4), +16) of the even (w < 4) or odd chunks of the hidden size; the
 // two halves are added through shared memory at the end of the tile.
 // ---------------------------------------------------------------------------
-constexpr int kDpTok = 64, kDpK = 64, kDpStages = 8, kDpWarps = 8;
+constexpr int kDpTok = 64, kDpK = 128, kDpStages = 4, kDpWarps = 8;  // a stage: two 64-element boxes
 constexpr int kDpThreads = (kDpWarps + 1) * 32;
 
-__host__ __device__ inline int dp_wrow(int hid) { return hid + 8; }  // table row (bf16), 16-byte pad
+// table row (bf16): the hidden size rounded up to whole chunks (zero-filled,
+// so the last chunk's columns past the hidden size read zeros) plus a
+// 16-byte pad that keeps the ldmatrix rows on distinct banks
+__host__ __device__ inline int dp_wrow(int hid) { return (hid + kDpK - 1) / kDpK * kDpK + 8; }
 // byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled TMA tile
 __device__ __forceinline__ uint32_t dp_sw128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 __host__ __device__ inline size_t dp_smem(int hid) {
-  return 1024 + static_cast<size_t>(kDpStages) * kDpTok * 128 + 2ull * 8 * dp_wrow(hid) * 2;
+  return 1024 + static_cast<size_t>(kDpStages) * kDpTok * 2 * kDpK + 2ull * 8 * dp_wrow(hid) * 2;
 }
 
 __global__ void __launch_bounds__(kDpThreads, 1)
     k_decide_proj_tc(CacheView c, int T, DecideArgs a, float* alpha, const __grid_constant__ CUtensorMap hmap) {
   extern __shared__ __align__(1024) unsigned char dp_raw[];
   unsigned char* sb = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dp_raw) + 1023) & ~uintptr_t(1023));
-  __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(sb + kDpStages * kDpTok * 128);  // [2][8][wrow]
+  __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(sb + kDpStages * kDpTok * 2 * kDpK);  // [2][8][wrow]
   __shared__ __align__(8) uint64_t full[kDpStages], empty[kDpStages];
   __shared__ float red[4][6][32];  // odd-chunk halves: acc[4], ss[2] per lane of warps 4..7
   const int H = c.Hkv, hid = c.hidden, wrow = dp_wrow(hid);
@@ -306,8 +309,10 @@ __global__ void __launch_bounds__(kDpThreads, 1)
             set_status(c.ctrl, DMS_ST_TIMEOUT);
             return;
           }
-          mbar_expect_tx(&full[st], kDpTok * 128);
-          tma_load_2d(sb + st * kDpTok * 128, &hmap, kc * kDpK, tile * kDpTok, &full[st]);
+          mbar_expect_tx(&full[st], kDpTok * 2 * kDpK);
+          for (int hb = 0; hb < kDpK / 64; ++hb)
+            tma_load_2d(sb + st * kDpTok * 2 * kDpK + hb * kDpTok * 128, &hmap, kc * kDpK + 64 * hb, tile * kDpTok,
+                        &full[st]);
         }
     }
     return;
@@ -332,11 +337,12 @@ __global__ void __launch_bounds__(kDpThreads, 1)
         if (lane == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
       }
       if (ok) {
-        const uint32_t xs = smem_u32(sb + st * kDpTok * 128);
+        const uint32_t xs = smem_u32(sb + st * kDpTok * 2 * kDpK);
 #pragma unroll
         for (int ks = 0; ks < kDpK / 16; ++ks) {
           uint32_t af[4], bf[4];
-          ldmatrix_x4(af[0], af[1], af[2], af[3], xs + dp_sw128(arow, 2 * ks + (mi >> 1)));
+          ldmatrix_x4(af[0], af[1], af[2], af[3],
+                      xs + (ks / 4) * (kDpTok * 128) + dp_sw128(arow, 2 * (ks % 4) + (mi >> 1)));
           ldmatrix_x4(bf[0], bf[1], bf[2], bf[3], wbase + 2u * static_cast<uint32_t>(kc * kDpK + ks * 16));
           mma_bf16_16816(acc, af, bf);
           mma_bf16_16816(acc, af, bf + 2);

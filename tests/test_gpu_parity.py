@@ -17,6 +17,9 @@ CASES = {
                                    source="input", keep=0.3, prealloc=64, seed=2),
     "bf16_d128_proj": Case(B=2, T=515, steps=24, Hq=8, Hkv=4, D=128, hidden=512, w=96, P=32, act="bf16",
                            kv="bf16", source="proj", keep=(1 / 16, 1 / 4), seed=3),
+    # a hidden size that is a multiple of 8 but not of the adapter kernel's chunks
+    "bf16_proj_hidden_ragged": Case(B=2, T=300, steps=12, Hq=8, Hkv=4, D=64, hidden=328, w=64, P=32, act="bf16",
+                                    kv="bf16", source="proj", keep=0.25, seed=31),
     "bf16_d64_proj_layer": Case(B=2, T=333, steps=20, Hq=4, Hkv=4, D=64, hidden=256, w=48, P=16, act="bf16",
                                 kv="bf16", source="proj", per="layer", keep=0.25, seed=4),
     "fp8_key_rope_head": Case(B=2, T=700, steps=30, Hq=8, Hkv=2, D=64, w=64, P=32, act="bf16", kv="fp8",
