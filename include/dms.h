@@ -247,6 +247,31 @@ DMS_API int dms_cache_reset(dms_cache* cache, void* stream);
 /* Offsets of the cache's arrays in the caller buffer. */
 DMS_API int dms_cache_get_layout(const dms_cache* cache, dms_cache_layout* layout);
 
+/* ---- state export -----------------------------------------------------------------
+ * Host copies of one layer's cache state ([DMS-Qwen3], inference mode with the
+ * paged KV cache: what the append rule maintains).  Every pointer is a
+ * caller-owned host buffer of the size given (B = batch, H = num_kv_heads,
+ * maxp and cap from dms_cache_get_layout, w = window), or NULL to skip it:
+ *   pos        [B]            tokens appended so far per sequence
+ *   count      [B,H]          retained slots per head
+ *   npages     [B,H]          pages owned per head
+ *   page_table [B,H,maxp]     page ids (-1 past npages)
+ *   slot_pos   [B,H,cap]      position held by each slot (entries past count undefined)
+ *   ring       [B,H,w]        slot of position t at t % w, bit 31 = its eviction decision */
+typedef struct dms_cache_view {
+  int* pos;
+  int* count;
+  int* npages;
+  int* page_table;
+  int* slot_pos;
+  int* ring;
+} dms_cache_view;
+
+/* Copy layer `layer`'s state into `out` after the work already on `stream`
+ * (synchronises the stream).  DMS_ERR_INVALID for a bad handle or layer,
+ * DMS_ERR_CUDA if a copy fails. */
+DMS_API int dms_cache_export(dms_cache* cache, int layer, dms_cache_view* out, void* stream);
+
 /* Read the sticky device status word (DMS_ST_* bits).  Synchronises `stream`. */
 DMS_API int dms_cache_status(dms_cache* cache, void* stream, int* status);
 

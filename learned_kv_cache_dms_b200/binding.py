@@ -48,6 +48,10 @@ class dms_cache_desc(C.Structure):
                ("decode_kernel", C.c_int)]
 
 
+class dms_cache_view(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("pos", "count", "npages", "page_table", "slot_pos", "ring")]
+
+
 class dms_cache_layout(C.Structure):
     _fields_ = [(n, C.c_size_t) for n in ("total_bytes", "status", "next_page", "pos", "count", "npages",
                                           "page_table", "slot_pos", "ring", "k_pool", "v_pool", "k_scale",
@@ -80,6 +84,7 @@ _lib.dms_cache_free.argtypes = [_P]
 _lib.dms_cache_reset.argtypes = [_P, _P]
 _lib.dms_cache_get_layout.argtypes = [_P, C.POINTER(dms_cache_layout)]
 _lib.dms_cache_status.argtypes = [_P, _P, C.POINTER(C.c_int)]
+_lib.dms_cache_export.argtypes = [_P, C.c_int, C.POINTER(dms_cache_view), _P]
 _lib.dms_decide.argtypes = [_P, C.c_int, C.POINTER(dms_decide_params), _P, _P, _P]
 _lib.dms_prefill.argtypes = [_P, C.c_int, C.POINTER(dms_prefill_args), _P]
 _lib.dms_decode_step.argtypes = [_P, C.c_int, C.POINTER(dms_decode_args), _P]
@@ -92,13 +97,13 @@ _lib.dms_cache_positions.argtypes = [_P, C.c_int]
 for _f in ("dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset", "dms_cache_get_layout",
            "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step", "dms_cache_positions",
            "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append", "dms_decode_attention",
-           "dms_decode_attention_noalloc"):
+           "dms_decode_attention_noalloc", "dms_cache_export"):
     getattr(_lib, _f).restype = C.c_int
 
 EXPORTED = ("dms_cache_desc_default", "dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset",
             "dms_cache_get_layout", "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step",
             "dms_cache_positions", "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append",
-            "dms_decode_attention", "dms_decode_attention_noalloc")
+            "dms_decode_attention", "dms_decode_attention_noalloc", "dms_cache_export")
 
 
 def _check(code, where):
@@ -152,6 +157,21 @@ def dms_cache_get_layout(handle: int) -> dms_cache_layout:
     l = dms_cache_layout()
     _check(_lib.dms_cache_get_layout(handle, C.byref(l)), "dms_cache_get_layout")
     return l
+
+
+def dms_cache_export(handle: int, layer: int, desc, layout, stream=None) -> dict:
+    """Host (numpy int32) copies of one layer's state: pos [B], count and
+    npages [B,Hkv], page_table [B,Hkv,maxp], slot_pos [B,Hkv,cap], ring
+    [B,Hkv,w] (bit 31: eviction decision)."""
+    import numpy as np
+    B, H, w = desc.batch, desc.num_kv_heads, desc.window
+    maxp, cap = layout.max_pages_per_head, layout.slot_capacity
+    out = dict(pos=np.zeros(B, np.int32), count=np.zeros((B, H), np.int32), npages=np.zeros((B, H), np.int32),
+               page_table=np.zeros((B, H, maxp), np.int32), slot_pos=np.zeros((B, H, cap), np.int32),
+               ring=np.zeros((B, H, w), np.int32))
+    v = dms_cache_view(*[out[k].ctypes.data for k in ("pos", "count", "npages", "page_table", "slot_pos", "ring")])
+    _check(_lib.dms_cache_export(handle, layer, C.byref(v), _stream(stream)), "dms_cache_export")
+    return out
 
 
 def dms_cache_status(handle: int, stream=None) -> int:
@@ -288,6 +308,10 @@ class Cache:
             next_page=self._view(l.next_page, 1, i32),
             status=self._view(l.status, 1, i32),
         )
+
+    def export(self, layer: int, stream=None) -> dict:
+        """dms_cache_export of one layer (host numpy copies)."""
+        return dms_cache_export(self.handle, layer, self.desc, self.layout, stream)
 
     def counts(self):
         """Retained lengths of every layer, [L, B, Hkv] int32 (a view of the cache)."""

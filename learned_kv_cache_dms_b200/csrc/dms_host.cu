@@ -370,6 +370,24 @@ int dms_cache_get_layout(const dms_cache* c, dms_cache_layout* l) {
   return DMS_OK;
 }
 
+int dms_cache_export(dms_cache* c, int layer, dms_cache_view* out, void* stream) {
+  if (!c || !out || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const CacheView& v = c->view;
+  const long nb = static_cast<long>(v.B) * v.Hkv, lbase = static_cast<long>(layer) * nb;
+  // one plain copy per array (layer slices are contiguous)
+  auto copy = [&](void* dst, const int* src, long n) -> bool {
+    return !dst || cudaMemcpyAsync(dst, src, n * sizeof(int), cudaMemcpyDeviceToHost, s) == cudaSuccess;
+  };
+  const bool ok = copy(out->pos, v.pos + static_cast<long>(layer) * v.B, v.B) && copy(out->count, v.count + lbase, nb) &&
+                  copy(out->npages, v.npages + lbase, nb) &&
+                  copy(out->page_table, v.page_table + lbase * v.maxp, nb * v.maxp) &&
+                  copy(out->slot_pos, v.slot_pos + lbase * v.cap, nb * v.cap) &&
+                  copy(out->ring, v.ring + lbase * v.w, nb * v.w);
+  if (!ok || cudaStreamSynchronize(s) != cudaSuccess) return DMS_ERR_CUDA;
+  return DMS_OK;
+}
+
 int dms_cache_status(dms_cache* c, void* stream, int* status) {
   if (!c || !status) return DMS_ERR_INVALID;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
