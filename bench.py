@@ -481,6 +481,37 @@ def decode_step_bytes(wl, retained):
     return retained * D * 2 * elem + pages * per_page + fixed
 
 
+def measure_prefill_parts(B_, r, wl, passes=3):
+    """The decision logits (dms_decide) and the compaction (dms_prefill_compact)
+    of one (replica, layer) timed on their own, each after an L2 flush (a
+    512 MB write), the cache reset and the prompt restored before each pass.
+    Returns (decide ms or None for neuron sources, compaction ms), medians."""
+    u = r.units[0]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    alpha = torch.empty_like(u["alpha"])
+    proj = wl.alpha_source == "proj"
+    dec, comp = [], []
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for i in range(passes):
+        r.reset_all()
+        r.restore_prompt()
+        if proj:
+            flush.fill_(i)
+            ev[0].record()
+            B_.dms_decide(u["h"], wl.prompt, u["pargs"].decide.contents, None, alpha)
+            ev[1].record()
+            torch.cuda.synchronize()
+            dec.append(ev[0].elapsed_time(ev[1]))
+        flush.fill_(i + 100)
+        ev[0].record()
+        B_.dms_prefill_compact(u["h"], u["l"], u["pargs"])
+        ev[1].record()
+        torch.cuda.synchronize()
+        comp.append(ev[0].elapsed_time(ev[1]))
+    med = lambda x: sorted(x)[len(x) // 2]
+    return (med(dec) if proj else None), med(comp)
+
+
 def run_ours(args, world, rank, local):
     from learned_kv_cache_dms_b200 import binding as B_
     wl = I.WORKLOADS[args.workload]
@@ -542,6 +573,30 @@ def run_ours(args, world, rank, local):
     prefill_tflops = K * R * prefill_flops / (prefill_attn_ms / 1e3) / 1e12
     clocks = clk.summary()
 
+    # decision logits (A1) and compaction (A2) on their own, L2-cold
+    dec_ms1, comp_ms1 = measure_prefill_parts(B_, r, wl)
+    T_ = wl.prompt
+    ret_prefill = counts[0] / L  # retained slots of one layer after the prefill
+    kv_in = 2  # bf16 K/V input rows
+    kv_page = 1 if wl.kv_dtype == "fp8" else 2
+    dec_bytes = B * T_ * wl.hidden * 2 + wl.kv_heads * wl.hidden * 2 + wl.hidden * 2 + B * wl.kv_heads * T_ * 4
+    comp_bytes = B * wl.kv_heads * T_ * 4 + ret_prefill * wl.head_dim * 2 * (kv_in + kv_page)
+    neuron_pass = wl.alpha_source != "proj"
+    if neuron_pass:  # q and k rewritten in place by the neuron/rotary pass, inside the compaction call
+        comp_bytes += 2 * B * T_ * (wl.q_heads + wl.kv_heads) * wl.head_dim * 2
+    comp_only_ms = comp_ms1 - (dec_ms1 or 0.0)
+    decide_roof = None if dec_ms1 is None else {
+        "bound": "hbm", "achieved": round(dec_bytes / (dec_ms1 / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+        "frac": round(dec_bytes / (dec_ms1 / 1e3) / 1e9 / pk["hbm_gbs"], 4), "ms": round(dec_ms1, 4),
+        "algorithmic_bytes": int(dec_bytes),
+        "kernel": "k_decide_proj_tc (adapter RMSNorm + linear) via dms_decide, L2-cold"}
+    compact_roof = {
+        "bound": "hbm", "achieved": round(comp_bytes / (comp_only_ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"],
+        "unit": "GB/s", "frac": round(comp_bytes / (comp_only_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+        "ms": round(comp_only_ms, 4), "algorithmic_bytes": int(comp_bytes),
+        "kernel": ("k_neuron_rope4 + " if neuron_pass else "") + "k_prefill_scan + k_prefill_scatter "
+                  "(dms_prefill_compact minus dms_decide), L2-cold"}
+
     e2e = None if args.no_e2e else run_e2e(B_, r, args, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -588,6 +643,8 @@ def run_ours(args, world, rank, local):
                               "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                               "frac": round(prefill_tflops / pk["bf16_tflops"], 4),
                               "flops_per_launch": prefill_flops / L, "visible_pairs": pairs},
+        "decide": decide_roof,
+        "compaction": compact_roof,
         "achieved_cr": round(wl.max_positions / retained_last, 3) if S == wl.decode_steps else None,
         "region_ms_per_step": round(region_ms / K, 3),
         "roofline": roof, "e2e": e2e, "gpu_launches": kernel_launches_per_step(wl, S) * K * R,
