@@ -594,7 +594,7 @@ def run_ours(args, world, rank, local):
         "bound": "hbm", "achieved": round(comp_bytes / (comp_only_ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"],
         "unit": "GB/s", "frac": round(comp_bytes / (comp_only_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
         "ms": round(comp_only_ms, 4), "algorithmic_bytes": int(comp_bytes),
-        "kernel": ("k_neuron_rope4 + " if neuron_pass else "") + "k_prefill_scan + k_prefill_scatter "
+        "kernel": ("k_neuron_rope8 + " if neuron_pass else "") + "k_prefill_scan + k_prefill_scatter "
                   "(dms_prefill_compact minus dms_decide), L2-cold"}
 
     e2e = None if args.no_e2e else run_e2e(B_, r, args, world)

@@ -586,11 +586,98 @@ __global__ void k_neuron_rope4(CacheView c, int T, const int* pos_dev, TA* q, TA
   }
 }
 
+// bf16 rows, large launches (prefill): one thread per (token, eight
+// consecutive pairs i .. i+7 < D/2).  The thread loads its cos/sin entries
+// once and walks the token's Hq + Hkv rows kRopeRows at a time, issuing all of
+// a group's loads before the first rotation; 32-bit indices (the launcher
+// checks that the item count fits).  The same arithmetic as above.
+constexpr int kRopeRows = 4;
+
+__global__ void __launch_bounds__(256, 3) k_neuron_rope8(CacheView c, int T, const int* pos_dev, __nv_bfloat16* q,
+                                                      __nv_bfloat16* k, const float* offset, int ostride,
+                                                      int do_alpha, float* alpha, const float* cos_t,
+                                                      const float* sin_t) {
+  const int D = c.D, half = D / 2, nq = half / 8, g = c.Hq / c.Hkv;
+  const bool key = c.alpha_source == DMS_ALPHA_KEY_NEURON;
+  const int nrow = c.Hq + c.Hkv;
+  const int total = c.B * T * nq;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
+    const int i = (idx % nq) * 8, tok = idx / nq;
+    const int b = tok / T, t = tok - b * T;
+    const long p = static_cast<long>(pos_dev ? pos_dev[b] + t : t) * half + i;
+    float cv[8], sv[8];
+    {
+      const float4 c0 = *reinterpret_cast<const float4*>(cos_t + p), c1 = *reinterpret_cast<const float4*>(cos_t + p + 4);
+      const float4 s0 = *reinterpret_cast<const float4*>(sin_t + p), s1 = *reinterpret_cast<const float4*>(sin_t + p + 4);
+      cv[0] = c0.x, cv[1] = c0.y, cv[2] = c0.z, cv[3] = c0.w, cv[4] = c1.x, cv[5] = c1.y, cv[6] = c1.z, cv[7] = c1.w;
+      sv[0] = s0.x, sv[1] = s0.y, sv[2] = s0.z, sv[3] = s0.w, sv[4] = s1.x, sv[5] = s1.y, sv[6] = s1.z, sv[7] = s1.w;
+    }
+    __nv_bfloat16* qrow = q + static_cast<long>(tok) * c.Hq * D + i;
+    __nv_bfloat16* krow = k + static_cast<long>(tok) * c.Hkv * D + i;
+    for (int r0 = 0; r0 < nrow; r0 += kRopeRows) {
+      uint4 x0[kRopeRows], x1[kRopeRows];
+#pragma unroll
+      for (int u = 0; u < kRopeRows; ++u) {
+        const int r = r0 + u;
+        if (r >= nrow) continue;
+        const __nv_bfloat16* row = r < c.Hq ? qrow + r * D : krow + (r - c.Hq) * D;
+        x0[u] = *reinterpret_cast<const uint4*>(row);
+        x1[u] = *reinterpret_cast<const uint4*>(row + half);
+      }
+#pragma unroll
+      for (int u = 0; u < kRopeRows; ++u) {
+        const int r = r0 + u;
+        if (r >= nrow) continue;
+        float a0[8], a1[8];
+        unpack16(x0[u], a0, static_cast<const __nv_bfloat16*>(nullptr));
+        unpack16(x1[u], a1, static_cast<const __nv_bfloat16*>(nullptr));
+        // the decision neuron (pair half - 1: the last element of the row) is
+        // read, then zeroed, before the rotation
+        const bool neuron_row = key ? r >= c.Hq : (r < c.Hq && r % g == 0);
+        if (do_alpha && neuron_row && i + 7 == half - 1) {
+          const int h = key ? r - c.Hq : r / g;
+          if (c.alpha_per == DMS_ALPHA_PER_LAYER) {
+            if (h == 0) {
+              const float av = fmaf(a1[7], c.alpha_scale, -offset[b * ostride]);
+              for (int hh = 0; hh < c.Hkv; ++hh) alpha[(static_cast<long>(b) * c.Hkv + hh) * T + t] = av;
+            }
+          } else {
+            alpha[(static_cast<long>(b) * c.Hkv + h) * T + t] = fmaf(a1[7], c.alpha_scale, -offset[b * ostride + h]);
+          }
+          a1[7] = 0.f;
+        }
+        uint32_t y0[4], y1[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          // each product and sum rounded separately (no fused multiply-add)
+          const int j = 2 * e;
+          y0[e] = pack_bf16(__fsub_rn(__fmul_rn(a0[j], cv[j]), __fmul_rn(a1[j], sv[j])),
+                            __fsub_rn(__fmul_rn(a0[j + 1], cv[j + 1]), __fmul_rn(a1[j + 1], sv[j + 1])));
+          y1[e] = pack_bf16(__fadd_rn(__fmul_rn(a1[j], cv[j]), __fmul_rn(a0[j], sv[j])),
+                            __fadd_rn(__fmul_rn(a1[j + 1], cv[j + 1]), __fmul_rn(a0[j + 1], sv[j + 1])));
+        }
+        __nv_bfloat16* row = r < c.Hq ? qrow + r * D : krow + (r - c.Hq) * D;
+        *reinterpret_cast<uint4*>(row) = make_uint4(y0[0], y0[1], y0[2], y0[3]);
+        *reinterpret_cast<uint4*>(row + half) = make_uint4(y1[0], y1[1], y1[2], y1[3]);
+      }
+    }
+  }
+}
+
 cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
                                int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
                                const float* sin_t, cudaStream_t s) {
   const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                        reinterpret_cast<uintptr_t>(cos_t) | reinterpret_cast<uintptr_t>(sin_t);
+  // large bf16 launches: one thread per (token, 8 pairs), rows walked in groups
+  const long total8 = static_cast<long>(c.B) * T * (c.D / 16);
+  if (cos_t && (al & 15) == 0 && (c.D / 2) % 8 == 0 && c.act_dtype == DMS_BF16 &&
+      total8 >= static_cast<long>(c.num_sms) * 256 && total8 < (1L << 30)) {
+    const int grid8 = static_cast<int>(min((total8 + 255) / 256, static_cast<long>(c.num_sms) * 3));
+    k_neuron_rope8<<<grid8, 256, 0, s>>>(c, T, pos_dev, static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
+                                         offset, offset_bstride, do_alpha ? 1 : 0, alpha, cos_t, sin_t);
+    return cudaGetLastError();
+  }
   if (cos_t && (al & 15) == 0 && (c.D / 2) % 4 == 0) {
     const long total4 = static_cast<long>(c.B) * T * (c.Hq + c.Hkv) * (c.D / 8);
     const int grid4 = static_cast<int>(max(1L, min((total4 + 255) / 256, static_cast<long>(c.num_sms) * 16)));

@@ -16,6 +16,9 @@ namespace dms {
 
 __device__ __forceinline__ bool bit_at(const unsigned* bits, int t) { return (bits[t >> 5] >> (t & 31)) & 1u; }
 
+constexpr int kScanU = 16;    // decision-logit words a warp loads before its ballots
+constexpr int kScatterU = 4;  // 16-byte row chunks a thread loads before it stores any
+
 // One CTA per (b, h).  Shared memory: five arrays of ceil(T/32) words.
 __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, int T, const float* alpha) {
   extern __shared__ unsigned sm[];
@@ -36,12 +39,22 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
   const int tid = threadIdx.x, lane = tid & 31, bd = blockDim.x;
   const int w = c.w;
 
-  // 1. evict bits (coalesced read, one ballot per 32 tokens)
-  for (int t0 = (tid & ~31); t0 < nw * 32; t0 += bd) {
-    const int t = t0 + lane;
-    const bool e = t < T && !c.disable && arow[t] > 0.0f;
-    const unsigned m = __ballot_sync(0xffffffffu, e);
-    if (lane == 0) ev[t0 >> 5] = m;
+  // 1. evict bits (coalesced read, one ballot per 32 tokens).  Warp wid owns
+  //    words wid, wid + nwarp, ...; it issues the loads of kScanU words before
+  //    the first ballot so that they are in flight together.
+  const int wid = tid >> 5, nwarp = bd >> 5;
+  for (int w0 = wid; w0 < nw; w0 += nwarp * kScanU) {
+    bool e[kScanU];
+#pragma unroll
+    for (int u = 0; u < kScanU; ++u) {
+      const int t = (w0 + u * nwarp) * 32 + lane;
+      e[u] = t < T && arow[t] > 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < kScanU; ++u) {
+      const unsigned m = __ballot_sync(0xffffffffu, e[u] && !c.disable);
+      if (lane == 0 && w0 + u * nwarp < nw) ev[w0 + u * nwarp] = m;
+    }
   }
   __syncthreads();
   // 2. open bits and kept-list bits
@@ -155,42 +168,69 @@ cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T, const floa
 }
 
 // ---------------------------------------------------------------------------
-// Scatter of the survivors into their pages: one CTA per (page, (b, h)).
-// Slot s of the page holds token slot_pos[s]; rows are copied as 16-byte
-// vectors.  FP8 pages: scale = max |x| / 448 over the page's rows (K and V
-// separately), code = RNE-satfinite(x / scale); eviction is applied before
-// quantisation ([FastDMS], quality section).
+// Scatter of the survivors into their pages.  Slot s of a page holds token
+// slot_pos[s]; rows are copied as 16-byte chunks.  FP8 pages: scale = max |x| /
+// 448 over the page's rows (K and V separately), code = RNE-satfinite(x /
+// scale); eviction is applied before quantisation ([FastDMS], quality section).
+//
+// Every thread gathers up to kScatterU chunks per batch: the slot positions,
+// then the K/V chunks (and the kept-list ranks), all loads issued before the
+// first store, so a batch costs two dependent DRAM round trips.
 // ---------------------------------------------------------------------------
+
+// bf16 / fp32 pages: one CTA per (group of rg rows of a page, (b, h)), with
+// rg * 16-byte chunks per row <= kScatterU * blockDim.x (one batch per thread).
 template <typename TA>
-__global__ void __launch_bounds__(256) k_prefill_scatter(CacheView c, int layer, int T, const TA* k, const TA* v) {
-  const int p = blockIdx.x, bh = blockIdx.y;
+__global__ void __launch_bounds__(256) k_prefill_scatter(CacheView c, int layer, int T, int rg, const TA* k,
+                                                         const TA* v) {
+  const int gpp = (c.P + rg - 1) / rg;
+  const int p = blockIdx.x / gpp, r0 = (blockIdx.x % gpp) * rg, bh = blockIdx.y;
   const int b = bh / c.Hkv, h = bh % c.Hkv;
   const long lbh = static_cast<long>(layer) * c.B * c.Hkv + bh;
   const int cnt = c.count[lbh];
-  if (p * c.P >= cnt) return;
+  const int s0 = p * c.P + r0;  // first slot of this CTA
+  if (s0 >= cnt) return;
   const int id = c.page_table[lbh * c.maxp + p];
   if (id < 0) return;
-  const int rows = min(c.P, cnt - p * c.P);
-  const int* slot_pos = c.slot_pos + lbh * c.cap + static_cast<long>(p) * c.P;
+  const int rows = min(rg, min(c.P - r0, cnt - s0));
+  const int* slot_pos = c.slot_pos + lbh * c.cap + s0;
   constexpr int V = 16 / sizeof(TA);
   const int cpr = c.D / V;  // 16-byte chunks per row
-  TA* kp = static_cast<TA*>(c.k_pool) + static_cast<long>(id) * c.P * c.D;
-  TA* vp = static_cast<TA*>(c.v_pool) + static_cast<long>(id) * c.P * c.D;
+  TA* kp = static_cast<TA*>(c.k_pool) + (static_cast<long>(id) * c.P + r0) * c.D;
+  TA* vp = static_cast<TA*>(c.v_pool) + (static_cast<long>(id) * c.P + r0) * c.D;
   const int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
-  for (int idx = threadIdx.x; idx < rows * cpr; idx += blockDim.x) {
-    const int r = idx / cpr, ch = idx % cpr;
-    const int t = slot_pos[r];
-    const long src = ((static_cast<long>(b) * T + t) * c.Hkv + h) * c.D;
-    const uint4 kq = reinterpret_cast<const uint4*>(k + src)[ch];
-    const uint4 vq = reinterpret_cast<const uint4*>(v + src)[ch];
-    reinterpret_cast<uint4*>(kp + static_cast<long>(r) * c.D)[ch] = kq;
-    reinterpret_cast<uint4*>(vp + static_cast<long>(r) * c.D)[ch] = vq;
-    if (sizeof(TA) == 2 && c.kept_k && t < T - c.w) {
-      // a kept token before the last window: also into the position-sorted
-      // kept copy read by the tcgen05 prefill attention
-      const long kr = (static_cast<long>(bh) * c.max_pos + kept_upto[t]) * c.D;
-      reinterpret_cast<uint4*>(static_cast<TA*>(c.kept_k) + kr)[ch] = kq;
-      reinterpret_cast<uint4*>(static_cast<TA*>(c.kept_v) + kr)[ch] = vq;
+  // a kept token before the last window also goes into the position-sorted
+  // kept copy read by the tcgen05 prefill attention
+  const bool kept_copy = sizeof(TA) == 2 && c.kept_k != nullptr;
+  const int n = rows * cpr;
+  for (int base = threadIdx.x; base < n; base += kScatterU * blockDim.x) {
+    int tt[kScatterU], kr[kScatterU];
+    uint4 kq[kScatterU], vq[kScatterU];
+#pragma unroll
+    for (int u = 0; u < kScatterU; ++u) {
+      const int idx = base + u * blockDim.x;
+      tt[u] = idx < n ? slot_pos[idx / cpr] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kScatterU; ++u) {
+      if (tt[u] < 0) continue;
+      const int ch = (base + u * blockDim.x) % cpr;
+      const long src = ((static_cast<long>(b) * T + tt[u]) * c.Hkv + h) * c.D;
+      kq[u] = reinterpret_cast<const uint4*>(k + src)[ch];
+      vq[u] = reinterpret_cast<const uint4*>(v + src)[ch];
+      kr[u] = kept_copy && tt[u] < T - c.w ? kept_upto[tt[u]] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kScatterU; ++u) {
+      if (tt[u] < 0) continue;
+      const int idx = base + u * blockDim.x, r = idx / cpr, ch = idx % cpr;
+      reinterpret_cast<uint4*>(kp + static_cast<long>(r) * c.D)[ch] = kq[u];
+      reinterpret_cast<uint4*>(vp + static_cast<long>(r) * c.D)[ch] = vq[u];
+      if (kr[u] >= 0) {
+        const long dst = (static_cast<long>(bh) * c.max_pos + kr[u]) * c.D;
+        reinterpret_cast<uint4*>(static_cast<TA*>(c.kept_k) + dst)[ch] = kq[u];
+        reinterpret_cast<uint4*>(static_cast<TA*>(c.kept_v) + dst)[ch] = vq[u];
+      }
     }
   }
 }
@@ -207,6 +247,32 @@ __device__ __forceinline__ float block_max(float x, float* red) {
   return m;
 }
 
+// FP8 pages: one CTA per (page, (b, h)); the scale needs the whole page.  Pass 1
+// takes max |x| of K and V and writes the kept copy; pass 2 re-reads the rows
+// (now in L2) and writes the codes.
+__device__ __forceinline__ uint2 encode8(const uint4 x, float scale) {
+  float f[8];
+  unpack16(x, f, static_cast<const __nv_bfloat16*>(nullptr));
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint32_t q = scale > 0.f ? fp8_encode(__fdiv_rn(f[e], scale)) : 0u;
+    if (e < 4)
+      lo |= q << (8 * e);
+    else
+      hi |= q << (8 * (e - 4));
+  }
+  return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ float amax8(const uint4 x, float m) {
+  float f[8];
+  unpack16(x, f, static_cast<const __nv_bfloat16*>(nullptr));
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+  return m;
+}
+
 __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int layer, int T, const __nv_bfloat16* k,
                                                             const __nv_bfloat16* v) {
   __shared__ float red[32];
@@ -220,49 +286,72 @@ __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int la
   const int rows = min(c.P, cnt - p * c.P);
   const int* slot_pos = c.slot_pos + lbh * c.cap + static_cast<long>(p) * c.P;
   const int cpr = c.D / 8;  // 8 bf16 per 16-byte input chunk
-  if (c.kept_k) {
-    // kept tokens before the last window: into the position-sorted kept copy
-    const int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
-    for (int idx = threadIdx.x; idx < rows * cpr; idx += blockDim.x) {
-      const int r = idx / cpr, ch = idx % cpr;
-      const int t = slot_pos[r];
-      if (t >= T - c.w) continue;
-      const long src = ((static_cast<long>(b) * T + t) * c.Hkv + h) * c.D;
-      const long kr = (static_cast<long>(bh) * c.max_pos + kept_upto[t]) * c.D;
-      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.kept_k) + kr)[ch] = reinterpret_cast<const uint4*>(k + src)[ch];
-      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.kept_v) + kr)[ch] = reinterpret_cast<const uint4*>(v + src)[ch];
+  const int n = rows * cpr;
+  const int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
+  const bool kept_copy = c.kept_k != nullptr;
+  float ak = 0.f, av = 0.f;
+  for (int base = threadIdx.x; base < n; base += kScatterU * blockDim.x) {
+    int tt[kScatterU], kr[kScatterU];
+    uint4 kq[kScatterU], vq[kScatterU];
+#pragma unroll
+    for (int u = 0; u < kScatterU; ++u) {
+      const int idx = base + u * blockDim.x;
+      tt[u] = idx < n ? slot_pos[idx / cpr] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kScatterU; ++u) {
+      if (tt[u] < 0) continue;
+      const int ch = (base + u * blockDim.x) % cpr;
+      const long src = ((static_cast<long>(b) * T + tt[u]) * c.Hkv + h) * c.D;
+      kq[u] = reinterpret_cast<const uint4*>(k + src)[ch];
+      vq[u] = reinterpret_cast<const uint4*>(v + src)[ch];
+      kr[u] = kept_copy && tt[u] < T - c.w ? kept_upto[tt[u]] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kScatterU; ++u) {
+      if (tt[u] < 0) continue;
+      ak = amax8(kq[u], ak);
+      av = amax8(vq[u], av);
+      if (kr[u] >= 0) {
+        // kept tokens before the last window: into the position-sorted kept copy
+        const int ch = (base + u * blockDim.x) % cpr;
+        const long dst = (static_cast<long>(bh) * c.max_pos + kr[u]) * c.D;
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.kept_k) + dst)[ch] = kq[u];
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.kept_v) + dst)[ch] = vq[u];
+      }
     }
   }
-  for (int which = 0; which < 2; ++which) {
-    const __nv_bfloat16* x = which ? v : k;
-    float amax = 0.f;
-    for (int idx = threadIdx.x; idx < rows * cpr; idx += blockDim.x) {
-      const int r = idx / cpr, ch = idx % cpr;
-      const long src = ((static_cast<long>(b) * T + slot_pos[r]) * c.Hkv + h) * c.D;
-      float f[8];
-      unpack16(reinterpret_cast<const uint4*>(x + src)[ch], f, static_cast<const __nv_bfloat16*>(nullptr));
+  ak = block_max(ak, red);
+  av = block_max(av, red);
+  const float sk = __fdiv_rn(ak, 448.0f), sv = __fdiv_rn(av, 448.0f);
+  if (threadIdx.x == 0) {
+    c.k_scale[id] = sk;
+    c.v_scale[id] = sv;
+  }
+  uint8_t* kd = static_cast<uint8_t*>(c.k_pool) + static_cast<long>(id) * c.P * c.D;
+  uint8_t* vd = static_cast<uint8_t*>(c.v_pool) + static_cast<long>(id) * c.P * c.D;
+  for (int base = threadIdx.x; base < n; base += kScatterU * blockDim.x) {
+    int tt[kScatterU];
+    uint4 kq[kScatterU], vq[kScatterU];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+    for (int u = 0; u < kScatterU; ++u) {
+      const int idx = base + u * blockDim.x;
+      tt[u] = idx < n ? slot_pos[idx / cpr] : -1;
     }
-    amax = block_max(amax, red);
-    const float scale = __fdiv_rn(amax, 448.0f);
-    if (threadIdx.x == 0) (which ? c.v_scale : c.k_scale)[id] = scale;
-    uint8_t* dst = static_cast<uint8_t*>(which ? c.v_pool : c.k_pool) + static_cast<long>(id) * c.P * c.D;
-    for (int idx = threadIdx.x; idx < rows * cpr; idx += blockDim.x) {
-      const int r = idx / cpr, ch = idx % cpr;
-      const long src = ((static_cast<long>(b) * T + slot_pos[r]) * c.Hkv + h) * c.D;
-      float f[8];
-      unpack16(reinterpret_cast<const uint4*>(x + src)[ch], f, static_cast<const __nv_bfloat16*>(nullptr));
-      uint32_t lo = 0, hi = 0;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t q = scale > 0.f ? fp8_encode(__fdiv_rn(f[e], scale)) : 0u;
-        if (e < 4)
-          lo |= q << (8 * e);
-        else
-          hi |= q << (8 * (e - 4));
-      }
-      reinterpret_cast<uint2*>(dst + static_cast<long>(r) * c.D)[ch] = make_uint2(lo, hi);
+    for (int u = 0; u < kScatterU; ++u) {
+      if (tt[u] < 0) continue;
+      const int ch = (base + u * blockDim.x) % cpr;
+      const long src = ((static_cast<long>(b) * T + tt[u]) * c.Hkv + h) * c.D;
+      kq[u] = reinterpret_cast<const uint4*>(k + src)[ch];
+      vq[u] = reinterpret_cast<const uint4*>(v + src)[ch];
+    }
+#pragma unroll
+    for (int u = 0; u < kScatterU; ++u) {
+      if (tt[u] < 0) continue;
+      const int idx = base + u * blockDim.x, r = idx / cpr, ch = idx % cpr;
+      reinterpret_cast<uint2*>(kd + static_cast<long>(r) * c.D)[ch] = encode8(kq[u], sk);
+      reinterpret_cast<uint2*>(vd + static_cast<long>(r) * c.D)[ch] = encode8(vq[u], sv);
     }
   }
 }
@@ -270,15 +359,20 @@ __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int la
 cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T, const void* k, const void* v,
                                    cudaStream_t s) {
   const int pages = min(c.maxp, (T + c.P - 1) / c.P);
-  dim3 grid(pages, c.B * c.Hkv);
-  if (c.kv_dtype == DMS_FP8_E4M3)
-    k_prefill_scatter_fp8<<<grid, 256, 0, s>>>(c, layer, T, static_cast<const __nv_bfloat16*>(k),
-                                               static_cast<const __nv_bfloat16*>(v));
-  else if (c.kv_dtype == DMS_BF16)
-    k_prefill_scatter<__nv_bfloat16><<<grid, 256, 0, s>>>(c, layer, T, static_cast<const __nv_bfloat16*>(k),
+  if (c.kv_dtype == DMS_FP8_E4M3) {
+    k_prefill_scatter_fp8<<<dim3(pages, c.B * c.Hkv), 256, 0, s>>>(c, layer, T, static_cast<const __nv_bfloat16*>(k),
+                                                                   static_cast<const __nv_bfloat16*>(v));
+    return cudaGetLastError();
+  }
+  // rows per CTA: one batch of kScatterU chunks per thread
+  const int cpr = c.D * (c.kv_dtype == DMS_BF16 ? 2 : 4) / 16;
+  const int rg = max(1, min(c.P, kScatterU * 256 / cpr));
+  dim3 grid(pages * ((c.P + rg - 1) / rg), c.B * c.Hkv);
+  if (c.kv_dtype == DMS_BF16)
+    k_prefill_scatter<__nv_bfloat16><<<grid, 256, 0, s>>>(c, layer, T, rg, static_cast<const __nv_bfloat16*>(k),
                                                           static_cast<const __nv_bfloat16*>(v));
   else
-    k_prefill_scatter<float><<<grid, 256, 0, s>>>(c, layer, T, static_cast<const float*>(k),
+    k_prefill_scatter<float><<<grid, 256, 0, s>>>(c, layer, T, rg, static_cast<const float*>(k),
                                                   static_cast<const float*>(v));
   return cudaGetLastError();
 }

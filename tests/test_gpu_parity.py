@@ -52,6 +52,11 @@ CASES = {
     # fused decode over many heads (batch 8: decision logits inside the kernel)
     "bf16_b8_proj": Case(B=8, T=300, steps=40, Hq=16, Hkv=8, D=128, hidden=256, w=64, P=32, act="bf16", kv="bf16",
                          source="proj", keep=(1 / 16, 1 / 4), prealloc=96, seed=17),
+    # a prompt large enough for the row-walking rotary kernel (batch x tokens x
+    # 8-pair chunks above 148 x 256), 256-slot pages scattered by several CTAs
+    # each, the last page ragged
+    "bf16_key_rope_p256": Case(B=2, T=2500, steps=16, Hq=8, Hkv=2, D=128, w=320, P=256, act="bf16", kv="bf16",
+                               source="key", keep=0.2, rope=True, attn_rows=128, seed=21),
     # second layer of a two-layer cache with preallocation
     "layer1_of_2": Case(B=2, T=260, steps=12, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16",
                         source="input", keep=0.3, layers=2, layer=1, prealloc=64, seed=15),
