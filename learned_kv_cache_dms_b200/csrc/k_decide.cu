@@ -237,6 +237,11 @@ __global__ void __launch_bounds__(256) k_decide_proj_row(CacheView c, DecideArgs
 // two halves are added through shared memory at the end of the tile.
 // ---------------------------------------------------------------------------
 constexpr int kDpTok = 64, kDpK = 128, kDpStages = 4, kDpWarps = 8;  // a stage: two 64-element boxes
+// chunks the producer keeps warm in L2 ahead of the ring (the ring is bounded
+// by the shared memory the table leaves; the prefetches are not)
+constexpr int kDpPrefetch = 8;
+static_assert(kDpStages % 2 == 0, "a stage must keep one consumer parity");
+constexpr int kDpFillU = 8;  // table items a thread loads before it writes any
 constexpr int kDpThreads = (kDpWarps + 1) * 32;
 
 // table row (bf16): the hidden size rounded up to whole chunks (zero-filled,
@@ -262,25 +267,66 @@ __global__ void __launch_bounds__(kDpThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long ntok = static_cast<long>(c.B) * T;
   const int ntiles = static_cast<int>((ntok + kDpTok - 1) / kDpTok), nk = (hid + kDpK - 1) / kDpK;
-  if (tid == 0) {
+  // chunk q of this CTA: tile blockIdx.x + (q / nk) * gridDim.x, column chunk q % nk
+  const int nq = (ntiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                 static_cast<int>(gridDim.x) * nk;
+  auto chunk_x = [&](int q) { return (q % nk) * kDpK; };
+  auto chunk_y = [&](int q) { return (static_cast<int>(blockIdx.x) + (q / nk) * static_cast<int>(gridDim.x)) * kDpTok; };
+  auto issue = [&](int q) {
+    const int st = q % kDpStages;
+    mbar_expect_tx(&full[st], kDpTok * 2 * kDpK);
+    for (int hb = 0; hb < kDpK / 64; ++hb)
+      tma_load_2d(sb + st * kDpTok * 2 * kDpK + hb * kDpTok * 128, &hmap, chunk_x(q) + 64 * hb, chunk_y(q), &full[st]);
+  };
+  auto prefetch = [&](int q) {
+    for (int hb = 0; hb < kDpK / 64; ++hb) tma_prefetch_2d(&hmap, chunk_x(q) + 64 * hb, chunk_y(q));
+  };
+  if (warp == kDpWarps && lane == 0) {
+    // the producer sets up the ring and starts it (and the L2 prefetches)
+    // before the table is built
     for (int i = 0; i < kDpStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kDpWarps / 2);  // the four warps of the chunk's parity
     }
     fence_mbar_init();
+    fence_proxy_async();  // the initialised barriers before this thread's first TMA (async proxy)
+    for (int q = 0; q < min(kDpStages, nq); ++q) issue(q);
+    for (int q = kDpStages; q < min(kDpStages + kDpPrefetch, nq); ++q) prefetch(q);
   }
-  // folded table hi / lo (rows >= H and the pad are zero)
+  // folded table hi / lo (rows >= H and the pad are zero).  Each thread loads
+  // kDpFillU items' W and gamma vectors before it writes any (the table is
+  // written through a generic pointer, which would otherwise order every load
+  // after the previous item's stores); CTAs start at different items so that
+  // they do not all read the same L2 lines at once.
   const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(a.W);
   const __nv_bfloat16* gamma = static_cast<const __nv_bfloat16*>(a.gamma);
-  const int nvec = hid / 8;
-#pragma unroll 4
-  for (int i = tid; i < 8 * (wrow / 8); i += kDpThreads) {
-    const int n = i / (wrow / 8), v = i % (wrow / 8);
-    uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
-    if (n < H && v < nvec) {
+  const int nvec = hid / 8, rvec = wrow / 8, nitem = 8 * rvec;
+  const int rot = static_cast<int>((blockIdx.x * 613u) % static_cast<unsigned>(nitem));
+  for (int i0 = tid; i0 < nitem; i0 += kDpThreads * kDpFillU) {
+    uint4 wq[kDpFillU], gq[kDpFillU];
+    int it[kDpFillU];
+#pragma unroll
+    for (int u = 0; u < kDpFillU; ++u) {
+      int i = i0 + u * kDpThreads;
+      it[u] = -1;
+      wq[u] = gq[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (i >= nitem) continue;
+      i += rot;
+      if (i >= nitem) i -= nitem;
+      it[u] = i;
+      const int n = i / rvec, v = i % rvec;
+      if (n < H && v < nvec) {
+        wq[u] = reinterpret_cast<const uint4*>(W + static_cast<long>(n) * hid)[v];
+        gq[u] = reinterpret_cast<const uint4*>(gamma)[v];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kDpFillU; ++u) {
+      if (it[u] < 0) continue;
+      const int n = it[u] / rvec, v = it[u] % rvec;
       float wv[8], gv[8];
-      unpack16(reinterpret_cast<const uint4*>(W + static_cast<long>(n) * hid)[v], wv, static_cast<const __nv_bfloat16*>(nullptr));
-      unpack16(reinterpret_cast<const uint4*>(gamma)[v], gv, static_cast<const __nv_bfloat16*>(nullptr));
+      unpack16(wq[u], wv, static_cast<const __nv_bfloat16*>(nullptr));
+      unpack16(gq[u], gv, static_cast<const __nv_bfloat16*>(nullptr));
       uint32_t h4[4], l4[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -290,30 +336,24 @@ __global__ void __launch_bounds__(kDpThreads, 1)
         h4[e] = *reinterpret_cast<const uint32_t*>(&hv);
         l4[e] = pack_bf16(p0 - hf.x, p1 - hf.y);
       }
-      hi = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-      lo = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+      reinterpret_cast<uint4*>(wt + static_cast<long>(n) * wrow)[v] = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+      reinterpret_cast<uint4*>(wt + static_cast<long>(8 + n) * wrow)[v] = make_uint4(l4[0], l4[1], l4[2], l4[3]);
     }
-    reinterpret_cast<uint4*>(wt + static_cast<long>(n) * wrow)[v] = hi;
-    reinterpret_cast<uint4*>(wt + static_cast<long>(8 + n) * wrow)[v] = lo;
   }
   __syncthreads();
 
   if (warp == kDpWarps) {
     // ---- producer: hidden tiles of this CTA's token tiles ----------------
     if (lane == 0) {
-      int q = 0;
-      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x)
-        for (int kc = 0; kc < nk; ++kc, ++q) {
-          const int st = q % kDpStages, use = q / kDpStages;
-          if (use > 0 && !mbar_wait_bounded(&empty[st], (use - 1) & 1)) {
-            set_status(c.ctrl, DMS_ST_TIMEOUT);
-            return;
-          }
-          mbar_expect_tx(&full[st], kDpTok * 2 * kDpK);
-          for (int hb = 0; hb < kDpK / 64; ++hb)
-            tma_load_2d(sb + st * kDpTok * 2 * kDpK + hb * kDpTok * 128, &hmap, kc * kDpK + 64 * hb, tile * kDpTok,
-                        &full[st]);
+      for (int q = kDpStages; q < nq; ++q) {
+        const int st = q % kDpStages, use = q / kDpStages;
+        if (!mbar_wait_bounded(&empty[st], (use - 1) & 1)) {
+          set_status(c.ctrl, DMS_ST_TIMEOUT);
+          return;
         }
+        issue(q);
+        if (q + kDpPrefetch < nq) prefetch(q + kDpPrefetch);
+      }
     }
     return;
   }
@@ -330,7 +370,9 @@ __global__ void __launch_bounds__(kDpThreads, 1)
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, qbase += nk) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     float ss[2] = {0.f, 0.f};
-    for (int kc = par; kc < nk; kc += 2) {
+    // chunk q goes to the warps of parity q % 2: with an even stage count a
+    // stage is always consumed by the same four warps, in order
+    for (int kc = par ^ (qbase & 1); kc < nk; kc += 2) {
       const int q = qbase + kc, st = q % kDpStages;
       if (ok && !mbar_wait_bounded(&full[st], (q / kDpStages) & 1)) {
         ok = false;

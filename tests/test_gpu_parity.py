@@ -20,6 +20,11 @@ CASES = {
     # a hidden size that is a multiple of 8 but not of the adapter kernel's chunks
     "bf16_proj_hidden_ragged": Case(B=2, T=300, steps=12, Hq=8, Hkv=4, D=64, hidden=328, w=64, P=32, act="bf16",
                                     kv="bf16", source="proj", keep=0.25, seed=31),
+    # the same hidden size (3 chunks) over 157 token tiles: some CTAs take two
+    # tiles, the second starting at an odd chunk index
+    "bf16_proj_hidden_ragged_multitile": Case(B=2, T=5000, steps=8, Hq=8, Hkv=4, D=64, hidden=328, w=64, P=32,
+                                              act="bf16", kv="bf16", source="proj", keep=0.25, attn_rows=64,
+                                              seed=32),
     "bf16_d64_proj_layer": Case(B=2, T=333, steps=20, Hq=4, Hkv=4, D=64, hidden=256, w=48, P=16, act="bf16",
                                 kv="bf16", source="proj", per="layer", keep=0.25, seed=4),
     "fp8_key_rope_head": Case(B=2, T=700, steps=30, Hq=8, Hkv=2, D=64, w=64, P=32, act="bf16", kv="fp8",
