@@ -20,6 +20,7 @@ enum Ctrl {
   CTRL_DONE_SCAN = 2,    // arrival counter of the prefill scan CTAs
   CTRL_GRID_DONE = 3,    // arrival counter of the fused decode CTAs
   CTRL_STEP_PAGES = 4,   // pages granted by the running fused decode step
+  CTRL_CLUSTER_STEP = 6, // (64-bit, words 6-7) cluster decode step: owners arrived, pages granted
   CTRL_WORDS = 64
 };
 

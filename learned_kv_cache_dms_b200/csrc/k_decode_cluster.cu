@@ -296,19 +296,20 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   if (!landed && tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
   DMS_TRACE_MARK(0, 4);
 
-  if (FUSED) {
-    // append of this head's token at the planned slot (every CTA of the
-    // cluster has finished reading the pages: their partials have landed)
+  if (FUSED && warp == 3) {
+    // Warp 3 appends this head's token at the planned slot (every CTA of the
+    // cluster has finished reading the pages: their partials have landed) and
+    // counts the step, while warps 0-2 merge the output.
     const int flags = pl.y, slot = pl.x;
     int id = -1;
     bool ok = !(flags & 4);
     if (ok && (flags & 2)) {
+      // a new page: numbered by this head's rank among the heads that need one
       int n_before = 0;
-      for (int i = tid; i < bh; i += kThreads)
+      for (int i = lane; i < bh; i += 32)
         n_before += (plan_at(c, static_cast<long>(layer) * c.B * c.Hkv + i, t)->y & 2) ? 1 : 0;
-      int before;
-      block_exclusive_scan(n_before, s_red, &before);
-      id = next_page0 + before;
+      n_before = __reduce_add_sync(0xffffffffu, n_before);
+      id = next_page0 + n_before;
       if (id >= c.pool_pages || pl.w >= c.maxp) ok = false;
     } else if (ok) {
       const int pi = slot / c.P;
@@ -317,19 +318,18 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     int cnt_new = cnt, np_new = pl.w;  // pages before the append (plan snapshot)
     if (ok) {
       const long row = static_cast<long>(id) * c.P + slot % c.P;
-      if (tid < D / 8) {
-        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.k_pool) + row * D)[tid] =
-            reinterpret_cast<const uint4*>(s_knew)[tid];
-        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.v_pool) + row * D)[tid] =
-            reinterpret_cast<const uint4*>(s_vnew)[tid];
+      if (lane < D / 8) {
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.k_pool) + row * D)[lane] =
+            reinterpret_cast<const uint4*>(s_knew)[lane];
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.v_pool) + row * D)[lane] =
+            reinterpret_cast<const uint4*>(s_vnew)[lane];
       }
       if (!(flags & 1)) cnt_new = cnt + 1;
       if (flags & 2) np_new += 1;
-      if (tid == 0) {
+      if (lane == 0) {
         if (flags & 2) {
           c.page_table[li * c.maxp + np_new - 1] = id;
           c.npages[li] = np_new;
-          atomicAdd(&c.ctrl[CTRL_STEP_PAGES], 1);
         }
         const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
         const float a = fuse_decide ? s_alpha : __ldcg(&alpha[b * c.Hkv + hs]);
@@ -338,35 +338,32 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
         c.ring[li * c.w + t % c.w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
         if (!(flags & 1)) c.count[li] = cnt_new;
       }
-    } else if (tid == 0) {
+    } else if (lane == 0) {
       set_status(c.ctrl, (flags & 4) ? DMS_ST_CAPACITY : DMS_ST_POOL_EXHAUSTED);
     }
-    if (tid == 0) {
-      // plan of the next append (token t + 1), from the values just written
-      *plan_at(c, li, t + 1) = make_plan(s_ring_next, t + 1, cnt_new, np_new, c);
-    }
-    __syncthreads();  // the append (thread 0's page grant included) precedes warp 3's release below
-  }
-  DMS_TRACE_MARK(0, 8);
-
-  if (FUSED && warp == 3) {
-    // warp 3, while warps 0-2 merge: count this owner (the fence releases the
-    // page grant ordered before it by the barrier above); the grid's last
-    // owner advances the page counter and the positions
+    DMS_TRACE_MARK(0, 8);
     int last = 0;
     if (lane == 0) {
-      __threadfence();
-      last = atomicAdd(&c.ctrl[CTRL_GRID_DONE], 1) == static_cast<int>(gridDim.x) / cs - 1;
+      // plan of the next append (token t + 1), from the values just written
+      *plan_at(c, li, t + 1) = make_plan(s_ring_next, t + 1, cnt_new, np_new, c);
+      // Step accounting: one 64-bit add per owner, the owners that arrived in
+      // the low word and the pages they granted in the high word, so the
+      // grid's last owner learns the step's total from its own add.  Every
+      // CTA read the page counter (next_page0) after the wait and before its
+      // owner counted itself, so the last owner may advance it; what the
+      // other owners wrote is read only by later launches.
+      const unsigned long long mine = (static_cast<unsigned long long>(ok && (flags & 2)) << 32) | 1ull;
+      unsigned long long* done = reinterpret_cast<unsigned long long*>(&c.ctrl[CTRL_CLUSTER_STEP]);
+      const unsigned long long old = atomicAdd(done, mine);
+      last = static_cast<int>(old & 0xffffffffull) == static_cast<int>(gridDim.x) / cs - 1;
       if (last) {
-        __threadfence();  // every owner's grant, released before its count, is visible
-        const int granted = __ldcg(&c.ctrl[CTRL_STEP_PAGES]);
-        c.ctrl[CTRL_NEXT_PAGE] = min(__ldcg(&c.ctrl[CTRL_NEXT_PAGE]) + granted, c.pool_pages);
-        c.ctrl[CTRL_STEP_PAGES] = 0;
-        c.ctrl[CTRL_GRID_DONE] = 0;
+        const int granted = static_cast<int>((old + mine) >> 32);
+        c.ctrl[CTRL_NEXT_PAGE] = min(next_page0 + granted, c.pool_pages);
+        *done = 0ull;
       }
     }
     if (__shfl_sync(0xffffffffu, last, 0))
-      for (int bb = lane; bb < c.B; bb += 32) c.pos[layer * c.B + bb] += 1;
+      for (int bb = lane; bb < c.B; bb += 32) atomicAdd(&c.pos[layer * c.B + bb], 1);
     DMS_TRACE_MARK(0, 6);
     return;
   }
