@@ -528,6 +528,26 @@ __device__ __forceinline__ float ld_dsmem(uint32_t addr) {
 // the head's retained count and pages before the append.
 // Loads bypass L1: the state may have been written by other CTAs of the same
 // launch (made visible by their fences).
+// Step accounting of a fused decode launch: one 64-bit add per counting CTA,
+// the CTAs arrived in the low word and the pages they granted in the high
+// word, so the last CTA learns the step's total from its own add.  Every CTA
+// has read the page counter and the positions before it counts itself, so
+// the last one advances the counter (from next_page0, the value every CTA
+// read) and the positions; what the other CTAs wrote is read only by later
+// launches.  Returns true in the last CTA (thread that calls it).
+__device__ __forceinline__ bool count_step(const CacheView& c, int granted, int ncount, int next_page0) {
+  unsigned long long* done = reinterpret_cast<unsigned long long*>(&c.ctrl[CTRL_STEP64]);
+  const unsigned long long mine = (static_cast<unsigned long long>(granted) << 32) | 1ull;
+  const unsigned long long old = atomicAdd(done, mine);
+  if (static_cast<int>(old & 0xffffffffull) != ncount - 1) return false;
+  c.ctrl[CTRL_NEXT_PAGE] = min(next_page0 + static_cast<int>((old + mine) >> 32), c.pool_pages);
+  *done = 0ull;
+  return true;
+}
+__device__ __forceinline__ void advance_positions(const CacheView& c, int layer, int first, int stride) {
+  for (int bb = first; bb < c.B; bb += stride) atomicAdd(&c.pos[layer * c.B + bb], 1);
+}
+
 __device__ __forceinline__ int4 make_plan(int ringv, int t, int cnt, int have, const CacheView& c) {
   if (t >= c.w && (static_cast<unsigned>(ringv) & RING_EVICT)) return make_int4(ringv & RING_SLOT_MASK, 1, cnt, have);
   if (cnt >= c.cap) return make_int4(-1, 4, cnt, have);

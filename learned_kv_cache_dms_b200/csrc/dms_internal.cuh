@@ -18,9 +18,7 @@ enum Ctrl {
   CTRL_STATUS = 0,       // sticky DMS_ST_* bits
   CTRL_NEXT_PAGE = 1,    // next page id the ascending counter hands out
   CTRL_DONE_SCAN = 2,    // arrival counter of the prefill scan CTAs
-  CTRL_GRID_DONE = 3,    // arrival counter of the fused decode CTAs
-  CTRL_STEP_PAGES = 4,   // pages granted by the running fused decode step
-  CTRL_CLUSTER_STEP = 6, // (64-bit, words 6-7) cluster decode step: owners arrived, pages granted
+  CTRL_STEP64 = 4,       // (64-bit, words 4-5) fused decode step: CTAs arrived, pages granted
   CTRL_WORDS = 64
 };
 

@@ -174,7 +174,6 @@ __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, i
       if (flags & 2) {
         c.page_table[li * c.maxp + have] = id;
         c.npages[li] = np_new;
-        atomicAdd(&c.ctrl[CTRL_STEP_PAGES], 1);
       }
       if (!(flags & 1)) c.count[li] = cnt_new;
       const float a = fuse_decide ? a_dec : alpha[b * c.Hkv + hs];
@@ -188,20 +187,10 @@ __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, i
     *plan_at(c, li, t + 1) = make_plan(ring_next, t + 1, cnt_new, np_new, c);
     // the grid's last CTA advances the page counter and the positions (every
     // CTA has read them by the time it counts itself)
-    __threadfence();
-    s_last = atomicAdd(&c.ctrl[CTRL_GRID_DONE], 1) == BH - 1;
+    s_last = count_step(c, ok && (flags & 2) ? 1 : 0, BH, next_page0) ? 1 : 0;
   }
   __syncthreads();
-  if (s_last) {
-    if (tid == 0) {
-      __threadfence();
-      const int granted = __ldcg(&c.ctrl[CTRL_STEP_PAGES]);
-      c.ctrl[CTRL_NEXT_PAGE] = min(__ldcg(&c.ctrl[CTRL_NEXT_PAGE]) + granted, c.pool_pages);
-      c.ctrl[CTRL_STEP_PAGES] = 0;
-      c.ctrl[CTRL_GRID_DONE] = 0;
-    }
-    for (int bb = tid; bb < c.B; bb += kAppendThreads) c.pos[layer * c.B + bb] += 1;
-  }
+  if (s_last) advance_positions(c, layer, tid, kAppendThreads);
   DMS_TRACE_MARK(1, 3);
 }
 

@@ -346,24 +346,11 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     if (lane == 0) {
       // plan of the next append (token t + 1), from the values just written
       *plan_at(c, li, t + 1) = make_plan(s_ring_next, t + 1, cnt_new, np_new, c);
-      // Step accounting: one 64-bit add per owner, the owners that arrived in
-      // the low word and the pages they granted in the high word, so the
-      // grid's last owner learns the step's total from its own add.  Every
-      // CTA read the page counter (next_page0) after the wait and before its
-      // owner counted itself, so the last owner may advance it; what the
-      // other owners wrote is read only by later launches.
-      const unsigned long long mine = (static_cast<unsigned long long>(ok && (flags & 2)) << 32) | 1ull;
-      unsigned long long* done = reinterpret_cast<unsigned long long*>(&c.ctrl[CTRL_CLUSTER_STEP]);
-      const unsigned long long old = atomicAdd(done, mine);
-      last = static_cast<int>(old & 0xffffffffull) == static_cast<int>(gridDim.x) / cs - 1;
-      if (last) {
-        const int granted = static_cast<int>((old + mine) >> 32);
-        c.ctrl[CTRL_NEXT_PAGE] = min(next_page0 + granted, c.pool_pages);
-        *done = 0ull;
-      }
+      // the owners count the step (every CTA of the cluster has read the page
+      // counter and the positions before its partial landed here)
+      last = count_step(c, ok && (flags & 2) ? 1 : 0, static_cast<int>(gridDim.x) / cs, next_page0) ? 1 : 0;
     }
-    if (__shfl_sync(0xffffffffu, last, 0))
-      for (int bb = lane; bb < c.B; bb += 32) atomicAdd(&c.pos[layer * c.B + bb], 1);
+    if (__shfl_sync(0xffffffffu, last, 0)) advance_positions(c, layer, lane, 32);
     DMS_TRACE_MARK(0, 6);
     return;
   }

@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
   __shared__ int s_part[kFlatThreads / 32][8];  // per-warp candidate unit sums
   __shared__ int s_ctot[kFlatThreads / 32][2];  // per-warp chunk totals (units, new pages)
   __shared__ int s_stot[2][3];                  // per-warp segment totals (sub-tiles, page ids, ring entries)
-  __shared__ int s_nseg, s_nsub, s_npt, s_nring, s_last, s_next_page0;
+  __shared__ int s_nseg, s_nsub, s_npt, s_nring, s_last, s_next_page0, s_grants;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
@@ -415,6 +415,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     }
     mbar_init(&aux_done, 1);
     s_nfin = 0;
+    s_grants = 0;
     fence_mbar_init();
   }
   // Heads are split into one contiguous chunk per warp.  Each warp loads its
@@ -828,7 +829,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
               if (flags & 2) {
                 c.page_table[li * c.maxp + np_new - 1] = id;
                 c.npages[li] = np_new;
-                atomicAdd(&c.ctrl[CTRL_STEP_PAGES], 1);
+                atomicAdd(&s_grants, 1);
               }
               const int hs = (fuse_decide || c.alpha_per != DMS_ALPHA_PER_LAYER) ? h : 0;
               const float av = s_alpha[k] == s_alpha[k] ? s_alpha[k] : __ldcg(&alpha[b * c.Hkv + hs]);
@@ -1125,23 +1126,13 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
   }
 
   if (FUSED) {
-    // the grid's last CTA advances the page counter and the positions
+    // the grid's last CTA advances the page counter and the positions (every
+    // CTA's aux warp read the counter, and every head its position, before
+    // this barrier)
     __syncthreads();
-    if (tid == 0) {
-      __threadfence();
-      s_last = (atomicAdd(&c.ctrl[CTRL_GRID_DONE], 1) == G - 1) ? 1 : 0;
-    }
+    if (tid == 0) s_last = count_step(c, s_grants, G, s_next_page0) ? 1 : 0;
     __syncthreads();
-    if (s_last) {
-      __threadfence();
-      if (tid == 0) {
-        const int granted = __ldcg(&c.ctrl[CTRL_STEP_PAGES]);
-        c.ctrl[CTRL_NEXT_PAGE] = min(__ldcg(&c.ctrl[CTRL_NEXT_PAGE]) + granted, c.pool_pages);
-        c.ctrl[CTRL_STEP_PAGES] = 0;
-        c.ctrl[CTRL_GRID_DONE] = 0;
-      }
-      for (int bb = tid; bb < c.B; bb += kFlatThreads) c.pos[layer * c.B + bb] += 1;
-    }
+    if (s_last) advance_positions(c, layer, tid, kFlatThreads);
   }
   FLAT_MARK(9);
 }
