@@ -85,3 +85,42 @@ def test_null_handles_rejected(B):
     assert B._lib.dms_cache_reset(None, None) == B.DMS_ERR_INVALID
     assert B._lib.dms_prefill(None, 0, None, None) == B.DMS_ERR_INVALID
     assert B._lib.dms_decode_step(None, 0, None, None) == B.DMS_ERR_INVALID
+
+
+def test_every_entry_point_rejects_bad_arguments(B):
+    """Argument checks happen on the host before any CUDA call: null handles,
+    null outputs, layers out of range and caller buffers that are missing,
+    misaligned or too small all come back as error codes."""
+    import ctypes as C
+    L = B._lib
+    inv = B.DMS_ERR_INVALID
+    d = good_desc(B)
+    n = C.c_size_t(0)
+    assert L.dms_cache_bytes(None, C.byref(n)) == inv
+    assert L.dms_cache_bytes(C.byref(d), None) == inv
+    # alloc: output handle, descriptor, buffer (never dereferenced: every
+    # check below returns before the pointer is used)
+    out = C.c_void_p(1)
+    need = B.dms_cache_bytes(d)
+    fake = 1 << 20  # 256-byte aligned, not a real allocation
+    assert L.dms_cache_alloc(C.byref(d), C.c_void_p(fake), need, None, None) == inv
+    assert L.dms_cache_alloc(None, C.c_void_p(fake), need, None, C.byref(out)) == inv and out.value is None
+    assert L.dms_cache_alloc(C.byref(d), None, need, None, C.byref(out)) == inv
+    assert L.dms_cache_alloc(C.byref(d), C.c_void_p(fake + 8), need, None, C.byref(out)) == inv
+    assert L.dms_cache_alloc(C.byref(d), C.c_void_p(fake), need - 1, None, C.byref(out)) == B.DMS_ERR_NOMEM
+    # every call on a null cache
+    lay = B.dms_cache_layout()
+    view = B.dms_cache_view()
+    st = C.c_int(0)
+    alpha = C.c_void_p(fake)
+    assert L.dms_cache_get_layout(None, C.byref(lay)) == inv
+    assert L.dms_cache_export(None, 0, C.byref(view), None) == inv
+    assert L.dms_cache_status(None, None, C.byref(st)) == inv
+    assert L.dms_cache_positions(None, 0) == inv
+    assert L.dms_decide(None, 16, None, None, alpha, None) == inv
+    assert L.dms_prefill_compact(None, 0, None, None) == inv
+    assert L.dms_prefill_attention(None, 0, None, None) == inv
+    assert L.dms_decode_append(None, 0, None, None) == inv
+    assert L.dms_decode_attention(None, 0, alpha, alpha, None) == inv
+    assert L.dms_decode_attention_noalloc(None, 0, alpha, alpha, None) == inv
+
