@@ -1,0 +1,37 @@
+"""Host logic of bench.py (no GPU): which decode kernel a workload's line
+names, and the recorded DRAM traffic, which is reported only while the
+kernel's sources are the ones the capture was taken on."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+@pytest.mark.parametrize("name,kernel", [("qwen8b", "k_decode_cluster"), ("qwen8b_c8", "k_decode_flat"),
+                                         ("llama1b", "k_decode_cluster"), ("reason36", "k_decode_flat")])
+def test_decode_kernel_name_follows_auto_rule(name, kernel):
+    wl = bench.I.WORKLOADS[name]
+    assert bench.decode_kernel_name(wl, "auto", 148) == kernel
+    # an explicit choice is taken as given
+    assert bench.decode_kernel_name(wl, "flat", 148) == "k_decode_flat"
+    assert bench.decode_kernel_name(wl, "cluster", 148) == "k_decode_cluster"
+
+
+def test_recorded_traffic_only_for_current_sources(monkeypatch):
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    assert rows, "profiles/traffic.txt lists no capture"
+    kernel, workload, nbytes, digest = rows[0][:4]
+    expect = int(nbytes) if bench.source_digest(kernel) == digest else None
+    assert bench.recorded_traffic(kernel, workload) == expect
+    # once the sources differ from the captured ones, nothing is reported
+    monkeypatch.setattr(bench, "source_digest", lambda k: "0" * 16)
+    assert bench.recorded_traffic(kernel, workload) is None
+    monkeypatch.undo()
+    assert bench.recorded_traffic(kernel, "no_such_workload") is None
+    assert bench.recorded_traffic("k_not_recorded", workload) is None
+
