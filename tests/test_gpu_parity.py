@@ -62,6 +62,9 @@ CASES = {
     # each, the last page ragged
     "bf16_key_rope_p256": Case(B=2, T=2500, steps=16, Hq=8, Hkv=2, D=128, w=320, P=256, act="bf16", kv="bf16",
                                source="key", keep=0.2, rope=True, attn_rows=128, seed=21),
+    # fp32 pages of 256 slots: eight 32-row scatter groups per page, the last page ragged
+    "f32_p256_scatter": Case(B=1, T=700, steps=10, Hq=4, Hkv=2, D=128, w=320, P=256, act="f32", kv="f32",
+                             source="input", keep=0.3, attn_rows=64, seed=33),
     # second layer of a two-layer cache with preallocation
     "layer1_of_2": Case(B=2, T=260, steps=12, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16",
                         source="input", keep=0.3, layers=2, layer=1, prealloc=64, seed=15),
