@@ -104,6 +104,33 @@ __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// Rotary embedding of one pair (x_i, x_{i+D/2}) by the table entries (c, s), in
+// fp64.  Each product of a bf16 or fp32 element with an fp32 table entry has at
+// most 48 significant bits and is exact in fp64, so each output is the exact
+// rotation rounded once.
+__device__ __forceinline__ void rotate64(double a, double b, double c, double s, double& y0, double& y1) {
+  y0 = __dsub_rn(__dmul_rn(a, c), __dmul_rn(b, s));
+  y1 = __dadd_rn(__dmul_rn(b, c), __dmul_rn(a, s));
+}
+
+// fp64 -> bf16 with one round-to-nearest-even step: the value is first
+// narrowed to fp32 rounding to odd (truncate, then set the last bit when
+// anything was dropped), which keeps 16 more bits than bf16 carries, so the
+// final fp32 -> bf16 rounding decides exactly as a direct rounding would.
+__device__ __forceinline__ float f64_to_f32_odd(double x) {
+  float r = __double2float_rz(x);
+  if (static_cast<double>(r) != x) r = __int_as_float(__float_as_int(r) | 1);
+  return r;
+}
+template <typename T>
+__device__ __forceinline__ T from_f64(double x);
+template <>
+__device__ __forceinline__ float from_f64<float>(double x) { return __double2float_rn(x); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f64<__nv_bfloat16>(double x) {
+  return __float2bfloat16_rn(f64_to_f32_odd(x));
+}
+
 // Unpack a 16-byte vector into floats (8 bf16 or 4 fp32).
 template <typename T>
 struct Vec16 {
@@ -212,6 +239,10 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, cons
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+// Two fp64 values rounded once each (see f64_to_f32_odd) into a bf16 pair.
+__device__ __forceinline__ uint32_t pack_bf16_f64(double lo, double hi) {
+  return pack_bf16(f64_to_f32_odd(lo), f64_to_f32_odd(hi));
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, int count) {

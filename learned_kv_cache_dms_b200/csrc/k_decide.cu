@@ -536,10 +536,11 @@ __global__ void k_neuron_rope(CacheView c, int T, const int* pos_dev, TA* q, TA*
     if (cos_t) {
       const int p = pos_dev ? pos_dev[b] + t : t;
       const float cv = cos_t[static_cast<long>(p) * half + i], sv = sin_t[static_cast<long>(p) * half + i];
-      // each product and sum rounded separately (no fused multiply-add), so
-      // the stored value does not depend on contraction choices
-      row[i] = from_f<TA>(__fsub_rn(__fmul_rn(x0, cv), __fmul_rn(x1, sv)));
-      row[i + half] = from_f<TA>(__fadd_rn(__fmul_rn(x1, cv), __fmul_rn(x0, sv)));
+      // the rotation in fp64, rounded once into the activation dtype
+      double y0, y1;
+      rotate64(x0, x1, cv, sv, y0, y1);
+      row[i] = from_f64<TA>(y0);
+      row[i + half] = from_f64<TA>(y1);
     } else {
       row[i + half] = from_f<TA>(x1);
     }
@@ -580,6 +581,16 @@ __device__ __forceinline__ void st4<float>(float* p, const float* f) {
   *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
 }
 
+// An fp64 rotation result narrowed to fp32 so that st4's conversion into the
+// activation dtype rounds it exactly once: bf16 rows keep it rounded to odd
+// (st4 then rounds to nearest even), fp32 rows round it to nearest even here.
+template <typename TA>
+__device__ __forceinline__ float narrow_f64(double x);
+template <>
+__device__ __forceinline__ float narrow_f64<float>(double x) { return __double2float_rn(x); }
+template <>
+__device__ __forceinline__ float narrow_f64<__nv_bfloat16>(double x) { return f64_to_f32_odd(x); }
+
 template <typename TA>
 __global__ void k_neuron_rope4(CacheView c, int T, const int* pos_dev, TA* q, TA* k, const float* offset, int ostride,
                                int do_alpha, float* alpha, const float* cos_t, const float* sin_t) {
@@ -619,9 +630,12 @@ __global__ void k_neuron_rope4(CacheView c, int T, const int* pos_dev, TA* q, TA
     float y0[4], y1[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      // each product and sum rounded separately (no fused multiply-add)
-      y0[e] = __fsub_rn(__fmul_rn(x0[e], cv[e]), __fmul_rn(x1[e], sv[e]));
-      y1[e] = __fadd_rn(__fmul_rn(x1[e], cv[e]), __fmul_rn(x0[e], sv[e]));
+      // the rotation in fp64, narrowed so that st4's rounding into the
+      // activation dtype is the only rounding of the exact rotation's fp64 value
+      double r0, r1;
+      rotate64(x0[e], x1[e], cv[e], sv[e], r0, r1);
+      y0[e] = narrow_f64<TA>(r0);
+      y1[e] = narrow_f64<TA>(r1);
     }
     st4<TA>(row + i, y0);
     st4<TA>(row + i + half, y1);
@@ -691,12 +705,13 @@ __global__ void __launch_bounds__(256, 3) k_neuron_rope8(CacheView c, int T, con
         uint32_t y0[4], y1[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          // each product and sum rounded separately (no fused multiply-add)
+          // the rotation in fp64, rounded once into bf16
           const int j = 2 * e;
-          y0[e] = pack_bf16(__fsub_rn(__fmul_rn(a0[j], cv[j]), __fmul_rn(a1[j], sv[j])),
-                            __fsub_rn(__fmul_rn(a0[j + 1], cv[j + 1]), __fmul_rn(a1[j + 1], sv[j + 1])));
-          y1[e] = pack_bf16(__fadd_rn(__fmul_rn(a1[j], cv[j]), __fmul_rn(a0[j], sv[j])),
-                            __fadd_rn(__fmul_rn(a1[j + 1], cv[j + 1]), __fmul_rn(a0[j + 1], sv[j + 1])));
+          double r0a, r1a, r0b, r1b;
+          rotate64(a0[j], a1[j], cv[j], sv[j], r0a, r1a);
+          rotate64(a0[j + 1], a1[j + 1], cv[j + 1], sv[j + 1], r0b, r1b);
+          y0[e] = pack_bf16_f64(r0a, r0b);
+          y1[e] = pack_bf16_f64(r1a, r1b);
         }
         __nv_bfloat16* row = r < c.Hq ? qrow + r * D : krow + (r - c.Hq) * D;
         *reinterpret_cast<uint4*>(row) = make_uint4(y0[0], y0[1], y0[2], y0[3]);

@@ -15,7 +15,7 @@
 // precision": the FP8 page scale and the FP8 codes are computed in fp32, which is
 // the precision the quantiser on the GPU uses (the pages fix no precision).
 //
-// Conventions the pages leave open (each is also listed in the design notes):
+// Conventions the pages leave open:
 //  * A decision logit alpha_t is computed from token t's own hidden state (or
 //    key/query neuron) and decides the fate of key t (no shift).
 //  * Key j is visible to query i iff j <= i and (i - j < w or alpha_j <= 0).
@@ -333,11 +333,10 @@ void oracle_decide_neuron(int B, int T, int Hsrc, int D, int group, int Hkv, dou
 
 // Rotary embedding, half-split form: for i < D/2 the pair (x_i, x_{i+D/2}) is
 // rotated by the angle of (position, i), with cos/sin read from caller tables
-// [max_pos, D/2].  x is [B,T,H,D]; token t sits at position pos0 + t.
-// Computed in fp32 with each product and sum rounded separately
-// (x_i' = fl(fl(x_i c) - fl(x_{i+D/2} s)), x_{i+D/2}' = fl(fl(x_{i+D/2} c) + fl(x_i s))):
-// the rotated keys are stored in the activation dtype and their FP8 codes are
-// integer decisions, so the oracle rounds exactly as the kernel does.
+// [max_pos, D/2]:  x_i' = x_i c - x_{i+D/2} s,  x_{i+D/2}' = x_{i+D/2} c + x_i s.
+// x is [B,T,H,D] (fp64, modified in place); token t sits at position pos0 + t.
+// Plain fp64; the caller rounds the result once into the activation dtype when
+// it is stored (oracle_round_bf16_n for bf16).
 void oracle_rope(int B, int T, int H, int D, double* x, int pos0, const double* cos_t,
                  const double* sin_t) {
   const int half = D / 2;
@@ -348,13 +347,33 @@ void oracle_rope(int B, int T, int H, int D, double* x, int pos0, const double* 
         const double* c = cos_t + static_cast<size_t>(pos0 + t) * half;
         const double* s = sin_t + static_cast<size_t>(pos0 + t) * half;
         for (int i = 0; i < half; ++i) {
-          const float a = static_cast<float>(e[i]), bb = static_cast<float>(e[i + half]);
-          const float cf = static_cast<float>(c[i]), sf = static_cast<float>(s[i]);
-          const float ac = a * cf, bs = bb * sf, bc = bb * cf, as = a * sf;
-          e[i] = static_cast<double>(ac - bs);
-          e[i + half] = static_cast<double>(bc + as);
+          const double a = e[i], bb = e[i + half];
+          e[i] = a * c[i] - bb * s[i];
+          e[i + half] = bb * c[i] + a * s[i];
         }
       }
+}
+
+// Round fp64 values to bfloat16 (1 sign bit, 8 exponent bits with bias 127, 7
+// stored mantissa bits: 8 significant bits for normal numbers, a fixed quantum
+// of 2^-133 below the smallest normal 2^-126), to nearest with ties to even, in
+// one step.  Results are returned as the fp32 numbers they denote; values that
+// round past the largest finite bf16 (0x7F7F) become infinities.
+void oracle_round_bf16_n(const double* x, float* out, long n) {
+  const double max_bf16 = std::ldexp(255.0, 120);  // 1.9921875 * 2^127
+  for (long idx = 0; idx < n; ++idx) {
+    const double v = x[idx];
+    if (std::isnan(v) || std::isinf(v) || v == 0.0) {
+      out[idx] = static_cast<float>(v);
+      continue;
+    }
+    int e;
+    std::frexp(std::fabs(v), &e);  // |v| in [2^(e-1), 2^e)
+    const int q = std::max(e - 8, -133);  // exponent of the quantum
+    double r = std::ldexp(rne(std::ldexp(std::fabs(v), -q)), q);
+    if (r > max_bf16) r = INFINITY;
+    out[idx] = static_cast<float>(std::signbit(v) ? -r : r);
+  }
 }
 
 // DMS-masked prefill attention ([DMS-Qwen3], attention: the sliding window plus

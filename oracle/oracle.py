@@ -30,6 +30,7 @@ def lib():
         L.oracle_decide_proj.argtypes = [C.c_int] * 4 + [dp] * 5 + [C.c_double, C.c_double, C.c_int, dp]
         L.oracle_decide_neuron.argtypes = [C.c_int] * 6 + [dp, dp, C.c_double, C.c_int, dp]
         L.oracle_rope.argtypes = [C.c_int] * 4 + [dp, C.c_int, dp, dp]
+        L.oracle_round_bf16_n.argtypes = [dp, fp, C.c_long]
         L.oracle_prefill_attention.argtypes = [C.c_int] * 6 + [dp, dp, dp, up, ip, C.c_long, dp]
         L.oracle_cache_new.argtypes = [C.c_int] * 11
         L.oracle_cache_new.restype = C.c_void_p
@@ -122,6 +123,21 @@ def rope(x, pos0, cos, sin):
     sin = _f64(sin)
     lib().oracle_rope(B, T, H, D, _p(x, C.c_double), int(pos0), _p(cos, C.c_double), _p(sin, C.c_double))
     return x
+
+
+def round_bf16(x):
+    """fp64 values rounded once (nearest, ties to even) to bfloat16; returned as fp64."""
+    x = _f64(x)
+    out = np.empty(x.shape, np.float32)
+    lib().oracle_round_bf16_n(_p(x, C.c_double), _p(out, C.c_float), x.size)
+    return out.astype(np.float64)
+
+
+def round_to(x, dtype):
+    """fp64 values stored in the activation dtype ("f32" or "bf16"), one rounding."""
+    if dtype == "bf16":
+        return round_bf16(x)
+    return _f64(x).astype(np.float32).astype(np.float64)
 
 
 def evict_bits(alpha, disable_eviction=False):

@@ -121,8 +121,80 @@ def test_rope_matches_complex_rotation():
     ang = rng.uniform(-3, 3, (10, D // 2))
     y = O.rope(x, 2, np.cos(ang), np.sin(ang))
     z = (x[..., : D // 2] + 1j * x[..., D // 2:]) * np.exp(1j * ang[2:2 + T])[None, :, None, :]
-    assert np.allclose(y[..., : D // 2], z.real, atol=1e-5)
-    assert np.allclose(y[..., D // 2:], z.imag, atol=1e-5)
+    assert np.allclose(y[..., : D // 2], z.real, rtol=0, atol=1e-12)
+    assert np.allclose(y[..., D // 2:], z.imag, rtol=0, atol=1e-12)
+
+
+def test_rope_fp32_tables_exact_products():
+    # bf16 elements times fp32 table entries: both products are exact in fp64,
+    # so each rotated value is the exact rotation (rational arithmetic) rounded once
+    from fractions import Fraction as F
+    rng = np.random.default_rng(5)
+    D = 8
+    x = O.round_bf16(rng.standard_normal((1, 3, 1, D)) * 3)
+    ang = rng.uniform(-3, 3, (3, D // 2))
+    c, s = np.cos(ang).astype(np.float32).astype(np.float64), np.sin(ang).astype(np.float32).astype(np.float64)
+    y = O.rope(x, 0, c, s)
+    for t in range(3):
+        for i in range(D // 2):
+            a, b = F(x[0, t, 0, i]), F(x[0, t, 0, i + D // 2])
+            ex0 = a * F(c[t, i]) - b * F(s[t, i])
+            ex1 = b * F(c[t, i]) + a * F(s[t, i])
+            assert y[0, t, 0, i] == float(ex0)            # float(Fraction) rounds to nearest
+            assert y[0, t, 0, i + D // 2] == float(ex1)
+
+
+def _bf16_neighbours(v):
+    """The two bf16 values bracketing the rational v (exact, by enumeration of the grid)."""
+    from fractions import Fraction as F
+    import math
+    if v == 0:
+        return F(0), F(0)
+    a = abs(v)
+    e = math.floor(math.log2(a))
+    while F(2) ** e > a:
+        e -= 1
+    while F(2) ** (e + 1) <= a:
+        e += 1
+    q = F(2) ** max(e - 7, -133)          # quantum of bf16 at this magnitude
+    lo = (a // q) * q
+    hi = lo if lo == a else lo + q
+    return (lo, hi) if v > 0 else (-hi, -lo)
+
+
+def test_round_bf16_definition():
+    # nearest bf16, ties to the even mantissa, against exact rational arithmetic
+    from fractions import Fraction as F
+    rng = np.random.default_rng(6)
+    xs = list(rng.standard_normal(3000) * 10.0 ** rng.integers(-6, 6, 3000))
+    # exact midpoints and values one fp64 ulp either side of them
+    for m in rng.integers(128, 256, 200):
+        for e in (-20, -3, 0, 5):
+            mid = (float(m) + 0.5) * 2.0 ** (e - 7)
+            xs += [mid, np.nextafter(mid, 0), np.nextafter(mid, np.inf), -mid]
+    xs += [2.0 ** -130 * 1.37, -(2.0 ** -133) * 0.5, 2.0 ** -133 * 1.5]   # subnormal range
+    x = np.array(xs, np.float64)
+    r = O.round_bf16(x)
+    for xv, rv in zip(x, r):
+        v = F(float(xv))
+        lo, hi = _bf16_neighbours(v)
+        dlo, dhi = v - lo, hi - v
+        if dlo < dhi:
+            want = lo
+        elif dhi < dlo:
+            want = hi
+        else:   # tie: the neighbour whose last mantissa bit is 0
+            q = hi - lo
+            want = lo if (lo / q) % 2 == 0 else hi
+        assert F(float(rv)) == want, (xv, rv, float(want))
+
+
+def test_round_bf16_matches_torch_on_fp32_values():
+    # for inputs that are fp32 numbers, rounding to bf16 is a single step in torch too
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal(200000) * 10.0 ** rng.integers(-8, 8, 200000)).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(O.round_bf16(x.astype(np.float64)), want)
 
 
 def test_rope_relative_position():
