@@ -192,7 +192,8 @@ typedef struct dms_decide_params {
  * Page grants of one call go to (b, h) in row-major order from one ascending
  * counter. */
 typedef struct dms_prefill_args {
-  int seq_len;              /* T, 1 <= T <= max_positions                          */
+  int seq_len;              /* T, 1 <= T <= min(max_positions, 262144 = 2^18)
+                               (DMS_ERR_INVALID otherwise)                         */
   void* q;                  /* device [B,T,Hq,D] act dtype (rotated in place)     */
   void* k;                  /* device [B,T,Hkv,D] act dtype (rotated/zeroed in place) */
   const void* v;            /* device [B,T,Hkv,D] act dtype                        */
@@ -318,10 +319,14 @@ DMS_API int dms_decode_attention(dms_cache* cache, int layer, const void* q, voi
  * partials -- e.g. an engine whose device memory is handed out by its own
  * fixed pool at start-up and whose decode loop must never reach cudaMalloc
  * (cudaMalloc can synchronise the device and can fail once the pool owns the
- * memory).  Same arguments, same result as dms_decode_attention; the partial
+ * memory).  Same arguments as dms_decode_attention, and the same result within the
+ * decode attention tolerance (it runs another kernel, k_decode_attn, whose
+ * splits and merge order differ, so the two are not bit-identical); the partial
  * results of the splits live instead in one fixed array of device memory that
  * the library holds (4 MiB per GPU that loads the library, kept until exit).
- *  - Limit: the cache's worst case of split-K scratch, one int per (b, h) for
+ * fp32 caches need no partials: their attention runs one CTA per query head,
+ * with no limit and nothing shared.
+ *  - Limit (bf16 and FP8 pages): the cache's worst case of split-K scratch, one int per (b, h) for
  *    the per-head arrival counters (rounded up to 256 bytes) plus
  *    items_cap * (Hq/Hkv) * (head_dim + 2) * 4 bytes of partials with
  *    items_cap = max(B * Hkv * ceil(max_positions / block), 640) + B * Hkv,

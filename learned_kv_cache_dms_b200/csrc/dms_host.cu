@@ -664,20 +664,22 @@ constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB per device
 static __device__ __align__(256) unsigned char g_split_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
 void* g_split_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_split_scratch on `device`.  In host code the symbol is
 // only a host-side stand-in; the real address comes from cudaGetSymbolAddress
-// with that device current.
+// with that device current.  The lookup runs once per device, under a lock.
 int split_scratch_address(int device, void** out) {
   if (device < 0 || device >= kMaxDevices) return DMS_ERR_INVALID;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
   if (!g_split_scratch_addr[device]) {
     int prev = -1;
     if (cudaGetDevice(&prev) != cudaSuccess) return DMS_ERR_CUDA;
     if (prev != device && cudaSetDevice(device) != cudaSuccess) return DMS_ERR_CUDA;
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_split_scratch);
-    if (prev != device) cudaSetDevice(prev);
+    if (prev != device && cudaSetDevice(prev) != cudaSuccess) return DMS_ERR_CUDA;
     if (e != cudaSuccess || p == nullptr) return DMS_ERR_CUDA;
     g_split_scratch_addr[device] = p;
   }
@@ -690,6 +692,14 @@ int split_scratch_address(int device, void** out) {
 extern "C" int dms_decode_attention_noalloc(dms_cache* c, int layer, const void* q, void* o, void* stream) {
   if (!c || !q || !o || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
   if (c->worklist_layer != layer) return DMS_ERR_STATE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (c->desc.kv_dtype == DMS_F32) {
+    // fp32 pages: one CTA per query head, no split-K partials, no scratch
+    track_launch(c, layer, st);
+    return launch_decode_attention(c->view, layer, q, o, nullptr, nullptr, c->num_sms, st) == cudaSuccess
+               ? DMS_OK
+               : DMS_ERR_CUDA;
+  }
   const size_t g = static_cast<size_t>(c->desc.num_q_heads / c->desc.num_kv_heads);
   const size_t items = static_cast<size_t>(c->plan.items_cap);
   const size_t heads = static_cast<size_t>(c->desc.batch) * c->desc.num_kv_heads;
@@ -705,10 +715,10 @@ extern "C" int dms_decode_attention_noalloc(dms_cache* c, int layer, const void*
   v.head_done = reinterpret_cast<int*>(p);  // per-head arrival counters: must start at zero
   v.part_acc = reinterpret_cast<float*>(p + cnt_bytes);
   v.part_ml = reinterpret_cast<float*>(p + cnt_bytes + acc_bytes);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  track_launch(c, layer, st);
   if (cudaMemsetAsync(v.head_done, 0, heads * sizeof(int), st) != cudaSuccess) return DMS_ERR_CUDA;
   if (launch_decode_attention(v, layer, q, o, c->has_maps ? &c->kmap : nullptr, c->has_maps ? &c->vmap : nullptr,
-                              c->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+                              c->num_sms, st) != cudaSuccess)
     return DMS_ERR_CUDA;
   return DMS_OK;
 }

@@ -68,25 +68,6 @@ __device__ __forceinline__ int4* plan_at(const CacheView& c, long li, int t) {
   return c.plan + static_cast<long>(t & 1) * c.L * c.B * c.Hkv + li;
 }
 
-// Phase timeline (tracing builds only, compiled with -DDMS_TRACE): thread 0 of
-// each CTA stores %globaltimer for phase `slot` of kernel `kid` into a
-// per-translation-unit device array read back by dms_debug_trace_read.
-#ifdef DMS_TRACE
-constexpr int kTraceCtas = 4096, kTraceSlots = 32;
-#define DMS_TRACE_MARK(kid, slot)                                                                   \
-  do {                                                                                              \
-    if (threadIdx.x == 0 && blockIdx.x < kTraceCtas) {                                              \
-      unsigned long long t_;                                                                        \
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                        \
-      g_dms_trace[((kid) * kTraceCtas + blockIdx.x) * kTraceSlots + (slot)] = t_;                   \
-    }                                                                                               \
-  } while (0)
-#else
-#define DMS_TRACE_MARK(kid, slot) \
-  do {                            \
-  } while (0)
-#endif
-
 // ---------------------------------------------------------------------------
 // Element helpers
 // ---------------------------------------------------------------------------

@@ -40,22 +40,6 @@
 
 namespace dms {
 
-#ifdef DMS_TRACE
-__device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
-// per-tile marks of the first CTA of the grid (row = tile), by one thread
-#define PF_MARK(tile, slot)                                                                          \
-  do {                                                                                               \
-    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (tile) < kTraceCtas) {              \
-      unsigned long long t_;                                                                         \
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                         \
-      g_dms_trace[static_cast<long>(tile) * kTraceSlots + (slot)] = t_;                              \
-    }                                                                                                \
-  } while (0)
-#else
-#define PF_MARK(tile, slot) \
-  do {                      \
-  } while (0)
-#endif
 
 constexpr int kPfRows = 128;     // query rows per Q tile (TMEM lanes)
 constexpr int kPfQT = 2;         // Q tiles per CTA
@@ -320,7 +304,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             give_up();
             break;
           }
-          PF_MARK(t, 12);
           const bool kt = j < it.nkt;
           const int jb = kt ? j * kPfBN : it.jlo + (j - it.nkt) * kPfBN;
           mbar_expect_tx(&k_full[st], L::KV_BYTES);
@@ -331,7 +314,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             else
               tma_load_3d(dk, &kmap, hf * 64, it.h, it.b * T + jb, &k_full[st]);
           }
-          PF_MARK(t, 13);
         }
         it = item(k + 1, use_late(nk_next));
       }
@@ -372,9 +354,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // S(t) = Q K(t)^T; after the item's last scores Q may be replaced
       auto issue_s = [&](int t, bool last_of_item) -> bool {
         const int st = t % ST;
-        PF_MARK(t, 16 * qt + 8);
         if (!mbar_wait_bounded(&k_full[st], (t / ST) & 1)) return false;
-        PF_MARK(t, 16 * qt + 9);
         tc_fence_after();
         const uint32_t qa = smem_u32(sb + L::OFF_Q + qt * L::Q_BYTES);
         const uint32_t ka = smem_u32(sb + L::OFF_K + st * L::KV_BYTES);
@@ -395,10 +375,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       auto issue_pv = [&](int t, int j, int k) -> bool {
         const int st = t % ST;
         if (!mbar_wait_bounded(&v_full[st], (t / ST) & 1)) return false;
-        PF_MARK(t, 16 * qt + 10);
         if (!mbar_wait_bounded(&p_full[qt], t & 1)) return false;
         if (j == 0 && k > 0 && !mbar_wait_bounded(&o_free[qt], (k - 1) & 1)) return false;
-        PF_MARK(t, 16 * qt + 11);
         tc_fence_after();
         const uint32_t va = smem_u32(sb + L::OFF_V + st * L::KV_BYTES);
 #pragma unroll
@@ -469,9 +447,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int jb = kt ? j * kPfBN : it.jlo + (j - it.nkt) * kPfBN;
         const int c_lo = max(kt ? 0 : blo - jb, 0), c_hi = min(kt ? ck - 1 - jb : bhi - jb, kPfBN - 1);
         const bool row_full = c_lo == 0 && c_hi == kPfBN - 1;
-        if (row == 0) PF_MARK(t, 16 * qt + 0);
         ok = ok && mbar_wait_bounded(&s_full[qt], t & 1);
-        if (row == 0) PF_MARK(t, 16 * qt + 1);
         tc_fence_after();
         uint32_t sr[kPfBN];
         if (ok) {
@@ -485,7 +461,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (ok && lane == 0) mbar_arrive(&s_free[qt]);  // S may be overwritten by the next tile's scores
-        if (row == 0) PF_MARK(t, 16 * qt + 2);
         // raw scores with the invisible ones at -inf; row max over 4 chains
         float sv[kPfBN];
         if (__all_sync(0xffffffffu, row_full)) {
@@ -516,13 +491,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           l_row *= factor;
         }
         const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a fully masked row so far: all p = 0
-        if (row == 0) PF_MARK(t, 16 * qt + 6);
         if (qt == 0) {
           if (t > 0) named_sync<2>();
         } else {
           named_sync<1>();
         }
-        if (row == 0) PF_MARK(t, 16 * qt + 7);
         const float neg_m = *reinterpret_cast<volatile float*>(&s_turn_zero) - m_use;
         const uint64_t nm2 = f2_pack(neg_m, neg_m);
         uint32_t pk[kPfBN / 2];
@@ -549,12 +522,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             named_arrive<2>();
         }
         l_row += psum;
-        if (row == 0) PF_MARK(t, 16 * qt + 3);
         // P V of the previous tile has finished with P and with O (for the
         // item's first tile the previous item's epilogue waited for it)
         if (j > 0) ok = ok && mbar_wait_bounded(&pv_done[qt], (t - 1) & 1);
         tc_fence_after();
-        if (row == 0) PF_MARK(t, 16 * qt + 4);
         if (ok && j > 0 && __any_sync(0xffffffffu, raise && factor != 1.0f)) {
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
@@ -570,13 +541,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_before();
         __syncwarp();  // the warp's P rows and O rescale precede lane 0's release
         if (ok && lane == 0) mbar_arrive(&p_full[qt]);
-        if (row == 0) PF_MARK(t, 16 * qt + 5);
         if (s_abort) ok = false;
       }
       // the item's last P V, then O / l; O is released to the next item as
       // soon as it is in registers
       ok = ok && mbar_wait_bounded(&pv_done[qt], (t - 1) & 1);
-      if (row == 0) PF_MARK(t - 1, 16 * qt + 14);
       tc_fence_after();
       // read O, release it, write O / l (bf16, 64-column boxes) to this
       // group's staging tile once the previous item's TMA stores have read
@@ -605,7 +574,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (row == 0) PF_MARK(t - 1, 16 * qt + 15);
       if (ok && lane == 0) mbar_arrive(&o_free[qt]);
       if (store) {
         fence_proxy_async();  // the tile visible to the TMA
@@ -616,10 +584,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           bulk_commit();
         }
       }
-      if (row == 0) PF_MARK(t, 16 * qt + 14);
       it = item(k + 1, use_late(nk_next));
       ck = use_late(ck_next);
-      if (row == 0) PF_MARK(t, 16 * qt + 15);
     }
     if (qt == 0 && t > 0) named_sync<2>();  // WG1's last hand-back
     if (row == 0) bulk_wait0();                 // this group's stores complete before the CTA ends
@@ -650,9 +616,3 @@ cudaError_t launch_prefill_attention_tc(const CacheView& c, int T, void* o, cons
 
 }  // namespace dms
 
-#ifdef DMS_TRACE
-extern "C" __attribute__((visibility("default"))) int dms_debug_trace_read_prefill(void* host, size_t bytes) {
-  const size_t n = sizeof(dms::g_dms_trace) < bytes ? sizeof(dms::g_dms_trace) : bytes;
-  return cudaMemcpyFromSymbol(host, dms::g_dms_trace, n) == cudaSuccess ? 0 : -3;
-}
-#endif

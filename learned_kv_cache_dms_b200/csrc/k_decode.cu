@@ -4,9 +4,6 @@
 
 namespace dms {
 
-#ifdef DMS_TRACE
-__device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
-#endif
 
 // ---------------------------------------------------------------------------
 // Append of token t for every (b, h) of one layer, one CTA per (b, h):
@@ -37,7 +34,6 @@ __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, i
   const int b = bh / c.Hkv, h = bh % c.Hkv;
   const long lbase = static_cast<long>(layer) * BH, li = lbase + bh;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, w = c.w, P = c.P, D = c.D;
-  DMS_TRACE_MARK(1, 0);
   // every read of this CTA's state first (one round trip; the plan needs t)
   const int t = c.pos[layer * c.B + b];
   const int next_page0 = c.ctrl[CTRL_NEXT_PAGE];
@@ -91,7 +87,6 @@ __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, i
     }
     __syncthreads();
   }
-  DMS_TRACE_MARK(1, 1);
 
   // rank among the lower heads needing a new page (their plans for t)
   const int flags = pl.y, slot = pl.x, cnt = pl.z, have = pl.w;
@@ -191,7 +186,6 @@ __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, i
   }
   __syncthreads();
   if (s_last) advance_positions(c, layer, tid, kAppendThreads);
-  DMS_TRACE_MARK(1, 3);
 }
 
 template <typename TA, bool FP8>
@@ -288,7 +282,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_attn(CacheView c, int layer
 
   const int tid = threadIdx.x;
   const long lbase = static_cast<long>(layer) * BH;
-  DMS_TRACE_MARK(0, 0);
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&full_bar[i], 1);
     fence_mbar_init();
@@ -296,7 +289,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_attn(CacheView c, int layer
   }
   const int C = decode_partition(c.count + lbase, BH, c.P, target_items, s_cnt, s_off, s_red);
   const int nitems = s_off[BH];
-  DMS_TRACE_MARK(0, 1);
 
   // producer iterator (thread 0 only)
   int p_item = blockIdx.x, p_sub = 0, p_bh = 0;
@@ -355,7 +347,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_attn(CacheView c, int layer
     }
     const StageMeta m = meta[stage];
     const int bh = m.bh, b = bh / c.Hkv, h = bh % c.Hkv;
-    if (n == 0) DMS_TRACE_MARK(0, 2);
     const unsigned char* kt = stage_buf + stage * S::STAGE;
     if (FP8) {
       widen_fp8_subtile<D>(kt, conv_buf);
@@ -381,7 +372,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_attn(CacheView c, int layer
     if (tid == 0 && produce(stage)) ++produced;
 
     if (m.last) {
-      if (n == 0) DMS_TRACE_MARK(0, 3);
       warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
       __syncthreads();
       merge_to_global<D>(merge, 4, g, 1.0f, c.part_acc, c.part_ml, m.item);
@@ -394,17 +384,14 @@ __global__ void __launch_bounds__(kThreads) k_decode_attn(CacheView c, int layer
         s_last = (atomicAdd(&c.head_done[bh], 1) == nh - 1) ? 1 : 0;
       }
       __syncthreads();
-      DMS_TRACE_MARK(0, 4);
       if (s_last) {
         __threadfence();
         combine_head<D>(c.part_acc, c.part_ml, g, s_off[bh], s_off[bh + 1],
                         o + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D, wbuf);
         if (tid == 0) c.head_done[bh] = 0;
-        DMS_TRACE_MARK(0, 5);
       }
     }
   }
-  DMS_TRACE_MARK(0, 6);
 }
 
 template <int D, bool FP8>
@@ -441,14 +428,3 @@ cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q
 
 }  // namespace dms
 
-#ifdef DMS_TRACE
-// Copy the phase timeline to the host (tracing builds only).
-extern "C" __attribute__((visibility("default"))) int dms_debug_trace_read(void* host, size_t bytes) {
-  const size_t n = sizeof(dms::g_dms_trace) < bytes ? sizeof(dms::g_dms_trace) : bytes;
-  return cudaMemcpyFromSymbol(host, dms::g_dms_trace, n) == cudaSuccess ? 0 : -3;
-}
-extern "C" __attribute__((visibility("default"))) int dms_debug_trace_clear() {
-  static unsigned long long zeros[2 * dms::kTraceCtas * dms::kTraceSlots];
-  return cudaMemcpyToSymbol(dms::g_dms_trace, zeros, sizeof(zeros)) == cudaSuccess ? 0 : -3;
-}
-#endif

@@ -30,9 +30,6 @@
 
 namespace dms {
 
-#ifdef DMS_TRACE
-__device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
-#endif
 
 constexpr int kMaxCluster = 16;  // shared-memory staging bound
 constexpr int kPickCluster = 8;  // largest cluster launched: every cluster of the grid co-resident
@@ -99,7 +96,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   const int owner = cs - 1;  // the rank that appends: its slice of the slots is the shortest
   const int b = bh / c.Hkv, h = bh % c.Hkv;
   const long li = static_cast<long>(layer) * c.B * c.Hkv + bh;
-  DMS_TRACE_MARK(0, 0);
   // Programmatic dependent launch.  With `early` (the previous launch of this
   // library on the stream was for another layer or cache) this layer's state
   // is read and the first tiles are requested before waiting for the previous
@@ -210,7 +206,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
       break;
     }
     const SubMeta m = meta[stage];
-    if (n == 0) DMS_TRACE_MARK(0, 2);
     const unsigned char* kt = stage_buf + stage * S::STAGE;
     if (FP8) {
       widen_fp8_subtile<D>(kt, conv_buf);
@@ -227,7 +222,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     if (tid == 0 && produce(stage)) ++produced;
   }
 
-  DMS_TRACE_MARK(0, 3);
   // merge the warps (and, for the owner of a fused step, the new token) into
   // this CTA's partial, written into slot `rank` of the owner's inbox
   warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
@@ -286,15 +280,12 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     }
   }
   if (rank != owner) {
-    DMS_TRACE_MARK(0, 4);
-    DMS_TRACE_MARK(0, 6);
     return;  // nothing reads this CTA's shared memory
   }
   if (tid == 0) mbar_expect_tx(&inbox_bar, static_cast<uint32_t>((cs - 1) * g * (D + 2) * 4));
   bool landed = cs == 1 || mbar_wait_bounded(&inbox_bar, 0);
   landed = __syncthreads_and(landed);  // (one answer for the block); the owner's own partial is in place too
   if (!landed && tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
-  DMS_TRACE_MARK(0, 4);
 
   if (FUSED && warp == 3) {
     // Warp 3 appends this head's token at the planned slot (every CTA of the
@@ -341,7 +332,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     } else if (lane == 0) {
       set_status(c.ctrl, (flags & 4) ? DMS_ST_CAPACITY : DMS_ST_POOL_EXHAUSTED);
     }
-    DMS_TRACE_MARK(0, 8);
     int last = 0;
     if (lane == 0) {
       // plan of the next append (token t + 1), from the values just written
@@ -351,7 +341,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
       last = count_step(c, ok && (flags & 2) ? 1 : 0, static_cast<int>(gridDim.x) / cs, next_page0) ? 1 : 0;
     }
     if (__shfl_sync(0xffffffffu, last, 0)) advance_positions(c, layer, lane, 32);
-    DMS_TRACE_MARK(0, 6);
     return;
   }
 
@@ -410,9 +399,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
       }
     }
   }
-  DMS_TRACE_MARK(0, 7);
-  DMS_TRACE_MARK(0, 5);
-  DMS_TRACE_MARK(0, 6);
 }
 
 // Cluster size: the largest power of two <= 8 with cs * B * Hkv <= 2 * SMs
@@ -510,10 +496,3 @@ cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, 
 
 }  // namespace dms
 
-#ifdef DMS_TRACE
-// Copy the cluster kernel's phase timeline to the host (tracing builds only).
-extern "C" __attribute__((visibility("default"))) int dms_debug_trace_read_cluster(void* host, size_t bytes) {
-  const size_t n = sizeof(dms::g_dms_trace) < bytes ? sizeof(dms::g_dms_trace) : bytes;
-  return cudaMemcpyFromSymbol(host, dms::g_dms_trace, n) == cudaSuccess ? 0 : -3;
-}
-#endif

@@ -46,29 +46,6 @@
 
 namespace dms {
 
-#ifdef DMS_TRACE
-__device__ unsigned long long g_dms_trace[2 * kTraceCtas * kTraceSlots];
-// phase marks of the kernel of layer l (27 layers kept, 148 CTAs each), by
-// thread 0 or by any one thread (the producer's or the aux warp's lane 0)
-#define FLAT_TRACE_ROW (((layer) % 27) * 148 + blockIdx.x)
-#define FLAT_MARK_ANY(slot)                                                                            \
-  do {                                                                                                 \
-    unsigned long long t_;                                                                             \
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                             \
-    if (blockIdx.x < 148) g_dms_trace[static_cast<long>(FLAT_TRACE_ROW) * kTraceSlots + (slot)] = t_; \
-  } while (0)
-#define FLAT_MARK(slot)                   \
-  do {                                    \
-    if (threadIdx.x == 0) FLAT_MARK_ANY(slot); \
-  } while (0)
-#else
-#define FLAT_MARK_ANY(slot) \
-  do {                      \
-  } while (0)
-#define FLAT_MARK(slot) \
-  do {                  \
-  } while (0)
-#endif
 
 constexpr int kFlatConsumers = 4;                        // warps computing
 constexpr int kFlatProducer = kFlatConsumers;            // warp issuing the TMA loads
@@ -377,7 +354,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
   const int BH = c.B * c.Hkv;
   const long lbase = static_cast<long>(layer) * BH;
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-  FLAT_MARK(0);
   // Programmatic dependent launch.  With `early` (the previous launch of this
   // library on the stream was for another layer or cache) the partition below
   // reads only this layer's state before waiting for the previous kernel:
@@ -513,7 +489,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
       s_ctot[warp][1] = gcarry;
     }
   }
-  FLAT_MARK(16);
   __syncthreads();
   {
     int base = 0, gbase = 0, total = 0;
@@ -532,7 +507,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     if (tid == 0) s_off[BH] = total;
   }
   __syncthreads();
-  FLAT_MARK(17);
   const long U = s_off[BH];
   const long u0 = static_cast<long>(cta) * U / G, u1 = static_cast<long>(cta + 1) * U / G;
   auto cta_of = [&](long u) {
@@ -662,7 +636,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     }
   }
   __syncthreads();
-  FLAT_MARK(18);
   nseg = s_nseg;
   const int nsub = s_nsub;
   const bool table = nsub <= kFlatSubMax;
@@ -715,7 +688,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     }
   }
   __syncthreads();
-  FLAT_MARK(1);
   // Early: the producer starts the first ring of K/V loads (this layer's
   // pages) before waiting; the aux warp waits before reading the inputs and
   // the shared counters; the consumers see only what those two publish.
@@ -796,7 +768,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
           *reinterpret_cast<uint2*>(o + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g + r) * D + 4 * d4) =
               pk;
         }
-        if (tix == 0) FLAT_MARK_ANY(13);
         if (FUSED) {
           // append of the token at the planned slot: every CTA reading this
           // head has arrived, so its pages are no longer read in this launch
@@ -844,7 +815,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
             const int tn = t + 1;
             const int rn = sg.ring_idx >= 0 ? s_ring[sg.ring_idx] : 0;
             *plan_at(c, li, tn) = make_plan(rn, tn, cnt_new, np_new, c);
-            FLAT_MARK_ANY(15);
           }
         }
       };
@@ -906,7 +876,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
       __threadfence();  // the logits written here are visible before any hand-over
     }
     __syncwarp();
-    if (lane == 0) FLAT_MARK_ANY(2);
     // ---- hand-overs, in segment order: the consumers' merged state of
     // segment k arrives in cpart[k & 1].  A head held here alone is finished
     // here from it; a head shared with other CTAs leaves its partial and
@@ -937,7 +906,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
           if (last) c.head_done[bh] = 0;
         }
         finish = __shfl_sync(0xffffffffu, last, 0) != 0;
-        if (k == 0 && lane == 0) FLAT_MARK_ANY(finish ? 4 : 6);
       }
       if (finish && sg.nparts == 1) {
         finish_head(k, cp, lane, 32);  // held here alone: sources in shared memory
@@ -985,9 +953,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
             }
           }
         }
-        if (n == 0) FLAT_MARK_ANY(10);
-        if (n == 1) FLAT_MARK_ANY(14);
-        if (n == nst - 1) FLAT_MARK_ANY(11);
         return dst;
       };
       auto issue_q = [&](int n, int qoff) {
@@ -1012,7 +977,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
         griddep_wait();
         griddep_launch_dependents();
       }
-      FLAT_MARK_ANY(21);
       for (int n = 0; n < n_early; ++n) issue_q(n, segs[s_sub[n].y >> 8].qoff);
       if (table) {
         for (int n = n_early; n < nsub; ++n) {
@@ -1051,7 +1015,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
         flat_stage(j, mper, &st, &use);
         if (!mbar_wait_bounded(&full_bar[st], use & 1)) timed_out = true;
       }
-      FLAT_MARK_ANY(12);
       if (timed_out) set_status(c.ctrl, DMS_ST_TIMEOUT);
     }
     __syncwarp();
@@ -1076,7 +1039,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
         flat_stage(n, nst / kFlatConsumers, &st, &use);
         const bool ok = mbar_wait_bounded(&full_bar[st], use & 1);
         if (!ok) timed_out = true;
-        if (n == 0) FLAT_MARK(3);
         const FlatMeta m = meta[st];
         const unsigned char* stage = sbase + st * stride;
         if (!have_q) {
@@ -1108,7 +1070,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
 
       // ---- end of a segment: merge the four warps' states into cpart[k & 1]
       // (once the aux warp has released it) and hand it over -----------------
-      if (k == 0) FLAT_MARK(5);
       const int j = k & 1;
       warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
       if (k >= 2 && !mbar_wait_bounded(&hq_empty[j], ((k >> 1) - 1) & 1)) timed_out = true;
@@ -1118,7 +1079,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
       consumers_sync();
       if (tid == 0) mbar_arrive(&hq_full[j]);
     }
-    FLAT_MARK(8);
     // the heads whose last part arrived here, once every hand-over is done
     if (!mbar_wait_bounded(&aux_done, 0)) timed_out = true;
     for (int f = 0; f < s_nfin; ++f) finish_head(s_fin[f], nullptr, tid, 128);
@@ -1134,7 +1094,6 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     __syncthreads();
     if (s_last) advance_positions(c, layer, tid, kFlatThreads);
   }
-  FLAT_MARK(9);
 }
 
 // Launch geometry of the flat kernel, or false when the shape is outside what
@@ -1219,10 +1178,3 @@ cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, voi
 
 }  // namespace dms
 
-#ifdef DMS_TRACE
-// Copy the flat kernel's phase timeline to the host (tracing builds only).
-extern "C" __attribute__((visibility("default"))) int dms_debug_trace_read_flat(void* host, size_t bytes) {
-  const size_t n = sizeof(dms::g_dms_trace) < bytes ? sizeof(dms::g_dms_trace) : bytes;
-  return cudaMemcpyFromSymbol(host, dms::g_dms_trace, n) == cudaSuccess ? 0 : -3;
-}
-#endif
