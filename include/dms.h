@@ -33,6 +33,9 @@
  *    unspecified until dms_cache_reset.
  *  - All calls on one cache must be issued on one stream (or ordered by the
  *    caller); calls on different caches are independent.
+ *  - q, k, v and o (prefill and decode) are read and written as 16-byte
+ *    vectors: their base pointers must be 16-byte aligned (DMS_ERR_INVALID
+ *    otherwise).
  */
 #ifndef DMS_H
 #define DMS_H
@@ -341,6 +344,16 @@ DMS_API int dms_decode_attention(dms_cache* cache, int layer, const void* q, voi
  *    the same device without ordering) race on the array and give wrong
  *    results; order them. */
 DMS_API int dms_decode_attention_noalloc(dms_cache* cache, int layer, const void* q, void* o, void* stream);
+
+/* Self-check of the device failure path (the pages have no counterpart): one
+ * thread waits, with the same bounded wait every kernel of the library uses,
+ * on a shared-memory barrier that nothing ever completes, gives up after
+ * `tries` tries (1 <= tries <= 2^24, each try suspends the thread for a few
+ * microseconds at most) and sets DMS_ST_TIMEOUT in the cache's status word, as
+ * a kernel whose tile never arrives would.  Nothing is left in flight and the
+ * context stays usable; dms_cache_reset clears the bit.  For tests of a
+ * caller's error handling. */
+DMS_API int dms_selftest_wait_timeout(dms_cache* cache, int tries, void* stream);
 
 /* Tokens appended so far to `layer` (host-side counter, no device access). */
 DMS_API int dms_cache_positions(const dms_cache* cache, int layer);

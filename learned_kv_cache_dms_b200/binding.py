@@ -94,16 +94,18 @@ _lib.dms_decode_append.argtypes = [_P, C.c_int, C.POINTER(dms_decode_args), _P]
 _lib.dms_decode_attention.argtypes = [_P, C.c_int, _P, _P, _P]
 _lib.dms_decode_attention_noalloc.argtypes = [_P, C.c_int, _P, _P, _P]
 _lib.dms_cache_positions.argtypes = [_P, C.c_int]
+_lib.dms_selftest_wait_timeout.argtypes = [_P, C.c_int, _P]
 for _f in ("dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset", "dms_cache_get_layout",
            "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step", "dms_cache_positions",
            "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append", "dms_decode_attention",
-           "dms_decode_attention_noalloc", "dms_cache_export"):
+           "dms_decode_attention_noalloc", "dms_cache_export", "dms_selftest_wait_timeout"):
     getattr(_lib, _f).restype = C.c_int
 
 EXPORTED = ("dms_cache_desc_default", "dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset",
             "dms_cache_get_layout", "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step",
             "dms_cache_positions", "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append",
-            "dms_decode_attention", "dms_decode_attention_noalloc", "dms_cache_export")
+            "dms_decode_attention", "dms_decode_attention_noalloc", "dms_cache_export",
+            "dms_selftest_wait_timeout")
 
 
 def _check(code, where):
@@ -218,6 +220,10 @@ def dms_decode_attention_noalloc(handle: int, layer: int, q, o, stream=None) -> 
 
 def dms_cache_positions(handle: int, layer: int) -> int:
     return _check(_lib.dms_cache_positions(handle, layer), "dms_cache_positions")
+
+
+def dms_selftest_wait_timeout(handle: int, tries: int, stream=None) -> None:
+    _check(_lib.dms_selftest_wait_timeout(handle, tries, _stream(stream)), "dms_selftest_wait_timeout")
 
 
 # ---- convenience wrapper over torch tensors (still marshalling only) ---------

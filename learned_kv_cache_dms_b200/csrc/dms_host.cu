@@ -446,11 +446,16 @@ int dms_decide(dms_cache* c, int T, const dms_decide_params* d, void* neuron_src
   return r == cudaSuccess ? DMS_OK : DMS_ERR_CUDA;
 }
 
+// q, k, v and o rows are moved as 16-byte vectors (and by TMA): their base
+// pointers must be 16-byte aligned.
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 static int check_prefill(const dms_cache* c, int layer, const dms_prefill_args* a) {
   if (!c || !a || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
   const int T = a->seq_len;
   if (T <= 0 || T > c->desc.max_positions || T > kMaxPrefillTokens) return DMS_ERR_INVALID;
   if (!a->q || !a->k || !a->v || !a->o || !a->alpha) return DMS_ERR_INVALID;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o)) return DMS_ERR_INVALID;
   if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
   if (a->decide) return check_decide(c, a->decide);
   return DMS_OK;
@@ -529,6 +534,7 @@ int dms_prefill(dms_cache* c, int layer, const dms_prefill_args* a, void* stream
 int dms_decode_append(dms_cache* c, int layer, const dms_decode_args* a, void* stream) {
   if (!c || !a || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
   if (!a->q || !a->k || !a->v || !a->alpha) return DMS_ERR_INVALID;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v)) return DMS_ERR_INVALID;
   if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
   if (a->decide) {
     int e = check_decide(c, a->decide);
@@ -595,6 +601,7 @@ extern "C" {
 
 int dms_decode_attention(dms_cache* c, int layer, const void* q, void* o, void* stream) {
   if (!c || !q || !o || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(o)) return DMS_ERR_INVALID;
   if (c->worklist_layer != layer) return DMS_ERR_STATE;
   if (c->has_maps && c->desc.kv_dtype != DMS_F32)
     return run_decode_kernel(c, layer, q, o, false, nullptr, nullptr, nullptr, nullptr,
@@ -607,7 +614,7 @@ int dms_decode_attention(dms_cache* c, int layer, const void* q, void* o, void* 
 }
 
 int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* stream) {
-  if (!c || !a || !a->o) return DMS_ERR_INVALID;
+  if (!c || !a || !a->o || !aligned16(a->o)) return DMS_ERR_INVALID;
   if (c->desc.kv_dtype == DMS_F32) {
     int e = dms_decode_append(c, layer, a, stream);
     if (e) return e;
@@ -623,6 +630,7 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   }
   if (layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
   if (!a->q || !a->k || !a->v || !a->alpha) return DMS_ERR_INVALID;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v)) return DMS_ERR_INVALID;
   if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
   if (a->decide) {
     int e = check_decide(c, a->decide);
@@ -651,6 +659,33 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Self-check of the failure path of a bounded device wait: one thread waits,
+// with the library's bounded wait, on a shared-memory barrier that nothing
+// completes (no copy or arrival is ever issued for it), gives up after `tries`
+// tries and records DMS_ST_TIMEOUT in the cache's status word, exactly as a
+// kernel whose copy never lands does.  Nothing is in flight when it returns.
+// ---------------------------------------------------------------------------
+namespace {
+__global__ void k_wait_selftest(int* ctrl, long long tries) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, tries)) set_status(ctrl, DMS_ST_TIMEOUT);
+}
+}  // namespace
+
+extern "C" int dms_selftest_wait_timeout(dms_cache* c, int tries, void* stream) {
+  if (!c || tries <= 0 || tries > (1 << 24)) return DMS_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  track_launch(c, -1, s);
+  k_wait_selftest<<<1, 32, 0, s>>>(c->view.ctrl, tries);
+  return cudaGetLastError() == cudaSuccess ? DMS_OK : DMS_ERR_CUDA;
+}
 
 // ---------------------------------------------------------------------------
 // Decode attention with its split-K partials in a fixed device array owned by
@@ -691,6 +726,7 @@ int split_scratch_address(int device, void** out) {
 
 extern "C" int dms_decode_attention_noalloc(dms_cache* c, int layer, const void* q, void* o, void* stream) {
   if (!c || !q || !o || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(o)) return DMS_ERR_INVALID;
   if (c->worklist_layer != layer) return DMS_ERR_STATE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (c->desc.kv_dtype == DMS_F32) {

@@ -274,9 +274,10 @@ __device__ __forceinline__ bool mbar_wait_parked(uint64_t* bar, uint32_t parity)
   }
   return false;
 }
-// Bounded wait: returns false (and the caller must give up) after kSpinLimit tries.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  for (long long i = 0; i < kSpinLimit; ++i)
+// Bounded wait: returns false (and the caller must give up) after `tries`
+// tries (kSpinLimit unless a caller asks for fewer).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, long long tries = kSpinLimit) {
+  for (long long i = 0; i < tries; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }

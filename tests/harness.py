@@ -179,11 +179,16 @@ def make_desc(B_, case: Case):
     return d
 
 
-def run_gpu(case: Case, ins):
-    """Run prefill + decode steps through the C ABI; returns GPU results on the CPU."""
+def run_gpu(case: Case, ins, cache=None):
+    """Run prefill + decode steps through the C ABI; returns GPU results on the CPU.
+
+    With `cache` (an open binding.Cache of this case's descriptor) the run uses
+    it as it is and leaves it open; otherwise a fresh cache is made and closed."""
     from learned_kv_cache_dms_b200 import binding as B_
     dev = torch.device("cuda")
-    cache = B_.Cache(make_desc(B_, case), dev)
+    own = cache is None
+    if own:
+        cache = B_.Cache(make_desc(B_, case), dev)
     T, N, B = case.T, case.N, case.B
     q = ins["q"].to(dev)
     k = ins["k"].to(dev)
@@ -253,7 +258,8 @@ def run_gpu(case: Case, ins):
     res["pages_final"] = {k_: t.cpu().clone() for k_, t in cache.pages().items()}
     res["status"] = cache.status()
     res["positions"] = cache.positions(case.layer)
-    cache.close()
+    if own:
+        cache.close()
     return res
 
 
@@ -298,9 +304,9 @@ def compare_pages(case, so, po, pg):
                     assert np.array_equal(po["vval"][pid, :rows], pg["v"][pid, :rows].double().numpy()), ("v", b, h, p)
 
 
-def check_case(case: Case, ins=None):
+def check_case(case: Case, ins=None, cache=None):
     ins = ins if ins is not None else build(case)
-    res = run_gpu(case, ins)
+    res = run_gpu(case, ins, cache)
     tol = TOL[case.act]
     T = case.T
     # decisions

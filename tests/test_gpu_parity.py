@@ -65,6 +65,12 @@ CASES = {
     # fp32 pages of 256 slots: eight 32-row scatter groups per page, the last page ragged
     "f32_p256_scatter": Case(B=1, T=700, steps=10, Hq=4, Hkv=2, D=128, w=320, P=256, act="f32", kv="f32",
                              source="input", keep=0.3, attn_rows=64, seed=33),
+    # GQA groups that are not a power of two: the prefill attention takes the
+    # mma.sync kernel (the tcgen05 kernel tiles 128 / g positions x g heads)
+    "bf16_g3_mma_prefill": Case(B=2, T=450, steps=12, Hq=12, Hkv=4, D=128, w=64, P=32, act="bf16", kv="bf16",
+                                source="input", keep=0.3, seed=51),
+    "bf16_g6_d64_proj_mma_prefill": Case(B=1, T=380, steps=10, Hq=12, Hkv=2, D=64, hidden=256, w=48, P=16,
+                                         act="bf16", kv="bf16", source="proj", keep=0.25, seed=52),
     # second layer of a two-layer cache with preallocation
     "layer1_of_2": Case(B=2, T=260, steps=12, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16",
                         source="input", keep=0.3, layers=2, layer=1, prealloc=64, seed=15),
