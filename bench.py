@@ -16,11 +16,21 @@ outside the window; synthetic seeded bf16 inputs resident in HBM.  --workload
 selects the batch-8 Qwen3-8B layer, the FP8 Llama-3.2-1B layer (32K context,
 key-neuron decisions, rotary tables) or the 36-layer batch-32 stack.
 
-L2: a single layer's decode working set (6-60 MB) fits in the 126 MB L2, so a
-512 MB buffer is written before every decode step (outside the timed
-segments) and the KV bytes come from DRAM; the 36-layer stack reads gigabytes
-per step and runs its steps back to back.  Times are CUDA events on the
-launching stream.
+L2: a single layer's decode working set (6-60 MB) fits in the 126 MB L2, so
+each decode step runs R independent replicas of the cache back to back (R
+chosen so that together they hold >= 4x L2): no replica's KV is still in L2
+when it is read again, and no flush kernel sits between decode kernels.  The
+36-layer stack reads gigabytes per step and runs its steps back to back.
+Times are CUDA events on the launching stream.
+
+The JSON line also carries: `e2e` (the whole request -- prompt copies,
+prefill, every decode step with its host copies -- through the public API with
+host buffers), `decode_step_us_single` (one replica's step, L2 flushed before
+it), the prefill attention's fraction on executed tiles, the decision and
+compaction kernels on their own, `cpu_baseline` (the oracle on the host cores:
+decode on all cores and on one core, and a prefill sample), and `secondary`
+records for the other workloads (batch 8, the FP8 Llama-3.2-1B layer, the
+first 512 steps of the 36-layer stack).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME] [--decode-steps N]
@@ -57,6 +67,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiler runs)")
+    p.add_argument("--no-secondary", action="store_true",
+                   help="measure only --workload (the default run also measures the other workloads)")
     p.add_argument("--workload", choices=BENCH_WORKLOADS, default="qwen8b",
                    help="qwen8b (default): one Qwen3-8B layer, batch 1; qwen8b_c8: batch 8; llama1b(_layer): "
                         "FP8 pages, key-neuron decisions, 32K context; reason36: 36 layers, batch 32")
@@ -465,6 +477,31 @@ def visible_pairs(alpha, wl):
     return int((band[None, None, :] + cum[:, :, upto]).sum())
 
 
+def executed_tile_flops(alpha, wl):
+    """Tensor-core flops the tcgen05 prefill attention executes (whole 128 x 64
+    tiles, masked elements included), from the prefill decisions: a work item
+    is 2 Q tiles of 128 rows (128/g positions x the g query heads of one KV
+    head); it runs ceil(nk / 64) kept-prefix tiles (nk = kept tokens before
+    position i1 - w) and the band tiles of keys [max(0, i0 - w + 1), i1 - 1],
+    each tile 4 * 128 * 64 * D flops (Q K^T and P V) per Q tile."""
+    ev = (alpha > 0).cpu().numpy()  # [B,H,T]
+    B, H, T = ev.shape
+    w, D, g = wl.window, wl.head_dim, wl.gqa
+    NP = 128 // g
+    span = 2 * NP
+    kept = ~ev
+    kept[:, :, max(0, T - w):] = False
+    cum = np.concatenate([np.zeros((B, H, 1), np.int64), np.cumsum(kept, -1)], -1)  # kept before x
+    i0 = np.arange(0, T, span)
+    i1 = np.minimum(T, i0 + span)
+    nk = cum[:, :, np.clip(i1 - w, 0, T)] * (i1 - w > 0)
+    nkt = (nk + 63) // 64
+    jlo = np.maximum(0, i0 - w + 1)
+    band = (i1 - 1 - jlo + 64) // 64
+    tiles = int((nkt + band[None, None, :]).sum())
+    return tiles * 2 * 4 * 128 * 64 * D
+
+
 def decode_step_bytes(wl, retained):
     """Algorithmic HBM bytes of one decode step over the stack, given the
     retained slots summed over (layer, b, h) before the append: the retained
@@ -512,7 +549,54 @@ def measure_prefill_parts(B_, r, wl, passes=3):
     return (med(dec) if proj else None), med(comp)
 
 
-def run_ours(args, world, rank, local):
+def measure_single_step(B_, r, steps=32):
+    """One replica's decode step on its own: a CUDA graph per step holding
+    only that replica's launch(es) between two events, replayed after a 512 MB
+    write that evicts its KV from L2.  Returns the median step time in us."""
+    wl = r.wl
+    units = [u for u in r.units if u["r"] == 0]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    n = min(steps, r.S)
+    r.reset_all()
+    r.restore_prompt()
+    for u in units:
+        B_.dms_prefill(u["h"], u["l"], u["pargs"])
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    graphs = []
+    for i in range(n):
+        r.restore_token(i % r.pool)
+        torch.cuda.synchronize()
+        ga = torch.cuda.CUDAGraph()
+        ev = (torch.cuda.Event(enable_timing=True, external=True),
+              torch.cuda.Event(enable_timing=True, external=True))
+        with torch.cuda.graph(ga, stream=side):
+            ev[0].record()
+            for u in units:
+                B_.dms_decode_step(u["h"], u["l"], u["dargs"][i % r.pool])
+            ev[1].record()
+        graphs.append((ga, ev))
+    torch.cuda.synchronize()
+    # replays from a fresh prefill: the captures above advanced the caches
+    r.reset_all()
+    r.restore_prompt()
+    for u in units:
+        B_.dms_prefill(u["h"], u["l"], u["pargs"])
+    times = []
+    for i, (ga, ev) in enumerate(graphs):
+        r.restore_token(i % r.pool)
+        flush.fill_(i & 0xFF)
+        ga.replay()
+        torch.cuda.synchronize()
+        times.append(ev[0].elapsed_time(ev[1]) * 1e3 / wl.layers)
+    del graphs
+    return float(np.median(times))
+
+
+def run_ours(args, world, rank, local, primary=True):
+    """Measure one workload.  The primary record (the JSON line) carries every
+    leg; a secondary record (another workload in the same run) carries the
+    device-timed decode and prefill figures and the single-replica latency."""
     from learned_kv_cache_dms_b200 import binding as B_
     wl = I.WORKLOADS[args.workload]
     pk, pk_kind = peaks()
@@ -525,6 +609,7 @@ def run_ours(args, world, rank, local):
     counts = [int(c.item()) for c in torch.stack(counts).cpu()]
     assert r.cache.status() == 0, "cache status %d" % r.cache.status()
     pairs = sum(visible_pairs(u["alpha"], wl) for u in r.units if u["r"] == 0)
+    tile_flops = sum(executed_tile_flops(u["alpha"], wl) for u in r.units if u["r"] == 0)
     o_eager = r.od.clone()
     r.capture()
     for _ in range(max(1, args.warmup - 1)):
@@ -571,6 +656,7 @@ def run_ours(args, world, rank, local):
     decode_gbs = K * R * attn_bytes / (decode_ms / 1e3) / 1e9
     prefill_flops = 4.0 * wl.head_dim * wl.gqa * pairs  # one replica, every layer
     prefill_tflops = K * R * prefill_flops / (prefill_attn_ms / 1e3) / 1e12
+    exec_tflops = K * R * tile_flops / (prefill_attn_ms / 1e3) / 1e12
     clocks = clk.summary()
 
     # decision logits (A1) and compaction (A2) on their own, L2-cold
@@ -597,9 +683,10 @@ def run_ours(args, world, rank, local):
         "kernel": ("k_neuron_rope8 + " if neuron_pass else "") + "k_prefill_scan + k_prefill_scatter "
                   "(dms_prefill_compact minus dms_decide), L2-cold"}
 
-    e2e = None if args.no_e2e else run_e2e(B_, r, args, world)
+    single_us = measure_single_step(B_, r)
+    e2e = None if (args.no_e2e or not primary) else run_e2e(B_, r, args, world)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if primary and rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, args.cpu_seconds)
     kern = decode_kernel_name(wl, args.decode_kernel, torch.cuda.get_device_properties(0).multi_processor_count)
     kname = ("decode step: %s<%d,%s> (split-K attention, %s%s)%s"
@@ -642,7 +729,12 @@ def run_ours(args, world, rank, local):
         "prefill_attention": {"bound": "tensor", "achieved": round(prefill_tflops, 2),
                               "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                               "frac": round(prefill_tflops / pk["bf16_tflops"], 4),
-                              "flops_per_launch": prefill_flops / L, "visible_pairs": pairs},
+                              "flops_per_launch": prefill_flops / L, "visible_pairs": pairs,
+                              "executed_tile_tflops": round(exec_tflops, 2),
+                              "frac_executed_tiles": round(exec_tflops / pk["bf16_tflops"], 4),
+                              "executed_over_algorithmic": round(tile_flops / prefill_flops, 4),
+                              "kernel": "k_attn_prefill_tc<%d> (tcgen05/TMEM)" % wl.head_dim},
+        "decode_step_us_single": round(single_us, 3),
         "decide": decide_roof,
         "compaction": compact_roof,
         "achieved_cr": round(wl.max_positions / retained_last, 3) if S == wl.decode_steps else None,
@@ -659,70 +751,92 @@ def _op(name):
 
 
 def run_e2e(B_, r, args, world):
-    """Same workload through the public API with host (pinned) buffers on one
-    replica: the prompt and every decode token are copied host->device and
-    every output device->host inside the timed segments, and L2 is flushed
-    (a 512 MB buffer written) before every step.  A multi-layer stack is
-    sampled over its first E2E_STEPS_STACK decode steps."""
+    """The whole request through the public API with host (pinned) buffers,
+    for the R replicas the device-timed measurement uses (R independent
+    requests served together; their caches together hold >= 4x L2).  Inside
+    the timed region, per request: each replica's prompt (q, k, v, hidden)
+    copied host->device and dms_prefill of every layer, the last prompt
+    position's outputs copied back; then per decode step one host->device copy
+    of every replica's token inputs, one dms_decode_step per (replica, layer),
+    one device->host copy of the step's outputs.  Eager calls, no graphs.  A
+    multi-layer stack is sampled over its first E2E_STEPS_STACK decode steps."""
     wl = r.wl
     S = r.S if r.L == 1 else min(r.S, E2E_STEPS_STACK)
+    R, L = r.R, r.L
     names_p = ("q", "k", "v") + (() if r.neuron else ("h",))
     names_d = ("qd", "kd", "vd") + (() if r.neuron else ("hd",))
-    units = [u for u in r.units if u["r"] == 0]
-    host = [{k: x[k].cpu().pin_memory() for k in names_p + names_d} for x in r.lay]
-    dev = [{k: torch.empty_like(x[k]) for k in names_p + names_d} for x in r.lay]
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
-    o_host = torch.empty(tuple(r.o.shape), dtype=r.o.dtype).pin_memory()
-    od_host = torch.empty(tuple(r.od.shape), dtype=r.od.dtype).pin_memory()
-    pargs, dargs, keep = [], [], []
-    for x, d, u in zip(r.lay, dev, units):
-        if r.neuron:
-            pd = B_.decide_params(x["off"])
-            dd = [pd] * r.pool
-        else:
-            pd = B_.decide_params(x["off"], hidden=d["h"], norm_weight=x["gamma"], proj_weight=x["W"])
-            dd = [B_.decide_params(x["off"], hidden=d["hd"][i], norm_weight=x["gamma"], proj_weight=x["W"])
-                  for i in range(r.pool)]
-        keep.append((pd, dd))
-        pargs.append(B_.Cache.prefill_args(d["q"], d["k"], d["v"], r.o, u["alpha"], pd, r.rope))
-        dargs.append([B_.Cache.decode_args(d["qd"][i], d["kd"][i], d["vd"][i], r.od[i], u["ad"][i], dd[i], r.rope)
-                      for i in range(r.pool)])
+    host_p = [{k: x[k].cpu().pin_memory() for k in names_p} for x in r.lay]
+    dev_p = [{k: torch.empty_like(x[k]) for k in names_p} for x in r.lay]
+    # token inputs: per step, every (replica, layer)'s rows packed in one buffer
+    row_elems = [sum(r.lay[l][k][0].numel() for k in names_d) for l in range(L)]
+    unit_off = np.cumsum([0] + [row_elems[l] for _ in range(R) for l in range(L)])
+    tok_n = int(unit_off[-1])
+    one = torch.cat([torch.cat([r.lay[l][k].reshape(r.pool, -1) for k in names_d], 1) for l in range(L)], 1).cpu()
+    packed = one.repeat(1, R)  # every replica serves the same token inputs
+    assert packed.shape[1] == tok_n
+    host_t = torch.empty(S, tok_n, dtype=torch.bfloat16).pin_memory()
+    for i in range(S):
+        host_t[i].copy_(packed[i % r.pool])
+    dev_t = torch.empty(tok_n, dtype=torch.bfloat16, device="cuda")
+    od_dev = torch.empty(R, L, *r.od.shape[1:], dtype=r.od.dtype, device="cuda")
+    od_host = torch.empty(S, *od_dev.shape, dtype=od_dev.dtype).pin_memory()
+    olast_host = torch.empty(R, L, wl.batch, wl.q_heads, wl.head_dim, dtype=r.o.dtype).pin_memory()
+    keep, pargs, dargs, alphas = [], [], [], []
+    for rr in range(R):
+        for l in range(L):
+            x, d = r.lay[l], dev_p[l]
+            u = r.units[rr * L + l]
+            base = int(unit_off[rr * L + l])
+            views, o = {}, base
+            for k in names_d:
+                n = x[k][0].numel()
+                views[k] = dev_t[o:o + n].view(x[k][0].shape)
+                o += n
+            if r.neuron:
+                pd = B_.decide_params(x["off"])
+                dd = pd
+            else:
+                pd = B_.decide_params(x["off"], hidden=d["h"], norm_weight=x["gamma"], proj_weight=x["W"])
+                dd = B_.decide_params(x["off"], hidden=views["hd"], norm_weight=x["gamma"], proj_weight=x["W"])
+            a_tok = torch.empty(wl.batch, wl.kv_heads, dtype=torch.float32, device="cuda")
+            keep.append((pd, dd, views, a_tok))
+            pargs.append(B_.Cache.prefill_args(d["q"], d["k"], d["v"], r.o, u["alpha"], pd, r.rope))
+            dargs.append(B_.Cache.decode_args(views["qd"], views["kd"], views["vd"], od_dev[rr, l], a_tok, dd,
+                                              r.rope))
     E = torch.cuda.Event
-    dec_ms = 0.0
-    h = r.cache.handle
+    total_ms = 0.0
     for it in range(args.steps + 1):
-        r.cache.reset()
-        flush.fill_(3)
-        for l in range(r.L):
-            for k in names_p:
-                dev[l][k].copy_(host[l][k], non_blocking=True)
-            B_.dms_prefill(h, l, pargs[l])
-        o_host.copy_(r.o, non_blocking=True)
-        evs = []
-        for s in range(S):
-            i = s % r.pool
-            if not r.cycled:
-                flush.fill_(s & 0xFF)
-            a, c = E(enable_timing=True), E(enable_timing=True)
-            a.record()
-            for l in range(r.L):
-                for k in names_d:
-                    dev[l][k][i].copy_(host[l][k][i], non_blocking=True)
-                B_.dms_decode_step(h, l, dargs[l][i])
-            od_host[i].copy_(r.od[i], non_blocking=True)
-            c.record()
-            evs.append((a, c))
+        r.reset_all()
+        torch.cuda.synchronize()
+        a, c = E(enable_timing=True), E(enable_timing=True)
+        a.record()
+        for rr in range(R):
+            h = r.caches[rr].handle
+            for l in range(L):
+                for k in names_p:
+                    dev_p[l][k].copy_(host_p[l][k], non_blocking=True)
+                B_.dms_prefill(h, l, pargs[rr * L + l])
+                olast_host[rr, l].copy_(r.o[:, wl.prompt - 1], non_blocking=True)
+        for i in range(S):
+            dev_t.copy_(host_t[i], non_blocking=True)
+            for rr in range(R):
+                h = r.caches[rr].handle
+                for l in range(L):
+                    B_.dms_decode_step(h, l, dargs[rr * L + l])
+            od_host[i].copy_(od_dev, non_blocking=True)
+        c.record()
         torch.cuda.synchronize()
         if it == 0:
-            continue  # warm-up
-        dec_ms += sum(a.elapsed_time(c) for a, c in evs)
-    h2d = sum(host[l][k].numel() * 2 for l in range(r.L) for k in names_p)
-    h2d += S * sum(host[l][k][0].numel() * 2 for l in range(r.L) for k in names_d)
-    d2h = o_host.numel() * 2 + S * od_host[0].numel() * 2
-    dec_ms_max = allreduce(dec_ms, _op("max"), world)
-    val = args.steps * S * wl.batch * world / (dec_ms_max / 1e3)
+            continue  # warm-up request
+        total_ms += a.elapsed_time(c)
+    h2d = R * sum(host_p[l][k].numel() * 2 for l in range(L) for k in names_p) + S * tok_n * 2
+    d2h = olast_host.numel() * 2 + S * od_dev.numel() * 2
+    total_max = allreduce(total_ms, _op("max"), world)
+    val = args.steps * R * S * wl.batch * world / (total_max / 1e3)
     out = {"value": round(val, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-           "l2": "512 MB buffer written before every decode step (untimed), one replica"}
+           "request_ms": round(total_ms / args.steps, 3),
+           "timed": "whole request: %d replica prompts copied in and prefilled, %d decode steps with their "
+                    "token copies in and outputs out; generated tokens / request time" % (R, S)}
     if S < r.S:
         out["sample"] = "first %d decode steps" % S
     return out
@@ -771,14 +885,63 @@ def oracle_decode_sample(wl, seconds, n_steps_max=None):
     return n * B / (dt * wl.layers), cores, n, dt, passes
 
 
+def oracle_prefill_sample(wl, seconds):
+    """Time the oracle's prefill of one layer on the host cores: the sequential
+    replay of the append rule over the whole prompt (slots, pages, stored
+    values) and the fp64 masked attention of a sample of prompt rows (b, hq, i)
+    drawn uniformly, extrapolated to all B * T * Hq rows.  Returns (prompt
+    tok/s over the layer stack, replay s, rows timed, attention s, cores)."""
+    from oracle import oracle as O
+    cores = O.set_threads(os.cpu_count() or 1)
+    B, T, s = wl.batch, wl.prompt, wl.seed
+    q = I.normal(s, (0, 1), (B, T, wl.q_heads, wl.head_dim), "bf16").double().numpy()
+    k = I.normal(s, (0, 2), (B, T, wl.kv_heads, wl.head_dim), "bf16")
+    v = I.normal(s, (0, 3), (B, T, wl.kv_heads, wl.head_dim), "bf16")
+    alpha = I.synthetic_alpha(s, (0, 5), B, wl.kv_heads, T, I.keep_fractions(wl)).numpy()
+    ev = np.ascontiguousarray((alpha > 0).astype(np.uint8))
+    maxp = -(-wl.max_positions // wl.block)
+    c = O.Cache(1, B, wl.kv_heads, wl.head_dim, wl.window, wl.block, wl.max_positions,
+                B * wl.kv_heads * maxp, wl.prealloc_tokens, fp8=wl.kv_dtype == "fp8")
+    k32, v32 = k.float().numpy(), v.float().numpy()
+    t0 = time.perf_counter()
+    c.prefill(0, ev, k32, v32)
+    replay_s = time.perf_counter() - t0
+    k64, v64 = k.double().numpy(), v.double().numpy()
+    rng = np.random.default_rng(s)
+    n, attn_s = 0, 0.0
+    batch = 64 * cores
+    while attn_s < seconds:
+        rows = np.stack([rng.integers(0, B, batch), rng.integers(0, wl.q_heads, batch),
+                         rng.integers(0, T, batch)], 1)
+        t0 = time.perf_counter()
+        O.prefill_attention(q, k64, v64, ev, wl.window, rows=rows)
+        attn_s += time.perf_counter() - t0
+        n += batch
+    total = replay_s + attn_s * (B * T * wl.q_heads) / n
+    return B * T / (total * wl.layers), replay_s, n, attn_s, cores
+
+
 def cpu_baseline(wl, seconds):
-    tps, cores, n, dt, passes = oracle_decode_sample(wl, seconds)
-    return {"value": round(tps, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    """The oracle as it stands, on the host cores: decode steps on all cores
+    (the reported value) and on one core, and a prefill sample on all cores."""
+    from oracle import oracle as O
+    tps, cores, n, dt, passes = oracle_decode_sample(wl, 0.5 * seconds)
+    O.set_threads(1)
+    tps1, _, n1, dt1, _ = oracle_decode_sample(wl, 0.2 * seconds)
+    O.set_threads(os.cpu_count() or 1)
+    ptps, replay_s, prow, pattn_s, pcores = oracle_prefill_sample(wl, 0.3 * seconds)
+    return {"value": round(tps, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle", "nproc": os.cpu_count(),
             "sample": "%d decode steps of one layer (append + fp64 decode attention over the retained slots) in %d "
                       "pass(es) over the workload's %d steps, each from the cache after an untimed prefill replay of "
-                      "the %d-token prompt, %.1f s timed%s"
-                      % (n, passes, wl.decode_steps, wl.prompt, dt,
-                         "; scaled to the %d-layer stack" % wl.layers if wl.layers > 1 else "")}
+                      "the %d-token prompt, %.1f s timed on %d cores%s"
+                      % (n, passes, wl.decode_steps, wl.prompt, dt, cores,
+                         "; scaled to the %d-layer stack" % wl.layers if wl.layers > 1 else ""),
+            "decode_one_core": {"value": round(tps1, 2), "unit": "tokens/s", "cores": 1,
+                                "sample": "%d decode steps, %.1f s" % (n1, dt1)},
+            "prefill": {"value": round(ptps, 2), "unit": "prompt tokens/s", "cores": pcores,
+                        "sample": "append-rule replay of the %d-token prompt (%.2f s, measured) + fp64 masked "
+                                  "attention of %d sampled prompt rows (%.1f s), extrapolated to all %d rows"
+                                  % (wl.prompt, replay_s, prow, pattn_s, wl.batch * wl.prompt * wl.q_heads)}}
 
 
 def run_reference(args, world, rank):
@@ -805,6 +968,13 @@ def run_reference(args, world, rank):
             "e2e": {"value": round(val, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+SECONDARY = (("qwen8b_c8", None), ("llama1b", None), ("llama1b_layer", None), ("reason36", 512))
+SECONDARY_KEYS = ("value", "unit", "steps", "warmup", "ms_per_step", "config", "roofline", "retained_kv_gbps",
+                  "retained_per_head", "decode_ms_per_token_step", "decode_step_us_single", "prefill_tok_s",
+                  "prefill_ms", "prefill_compact_ms", "prefill_attention_ms", "prefill_attention", "decide",
+                  "compaction", "gpu_launches", "clocks")
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -816,6 +986,18 @@ def main():
         return
     world, rank, local = dist_setup()
     line = run_ours(args, world, rank, local)
+    if world == 1 and args.workload == "qwen8b" and not args.no_secondary:
+        # the other workloads, measured in the same run (device-timed legs);
+        # the 36-layer stack over its first 512 decode steps
+        torch.cuda.empty_cache()
+        line["secondary"] = {}
+        for name, n_dec in SECONDARY:
+            sub = argparse.Namespace(**vars(args))
+            sub.workload, sub.decode_steps, sub.replicas = name, n_dec, None
+            sub.steps = min(args.steps, 3)
+            rec = run_ours(sub, world, rank, local, primary=False)
+            line["secondary"][name] = {k: rec[k] for k in SECONDARY_KEYS if k in rec}
+            torch.cuda.empty_cache()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

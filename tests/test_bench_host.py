@@ -35,3 +35,25 @@ def test_recorded_traffic_only_for_current_sources(monkeypatch):
     assert bench.recorded_traffic(kernel, "no_such_workload") is None
     assert bench.recorded_traffic("k_not_recorded", workload) is None
 
+
+
+def test_executed_tiles_cover_the_visible_pairs():
+    """The tile count of the tcgen05 prefill schedule covers every visible
+    (query, key) pair, and with every key kept inside one band it is the
+    causal band's tile count."""
+    import numpy as np
+    import torch
+    wl = bench.I.WORKLOADS["qwen8b"]
+    rng = np.random.default_rng(0)
+    alpha = torch.from_numpy(np.where(rng.random((1, 8, wl.prompt)) < 0.125, -1.0, 1.0).astype(np.float32))
+    flops = bench.executed_tile_flops(alpha, wl)
+    algo = 4.0 * wl.head_dim * wl.gqa * bench.visible_pairs(alpha, wl)
+    assert algo <= flops <= 4 * algo
+    # all evicted: only the band; items of 2 * 128 / g positions see keys [i0 - w + 1, i1 - 1]
+    allev = torch.ones_like(alpha)
+    span = 2 * 128 // wl.gqa
+    tiles = 0
+    for i0 in range(0, wl.prompt, span):
+        i1 = min(wl.prompt, i0 + span)
+        tiles += (i1 - 1 - max(0, i0 - wl.window + 1) + 64) // 64
+    assert bench.executed_tile_flops(allev, wl) == 8 * tiles * 2 * 4 * 128 * 64 * wl.head_dim
