@@ -171,24 +171,53 @@ void store_row(Cache& c, int id, int row, int rows_in_page, const float* krow, c
   }
 }
 
-void fp8_encode_prefill_page(Cache& c, int id, int rows) {
+// FP8 encoding of page p of head i once a prefill call has staged its rows.
+// Rows holding positions >= pos0 were written by this call ("new"); the others
+// were written by an earlier call and hold codes at the page's scale ("old").
+// For K and for V separately: the scale becomes the larger of the old scale
+// (when the page holds old rows) and max amax(new row) / 448; when it grows the
+// old rows are first re-encoded from their decoded values, exactly as a decode
+// append re-encodes a page; then the new rows are encoded.  In a first prefill
+// every row is new and the scale is max amax(row) / 448 over the page.
+void fp8_encode_prefill_page(Cache& c, size_t i, int p, int pos0) {
+  const int id = c.page_table[i * c.maxp + p];
+  const int rows = std::min(c.P, c.count[i] - p * c.P);
+  const int* sp = &c.slot_pos[i * c.cap + static_cast<size_t>(p) * c.P];
+  bool any_new = false, any_old = false;
+  for (int r = 0; r < rows; ++r) (sp[r] >= pos0 ? any_new : any_old) = true;
+  if (!any_new) return;
   for (int which = 0; which < 2; ++which) {
     const std::vector<float>& raw = which ? c.vraw : c.kraw;
     std::vector<uint8_t>& code = which ? c.vcode : c.kcode;
     std::vector<double>& val = which ? c.vval : c.kval;
+    float& scale = (which ? c.vscale : c.kscale)[id];
     float amax = 0.0f;
     for (int r = 0; r < rows; ++r)
-      for (int d = 0; d < c.D; ++d)
-        amax = std::max(amax, std::fabs(raw[(static_cast<size_t>(id) * c.P + r) * c.D + d]));
-    float scale = amax / 448.0f;
-    (which ? c.vscale : c.kscale)[id] = scale;
-    for (int r = 0; r < rows; ++r)
-      for (int d = 0; d < c.D; ++d) {
-        size_t o = (static_cast<size_t>(id) * c.P + r) * c.D + d;
-        uint8_t q = scale > 0.0f ? e4m3_encode(raw[o] / scale) : 0;
-        code[o] = q;
-        val[o] = static_cast<double>(static_cast<float>(e4m3_decode(q)) * scale);
+      if (sp[r] >= pos0)
+        for (int d = 0; d < c.D; ++d)
+          amax = std::max(amax, std::fabs(raw[(static_cast<size_t>(id) * c.P + r) * c.D + d]));
+    const float s_old = any_old ? scale : 0.0f;
+    const float s = std::max(s_old, amax / 448.0f);
+    if (any_old && s > s_old)
+      for (int r = 0; r < rows; ++r) {
+        if (sp[r] >= pos0) continue;
+        for (int d = 0; d < c.D; ++d) {
+          const size_t o = (static_cast<size_t>(id) * c.P + r) * c.D + d;
+          const float dec = static_cast<float>(e4m3_decode(code[o])) * s_old;  // fp32 multiply
+          code[o] = e4m3_encode(dec / s);                                       // fp32 divide
+          val[o] = static_cast<double>(static_cast<float>(e4m3_decode(code[o])) * s);
+        }
       }
+    scale = s;
+    for (int r = 0; r < rows; ++r) {
+      if (sp[r] < pos0) continue;
+      for (int d = 0; d < c.D; ++d) {
+        const size_t o = (static_cast<size_t>(id) * c.P + r) * c.D + d;
+        const uint8_t q = s > 0.0f ? e4m3_encode(raw[o] / s) : 0;
+        code[o] = q;
+        val[o] = static_cast<double>(static_cast<float>(e4m3_decode(q)) * s);
+      }
+    }
   }
 }
 
@@ -474,13 +503,16 @@ void* oracle_cache_clone(void* h) { return new Cache(*static_cast<const Cache*>(
 int oracle_cache_status(void* h) { return static_cast<Cache*>(h)->status; }
 
 // Prefill of layer l: replay the append rule token by token, for each (b, h) in
-// row-major order.  evict [B,Hkv,T] (0/1); k/v [B,T,Hkv,D] fp32 values or null
-// (index-only replay).  FP8 pages are encoded from the survivors at the end.
+// row-major order, continuing from the tokens the layer already holds (a
+// later chunk of a chunked prefill).  evict [B,Hkv,T] (0/1); k/v [B,T,Hkv,D] fp32 values or null
+// (index-only replay).  FP8 pages the call wrote rows into are encoded at the
+// end (fp8_encode_prefill_page).
 void oracle_cache_prefill(void* hc, int l, int T, const uint8_t* evict, const float* k,
                           const float* v) {
   Cache& c = *static_cast<Cache*>(hc);
   for (int b = 0; b < c.B; ++b)
     for (int h = 0; h < c.Hkv; ++h) {
+      const int pos0 = c.npos[c.bh(l, b, h)];  // tokens held before this call
       for (int t = 0; t < T; ++t) {
         const float* kr = k ? k + ((static_cast<size_t>(b) * T + t) * c.Hkv + h) * c.D : nullptr;
         const float* vr = v ? v + ((static_cast<size_t>(b) * T + t) * c.Hkv + h) * c.D : nullptr;
@@ -488,8 +520,7 @@ void oracle_cache_prefill(void* hc, int l, int T, const uint8_t* evict, const fl
       }
       if (c.fp8 && c.store_values && k) {
         const size_t i = c.bh(l, b, h);
-        for (int p = 0; p * c.P < c.count[i]; ++p)
-          fp8_encode_prefill_page(c, c.page_table[i * c.maxp + p], std::min(c.P, c.count[i] - p * c.P));
+        for (int p = 0; p * c.P < c.count[i]; ++p) fp8_encode_prefill_page(c, i, p, pos0);
       }
     }
 }
@@ -558,6 +589,64 @@ void oracle_cache_decode_attention(void* hc, int l, int Hq, const double* q, dou
       softmax_attend(q + (static_cast<size_t>(b) * Hq + hq) * c.D, c.D, keys, vals,
                      o + (static_cast<size_t>(b) * Hq + hq) * c.D);
     }
+}
+
+
+// Attention of the T rows of a prefill call into layer l, computed with the
+// cache as it is before the call's appends ([DMS-Qwen3], chunked prefill: a
+// chunk's queries attend to the cache plus the chunk itself).  Row i of the
+// call sits at position pos0 + i (pos0 = tokens the layer already holds) and
+// sees, under the DMS mask (key j visible iff j <= i and (i - j < w or j was
+// kept)):
+//   * every key the cache holds: a slot at position j older than the last w
+//     positions is a kept token (a marked one would have been overwritten), a
+//     younger one is kept or marked as its ring entry says; values as stored
+//     (decoded for FP8 pages);
+//   * the call's own keys j <= i, from its inputs.
+// q [B,T,Hq,D], k/v [B,T,Hkv,D], evict [B,Hkv,T]; rows: optional (b, hq, i)
+// triples (i a row of this call), else every row.  With an empty layer this is
+// oracle_prefill_attention.
+void oracle_cache_prefill_attention(void* hc, int l, int T, int Hq, const double* q, const double* k,
+                                    const double* v, const uint8_t* evict, const int* rows, long n_rows,
+                                    double* o) {
+  Cache& c = *static_cast<Cache*>(hc);
+  const int g = Hq / c.Hkv, w = c.w, D = c.D;
+  const long total = rows ? n_rows : static_cast<long>(c.B) * Hq * T;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (long r = 0; r < total; ++r) {
+    int b, hq, i;
+    if (rows) {
+      b = rows[3 * r];
+      hq = rows[3 * r + 1];
+      i = rows[3 * r + 2];
+    } else {
+      b = static_cast<int>(r / (static_cast<long>(Hq) * T));
+      hq = static_cast<int>((r / T) % Hq);
+      i = static_cast<int>(r % T);
+    }
+    const int h = hq / g;
+    const size_t bh = c.bh(l, b, h);
+    const int pos0 = c.npos[bh], qi = pos0 + i;
+    std::vector<const double*> keys, vals;
+    for (int s = 0; s < c.count[bh]; ++s) {
+      const int j = c.slot_pos[bh * c.cap + s];
+      const bool marked = j >= pos0 - w && c.ring_evict[bh * w + j % w];
+      if (marked && qi - j >= w) continue;
+      const int id = c.page_table[bh * c.maxp + s / c.P];
+      const size_t off = (static_cast<size_t>(id) * c.P + s % c.P) * D;
+      keys.push_back(&c.kval[off]);
+      vals.push_back(&c.vval[off]);
+    }
+    for (int jj = 0; jj <= i; ++jj) {
+      const bool visible = (i - jj < w) || evict[(static_cast<size_t>(b) * c.Hkv + h) * T + jj] == 0;
+      if (!visible) continue;
+      keys.push_back(k + ((static_cast<size_t>(b) * T + jj) * c.Hkv + h) * D);
+      vals.push_back(v + ((static_cast<size_t>(b) * T + jj) * c.Hkv + h) * D);
+    }
+    const double* qq = q + ((static_cast<size_t>(b) * T + i) * Hq + hq) * D;
+    double* out = rows ? o + static_cast<size_t>(r) * D : o + ((static_cast<size_t>(b) * T + i) * Hq + hq) * D;
+    softmax_attend(qq, D, keys, vals, out);
+  }
 }
 
 }  // extern "C"

@@ -44,6 +44,8 @@ def lib():
         L.oracle_cache_export.argtypes = [C.c_void_p, C.c_int, ip, ip, ip, ip, ip, ip, up, ip]
         L.oracle_cache_pages.argtypes = [C.c_void_p, dp, dp, up, up, fp, fp]
         L.oracle_cache_decode_attention.argtypes = [C.c_void_p, C.c_int, C.c_int, dp, dp]
+        L.oracle_cache_prefill_attention.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, dp, dp, dp, up, ip,
+                                                     C.c_long, dp]
         _lib = L
     return _lib
 
@@ -239,4 +241,24 @@ class Cache:
         B, Hq, D = q.shape
         o = np.empty_like(q)
         lib().oracle_cache_decode_attention(self._h, layer, Hq, _p(q, C.c_double), _p(o, C.c_double))
+        return o
+
+    def prefill_attention(self, layer, q, k, v, evict, rows=None):
+        """Attention of a prefill call's rows against the cache as it is now
+        (call before prefill() of the same tokens) plus the call's own keys.
+        q [B,T,Hq,D], k/v [B,T,Hkv,D], evict [B,Hkv,T]; returns o[B,T,Hq,D] or
+        o[len(rows),D] for (b, hq, i) rows."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, T, Hq, D = q.shape
+        ev = _u8(evict)
+        assert ev.shape == (B, self.Hkv, T)
+        if rows is None:
+            o = np.empty((B, T, Hq, D), np.float64)
+            rp, n = None, 0
+        else:
+            r = np.ascontiguousarray(np.asarray(rows, np.int32).reshape(-1, 3))
+            o = np.empty((r.shape[0], D), np.float64)
+            rp, n = _p(r, C.c_int), r.shape[0]
+        lib().oracle_cache_prefill_attention(self._h, layer, T, Hq, _p(q, C.c_double), _p(k, C.c_double),
+                                             _p(v, C.c_double), _p(ev, C.c_uint8), rp, n, _p(o, C.c_double))
         return o

@@ -500,3 +500,127 @@ def test_fp8_decode_rescale_rule():
     dq = (O.e4m3_decode(c0).astype(np.float32) * s0).astype(np.float32)
     assert np.array_equal(pg["kcode"][0, 0], O.e4m3_encode(dq / s1))
     assert np.array_equal(pg["kcode"][0, 1], O.e4m3_encode(r1[0] / s1))
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill ([DMS-Qwen3], advanced options: the prompt is prefilled in
+# fixed-size chunks, each attending to the cache and to itself, and the chunks'
+# outputs are concatenated)
+# ---------------------------------------------------------------------------
+def _chunked(c, layer, q, k, v, ev, splits, rows_per_call=None):
+    outs, t0 = [], 0
+    for n in splits:
+        sl = slice(t0, t0 + n)
+        outs.append(c.prefill_attention(layer, np.ascontiguousarray(q[:, sl]), np.ascontiguousarray(k[:, sl]),
+                                        np.ascontiguousarray(v[:, sl]), np.ascontiguousarray(ev[:, :, sl])))
+        c.prefill(layer, np.ascontiguousarray(ev[:, :, sl]), np.ascontiguousarray(k[:, sl]).astype(np.float32),
+                  np.ascontiguousarray(v[:, sl]).astype(np.float32))
+        t0 += n
+    return np.concatenate(outs, 1)
+
+
+@pytest.mark.parametrize("splits", [[50], [13, 1, 20, 16], [3, 47], [8, 8, 8, 8, 8, 10], [7, 30, 13]])
+def test_chunked_prefill_equals_one_prefill(splits):
+    """With exact pages (bf16/fp32 values) a chunked prefill leaves the same
+    cache state and pages as one prefill of the whole prompt, and its rows'
+    attention equals the whole prompt's masked attention."""
+    B, T, Hq, Hkv, D, w, P = 2, 50, 4, 2, 16, 8, 4
+    # values the pages hold exactly (fp32 numbers)
+    q, k, v = (x.astype(np.float32).astype(np.float64) for x in rand_qkv(21, B, T, Hq, Hkv, D))
+    ev = (np.random.default_rng(22).random((B, Hkv, T)) < 0.6).astype(np.uint8)
+    one = O.Cache(1, B, Hkv, D, w, P, T + 4, 64, 0)
+    one.prefill(0, ev, k.astype(np.float32), v.astype(np.float32))
+    ref = O.prefill_attention(q, k, v, ev, w)
+    ch = O.Cache(1, B, Hkv, D, w, P, T + 4, 64, 0)
+    got = _chunked(ch, 0, q, k, v, ev, splits)
+    assert np.allclose(got, ref, rtol=0, atol=1e-12)
+    a, b = one.export(0), ch.export(0)
+    for key in ("npos", "count", "npages", "ring_slot", "ring_evict", "next_page"):
+        assert np.array_equal(a[key], b[key]), key
+    # page ids follow each call's grant order (one counter, (b, h) row-major
+    # per call), so they differ between one call and several; the pages used
+    # and every slot's stored row do not
+    pa, pb = one.pages(), ch.pages()
+    used_a, used_b = set(), set()
+    for bb in range(B):
+        for h in range(Hkv):
+            n = a["count"][bb, h]
+            assert np.array_equal(a["slot_pos"][bb, h, :n], b["slot_pos"][bb, h, :n])
+            ida = a["page_table"][bb, h, :a["npages"][bb, h]]
+            idb = b["page_table"][bb, h, :b["npages"][bb, h]]
+            used_a |= set(ida.tolist())
+            used_b |= set(idb.tolist())
+            for key in ("kval", "vval"):
+                ra = pa[key][ida].reshape(-1, D)[:n]
+                rb = pb[key][idb].reshape(-1, D)[:n]
+                assert np.array_equal(ra, rb), key
+    assert used_a == used_b
+    # and the decode steps after it see the same cache
+    qd = np.ascontiguousarray(q[:, T - 1])
+    assert np.array_equal(one.decode_attention(0, qd), ch.decode_attention(0, qd))
+
+
+def test_chunk_attention_sees_marked_window_keys_until_they_leave():
+    """A marked token of the previous chunk stays visible to the next chunk's
+    queries while it is inside their window, then disappears: brute force over
+    the visible set, with a single marked token."""
+    B, Hq, Hkv, D, w, P = 1, 1, 1, 8, 4, 4
+    T0, C = 6, 6
+    q, k, v = (x.astype(np.float32).astype(np.float64) for x in rand_qkv(23, B, T0 + C, Hq, Hkv, D))
+    ev = np.zeros((B, Hkv, T0 + C), np.uint8)
+    ev[0, 0, 4] = 1  # position 4 marked: visible to queries 4..7, gone from query 8 on
+    c = O.Cache(1, B, Hkv, D, w, P, T0 + C, 8, 0)
+    c.prefill(0, np.ascontiguousarray(ev[:, :, :T0]), k[:, :T0].astype(np.float32), v[:, :T0].astype(np.float32))
+    got = c.prefill_attention(0, q[:, T0:], k[:, T0:], v[:, T0:], np.ascontiguousarray(ev[:, :, T0:]))
+    sc = 1 / np.sqrt(D)
+    for i in range(C):
+        qi = T0 + i
+        vis = [j for j in range(qi + 1) if not (j == 4 and qi - j >= w)]
+        s = np.array([q[0, qi, 0] @ k[0, j, 0] * sc for j in vis])
+        p = np.exp(s - s.max())
+        want = (p[:, None] * v[0, vis, 0]).sum(0) / p.sum()
+        assert np.allclose(got[0, i, 0], want, rtol=0, atol=1e-12), i
+
+
+def test_fp8_chunk_of_one_token_is_a_decode_append():
+    """The FP8 rule for a prefill call whose rows land in a page that already
+    holds rows reduces, for a one-token call, to the decode append's rule."""
+    B, H, D, w, P, T0 = 1, 2, 8, 4, 4, 9
+    rng = np.random.default_rng(24)
+    k = (rng.standard_normal((B, T0 + 1, H, D)) * np.linspace(0.5, 4, T0 + 1)[None, :, None, None]).astype(np.float32)
+    v = rng.standard_normal((B, T0 + 1, H, D)).astype(np.float32)
+    ev = (rng.random((B, H, T0 + 1)) < 0.5).astype(np.uint8)
+    a = O.Cache(1, B, H, D, w, P, T0 + 1, 16, 0, fp8=True)
+    a.prefill(0, np.ascontiguousarray(ev[:, :, :T0]), np.ascontiguousarray(k[:, :T0]), np.ascontiguousarray(v[:, :T0]))
+    b = a.clone()
+    a.prefill(0, np.ascontiguousarray(ev[:, :, T0:]), np.ascontiguousarray(k[:, T0:]), np.ascontiguousarray(v[:, T0:]))
+    b.append(0, np.ascontiguousarray(ev[:, :, T0]), np.ascontiguousarray(k[:, T0]), np.ascontiguousarray(v[:, T0]))
+    pa, pb = a.pages(), b.pages()
+    for key in ("kcode", "vcode", "kscale", "vscale", "kval", "vval"):
+        assert np.array_equal(pa[key], pb[key]), key
+    sa, sb = a.export(0), b.export(0)
+    assert np.array_equal(sa["count"], sb["count"]) and np.array_equal(sa["slot_pos"], sb["slot_pos"])
+
+
+def test_fp8_chunked_scales_cover_every_row():
+    """After a chunked FP8 prefill every page's scale is at least each of its
+    rows' max |x| / 448, and every stored row decodes to within half a code
+    step of its input (the rescale only coarsens the grid)."""
+    B, H, D, w, P, T = 1, 2, 8, 6, 4, 40
+    rng = np.random.default_rng(25)
+    k = (rng.standard_normal((B, T, H, D)) * rng.uniform(0.2, 5, (1, T, 1, 1))).astype(np.float32)
+    v = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    ev = (rng.random((B, H, T)) < 0.5).astype(np.uint8)
+    c = O.Cache(1, B, H, D, w, P, T, 32, 0, fp8=True)
+    q = np.zeros((B, T, 2, D))
+    _chunked(c, 0, q, k, v, ev, [9, 5, 17, 9])
+    s, pg = c.export(0), c.pages()
+    for h in range(H):
+        for sl in range(s["count"][0, h]):
+            t = s["slot_pos"][0, h, sl]
+            pid = s["page_table"][0, h, sl // P]
+            sc = pg["kscale"][pid]
+            assert sc >= np.float32(np.max(np.abs(k[0, t, h]))) / np.float32(448.0)
+            # E4M3 has 3 mantissa bits: relative step 2^-3 above the subnormals
+            err = np.abs(pg["kval"][pid, sl % P] - k[0, t, h])
+            assert np.all(err <= np.maximum(np.abs(k[0, t, h]) * 2.0 ** -3, sc * 2.0 ** -8) + 1e-12)
