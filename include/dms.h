@@ -174,9 +174,18 @@ typedef struct dms_decide_params {
 } dms_decide_params;
 
 /* ---- prefill -------------------------------------------------------------------
- * One prompt of T tokens for every sequence of one layer ([DMS-Qwen3]: the
- * supported workflow is a single prefill followed by generation; a second
- * prefill into a non-empty layer is DMS_ERR_STATE).  In order, on `stream`:
+ * T prompt tokens for every sequence of one layer, at positions T0 .. T0+T-1
+ * where T0 is the number of tokens the layer already holds.  A prompt may be
+ * prefilled in several calls (chunked prefill, [DMS-Qwen3] "高级选项": the
+ * prompt split into fixed-size chunks, 4096 tokens by default): each call's
+ * queries attend to the keys the cache holds, as stored (FP8 pages decoded),
+ * plus the call's own keys, under the mask below, so with bf16/fp32 pages the
+ * chunks' outputs equal one prefill of the whole prompt.  Prefill calls may
+ * follow each other until the layer's first decode step; after it a prefill
+ * is DMS_ERR_STATE ([DMS-Qwen3] "当前限制": prefill-then-generate; reset the
+ * cache for a new prompt).  A call with T0 > 0 needs bf16 activations and a
+ * GQA group Hq/Hkv that is a power of two up to 16 (else DMS_ERR_INVALID), and
+ * T0 + T <= max_positions.  In order, on `stream`:
  *  1. decision logits alpha[B,Hkv,T] (when `decide` is non-NULL; else `alpha`
  *     is read as an input);
  *  2. for neuron sources the decision element is zeroed in place, then, when
@@ -286,19 +295,24 @@ DMS_API int dms_cache_status(dms_cache* cache, void* stream, int* status);
 DMS_API int dms_decide(dms_cache* cache, int seq_len, const dms_decide_params* decide, void* neuron_src,
                float* alpha, void* stream);
 
-/* Prefill layer `layer` (0 <= layer < L) of an empty cache; see dms_prefill_args.
- * Equivalent to dms_prefill_compact followed by dms_prefill_attention. */
+/* Prefill T tokens into layer `layer` (0 <= layer < L) after the tokens it
+ * already holds; see dms_prefill_args.  Equivalent to dms_prefill_compact
+ * followed by dms_prefill_attention. */
 DMS_API int dms_prefill(dms_cache* cache, int layer, const dms_prefill_args* args, void* stream);
 
 /* Steps 1-3 of dms_prefill: decision logits, neuron zeroing / rotation, and the
- * compaction of the prompt into the layer's pages ([FastDMS] prefill kernel).
- * Leaves the position-sorted list of kept tokens in the cache's scratch for
- * dms_prefill_attention.  DMS_ERR_STATE if the layer was already filled. */
+ * compaction of the tokens into the layer's pages ([FastDMS] prefill kernel),
+ * continuing from the layer's state.  Leaves the position-sorted list of kept
+ * tokens (and, for a later chunk, the keys and values of the last w positions
+ * before it) in the cache's scratch for dms_prefill_attention; that scratch is
+ * shared by the layers, so the attention must follow before another layer's
+ * compaction.  DMS_ERR_STATE after the layer's first decode step. */
 DMS_API int dms_prefill_compact(dms_cache* cache, int layer, const dms_prefill_args* args, void* stream);
 
-/* Step 4 of dms_prefill: the DMS-masked attention of the prompt.  Must follow
- * dms_prefill_compact of the same layer and length (else DMS_ERR_STATE); reads
- * args->q, k, v (as rotated by the compaction) and writes args->o. */
+/* Step 4 of dms_prefill: the DMS-masked attention of the call's tokens.  Must
+ * follow dms_prefill_compact of the same layer and length, with no other
+ * layer's compaction in between (else DMS_ERR_STATE); reads args->q, k, v (as
+ * rotated by the compaction) and writes args->o. */
 DMS_API int dms_prefill_attention(dms_cache* cache, int layer, const dms_prefill_args* args, void* stream);
 
 /* One decode step of layer `layer` after its prefill; DMS_ERR_STATE before the

@@ -23,8 +23,8 @@ constexpr int kMaxSmsForWork = 160;  // bound used to size the decode work list
 constexpr int kFuseDecideHeads = 64;  // decode decisions fused into the append up to B*Hkv heads
 
 struct Plan {
-  size_t ctrl, pos, count, npages, page_table, slot_pos, ring, plan, kept, kept_count, kept_upto, kept_k, kept_v, head_done, part_acc,
-      part_ml, k_scale, v_scale, k_pool, v_pool, total;
+  size_t ctrl, pos, count, npages, page_table, slot_pos, ring, plan, kept, kept_count, kept_upto, kept_k, kept_v, win_k,
+      win_v, head_done, part_acc, part_ml, k_scale, v_scale, k_pool, v_pool, total;
   int maxp, cap, pre_pages, items_cap, first_free;
 };
 
@@ -86,6 +86,9 @@ Plan make_plan(const dms_cache_desc* d) {
   const size_t kept_rows_bytes = d->act_dtype == DMS_BF16 ? B * H * d->max_positions * d->head_dim * 2 : 0;
   p.kept_k = take(kept_rows_bytes, 1024);
   p.kept_v = take(kept_rows_bytes, 1024);
+  const size_t win_rows_bytes = d->act_dtype == DMS_BF16 ? B * H * d->window * d->head_dim * 2 : 0;
+  p.win_k = take(win_rows_bytes, 1024);
+  p.win_v = take(win_rows_bytes, 1024);
   p.head_done = take(B * H * 4, 256);
   p.part_acc = take(static_cast<size_t>(p.items_cap) * g * d->head_dim * 4, 256);
   p.part_ml = take(static_cast<size_t>(p.items_cap) * g * 2 * 4, 256);
@@ -193,9 +196,12 @@ struct dms_cache {
   CUtensorMap kmap64, vmap64;  // pool pages, 64-row boxes (flat decode kernel)
   bool has_maps;
   CUtensorMap kept_kmap, kept_vmap;  // tcgen05 prefill: kept copies
+  CUtensorMap win_kmap, win_vmap;    // tcgen05 prefill of a later chunk: window copies
   bool has_kept_maps = false;
+  std::vector<char> decoded;  // a decode step ran on the layer since its last reset
   int compacted_layer = -1;  // layer whose kept list the prefill attention may use
   int compacted_len = 0;
+  int compacted_pos0 = 0;    // position of that call's first token
   int worklist_layer = -1;   // layer whose decode work list is current
 };
 
@@ -255,6 +261,7 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   }
   c->positions.assign(desc->num_layers, 0);
   c->prefilled.assign(desc->num_layers, 0);
+  c->decoded.assign(desc->num_layers, 0);
   CacheView& v = c->view;
   v.L = desc->num_layers;
   v.B = desc->batch;
@@ -292,6 +299,8 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   v.kept_upto = reinterpret_cast<int*>(b + p.kept_upto);
   v.kept_k = desc->act_dtype == DMS_BF16 ? b + p.kept_k : nullptr;
   v.kept_v = desc->act_dtype == DMS_BF16 ? b + p.kept_v : nullptr;
+  v.win_k = desc->act_dtype == DMS_BF16 ? b + p.win_k : nullptr;
+  v.win_v = desc->act_dtype == DMS_BF16 ? b + p.win_v : nullptr;
   v.head_done = reinterpret_cast<int*>(b + p.head_done);
   v.part_acc = reinterpret_cast<float*>(b + p.part_acc);
   v.part_ml = reinterpret_cast<float*>(b + p.part_ml);
@@ -318,8 +327,12 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
                                 static_cast<cuuint64_t>(desc->batch) * desc->num_kv_heads * desc->max_positions};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
     const cuuint32_t box[2] = {64u, 64u};  // 64-key tiles of the prefill attention
+    const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(D),
+                                 static_cast<cuuint64_t>(desc->batch) * desc->num_kv_heads * desc->window};
     c->has_kept_maps = make_bf16_map(&c->kept_kmap, v.kept_k, 2, dims, strides, box) &&
-                       make_bf16_map(&c->kept_vmap, v.kept_v, 2, dims, strides, box);
+                       make_bf16_map(&c->kept_vmap, v.kept_v, 2, dims, strides, box) &&
+                       make_bf16_map(&c->win_kmap, v.win_k, 2, wdims, strides, box) &&
+                       make_bf16_map(&c->win_vmap, v.win_v, 2, wdims, strides, box);
   }
   if (launch_init(v, true, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     delete c;
@@ -342,6 +355,7 @@ int dms_cache_reset(dms_cache* c, void* stream) {
   if (launch_init(c->view, false, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DMS_ERR_CUDA;
   std::fill(c->positions.begin(), c->positions.end(), 0);
   std::fill(c->prefilled.begin(), c->prefilled.end(), 0);
+  std::fill(c->decoded.begin(), c->decoded.end(), 0);
   c->compacted_layer = -1;
   c->worklist_layer = -1;
   return DMS_OK;
@@ -461,11 +475,23 @@ static int check_prefill(const dms_cache* c, int layer, const dms_prefill_args* 
   return DMS_OK;
 }
 
+// A later chunk of a chunked prefill (the layer already holds tokens) runs on
+// the tcgen05 attention, which reads the window and kept copies: bf16
+// activations and a GQA group that is a power of two up to 16.
+static bool chunk_capable(const dms_cache* c) {
+  const int g = c->desc.num_q_heads / c->desc.num_kv_heads;
+  return c->has_kept_maps && g <= 16 && (g & (g - 1)) == 0;
+}
+
 int dms_prefill_compact(dms_cache* c, int layer, const dms_prefill_args* a, void* stream) {
   int e = check_prefill(c, layer, a);
   if (e) return e;
-  if (c->prefilled[layer]) return DMS_ERR_STATE;
-  const int T = a->seq_len;
+  // prefill-then-generate: prefills (chunks) may follow each other until the
+  // layer's first decode step
+  if (c->decoded[layer]) return DMS_ERR_STATE;
+  const int T = a->seq_len, T0 = c->positions[layer];
+  if (T0 + T > c->desc.max_positions) return DMS_ERR_INVALID;
+  if (T0 > 0 && (!chunk_capable(c) || prefill_scan_smem(c->view, T0, T) > (200u << 10))) return DMS_ERR_INVALID;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   track_launch(c, layer, s);
   const CacheView& v = c->view;
@@ -477,24 +503,30 @@ int dms_prefill_compact(dms_cache* c, int layer, const dms_prefill_args* a, void
       return DMS_ERR_CUDA;
   }
   if (neuron || a->rope_cos) {
-    if (launch_neuron_rope(v, T, nullptr, a->q, a->k, neuron ? a->decide->offset : nullptr,
-                           neuron ? a->decide->offset_batch_stride : 0, neuron, a->alpha, a->rope_cos, a->rope_sin,
-                           s) != cudaSuccess)
+    // a later chunk's tokens sit at positions T0 + t (read on the device)
+    if (launch_neuron_rope(v, T, T0 > 0 ? v.pos + static_cast<long>(layer) * v.B : nullptr, a->q, a->k,
+                           neuron ? a->decide->offset : nullptr, neuron ? a->decide->offset_batch_stride : 0, neuron,
+                           a->alpha, a->rope_cos, a->rope_sin, s) != cudaSuccess)
       return DMS_ERR_CUDA;
   }
-  if (launch_prefill_scan(v, layer, T, a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
-  if (launch_prefill_scatter(v, layer, T, a->k, a->v, s) != cudaSuccess) return DMS_ERR_CUDA;
+  if (T0 > 0 && launch_prefill_context(v, layer, T0, s) != cudaSuccess) return DMS_ERR_CUDA;
+  if (launch_prefill_scan(v, layer, T0, T, a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
+  if (launch_prefill_scatter(v, layer, T0, T, a->k, a->v, s) != cudaSuccess) return DMS_ERR_CUDA;
   c->prefilled[layer] = 1;
-  c->positions[layer] = T;
+  c->positions[layer] = T0 + T;
   c->compacted_layer = layer;
   c->compacted_len = T;
+  c->compacted_pos0 = T0;
   return DMS_OK;
 }
 
 int dms_prefill_attention(dms_cache* c, int layer, const dms_prefill_args* a, void* stream) {
   int e = check_prefill(c, layer, a);
   if (e) return e;
-  if (c->compacted_layer != layer || c->compacted_len != a->seq_len) return DMS_ERR_STATE;
+  if (c->compacted_layer != layer || c->compacted_len != a->seq_len ||
+      c->compacted_pos0 + a->seq_len != c->positions[layer] || c->decoded[layer])
+    return DMS_ERR_STATE;
+  const int T0 = c->compacted_pos0;
   track_launch(c, layer, static_cast<cudaStream_t>(stream));
   // tensor maps of this call's q, k, v for the tcgen05 kernel
   PrefillMaps maps{};
@@ -518,9 +550,12 @@ int dms_prefill_attention(dms_cache* c, int layer, const dms_prefill_args* a, vo
                  make_bf16_map(&maps.v, a->v, 3, kd, ks, kbx) && make_bf16_map(&maps.o, a->o, 4, od, os, ob);
     maps.kept_k = c->kept_kmap;
     maps.kept_v = c->kept_vmap;
+    maps.win_k = c->win_kmap;
+    maps.win_v = c->win_vmap;
   }
-  if (launch_prefill_attention(c->view, a->seq_len, a->q, a->k, a->v, a->o, &maps, static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  if (T0 > 0 && !maps.valid) return DMS_ERR_INVALID;
+  if (launch_prefill_attention(c->view, T0, a->seq_len, a->q, a->k, a->v, a->o, &maps,
+                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DMS_ERR_CUDA;
   return DMS_OK;
 }
@@ -563,6 +598,7 @@ int dms_decode_append(dms_cache* c, int layer, const dms_decode_args* a, void* s
   }
   if (launch_decode_append(v, layer, a->k, a->v, a->alpha, fuse ? &da : nullptr, c->num_sms, s) != cudaSuccess)
     return DMS_ERR_CUDA;
+  c->decoded[layer] = 1;
   c->positions[layer] += 1;
   c->worklist_layer = layer;
   return DMS_OK;
@@ -653,6 +689,7 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   // bf16 pages: one launch -- attention over the pre-append slots plus the new
   // token, then the append, with the adapter's decision logits computed inside.
   if (int e = run_decode_kernel(c, layer, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, s)) return e;
+  c->decoded[layer] = 1;
   c->positions[layer] += 1;
   c->worklist_layer = layer;
   return DMS_OK;

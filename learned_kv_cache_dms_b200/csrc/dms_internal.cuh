@@ -41,6 +41,8 @@ struct CacheView {
   int* kept_upto;   // [B,Hkv,max_pos+1] prefill scratch: kept tokens before position t
   void* kept_k;     // [B*Hkv, max_pos, D] prefill scratch (bf16 activations): kept keys in list order
   void* kept_v;     //                      and values
+  void* win_k;      // [B*Hkv, w, D] prefill scratch (bf16 activations): the keys of the last w positions
+  void* win_v;      //                before a later chunk of a chunked prefill, and the values
   int* head_done;   // [B*Hkv] arrival counters of the attention CTAs (self-resetting)
   float* part_acc;  // [items_cap, g, D]   decode split-K partials, indexed by work item
   float* part_ml;   // [items_cap, g, 2]  (running max, running sum)
@@ -414,19 +416,26 @@ cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, f
 cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
                                int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
                                const float* sin_t, cudaStream_t s);
-cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T, const float* alpha, cudaStream_t s);
-cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T, const void* k, const void* v,
+// Prefill of T tokens at positions T0 .. T0 + T - 1 (T0 > 0: a later chunk of
+// a chunked prefill; launch_prefill_context rebuilds the kept list, kept copy
+// and window copy of the layer first).
+size_t prefill_scan_smem(const CacheView& c, int T0, int T);
+cudaError_t launch_prefill_context(const CacheView& c, int layer, int T0, cudaStream_t s);
+cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T0, int T, const float* alpha, cudaStream_t s);
+cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T0, int T, const void* k, const void* v,
                                    cudaStream_t s);
 // Tensor maps of the tcgen05 prefill attention: q [B*T, Hq, D] (box 64 x g x 128/g),
-// k and v [B*T, Hkv, D] (box 64 x 1 x 128), kept copies [B*Hkv*max_pos, D] (box 64 x 128),
-// all bf16 with the 128-byte swizzle.  `valid` is false when the shape is not covered.
+// k and v [B*T, Hkv, D] (box 64 x 1 x 128), kept copies [B*Hkv*max_pos, D] and
+// window copies [B*Hkv*w, D] (box 64 x 64), all bf16 with the 128-byte
+// swizzle.  `valid` is false when the shape is not covered.
 struct PrefillMaps {
-  CUtensorMap q, k, v, o, kept_k, kept_v;
+  CUtensorMap q, k, v, o, kept_k, kept_v, win_k, win_v;
   bool valid;
 };
-cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, const void* k, const void* v,
+cudaError_t launch_prefill_attention(const CacheView& c, int T0, int T, const void* q, const void* k, const void* v,
                                      void* o, const PrefillMaps* maps, cudaStream_t s);
-cudaError_t launch_prefill_attention_tc(const CacheView& c, int T, void* o, const PrefillMaps& maps, cudaStream_t s);
+cudaError_t launch_prefill_attention_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& maps,
+                                        cudaStream_t s);
 cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, const void* v, float* alpha,
                                  const DecideArgs* fused_decide, int num_sms, cudaStream_t s);
 cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q, void* o,

@@ -292,8 +292,11 @@ static cudaError_t launch_bf16(const CacheView& c, int T, const void* q, const v
   return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, const void* k, const void* v,
+cudaError_t launch_prefill_attention(const CacheView& c, int T0, int T, const void* q, const void* k, const void* v,
                                      void* o, const PrefillMaps* maps, cudaStream_t s) {
+  // a later chunk of a chunked prefill reads the window and kept copies: the
+  // tcgen05 kernel only (the host refuses other shapes for such calls)
+  if (T0 > 0) return maps && maps->valid ? launch_prefill_attention_tc(c, T0, T, o, *maps, s) : cudaErrorNotSupported;
   if (c.act_dtype == DMS_F32) {
     const long nrows = static_cast<long>(c.B) * T * c.Hq;
     const int grid = static_cast<int>((nrows * 32 + 255) / 256);
@@ -303,7 +306,7 @@ cudaError_t launch_prefill_attention(const CacheView& c, int T, const void* q, c
   }
   // bf16: the tcgen05 kernel; shapes it does not cover (g not a power of two
   // up to 16, or inputs not 16-byte aligned for TMA) take the mma.sync kernel
-  if (maps && maps->valid) return launch_prefill_attention_tc(c, T, o, *maps, s);
+  if (maps && maps->valid) return launch_prefill_attention_tc(c, 0, T, o, *maps, s);
   return c.D == 64 ? launch_bf16<64>(c, T, q, k, v, o, s) : launch_bf16<128>(c, T, q, k, v, o, s);
 }
 

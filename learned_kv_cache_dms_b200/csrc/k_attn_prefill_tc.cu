@@ -159,9 +159,13 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// One work item: a block of kPfQT * NP query positions of one (batch, KV head).
+// One work item: a block of kPfQT * NP query rows of one (batch, KV head);
+// i0, i1 index the call's rows, whose positions are T0 + i.  Its key tiles:
+// nkt kept-list tiles, npre band tiles of positions [jlo, T0) from the window
+// copy (a later chunk of a chunked prefill only), then the band tiles of the
+// call's own positions [jin, jhi].
 struct PfItem {
-  int h, b, bh, i0, i1, nk, jlo, jhi, nkt, ntiles;
+  int h, b, bh, i0, i1, nk, jlo, jhi, jin, nkt, npre, ntiles;
   bool valid;
 };
 
@@ -174,7 +178,8 @@ __device__ __forceinline__ int pf_item_index(int k, int G, int cta) {
 
 // The item's geometry; nk (kept keys before i1 - w, a table read) is passed in
 // so that callers can fetch it one item ahead.
-__device__ __forceinline__ PfItem pf_item(const CacheView& c, int T, int NP, int nblk, int nitems, int u, int nk) {
+__device__ __forceinline__ PfItem pf_item(const CacheView& c, int T0, int T, int NP, int nblk, int nitems, int u,
+                                          int nk) {
   PfItem it{};
   it.valid = u < nitems;
   if (!it.valid) return it;
@@ -185,11 +190,28 @@ __device__ __forceinline__ PfItem pf_item(const CacheView& c, int T, int NP, int
   it.i0 = blk * kPfQT * NP;
   it.i1 = min(T, it.i0 + kPfQT * NP);
   it.nk = nk;
-  it.jlo = max(0, it.i0 - c.w + 1);
-  it.jhi = it.i1 - 1;
+  it.jlo = max(0, T0 + it.i0 - c.w + 1);  // band positions [jlo, jhi]
+  it.jhi = T0 + it.i1 - 1;
+  it.jin = max(it.jlo, T0);
   it.nkt = (it.nk + kPfBN - 1) / kPfBN;  // kept tiles
-  it.ntiles = it.nkt + (it.jhi - it.jlo + kPfBN) / kPfBN;
+  it.npre = it.jlo < T0 ? (min(T0, it.jhi + 1) - it.jlo + kPfBN - 1) / kPfBN : 0;
+  it.ntiles = it.nkt + it.npre + (it.jhi - it.jin + kPfBN) / kPfBN;
   return it;
+}
+
+// Position of the first key of tile j of an item, and its source (0: kept
+// copy, 1: window copy, 2: the call's own rows).
+__device__ __forceinline__ int pf_tile(const PfItem& it, int j, int& src) {
+  if (j < it.nkt) {
+    src = 0;
+    return j * kPfBN;  // a kept-list rank
+  }
+  if (j < it.nkt + it.npre) {
+    src = 1;
+    return it.jlo + (j - it.nkt) * kPfBN;
+  }
+  src = 2;
+  return it.jin + (j - it.nkt - it.npre) * kPfBN;
 }
 
 // A table read issued where it is written (the asm keeps the compiler from
@@ -207,21 +229,23 @@ __device__ __forceinline__ int use_late(int v) {
   return r;
 }
 
-// kept_upto(bh, x) of item u's (batch, KV head) at position x = i0 + dx
-// (0 when x <= 0 or the item does not exist; x is clamped to T)
-__device__ __forceinline__ int pf_kept_upto(const CacheView& c, int T, int NP, int nblk, int nitems, int u, int dx) {
+// kept_upto(bh, x) of item u's (batch, KV head) at position x = T0 + i0 + dx
+// (0 when x <= 0 or the item does not exist; x is clamped to T0 + T)
+__device__ __forceinline__ int pf_kept_upto(const CacheView& c, int T0, int T, int NP, int nblk, int nitems, int u,
+                                           int dx) {
   if (u >= nitems) return 0;
   const int per = c.Hkv * c.B, blk = nblk - 1 - u / per, rem = u % per;
-  const int x = min(blk * kPfQT * NP + dx, T);
+  const int x = min(T0 + blk * kPfQT * NP + dx, T0 + T);
   return x > 0 ? ld_early_i32(c.kept_upto + static_cast<long>((rem / c.Hkv) * c.Hkv + rem % c.Hkv) * (c.max_pos + 1) + x)
                : 0;
 }
 
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
-    k_attn_prefill_tc(CacheView c, int T, __nv_bfloat16* o, const __grid_constant__ CUtensorMap qmap,
+    k_attn_prefill_tc(CacheView c, int T0, int T, __nv_bfloat16* o, const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                       const __grid_constant__ CUtensorMap kkmap, const __grid_constant__ CUtensorMap kvmap,
+                      const __grid_constant__ CUtensorMap wkmap, const __grid_constant__ CUtensorMap wvmap,
                       const __grid_constant__ CUtensorMap omap) {
   using L = PfSmem<D>;
   constexpr int ST = L::ST;
@@ -247,9 +271,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int u = pf_item_index(k, G, cta);
     if (u >= nitems) return 0;
     const int i0 = (nblk - 1 - u / (c.Hkv * c.B)) * kPfQT * NP, i1 = min(T, i0 + kPfQT * NP);
-    return pf_kept_upto(c, T, NP, nblk, nitems, u, i1 - i0 - w);
+    return pf_kept_upto(c, T0, T, NP, nblk, nitems, u, i1 - i0 - w);
   };
-  auto item = [&](int k, int nk) { return pf_item(c, T, NP, nblk, nitems, pf_item_index(k, G, cta), nk); };
+  auto item = [&](int k, int nk) { return pf_item(c, T0, T, NP, nblk, nitems, pf_item_index(k, G, cta), nk); };
 
   if (tid == 0) {
     mbar_init(&bar_q, 1);
@@ -304,15 +328,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             give_up();
             break;
           }
-          const bool kt = j < it.nkt;
-          const int jb = kt ? j * kPfBN : it.jlo + (j - it.nkt) * kPfBN;
+          int src;
+          const int jb = pf_tile(it, j, src);
           mbar_expect_tx(&k_full[st], L::KV_BYTES);
           for (int hf = 0; hf < L::HALVES; ++hf) {
             unsigned char* dk = sb + L::OFF_K + st * L::KV_BYTES + hf * (kPfBN * 128);
-            if (kt)
+            if (src == 0)
               tma_load_2d(dk, &kkmap, hf * 64, it.bh * c.max_pos + jb, &k_full[st]);
+            else if (src == 1)
+              tma_load_2d(dk, &wkmap, hf * 64, it.bh * w + (jb - (T0 - w)), &k_full[st]);
             else
-              tma_load_3d(dk, &kmap, hf * 64, it.h, it.b * T + jb, &k_full[st]);
+              tma_load_3d(dk, &kmap, hf * 64, it.h, it.b * T + (jb - T0), &k_full[st]);
           }
         }
         it = item(k + 1, use_late(nk_next));
@@ -331,15 +357,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             give_up();
             break;
           }
-          const bool kt = j < it.nkt;
-          const int jb = kt ? j * kPfBN : it.jlo + (j - it.nkt) * kPfBN;
+          int src;
+          const int jb = pf_tile(it, j, src);
           mbar_expect_tx(&v_full[st], L::KV_BYTES);
           for (int hf = 0; hf < L::HALVES; ++hf) {
             unsigned char* dv = sb + L::OFF_V + st * L::KV_BYTES + hf * (kPfBN * 128);
-            if (kt)
+            if (src == 0)
               tma_load_2d(dv, &kvmap, hf * 64, it.bh * c.max_pos + jb, &v_full[st]);
+            else if (src == 1)
+              tma_load_2d(dv, &wvmap, hf * 64, it.bh * w + (jb - (T0 - w)), &v_full[st]);
             else
-              tma_load_3d(dv, &vmap, hf * 64, it.h, it.b * T + jb, &v_full[st]);
+              tma_load_3d(dv, &vmap, hf * 64, it.h, it.b * T + (jb - T0), &v_full[st]);
           }
         }
         it = item(k + 1, use_late(nk_next));
@@ -424,7 +452,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // the row's count of visible kept keys: kept-list entries [0, ck) are the
     // positions <= i - w
     auto kept_visible = [&](int k) {
-      return pf_kept_upto(c, T, NP, nblk, nitems, pf_item_index(k, G, cta), p_row - w + 1);
+      return pf_kept_upto(c, T0, T, NP, nblk, nitems, pf_item_index(k, G, cta), p_row - w + 1);
     };
     bool ok = true;
     int t = 0;
@@ -438,14 +466,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // wait, so neither group can be left waiting.
     for (int k = 0; it.valid; ++k) {
       const int nk_next = item_nk(k + 1), ck_next = kept_visible(k + 1);
-      const int i_row = it.i0 + p_row;
+      const int i_row = T0 + it.i0 + p_row;                               // the row's position
       const int blo = max(0, i_row - w + 1), bhi = min(i_row, it.jhi);  // band positions of the row
       float m_ref = -INFINITY, l_row = 0.f;
       for (int j = 0; j < it.ntiles; ++j, ++t) {
         // visible columns [c_lo, c_hi] of this tile for the row
-        const bool kt = j < it.nkt;
-        const int jb = kt ? j * kPfBN : it.jlo + (j - it.nkt) * kPfBN;
-        const int c_lo = max(kt ? 0 : blo - jb, 0), c_hi = min(kt ? ck - 1 - jb : bhi - jb, kPfBN - 1);
+        int src;
+        const int jb = pf_tile(it, j, src);
+        const bool kt = src == 0;
+        // window-copy tiles end before the call's first position T0
+        const int hi = src == 1 ? min(bhi, T0 - 1) : bhi;
+        const int c_lo = max(kt ? 0 : blo - jb, 0), c_hi = min(kt ? ck - 1 - jb : hi - jb, kPfBN - 1);
         const bool row_full = c_lo == 0 && c_hi == kPfBN - 1;
         ok = ok && mbar_wait_bounded(&s_full[qt], t & 1);
         tc_fence_after();
@@ -597,7 +628,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 }
 
 template <int D>
-static cudaError_t launch_tc(const CacheView& c, int T, void* o, const PrefillMaps& m, cudaStream_t s) {
+static cudaError_t launch_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& m, cudaStream_t s) {
   const size_t smem = PfSmem<D>::BYTES + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_attn_prefill_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -605,13 +636,14 @@ static cudaError_t launch_tc(const CacheView& c, int T, void* o, const PrefillMa
   const int g = c.Hq / c.Hkv, NP = kPfRows / g;
   const long nitems = static_cast<long>((T + kPfQT * NP - 1) / (kPfQT * NP)) * c.Hkv * c.B;
   const int grid = static_cast<int>(min(nitems, static_cast<long>(c.num_sms)));  // persistent: one CTA per SM
-  k_attn_prefill_tc<D><<<grid, kPfThreads, smem, s>>>(c, T, static_cast<__nv_bfloat16*>(o), m.q, m.k, m.v, m.kept_k,
-                                                      m.kept_v, m.o);
+  k_attn_prefill_tc<D><<<grid, kPfThreads, smem, s>>>(c, T0, T, static_cast<__nv_bfloat16*>(o), m.q, m.k, m.v,
+                                                      m.kept_k, m.kept_v, m.win_k, m.win_v, m.o);
   return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_attention_tc(const CacheView& c, int T, void* o, const PrefillMaps& maps, cudaStream_t s) {
-  return c.D == 64 ? launch_tc<64>(c, T, o, maps, s) : launch_tc<128>(c, T, o, maps, s);
+cudaError_t launch_prefill_attention_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& maps,
+                                        cudaStream_t s) {
+  return c.D == 64 ? launch_tc<64>(c, T0, T, o, maps, s) : launch_tc<128>(c, T0, T, o, maps, s);
 }
 
 }  // namespace dms

@@ -47,6 +47,10 @@ cudaError_t launch_init(const CacheView& c, bool full, cudaStream_t s) {
     const size_t kept_bytes = static_cast<size_t>(c.B) * c.Hkv * c.max_pos * c.D * 2;
     if (e == cudaSuccess && c.kept_k) e = cudaMemsetAsync(c.kept_k, 0, kept_bytes, s);
     if (e == cudaSuccess && c.kept_v) e = cudaMemsetAsync(c.kept_v, 0, kept_bytes, s);
+    // and the window copies (rows of positions before 0 are read and masked)
+    const size_t win_bytes = static_cast<size_t>(c.B) * c.Hkv * c.w * c.D * 2;
+    if (e == cudaSuccess && c.win_k) e = cudaMemsetAsync(c.win_k, 0, win_bytes, s);
+    if (e == cudaSuccess && c.win_v) e = cudaMemsetAsync(c.win_v, 0, win_bytes, s);
     if (e != cudaSuccess) return e;
   }
   const long nbh = static_cast<long>(c.L) * c.B * c.Hkv;

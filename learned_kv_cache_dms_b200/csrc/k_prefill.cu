@@ -19,17 +19,27 @@ __device__ __forceinline__ bool bit_at(const unsigned* bits, int t) { return (bi
 constexpr int kScanU = 16;    // decision-logit words a warp loads before its ballots
 constexpr int kScatterU = 4;  // 16-byte row chunks a thread loads before it stores any
 
-// One CTA per (b, h).  Shared memory: five arrays of ceil(T/32) words.
-__global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, int T, const float* alpha) {
+// One CTA per (b, h), over the T tokens of one prefill call at positions
+// T0 .. T0 + T - 1 (T0 > 0: a later chunk of a chunked prefill, continuing
+// from the layer's state).  Shared memory: five arrays of ceil(T/32) words,
+// then (T0 > 0) a snapshot of the ring: the slots and decisions of positions
+// T0 - w .. T0 - 1, read while this kernel rewrites the ring.  With T0 > 0:
+//   open(t)  also holds when t - w < T0 and token t - w was kept;
+//   root(t)  stops at the first r with r - w < T0: token r takes a fresh slot
+//            (r open), or the slot of the marked token r - w (its ring entry);
+//   fresh slots are numbered from the layer's count; kept-list entries from
+//   the context's kept count (k_prefill_context).
+__global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, int T0, int T, const float* alpha) {
   extern __shared__ unsigned sm[];
   const int nw = (T + 31) >> 5;
   unsigned* ev = sm;                                       // evict bits
   unsigned* op = sm + nw;                                  // open bits
-  unsigned* kb = sm + 2 * nw;                              // kept-list bits: kept and t < T - w
+  unsigned* kb = sm + 2 * nw;                              // kept-list bits: kept and t < T0 + T - w
   int* opre = reinterpret_cast<int*>(sm + 3 * nw);         // exclusive prefix of open bits per word
   int* kpre = reinterpret_cast<int*>(sm + 4 * nw);         // exclusive prefix of kept-list bits per word
+  int* rs = reinterpret_cast<int*>(sm + 5 * nw);           // ring snapshot (T0 > 0)
   __shared__ int tmp[32];
-  __shared__ int s_last;
+  __shared__ int s_last, s_count0, s_kept0;
 
   const int BH = c.B * c.Hkv;
   const int bh = blockIdx.x, b = bh / c.Hkv, h = bh % c.Hkv;
@@ -38,6 +48,21 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
   const float* arow = alpha + (static_cast<long>(b) * c.Hkv + hs) * T;
   const int tid = threadIdx.x, lane = tid & 31, bd = blockDim.x;
   const int w = c.w;
+  const int end = T0 + T;  // positions held after this call
+  int* ring = c.ring + lbh * w;
+
+  if (T0 > 0) {
+    for (int i = tid; i < w; i += bd) rs[i] = ring[i];
+    if (tid == 0) {
+      s_count0 = c.count[lbh];
+      s_kept0 = c.kept_count[bh];
+    }
+  } else if (tid == 0) {
+    s_count0 = 0;
+    s_kept0 = 0;
+  }
+  // decision of an earlier token e (0 <= e < T0): its ring entry
+  auto evict_before = [&](int e) { return (rs[e % w] & static_cast<int>(RING_EVICT)) != 0; };
 
   // 1. evict bits (coalesced read, one ballot per 32 tokens).  Warp wid owns
   //    words wid, wid + nwarp, ...; it issues the loads of kScanU words before
@@ -57,11 +82,11 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
     }
   }
   __syncthreads();
-  // 2. open bits and kept-list bits
+  // 2. open bits and kept-list bits (t is the call's token index, T0 + t its position)
   for (int t0 = (tid & ~31); t0 < nw * 32; t0 += bd) {
-    const int t = t0 + lane;
-    const bool o = t < T && (t < w || !bit_at(ev, t - w));
-    const bool k = t < T - w && !bit_at(ev, t);
+    const int t = t0 + lane, e = T0 + t - w;
+    const bool o = t < T && (e < 0 || (e >= T0 ? !bit_at(ev, e - T0) : !evict_before(e)));
+    const bool k = T0 + t < end - w && t < T && !bit_at(ev, t);
     const unsigned mo = __ballot_sync(0xffffffffu, o);
     const unsigned mk = __ballot_sync(0xffffffffu, k);
     if (lane == 0) {
@@ -89,28 +114,34 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
   }
   __syncthreads();
   // 4. slots of the retained tokens; ring of the last w tokens; kept list
+  const int count0 = s_count0, kept0 = s_kept0;
   int* slot_pos = c.slot_pos + lbh * c.cap;
-  int* ring = c.ring + lbh * w;
   int* kept = c.kept + static_cast<long>(bh) * c.max_pos;
   int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
   for (int t = tid; t < T; t += bd) {
+    const int pos = T0 + t;
     const bool evt = bit_at(ev, t);
     const unsigned below = (1u << (t & 31)) - 1u;
-    kept_upto[t] = kpre[t >> 5] + __popc(kb[t >> 5] & below);
-    const bool retained = (t >= T - w) || !evt;
+    kept_upto[pos] = kept0 + kpre[t >> 5] + __popc(kb[t >> 5] & below);
+    const bool retained = (pos >= end - w) || !evt;
     if (!retained) continue;
     int r = t;
-    while (r >= w && bit_at(ev, r - w)) r -= w;
-    const int slot = opre[r >> 5] + __popc(op[r >> 5] & ((1u << (r & 31)) - 1u));
-    slot_pos[slot] = t;
-    if (t >= T - w) ring[t % w] = slot | (evt ? static_cast<int>(RING_EVICT) : 0);
-    if (t < T - w) kept[kpre[t >> 5] + __popc(kb[t >> 5] & below)] = t;
+    while (T0 + r - w >= T0 && bit_at(ev, r - w)) r -= w;
+    const int e = T0 + r - w;
+    int slot;
+    if (e >= 0 && e < T0 && evict_before(e))
+      slot = rs[e % w] & RING_SLOT_MASK;  // the marked token of the previous call leaves: its slot
+    else
+      slot = count0 + opre[r >> 5] + __popc(op[r >> 5] & ((1u << (r & 31)) - 1u));
+    slot_pos[slot] = pos;
+    if (pos >= end - w) ring[pos % w] = slot | (evt ? static_cast<int>(RING_EVICT) : 0);
+    if (pos < end - w) kept[kept0 + kpre[t >> 5] + __popc(kb[t >> 5] & below)] = pos;
   }
   if (tid == 0) {
-    kept_upto[T] = tot_keep;
-    c.count[lbh] = tot_open;
-    c.kept_count[bh] = tot_keep;
-    if (h == 0) c.pos[layer * c.B + b] = T;
+    kept_upto[end] = kept0 + tot_keep;
+    c.count[lbh] = count0 + tot_open;
+    c.kept_count[bh] = kept0 + tot_keep;
+    if (h == 0) c.pos[layer * c.B + b] = end;
   }
   // 5. the last CTA to arrive grants the extra pages of every head, in (b, h)
   //    row-major order, from the ascending page counter.
@@ -149,21 +180,131 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
     c.ctrl[CTRL_NEXT_PAGE] = min(next, c.pool_pages);
     c.ctrl[CTRL_DONE_SCAN] = 0;
   }
-  // slot plan of the first decode append (token T) of every head
+  // slot plan of the first decode append (token end) of every head
   __syncthreads();
   for (int i = tid; i < BH; i += bd) {
     const long li = static_cast<long>(layer) * BH + i;
-    *plan_at(c, li, T) = next_plan(c, li, T);
+    *plan_at(c, li, end) = next_plan(c, li, end);
   }
 }
 
-cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T, const float* alpha, cudaStream_t s) {
-  const int nw = (T + 31) / 32;
-  const size_t smem = static_cast<size_t>(nw) * 5 * 4;
+size_t prefill_scan_smem(const CacheView& c, int T0, int T) {
+  return (static_cast<size_t>((T + 31) / 32) * 5 + (T0 > 0 ? c.w : 0)) * 4;
+}
+
+cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T0, int T, const float* alpha, cudaStream_t s) {
+  const size_t smem = prefill_scan_smem(c, T0, T);
   cudaError_t e = cudaFuncSetAttribute(k_prefill_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  k_prefill_scan<<<c.B * c.Hkv, 1024, smem, s>>>(c, layer, T, alpha);
+  k_prefill_scan<<<c.B * c.Hkv, 1024, smem, s>>>(c, layer, T0, T, alpha);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Context of a prefill call into a layer that already holds T0 tokens (a later
+// chunk of a chunked prefill), rebuilt from the cache before the call's
+// compaction; one CTA per (b, h):
+//  1. the position-sorted list of the kept tokens before T0: kept_upto[x] =
+//     kept tokens at positions < x (x <= T0), kept[r] = the r-th kept
+//     position, and their K/V rows in the kept copy in that order.  A token
+//     held at position j < T0 - w is kept (a marked one would have been
+//     overwritten); a younger one is kept or marked as its ring entry says;
+//  2. the K/V rows of the last w positions T0 - w .. T0 - 1 in position order
+//     (window copy): the band keys the call's first queries see before its
+//     own.
+// The kept list and kept copy are scratch shared by the layers, so every call
+// rebuilds them for its own layer.  Rows are bf16: FP8 pages are decoded with
+// their page scale and rounded.
+// ---------------------------------------------------------------------------
+template <bool FP8>
+__device__ __forceinline__ uint4 page_row_chunk(const CacheView& c, const void* pool, const float* scales, int id,
+                                                int row, int ch) {
+  if (!FP8) {
+    return reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(pool) +
+                                          (static_cast<long>(id) * c.P + row) * c.D)[ch];
+  } else {
+    const uint2 q = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(pool) +
+                                                   (static_cast<long>(id) * c.P + row) * c.D)[ch];
+    const float sc = scales[id];
+    float f[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = fp8_decode(static_cast<uint8_t>(((e < 4 ? q.x : q.y) >> (8 * (e & 3))) & 0xFF)) * sc;
+    return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
+  }
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(1024) k_prefill_context(CacheView c, int layer, int T0) {
+  __shared__ int tmp[32];
+  const int bh = blockIdx.x, tid = threadIdx.x, bd = blockDim.x, w = c.w;
+  const long lbh = static_cast<long>(layer) * c.B * c.Hkv + bh;
+  const int count0 = c.count[lbh];
+  int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
+  int* kept = c.kept + static_cast<long>(bh) * c.max_pos;
+  const int* slot_pos = c.slot_pos + lbh * c.cap;
+  const int* ring = c.ring + lbh * w;
+  const int* pt = c.page_table + lbh * c.maxp;
+  auto is_kept = [&](int j) { return j < T0 - w || (ring[j % w] & static_cast<int>(RING_EVICT)) == 0; };
+  // 1. flags at the kept positions, then an exclusive scan in place
+  for (int x = tid; x <= T0; x += bd) kept_upto[x] = 0;
+  __syncthreads();
+  for (int s = tid; s < count0; s += bd) {
+    const int j = slot_pos[s];
+    if (is_kept(j)) kept_upto[j] = 1;
+  }
+  __syncthreads();
+  const int n = T0 + 1, per = (n + bd - 1) / bd;
+  const int x0 = min(n, tid * per), x1 = min(n, x0 + per);
+  int sum = 0;
+  for (int x = x0; x < x1; ++x) sum += kept_upto[x];
+  int total;
+  int base = block_exclusive_scan(sum, tmp, &total);
+  for (int x = x0; x < x1; ++x) {
+    const int f = kept_upto[x];
+    kept_upto[x] = base;
+    base += f;
+  }
+  __syncthreads();
+  if (tid == 0) c.kept_count[bh] = total;
+  // kept list and kept copy (16-byte chunks of bf16 rows)
+  const int cpr = c.D / 8;
+  __nv_bfloat16* kk = static_cast<__nv_bfloat16*>(c.kept_k) + static_cast<long>(bh) * c.max_pos * c.D;
+  __nv_bfloat16* kv = static_cast<__nv_bfloat16*>(c.kept_v) + static_cast<long>(bh) * c.max_pos * c.D;
+  for (int idx = tid; idx < count0 * cpr; idx += bd) {
+    const int s = idx / cpr, ch = idx % cpr;
+    const int j = slot_pos[s];
+    if (!is_kept(j)) continue;
+    const int r = kept_upto[j];
+    if (ch == 0) kept[r] = j;
+    const int id = pt[s / c.P];
+    if (id < 0) continue;  // no page (pool exhausted): the status word says so
+    reinterpret_cast<uint4*>(kk + static_cast<long>(r) * c.D)[ch] =
+        page_row_chunk<FP8>(c, c.k_pool, c.k_scale, id, s % c.P, ch);
+    reinterpret_cast<uint4*>(kv + static_cast<long>(r) * c.D)[ch] =
+        page_row_chunk<FP8>(c, c.v_pool, c.v_scale, id, s % c.P, ch);
+  }
+  // 2. window copy: position T0 - w + i at row i
+  __nv_bfloat16* wk = static_cast<__nv_bfloat16*>(c.win_k) + static_cast<long>(bh) * w * c.D;
+  __nv_bfloat16* wv = static_cast<__nv_bfloat16*>(c.win_v) + static_cast<long>(bh) * w * c.D;
+  for (int idx = tid; idx < w * cpr; idx += bd) {
+    const int i = idx / cpr, ch = idx % cpr, j = T0 - w + i;
+    if (j < 0) continue;
+    const int s = ring[j % w] & RING_SLOT_MASK;
+    const int id = pt[s / c.P];
+    if (id < 0) continue;
+    reinterpret_cast<uint4*>(wk + static_cast<long>(i) * c.D)[ch] =
+        page_row_chunk<FP8>(c, c.k_pool, c.k_scale, id, s % c.P, ch);
+    reinterpret_cast<uint4*>(wv + static_cast<long>(i) * c.D)[ch] =
+        page_row_chunk<FP8>(c, c.v_pool, c.v_scale, id, s % c.P, ch);
+  }
+}
+
+cudaError_t launch_prefill_context(const CacheView& c, int layer, int T0, cudaStream_t s) {
+  if (c.kv_dtype == DMS_FP8_E4M3)
+    k_prefill_context<true><<<c.B * c.Hkv, 1024, 0, s>>>(c, layer, T0);
+  else
+    k_prefill_context<false><<<c.B * c.Hkv, 1024, 0, s>>>(c, layer, T0);
   return cudaGetLastError();
 }
 
@@ -180,8 +321,10 @@ cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T, const floa
 
 // bf16 / fp32 pages: one CTA per (group of rg rows of a page, (b, h)), with
 // rg * 16-byte chunks per row <= kScatterU * blockDim.x (one batch per thread).
+// With T0 > 0 (a later chunk) only slots holding this call's tokens (positions
+// >= T0) are written; the others keep their rows.
 template <typename TA>
-__global__ void __launch_bounds__(256) k_prefill_scatter(CacheView c, int layer, int T, int rg, const TA* k,
+__global__ void __launch_bounds__(256) k_prefill_scatter(CacheView c, int layer, int T0, int T, int rg, const TA* k,
                                                          const TA* v) {
   const int gpp = (c.P + rg - 1) / rg;
   const int p = blockIdx.x / gpp, r0 = (blockIdx.x % gpp) * rg, bh = blockIdx.y;
@@ -209,7 +352,7 @@ __global__ void __launch_bounds__(256) k_prefill_scatter(CacheView c, int layer,
 #pragma unroll
     for (int u = 0; u < kScatterU; ++u) {
       const int idx = base + u * blockDim.x;
-      tt[u] = idx < n ? slot_pos[idx / cpr] : -1;
+      tt[u] = idx < n ? slot_pos[idx / cpr] - T0 : -1;  // the call's token index (< 0: an older row)
     }
 #pragma unroll
     for (int u = 0; u < kScatterU; ++u) {
@@ -218,7 +361,7 @@ __global__ void __launch_bounds__(256) k_prefill_scatter(CacheView c, int layer,
       const long src = ((static_cast<long>(b) * T + tt[u]) * c.Hkv + h) * c.D;
       kq[u] = reinterpret_cast<const uint4*>(k + src)[ch];
       vq[u] = reinterpret_cast<const uint4*>(v + src)[ch];
-      kr[u] = kept_copy && tt[u] < T - c.w ? kept_upto[tt[u]] : -1;
+      kr[u] = kept_copy && tt[u] < T - c.w ? kept_upto[T0 + tt[u]] : -1;
     }
 #pragma unroll
     for (int u = 0; u < kScatterU; ++u) {
@@ -273,8 +416,14 @@ __device__ __forceinline__ float amax8(const uint4 x, float m) {
   return m;
 }
 
-__global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int layer, int T, const __nv_bfloat16* k,
-                                                            const __nv_bfloat16* v) {
+// With T0 > 0 (a later chunk) a page may already hold rows of earlier calls
+// ("old" rows, positions < T0): its scale becomes max(old scale, amax of the
+// new rows / 448) and, when it grows, the old rows are first re-encoded from
+// their decoded values (code' = RNE(fl32(fl32(dec(code) * s_old) / s_new))),
+// the decode append's rule applied once for the call; pages without new rows
+// are left as they are.
+__global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int layer, int T0, int T,
+                                                            const __nv_bfloat16* k, const __nv_bfloat16* v) {
   __shared__ float red[32];
   const int p = blockIdx.x, bh = blockIdx.y;
   const int b = bh / c.Hkv, h = bh % c.Hkv;
@@ -285,6 +434,12 @@ __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int la
   if (id < 0) return;
   const int rows = min(c.P, cnt - p * c.P);
   const int* slot_pos = c.slot_pos + lbh * c.cap + static_cast<long>(p) * c.P;
+  // which rows this call wrote (new) and which it did not (old)
+  bool any_new = false, any_old = false;
+  for (int r = threadIdx.x; r < rows; r += blockDim.x) (slot_pos[r] >= T0 ? any_new : any_old) = true;
+  any_new = __syncthreads_or(any_new);
+  any_old = __syncthreads_or(any_old);
+  if (!any_new) return;
   const int cpr = c.D / 8;  // 8 bf16 per 16-byte input chunk
   const int n = rows * cpr;
   const int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
@@ -296,7 +451,7 @@ __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int la
 #pragma unroll
     for (int u = 0; u < kScatterU; ++u) {
       const int idx = base + u * blockDim.x;
-      tt[u] = idx < n ? slot_pos[idx / cpr] : -1;
+      tt[u] = idx < n ? slot_pos[idx / cpr] - T0 : -1;  // the call's token index (< 0: an old row)
     }
 #pragma unroll
     for (int u = 0; u < kScatterU; ++u) {
@@ -305,7 +460,7 @@ __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int la
       const long src = ((static_cast<long>(b) * T + tt[u]) * c.Hkv + h) * c.D;
       kq[u] = reinterpret_cast<const uint4*>(k + src)[ch];
       vq[u] = reinterpret_cast<const uint4*>(v + src)[ch];
-      kr[u] = kept_copy && tt[u] < T - c.w ? kept_upto[tt[u]] : -1;
+      kr[u] = kept_copy && tt[u] < T - c.w ? kept_upto[T0 + tt[u]] : -1;
     }
 #pragma unroll
     for (int u = 0; u < kScatterU; ++u) {
@@ -323,20 +478,30 @@ __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int la
   }
   ak = block_max(ak, red);
   av = block_max(av, red);
-  const float sk = __fdiv_rn(ak, 448.0f), sv = __fdiv_rn(av, 448.0f);
+  const float sk_old = any_old ? c.k_scale[id] : 0.f, sv_old = any_old ? c.v_scale[id] : 0.f;
+  const float sk = fmaxf(sk_old, __fdiv_rn(ak, 448.0f)), sv = fmaxf(sv_old, __fdiv_rn(av, 448.0f));
+  uint8_t* kd = static_cast<uint8_t*>(c.k_pool) + static_cast<long>(id) * c.P * c.D;
+  uint8_t* vd = static_cast<uint8_t*>(c.v_pool) + static_cast<long>(id) * c.P * c.D;
+  // old rows at a grown scale: re-encoded from their decoded values
+  const bool grow_k = any_old && sk > sk_old, grow_v = any_old && sv > sv_old;
+  if (grow_k || grow_v) {
+    for (int idx = threadIdx.x; idx < rows * c.D; idx += blockDim.x) {
+      if (slot_pos[idx / c.D] >= T0) continue;
+      if (grow_k) kd[idx] = fp8_encode(__fdiv_rn(__fmul_rn(fp8_decode(kd[idx]), sk_old), sk));
+      if (grow_v) vd[idx] = fp8_encode(__fdiv_rn(__fmul_rn(fp8_decode(vd[idx]), sv_old), sv));
+    }
+  }
   if (threadIdx.x == 0) {
     c.k_scale[id] = sk;
     c.v_scale[id] = sv;
   }
-  uint8_t* kd = static_cast<uint8_t*>(c.k_pool) + static_cast<long>(id) * c.P * c.D;
-  uint8_t* vd = static_cast<uint8_t*>(c.v_pool) + static_cast<long>(id) * c.P * c.D;
   for (int base = threadIdx.x; base < n; base += kScatterU * blockDim.x) {
     int tt[kScatterU];
     uint4 kq[kScatterU], vq[kScatterU];
 #pragma unroll
     for (int u = 0; u < kScatterU; ++u) {
       const int idx = base + u * blockDim.x;
-      tt[u] = idx < n ? slot_pos[idx / cpr] : -1;
+      tt[u] = idx < n ? slot_pos[idx / cpr] - T0 : -1;
     }
 #pragma unroll
     for (int u = 0; u < kScatterU; ++u) {
@@ -356,11 +521,14 @@ __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int la
   }
 }
 
-cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T, const void* k, const void* v,
+cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T0, int T, const void* k, const void* v,
                                    cudaStream_t s) {
-  const int pages = min(c.maxp, (T + c.P - 1) / c.P);
+  // pages that can hold the call's tokens: every page up to the layer's
+  // count (slots reused in place may sit in any earlier page)
+  const int pages = min(c.maxp, (T0 + T + c.P - 1) / c.P);
   if (c.kv_dtype == DMS_FP8_E4M3) {
-    k_prefill_scatter_fp8<<<dim3(pages, c.B * c.Hkv), 256, 0, s>>>(c, layer, T, static_cast<const __nv_bfloat16*>(k),
+    k_prefill_scatter_fp8<<<dim3(pages, c.B * c.Hkv), 256, 0, s>>>(c, layer, T0, T,
+                                                                   static_cast<const __nv_bfloat16*>(k),
                                                                    static_cast<const __nv_bfloat16*>(v));
     return cudaGetLastError();
   }
@@ -369,10 +537,10 @@ cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T, const v
   const int rg = max(1, min(c.P, kScatterU * 256 / cpr));
   dim3 grid(pages * ((c.P + rg - 1) / rg), c.B * c.Hkv);
   if (c.kv_dtype == DMS_BF16)
-    k_prefill_scatter<__nv_bfloat16><<<grid, 256, 0, s>>>(c, layer, T, rg, static_cast<const __nv_bfloat16*>(k),
+    k_prefill_scatter<__nv_bfloat16><<<grid, 256, 0, s>>>(c, layer, T0, T, rg, static_cast<const __nv_bfloat16*>(k),
                                                           static_cast<const __nv_bfloat16*>(v));
   else
-    k_prefill_scatter<float><<<grid, 256, 0, s>>>(c, layer, T, rg, static_cast<const float*>(k),
+    k_prefill_scatter<float><<<grid, 256, 0, s>>>(c, layer, T0, T, rg, static_cast<const float*>(k),
                                                   static_cast<const float*>(v));
   return cudaGetLastError();
 }

@@ -47,6 +47,7 @@ class Case:
     attn_rows: int | None = None  # sample this many prefill rows (None: all)
     staged: bool = False          # decode through dms_decode_append + dms_decode_attention
     kernel: str = "auto"          # decode attention kernel: auto | cluster | flat
+    chunks: tuple | None = None   # chunked prefill: the prompt's chunk sizes (summing to T)
 
     @property
     def N(self):
@@ -140,12 +141,37 @@ def build(case: Case):
                          rng.integers(0, T, case.attn_rows)], 1)
         rows[: min(B, case.attn_rows), 2] = T - 1  # always include the last rows
         out["rows"] = rows
-    out["o_prefill"] = O.prefill_attention(qs[:, :T], ks[:, :T], vs[:, :T], np.ascontiguousarray(evict[:, :, :T]),
-                                           case.w, rows=rows)
     cache = O.Cache(case.layers, B, case.Hkv, case.D, case.w, case.P, N, case.pool, case.prealloc,
                     fp8=case.kv == "fp8")
-    cache.prefill(case.layer, np.ascontiguousarray(evict[:, :, :T]), ks[:, :T].astype(np.float32),
-                  vs[:, :T].astype(np.float32))
+    if case.chunks is None:
+        out["o_prefill"] = O.prefill_attention(qs[:, :T], ks[:, :T], vs[:, :T],
+                                               np.ascontiguousarray(evict[:, :, :T]), case.w, rows=rows)
+        cache.prefill(case.layer, np.ascontiguousarray(evict[:, :, :T]), ks[:, :T].astype(np.float32),
+                      vs[:, :T].astype(np.float32))
+    else:
+        # each chunk attends to the cache as the earlier chunks left it, then is appended
+        assert sum(case.chunks) == T
+        outs, t0 = [], 0
+        for n in case.chunks:
+            sl = slice(t0, t0 + n)
+            ev_c = np.ascontiguousarray(evict[:, :, sl])
+            r_c = None
+            if rows is not None:
+                sel = (rows[:, 2] >= t0) & (rows[:, 2] < t0 + n)
+                r_c = rows[sel] - np.array([0, 0, t0])
+            o_c = cache.prefill_attention(case.layer, np.ascontiguousarray(qs[:, sl]), np.ascontiguousarray(ks[:, sl]),
+                                          np.ascontiguousarray(vs[:, sl]), ev_c, rows=r_c)
+            outs.append((sel, o_c) if rows is not None else o_c)
+            cache.prefill(case.layer, ev_c, np.ascontiguousarray(ks[:, sl]).astype(np.float32),
+                          np.ascontiguousarray(vs[:, sl]).astype(np.float32))
+            t0 += n
+        if rows is None:
+            out["o_prefill"] = np.concatenate(outs, 1)
+        else:
+            o = np.empty((rows.shape[0], case.D))
+            for sel, o_c in outs:
+                o[sel] = o_c
+            out["o_prefill"] = o
     out["state_prefill"] = cache.export(case.layer)
     out["pages_prefill"] = cache.pages() if case.steps == 0 else None
     o_dec = []
@@ -204,23 +230,34 @@ def run_gpu(case: Case, ins, cache=None):
     elif case.source in ("key", "query"):
         off = ins["offset"].to(dev)
         keep_alive.append(off)
-    qp = q[:, :T].contiguous()
-    kp = k[:, :T].contiguous()
-    vp = v[:, :T].contiguous()
-    o = torch.empty_like(qp)
-    if case.source == "input":
-        alpha = ins["alpha_in"][:, :, :T].contiguous().to(dev)
-    else:
-        alpha = torch.empty(B, case.Hkv, T, dtype=torch.float32, device=dev)
-        if case.source == "proj":
-            hp = h[:, :T].contiguous()
-            keep_alive.append(hp)
-            decide = B_.decide_params(off, hidden=hp, norm_weight=gamma, proj_weight=W)
+    chunks = case.chunks or (T,)
+    o_parts, a_parts, q_parts, k_parts = [], [], [], []
+    t0 = 0
+    for n in chunks:
+        qp = q[:, t0:t0 + n].contiguous()
+        kp = k[:, t0:t0 + n].contiguous()
+        vp = v[:, t0:t0 + n].contiguous()
+        o = torch.empty_like(qp)
+        if case.source == "input":
+            alpha = ins["alpha_in"][:, :, t0:t0 + n].contiguous().to(dev)
         else:
-            decide = B_.decide_params(off)
-    cache.prefill(case.layer, qp, kp, vp, o, alpha, decide=decide, rope=rope)
+            alpha = torch.empty(B, case.Hkv, n, dtype=torch.float32, device=dev)
+            if case.source == "proj":
+                hp = h[:, t0:t0 + n].contiguous()
+                keep_alive.append(hp)
+                decide = B_.decide_params(off, hidden=hp, norm_weight=gamma, proj_weight=W)
+            else:
+                decide = B_.decide_params(off)
+        cache.prefill(case.layer, qp, kp, vp, o, alpha, decide=decide, rope=rope)
+        o_parts.append(o)
+        a_parts.append(alpha)
+        q_parts.append(qp)
+        k_parts.append(kp)
+        keep_alive += [vp]
+        t0 += n
     torch.cuda.synchronize()
-    res = dict(o_prefill=o.cpu(), alpha_prefill=alpha.cpu(), k_prefill=kp.cpu(), q_prefill=qp.cpu())
+    res = dict(o_prefill=torch.cat(o_parts, 1).cpu(), alpha_prefill=torch.cat(a_parts, 2).cpu(),
+               k_prefill=torch.cat(k_parts, 1).cpu(), q_prefill=torch.cat(q_parts, 1).cpu())
     res["state_prefill"] = {k_: t.cpu().clone() for k_, t in cache.state(case.layer).items()}
     if case.steps == 0:
         res["pages_prefill"] = {k_: t.cpu().clone() for k_, t in cache.pages().items()}
