@@ -110,6 +110,10 @@ struct Cache {
   std::vector<uint8_t> kcode, vcode;     // [pool_pages, P, D]
   std::vector<float> kscale, vscale;     // [pool_pages]
   int store_values;
+  // Which token's decision logit marks token t (see append): 0 its own, +1
+  // token t - 1's (carried per head), -1 token t + 1's (set when it arrives).
+  int shift;
+  std::vector<uint8_t> carry;  // [L,B,Hkv] shift +1: the last token's own decision
 
   size_t bh(int l, int b, int h) const { return (static_cast<size_t>(l) * B + b) * Hkv + h; }
 };
@@ -227,12 +231,29 @@ void fp8_encode_prefill_page(Cache& c, size_t i, int p, int pos0) {
 // otherwise t takes the next free slot, and the block table grows by one page
 // whenever that slot starts a page.  Returns false if the append was dropped
 // (pool exhausted or capacity exceeded; the status word records which).
-bool append(Cache& c, int l, int b, int h, bool evict, const float* krow, const float* vrow,
+//
+// `decision` is token t's own decision (its logit > 0).  Which token it marks
+// follows the cache's shift ([DMS-Qwen3], attention: the training path shifts
+// the decision logits by one position):
+//   0   token t is marked by its own decision;
+//   +1  token t is marked by token t - 1's decision (the logits shifted right
+//       by one; token 0 takes the padding, "keep");
+//   -1  token t's decision marks token t - 1 (set now, in t - 1's ring entry);
+//       token t stays unmarked until token t + 1 arrives.
+bool append(Cache& c, int l, int b, int h, bool decision, const float* krow, const float* vrow,
             bool prefill_mode) {
   const size_t i = c.bh(l, b, h);
   const int t = c.npos[i];
   int* ring_slot = &c.ring_slot[i * c.w];
   uint8_t* ring_evict = &c.ring_evict[i * c.w];
+  bool evict = decision;
+  if (c.shift == 1) {
+    evict = c.carry[i] != 0;
+    c.carry[i] = decision ? 1 : 0;
+  } else if (c.shift == -1) {
+    evict = false;
+    if (t >= 1) ring_evict[(t - 1) % c.w] = decision ? 1 : 0;
+  }
   int slot;
   if (t >= c.w && ring_evict[t % c.w]) {
     slot = ring_slot[t % c.w];  // overwrite the evicted token in place
@@ -447,8 +468,10 @@ void oracle_prefill_attention(int B, int T, int Hq, int Hkv, int D, int w, const
 // Paged cache simulation
 // ---------------------------------------------------------------------------
 void* oracle_cache_new(int L, int B, int Hkv, int D, int w, int P, int max_pos, int pool_pages,
-                       int prealloc_tokens, int fp8, int store_values) {
+                       int prealloc_tokens, int fp8, int store_values, int shift) {
   Cache* c = new Cache();
+  c->shift = shift;
+  c->carry.assign(static_cast<size_t>(L) * B * Hkv, 0);
   c->L = L; c->B = B; c->Hkv = Hkv; c->D = D; c->w = w; c->P = P;
   c->max_pos = max_pos;
   c->maxp = (max_pos + P - 1) / P;
@@ -603,9 +626,10 @@ void oracle_cache_decode_attention(void* hc, int l, int Hq, const double* q, dou
 //     younger one is kept or marked as its ring entry says; values as stored
 //     (decoded for FP8 pages);
 //   * the call's own keys j <= i, from its inputs.
-// q [B,T,Hq,D], k/v [B,T,Hkv,D], evict [B,Hkv,T]; rows: optional (b, hq, i)
-// triples (i a row of this call), else every row.  With an empty layer this is
-// oracle_prefill_attention.
+// q [B,T,Hq,D], k/v [B,T,Hkv,D], evict [B,Hkv,T] (the call's tokens' own
+// decisions; which token each marks follows the cache's shift, as in append);
+// rows: optional (b, hq, i) triples (i a row of this call), else every row.
+// With an empty layer and no shift this is oracle_prefill_attention.
 void oracle_cache_prefill_attention(void* hc, int l, int T, int Hq, const double* q, const double* k,
                                     const double* v, const uint8_t* evict, const int* rows, long n_rows,
                                     double* o) {
@@ -627,10 +651,20 @@ void oracle_cache_prefill_attention(void* hc, int l, int T, int Hq, const double
     const int h = hq / g;
     const size_t bh = c.bh(l, b, h);
     const int pos0 = c.npos[bh], qi = pos0 + i;
+    const uint8_t* ev = evict + (static_cast<size_t>(b) * c.Hkv + h) * T;  // the call's own decisions
+    // the mark of the call's token jj under the cache's shift
+    auto call_mark = [&](int jj) -> bool {
+      if (c.shift == 1) return jj == 0 ? c.carry[bh] != 0 : ev[jj - 1] != 0;
+      if (c.shift == -1) return jj + 1 < T ? ev[jj + 1] != 0 : false;
+      return ev[jj] != 0;
+    };
     std::vector<const double*> keys, vals;
     for (int s = 0; s < c.count[bh]; ++s) {
       const int j = c.slot_pos[bh * c.cap + s];
-      const bool marked = j >= pos0 - w && c.ring_evict[bh * w + j % w];
+      // the layer's last token is marked by this call's first decision when
+      // a token's decision marks the one before it
+      const bool mark = (c.shift == -1 && j == pos0 - 1) ? ev[0] != 0 : c.ring_evict[bh * w + j % w] != 0;
+      const bool marked = j >= pos0 - w && mark;
       if (marked && qi - j >= w) continue;
       const int id = c.page_table[bh * c.maxp + s / c.P];
       const size_t off = (static_cast<size_t>(id) * c.P + s % c.P) * D;
@@ -638,7 +672,7 @@ void oracle_cache_prefill_attention(void* hc, int l, int T, int Hq, const double
       vals.push_back(&c.vval[off]);
     }
     for (int jj = 0; jj <= i; ++jj) {
-      const bool visible = (i - jj < w) || evict[(static_cast<size_t>(b) * c.Hkv + h) * T + jj] == 0;
+      const bool visible = (i - jj < w) || !call_mark(jj);
       if (!visible) continue;
       keys.push_back(k + ((static_cast<size_t>(b) * T + jj) * c.Hkv + h) * D);
       vals.push_back(v + ((static_cast<size_t>(b) * T + jj) * c.Hkv + h) * D);

@@ -32,7 +32,7 @@ def lib():
         L.oracle_rope.argtypes = [C.c_int] * 4 + [dp, C.c_int, dp, dp]
         L.oracle_round_bf16_n.argtypes = [dp, fp, C.c_long]
         L.oracle_prefill_attention.argtypes = [C.c_int] * 6 + [dp, dp, dp, up, ip, C.c_long, dp]
-        L.oracle_cache_new.argtypes = [C.c_int] * 11
+        L.oracle_cache_new.argtypes = [C.c_int] * 12
         L.oracle_cache_new.restype = C.c_void_p
         L.oracle_cache_delete.argtypes = [C.c_void_p]
         L.oracle_cache_clone.argtypes = [C.c_void_p]
@@ -173,7 +173,7 @@ class Cache:
     """Sequential simulation of the paged DMS cache (one object per test)."""
 
     def __init__(self, L, B, Hkv, D, window, block, max_pos, pool_pages, prealloc_tokens=0,
-                 fp8=False, store_values=True):
+                 fp8=False, store_values=True, shift=0):
         self.L, self.B, self.Hkv, self.D = L, B, Hkv, D
         self.w, self.P, self.max_pos = window, block, max_pos
         self.maxp = (max_pos + block - 1) // block
@@ -181,8 +181,9 @@ class Cache:
         self.pool_pages = pool_pages
         self.fp8 = bool(fp8)
         self.store_values = bool(store_values)
+        self.shift = int(shift)
         self._h = lib().oracle_cache_new(L, B, Hkv, D, window, block, max_pos, pool_pages,
-                                         prealloc_tokens, int(self.fp8), int(self.store_values))
+                                         prealloc_tokens, int(self.fp8), int(self.store_values), self.shift)
 
     def clone(self):
         """An independent copy (state and pages) of this cache."""

@@ -624,3 +624,67 @@ def test_fp8_chunked_scales_cover_every_row():
             # E4M3 has 3 mantissa bits: relative step 2^-3 above the subnormals
             err = np.abs(pg["kval"][pid, sl % P] - k[0, t, h])
             assert np.all(err <= np.maximum(np.abs(k[0, t, h]) * 2.0 ** -3, sc * 2.0 ** -8) + 1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Decision shift ([DMS-Qwen3], attention: the training path shifts the decision
+# logits by one position).  +1: token t is marked by token t - 1's decision
+# (token 0 by the padding, "keep"); -1: token t's decision marks token t - 1.
+# Each reduces to the unshifted rule applied to the correspondingly shifted
+# decisions.
+# ---------------------------------------------------------------------------
+def _shifted_bits(bits, shift):
+    out = np.zeros_like(bits)
+    if shift == 1:
+        out[..., 1:] = bits[..., :-1]
+    elif shift == -1:
+        out[..., :-1] = bits[..., 1:]   # the last token's mark is still pending (keep)
+    else:
+        out[:] = bits
+    return out
+
+
+@pytest.mark.parametrize("shift", [1, -1])
+@pytest.mark.parametrize("splits", [[40], [11, 17, 12]])
+def test_shift_reduces_to_the_unshifted_rule(shift, splits):
+    B, H, D, w, P, T, n = 2, 2, 8, 5, 4, 40, 15
+    rng = np.random.default_rng(30 + shift)
+    bits = (rng.random((B, H, T + n)) < 0.55).astype(np.uint8)
+    k = rng.standard_normal((B, T + n, H, D)).astype(np.float32)
+    a = O.Cache(1, B, H, D, w, P, T + n, 120, 0, shift=shift)
+    t0 = 0
+    for m in splits:
+        a.prefill(0, np.ascontiguousarray(bits[:, :, t0:t0 + m]), np.ascontiguousarray(k[:, t0:t0 + m]),
+                  np.ascontiguousarray(k[:, t0:t0 + m]))
+        t0 += m
+    for t in range(T, T + n):
+        a.append(0, np.ascontiguousarray(bits[:, :, t]), np.ascontiguousarray(k[:, t]), np.ascontiguousarray(k[:, t]))
+    ref_bits = _shifted_bits(bits, shift)
+    b = O.Cache(1, B, H, D, w, P, T + n, 120, 0)
+    b.prefill(0, np.ascontiguousarray(ref_bits[:, :, :T]), np.ascontiguousarray(k[:, :T]), np.ascontiguousarray(k[:, :T]))
+    for t in range(T, T + n):
+        b.append(0, np.ascontiguousarray(ref_bits[:, :, t]), np.ascontiguousarray(k[:, t]), np.ascontiguousarray(k[:, t]))
+    sa, sb = a.export(0), b.export(0)
+    for key in ("count", "npages", "ring_slot", "ring_evict", "next_page", "slot_pos"):
+        if key == "slot_pos":
+            for bb in range(B):
+                for h in range(H):
+                    c = sa["count"][bb, h]
+                    assert np.array_equal(sa[key][bb, h, :c], sb[key][bb, h, :c])
+        elif key != "page_table":
+            assert np.array_equal(sa[key], sb[key]), key
+    if len(splits) == 1:  # one prefill call: the same page ids, so the same pages
+        assert np.array_equal(a.pages()["kval"], b.pages()["kval"])
+
+
+@pytest.mark.parametrize("shift", [1, -1])
+def test_shift_attention_reduces_to_masked_attention(shift):
+    """A prefill's rows under a shift see exactly the keys the unshifted mask
+    gives for the shifted decisions; across a chunk boundary too."""
+    B, Hq, Hkv, D, w, P, T = 1, 2, 1, 8, 6, 4, 36
+    q, k, v = (x.astype(np.float32).astype(np.float64) for x in rand_qkv(33, B, T, Hq, Hkv, D))
+    bits = (np.random.default_rng(34).random((B, Hkv, T)) < 0.6).astype(np.uint8)
+    ref = O.prefill_attention(q, k, v, _shifted_bits(bits, shift), w)
+    c = O.Cache(1, B, Hkv, D, w, P, T, 40, 0, shift=shift)
+    got = _chunked(c, 0, q, k, v, bits, [13, 23])
+    assert np.allclose(got, ref, rtol=0, atol=1e-12)
