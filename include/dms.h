@@ -120,6 +120,16 @@ typedef struct dms_cache_desc {
   int disable_eviction; /* nonzero: every decision is "keep" (vanilla model)    */
   int decode_kernel;    /* enum dms_decode_kernel: how a decode step splits the
                            attention over the SMs (0: chosen from the shape)  */
+  int decision_shift;   /* which token's decision marks token t for eviction
+                           ([DMS-Qwen3] "注意力实现": the training path shifts
+                           the decision logits by one position; the operators
+                           of the page are garbled, so both directions exist):
+                             0  token t's own decision (default);
+                            +1  token t-1's decision: the logits shifted right
+                                by one, token 0 padded with "keep";
+                            -1  token t+1's decision: a token's decision marks
+                                the token before it, so the newest token is
+                                unmarked until the next one arrives        */
 } dms_cache_desc;
 
 /* Fill `desc` with the defaults of the DMS configuration record: window 512,
@@ -318,6 +328,21 @@ DMS_API int dms_prefill_attention(dms_cache* cache, int layer, const dms_prefill
 /* One decode step of layer `layer` after its prefill; DMS_ERR_STATE before the
  * prefill or when max_positions tokens are already held. */
 DMS_API int dms_decode_step(dms_cache* cache, int layer, const dms_decode_args* args, void* stream);
+
+/* One decode step of the layers [layer, layer + num_layers) in one launch of
+ * the attention kernel (one thread-block cluster per (layer, b, h)), for a
+ * stack whose layers do not feed each other within a step -- the same result
+ * as dms_decode_step on each layer in turn (page grants in (layer, b, h)
+ * order).  Every array of `args` holds the num_layers layers back to back:
+ * q/o [L',B,Hq,D], k/v [L',B,Hkv,D], alpha [L',B,Hkv]; with decision
+ * parameters, hidden [L',B,hidden], norm_weight [L',hidden], proj_weight
+ * [L',Hkv,hidden], proj_bias [L',Hkv] (or NULL) and offset [L',B,Hkv] (batch
+ * stride Hkv) or [L',Hkv] (batch stride 0).  bf16 pages only
+ * (DMS_ERR_INVALID otherwise: FP8 pages are re-encoded before they are
+ * attended); every layer of the range must be prefilled and hold the same
+ * number of tokens (else DMS_ERR_STATE). */
+DMS_API int dms_decode_step_layers(dms_cache* cache, int layer, int num_layers, const dms_decode_args* args,
+                                   void* stream);
 
 /* First half of dms_decode_step: decision logit, rotation and the append of
  * the new token ([FastDMS] decode kernel), plus the work list of the attention.

@@ -45,7 +45,7 @@ class dms_cache_desc(C.Structure):
                                        "window", "block", "max_positions", "prealloc_tokens", "pool_pages",
                                        "act_dtype", "kv_dtype", "alpha_per", "alpha_source")] + \
               [("alpha_scale", C.c_float), ("rms_eps", C.c_float), ("disable_eviction", C.c_int),
-               ("decode_kernel", C.c_int)]
+               ("decode_kernel", C.c_int), ("decision_shift", C.c_int)]
 
 
 class dms_cache_view(C.Structure):
@@ -95,17 +95,19 @@ _lib.dms_decode_attention.argtypes = [_P, C.c_int, _P, _P, _P]
 _lib.dms_decode_attention_noalloc.argtypes = [_P, C.c_int, _P, _P, _P]
 _lib.dms_cache_positions.argtypes = [_P, C.c_int]
 _lib.dms_selftest_wait_timeout.argtypes = [_P, C.c_int, _P]
+_lib.dms_decode_step_layers.argtypes = [_P, C.c_int, C.c_int, C.POINTER(dms_decode_args), _P]
 for _f in ("dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset", "dms_cache_get_layout",
            "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step", "dms_cache_positions",
            "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append", "dms_decode_attention",
-           "dms_decode_attention_noalloc", "dms_cache_export", "dms_selftest_wait_timeout"):
+           "dms_decode_attention_noalloc", "dms_cache_export", "dms_selftest_wait_timeout",
+           "dms_decode_step_layers"):
     getattr(_lib, _f).restype = C.c_int
 
 EXPORTED = ("dms_cache_desc_default", "dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset",
             "dms_cache_get_layout", "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step",
             "dms_cache_positions", "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append",
             "dms_decode_attention", "dms_decode_attention_noalloc", "dms_cache_export",
-            "dms_selftest_wait_timeout")
+            "dms_selftest_wait_timeout", "dms_decode_step_layers")
 
 
 def _check(code, where):
@@ -220,6 +222,11 @@ def dms_decode_attention_noalloc(handle: int, layer: int, q, o, stream=None) -> 
 
 def dms_cache_positions(handle: int, layer: int) -> int:
     return _check(_lib.dms_cache_positions(handle, layer), "dms_cache_positions")
+
+
+def dms_decode_step_layers(handle: int, layer: int, num_layers: int, args: dms_decode_args, stream=None) -> None:
+    _check(_lib.dms_decode_step_layers(handle, layer, num_layers, C.byref(args), _stream(stream)),
+           "dms_decode_step_layers")
 
 
 def dms_selftest_wait_timeout(handle: int, tries: int, stream=None) -> None:

@@ -544,8 +544,8 @@ __device__ __forceinline__ bool count_step(const CacheView& c, int granted, int 
   *done = 0ull;
   return true;
 }
-__device__ __forceinline__ void advance_positions(const CacheView& c, int layer, int first, int stride) {
-  for (int bb = first; bb < c.B; bb += stride) atomicAdd(&c.pos[layer * c.B + bb], 1);
+__device__ __forceinline__ void advance_positions(const CacheView& c, int layer, int first, int stride, int nl = 1) {
+  for (int bb = first; bb < nl * c.B; bb += stride) atomicAdd(&c.pos[layer * c.B + bb], 1);
 }
 
 __device__ __forceinline__ int4 make_plan(int ringv, int t, int cnt, int have, const CacheView& c) {

@@ -23,7 +23,7 @@ constexpr int kMaxSmsForWork = 160;  // bound used to size the decode work list
 constexpr int kFuseDecideHeads = 64;  // decode decisions fused into the append up to B*Hkv heads
 
 struct Plan {
-  size_t ctrl, pos, count, npages, page_table, slot_pos, ring, plan, kept, kept_count, kept_upto, kept_k, kept_v, win_k,
+  size_t ctrl, pos, count, carry, npages, page_table, slot_pos, ring, plan, kept, kept_count, kept_upto, kept_k, kept_v, win_k,
       win_v, head_done, part_acc, part_ml, k_scale, v_scale, k_pool, v_pool, total;
   int maxp, cap, pre_pages, items_cap, first_free;
 };
@@ -54,6 +54,7 @@ int check_desc(const dms_cache_desc* d) {
   if (d->alpha_source != DMS_ALPHA_PROJ && d->num_kv_heads > 32) return DMS_ERR_INVALID;
   if (!(d->alpha_scale == d->alpha_scale) || !(d->rms_eps >= 0.0f)) return DMS_ERR_INVALID;
   if (d->decode_kernel < DMS_DECODE_AUTO || d->decode_kernel > DMS_DECODE_FLAT) return DMS_ERR_INVALID;
+  if (d->decision_shift < -1 || d->decision_shift > 1) return DMS_ERR_INVALID;
   return DMS_OK;
 }
 
@@ -75,6 +76,7 @@ Plan make_plan(const dms_cache_desc* d) {
   p.ctrl = take(CTRL_WORDS * 4, 256);
   p.pos = take(L * B * 4, 256);
   p.count = take(L * B * H * 4, 256);
+  p.carry = take(L * B * H * 4, 256);
   p.npages = take(L * B * H * 4, 256);
   p.page_table = take(L * B * H * p.maxp * 4, 256);
   p.slot_pos = take(L * B * H * p.cap * 4, 256);
@@ -282,6 +284,7 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   v.alpha_source = desc->alpha_source;
   v.disable = desc->disable_eviction ? 1 : 0;
   v.decode_kernel = desc->decode_kernel;
+  v.shift = desc->decision_shift;
   v.alpha_scale = desc->alpha_scale;
   v.rms_eps = desc->rms_eps;
   v.num_sms = c->num_sms;
@@ -289,6 +292,7 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   v.ctrl = reinterpret_cast<int*>(b + p.ctrl);
   v.pos = reinterpret_cast<int*>(b + p.pos);
   v.count = reinterpret_cast<int*>(b + p.count);
+  v.carry = reinterpret_cast<int*>(b + p.carry);
   v.npages = reinterpret_cast<int*>(b + p.npages);
   v.page_table = reinterpret_cast<int*>(b + p.page_table);
   v.slot_pos = reinterpret_cast<int*>(b + p.slot_pos);
@@ -431,7 +435,7 @@ static int check_decide(const dms_cache* c, const dms_decide_params* d) {
 }
 
 static DecideArgs decide_args(const dms_decide_params* d) {
-  DecideArgs a;
+  DecideArgs a{};
   a.hidden = d->hidden;
   a.gamma = d->norm_weight;
   a.W = d->proj_weight;
@@ -509,7 +513,7 @@ int dms_prefill_compact(dms_cache* c, int layer, const dms_prefill_args* a, void
                            a->alpha, a->rope_cos, a->rope_sin, s) != cudaSuccess)
       return DMS_ERR_CUDA;
   }
-  if (T0 > 0 && launch_prefill_context(v, layer, T0, s) != cudaSuccess) return DMS_ERR_CUDA;
+  if (T0 > 0 && launch_prefill_context(v, layer, T0, T, a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
   if (launch_prefill_scan(v, layer, T0, T, a->alpha, s) != cudaSuccess) return DMS_ERR_CUDA;
   if (launch_prefill_scatter(v, layer, T0, T, a->k, a->v, s) != cudaSuccess) return DMS_ERR_CUDA;
   c->prefilled[layer] = 1;
@@ -692,6 +696,60 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   c->decoded[layer] = 1;
   c->positions[layer] += 1;
   c->worklist_layer = layer;
+  return DMS_OK;
+}
+
+int dms_decode_step_layers(dms_cache* c, int layer0, int num_layers, const dms_decode_args* a, void* stream) {
+  if (!c || !a || num_layers < 1 || layer0 < 0 || layer0 + num_layers > c->desc.num_layers) return DMS_ERR_INVALID;
+  if (!a->q || !a->k || !a->v || !a->o || !a->alpha) return DMS_ERR_INVALID;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o)) return DMS_ERR_INVALID;
+  if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
+  // one fused launch: bf16 pages (FP8 pages append before they are attended)
+  if (c->desc.kv_dtype != DMS_BF16 || !c->has_maps) return DMS_ERR_INVALID;
+  if (a->decide) {
+    int e = check_decide(c, a->decide);
+    if (e) return e;
+  }
+  const int t = c->positions[layer0];
+  for (int l = layer0; l < layer0 + num_layers; ++l)
+    if (!c->prefilled[l] || c->positions[l] != t || t >= c->desc.max_positions) return DMS_ERR_STATE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const CacheView& v = c->view;
+  const int B = c->desc.batch, Hq = c->desc.num_q_heads, Hkv = c->desc.num_kv_heads, D = c->desc.head_dim;
+  const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
+  const long ostride_layer = a->decide ? static_cast<long>(a->decide->offset_batch_stride ? B * Hkv : Hkv) : 0;
+  if (neuron || a->rope_cos) {
+    // the decision neuron / rotary pass of each layer (its rows of q and k)
+    track_launch(c, -1, s);
+    for (int l = 0; l < num_layers; ++l) {
+      char* ql = static_cast<char*>(a->q) + static_cast<long>(l) * B * Hq * D * 2;
+      char* kl = static_cast<char*>(a->k) + static_cast<long>(l) * B * Hkv * D * 2;
+      if (launch_neuron_rope(v, 1, v.pos + static_cast<long>(layer0 + l) * B, ql, kl,
+                             neuron ? a->decide->offset + l * ostride_layer : nullptr,
+                             neuron ? a->decide->offset_batch_stride : 0, neuron, a->alpha + static_cast<long>(l) * B * Hkv,
+                             a->rope_cos, a->rope_sin, s) != cudaSuccess)
+        return DMS_ERR_CUDA;
+    }
+  }
+  DecideArgs da{};
+  const bool proj = a->decide && !neuron;
+  if (proj) {
+    da = decide_args(a->decide);
+    da.gamma_lstride = c->desc.hidden;
+    da.w_lstride = static_cast<long>(Hkv) * c->desc.hidden;
+    da.bias_lstride = Hkv;
+    da.offset_lstride = ostride_layer;
+  }
+  // every layer of the range in one launch (early reads only after the wait)
+  track_launch(c, -1, s);
+  if (launch_decode_cluster(v, layer0, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, &c->kmap,
+                            &c->vmap, c->num_sms, s, false, num_layers) != cudaSuccess)
+    return DMS_ERR_CUDA;
+  for (int l = layer0; l < layer0 + num_layers; ++l) {
+    c->decoded[l] = 1;
+    c->positions[l] += 1;
+  }
+  c->worklist_layer = -1;
   return DMS_OK;
 }
 

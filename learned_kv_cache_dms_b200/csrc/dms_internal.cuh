@@ -25,7 +25,7 @@ enum Ctrl {
 // Device view of one cache: sizes and device pointers into the caller buffer.
 struct CacheView {
   int L, B, Hq, Hkv, D, hidden, w, P, maxp, cap, pool_pages, pre_pages, max_pos;
-  int kv_dtype, act_dtype, alpha_per, alpha_source, disable, decode_kernel;
+  int kv_dtype, act_dtype, alpha_per, alpha_source, disable, decode_kernel, shift;
   float alpha_scale, rms_eps;
   int num_sms;
   int* ctrl;
@@ -35,6 +35,7 @@ struct CacheView {
   int* page_table;  // [L,B,Hkv,maxp]
   int* slot_pos;    // [L,B,Hkv,cap]
   int* ring;        // [L,B,Hkv,w]
+  int* carry;       // [L,B,Hkv] decision shift +1: the newest token's own decision
   int4* plan;       // [2][L,B,Hkv] plan of the next append, by parity of its position (next_plan)
   int* kept;        // [B,Hkv,max_pos]   prefill scratch: kept positions, ascending
   int* kept_count;  // [B,Hkv]
@@ -55,6 +56,27 @@ struct CacheView {
 
 constexpr unsigned RING_EVICT = 0x80000000u;
 constexpr int RING_SLOT_MASK = 0x7FFFFFFF;
+
+// The eviction mark stored with token t, appended with its own decision `dec`
+// (logit > 0, eviction enabled), under the cache's decision shift: 0, its own
+// decision; +1, the previous token's (carried per head); -1, unmarked until the
+// next token, and `dec` marks token t - 1 in its ring entry now.  Called by the
+// one thread that appends to head li.
+__device__ __forceinline__ bool shifted_mark(const CacheView& c, long li, int t, bool dec) {
+  if (c.shift == 1) {
+    const bool m = c.carry[li] != 0;
+    c.carry[li] = dec ? 1 : 0;
+    return m;
+  }
+  if (c.shift == -1) {
+    if (t >= 1 && dec) {
+      int* e = c.ring + li * c.w + (t - 1) % c.w;
+      *e = *e | static_cast<int>(RING_EVICT);
+    }
+    return false;
+  }
+  return dec;
+}
 
 // Bounded spin limit for every device-side wait.
 constexpr long long kSpinLimit = 1ll << 26;
@@ -406,6 +428,9 @@ struct DecideArgs {
   const void* bias;
   const float* offset;
   int offset_bstride;
+  // a decode launch over several layers: elements from one layer's gamma, W,
+  // bias and offsets to the next (hidden rows continue layer by layer)
+  long gamma_lstride, w_lstride, bias_lstride, offset_lstride;
 };
 
 cudaError_t launch_init(const CacheView& c, bool full, cudaStream_t s);
@@ -420,7 +445,7 @@ cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, vo
 // a chunked prefill; launch_prefill_context rebuilds the kept list, kept copy
 // and window copy of the layer first).
 size_t prefill_scan_smem(const CacheView& c, int T0, int T);
-cudaError_t launch_prefill_context(const CacheView& c, int layer, int T0, cudaStream_t s);
+cudaError_t launch_prefill_context(const CacheView& c, int layer, int T0, int T, const float* alpha, cudaStream_t s);
 cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T0, int T, const float* alpha, cudaStream_t s);
 cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T0, int T, const void* k, const void* v,
                                    cudaStream_t s);
@@ -449,8 +474,11 @@ cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q
 cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
                                const CUtensorMap* vmap, cudaStream_t s, bool early, bool* taken);
+// One cluster per (layer, b, h) of layers [layer, layer + nl): with nl > 1
+// every input and output array holds the nl layers back to back (rows
+// layer-major), and the fused step appends to all of them in one launch.
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
-                                  const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early);
+                                  const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early, int nl = 1);
 
 }  // namespace dms

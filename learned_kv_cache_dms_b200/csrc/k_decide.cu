@@ -22,6 +22,7 @@ __global__ void k_init(CacheView c) {
     if (i < nbh) {
       c.npages[i] = c.pre_pages;
       c.count[i] = 0;
+      c.carry[i] = 0;
       c.plan[i] = make_int4(0, 0, 0, 0);
       c.plan[nbh + i] = make_int4(0, 0, 0, 0);
     }

@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, i
       }
       if (!(flags & 1)) c.count[li] = cnt_new;
       const float a = fuse_decide ? a_dec : alpha[b * c.Hkv + hs];
-      const bool evict = !c.disable && a > 0.0f;
+      const bool evict = shifted_mark(c, li, t, !c.disable && a > 0.0f);
       c.slot_pos[li * c.cap + slot] = t;
       c.ring[li * w + t % w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
     } else {

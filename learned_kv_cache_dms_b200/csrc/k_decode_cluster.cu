@@ -63,10 +63,10 @@ struct SubMeta {
 };
 
 template <int D, bool FP8, bool FUSED>
-__global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int layer, int early, const __nv_bfloat16* q,
-                                                            __nv_bfloat16* o, int cs, const __nv_bfloat16* k_new,
-                                                            const __nv_bfloat16* v_new, float* alpha, DecideArgs da,
-                                                            int fuse_decide,
+__global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int layer, int nl, int early,
+                                                            const __nv_bfloat16* q, __nv_bfloat16* o, int cs,
+                                                            const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                                                            float* alpha, DecideArgs da, int fuse_decide,
                                                             const __grid_constant__ CUtensorMap kmap,
                                                             const __grid_constant__ CUtensorMap vmap) {
   using S = DecodeSmem<D, FP8>;
@@ -91,11 +91,14 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   __shared__ int s_pt[kPtCache];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x / cs;
+  // head vh of the launch: (layer + lrel, b, h); the inputs of a multi-layer
+  // launch hold its layers back to back, so their row is bb = lrel * B + b
+  const int vh = blockIdx.x / cs, BH = c.B * c.Hkv;
+  const int lrel = vh / BH, bh = vh % BH;
   const int rank = static_cast<int>(cluster_rank());
   const int owner = cs - 1;  // the rank that appends: its slice of the slots is the shortest
-  const int b = bh / c.Hkv, h = bh % c.Hkv;
-  const long li = static_cast<long>(layer) * c.B * c.Hkv + bh;
+  const int b = bh / c.Hkv, h = bh % c.Hkv, bb = vh / c.Hkv;
+  const long li = static_cast<long>(layer) * BH + vh;
   // Programmatic dependent launch.  With `early` (the previous launch of this
   // library on the stream was for another layer or cache) this layer's state
   // is read and the first tiles are requested before waiting for the previous
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   // the head's page-table row is fetched together with the count (no dependent round trip)
   for (int i = tid; i < min(c.maxp, kPtCache); i += kThreads) s_pt[i] = c.page_table[li * c.maxp + i];
   const int cnt = c.count[li];
-  const int t = FUSED ? c.pos[layer * c.B + b] : 0;
+  const int t = FUSED ? c.pos[layer * c.B + bb] : 0;
   const int4 pl = FUSED ? *plan_at(c, li, t) : make_int4(0, 0, 0, 0);
   const int masked_slot = (FUSED && (pl.y & 1)) ? pl.x : -1;
   // ranks 0 .. cs-2 take `per` slots each, the owner the rest: a quarter share
@@ -155,14 +158,14 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   }
   const int next_page0 = FUSED ? c.ctrl[CTRL_NEXT_PAGE] : 0;
   uint32_t qa[KS][4];
-  const __nv_bfloat16* qb = q + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D;
+  const __nv_bfloat16* qb = q + (static_cast<long>(bb) * c.Hq + static_cast<long>(h) * g) * D;
   load_q_frags<D>(qb, g, qa);
   if (FUSED && rank == owner) {
     // everything the append needs, fetched while the first tiles are in flight:
     // the new key/value row, the new token's scores, the ring entry of t + 1
     if (tid < D / 8) {
-      reinterpret_cast<uint4*>(s_knew)[tid] = reinterpret_cast<const uint4*>(k_new + static_cast<long>(bh) * D)[tid];
-      reinterpret_cast<uint4*>(s_vnew)[tid] = reinterpret_cast<const uint4*>(v_new + static_cast<long>(bh) * D)[tid];
+      reinterpret_cast<uint4*>(s_knew)[tid] = reinterpret_cast<const uint4*>(k_new + static_cast<long>(vh) * D)[tid];
+      reinterpret_cast<uint4*>(s_vnew)[tid] = reinterpret_cast<const uint4*>(v_new + static_cast<long>(vh) * D)[tid];
     }
     if (tid == 32) s_ring_next = (t + 1 >= c.w) ? c.ring[li * c.w + (t + 1) % c.w] : 0;
     __syncthreads();
@@ -183,10 +186,19 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   if (FUSED && rank == owner && fuse_decide) {
     // decision logit of the new token (layer granularity: head 0's)
     const int src = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
-    const float a = decide_cta<4>(c, da, b, src, s_fred);
+    // this layer's adapter (hidden rows of the layer, its weights and offsets)
+    DecideArgs dl = da;
+    if (lrel > 0) {
+      dl.hidden = static_cast<const __nv_bfloat16*>(da.hidden) + static_cast<long>(lrel) * c.B * c.hidden;
+      dl.gamma = static_cast<const __nv_bfloat16*>(da.gamma) + lrel * da.gamma_lstride;
+      dl.W = static_cast<const __nv_bfloat16*>(da.W) + lrel * da.w_lstride;
+      if (da.bias) dl.bias = static_cast<const __nv_bfloat16*>(da.bias) + lrel * da.bias_lstride;
+      dl.offset = da.offset + lrel * da.offset_lstride;
+    }
+    const float a = decide_cta<4>(c, dl, b, src, s_fred);
     if (tid == 0) {
       s_alpha = a;
-      alpha[b * c.Hkv + h] = a;
+      alpha[bb * c.Hkv + h] = a;
     }
   }
 
@@ -297,8 +309,8 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     if (ok && (flags & 2)) {
       // a new page: numbered by this head's rank among the heads that need one
       int n_before = 0;
-      for (int i = lane; i < bh; i += 32)
-        n_before += (plan_at(c, static_cast<long>(layer) * c.B * c.Hkv + i, t)->y & 2) ? 1 : 0;
+      for (int i = lane; i < vh; i += 32)
+        n_before += (plan_at(c, static_cast<long>(layer) * BH + i, t)->y & 2) ? 1 : 0;
       n_before = __reduce_add_sync(0xffffffffu, n_before);
       id = next_page0 + n_before;
       if (id >= c.pool_pages || pl.w >= c.maxp) ok = false;
@@ -323,8 +335,8 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
           c.npages[li] = np_new;
         }
         const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
-        const float a = fuse_decide ? s_alpha : __ldcg(&alpha[b * c.Hkv + hs]);
-        const bool evict = !c.disable && a > 0.0f;
+        const float a = fuse_decide ? s_alpha : __ldcg(&alpha[bb * c.Hkv + hs]);
+        const bool evict = shifted_mark(c, li, t, !c.disable && a > 0.0f);
         c.slot_pos[li * c.cap + slot] = t;
         c.ring[li * c.w + t % c.w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
         if (!(flags & 1)) c.count[li] = cnt_new;
@@ -340,7 +352,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
       // counter and the positions before its partial landed here)
       last = count_step(c, ok && (flags & 2) ? 1 : 0, static_cast<int>(gridDim.x) / cs, next_page0) ? 1 : 0;
     }
-    if (__shfl_sync(0xffffffffu, last, 0)) advance_positions(c, layer, lane, 32);
+    if (__shfl_sync(0xffffffffu, last, 0)) advance_positions(c, layer, lane, 32, nl);
     return;
   }
 
@@ -369,7 +381,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     constexpr int kMergeThreads = FUSED ? kThreads - 32 : kThreads;
     asm volatile("bar.sync 1, %0;\n" ::"n"(kMergeThreads) : "memory");
     // four consecutive elements of one row per thread and pass
-    __nv_bfloat16* ob = o + (static_cast<long>(b) * c.Hq + static_cast<long>(h) * g) * D;
+    __nv_bfloat16* ob = o + (static_cast<long>(bb) * c.Hq + static_cast<long>(h) * g) * D;
     const bool vec_out = (reinterpret_cast<uintptr_t>(ob) & 7) == 0;
     for (int e4 = tid; e4 < g * (D / 4); e4 += kMergeThreads) {
       const int r = e4 / (D / 4), d = 4 * (e4 % (D / 4));
@@ -448,12 +460,12 @@ static int pick_cluster(int heads, int g, int num_sms) {
 template <int D, bool FP8, bool FUSED>
 static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q, void* o, const void* k,
                                    const void* v, float* alpha, const DecideArgs* da, const CUtensorMap* kmap,
-                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early) {
+                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early, int nl) {
   const int g = c.Hq / c.Hkv;
   auto kern = k_decode_cluster<D, FP8, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
-  const int heads = c.B * c.Hkv;
+  const int heads = nl * c.B * c.Hkv;
   const int cs = pick_cluster<D, FP8, FUSED>(heads, g, num_sms);
   const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -473,25 +485,31 @@ static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   DecideArgs none{};
-  return cudaLaunchKernelEx(&cfg, kern, c, layer, early ? 1 : 0, static_cast<const __nv_bfloat16*>(q),
+  return cudaLaunchKernelEx(&cfg, kern, c, layer, nl, early ? 1 : 0, static_cast<const __nv_bfloat16*>(q),
                             static_cast<__nv_bfloat16*>(o), cs, static_cast<const __nv_bfloat16*>(k),
                             static_cast<const __nv_bfloat16*>(v), alpha, da ? *da : none, da ? 1 : 0, *kmap, *vmap);
 }
 
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
-                                  const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early) {
-  if (!kmap || !vmap || c.kv_dtype == DMS_F32) return cudaErrorInvalidValue;
+                                  const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early, int nl) {
+  if (!kmap || !vmap || c.kv_dtype == DMS_F32 || nl < 1) return cudaErrorInvalidValue;
   if (fused) {
     if (c.kv_dtype != DMS_BF16) return cudaErrorInvalidValue;
-    return c.D == 64 ? launch_cluster_t<64, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s, early)
-                     : launch_cluster_t<128, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s, early);
+    return c.D == 64 ? launch_cluster_t<64, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms,
+                                                         s, early, nl)
+                     : launch_cluster_t<128, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap,
+                                                          num_sms, s, early, nl);
   }
   if (c.kv_dtype == DMS_FP8_E4M3)
-    return c.D == 64 ? launch_cluster_t<64, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early)
-                     : launch_cluster_t<128, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early);
-  return c.D == 64 ? launch_cluster_t<64, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early)
-                   : launch_cluster_t<128, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early);
+    return c.D == 64 ? launch_cluster_t<64, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s,
+                                                         early, nl)
+                     : launch_cluster_t<128, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s,
+                                                          early, nl);
+  return c.D == 64 ? launch_cluster_t<64, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s,
+                                                        early, nl)
+                   : launch_cluster_t<128, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s,
+                                                         early, nl);
 }
 
 }  // namespace dms

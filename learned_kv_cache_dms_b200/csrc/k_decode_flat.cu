@@ -804,7 +804,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
               }
               const int hs = (fuse_decide || c.alpha_per != DMS_ALPHA_PER_LAYER) ? h : 0;
               const float av = s_alpha[k] == s_alpha[k] ? s_alpha[k] : __ldcg(&alpha[b * c.Hkv + hs]);
-              const bool evict = !c.disable && av > 0.0f;
+              const bool evict = shifted_mark(c, li, t, !c.disable && av > 0.0f);
               c.slot_pos[li * c.cap + slot] = t;
               c.ring[li * c.w + t % c.w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
               if (!(flags & 1)) c.count[li] = cnt_new;

@@ -50,6 +50,9 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
   const int w = c.w;
   const int end = T0 + T;  // positions held after this call
   int* ring = c.ring + lbh * w;
+  // decision shift +1: the mark of the call's first token is the previous
+  // token's decision, carried from the previous call (0: the padding, keep)
+  const bool carry_in = c.shift == 1 && T0 > 0 && c.carry[lbh] != 0;
 
   if (T0 > 0) {
     for (int i = tid; i < w; i += bd) rs[i] = ring[i];
@@ -66,14 +69,16 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
 
   // 1. evict bits (coalesced read, one ballot per 32 tokens).  Warp wid owns
   //    words wid, wid + nwarp, ...; it issues the loads of kScanU words before
-  //    the first ballot so that they are in flight together.
+  //    the first ballot so that they are in flight together.  Token t's mark
+  //    is the decision of token t - shift: +1 the previous token's (the
+  //    carried one for t = 0), -1 the next token's (none yet for the last).
   const int wid = tid >> 5, nwarp = bd >> 5;
   for (int w0 = wid; w0 < nw; w0 += nwarp * kScanU) {
     bool e[kScanU];
 #pragma unroll
     for (int u = 0; u < kScanU; ++u) {
-      const int t = (w0 + u * nwarp) * 32 + lane;
-      e[u] = t < T && arow[t] > 0.0f;
+      const int t = (w0 + u * nwarp) * 32 + lane, src = t - c.shift;
+      e[u] = t < T && (src >= 0 && src < T ? arow[src] > 0.0f : (src < 0 && carry_in));
     }
 #pragma unroll
     for (int u = 0; u < kScanU; ++u) {
@@ -141,6 +146,7 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
     kept_upto[end] = kept0 + tot_keep;
     c.count[lbh] = count0 + tot_open;
     c.kept_count[bh] = kept0 + tot_keep;
+    if (c.shift == 1) c.carry[lbh] = (!c.disable && arow[T - 1] > 0.0f) ? 1 : 0;
     if (h == 0) c.pos[layer * c.B + b] = end;
   }
   // 5. the last CTA to arrive grants the extra pages of every head, in (b, h)
@@ -235,7 +241,7 @@ __device__ __forceinline__ uint4 page_row_chunk(const CacheView& c, const void* 
 }
 
 template <bool FP8>
-__global__ void __launch_bounds__(1024) k_prefill_context(CacheView c, int layer, int T0) {
+__global__ void __launch_bounds__(1024) k_prefill_context(CacheView c, int layer, int T0, int T, const float* alpha) {
   __shared__ int tmp[32];
   const int bh = blockIdx.x, tid = threadIdx.x, bd = blockDim.x, w = c.w;
   const long lbh = static_cast<long>(layer) * c.B * c.Hkv + bh;
@@ -243,8 +249,15 @@ __global__ void __launch_bounds__(1024) k_prefill_context(CacheView c, int layer
   int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
   int* kept = c.kept + static_cast<long>(bh) * c.max_pos;
   const int* slot_pos = c.slot_pos + lbh * c.cap;
-  const int* ring = c.ring + lbh * w;
+  int* ring = c.ring + lbh * w;
   const int* pt = c.page_table + lbh * c.maxp;
+  // decision shift -1: the call's first decision marks the layer's last token
+  if (c.shift == -1 && tid == 0) {
+    const int b = bh / c.Hkv, hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : bh % c.Hkv;
+    if (!c.disable && alpha[(static_cast<long>(b) * c.Hkv + hs) * T] > 0.0f)
+      ring[(T0 - 1) % w] |= static_cast<int>(RING_EVICT);
+  }
+  __syncthreads();
   auto is_kept = [&](int j) { return j < T0 - w || (ring[j % w] & static_cast<int>(RING_EVICT)) == 0; };
   // 1. flags at the kept positions, then an exclusive scan in place
   for (int x = tid; x <= T0; x += bd) kept_upto[x] = 0;
@@ -300,11 +313,11 @@ __global__ void __launch_bounds__(1024) k_prefill_context(CacheView c, int layer
   }
 }
 
-cudaError_t launch_prefill_context(const CacheView& c, int layer, int T0, cudaStream_t s) {
+cudaError_t launch_prefill_context(const CacheView& c, int layer, int T0, int T, const float* alpha, cudaStream_t s) {
   if (c.kv_dtype == DMS_FP8_E4M3)
-    k_prefill_context<true><<<c.B * c.Hkv, 1024, 0, s>>>(c, layer, T0);
+    k_prefill_context<true><<<c.B * c.Hkv, 1024, 0, s>>>(c, layer, T0, T, alpha);
   else
-    k_prefill_context<false><<<c.B * c.Hkv, 1024, 0, s>>>(c, layer, T0);
+    k_prefill_context<false><<<c.B * c.Hkv, 1024, 0, s>>>(c, layer, T0, T, alpha);
   return cudaGetLastError();
 }
 

@@ -48,6 +48,7 @@ class Case:
     staged: bool = False          # decode through dms_decode_append + dms_decode_attention
     kernel: str = "auto"          # decode attention kernel: auto | cluster | flat
     chunks: tuple | None = None   # chunked prefill: the prompt's chunk sizes (summing to T)
+    shift: int = 0                # decision shift: 0 own, +1 previous token's, -1 next token's decision
 
     @property
     def N(self):
@@ -142,17 +143,19 @@ def build(case: Case):
         rows[: min(B, case.attn_rows), 2] = T - 1  # always include the last rows
         out["rows"] = rows
     cache = O.Cache(case.layers, B, case.Hkv, case.D, case.w, case.P, N, case.pool, case.prealloc,
-                    fp8=case.kv == "fp8")
-    if case.chunks is None:
+                    fp8=case.kv == "fp8", shift=case.shift)
+    if case.chunks is None and case.shift == 0:
         out["o_prefill"] = O.prefill_attention(qs[:, :T], ks[:, :T], vs[:, :T],
                                                np.ascontiguousarray(evict[:, :, :T]), case.w, rows=rows)
         cache.prefill(case.layer, np.ascontiguousarray(evict[:, :, :T]), ks[:, :T].astype(np.float32),
                       vs[:, :T].astype(np.float32))
     else:
-        # each chunk attends to the cache as the earlier chunks left it, then is appended
-        assert sum(case.chunks) == T
+        # each chunk attends to the cache as the earlier chunks left it, then is
+        # appended (a shifted-decision prompt in one call goes the same way)
+        chunks = case.chunks or (T,)
+        assert sum(chunks) == T
         outs, t0 = [], 0
-        for n in case.chunks:
+        for n in chunks:
             sl = slice(t0, t0 + n)
             ev_c = np.ascontiguousarray(evict[:, :, sl])
             r_c = None
@@ -186,6 +189,20 @@ def build(case: Case):
     return out
 
 
+def marks(evict, shift):
+    """Eviction marks of the tokens from their own decisions under a decision
+    shift (+1: the previous token's decision, the first token keeps; -1: the
+    next token's, the last token not yet marked)."""
+    out = np.zeros_like(evict)
+    if shift == 1:
+        out[..., 1:] = evict[..., :-1]
+    elif shift == -1:
+        out[..., :-1] = evict[..., 1:]
+    else:
+        out[:] = evict
+    return out
+
+
 def make_desc(B_, case: Case):
     d = B_.dms_cache_desc_default()
     d.num_layers, d.batch, d.num_q_heads, d.num_kv_heads = case.layers, case.B, case.Hq, case.Hkv
@@ -200,6 +217,7 @@ def make_desc(B_, case: Case):
         d.hidden = max(d.hidden, 8)
     d.alpha_scale, d.rms_eps = ALPHA_SCALE, RMS_EPS
     d.disable_eviction = int(case.disable)
+    d.decision_shift = case.shift
     d.decode_kernel = {"auto": B_.DMS_DECODE_AUTO, "cluster": B_.DMS_DECODE_CLUSTER,
                        "flat": B_.DMS_DECODE_FLAT}[case.kernel]
     return d

@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from harness import Case, build, check_case, compare_pages, compare_state, make_desc, run_gpu
+from harness import Case, build, check_case, marks, compare_pages, compare_state, make_desc, run_gpu
 
 CASES = {
     # three ragged chunks, each spanning several 64-key tiles
@@ -29,6 +29,12 @@ CASES = {
     # FP8 pages, key-neuron decisions, rotary tables at the chunks' positions
     "fp8_key_rope_chunks": Case(B=2, T=700, steps=20, Hq=8, Hkv=2, D=64, w=64, P=32, act="bf16", kv="fp8",
                                 source="key", keep=0.125, rope=True, chunks=(250, 250, 200), seed=64),
+    # decision shifts across chunk boundaries: the carried decision (+1) and
+    # the previous chunk's last token marked by the next chunk's first (-1)
+    "bf16_shift_right_chunks": Case(B=2, T=600, steps=10, Hq=8, Hkv=2, D=128, w=64, P=32, act="bf16", kv="bf16",
+                                    source="input", keep=0.3, chunks=(200, 1, 399), shift=1, seed=68),
+    "bf16_shift_left_chunks": Case(B=2, T=600, steps=10, Hq=8, Hkv=2, D=64, hidden=256, w=64, P=32, act="bf16",
+                                   kv="bf16", source="proj", keep=0.3, chunks=(150, 250, 200), shift=-1, seed=69),
     # per-layer decisions and the query neuron over two chunks
     "bf16_query_layer_chunks": Case(B=1, T=520, steps=6, Hq=8, Hkv=2, D=128, w=96, P=32, act="bf16", kv="bf16",
                                     source="query", per="layer", keep=0.2, chunks=(256, 264), seed=65),
@@ -49,7 +55,7 @@ def test_chunked_case_builds(name):
     if name in FULL:
         pytest.skip("full-size oracle replay runs with the GPU test")
     ins = build(case)
-    ev, T, w = ins["evict"], case.T, case.w
+    ev, T, w = marks(ins["evict"][:, :, :case.T], case.shift), case.T, case.w
     expect = min(T, w) + (1 - ev[:, :, : max(0, T - w)]).sum(-1)
     assert np.array_equal(ins["state_prefill"]["count"], expect)
 

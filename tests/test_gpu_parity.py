@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-from harness import Case, build, check_case
+from harness import Case, build, check_case, marks
 
 CASES = {
     # the tiny fp32 workload: B1, hidden 256, 4/2 heads, D64, 256 + 16 tokens, w32, P16, keep 1/2
@@ -71,6 +71,18 @@ CASES = {
                                 source="input", keep=0.3, seed=51),
     "bf16_g6_d64_proj_mma_prefill": Case(B=1, T=380, steps=10, Hq=12, Hkv=2, D=64, hidden=256, w=48, P=16,
                                          act="bf16", kv="bf16", source="proj", keep=0.25, seed=52),
+    # decision shifts: +1 (token t marked by token t-1's decision) with the
+    # adapter, -1 (token t's decision marks token t-1) on FP8 pages with the
+    # key neuron and rotary tables, +1 on fp32 pages
+    "bf16_shift_right_proj": Case(B=2, T=515, steps=24, Hq=8, Hkv=4, D=128, hidden=512, w=96, P=32, act="bf16",
+                                  kv="bf16", source="proj", keep=(1 / 16, 1 / 4), shift=1, seed=71),
+    "fp8_shift_left_key_rope": Case(B=2, T=700, steps=30, Hq=8, Hkv=2, D=64, w=64, P=32, act="bf16", kv="fp8",
+                                    source="key", keep=0.125, rope=True, shift=-1, seed=72),
+    "f32_shift_right_input": Case(B=1, T=256, steps=16, Hq=4, Hkv=2, D=64, w=32, P=16, act="f32", kv="f32",
+                                  source="input", keep=0.5, shift=1, seed=73),
+    "bf16_shift_left_layer_b8": Case(B=8, T=300, steps=40, Hq=16, Hkv=8, D=128, hidden=256, w=64, P=32,
+                                     act="bf16", kv="bf16", source="proj", per="layer", keep=(1 / 16, 1 / 4),
+                                     prealloc=96, shift=-1, seed=74),
     # second layer of a two-layer cache with preallocation
     "layer1_of_2": Case(B=2, T=260, steps=12, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16",
                         source="input", keep=0.3, layers=2, layer=1, prealloc=64, seed=15),
@@ -83,7 +95,7 @@ def test_case_inputs_and_oracle(name):
     the oracle's own invariants hold (retained count)."""
     case = CASES[name]
     ins = build(case)
-    ev = ins["evict"]
+    ev = marks(ins["evict"][:, :, :case.T], case.shift)
     T, w = case.T, case.w
     cnt = ins["state_prefill"]["count"]
     expect = min(T, w) + (1 - ev[:, :, : max(0, T - w)]).sum(-1)
