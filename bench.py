@@ -75,6 +75,9 @@ def parse():
     p.add_argument("--decode-steps", type=int, default=None, help="decode only the first N steps")
     p.add_argument("--decode-kernel", choices=["auto", "cluster", "flat"], default="auto",
                    help="decode attention kernel (auto: by the number of heads)")
+    p.add_argument("--decode-api", choices=["auto", "step", "layers"], default="auto",
+                   help="multi-layer stacks: one dms_decode_step_layers launch per step (auto, layers) or one "
+                        "dms_decode_step per layer (step)")
     p.add_argument("--replicas", type=int, default=None,
                    help="cache replicas per step (default: enough that each step's KV is >= 4x L2; 1 gives a "
                         "small case for profiler captures, whose numbers are then not L2-cold)")
@@ -216,10 +219,12 @@ def decode_launches_per_step(wl):
     return pre + 1      # one fused kernel: decision, attention, combine, append
 
 
-def kernel_launches_per_step(wl, n_dec):
+def kernel_launches_per_step(wl, n_dec, stacked=False):
     # reset (1) + per layer: compaction (decide or neuron/rotary pass, scan,
-    # scatter) + prefill attention (1) + the decode steps
-    return 1 + wl.layers * (3 + 1) + wl.layers * n_dec * decode_launches_per_step(wl)
+    # scatter) + prefill attention (1) + the decode steps (one launch for the
+    # whole stack with dms_decode_step_layers)
+    per_step = 1 if stacked else wl.layers * decode_launches_per_step(wl)
+    return 1 + wl.layers * (3 + 1) + n_dec * per_step
 
 
 def decode_kernel_name(wl, choice, num_sms):
@@ -280,7 +285,7 @@ class Runner:
     (each holding every layer), and the decode steps captured as CUDA graphs
     that run every (replica, layer) back to back."""
 
-    def __init__(self, B_, wl, seed, n_dec=None, kernel="auto", replicas=None):
+    def __init__(self, B_, wl, seed, n_dec=None, kernel="auto", replicas=None, api="auto"):
         self.B_, self.wl = B_, wl
         self.S = n_dec or wl.decode_steps
         self.L = wl.layers
@@ -311,6 +316,51 @@ class Runner:
         self.od = self.units[0]["od"]
         self.graphs = None
         self.cycled = self.pool < self.S
+        # a stack of bf16 layers decodes all its layers in one launch
+        # (dms_decode_step_layers) unless asked otherwise
+        self.stacked = (api in ("auto", "layers") and self.L > 1 and wl.kv_dtype == "bf16" and not self.inplace)
+        if self.stacked:
+            self._stack_inputs()
+
+    def _stack_inputs(self):
+        """Decode inputs of every layer stacked layer by layer ([pool, L, B, ...])
+        and one dms_decode_step_layers argument set per (replica, token)."""
+        B_, wl, P = self.B_, self.wl, self.pool
+        st = {k_: torch.stack([x[k_] for x in self.lay], 1).contiguous() for k_ in ("qd", "kd", "vd")}
+        proj = not self.neuron
+        if proj:
+            st["hd"] = torch.stack([x["hd"] for x in self.lay], 1).contiguous()
+            st["gamma"] = torch.stack([x["gamma"] for x in self.lay]).contiguous()
+            st["W"] = torch.stack([x["W"] for x in self.lay]).contiguous()
+            st["off"] = torch.stack([x["off"] for x in self.lay]).contiguous()  # [L, B, Hkv]
+        self.st = st
+        self.sargs = []
+        for r in range(self.R):
+            ad = torch.empty(P, self.L, wl.batch, wl.kv_heads, dtype=torch.float32, device="cuda")
+            od = torch.empty_like(st["qd"])
+            args, keep = [], []
+            for i in range(P):
+                dp = None
+                if proj:
+                    dp = B_.decide_params(st["off"][0], hidden=st["hd"][i], norm_weight=st["gamma"], proj_weight=st["W"])
+                    dp.offset = st["off"].data_ptr()
+                    keep.append(dp)
+                args.append(B_.Cache.decode_args(st["qd"][i], st["kd"][i], st["vd"][i], od[i], ad[i], dp))
+            self.sargs.append(dict(h=self.caches[r].handle, args=args, ad=ad, od=od, keep=keep))
+        self.od = self.sargs[0]["od"][:, 0]
+
+    def decode_replica(self, r, i):
+        """Decode step i of replica r: every layer."""
+        if self.stacked:
+            sa = self.sargs[r]
+            self.B_.dms_decode_step_layers(sa["h"], 0, self.L, sa["args"][i])
+        else:
+            for u in self.units[r * self.L:(r + 1) * self.L]:
+                self.B_.dms_decode_step(u["h"], u["l"], u["dargs"][i])
+
+    def decode_all(self, i):
+        for r in range(self.R):
+            self.decode_replica(r, i)
 
     def _layer(self, l, seed):
         B_, wl = self.B_, self.wl
@@ -409,8 +459,7 @@ class Runner:
                   torch.cuda.Event(enable_timing=True, external=True))
             with torch.cuda.graph(ga, stream=side):
                 ev[0].record()
-                for u in self.units:
-                    B_.dms_decode_step(u["h"], u["l"], u["dargs"][i])
+                self.decode_all(i)
                 ev[1].record()
             gs.append((ga, ev))
         torch.cuda.synchronize()
@@ -445,8 +494,7 @@ class Runner:
             else:
                 a, c = E(enable_timing=True), E(enable_timing=True)
                 a.record()
-                for u in self.units:
-                    B_.dms_decode_step(u["h"], u["l"], u["dargs"][i])
+                self.decode_all(i)
                 c.record()
                 dec.append((a, c))
             if counts is not None:
@@ -572,8 +620,7 @@ def measure_single_step(B_, r, steps=32):
               torch.cuda.Event(enable_timing=True, external=True))
         with torch.cuda.graph(ga, stream=side):
             ev[0].record()
-            for u in units:
-                B_.dms_decode_step(u["h"], u["l"], u["dargs"][i % r.pool])
+            r.decode_replica(0, i % r.pool)
             ev[1].record()
         graphs.append((ga, ev))
     torch.cuda.synchronize()
@@ -600,7 +647,8 @@ def run_ours(args, world, rank, local, primary=True):
     from learned_kv_cache_dms_b200 import binding as B_
     wl = I.WORKLOADS[args.workload]
     pk, pk_kind = peaks()
-    r = Runner(B_, wl, seed=wl.seed + rank, n_dec=args.decode_steps, kernel=args.decode_kernel, replicas=args.replicas)
+    r = Runner(B_, wl, seed=wl.seed + rank, n_dec=args.decode_steps, kernel=args.decode_kernel, replicas=args.replicas,
+               api=args.decode_api)
     S, L = r.S, r.L
     # untimed pass: retained counts after the prefill and after each append
     counts = []
@@ -688,16 +736,19 @@ def run_ours(args, world, rank, local, primary=True):
     cpu = None
     if primary and rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, args.cpu_seconds)
-    kern = decode_kernel_name(wl, args.decode_kernel, torch.cuda.get_device_properties(0).multi_processor_count)
+    kern = ("k_decode_cluster" if r.stacked else
+            decode_kernel_name(wl, args.decode_kernel, torch.cuda.get_device_properties(0).multi_processor_count))
     kname = ("decode step: %s<%d,%s> (split-K attention, %s%s)%s"
              % (kern, wl.head_dim, wl.kv_dtype,
                 "on-chip combine" if kern == "k_decode_cluster" else "partials merged by the last CTA of a head",
                 ", append, decision logit" if wl.kv_dtype == "bf16" else "",
                 " after k_decode_append" if wl.kv_dtype == "fp8" else ""))
+    if r.stacked:
+        kname += ", all %d layers in one launch (dms_decode_step_layers)" % L
     traffic = recorded_traffic(kern, workload_label(wl, S)) if args.replicas is None else None
     roof = {"bound": "hbm", "achieved": round(decode_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(decode_gbs / pk["hbm_gbs"], 4), "traffic": traffic, "kernel": kname,
-            "algorithmic_bytes_per_launch": int(attn_bytes / (S * L)), "peak_source": pk_kind}
+            "algorithmic_bytes_per_launch": int(attn_bytes / (S * (1 if r.stacked else L))), "peak_source": pk_kind}
     retained_first = counts[0] / (L * B * wl.kv_heads)
     retained_last = counts[-1] / (L * B * wl.kv_heads)
     cfg = {"workload": workload_label(wl, S), "layers": L, "batch": B, "prompt": wl.prompt, "decode_steps": S,
@@ -710,7 +761,8 @@ def run_ours(args, world, rank, local, primary=True):
                   "KV per step, >= 4x L2), so no replica's KV is in L2 when it is read; no flush"
                   % (R, R * step_bytes[0] / 1e6)),
            "replicas": R,
-           "parallelism": "dp%d replicas" % world, "decode_kernel": args.decode_kernel}
+           "parallelism": "dp%d replicas" % world, "decode_kernel": args.decode_kernel,
+           "decode_api": "dms_decode_step_layers" if r.stacked else "dms_decode_step"}
     if r.cycled:
         cfg["decode_inputs"] = "%d distinct token inputs per layer, cycled" % r.pool
     line = {
@@ -739,7 +791,7 @@ def run_ours(args, world, rank, local, primary=True):
         "compaction": compact_roof,
         "achieved_cr": round(wl.max_positions / retained_last, 3) if S == wl.decode_steps else None,
         "region_ms_per_step": round(region_ms / K, 3),
-        "roofline": roof, "e2e": e2e, "gpu_launches": kernel_launches_per_step(wl, S) * K * R,
+        "roofline": roof, "e2e": e2e, "gpu_launches": kernel_launches_per_step(wl, S, r.stacked) * K * R,
         "clocks": clocks, "cpu_baseline": cpu,
     }
     return line
