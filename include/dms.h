@@ -77,9 +77,18 @@ enum dms_dtype { DMS_F32 = 0, DMS_BF16 = 1, DMS_FP8_E4M3 = 2 };
 /* [DMS-Qwen3] "驱逐决策的两种来源与两种粒度": dms_alpha_per is head or layer. */
 enum dms_alpha_per { DMS_ALPHA_PER_HEAD = 0, DMS_ALPHA_PER_LAYER = 1 };
 /* Source of the decision logit: the separate adapter (RMSNorm + Linear over the
- * pre-attention hidden state, dms_separate_alpha=True), or the last neuron of
- * each key / of the first query head of each GQA group (separate_alpha=False). */
-enum dms_alpha_source { DMS_ALPHA_PROJ = 0, DMS_ALPHA_KEY_NEURON = 1, DMS_ALPHA_QUERY_NEURON = 2 };
+ * pre-attention hidden state, dms_separate_alpha=True), the last neuron of
+ * each key / of the first query head of each GQA group (separate_alpha=False),
+ * or an importance score (the KVzap-linear page: one Linear from the hidden
+ * state to one score per KV head, no normalisation; a token scoring below the
+ * threshold is pruned, the most recent tokens kept -- the DMS rule with
+ * window = that number of recent tokens, e.g. 128). */
+enum dms_alpha_source {
+  DMS_ALPHA_PROJ = 0,
+  DMS_ALPHA_KEY_NEURON = 1,
+  DMS_ALPHA_QUERY_NEURON = 2,
+  DMS_ALPHA_SCORE_LINEAR = 3
+};
 
 /* Decode attention kernels.  CLUSTER: one thread-block cluster per (b, h),
  * partials combined on chip (lowest latency when B * Hkv is small).  FLAT: one
@@ -169,15 +178,18 @@ typedef struct dms_cache_layout {
  *   *_NEURON: alpha = x[D-1] * alpha_scale - offset[b,h], x the key of head h
  *            (KEY) or the query of head h*g (QUERY); that element is then set
  *            to zero in the caller's k (or q) before the rotary embedding.
+ *   SCORE_LINEAR: alpha[b,h,t] = offset[b,h] - (W_h . h_t + bias_h), the offset
+ *            holding the pruning threshold (-4 on the KVzap page): a token whose
+ *            score is below it is marked; norm_weight is not read.
  *   Layer granularity: every head takes head 0's logit.
  *   [DMS-Qwen3] "Gumbel 噪声与可微门控": at inference a token is evicted iff
  *   alpha > 0 (alpha == 0 keeps), and never when disable_eviction is set. */
 typedef struct dms_decide_params {
   /* PROJ: hidden, norm_weight and proj_weight are read as 16-byte vectors and
    * must be 16-byte aligned (DMS_ERR_INVALID otherwise). */
-  const void* hidden;      /* device [B,T,hidden] (decode: [B,hidden]), act dtype; PROJ only */
-  const void* norm_weight; /* device gamma [hidden], act dtype; PROJ only                 */
-  const void* proj_weight; /* device W [Hkv,hidden], act dtype; PROJ only                 */
+  const void* hidden;      /* device [B,T,hidden] (decode: [B,hidden]), act dtype; PROJ, SCORE_LINEAR */
+  const void* norm_weight; /* device gamma [hidden], act dtype; PROJ only (not read by SCORE_LINEAR) */
+  const void* proj_weight; /* device W [Hkv,hidden], act dtype; PROJ, SCORE_LINEAR        */
   const void* proj_bias;   /* device [Hkv] act dtype, or NULL                             */
   const float* offset;     /* device fp32 offset[b*offset_batch_stride + h]               */
   int offset_batch_stride; /* 0 (one offset per head) or Hkv (per sequence and head)      */

@@ -27,7 +27,7 @@ DMS_OK, DMS_ERR_INVALID, DMS_ERR_STATE, DMS_ERR_CUDA, DMS_ERR_NOMEM, DMS_ERR_SCR
 DMS_ST_POOL_EXHAUSTED, DMS_ST_CAPACITY, DMS_ST_TIMEOUT, DMS_ST_SPLIT_LIMIT = 1, 2, 4, 8
 DMS_F32, DMS_BF16, DMS_FP8_E4M3 = 0, 1, 2
 DMS_ALPHA_PER_HEAD, DMS_ALPHA_PER_LAYER = 0, 1
-DMS_ALPHA_PROJ, DMS_ALPHA_KEY_NEURON, DMS_ALPHA_QUERY_NEURON = 0, 1, 2
+DMS_ALPHA_PROJ, DMS_ALPHA_KEY_NEURON, DMS_ALPHA_QUERY_NEURON, DMS_ALPHA_SCORE_LINEAR = 0, 1, 2, 3
 DMS_DECODE_AUTO, DMS_DECODE_CLUSTER, DMS_DECODE_FLAT = 0, 1, 2
 
 _ERRORS = {DMS_ERR_INVALID: "DMS_ERR_INVALID", DMS_ERR_STATE: "DMS_ERR_STATE", DMS_ERR_CUDA: "DMS_ERR_CUDA",

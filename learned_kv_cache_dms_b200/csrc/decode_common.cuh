@@ -412,7 +412,6 @@ __device__ __forceinline__ float decide_cta(const CacheView& c, const DecideArgs
       reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.hidden) + static_cast<long>(b) * hid);
   const uint4* wr =
       reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.W) + static_cast<long>(src) * hid);
-  const uint4* gr = reinterpret_cast<const uint4*>(a.gamma);
   float ss = 0.f, dot = 0.f;
   for (int v0 = 0; v0 < nvec; v0 += kThreads * VPT) {
     uint4 xu[VPT], wu[VPT], gu[VPT];
@@ -422,7 +421,7 @@ __device__ __forceinline__ float decide_cta(const CacheView& c, const DecideArgs
       const bool ok = vi < nvec;
       xu[u] = ok ? xr[vi] : make_uint4(0, 0, 0, 0);
       wu[u] = ok ? wr[vi] : make_uint4(0, 0, 0, 0);
-      gu[u] = ok ? gr[vi] : make_uint4(0, 0, 0, 0);
+      gu[u] = ok ? gamma16<__nv_bfloat16>(a.gamma, vi) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < VPT; ++u) {
@@ -453,9 +452,7 @@ __device__ __forceinline__ float decide_cta(const CacheView& c, const DecideArgs
     const float s2 = red[0] + red[1] + red[2] + red[3];
     const float d2 = red[4] + red[5] + red[6] + red[7];
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
-    const float inv = 1.0f / sqrtf(s2 / static_cast<float>(hid) + c.rms_eps);
-    const float z = d2 * inv + (bias ? __bfloat162float(bias[src]) : 0.f);
-    alpha = z * c.alpha_scale - a.offset[b * a.offset_bstride + src];
+    alpha = adapter_logit(c, d2, s2, hid, bias ? __bfloat162float(bias[src]) : 0.f, a.offset[b * a.offset_bstride + src]);
   }
   return alpha;
 }

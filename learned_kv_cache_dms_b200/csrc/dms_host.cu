@@ -32,6 +32,10 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int elem_bytes(int dt) { return dt == DMS_F32 ? 4 : dt == DMS_BF16 ? 2 : 1; }
 
+// Sources whose decision logit comes from a product of the hidden state with
+// a weight table (the adapter with RMSNorm, and the importance score).
+bool adapter_source(int src) { return src == DMS_ALPHA_PROJ || src == DMS_ALPHA_SCORE_LINEAR; }
+
 int check_desc(const dms_cache_desc* d) {
   if (!d) return DMS_ERR_INVALID;
   if (d->num_layers <= 0 || d->batch <= 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0) return DMS_ERR_INVALID;
@@ -46,12 +50,12 @@ int check_desc(const dms_cache_desc* d) {
   if (!(d->kv_dtype == d->act_dtype || (d->kv_dtype == DMS_FP8_E4M3 && d->act_dtype == DMS_BF16)))
     return DMS_ERR_INVALID;
   if (d->alpha_per != DMS_ALPHA_PER_HEAD && d->alpha_per != DMS_ALPHA_PER_LAYER) return DMS_ERR_INVALID;
-  if (d->alpha_source < DMS_ALPHA_PROJ || d->alpha_source > DMS_ALPHA_QUERY_NEURON) return DMS_ERR_INVALID;
-  if (d->alpha_source == DMS_ALPHA_PROJ) {
+  if (d->alpha_source < DMS_ALPHA_PROJ || d->alpha_source > DMS_ALPHA_SCORE_LINEAR) return DMS_ERR_INVALID;
+  if (adapter_source(d->alpha_source)) {
     if (d->hidden <= 0 || d->hidden % 8) return DMS_ERR_INVALID;
     if (d->num_kv_heads > 8 || static_cast<long>(d->num_kv_heads) * d->hidden > 40960) return DMS_ERR_INVALID;
   }
-  if (d->alpha_source != DMS_ALPHA_PROJ && d->num_kv_heads > 32) return DMS_ERR_INVALID;
+  if (!adapter_source(d->alpha_source) && d->num_kv_heads > 32) return DMS_ERR_INVALID;
   if (!(d->alpha_scale == d->alpha_scale) || !(d->rms_eps >= 0.0f)) return DMS_ERR_INVALID;
   if (d->decode_kernel < DMS_DECODE_AUTO || d->decode_kernel > DMS_DECODE_FLAT) return DMS_ERR_INVALID;
   if (d->decision_shift < -1 || d->decision_shift > 1) return DMS_ERR_INVALID;
@@ -425,19 +429,22 @@ int dms_cache_positions(const dms_cache* c, int layer) {
 static int check_decide(const dms_cache* c, const dms_decide_params* d) {
   if (!d || !d->offset) return DMS_ERR_INVALID;
   if (d->offset_batch_stride != 0 && d->offset_batch_stride != c->desc.num_kv_heads) return DMS_ERR_INVALID;
-  if (c->desc.alpha_source == DMS_ALPHA_PROJ) {
-    if (!d->hidden || !d->norm_weight || !d->proj_weight) return DMS_ERR_INVALID;
-    const uintptr_t any = reinterpret_cast<uintptr_t>(d->hidden) | reinterpret_cast<uintptr_t>(d->norm_weight) |
+  if (adapter_source(c->desc.alpha_source)) {
+    // the score source has no normalisation: norm_weight is not read
+    const bool norm = c->desc.alpha_source == DMS_ALPHA_PROJ;
+    if (!d->hidden || !d->proj_weight || (norm && !d->norm_weight)) return DMS_ERR_INVALID;
+    const uintptr_t any = reinterpret_cast<uintptr_t>(d->hidden) |
+                          (norm ? reinterpret_cast<uintptr_t>(d->norm_weight) : 0) |
                           reinterpret_cast<uintptr_t>(d->proj_weight);
     if (any & 15) return DMS_ERR_INVALID;  // read as 16-byte vectors
   }
   return DMS_OK;
 }
 
-static DecideArgs decide_args(const dms_decide_params* d) {
+static DecideArgs decide_args(const dms_cache* c, const dms_decide_params* d) {
   DecideArgs a{};
   a.hidden = d->hidden;
-  a.gamma = d->norm_weight;
+  a.gamma = c->desc.alpha_source == DMS_ALPHA_PROJ ? d->norm_weight : nullptr;  // none: ones
   a.W = d->proj_weight;
   a.bias = d->proj_bias;
   a.offset = d->offset;
@@ -451,10 +458,10 @@ int dms_decide(dms_cache* c, int T, const dms_decide_params* d, void* neuron_src
   if (e) return e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t r;
-  if (c->desc.alpha_source == DMS_ALPHA_PROJ) {
+  if (adapter_source(c->desc.alpha_source)) {
     CUtensorMap hm;
     const bool have = make_hidden_map(&hm, &c->desc, d->hidden, T);
-    r = launch_decide_proj(c->view, T, decide_args(d), alpha, have ? &hm : nullptr, s);
+    r = launch_decide_proj(c->view, T, decide_args(c, d), alpha, have ? &hm : nullptr, s);
   } else {
     if (!neuron_src) return DMS_ERR_INVALID;
     const bool key = c->desc.alpha_source == DMS_ALPHA_KEY_NEURON;
@@ -499,11 +506,11 @@ int dms_prefill_compact(dms_cache* c, int layer, const dms_prefill_args* a, void
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   track_launch(c, layer, s);
   const CacheView& v = c->view;
-  const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
+  const bool neuron = a->decide && !adapter_source(c->desc.alpha_source);
   if (a->decide && !neuron) {
     CUtensorMap hm;
     const bool have = make_hidden_map(&hm, &c->desc, a->decide->hidden, T);
-    if (launch_decide_proj(v, T, decide_args(a->decide), a->alpha, have ? &hm : nullptr, s) != cudaSuccess)
+    if (launch_decide_proj(v, T, decide_args(c, a->decide), a->alpha, have ? &hm : nullptr, s) != cudaSuccess)
       return DMS_ERR_CUDA;
   }
   if (neuron || a->rope_cos) {
@@ -583,14 +590,14 @@ int dms_decode_append(dms_cache* c, int layer, const dms_decode_args* a, void* s
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   track_launch(c, layer, s);
   const CacheView& v = c->view;
-  const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
+  const bool neuron = a->decide && !adapter_source(c->desc.alpha_source);
   // The adapter's decision logits are computed inside the append kernel when
   // the batch has few heads (one warp per dot product); otherwise by their own
   // kernel with one CTA per (head, sequence).
   const bool fuse = a->decide && !neuron && c->desc.batch * c->desc.num_kv_heads <= kFuseDecideHeads;
   DecideArgs da{};
   if (a->decide && !neuron) {
-    da = decide_args(a->decide);
+    da = decide_args(c, a->decide);
     if (!fuse && launch_decide_proj(v, 1, da, a->alpha, nullptr, s) != cudaSuccess) return DMS_ERR_CUDA;
   }
   if (neuron || a->rope_cos) {
@@ -679,7 +686,7 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   if (!c->prefilled[layer] || c->positions[layer] >= c->desc.max_positions) return DMS_ERR_STATE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CacheView& v = c->view;
-  const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
+  const bool neuron = a->decide && !adapter_source(c->desc.alpha_source);
   if (neuron || a->rope_cos) {
     track_launch(c, layer, s);
     if (launch_neuron_rope(v, 1, v.pos + static_cast<long>(layer) * v.B, a->q, a->k,
@@ -689,7 +696,7 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   }
   DecideArgs da{};
   const bool proj = a->decide && !neuron;
-  if (proj) da = decide_args(a->decide);
+  if (proj) da = decide_args(c, a->decide);
   // bf16 pages: one launch -- attention over the pre-append slots plus the new
   // token, then the append, with the adapter's decision logits computed inside.
   if (int e = run_decode_kernel(c, layer, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, s)) return e;
@@ -716,7 +723,7 @@ int dms_decode_step_layers(dms_cache* c, int layer0, int num_layers, const dms_d
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CacheView& v = c->view;
   const int B = c->desc.batch, Hq = c->desc.num_q_heads, Hkv = c->desc.num_kv_heads, D = c->desc.head_dim;
-  const bool neuron = a->decide && c->desc.alpha_source != DMS_ALPHA_PROJ;
+  const bool neuron = a->decide && !adapter_source(c->desc.alpha_source);
   const long ostride_layer = a->decide ? static_cast<long>(a->decide->offset_batch_stride ? B * Hkv : Hkv) : 0;
   if (neuron || a->rope_cos) {
     // the decision neuron / rotary pass of each layer (its rows of q and k)
@@ -734,7 +741,7 @@ int dms_decode_step_layers(dms_cache* c, int layer0, int num_layers, const dms_d
   DecideArgs da{};
   const bool proj = a->decide && !neuron;
   if (proj) {
-    da = decide_args(a->decide);
+    da = decide_args(c, a->decide);
     da.gamma_lstride = c->desc.hidden;
     da.w_lstride = static_cast<long>(Hkv) * c->desc.hidden;
     da.bias_lstride = Hkv;

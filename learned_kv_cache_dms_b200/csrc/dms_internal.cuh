@@ -136,6 +136,28 @@ __device__ __forceinline__ __nv_bfloat16 from_f64<__nv_bfloat16>(double x) {
   return __float2bfloat16_rn(f64_to_f32_odd(x));
 }
 
+// 16 bytes of the RMSNorm weight gamma (vector vi), or of ones when there is
+// none (the score source has no normalisation).
+template <typename TA>
+__device__ __forceinline__ uint4 gamma16(const void* g, long vi) {
+  if (g) return reinterpret_cast<const uint4*>(g)[vi];
+  const unsigned one = sizeof(TA) == 2 ? 0x3F803F80u : 0x3F800000u;
+  return make_uint4(one, one, one, one);
+}
+
+// Decision logit of the adapter sources from dot = W_h . (x * gamma), the
+// sum of squares ss of the hidden row x (hid elements), the bias and the
+// offset: PROJ, alpha = (dot / rms(x) + bias) * alpha_scale - offset with
+// rms(x) = sqrt(ss / hid + rms_eps); SCORE_LINEAR (a KVzap-style importance
+// score, gamma absent), alpha = offset - (dot + bias) with the offset as the
+// pruning threshold: a token scoring below it is marked.
+__device__ __forceinline__ float adapter_logit(const CacheView& c, float dot, float ss, int hid, float bias,
+                                               float offset) {
+  if (c.alpha_source == DMS_ALPHA_SCORE_LINEAR) return offset - (dot + bias);
+  const float inv = 1.0f / sqrtf(ss / static_cast<float>(hid) + c.rms_eps);
+  return (dot * inv + bias) * c.alpha_scale - offset;
+}
+
 // Unpack a 16-byte vector into floats (8 bf16 or 4 fp32).
 template <typename T>
 struct Vec16 {

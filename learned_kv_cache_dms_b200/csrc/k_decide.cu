@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(256) k_decide_proj(CacheView c, int T, DecideA
   for (int i = threadIdx.x; i < H * nvec; i += blockDim.x) {
     float wv[V], gv[V];
     unpack16(reinterpret_cast<const uint4*>(W)[i], wv, static_cast<const TA*>(nullptr));
-    unpack16(reinterpret_cast<const uint4*>(gamma)[i % nvec], gv, static_cast<const TA*>(nullptr));
+    unpack16(gamma16<TA>(gamma, i % nvec), gv, static_cast<const TA*>(nullptr));
 #pragma unroll
     for (int e = 0; e < V; ++e) wg[i * V + e] = wv[e] * gv[e];
   }
@@ -165,14 +165,13 @@ __global__ void __launch_bounds__(256) k_decide_proj(CacheView c, int T, DecideA
         const long tok = tok0 + u;
         if (tok >= ntok) continue;
         const int b = static_cast<int>(tok / T), t = static_cast<int>(tok % T);
-        const float inv = 1.0f / sqrtf(ss[u] / static_cast<float>(hid) + c.rms_eps);
         float a0 = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (j >= H) continue;
           const int src = layer_mode ? 0 : j;
-          float z = dot[u][src] * inv + (bias ? to_f(bias[src]) : 0.f);
-          float al = z * c.alpha_scale - a.offset[b * a.offset_bstride + src];
+          const float al = adapter_logit(c, dot[u][src], ss[u], hid, bias ? to_f(bias[src]) : 0.f,
+                                         a.offset[b * a.offset_bstride + src]);
           if (j == 0) a0 = al;
           alpha[(static_cast<long>(b) * H + j) * T + t] = layer_mode ? a0 : al;
         }
@@ -191,13 +190,12 @@ __global__ void __launch_bounds__(256) k_decide_proj_row(CacheView c, DecideArgs
   constexpr int V = 16 / sizeof(TA);
   const uint4* x = reinterpret_cast<const uint4*>(static_cast<const TA*>(a.hidden) + static_cast<long>(b) * hid);
   const uint4* W = reinterpret_cast<const uint4*>(static_cast<const TA*>(a.W) + static_cast<long>(src) * hid);
-  const uint4* gamma = reinterpret_cast<const uint4*>(a.gamma);
   float ss = 0.f, dot = 0.f;
   for (int vi = threadIdx.x; vi < hid / V; vi += blockDim.x) {
     float xv[V], wv[V], gv[V];
     unpack16(x[vi], xv, static_cast<const TA*>(nullptr));
     unpack16(W[vi], wv, static_cast<const TA*>(nullptr));
-    unpack16(gamma[vi], gv, static_cast<const TA*>(nullptr));
+    unpack16(gamma16<TA>(a.gamma, vi), gv, static_cast<const TA*>(nullptr));
 #pragma unroll
     for (int e = 0; e < V; ++e) {
       ss = fmaf(xv[e], xv[e], ss);
@@ -223,9 +221,8 @@ __global__ void __launch_bounds__(256) k_decide_proj_row(CacheView c, DecideArgs
       d2 += red[1][i];
     }
     const TA* bias = static_cast<const TA*>(a.bias);
-    const float inv = 1.0f / sqrtf(s2 / static_cast<float>(hid) + c.rms_eps);
-    const float z = d2 * inv + (bias ? to_f(bias[src]) : 0.f);
-    alpha[b * c.Hkv + h] = z * c.alpha_scale - a.offset[b * a.offset_bstride + src];
+    alpha[b * c.Hkv + h] =
+        adapter_logit(c, d2, s2, hid, bias ? to_f(bias[src]) : 0.f, a.offset[b * a.offset_bstride + src]);
   }
 }
 
@@ -322,7 +319,7 @@ __global__ void __launch_bounds__(kDpThreads, 1)
       const int n = i / rvec, v = i % rvec;
       if (n < H && v < nvec) {
         wq[u] = reinterpret_cast<const uint4*>(W + static_cast<long>(n) * hid)[v];
-        gq[u] = reinterpret_cast<const uint4*>(gamma)[v];
+        gq[u] = gamma16<__nv_bfloat16>(gamma, v);
       }
     }
 #pragma unroll
@@ -432,15 +429,14 @@ __global__ void __launch_bounds__(kDpThreads, 1)
           const long tok = static_cast<long>(tile) * kDpTok + mt * 16 + (lane >> 2) + 8 * r;
           if (tok >= ntok) continue;
           const int b = static_cast<int>(tok / T), t = static_cast<int>(tok % T);
-          const float inv = 1.0f / sqrtf(ss[r] / static_cast<float>(hid) + c.rms_eps);
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int j = 2 * (lane & 3) + e;
             if (j >= H) continue;
             const int src = layer_mode ? 0 : j;
             const float dot = layer_mode ? h0[r] : acc[2 * r + e];
-            const float z = dot * inv + (bias ? __bfloat162float(bias[src]) : 0.f);
-            alpha[(static_cast<long>(b) * H + j) * T + t] = z * c.alpha_scale - a.offset[b * a.offset_bstride + src];
+            alpha[(static_cast<long>(b) * H + j) * T + t] = adapter_logit(
+                c, dot, ss[r], hid, bias ? __bfloat162float(bias[src]) : 0.f, a.offset[b * a.offset_bstride + src]);
           }
         }
       }

@@ -48,11 +48,10 @@ __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, i
     const int hid = c.hidden, nvec = hid / V;
     const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const TA*>(da.hidden) + static_cast<long>(b) * hid);
     const uint4* wr = reinterpret_cast<const uint4*>(static_cast<const TA*>(da.W) + static_cast<long>(hs) * hid);
-    const uint4* gr = reinterpret_cast<const uint4*>(da.gamma);
     float ss = 0.f, dot = 0.f;
 #pragma unroll 4
     for (int vi = tid; vi < nvec; vi += kAppendThreads) {
-      const uint4 xu = xr[vi], wu = wr[vi], gu = gr[vi];
+      const uint4 xu = xr[vi], wu = wr[vi], gu = gamma16<TA>(da.gamma, vi);
       float x[V], wv[V], gv[V];
       unpack16(xu, x, static_cast<const TA*>(nullptr));
       unpack16(wu, wv, static_cast<const TA*>(nullptr));
@@ -80,9 +79,7 @@ __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, i
         d2 += s_f[1][i];
       }
       const TA* bias = static_cast<const TA*>(da.bias);
-      const float inv = 1.0f / sqrtf(s2 / static_cast<float>(hid) + c.rms_eps);
-      const float z = d2 * inv + (bias ? to_f(bias[hs]) : 0.f);
-      a_dec = z * c.alpha_scale - da.offset[b * da.offset_bstride + hs];
+      a_dec = adapter_logit(c, d2, s2, hid, bias ? to_f(bias[hs]) : 0.f, da.offset[b * da.offset_bstride + hs]);
       alpha[b * c.Hkv + h] = a_dec;
     }
     __syncthreads();

@@ -131,7 +131,6 @@ __device__ __forceinline__ float decide_warp(const CacheView& c, const DecideArg
       reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.hidden) + static_cast<long>(b) * hid);
   const uint4* wr =
       reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.W) + static_cast<long>(src) * hid);
-  const uint4* gr = reinterpret_cast<const uint4*>(a.gamma);
   constexpr int VPT = 8;
   float ss = 0.f, dot = 0.f;
   for (int v0 = 0; v0 < nvec; v0 += 32 * VPT) {
@@ -142,7 +141,7 @@ __device__ __forceinline__ float decide_warp(const CacheView& c, const DecideArg
       const bool ok = vi < nvec;
       xu[u] = ok ? xr[vi] : make_uint4(0, 0, 0, 0);
       wu[u] = ok ? wr[vi] : make_uint4(0, 0, 0, 0);
-      gu[u] = ok ? gr[vi] : make_uint4(0, 0, 0, 0);
+      gu[u] = ok ? gamma16<__nv_bfloat16>(a.gamma, vi) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < VPT; ++u) {
@@ -163,9 +162,7 @@ __device__ __forceinline__ float decide_warp(const CacheView& c, const DecideArg
     dot += __shfl_xor_sync(0xffffffffu, dot, o);
   }
   const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
-  const float inv = 1.0f / sqrtf(ss / static_cast<float>(hid) + c.rms_eps);
-  const float z = dot * inv + (bias ? __bfloat162float(bias[src]) : 0.f);
-  return z * c.alpha_scale - a.offset[b * a.offset_bstride + src];
+  return adapter_logit(c, dot, ss, hid, bias ? __bfloat162float(bias[src]) : 0.f, a.offset[b * a.offset_bstride + src]);
 }
 
 // One warp's online-softmax update over KEYS consecutive keys of a staged tile

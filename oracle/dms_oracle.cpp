@@ -360,6 +360,28 @@ void oracle_decide_proj(int B, int T, int hidden, int Hkv, const double* h, cons
     }
 }
 
+// Decision logits from an importance score (the KVzap-linear page, workflow:
+// a Linear from the layer's hidden state to one score per KV head; tokens
+// scoring below the threshold are pruned while the most recent ones are
+// kept): score = W_h . x_t + bias_h, alpha = threshold_h - score, so a token
+// is marked iff its score is below the threshold.  No normalisation.
+//   h [B,T,hidden]  W [Hkv,hidden]  bias [Hkv] or null  threshold [B,Hkv]
+// With layer granularity every head takes head 0's logit.
+void oracle_decide_score(int B, int T, int hidden, int Hkv, const double* h, const double* W,
+                         const double* bias, const double* threshold, int layer_mode, double* alpha) {
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int t = 0; t < T; ++t) {
+      const double* x = h + (static_cast<size_t>(b) * T + t) * hidden;
+      for (int hd = 0; hd < Hkv; ++hd) {
+        const int src = layer_mode ? 0 : hd;
+        double score = bias ? bias[src] : 0.0;
+        for (int i = 0; i < hidden; ++i) score += W[static_cast<size_t>(src) * hidden + i] * x[i];
+        alpha[(static_cast<size_t>(b) * Hkv + hd) * T + t] = threshold[b * Hkv + src] - score;
+      }
+    }
+}
+
 // Decision logits from a single neuron ([DMS-Qwen3], source one): the last
 // element of a key (group = 1) or of the first query head of each GQA group
 // (group = Hq/Hkv), times the scale, minus the offset; that element is then set

@@ -29,6 +29,7 @@ def lib():
         L.oracle_e4m3_decode_n.argtypes = [up, dp, C.c_long]
         L.oracle_decide_proj.argtypes = [C.c_int] * 4 + [dp] * 5 + [C.c_double, C.c_double, C.c_int, dp]
         L.oracle_decide_neuron.argtypes = [C.c_int] * 6 + [dp, dp, C.c_double, C.c_int, dp]
+        L.oracle_decide_score.argtypes = [C.c_int] * 4 + [dp] * 4 + [C.c_int, dp]
         L.oracle_rope.argtypes = [C.c_int] * 4 + [dp, C.c_int, dp, dp]
         L.oracle_round_bf16_n.argtypes = [dp, fp, C.c_long]
         L.oracle_prefill_attention.argtypes = [C.c_int] * 6 + [dp, dp, dp, up, ip, C.c_long, dp]
@@ -100,6 +101,20 @@ def decide_proj(h, gamma, W, bias, offset, scale=100.0, eps=1e-6, layer_mode=Fal
     lib().oracle_decide_proj(B, T, hidden, Hkv, _p(h, C.c_double), _p(gamma, C.c_double),
                              _p(W, C.c_double), _p(bias, C.c_double), _p(off, C.c_double),
                              float(scale), float(eps), int(bool(layer_mode)), _p(alpha, C.c_double))
+    return alpha
+
+
+def decide_score(h, W, bias, threshold, layer_mode=False):
+    """alpha[B,Hkv,T] = threshold - (W . h + bias): the importance-score source."""
+    h = _f64(h)
+    B, T, hidden = h.shape
+    W = _f64(W)
+    Hkv = W.shape[0]
+    thr = _f64(np.broadcast_to(np.asarray(threshold, np.float64), (B, Hkv)))
+    bias = None if bias is None else _f64(bias)
+    alpha = np.empty((B, Hkv, T), np.float64)
+    lib().oracle_decide_score(B, T, hidden, Hkv, _p(h, C.c_double), _p(W, C.c_double), _p(bias, C.c_double),
+                              _p(thr, C.c_double), int(bool(layer_mode)), _p(alpha, C.c_double))
     return alpha
 
 

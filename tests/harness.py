@@ -34,7 +34,7 @@ class Case:
     P: int = 16
     act: str = "f32"
     kv: str = "f32"
-    source: str = "input"      # input | proj | key | query
+    source: str = "input"      # input | proj | key | query | score
     per: str = "head"          # head | layer
     keep: object = 0.5         # float, or (lo, hi) per (b, h)
     disable: bool = False
@@ -93,6 +93,20 @@ def build(case: Case):
         alpha_o = alpha.double().numpy()
         out["alpha_in"] = alpha
         kz, qz = _f64(k), _f64(q)
+    elif case.source == "score":
+        # the importance score: Linear(hidden -> Hkv) with a bias, no norm;
+        # thresholds calibrated per head like the adapter's offsets
+        h = I.normal(s, (case.layer, 4), (B, N, case.hidden), case.act)
+        W = I.normal(s, (case.layer, 11), (case.Hkv, case.hidden), case.act, std=case.hidden ** -0.5)
+        bias = I.normal(s, (case.layer, 12), (case.Hkv,), case.act, std=0.1)
+        neg_score = O.decide_score(_f64(h), _f64(W), _f64(bias), np.zeros((B, case.Hkv)), layer_mode)
+        off, _ = I.calibrate_offsets(neg_score, keep)
+        if layer_mode:
+            off[:] = off[:, :1]
+        thr = -off.astype(np.float64)
+        alpha_o = O.decide_score(_f64(h), _f64(W), _f64(bias), thr, layer_mode)
+        out.update(h=h, W=W, bias=bias, offset=torch.from_numpy(thr.astype(np.float32)))
+        kz, qz = _f64(k), _f64(q)
     elif case.source == "proj":
         h = I.normal(s, (case.layer, 4), (B, N, case.hidden), case.act)
         gamma = I.normal(s, (case.layer, 10), (case.hidden,), case.act)
@@ -119,8 +133,11 @@ def build(case: Case):
         kz = zeroed if case.source == "key" else _f64(k)
         qz = zeroed if case.source == "query" else _f64(q)
     if case.source != "input":
+        # the score is not multiplied by alpha_scale: the same margin on the
+        # raw dot product as the adapter's (0.02 / 100)
+        margin = MIN_MARGIN / ALPHA_SCALE if case.source == "score" else MIN_MARGIN
         m = np.min(np.abs(alpha_o))
-        assert m > MIN_MARGIN, "decision margin %.3g too small for a bit-exact comparison; change the seed" % m
+        assert m > margin, "decision margin %.3g too small for a bit-exact comparison; change the seed" % m
     if case.rope:
         cos, sin = I.rope_tables(N, case.D)
         out["rope"] = (cos, sin)
@@ -212,7 +229,7 @@ def make_desc(B_, case: Case):
     d.kv_dtype = {"f32": B_.DMS_F32, "bf16": B_.DMS_BF16, "fp8": B_.DMS_FP8_E4M3}[case.kv]
     d.alpha_per = B_.DMS_ALPHA_PER_LAYER if case.per == "layer" else B_.DMS_ALPHA_PER_HEAD
     d.alpha_source = {"input": B_.DMS_ALPHA_PROJ, "proj": B_.DMS_ALPHA_PROJ, "key": B_.DMS_ALPHA_KEY_NEURON,
-                      "query": B_.DMS_ALPHA_QUERY_NEURON}[case.source]
+                      "query": B_.DMS_ALPHA_QUERY_NEURON, "score": B_.DMS_ALPHA_SCORE_LINEAR}[case.source]
     if case.source in ("key", "query", "input"):
         d.hidden = max(d.hidden, 8)
     d.alpha_scale, d.rms_eps = ALPHA_SCALE, RMS_EPS
@@ -240,11 +257,16 @@ def run_gpu(case: Case, ins, cache=None):
     rope = tuple(t.to(dev) for t in ins["rope"]) if case.rope else None
     decide = None
     keep_alive = []
-    if case.source == "proj":
+    gamma = bias = None
+    if case.source in ("proj", "score"):
         h = ins["h"].to(dev)
-        gamma, W = ins["gamma"].to(dev), ins["W"].to(dev)
+        W = ins["W"].to(dev)
+        if case.source == "proj":
+            gamma = ins["gamma"].to(dev)
+        else:
+            bias = ins["bias"].to(dev)
         off = ins["offset"].to(dev)
-        keep_alive += [h, gamma, W, off]
+        keep_alive += [h, gamma, W, off, bias]
     elif case.source in ("key", "query"):
         off = ins["offset"].to(dev)
         keep_alive.append(off)
@@ -260,10 +282,10 @@ def run_gpu(case: Case, ins, cache=None):
             alpha = ins["alpha_in"][:, :, t0:t0 + n].contiguous().to(dev)
         else:
             alpha = torch.empty(B, case.Hkv, n, dtype=torch.float32, device=dev)
-            if case.source == "proj":
+            if case.source in ("proj", "score"):
                 hp = h[:, t0:t0 + n].contiguous()
                 keep_alive.append(hp)
-                decide = B_.decide_params(off, hidden=hp, norm_weight=gamma, proj_weight=W)
+                decide = B_.decide_params(off, hidden=hp, norm_weight=gamma, proj_weight=W, proj_bias=bias)
             else:
                 decide = B_.decide_params(off)
         cache.prefill(case.layer, qp, kp, vp, o, alpha, decide=decide, rope=rope)
@@ -288,9 +310,9 @@ def run_gpu(case: Case, ins, cache=None):
             dd = None
         else:
             at = torch.empty(B, case.Hkv, dtype=torch.float32, device=dev)
-            if case.source == "proj":
+            if case.source in ("proj", "score"):
                 ht = h[:, t].contiguous()
-                dd = B_.decide_params(off, hidden=ht, norm_weight=gamma, proj_weight=W)
+                dd = B_.decide_params(off, hidden=ht, norm_weight=gamma, proj_weight=W, proj_bias=bias)
                 keep_alive.append(ht)
             else:
                 dd = B_.decide_params(off)

@@ -61,7 +61,7 @@ def test_cache_bytes_and_validation(B):
         ("head_dim", 96),
         ("num_q_heads", 7),      # not a multiple of kv heads
         ("alpha_per", 2),
-        ("alpha_source", 3),
+        ("alpha_source", 4),
         ("kv_dtype", 2),         # FP8 pages need bf16 activations: ok here...
     ]
     for field, val in bad[:-1]:

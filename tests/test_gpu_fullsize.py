@@ -25,6 +25,12 @@ FULL = {
     "llama1b_layer": Case(B=4, T=32768, steps=256, Hq=32, Hkv=8, D=64, hidden=2048, w=512, P=256, act="bf16",
                           kv="fp8", source="key", per="layer", keep=1 / 8, rope=True, prealloc=4096,
                           attn_rows=256, seed=1014),
+    # the importance-score source on the Llama-3.1-8B attention shape (the
+    # KVzap-linear page: hidden 4096 -> 8 KV heads, threshold pruning outside
+    # the last 128 tokens), 8192 + 64, keep 1/4
+    "kvzap_llama8b_score": Case(B=1, T=8192, steps=64, Hq=32, Hkv=8, D=128, hidden=4096, w=128, P=64,
+                                act="bf16", kv="bf16", source="score", keep=1 / 4, prealloc=2048, attn_rows=256,
+                                seed=1006),
     # reasoning stack: batch 32, prompt 1024, keep 1/16, last of 36 layers
     "reason36_last_layer": Case(B=32, T=1024, steps=256, Hq=32, Hkv=8, D=128, hidden=4096, w=512, P=256,
                                 act="bf16", kv="bf16", source="proj", keep=1 / 16, layers=36, layer=35,

@@ -83,6 +83,14 @@ CASES = {
     "bf16_shift_left_layer_b8": Case(B=8, T=300, steps=40, Hq=16, Hkv=8, D=128, hidden=256, w=64, P=32,
                                      act="bf16", kv="bf16", source="proj", per="layer", keep=(1 / 16, 1 / 4),
                                      prealloc=96, shift=-1, seed=74),
+    # the importance-score source (KVzap-style: Linear with a bias, no norm,
+    # prune below a threshold, keep the last 128 tokens), bf16 and fp32
+    "bf16_score_w128": Case(B=2, T=700, steps=20, Hq=32, Hkv=8, D=128, hidden=512, w=128, P=64, act="bf16",
+                            kv="bf16", source="score", keep=0.25, seed=75),
+    "f32_score_w128_layer": Case(B=1, T=400, steps=12, Hq=8, Hkv=4, D=64, hidden=256, w=128, P=32, act="f32",
+                                 kv="f32", source="score", per="layer", keep=0.3, seed=76),
+    "fp8_score_w128": Case(B=2, T=600, steps=16, Hq=16, Hkv=4, D=64, hidden=320, w=128, P=64, act="bf16",
+                           kv="fp8", source="score", keep=0.2, seed=77),
     # second layer of a two-layer cache with preallocation
     "layer1_of_2": Case(B=2, T=260, steps=12, Hq=4, Hkv=2, D=64, w=32, P=16, act="bf16", kv="bf16",
                         source="input", keep=0.3, layers=2, layer=1, prealloc=64, seed=15),

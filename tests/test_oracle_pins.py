@@ -688,3 +688,46 @@ def test_shift_attention_reduces_to_masked_attention(shift):
     c = O.Cache(1, B, Hkv, D, w, P, T, 40, 0, shift=shift)
     got = _chunked(c, 0, q, k, v, bits, [13, 23])
     assert np.allclose(got, ref, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Importance-score source (the KVzap-linear page: one Linear per layer from the
+# hidden state to a score per KV head; prune below the threshold, keep the
+# most recent tokens)
+# ---------------------------------------------------------------------------
+def test_decide_score_is_threshold_minus_linear_score():
+    rng = np.random.default_rng(40)
+    B, T, hid, H = 2, 7, 64, 3
+    h = rng.standard_normal((B, T, hid))
+    W = rng.standard_normal((H, hid)) / 8
+    bias = rng.standard_normal(H)
+    thr = np.array([[-4.0, 0.5, 1.0], [2.0, -1.0, 0.0]])
+    a = O.decide_score(h, W, bias, thr)
+    want = thr[:, :, None] - (np.einsum("bti,hi->bht", h, W) + bias[None, :, None])
+    assert np.allclose(a, want, rtol=0, atol=1e-12)
+    # no normalisation: the score is linear in the hidden state (the adapter's
+    # RMSNorm would make it scale-invariant instead)
+    a2 = O.decide_score(2 * h, W, None, np.zeros((B, H)))
+    assert np.allclose(a2, 2 * O.decide_score(h, W, None, np.zeros((B, H))), rtol=0, atol=1e-12)
+    # zero weights: every token scores its bias; layer mode copies head 0
+    assert np.array_equal(O.decide_score(h, np.zeros((H, hid)), None, thr), np.broadcast_to(thr[:, :, None], (B, H, T)))
+    al = O.decide_score(h, W, bias, thr, layer_mode=True)
+    assert np.array_equal(al[:, 1], al[:, 0]) and np.array_equal(al[:, 0], a[:, 0])
+
+
+def test_score_pruning_keeps_recent_tokens_and_high_scores():
+    """With window 128 the delayed-eviction rule keeps exactly what the page's
+    pruning keeps: the last 128 tokens and every earlier token whose score is
+    not below the threshold."""
+    rng = np.random.default_rng(41)
+    T, hid, w, P = 700, 32, 128, 64
+    h = rng.standard_normal((1, T, hid))
+    W = rng.standard_normal((1, hid)) / 6
+    a = O.decide_score(h, W, None, np.array([[-0.3]]))
+    ev = O.evict_bits(a)
+    c = O.Cache(1, 1, 1, 8, w, P, T, 64, 0, store_values=False)
+    c.prefill(0, ev)
+    s = c.export(0)
+    score = (h[0] @ W[0])
+    keep = set(range(T - w, T)) | {j for j in range(T - w) if score[j] >= -0.3}
+    assert sorted(s["slot_pos"][0, 0, :s["count"][0, 0]]) == sorted(keep)
