@@ -487,6 +487,85 @@ void oracle_prefill_attention(int B, int T, int Hq, int Hkv, int D, int w, const
 }
 
 // ---------------------------------------------------------------------------
+// Training mode ([DMS-Qwen3], "Gumbel 噪声与可微门控" and "注意力实现": the
+// soft-gated attention of the training path, forward only)
+// ---------------------------------------------------------------------------
+// Gate of each token: gate logit l = (alpha + noise) / tau, probability
+// p = sigmoid(l), forward value of the straight-through decision
+// (p > 0.5) - p + p, which is exactly 1 or 0 (here: p > 0.5); and the eviction
+// penalty of each key from the logits shifted right by one position:
+// penalty[k] = logsigmoid(-l[k-1]) = log(1 - p[k-1]) for k >= 1, penalty[0] = 0
+// (the padding position is never penalised).  All [B,Hkv,T]; noise may be
+// null (zero).
+void oracle_train_gate(int B, int Hkv, int T, const double* alpha, const double* noise, double tau,
+                       double* prob, double* hard, double* penalty) {
+  for (long r = 0; r < static_cast<long>(B) * Hkv; ++r) {
+    const double* a = alpha + r * T;
+    const double* g = noise ? noise + r * T : nullptr;
+    for (int t = 0; t < T; ++t) {
+      const double l = (a[t] + (g ? g[t] : 0.0)) / tau;
+      const double p = 1.0 / (1.0 + std::exp(-l));
+      prob[r * T + t] = p;
+      hard[r * T + t] = p > 0.5 ? 1.0 : 0.0;
+      // logsigmoid(-l) = -log(1 + exp(l)), in a form that does not overflow
+      const double ls = l > 0 ? -(l + std::log1p(std::exp(-l))) : -std::log1p(std::exp(l));
+      if (t + 1 < T) penalty[r * T + t + 1] = ls;
+    }
+    penalty[r * T] = 0.0;
+  }
+}
+
+// The soft-gated attention of the training path: query i and key j of KV head
+// hq / (Hq/Hkv) score s = q.k / sqrt(D); a key inside the window (i - j < w)
+// keeps s, a key outside it gets s + penalty[j]; a causal violation (j > i)
+// gets the mask value -50000, whose weight exp(-50000 - max) is zero in fp64,
+// so those keys are left out; o = softmax(scores) v.  Dense over every key.
+//   q [B,T,Hq,D], k/v [B,T,Hkv,D], penalty [B,Hkv,T]; rows as in
+//   oracle_prefill_attention.
+void oracle_train_attention(int B, int T, int Hq, int Hkv, int D, int w, const double* q, const double* k,
+                            const double* v, const double* penalty, const int* rows, long n_rows, double* o) {
+  const int g = Hq / Hkv;
+  const long total = rows ? n_rows : static_cast<long>(B) * Hq * T;
+  const double scale = 1.0 / std::sqrt(static_cast<double>(D));
+#pragma omp parallel for schedule(dynamic, 16)
+  for (long r = 0; r < total; ++r) {
+    int b, hq, i;
+    if (rows) {
+      b = rows[3 * r];
+      hq = rows[3 * r + 1];
+      i = rows[3 * r + 2];
+    } else {
+      b = static_cast<int>(r / (static_cast<long>(Hq) * T));
+      hq = static_cast<int>((r / T) % Hq);
+      i = static_cast<int>(r % T);
+    }
+    const int h = hq / g;
+    const double* qq = q + ((static_cast<size_t>(b) * T + i) * Hq + hq) * D;
+    std::vector<double> s(i + 1);
+    double m = -INFINITY;
+    for (int j = 0; j <= i; ++j) {
+      const double* kk = k + ((static_cast<size_t>(b) * T + j) * Hkv + h) * D;
+      double acc = 0.0;
+      for (int d = 0; d < D; ++d) acc += qq[d] * kk[d];
+      s[j] = acc * scale + (i - j < w ? 0.0 : penalty[(static_cast<size_t>(b) * Hkv + h) * T + j]);
+      m = std::max(m, s[j]);
+    }
+    double l = 0.0;
+    for (int j = 0; j <= i; ++j) {
+      s[j] = std::exp(s[j] - m);
+      l += s[j];
+    }
+    double* out = rows ? o + static_cast<size_t>(r) * D : o + ((static_cast<size_t>(b) * T + i) * Hq + hq) * D;
+    for (int d = 0; d < D; ++d) out[d] = 0.0;
+    for (int j = 0; j <= i; ++j) {
+      const double* vv = v + ((static_cast<size_t>(b) * T + j) * Hkv + h) * D;
+      for (int d = 0; d < D; ++d) out[d] += s[j] * vv[d];
+    }
+    for (int d = 0; d < D; ++d) out[d] /= l;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Paged cache simulation
 // ---------------------------------------------------------------------------
 void* oracle_cache_new(int L, int B, int Hkv, int D, int w, int P, int max_pos, int pool_pages,

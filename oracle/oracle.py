@@ -34,6 +34,8 @@ def lib():
         L.oracle_round_bf16_n.argtypes = [dp, fp, C.c_long]
         L.oracle_prefill_attention.argtypes = [C.c_int] * 6 + [dp, dp, dp, up, ip, C.c_long, dp]
         L.oracle_cache_new.argtypes = [C.c_int] * 12
+        L.oracle_train_gate.argtypes = [C.c_int] * 3 + [dp, dp, C.c_double, dp, dp, dp]
+        L.oracle_train_attention.argtypes = [C.c_int] * 6 + [dp] * 4 + [ip, C.c_long, dp]
         L.oracle_cache_new.restype = C.c_void_p
         L.oracle_cache_delete.argtypes = [C.c_void_p]
         L.oracle_cache_clone.argtypes = [C.c_void_p]
@@ -181,6 +183,34 @@ def prefill_attention(q, k, v, evict, window, rows=None):
         rp, n = _p(r, C.c_int), r.shape[0]
     lib().oracle_prefill_attention(B, T, Hq, Hkv, D, int(window), _p(q, C.c_double), _p(k, C.c_double),
                                    _p(v, C.c_double), _p(ev, C.c_uint8), rp, n, _p(o, C.c_double))
+    return o
+
+
+def train_gate(alpha, noise, tau):
+    """(prob, hard, penalty) [B,Hkv,T] of the training path's gate (fp64)."""
+    a = _f64(alpha)
+    B, H, T = a.shape
+    g = None if noise is None else _f64(noise)
+    prob, hard, pen = (np.empty((B, H, T), np.float64) for _ in range(3))
+    lib().oracle_train_gate(B, H, T, _p(a, C.c_double), _p(g, C.c_double), float(tau), _p(prob, C.c_double),
+                            _p(hard, C.c_double), _p(pen, C.c_double))
+    return prob, hard, pen
+
+
+def train_attention(q, k, v, penalty, window, rows=None):
+    """The soft-gated training attention, o[B,T,Hq,D] (or o[len(rows),D])."""
+    q, k, v, pen = _f64(q), _f64(k), _f64(v), _f64(penalty)
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if rows is None:
+        o = np.empty((B, T, Hq, D), np.float64)
+        rp, n = None, 0
+    else:
+        r = np.ascontiguousarray(np.asarray(rows, np.int32).reshape(-1, 3))
+        o = np.empty((r.shape[0], D), np.float64)
+        rp, n = _p(r, C.c_int), r.shape[0]
+    lib().oracle_train_attention(B, T, Hq, Hkv, D, int(window), _p(q, C.c_double), _p(k, C.c_double),
+                                 _p(v, C.c_double), _p(pen, C.c_double), rp, n, _p(o, C.c_double))
     return o
 
 

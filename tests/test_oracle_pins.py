@@ -731,3 +731,72 @@ def test_score_pruning_keeps_recent_tokens_and_high_scores():
     score = (h[0] @ W[0])
     keep = set(range(T - w, T)) | {j for j in range(T - w) if score[j] >= -0.3}
     assert sorted(s["slot_pos"][0, 0, :s["count"][0, 0]]) == sorted(keep)
+
+
+# ---------------------------------------------------------------------------
+# Training mode: Gumbel-sigmoid gate and soft-gated attention ([DMS-Qwen3],
+# "Gumbel 噪声与可微门控" and "注意力实现")
+# ---------------------------------------------------------------------------
+def test_train_gate_definition():
+    rng = np.random.default_rng(50)
+    a = rng.standard_normal((2, 3, 40)) * 3
+    u = rng.random((2, 3, 40))
+    g = np.log(u) - np.log1p(-u)
+    tau = 0.1
+    prob, hard, pen = O.train_gate(a, g, tau)
+    l = (a + g) / tau
+    assert np.allclose(prob, torch.sigmoid(torch.from_numpy(l)).numpy(), rtol=1e-12, atol=1e-15)
+    assert np.array_equal(hard, (a + g > 0).astype(np.float64))
+    # penalty: logsigmoid of the negated logit of the previous position; none at 0
+    want = torch.nn.functional.logsigmoid(-torch.from_numpy(l)).numpy()
+    assert np.all(pen[:, :, 0] == 0)
+    assert np.allclose(pen[:, :, 1:], want[:, :, :-1], rtol=1e-12, atol=1e-14)
+    # = log(1 - p) of the previous position
+    assert np.allclose(np.exp(pen[:, :, 1:]), 1 - prob[:, :, :-1], rtol=1e-9, atol=1e-12)
+    # no noise: the gate of the logit itself
+    p0, h0, _ = O.train_gate(a, None, tau)
+    assert np.array_equal(h0, (a > 0).astype(np.float64))
+
+
+def test_train_attention_reduces_to_causal_and_window():
+    rng = np.random.default_rng(51)
+    B, T, Hq, Hkv, D, w = 1, 50, 4, 2, 16, 8
+    q, k, v = rand_qkv(52, B, T, Hq, Hkv, D)
+    def sdpa(mask):
+        qq = torch.from_numpy(q).permute(0, 2, 1, 3)
+        kk = torch.from_numpy(k).permute(0, 2, 1, 3).repeat_interleave(Hq // Hkv, 1)
+        vv = torch.from_numpy(v).permute(0, 2, 1, 3).repeat_interleave(Hq // Hkv, 1)
+        return torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask).permute(0, 2, 1, 3).numpy()
+    i, j = np.arange(T)[:, None], np.arange(T)[None, :]
+    causal = torch.from_numpy(j <= i)
+    # no penalty (every gate closed): dense causal attention
+    o = O.train_attention(q, k, v, np.zeros((B, Hkv, T)), w)
+    assert np.allclose(o, sdpa(causal), rtol=0, atol=1e-12)
+    # the window covers the prompt: the penalty is never applied
+    o = O.train_attention(q, k, v, rng.standard_normal((B, Hkv, T)) - 5, T)
+    assert np.allclose(o, sdpa(causal), rtol=0, atol=1e-12)
+    # a huge penalty everywhere: pure sliding-window attention
+    o = O.train_attention(q, k, v, np.full((B, Hkv, T), -1e4), w)
+    assert np.allclose(o, sdpa(torch.from_numpy((j <= i) & (i - j < w))), rtol=0, atol=1e-12)
+    # an additive per-key bias outside the window: SDPA with a float mask
+    pen = -np.abs(rng.standard_normal((B, Hkv, T)))
+    bias = np.where(i - j < w, 0.0, pen[0, 0][None, :])
+    bias = np.where(j <= i, bias, -np.inf)
+    o = O.train_attention(q[:, :, :1], k[:, :, :1], v[:, :, :1], pen[:, :1], w)
+    qq, kk, vv = (torch.from_numpy(x[:, :, :1]).permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=torch.from_numpy(bias)).permute(0, 2, 1, 3)
+    assert np.allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_train_attention_hard_limit_is_the_inference_mask():
+    """As tau -> 0 the gate's penalty is 0 or -inf: the training attention
+    becomes the inference DMS mask of the decisions shifted right by one
+    (the +1 decision shift)."""
+    B, T, Hq, Hkv, D, w = 2, 60, 4, 2, 16, 8
+    q, k, v = rand_qkv(53, B, T, Hq, Hkv, D)
+    a = np.where(np.random.default_rng(54).random((B, Hkv, T)) < 0.5, -1.0, 1.0)
+    _, hard, pen = O.train_gate(a, None, 1e-4)    # |l| = 1e4: penalty 0 or about -1e4
+    o = O.train_attention(q, k, v, pen, w)
+    marks = np.zeros((B, Hkv, T), np.uint8)
+    marks[:, :, 1:] = hard[:, :, :-1]
+    assert np.allclose(o, O.prefill_attention(q, k, v, marks, w), rtol=0, atol=1e-12)
