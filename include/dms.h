@@ -396,6 +396,32 @@ DMS_API int dms_decode_attention(dms_cache* cache, int layer, const void* q, voi
  *    results; order them. */
 DMS_API int dms_decode_attention_noalloc(dms_cache* cache, int layer, const void* q, void* o, void* stream);
 
+/* ---- training mode (forward) ------------------------------------------------------
+ * [DMS-Qwen3] "Gumbel 噪声与可微门控" and "注意力实现": while the eviction
+ * adapter is trained, decisions are soft.  Both calls use only the cache's
+ * shape (B, Hq, Hkv, D, window) and none of its state.
+ *
+ * dms_train_gate: for each of the B*Hkv rows of T tokens, l = (alpha + noise)
+ * / tau (tau = 0.1 on the page; noise drawn by the caller, NULL for none),
+ * prob = sigmoid(l), hard = 1 if l > 0 else 0 -- the forward value of the
+ * straight-through decision (prob > 0.5) - prob + prob -- and the eviction
+ * penalty of the attention, taken from the logits shifted right by one
+ * position: penalty[t] = logsigmoid(-l[t-1]) = log(1 - prob[t-1]),
+ * penalty[0] = 0.  alpha, noise, prob, hard, penalty: device [B,Hkv,T] fp32.
+ * DMS_ERR_INVALID for a null pointer, T <= 0 or tau not positive and finite.
+ *
+ * dms_train_attention: the soft-gated attention of the training score_mod:
+ * query i and key j <= i score q.k / sqrt(D), plus penalty[b,h,j] when j is
+ * outside the window (i - j >= w); causal violations (mask value -50000) carry
+ * no weight; o = softmax(scores) v over every key, on the tensor cores.
+ * q/o [B,T,Hq,D], k/v [B,T,Hkv,D] bf16 (16-byte aligned), penalty [B,Hkv,T]
+ * fp32.  Needs bf16 activations and Hq/Hkv a power of two up to 16
+ * (DMS_ERR_INVALID otherwise). */
+DMS_API int dms_train_gate(dms_cache* cache, int seq_len, const float* alpha, const float* noise, float tau,
+                           float* prob, float* hard, float* penalty, void* stream);
+DMS_API int dms_train_attention(dms_cache* cache, int seq_len, const void* q, const void* k, const void* v,
+                                const float* penalty, void* o, void* stream);
+
 /* Self-check of the device failure path (the pages have no counterpart): one
  * thread waits, with the same bounded wait every kernel of the library uses,
  * on a shared-memory barrier that nothing ever completes, gives up after

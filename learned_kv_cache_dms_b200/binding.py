@@ -96,18 +96,20 @@ _lib.dms_decode_attention_noalloc.argtypes = [_P, C.c_int, _P, _P, _P]
 _lib.dms_cache_positions.argtypes = [_P, C.c_int]
 _lib.dms_selftest_wait_timeout.argtypes = [_P, C.c_int, _P]
 _lib.dms_decode_step_layers.argtypes = [_P, C.c_int, C.c_int, C.POINTER(dms_decode_args), _P]
+_lib.dms_train_gate.argtypes = [_P, C.c_int, _P, _P, C.c_float, _P, _P, _P, _P]
+_lib.dms_train_attention.argtypes = [_P, C.c_int, _P, _P, _P, _P, _P, _P]
 for _f in ("dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset", "dms_cache_get_layout",
            "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step", "dms_cache_positions",
            "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append", "dms_decode_attention",
            "dms_decode_attention_noalloc", "dms_cache_export", "dms_selftest_wait_timeout",
-           "dms_decode_step_layers"):
+           "dms_decode_step_layers", "dms_train_gate", "dms_train_attention"):
     getattr(_lib, _f).restype = C.c_int
 
 EXPORTED = ("dms_cache_desc_default", "dms_cache_bytes", "dms_cache_alloc", "dms_cache_free", "dms_cache_reset",
             "dms_cache_get_layout", "dms_cache_status", "dms_decide", "dms_prefill", "dms_decode_step",
             "dms_cache_positions", "dms_prefill_compact", "dms_prefill_attention", "dms_decode_append",
             "dms_decode_attention", "dms_decode_attention_noalloc", "dms_cache_export",
-            "dms_selftest_wait_timeout", "dms_decode_step_layers")
+            "dms_selftest_wait_timeout", "dms_decode_step_layers", "dms_train_gate", "dms_train_attention")
 
 
 def _check(code, where):
@@ -227,6 +229,16 @@ def dms_cache_positions(handle: int, layer: int) -> int:
 def dms_decode_step_layers(handle: int, layer: int, num_layers: int, args: dms_decode_args, stream=None) -> None:
     _check(_lib.dms_decode_step_layers(handle, layer, num_layers, C.byref(args), _stream(stream)),
            "dms_decode_step_layers")
+
+
+def dms_train_gate(handle: int, seq_len: int, alpha, noise, tau: float, prob, hard, penalty, stream=None) -> None:
+    _check(_lib.dms_train_gate(handle, seq_len, _ptr(alpha), _ptr(noise), float(tau), _ptr(prob), _ptr(hard),
+                               _ptr(penalty), _stream(stream)), "dms_train_gate")
+
+
+def dms_train_attention(handle: int, seq_len: int, q, k, v, penalty, o, stream=None) -> None:
+    _check(_lib.dms_train_attention(handle, seq_len, _ptr(q), _ptr(k), _ptr(v), _ptr(penalty), _ptr(o),
+                                    _stream(stream)), "dms_train_attention")
 
 
 def dms_selftest_wait_timeout(handle: int, tries: int, stream=None) -> None:

@@ -475,6 +475,9 @@ int dms_decide(dms_cache* c, int T, const dms_decide_params* d, void* neuron_src
 // pointers must be 16-byte aligned.
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+static void prefill_maps(const dms_cache* c, int T, const void* q, const void* k, const void* v, void* o,
+                         PrefillMaps* out);
+
 static int check_prefill(const dms_cache* c, int layer, const dms_prefill_args* a) {
   if (!c || !a || layer < 0 || layer >= c->desc.num_layers) return DMS_ERR_INVALID;
   const int T = a->seq_len;
@@ -539,12 +542,24 @@ int dms_prefill_attention(dms_cache* c, int layer, const dms_prefill_args* a, vo
     return DMS_ERR_STATE;
   const int T0 = c->compacted_pos0;
   track_launch(c, layer, static_cast<cudaStream_t>(stream));
-  // tensor maps of this call's q, k, v for the tcgen05 kernel
   PrefillMaps maps{};
+  prefill_maps(c, a->seq_len, a->q, a->k, a->v, a->o, &maps);
+  if (T0 > 0 && !maps.valid) return DMS_ERR_INVALID;
+  if (launch_prefill_attention(c->view, T0, a->seq_len, a->q, a->k, a->v, a->o, &maps,
+                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DMS_ERR_CUDA;
+  return DMS_OK;
+}
+
+// Tensor maps of one call's q, k, v, o for the tcgen05 attention (valid only
+// for bf16 activations and a GQA group that is a power of two up to 16).
+static void prefill_maps(const dms_cache* c, int T, const void* q, const void* k, const void* v, void* o,
+                         PrefillMaps* out) {
+  PrefillMaps& maps = *out;
   maps.valid = false;
   const int g = c->desc.num_q_heads / c->desc.num_kv_heads;
   if (c->has_kept_maps && g <= 16 && (g & (g - 1)) == 0) {
-    const int D = c->desc.head_dim, T = a->seq_len;
+    const int D = c->desc.head_dim;
     const cuuint64_t bt = static_cast<cuuint64_t>(c->desc.batch) * T;
     const cuuint64_t qd[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(c->desc.num_q_heads), bt};
     const cuuint64_t qs[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(c->desc.num_q_heads) * D * 2};
@@ -557,16 +572,34 @@ int dms_prefill_attention(dms_cache* c, int layer, const dms_prefill_args* a, vo
                               static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(c->desc.batch)};
     const cuuint64_t os[3] = {qs[0], qs[1], qs[1] * T};
     const cuuint32_t ob[4] = {64u, static_cast<cuuint32_t>(g), static_cast<cuuint32_t>(128 / g), 1u};
-    maps.valid = make_bf16_map(&maps.q, a->q, 3, qd, qs, qb) && make_bf16_map(&maps.k, a->k, 3, kd, ks, kbx) &&
-                 make_bf16_map(&maps.v, a->v, 3, kd, ks, kbx) && make_bf16_map(&maps.o, a->o, 4, od, os, ob);
+    maps.valid = make_bf16_map(&maps.q, q, 3, qd, qs, qb) && make_bf16_map(&maps.k, k, 3, kd, ks, kbx) &&
+                 make_bf16_map(&maps.v, v, 3, kd, ks, kbx) && make_bf16_map(&maps.o, o, 4, od, os, ob);
     maps.kept_k = c->kept_kmap;
     maps.kept_v = c->kept_vmap;
     maps.win_k = c->win_kmap;
     maps.win_v = c->win_vmap;
   }
-  if (T0 > 0 && !maps.valid) return DMS_ERR_INVALID;
-  if (launch_prefill_attention(c->view, T0, a->seq_len, a->q, a->k, a->v, a->o, &maps,
-                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
+}
+
+int dms_train_gate(dms_cache* c, int T, const float* alpha, const float* noise, float tau, float* prob, float* hard,
+                   float* penalty, void* stream) {
+  if (!c || !alpha || !prob || !hard || !penalty || T <= 0) return DMS_ERR_INVALID;
+  if (!(tau > 0.0f) || !(tau < INFINITY)) return DMS_ERR_INVALID;
+  if (launch_train_gate(static_cast<long>(c->desc.batch) * c->desc.num_kv_heads, T, alpha, noise, tau, prob, hard,
+                        penalty, c->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DMS_ERR_CUDA;
+  return DMS_OK;
+}
+
+int dms_train_attention(dms_cache* c, int T, const void* q, const void* k, const void* v, const float* penalty,
+                        void* o, void* stream) {
+  if (!c || !q || !k || !v || !o || !penalty || T <= 0) return DMS_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DMS_ERR_INVALID;
+  PrefillMaps maps{};
+  prefill_maps(c, T, q, k, v, o, &maps);
+  if (!maps.valid) return DMS_ERR_INVALID;  // bf16 activations, g a power of two up to 16
+  track_launch(c, -1, static_cast<cudaStream_t>(stream));
+  if (launch_prefill_attention_tc(c->view, 0, T, o, maps, static_cast<cudaStream_t>(stream), penalty) != cudaSuccess)
     return DMS_ERR_CUDA;
   return DMS_OK;
 }

@@ -481,8 +481,12 @@ struct PrefillMaps {
 };
 cudaError_t launch_prefill_attention(const CacheView& c, int T0, int T, const void* q, const void* k, const void* v,
                                      void* o, const PrefillMaps* maps, cudaStream_t s);
+// pen: the training path's soft mode (every key before the window a prefix
+// key from the input rows, scored with its penalty); null: DMS-masked prefill
 cudaError_t launch_prefill_attention_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& maps,
-                                        cudaStream_t s);
+                                        cudaStream_t s, const float* pen = nullptr);
+cudaError_t launch_train_gate(long rows, int T, const float* alpha, const float* noise, float tau, float* prob,
+                              float* hard, float* penalty, int num_sms, cudaStream_t s);
 cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, const void* v, float* alpha,
                                  const DecideArgs* fused_decide, int num_sms, cudaStream_t s);
 cudaError_t launch_decode_attention(const CacheView& c, int layer, const void* q, void* o,

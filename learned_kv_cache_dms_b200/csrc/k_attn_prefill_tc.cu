@@ -230,12 +230,14 @@ __device__ __forceinline__ int use_late(int v) {
 }
 
 // kept_upto(bh, x) of item u's (batch, KV head) at position x = T0 + i0 + dx
-// (0 when x <= 0 or the item does not exist; x is clamped to T0 + T)
+// (0 when x <= 0 or the item does not exist; x is clamped to T0 + T).  In the
+// soft (training) mode every key is a prefix key: kept_upto(x) = x.
 __device__ __forceinline__ int pf_kept_upto(const CacheView& c, int T0, int T, int NP, int nblk, int nitems, int u,
-                                           int dx) {
+                                           int dx, bool soft) {
   if (u >= nitems) return 0;
   const int per = c.Hkv * c.B, blk = nblk - 1 - u / per, rem = u % per;
   const int x = min(T0 + blk * kPfQT * NP + dx, T0 + T);
+  if (soft) return max(x, 0);
   return x > 0 ? ld_early_i32(c.kept_upto + static_cast<long>((rem / c.Hkv) * c.Hkv + rem % c.Hkv) * (c.max_pos + 1) + x)
                : 0;
 }
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                       const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                       const __grid_constant__ CUtensorMap kkmap, const __grid_constant__ CUtensorMap kvmap,
                       const __grid_constant__ CUtensorMap wkmap, const __grid_constant__ CUtensorMap wvmap,
-                      const __grid_constant__ CUtensorMap omap) {
+                      const __grid_constant__ CUtensorMap omap, const float* pen) {
   using L = PfSmem<D>;
   constexpr int ST = L::ST;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -264,6 +266,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = c.Hq / c.Hkv, NP = kPfRows / g, w = c.w;
+  // soft mode (training attention, pen != null): every key at or before i - w
+  // is a prefix key read from the input rows, its score raised by pen[key]
+  const bool soft = pen != nullptr;
   const int nblk = (T + kPfQT * NP - 1) / (kPfQT * NP);
   const int nitems = nblk * c.Hkv * c.B, G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
   // item k of this CTA, and its nk (kept keys before i1 - w)
@@ -271,7 +276,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int u = pf_item_index(k, G, cta);
     if (u >= nitems) return 0;
     const int i0 = (nblk - 1 - u / (c.Hkv * c.B)) * kPfQT * NP, i1 = min(T, i0 + kPfQT * NP);
-    return pf_kept_upto(c, T0, T, NP, nblk, nitems, u, i1 - i0 - w);
+    return pf_kept_upto(c, T0, T, NP, nblk, nitems, u, i1 - i0 - w, soft);
   };
   auto item = [&](int k, int nk) { return pf_item(c, T0, T, NP, nblk, nitems, pf_item_index(k, G, cta), nk); };
 
@@ -333,7 +338,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           mbar_expect_tx(&k_full[st], L::KV_BYTES);
           for (int hf = 0; hf < L::HALVES; ++hf) {
             unsigned char* dk = sb + L::OFF_K + st * L::KV_BYTES + hf * (kPfBN * 128);
-            if (src == 0)
+            if (src == 0 && soft)
+              tma_load_3d(dk, &kmap, hf * 64, it.h, it.b * T + jb, &k_full[st]);
+            else if (src == 0)
               tma_load_2d(dk, &kkmap, hf * 64, it.bh * c.max_pos + jb, &k_full[st]);
             else if (src == 1)
               tma_load_2d(dk, &wkmap, hf * 64, it.bh * w + (jb - (T0 - w)), &k_full[st]);
@@ -362,7 +369,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           mbar_expect_tx(&v_full[st], L::KV_BYTES);
           for (int hf = 0; hf < L::HALVES; ++hf) {
             unsigned char* dv = sb + L::OFF_V + st * L::KV_BYTES + hf * (kPfBN * 128);
-            if (src == 0)
+            if (src == 0 && soft)
+              tma_load_3d(dv, &vmap, hf * 64, it.h, it.b * T + jb, &v_full[st]);
+            else if (src == 0)
               tma_load_2d(dv, &kvmap, hf * 64, it.bh * c.max_pos + jb, &v_full[st]);
             else if (src == 1)
               tma_load_2d(dv, &wvmap, hf * 64, it.bh * w + (jb - (T0 - w)), &v_full[st]);
@@ -452,7 +461,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // the row's count of visible kept keys: kept-list entries [0, ck) are the
     // positions <= i - w
     auto kept_visible = [&](int k) {
-      return pf_kept_upto(c, T0, T, NP, nblk, nitems, pf_item_index(k, G, cta), p_row - w + 1);
+      return pf_kept_upto(c, T0, T, NP, nblk, nitems, pf_item_index(k, G, cta), p_row - w + 1, soft);
     };
     bool ok = true;
     int t = 0;
@@ -508,6 +517,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
           for (int n = 0; n < kPfBN; ++n)
             sv[n] = (((n < 32 ? m0 : m1) >> (n & 31)) & 1u) ? __uint_as_float(sr[n]) : -INFINITY;
+        }
+        if (soft && kt && c_lo <= c_hi) {
+          // penalty of the prefix keys, in raw-score units (the softmax works
+          // in s * log2(e) / sqrt(D))
+          const float* pr = pen + static_cast<long>(it.bh) * T + jb;
+          const float rs = sqrtf(static_cast<float>(D));
+#pragma unroll
+          for (int n = 0; n < kPfBN; ++n)
+            if (n >= c_lo && n <= c_hi) sv[n] = fmaf(__ldg(pr + n), rs, sv[n]);
         }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -628,7 +646,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 }
 
 template <int D>
-static cudaError_t launch_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& m, cudaStream_t s) {
+static cudaError_t launch_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& m, cudaStream_t s,
+                             const float* pen) {
   const size_t smem = PfSmem<D>::BYTES + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_attn_prefill_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -637,13 +656,42 @@ static cudaError_t launch_tc(const CacheView& c, int T0, int T, void* o, const P
   const long nitems = static_cast<long>((T + kPfQT * NP - 1) / (kPfQT * NP)) * c.Hkv * c.B;
   const int grid = static_cast<int>(min(nitems, static_cast<long>(c.num_sms)));  // persistent: one CTA per SM
   k_attn_prefill_tc<D><<<grid, kPfThreads, smem, s>>>(c, T0, T, static_cast<__nv_bfloat16*>(o), m.q, m.k, m.v,
-                                                      m.kept_k, m.kept_v, m.win_k, m.win_v, m.o);
+                                                      m.kept_k, m.kept_v, m.win_k, m.win_v, m.o, pen);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_attention_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& maps,
-                                        cudaStream_t s) {
-  return c.D == 64 ? launch_tc<64>(c, T0, T, o, maps, s) : launch_tc<128>(c, T0, T, o, maps, s);
+                                        cudaStream_t s, const float* pen) {
+  return c.D == 64 ? launch_tc<64>(c, T0, T, o, maps, s, pen) : launch_tc<128>(c, T0, T, o, maps, s, pen);
+}
+
+// ---------------------------------------------------------------------------
+// Gate of the training path, one thread per token: l = (alpha + noise) / tau,
+// prob = sigmoid(l), hard = 1 if l > 0 else 0 (the forward value of the
+// straight-through decision, prob > 0.5), and the penalty of the next
+// position, logsigmoid(-l) (position 0 of each row gets 0).
+// ---------------------------------------------------------------------------
+__global__ void k_train_gate(long n, int T, const float* alpha, const float* noise, float tau, float* prob,
+                             float* hard, float* penalty) {
+  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const float l = __fdiv_rn(alpha[i] + (noise ? noise[i] : 0.f), tau);
+    prob[i] = 1.0f / (1.0f + expf(-l));
+    hard[i] = l > 0.f ? 1.0f : 0.0f;
+    // logsigmoid(-l) = -log(1 + exp(l)), without overflow for large l
+    const float ls = l > 0.f ? -(l + log1pf(expf(-l))) : -log1pf(expf(l));
+    const int t = static_cast<int>(i % T);
+    if (t + 1 < T) penalty[i + 1] = ls;
+    if (t == 0) penalty[i] = 0.f;
+  }
+}
+
+cudaError_t launch_train_gate(long rows, int T, const float* alpha, const float* noise, float tau, float* prob,
+                              float* hard, float* penalty, int num_sms, cudaStream_t s) {
+  const long n = rows * T;
+  const int grid = static_cast<int>(max(1L, min((n + 255) / 256, static_cast<long>(num_sms) * 8)));
+  k_train_gate<<<grid, 256, 0, s>>>(n, T, alpha, noise, tau, prob, hard, penalty);
+  return cudaGetLastError();
 }
 
 }  // namespace dms
