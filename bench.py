@@ -38,6 +38,7 @@ Multi-GPU (torchrun): every rank runs its own replica (independent sequences,
 weak scaling, no collective on the data path); rank 0 prints one JSON line.
 """
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -180,7 +181,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------
-BENCH_WORKLOADS = ("qwen8b", "qwen8b_c8", "llama1b", "llama1b_layer", "reason36")
+BENCH_WORKLOADS = ("qwen8b", "qwen8b_c8", "llama1b", "llama1b_layer", "reason36", "kvzap8b")
 STEP_POOL = 64  # distinct decode-token inputs per layer of a multi-layer stack (cycled)
 
 
@@ -206,14 +207,15 @@ def make_desc(B_, wl, kernel="auto"):
     d.pool_pages = wl.layers * wl.batch * wl.kv_heads * min(maxp, max(pre, need))
     d.act_dtype = B_.DMS_BF16
     d.kv_dtype = {"bf16": B_.DMS_BF16, "fp8": B_.DMS_FP8_E4M3}[wl.kv_dtype]
-    d.alpha_source = {"proj": B_.DMS_ALPHA_PROJ, "key": B_.DMS_ALPHA_KEY_NEURON}[wl.alpha_source]
+    d.alpha_source = {"proj": B_.DMS_ALPHA_PROJ, "key": B_.DMS_ALPHA_KEY_NEURON,
+                      "score": B_.DMS_ALPHA_SCORE_LINEAR}[wl.alpha_source]
     d.alpha_per = B_.DMS_ALPHA_PER_LAYER if wl.alpha_per == "layer" else B_.DMS_ALPHA_PER_HEAD
     return d
 
 
 def decode_launches_per_step(wl):
     """Kernels one dms_decode_step launches per layer."""
-    pre = 1 if (wl.alpha_source != "proj" or wl.rope) else 0  # decision neuron / rotary pass
+    pre = 1 if (wl.alpha_source not in ("proj", "score") or wl.rope) else 0  # decision neuron / rotary pass
     if wl.kv_dtype == "fp8":
         return pre + 2  # append (re-encodes pages), then the cluster attention
     return pre + 1      # one fused kernel: decision, attention, combine, append
@@ -296,7 +298,8 @@ class Runner:
         self.R = replicas or replicas_for(wl, l2)
         self.caches = [B_.Cache(self.desc) for _ in range(self.R)]
         self.cache = self.caches[0]
-        self.neuron = wl.alpha_source != "proj"
+        self.neuron = wl.alpha_source not in ("proj", "score")
+        self.score = wl.alpha_source == "score"
         # the compaction and the decode step rewrite q and k in place (neuron
         # zeroing, rotary): such inputs get a copy per replica, restored from
         # pristine copies outside the timed segments
@@ -375,7 +378,7 @@ class Runner:
         x = dict(q=rn(B, T, Hq, D), k=rn(B, T, H, D), v=rn(B, T, H, D),
                  qd=rn(P, B, Hq, D), kd=rn(P, B, H, D), vd=rn(P, B, H, D))
         if not self.neuron:
-            x.update(h=rn(B, T, wl.hidden), hd=rn(P, B, wl.hidden), gamma=rn(wl.hidden),
+            x.update(h=rn(B, T, wl.hidden), hd=rn(P, B, wl.hidden), gamma=None if self.score else rn(wl.hidden),
                      W=rn(H, wl.hidden, std=wl.hidden ** -0.5))
         # offsets that keep the workload's fraction of tokens per (b, h)
         keep = I.keep_fractions(wl, seed)
@@ -391,7 +394,9 @@ class Runner:
             raw = np.broadcast_to(raw[:, :1], raw.shape)
             keep = np.broadcast_to(keep[:, :1], keep.shape)
         off, _ = I.calibrate_offsets(raw, keep)
-        x["off"] = torch.from_numpy(off).cuda()
+        # the score source marks a token when threshold - score > 0: with a
+        # zero threshold the logit is -score, so the threshold is -offset
+        x["off"] = torch.from_numpy(-off if self.score else off).cuda()
         if self.neuron:
             x["pdec"] = B_.decide_params(x["off"])
             x["ddec"] = [x["pdec"]] * P
@@ -561,8 +566,8 @@ def decode_step_bytes(wl, retained):
     pages = -(-retained // wl.block)  # a lower bound on pages touched
     per_page = 4 + (8 if wl.kv_dtype == "fp8" else 0)
     fixed = L * (2 * B * wl.q_heads * D * 2 + 2 * BH * D * 2 + 2 * BH * D * elem)
-    if wl.alpha_source == "proj":
-        fixed += L * (B * wl.hidden * 2 + wl.kv_heads * wl.hidden * 2 + wl.hidden * 2)
+    if wl.alpha_source in ("proj", "score"):
+        fixed += L * (B * wl.hidden * 2 + wl.kv_heads * wl.hidden * 2 + (wl.hidden * 2 if wl.alpha_source == "proj" else 0))
     return retained * D * 2 * elem + pages * per_page + fixed
 
 
@@ -574,7 +579,7 @@ def measure_prefill_parts(B_, r, wl, passes=3):
     u = r.units[0]
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     alpha = torch.empty_like(u["alpha"])
-    proj = wl.alpha_source == "proj"
+    proj = wl.alpha_source in ("proj", "score")
     dec, comp = [], []
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     for i in range(passes):
@@ -713,9 +718,10 @@ def run_ours(args, world, rank, local, primary=True):
     ret_prefill = counts[0] / L  # retained slots of one layer after the prefill
     kv_in = 2  # bf16 K/V input rows
     kv_page = 1 if wl.kv_dtype == "fp8" else 2
-    dec_bytes = B * T_ * wl.hidden * 2 + wl.kv_heads * wl.hidden * 2 + wl.hidden * 2 + B * wl.kv_heads * T_ * 4
+    dec_bytes = (B * T_ * wl.hidden * 2 + wl.kv_heads * wl.hidden * 2 + B * wl.kv_heads * T_ * 4 +
+                 (wl.hidden * 2 if wl.alpha_source == "proj" else 0))
     comp_bytes = B * wl.kv_heads * T_ * 4 + ret_prefill * wl.head_dim * 2 * (kv_in + kv_page)
-    neuron_pass = wl.alpha_source != "proj"
+    neuron_pass = wl.alpha_source not in ("proj", "score")
     if neuron_pass:  # q and k rewritten in place by the neuron/rotary pass, inside the compaction call
         comp_bytes += 2 * B * T_ * (wl.q_heads + wl.kv_heads) * wl.head_dim * 2
     comp_only_ms = comp_ms1 - (dec_ms1 or 0.0)
@@ -723,7 +729,8 @@ def run_ours(args, world, rank, local, primary=True):
         "bound": "hbm", "achieved": round(dec_bytes / (dec_ms1 / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
         "frac": round(dec_bytes / (dec_ms1 / 1e3) / 1e9 / pk["hbm_gbs"], 4), "ms": round(dec_ms1, 4),
         "algorithmic_bytes": int(dec_bytes),
-        "kernel": "k_decide_proj_tc (adapter RMSNorm + linear) via dms_decide, L2-cold"}
+        "kernel": "k_decide_proj_tc (%s) via dms_decide, L2-cold"
+                  % ("importance score: linear, no norm" if wl.alpha_source == "score" else "adapter RMSNorm + linear")}
     compact_roof = {
         "bound": "hbm", "achieved": round(comp_bytes / (comp_only_ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"],
         "unit": "GB/s", "frac": round(comp_bytes / (comp_only_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
@@ -996,6 +1003,143 @@ def cpu_baseline(wl, seconds):
                                   % (wl.prompt, replay_s, prow, pattn_s, wl.batch * wl.prompt * wl.q_heads)}}
 
 
+def _flush_l2(buf, i):
+    buf.fill_(i & 0xFF)
+
+
+def _med(x):
+    return sorted(x)[len(x) // 2]
+
+
+def measure_chunked_prefill(B_, pk, passes=3, chunk=4096, n_chunks=3):
+    """Chunked prefill on the Qwen3-8B layer shape: a 12288-token prompt
+    prefilled as three calls of 4096 (each dms_prefill_compact, then
+    dms_prefill_attention), against the same prompt in one call; adapter
+    decisions calibrated for keep 1/8.  L2 flushed before each pass (the chunks
+    of a pass run back to back).  Attention flops: 4 * D per visible (query,
+    key) pair of the prompt, the same for both."""
+    wl = I.WORKLOADS["qwen8b"]
+    T = chunk * n_chunks
+    g = torch.Generator(device="cuda")
+    g.manual_seed(wl.seed * 7 + 1)
+    bf = torch.bfloat16
+    B, Hq, H, D = wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim
+
+    def rn(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g, device="cuda", dtype=torch.float32) * std).to(bf)
+
+    q, k, v, h = rn(B, T, Hq, D), rn(B, T, H, D), rn(B, T, H, D), rn(B, T, wl.hidden)
+    gamma, W = rn(wl.hidden), rn(H, wl.hidden, std=wl.hidden ** -0.5)
+    d = make_desc(B_, dataclasses.replace(wl, prompt=T, decode_steps=16))
+    cache = B_.Cache(d)
+    raw = torch.empty(B, H, T, dtype=torch.float32, device="cuda")
+    B_.dms_decide(cache.handle, T, B_.decide_params(torch.zeros(B, H, device="cuda"), hidden=h, norm_weight=gamma,
+                                                    proj_weight=W), None, raw)
+    off, _ = I.calibrate_offsets(raw.cpu().numpy(), I.keep_fractions(wl))
+    off = torch.from_numpy(off).cuda()
+    o = torch.empty_like(q)
+    alpha = torch.empty(B, H, T, dtype=torch.float32, device="cuda")
+    parts = []
+    for c0 in range(0, T, chunk):
+        sl = slice(c0, c0 + chunk)
+        qc, kc, vc, hc = (x[:, sl].contiguous() for x in (q, k, v, h))
+        oc, ac = torch.empty_like(qc), torch.empty(B, H, chunk, dtype=torch.float32, device="cuda")
+        dp = B_.decide_params(off, hidden=hc, norm_weight=gamma, proj_weight=W)
+        parts.append(dict(keep=(qc, kc, vc, hc, oc, ac, dp), args=B_.Cache.prefill_args(qc, kc, vc, oc, ac, dp)))
+    whole = B_.Cache.prefill_args(q, k, v, o, alpha, B_.decide_params(off, hidden=h, norm_weight=gamma, proj_weight=W))
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    ch_comp, ch_attn, one = [], [], []
+    for it in range(passes + 1):
+        cache.reset()
+        _flush_l2(flush, it)
+        ev = [(E(), E(), E()) for _ in parts]
+        for (e0, e1, e2), pt in zip(ev, parts):
+            e0.record()
+            B_.dms_prefill_compact(cache.handle, 0, pt["args"])
+            e1.record()
+            B_.dms_prefill_attention(cache.handle, 0, pt["args"])
+            e2.record()
+        cache.reset()
+        _flush_l2(flush, it + 50)
+        a0, a1 = E(), E()
+        a0.record()
+        B_.dms_prefill(cache.handle, 0, whole)
+        a1.record()
+        torch.cuda.synchronize()
+        if it == 0:
+            continue
+        ch_comp.append(sum(e0.elapsed_time(e1) for e0, e1, _ in ev))
+        ch_attn.append(sum(e1.elapsed_time(e2) for _, e1, e2 in ev))
+        one.append(a0.elapsed_time(a1))
+    assert cache.status() == 0
+    pairs = visible_pairs(alpha, dataclasses.replace(wl, prompt=T))
+    flops = 4.0 * D * wl.gqa * pairs
+    tot = _med([a + b for a, b in zip(ch_comp, ch_attn)])
+    att = _med(ch_attn)
+    tf = flops / (att / 1e3) / 1e12
+    cache.close()
+    return {"workload": "qwen8b_layer_b1_prompt%d_in_%d_chunks_of_%d" % (T, n_chunks, chunk),
+            "prefill_tok_s": round(B * T / (tot / 1e3), 1), "ms": round(tot, 4),
+            "compact_ms": round(_med(ch_comp), 4), "attention_ms": round(att, 4),
+            "one_call_ms": round(_med(one), 4),
+            "attention": {"bound": "tensor", "achieved": round(tf, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                          "frac": round(tf / pk["bf16_tflops"], 4), "flops": flops,
+                          "kernel": "k_attn_prefill_tc<128> with the window copy of the previous chunk"},
+            "passes": passes, "l2": "512 MB written before each pass"}
+
+
+def measure_train_attention(B_, pk, passes=3):
+    """The training path on the Qwen3-8B layer shape, 8192 tokens: the gate
+    (dms_train_gate) and the soft-gated attention (dms_train_attention), each
+    after an L2 flush, median of `passes`.  Algorithmic flops: 4 * D per causal
+    (query, key) pair, every key visible (dense causal)."""
+    wl = I.WORKLOADS["qwen8b"]
+    T, B, Hq, H, D = wl.prompt, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim
+    g = torch.Generator(device="cuda")
+    g.manual_seed(wl.seed * 7 + 2)
+    bf = torch.bfloat16
+    q, k, v = (torch.randn(*s_, generator=g, device="cuda").to(bf) for s_ in ((B, T, Hq, D), (B, T, H, D), (B, T, H, D)))
+    alpha = torch.randn(B, H, T, generator=g, device="cuda") * 2 - 0.5
+    u = torch.rand(B, H, T, generator=g, device="cuda").clamp(1e-6, 1 - 1e-6)
+    noise = torch.log(u) - torch.log1p(-u)
+    cache = B_.Cache(make_desc(B_, wl))
+    prob, hard, pen = (torch.empty(B, H, T, device="cuda") for _ in range(3))
+    o = torch.empty_like(q)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    tg, ta = [], []
+    for it in range(passes + 1):
+        _flush_l2(flush, it)
+        e0, e1, e2, e3 = E(), E(), E(), E()
+        e0.record()
+        B_.dms_train_gate(cache.handle, T, alpha, noise, 0.1, prob, hard, pen)
+        e1.record()
+        _flush_l2(flush, it + 50)
+        e2.record()
+        B_.dms_train_attention(cache.handle, T, q, k, v, pen, o)
+        e3.record()
+        torch.cuda.synchronize()
+        if it:
+            tg.append(e0.elapsed_time(e1))
+            ta.append(e2.elapsed_time(e3))
+    assert cache.status() == 0
+    cache.close()
+    flops = 4.0 * D * Hq * B * T * (T + 1) / 2
+    keep_all = -torch.ones(B, H, T)
+    tiles = executed_tile_flops(keep_all, wl)
+    att = _med(ta)
+    tf = flops / (att / 1e3) / 1e12
+    return {"workload": "qwen8b_layer_b1_T%d_dense_causal" % T, "gate_ms": round(_med(tg), 4),
+            "attention_ms": round(att, 4), "tok_s": round(B * T / (att / 1e3), 1),
+            "attention": {"bound": "tensor", "achieved": round(tf, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                          "frac": round(tf / pk["bf16_tflops"], 4), "flops": flops,
+                          "frac_executed_tiles": round(tiles / (att / 1e3) / 1e12 / pk["bf16_tflops"], 4),
+                          "executed_over_algorithmic": round(tiles / flops, 4),
+                          "kernel": "k_attn_prefill_tc<128>, soft mode (penalty on keys outside the window)"},
+            "passes": passes, "l2": "512 MB written before each kernel"}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return None
@@ -1020,7 +1164,7 @@ def run_reference(args, world, rank):
             "e2e": {"value": round(val, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-SECONDARY = (("qwen8b_c8", None), ("llama1b", None), ("llama1b_layer", None), ("reason36", 512))
+SECONDARY = (("qwen8b_c8", None), ("llama1b", None), ("llama1b_layer", None), ("reason36", 512), ("kvzap8b", None))
 SECONDARY_KEYS = ("value", "unit", "steps", "warmup", "ms_per_step", "config", "roofline", "retained_kv_gbps",
                   "retained_per_head", "decode_ms_per_token_step", "decode_step_us_single", "prefill_tok_s",
                   "prefill_ms", "prefill_compact_ms", "prefill_attention_ms", "prefill_attention", "decide",
@@ -1050,6 +1194,14 @@ def main():
             rec = run_ours(sub, world, rank, local, primary=False)
             line["secondary"][name] = {k: rec[k] for k in SECONDARY_KEYS if k in rec}
             torch.cuda.empty_cache()
+        # the rows beyond the first prefill-then-decode: chunked prefill and
+        # the training path's forward
+        from learned_kv_cache_dms_b200 import binding as B_
+        pk, _ = peaks()
+        line["next"] = {"chunked_prefill": measure_chunked_prefill(B_, pk)}
+        torch.cuda.empty_cache()
+        line["next"]["train_attention"] = measure_train_attention(B_, pk)
+        torch.cuda.empty_cache()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

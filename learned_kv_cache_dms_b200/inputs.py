@@ -18,6 +18,9 @@ no model weights or datasets are used):
            last key neuron, rotary tables; run per head and per layer.
   reason36 bf16, 36 independent layers, B32, prompt 1024 + 16384 steps, w512,
            block 256, keep 1/16, decisions online every step.
+  kvzap8b  bf16, Llama-3.1-8B attention shape, B1, prompt 8192 + 128 steps,
+           importance-score decisions (Linear, no norm, threshold), w128,
+           block 64, keep 1/4.
 """
 from __future__ import annotations
 
@@ -45,7 +48,7 @@ class Workload:
     kv_dtype: str           # "f32" | "bf16" | "fp8"
     keep: float             # mean keep fraction outside the window
     keep_range: tuple | None = None   # per-(b,h) keep ~ U[lo, hi]
-    alpha_source: str = "proj"        # "proj" | "key" | "query"
+    alpha_source: str = "proj"        # "proj" | "key" | "query" | "score"
     alpha_per: str = "head"           # "head" | "layer"
     rope: bool = False
     prealloc_tokens: int = 4096
@@ -74,6 +77,11 @@ WORKLOADS = {
                               seed=1004),
     "reason36": Workload("reason36", 36, 32, 4096, 32, 8, 128, 1024, 16384, 512, 256, "bf16", "bf16",
                          1 / 16, seed=1005),
+    # the importance-score source on the Llama-3.1-8B attention shape (the
+    # KVzap-linear page: hidden 4096 -> 8 KV-head scores, threshold pruning
+    # outside the last 128 tokens), batch 1, 8192 + 128, keep 1/4
+    "kvzap8b": Workload("kvzap8b", 1, 1, 4096, 32, 8, 128, 8192, 128, 128, 64, "bf16", "bf16", 1 / 4,
+                        alpha_source="score", seed=1006),
 }
 
 TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
