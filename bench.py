@@ -68,6 +68,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiler runs)")
+    p.add_argument("--measure", choices=["train_attention", "chunked_prefill"], default=None,
+                   help="run one of the extra measurements alone and print its record (profiler captures)")
     p.add_argument("--no-secondary", action="store_true",
                    help="measure only --workload (the default run also measures the other workloads)")
     p.add_argument("--workload", choices=BENCH_WORKLOADS, default="qwen8b",
@@ -1181,6 +1183,12 @@ def main():
             print(json.dumps(line), flush=True)
         return
     world, rank, local = dist_setup()
+    if args.measure:
+        from learned_kv_cache_dms_b200 import binding as B_
+        pk, _ = peaks()
+        fn = {"train_attention": measure_train_attention, "chunked_prefill": measure_chunked_prefill}[args.measure]
+        print(json.dumps({args.measure: fn(B_, pk)}), flush=True)
+        return
     line = run_ours(args, world, rank, local)
     if world == 1 and args.workload == "qwen8b" and not args.no_secondary:
         # the other workloads, measured in the same run (device-timed legs);

@@ -598,8 +598,22 @@ int dms_train_attention(dms_cache* c, int T, const void* q, const void* k, const
   PrefillMaps maps{};
   prefill_maps(c, T, q, k, v, o, &maps);
   if (!maps.valid) return DMS_ERR_INVALID;  // bf16 activations, g a power of two up to 16
+  // the penalties as a [B*Hkv, T] fp32 tensor map (rows of 16-byte multiples)
+  CUtensorMap pm;
+  bool have_pm = false;
+  if (T % 4 == 0 && (reinterpret_cast<uintptr_t>(penalty) & 15) == 0) {
+    auto enc = tensor_map_encoder();
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(T),
+                                static_cast<cuuint64_t>(c->desc.batch) * c->desc.num_kv_heads};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(T) * 4};
+    const cuuint32_t box[2] = {64u, 1u}, estr[2] = {1u, 1u};
+    have_pm = enc && enc(&pm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(penalty), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   track_launch(c, -1, static_cast<cudaStream_t>(stream));
-  if (launch_prefill_attention_tc(c->view, 0, T, o, maps, static_cast<cudaStream_t>(stream), penalty) != cudaSuccess)
+  if (launch_prefill_attention_tc(c->view, 0, T, o, maps, static_cast<cudaStream_t>(stream), penalty,
+                                  have_pm ? &pm : nullptr) != cudaSuccess)
     return DMS_ERR_CUDA;
   return DMS_OK;
 }

@@ -483,8 +483,11 @@ cudaError_t launch_prefill_attention(const CacheView& c, int T0, int T, const vo
                                      void* o, const PrefillMaps* maps, cudaStream_t s);
 // pen: the training path's soft mode (every key before the window a prefix
 // key from the input rows, scored with its penalty); null: DMS-masked prefill
+// penmap: optional tensor map of pen as [B*Hkv rows, T] fp32 (box 64 x 1), when
+// T % 4 == 0: the penalties then come by TMA with the V tiles
 cudaError_t launch_prefill_attention_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& maps,
-                                        cudaStream_t s, const float* pen = nullptr);
+                                        cudaStream_t s, const float* pen = nullptr,
+                                        const CUtensorMap* penmap = nullptr);
 cudaError_t launch_train_gate(long rows, int T, const float* alpha, const float* noise, float tau, float* prob,
                               float* hard, float* penalty, int num_sms, cudaStream_t s);
 cudaError_t launch_decode_append(const CacheView& c, int layer, const void* k, const void* v, float* alpha,

@@ -248,7 +248,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                       const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                       const __grid_constant__ CUtensorMap kkmap, const __grid_constant__ CUtensorMap kvmap,
                       const __grid_constant__ CUtensorMap wkmap, const __grid_constant__ CUtensorMap wvmap,
-                      const __grid_constant__ CUtensorMap omap, const float* pen) {
+                      const __grid_constant__ CUtensorMap omap, const float* pen,
+                      const __grid_constant__ CUtensorMap penmap, int pen_tma) {
   using L = PfSmem<D>;
   constexpr int ST = L::ST;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -263,6 +264,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   // these)
   __shared__ float s_turn_zero;
   __shared__ float s_turn_sink[kPfQT];
+  // soft mode: the penalties of each V stage's prefix keys, loaded with the
+  // V tile (the stage is free again only after P V, so after the softmax used them)
+  __shared__ __align__(128) float s_pen[ST][kPfBN];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = c.Hq / c.Hkv, NP = kPfRows / g, w = c.w;
@@ -366,7 +370,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           int src;
           const int jb = pf_tile(it, j, src);
-          mbar_expect_tx(&v_full[st], L::KV_BYTES);
+          const bool pen_tile = soft && pen_tma && src == 0;
+          mbar_expect_tx(&v_full[st], L::KV_BYTES + (pen_tile ? kPfBN * 4 : 0));
+          if (pen_tile) tma_load_2d(&s_pen[st][0], &penmap, jb, it.bh, &v_full[st]);
           for (int hf = 0; hf < L::HALVES; ++hf) {
             unsigned char* dv = sb + L::OFF_V + st * L::KV_BYTES + hf * (kPfBN * 128);
             if (src == 0 && soft)
@@ -520,12 +526,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         if (soft && kt && c_lo <= c_hi) {
           // penalty of the prefix keys, in raw-score units (the softmax works
-          // in s * log2(e) / sqrt(D))
-          const float* pr = pen + static_cast<long>(it.bh) * T + jb;
+          // in s * log2(e) / sqrt(D)): from the V stage, else from global memory
           const float rs = sqrtf(static_cast<float>(D));
+          if (pen_tma) {
+            const int st = t % ST;
+            ok = ok && mbar_wait_bounded(&v_full[st], (t / ST) & 1);
+            const float* pr = &s_pen[st][0];
 #pragma unroll
-          for (int n = 0; n < kPfBN; ++n)
-            if (n >= c_lo && n <= c_hi) sv[n] = fmaf(__ldg(pr + n), rs, sv[n]);
+            for (int n = 0; n < kPfBN; ++n)
+              if (n >= c_lo && n <= c_hi) sv[n] = fmaf(pr[n], rs, sv[n]);
+          } else {
+            const float* pr = pen + static_cast<long>(it.bh) * T + jb;
+#pragma unroll
+            for (int n = 0; n < kPfBN; ++n)
+              if (n >= c_lo && n <= c_hi) sv[n] = fmaf(__ldg(pr + n), rs, sv[n]);
+          }
         }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -647,7 +662,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
 template <int D>
 static cudaError_t launch_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& m, cudaStream_t s,
-                             const float* pen) {
+                             const float* pen, const CUtensorMap* penmap) {
   const size_t smem = PfSmem<D>::BYTES + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_attn_prefill_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -656,13 +671,15 @@ static cudaError_t launch_tc(const CacheView& c, int T0, int T, void* o, const P
   const long nitems = static_cast<long>((T + kPfQT * NP - 1) / (kPfQT * NP)) * c.Hkv * c.B;
   const int grid = static_cast<int>(min(nitems, static_cast<long>(c.num_sms)));  // persistent: one CTA per SM
   k_attn_prefill_tc<D><<<grid, kPfThreads, smem, s>>>(c, T0, T, static_cast<__nv_bfloat16*>(o), m.q, m.k, m.v,
-                                                      m.kept_k, m.kept_v, m.win_k, m.win_v, m.o, pen);
+                                                      m.kept_k, m.kept_v, m.win_k, m.win_v, m.o, pen,
+                                                      penmap ? *penmap : m.o, penmap ? 1 : 0);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_attention_tc(const CacheView& c, int T0, int T, void* o, const PrefillMaps& maps,
-                                        cudaStream_t s, const float* pen) {
-  return c.D == 64 ? launch_tc<64>(c, T0, T, o, maps, s, pen) : launch_tc<128>(c, T0, T, o, maps, s, pen);
+                                        cudaStream_t s, const float* pen, const CUtensorMap* penmap) {
+  return c.D == 64 ? launch_tc<64>(c, T0, T, o, maps, s, pen, penmap)
+                   : launch_tc<128>(c, T0, T, o, maps, s, pen, penmap);
 }
 
 // ---------------------------------------------------------------------------
