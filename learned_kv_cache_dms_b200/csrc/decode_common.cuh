@@ -58,6 +58,31 @@ __device__ __forceinline__ void issue_subtile(unsigned char* dst, const CUtensor
   }
 }
 
+// Issue the TMA loads of `rows` slots (<= TROWS, starting at pool row `row0`,
+// all inside one page) into a stage of TROWS-row tiles: K then V, 16-row
+// boxes; bf16 rows as 128-byte column halves with the 128-byte swizzle (half
+// hf at hf * TROWS * 128), FP8 rows unswizzled.  Called by one thread;
+// completes on `bar` with the exact byte count.
+template <int D, bool FP8, int TROWS>
+__device__ __forceinline__ void issue_rows(unsigned char* dst, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                           int row0, int rows, uint64_t* bar) {
+  constexpr int HALVES = D / 64, TILE = FP8 ? TROWS * D : TROWS * D * 2;
+  const int nbox = (rows + 15) / 16;
+  mbar_expect_tx(bar, static_cast<uint32_t>(nbox * 16 * D * (FP8 ? 1 : 2) * 2));
+  for (int bx = 0; bx < nbox; ++bx) {
+    if (FP8) {
+      tma_load_2d(dst + bx * 16 * D, kmap, 0, row0 + bx * 16, bar);
+      tma_load_2d(dst + TILE + bx * 16 * D, vmap, 0, row0 + bx * 16, bar);
+    } else {
+#pragma unroll
+      for (int hf = 0; hf < HALVES; ++hf) {
+        tma_load_2d(dst + hf * TROWS * 128 + bx * 16 * 128, kmap, hf * 64, row0 + bx * 16, bar);
+        tma_load_2d(dst + TILE + hf * TROWS * 128 + bx * 16 * 128, vmap, hf * 64, row0 + bx * 16, bar);
+      }
+    }
+  }
+}
+
 // Widen a staged FP8 sub-tile (K then V, unswizzled rows of D codes) to bf16
 // codes (exact) in the 128-byte swizzled layout of `conv` (K then V).
 template <int D>
@@ -220,6 +245,135 @@ __device__ __forceinline__ void warp_tile(const unsigned char* kt, const unsigne
     uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
     mma_bf16_16816(acc[2 * dp], pa, bb0);
     mma_bf16_16816(acc[2 * dp + 1], pa, bb1);
+  }
+}
+
+// One warp's online-softmax update over KEYS consecutive keys of a staged tile
+// (bf16, 128-byte swizzled, column halves of TROWS rows of 128 bytes; K and V
+// alike), keys numbered from 0 at the tile's first row.  Keys >= rows and key
+// `masked` are excluded.  Scores are in the log2 domain: s = q.k * kscale *
+// log2(e) / sqrt(D).  The probabilities entering PV are multiplied by `vscale`
+// (the FP8 page scale of V; 1 for bf16 pages), the row sums are not.  The
+// QK^T products of the KEYS/16 key pairs and the PV products of the D/16
+// column pairs are independent mma chains, so one warp keeps the tensor pipe
+// busy on its own.
+template <int D, int KEYS, int TROWS>
+__device__ __forceinline__ void warp_tile_keys(const unsigned char* kt, const unsigned char* vt, int rows, int masked,
+                                               float kscale_l2, float vscale, const uint32_t (&qa)[D / 16][4],
+                                               float (&acc)[D / 8][4], float (&mrow)[2], float (&lrow)[2]) {
+  constexpr int KS = D / 16, NT = D / 8, KP = KEYS / 16;
+  const int lane = threadIdx.x & 31;
+  const int mi = lane >> 3, rr = lane & 7;
+  float s[KP][2][4];
+#pragma unroll
+  for (int kp = 0; kp < KP; ++kp)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) s[kp][nt][0] = s[kp][nt][1] = s[kp][nt][2] = s[kp][nt][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int chunk = 2 * ks + (mi & 1);
+#pragma unroll
+    for (int kp = 0; kp < KP; ++kp) {
+      const int n_row = kp * 16 + (mi >> 1) * 8 + rr;
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4(b0, b1, b2, b3, smem_u32(kt + (chunk / 8) * TROWS * 128 + sw128(n_row, chunk % 8)));
+      uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+      mma_bf16_16816(s[kp][0], qa[ks], bb0);
+      mma_bf16_16816(s[kp][1], qa[ks], bb1);
+    }
+  }
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int kp = 0; kp < KP; ++kp)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = kp * 16 + nt * 8 + 2 * (lane & 3) + (e & 1);
+        const float x = (key < rows && key != masked) ? s[kp][nt][e] * kscale_l2 : -INFINITY;
+        s[kp][nt][e] = x;
+        mx[e >> 1] = fmaxf(mx[e >> 1], x);
+      }
+  float corr[2], mu[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+    const float mn = fmaxf(mrow[r], mx[r]);
+    mu[r] = mn == -INFINITY ? 0.f : mn;
+    corr[r] = exp2f(mrow[r] - mu[r]);
+    mrow[r] = mn;
+  }
+  float rs[2] = {0.f, 0.f};
+#pragma unroll
+  for (int kp = 0; kp < KP; ++kp)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float p = exp2f(s[kp][nt][e] - mu[e >> 1]);
+        s[kp][nt][e] = p;
+        rs[e >> 1] += p;
+      }
+  lrow[0] = lrow[0] * corr[0] + rs[0];
+  lrow[1] = lrow[1] * corr[1] + rs[1];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    acc[nt][0] *= corr[0];
+    acc[nt][1] *= corr[0];
+    acc[nt][2] *= corr[1];
+    acc[nt][3] *= corr[1];
+  }
+#pragma unroll
+  for (int kp = 0; kp < KP; ++kp) {
+    uint32_t pa[4];
+    pa[0] = pack_bf16(s[kp][0][0] * vscale, s[kp][0][1] * vscale);
+    pa[1] = pack_bf16(s[kp][0][2] * vscale, s[kp][0][3] * vscale);
+    pa[2] = pack_bf16(s[kp][1][0] * vscale, s[kp][1][1] * vscale);
+    pa[3] = pack_bf16(s[kp][1][2] * vscale, s[kp][1][3] * vscale);
+    const int n_row = kp * 16 + (mi & 1) * 8 + rr;
+#pragma unroll
+    for (int dp = 0; dp < NT / 2; ++dp) {
+      const int chunk = 2 * dp + (mi >> 1);
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(vt + (chunk / 8) * TROWS * 128 + sw128(n_row, chunk % 8)));
+      uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+      mma_bf16_16816(acc[2 * dp], pa, bb0);
+      mma_bf16_16816(acc[2 * dp + 1], pa, bb1);
+    }
+  }
+}
+
+// Widen rows [r0, r0 + CROWS) of a staged FP8 sub-tile (K then V, RAWROWS
+// unswizzled rows of D codes each) to bf16 (exact) in the 128-byte swizzled
+// layout of a CROWS-row tile pair at `conv` (K then V), by one warp.
+template <int D, int CROWS, int RAWROWS>
+__device__ __forceinline__ void widen_fp8_rows(const unsigned char* raw, unsigned char* conv, int r0) {
+  constexpr int TILE_RAW = RAWROWS * D, CTILE = CROWS * D * 2, CH = D / 16;
+  const int lane = threadIdx.x & 31;
+  for (int idx = lane; idx < 2 * CROWS * CH; idx += 32) {
+    const int which = idx / (CROWS * CH);
+    const int rem = idx % (CROWS * CH);
+    const int r = rem / CH, ch = rem % CH;  // 16 codes of row r0 + r
+    const uint4 u = *reinterpret_cast<const uint4*>(raw + which * TILE_RAW + (r0 + r) * D + ch * 16);
+    const uint32_t wsrc[4] = {u.x, u.y, u.z, u.w};
+    uint32_t wds[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __half2_raw lo =
+          __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(wsrc[e] & 0xFFFFu), __NV_E4M3);
+      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(wsrc[e] >> 16), __NV_E4M3);
+      const float2 fl = __half22float2(__half2(lo)), fh = __half22float2(__half2(hi));
+      wds[2 * e] = pack_bf16(fl.x, fl.y);
+      wds[2 * e + 1] = pack_bf16(fh.x, fh.y);
+    }
+    unsigned char* dstt = conv + which * CTILE;
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      const int chunk = 2 * ch + hc;
+      *reinterpret_cast<uint4*>(dstt + (chunk / 8) * CROWS * 128 + sw128(r, chunk % 8)) =
+          make_uint4(wds[4 * hc], wds[4 * hc + 1], wds[4 * hc + 2], wds[4 * hc + 3]);
+    }
   }
 }
 

@@ -1,11 +1,15 @@
 // Decode attention with one thread-block cluster per KV head, and the fused
 // decode step built on it.
 //
-// A cluster of `cs` CTAs (cs a power of two <= 8, chosen so the grid holds
-// about two CTAs per SM) covers one (b, h): CTA r attends a contiguous range of
-// the head's retained slots, staged by TMA in sub-tiles of at most 64 slots
-// that never cross a page, with the g query heads as the M dimension of
-// mma.sync tiles.  Each CTA merges its warps into one partial (acc, running
+// A cluster of `cs` CTAs (cs a power of two <= 8, chosen so the grid fits the
+// SMs at the CTAs per SM its shared memory allows, at most two) covers one
+// (b, h): CTA r attends a contiguous range of the head's retained slots, cut
+// at multiples of 32 slots (16 when the page size is not a multiple of 32) so
+// no sub-tile crosses a page.  Sub-tile n belongs to warp n mod 4, which
+// issues its TMA loads into stages of its own, waits on them and runs the
+// whole online-softmax update of its keys with the g query heads as the M
+// dimension of mma.sync tiles: the four warps stream independently, with no
+// block barrier between sub-tiles.  Each CTA merges its warps into one partial (acc, running
 // max, running sum, log2 domain) and writes it with st.async into the shared
 // memory of the cluster's last rank (the owner), completing bytes on an
 // mbarrier there; the owner, whose share of the slots is the smallest, merges
@@ -40,9 +44,15 @@ __device__ __forceinline__ float ex2_fast(float x) {
   return y;
 }
 
+constexpr int kCRows = 32;  // slots per warp sub-tile (two 16-row TMA boxes)
+
 template <int D, bool FP8>
 struct ClusterSmem {
-  using S = DecodeSmem<D, FP8>;
+  static constexpr int TILE = FP8 ? kCRows * D : kCRows * D * 2;  // K (or V) of one sub-tile, as loaded
+  static constexpr int STAGE = 2 * TILE;                           // K then V (a multiple of 1024 bytes)
+  static constexpr int MPER = D == 64 ? 4 : 2;                     // stages per warp
+  static constexpr int NST = 4 * MPER;
+  static constexpr int CONV_WARP = FP8 ? 2 * kCRows * D * 2 : 0;   // widened bf16 K and V, per warp
   static constexpr int MLD = D + 2;
   static constexpr int IMLD = D + 4;  // inbox row: D values, max, sum, 2 pad (16-byte rows)
   // floats of the merge buffer [5 sources][g][MLD], rounded up so the inbox
@@ -51,7 +61,7 @@ struct ClusterSmem {
   // stages, conversion tile, merge buffer, the owner's inbox [cs][g][IMLD],
   // weights [max(cs, 5)][g], row maxima and sums [2][16]
   static size_t bytes(int g, int cs) {
-    return 1024 + kStages * S::STAGE + S::CONV + (merge_floats(g) + cs * g * IMLD) * sizeof(float) +
+    return 1024 + NST * STAGE + 4 * CONV_WARP + (merge_floats(g) + cs * g * IMLD) * sizeof(float) +
            (kMaxCluster * 16 + 32) * sizeof(float);
   }
 };
@@ -69,26 +79,27 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
                                                             float* alpha, DecideArgs da, int fuse_decide,
                                                             const __grid_constant__ CUtensorMap kmap,
                                                             const __grid_constant__ CUtensorMap vmap) {
-  using S = DecodeSmem<D, FP8>;
-  constexpr int KS = D / 16, NT = D / 8, MLD = D + 2, IMLD = ClusterSmem<D, FP8>::IMLD;
+  using S = ClusterSmem<D, FP8>;
+  constexpr int KS = D / 16, NT = D / 8, MLD = D + 2, IMLD = S::IMLD;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sbase =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* stage_buf = sbase;
-  unsigned char* conv_buf = sbase + kStages * S::STAGE;
+  unsigned char* stage_buf = sbase;                              // [NST] stages; warp w owns w, w + 4, ...
+  unsigned char* conv_buf = sbase + S::NST * S::STAGE;           // FP8: [4 warps] widened K, V
   const int g = c.Hq / c.Hkv;
-  float* merge = reinterpret_cast<float*>(conv_buf + S::CONV);  // [5 sources][g][MLD]
-  float* inbox = merge + ClusterSmem<D, FP8>::merge_floats(g);  // [cs][g][IMLD] partials, on the owner (16-byte aligned)
+  float* merge = reinterpret_cast<float*>(conv_buf + 4 * S::CONV_WARP);  // [5 sources][g][MLD]
+  float* inbox = merge + S::merge_floats(g);  // [cs][g][IMLD] partials, on the owner (16-byte aligned)
   float* sm_w = inbox + cs * g * IMLD;                          // [sources][g] weights
   float* sm_L = sm_w + kMaxCluster * 16;                        // [g]
-  __shared__ uint64_t full_bar[kStages];
+  __shared__ uint64_t full_bar[S::NST];
   __shared__ uint64_t inbox_bar;  // the owner: every rank's partial has landed
-  __shared__ SubMeta meta[kStages];
-  __shared__ int s_abort, s_have, s_red[32], s_ring_next;
+  __shared__ SubMeta meta[S::NST];
+  __shared__ int s_ring_next;
   __shared__ float s_fred[8], s_alpha, s_xscore[16];
   __shared__ __align__(16) __nv_bfloat16 s_knew[D], s_vnew[D];
   constexpr int kPtCache = 256;  // page-table entries of the head kept in shared memory
   __shared__ int s_pt[kPtCache];
+  __shared__ float s_ksc[FP8 ? kPtCache : 1], s_vsc[FP8 ? kPtCache : 1];  // FP8 page scales
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // head vh of the launch: (layer + lrel, b, h); the inputs of a multi-layer
@@ -111,10 +122,9 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     griddep_launch_dependents();
   }
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) mbar_init(&full_bar[i], 1);
+    for (int i = 0; i < S::NST; ++i) mbar_init(&full_bar[i], 1);
     mbar_init(&inbox_bar, 1);
     fence_mbar_init();
-    s_abort = 0;
   }
   // state of this head (stable during the launch: only rank 0 of this head's
   // cluster writes it, after the cluster barrier; the position and the page
@@ -134,23 +144,34 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   __syncthreads();
   cluster_arrive_relaxed();  // this CTA's barriers are initialised (waited before the first remote store)
 
-  int p_s = s_begin;
-  auto produce = [&](int stage) -> bool {
-    if (p_s >= s_end) return false;
-    const int pi = p_s / c.P;
+  // sub-tile n of this CTA: slots [max(s_begin, (first + n) C), min(s_end, (first + n + 1) C)),
+  // inside one page (C divides P); warp n % 4 takes it into stage
+  // n % 4 + 4 ((n / 4) mod MPER), issued by the warp's lane 0
+  const int chunk = c.P % kCRows == 0 ? kCRows : 16;
+  const int first = s_begin / chunk;
+  const int nsub = s_end > s_begin ? (s_end - 1) / chunk - first + 1 : 0;
+  auto issue = [&](int n) {
+    const int st = warp + 4 * ((n >> 2) % S::MPER);
+    const int slot = max(s_begin, (first + n) * chunk);
+    const int rows = min(s_end, (first + n + 1) * chunk) - slot;
+    const int pi = slot / c.P;
     const int page = pi < kPtCache ? s_pt[pi] : c.page_table[li * c.maxp + pi];
-    const int rows = min(min(kSub, s_end - p_s), c.P - p_s % c.P);
-    meta[stage].slot = p_s;
-    meta[stage].rows = rows;
-    meta[stage].page = page;
-    issue_subtile<D, FP8>(stage_buf + stage * S::STAGE, &kmap, &vmap, page * c.P + p_s % c.P, rows, &full_bar[stage]);
-    p_s += rows;
-    return true;
+    meta[st].slot = slot;
+    meta[st].rows = rows;
+    meta[st].page = page;
+    issue_rows<D, FP8, kCRows>(stage_buf + st * S::STAGE, &kmap, &vmap, page * c.P + slot % c.P, rows,
+                               &full_bar[st]);
   };
-  int produced = 0;
-  if (tid == 0)
-    for (int st = 0; st < kStages; ++st)
-      if (produce(st)) ++produced;
+  if (lane == 0)
+    for (int n = warp; n < nsub && n < 4 * S::MPER; n += 4) issue(n);
+  if (FP8) {
+    // the scales of this CTA's pages, while the first tiles are in flight
+    const int pf = s_begin / c.P, pl = nsub ? min((s_end - 1) / c.P, kPtCache - 1) : pf - 1;
+    for (int pi = pf + tid; pi <= pl; pi += kThreads) {
+      s_ksc[pi] = c.k_scale[s_pt[pi]];
+      s_vsc[pi] = c.v_scale[s_pt[pi]];
+    }
+  }
 
   if (early) {
     griddep_wait();
@@ -202,36 +223,53 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     }
   }
 
-  for (int n = 0;; ++n) {
-    __syncthreads();
-    if (s_abort) break;
-    const int stage = n % kStages;
-    if (tid == 0) s_have = (n < produced) ? 1 : 0;
-    __syncthreads();
-    if (!s_have) break;
-    if (!mbar_wait_bounded(&full_bar[stage], (n / kStages) & 1)) {
-      if (tid == 0) {
-        set_status(c.ctrl, DMS_ST_TIMEOUT);
-        s_abort = 1;
+  if (FP8) __syncthreads();  // page scales staged
+  {
+    // this warp's sub-tiles n = warp, warp + 4, ...: local index j, stage
+    // use j / MPER; the refill of a stage follows the warp's own reads of it
+    unsigned char* conv = conv_buf + warp * S::CONV_WARP;
+    const int nmine = nsub > warp ? (nsub - warp + 3) / 4 : 0;
+    int j = 0;
+    bool timed_out = false;
+    for (; j < nmine; ++j) {
+      const int n = warp + 4 * j, st = warp + 4 * (j % S::MPER);
+      __syncwarp();
+      if (!mbar_wait_bounded(&full_bar[st], (j / S::MPER) & 1)) {
+        timed_out = true;
+        break;
       }
-      __syncthreads();
-      break;
+      const SubMeta m = meta[st];
+      const unsigned char* kt = stage_buf + st * S::STAGE;
+      const int masked = masked_slot >= 0 ? masked_slot - m.slot : -1;
+      float ks = 1.0f, vs = 1.0f;
+      if (FP8) {
+        const int pi = m.slot / c.P;
+        ks = pi < kPtCache ? s_ksc[pi] : c.k_scale[m.page];
+        vs = pi < kPtCache ? s_vsc[pi] : c.v_scale[m.page];
+        widen_fp8_rows<D, kCRows, kCRows>(kt, conv, 0);
+        __syncwarp();
+        kt = conv;
+      }
+      // a sub-tile of at most 16 slots had one box loaded: the rows after it
+      // hold whatever the stage held before, so only its 16 keys are read
+      const unsigned char* vt = kt + (FP8 ? kCRows * D * 2 : S::TILE);
+      const float kl2 = FP8 ? ks * sl2 : sl2;
+      if (m.rows > 16)
+        warp_tile_keys<D, kCRows, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
+      else
+        warp_tile_keys<D, 16, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
+      __syncwarp();
+      if (lane == 0 && n + 4 * S::MPER < nsub) {
+        fence_proxy_async();  // this warp's reads of the stage before the copy that refills it
+        issue(n + 4 * S::MPER);
+      }
     }
-    const SubMeta m = meta[stage];
-    const unsigned char* kt = stage_buf + stage * S::STAGE;
-    if (FP8) {
-      widen_fp8_subtile<D>(kt, conv_buf);
-      __syncthreads();
-      kt = conv_buf;
+    if (timed_out) {
+      // the copies of this warp still in flight land before the CTA exits
+      for (int jj = j; jj < min(nmine, j + S::MPER); ++jj)
+        mbar_wait_bounded(&full_bar[warp + 4 * (jj % S::MPER)], (jj / S::MPER) & 1);
+      if (lane == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
     }
-    const unsigned char* vt = kt + (FP8 ? S::TILE_BF16 : S::TILE_RAW);
-    if (warp * 16 < m.rows) {
-      const float kscale = FP8 ? c.k_scale[m.page] : 1.0f;
-      const float vscale = FP8 ? c.v_scale[m.page] : 1.0f;
-      warp_tile<D>(kt, vt, m.rows, masked_slot - m.slot, kscale * sl2, vscale, qa, acc, mrow, lrow);
-    }
-    __syncthreads();
-    if (tid == 0 && produce(stage)) ++produced;
   }
 
   // merge the warps (and, for the owner of a fused step, the new token) into
@@ -413,15 +451,17 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   }
 }
 
-// Cluster size: the largest power of two <= 8 with cs * B * Hkv <= 2 * SMs
-// (about two CTAs per SM) whose shared memory fits and which the device can
-// co-schedule.
+// Cluster size: the largest power of two <= 8 with cs * B * Hkv <= k * SMs,
+// k the CTAs per SM the kernel's shared memory allows (at most two), whose
+// shared memory fits and which the device can co-schedule.
 template <int D, bool FP8, bool FUSED>
 static int pick_cluster(int heads, int g, int num_sms) {
-  static int max_cs[17] = {0};  // by g (<= 16)
+  static int max_cs[17] = {0}, per_sm[17] = {0};  // by g (<= 16)
   int& m = max_cs[g < 16 ? g : 16];
+  int& k = per_sm[g < 16 ? g : 16];
   if (m == 0) {
     m = 1;
+    k = 1;
     int dev = 0, optin = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -447,13 +487,19 @@ static int pick_cluster(int heads, int g, int num_sms) {
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, k_decode_cluster<D, FP8, FUSED>, &cfg) == cudaSuccess && n > 0) {
         m = cs;
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode_cluster<D, FP8, FUSED>, kThreads, smem) ==
+                cudaSuccess &&
+            nb > 1)
+          k = 2;
+        cudaGetLastError();
         break;
       }
       cudaGetLastError();
     }
   }
   int cs = 1;
-  while (cs * 2 <= m && static_cast<long>(cs) * 2 * heads <= 2L * num_sms) cs *= 2;
+  while (cs * 2 <= m && static_cast<long>(cs) * 2 * heads <= static_cast<long>(k) * num_sms) cs *= 2;
   return cs;
 }
 
