@@ -377,6 +377,132 @@ __device__ __forceinline__ void widen_fp8_rows(const unsigned char* raw, unsigne
   }
 }
 
+// 8x8 bf16 matrix transpose across the warp (the mma fragment layout: lane
+// holds row lane / 4, columns 2 (lane % 4) + {0, 1}).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// warp_tile_keys with the keys as the M dimension of the mma tiles and the
+// g <= 8 query heads as N = 8: S^T = K Q^T, then O^T += V^T P^T.  For g <= 8
+// this takes half the tensor work of the query-major form (whose M = 16 rows
+// hold only g queries).  Lane state: queries 2 (lane % 4) + {0, 1}; running
+// maxima uniform over the lanes sharing lane % 4, sums partial per lane.
+//   qb[ks]: Q as the B operand: Q[lane / 4][16 ks + 2 (lane % 4) + {0, 1}]
+//           and the same + 8 (rows >= g zero).
+//   acc[dt][j], acc[dt][2 + j]: O^T[16 dt + lane / 4 (+ 8)][2 (lane % 4) + j].
+// The probability tiles go from the S^T accumulator layout to the B operand
+// of the PV product by an in-register 8x8 transpose (movmatrix).
+template <int D, int KEYS, int TROWS>
+__device__ __forceinline__ void warp_tile_keys_t(const unsigned char* kt, const unsigned char* vt, int rows,
+                                                 int masked, float kscale_l2, float vscale,
+                                                 const uint32_t (&qb)[D / 16][2], float (&acc)[D / 16][4],
+                                                 float (&mrow)[2], float (&lrow)[2]) {
+  constexpr int KS = D / 16, MT = KEYS / 16, DT = D / 16;
+  const int lane = threadIdx.x & 31;
+  float s[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int chunk = 2 * ks + (lane >> 4);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      uint32_t a[4];
+      ldmatrix_x4(a[0], a[1], a[2], a[3],
+                  smem_u32(kt + (chunk / 8) * TROWS * 128 + sw128(mt * 16 + (lane & 15), chunk % 8)));
+      mma_bf16_16816(s[mt], a, qb[ks]);
+    }
+  }
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = mt * 16 + (lane >> 2) + (e >> 1) * 8;
+      const float x = (key < rows && key != masked) ? s[mt][e] * kscale_l2 : -INFINITY;
+      s[mt][e] = x;
+      mx[e & 1] = fmaxf(mx[e & 1], x);
+    }
+  float corr[2], mu[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 4));
+    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 8));
+    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 16));
+    const float mn = fmaxf(mrow[j], mx[j]);
+    mu[j] = mn == -INFINITY ? 0.f : mn;
+    corr[j] = exp2f(mrow[j] - mu[j]);
+    mrow[j] = mn;
+  }
+  float rs[2] = {0.f, 0.f};
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float p = exp2f(s[mt][e] - mu[e & 1]);
+      s[mt][e] = p;
+      rs[e & 1] += p;
+    }
+  lrow[0] = lrow[0] * corr[0] + rs[0];
+  lrow[1] = lrow[1] * corr[1] + rs[1];
+#pragma unroll
+  for (int dt = 0; dt < DT; ++dt) {
+    acc[dt][0] *= corr[0];
+    acc[dt][1] *= corr[1];
+    acc[dt][2] *= corr[0];
+    acc[dt][3] *= corr[1];
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    uint32_t pb[2];
+    pb[0] = movmatrix_trans(pack_bf16(s[mt][0] * vscale, s[mt][1] * vscale));  // keys 16 mt + 0..7
+    pb[1] = movmatrix_trans(pack_bf16(s[mt][2] * vscale, s[mt][3] * vscale));  // keys 16 mt + 8..15
+    const int key = mt * 16 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+    for (int dt = 0; dt < DT; ++dt) {
+      const int chunk = 2 * dt + ((lane >> 3) & 1);
+      uint32_t a[4];
+      ldmatrix_x4_trans(a[0], a[1], a[2], a[3], smem_u32(vt + (chunk / 8) * TROWS * 128 + sw128(key, chunk % 8)));
+      mma_bf16_16816(acc[dt], a, pb);
+    }
+  }
+}
+
+// The state of warp_tile_keys_t (queries < g) into merge buffer slot `src`,
+// laid out as warp_state_to_smem's.
+template <int D>
+__device__ __forceinline__ void warp_state_t_to_smem(float* merge, int src, int g, const float (&acc)[D / 16][4],
+                                                     const float (&mrow)[2], const float (&lrow)[2]) {
+  constexpr int DT = D / 16, MLD = D + 2;
+  const int lane = threadIdx.x & 31;
+  float lsum[2] = {lrow[0], lrow[1]};
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    lsum[j] += __shfl_xor_sync(0xffffffffu, lsum[j], 4);
+    lsum[j] += __shfl_xor_sync(0xffffffffu, lsum[j], 8);
+    lsum[j] += __shfl_xor_sync(0xffffffffu, lsum[j], 16);
+  }
+  float* mw = merge + src * g * MLD;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int qr = 2 * (lane & 3) + j;
+    if (qr < g) {
+#pragma unroll
+      for (int dt = 0; dt < DT; ++dt) {
+        mw[qr * MLD + dt * 16 + (lane >> 2)] = acc[dt][j];
+        mw[qr * MLD + dt * 16 + (lane >> 2) + 8] = acc[dt][2 + j];
+      }
+      if (lane < 4) {
+        mw[qr * MLD + D] = mrow[j];
+        mw[qr * MLD + D + 1] = lsum[j];
+      }
+    }
+  }
+}
+
 // Store one warp's state (rows < g) into the merge buffer slot `src`:
 // merge[(src * g + r) * (D + 2) + {0..D-1: acc, D: max, D+1: sum}].
 template <int D>
@@ -553,6 +679,82 @@ __device__ void combine_head(const float* part_acc, const float* part_ml, int g,
     pk.y = pack_bf16(accv[k].z * inv, accv[k].w * inv);
     *reinterpret_cast<uint2*>(out + static_cast<long>(r) * D + d4 * 4) = pk;
   }
+}
+
+// The decision logit of one (b, head) in pieces, so that its loads join the
+// other loads of a prologue and its dot products can be shared by several
+// CTAs: decide_issue starts the loads of part `part` of `nparts` equal slices
+// of the hidden row (each at most kThreads * VPT 16-byte vectors; thread `who`
+// also loads the bias and offset), decide_partial gives one thread's sums
+// (x.x, (W * gamma).x), decide_reduce finishes a whole row in one CTA.
+template <int VPT>
+struct DecideLoads {
+  uint4 x[VPT], w[VPT], gm[VPT];
+  float bias, offset;
+};
+template <int VPT>
+__device__ __forceinline__ void decide_issue(const CacheView& c, const DecideArgs& a, int b, int src,
+                                             DecideLoads<VPT>& L, int part = 0, int nparts = 1, int who = 0) {
+  const int tid = threadIdx.x, nvec = c.hidden / 8;
+  const int per = (nvec + nparts - 1) / nparts, v0 = part * per, v1 = min(nvec, v0 + per);
+  const uint4* xr =
+      reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.hidden) + static_cast<long>(b) * c.hidden);
+  const uint4* wr =
+      reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.W) + static_cast<long>(src) * c.hidden);
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int vi = v0 + u * kThreads + tid;
+    const bool ok = vi < v1;
+    L.x[u] = ok ? xr[vi] : make_uint4(0, 0, 0, 0);
+    L.w[u] = ok ? wr[vi] : make_uint4(0, 0, 0, 0);
+    L.gm[u] = ok ? gamma16<__nv_bfloat16>(a.gamma, vi) : make_uint4(0, 0, 0, 0);
+  }
+  L.bias = 0.f;
+  L.offset = 0.f;
+  if (tid == who) {
+    const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+    L.bias = bias ? __bfloat162float(bias[src]) : 0.f;
+    L.offset = a.offset[b * a.offset_bstride + src];
+  }
+}
+template <int VPT>
+__device__ __forceinline__ float2 decide_partial(const DecideLoads<VPT>& L) {
+  float ss = 0.f, dot = 0.f;
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    float x[8], wv[8], gv[8];
+    unpack16(L.x[u], x, static_cast<const __nv_bfloat16*>(nullptr));
+    unpack16(L.w[u], wv, static_cast<const __nv_bfloat16*>(nullptr));
+    unpack16(L.gm[u], gv, static_cast<const __nv_bfloat16*>(nullptr));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      ss = fmaf(x[e], x[e], ss);
+      dot = fmaf(wv[e] * gv[e], x[e], dot);
+    }
+  }
+  return make_float2(ss, dot);
+}
+template <int VPT>
+__device__ __forceinline__ float decide_reduce(const CacheView& c, const DecideLoads<VPT>& L, float* red) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const float2 pd = decide_partial<VPT>(L);
+  float ss = pd.x, dot = pd.y;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  }
+  __syncthreads();
+  if (lane == 0) {
+    red[wid] = ss;
+    red[4 + wid] = dot;
+  }
+  __syncthreads();
+  float alpha = 0.f;
+  if (tid == 0)
+    alpha = adapter_logit(c, red[4] + red[5] + red[6] + red[7], red[0] + red[1] + red[2] + red[3], c.hidden, L.bias,
+                          L.offset);
+  return alpha;
 }
 
 // Adapter decision logit of the new token of sequence b for head `src`, by one

@@ -72,7 +72,7 @@ struct SubMeta {
   int page;  // page id
 };
 
-template <int D, bool FP8, bool FUSED>
+template <int D, bool FP8, bool FUSED, bool TQ>
 __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int layer, int nl, int early,
                                                             const __nv_bfloat16* q, __nv_bfloat16* o, int cs,
                                                             const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   __shared__ uint64_t inbox_bar;  // the owner: every rank's partial has landed
   __shared__ SubMeta meta[S::NST];
   __shared__ int s_ring_next;
-  __shared__ float s_fred[8], s_alpha, s_xscore[16];
+  __shared__ float s_fred[8], s_alpha;
   __shared__ __align__(16) __nv_bfloat16 s_knew[D], s_vnew[D];
   constexpr int kPtCache = 256;  // page-table entries of the head kept in shared memory
   __shared__ int s_pt[kPtCache];
@@ -117,6 +117,11 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   // start only once its own wait has returned), and it does not write this
   // state.  The page counter, the inputs and the outputs are touched only
   // after the wait.
+  if (tid == 32) {
+    // the pool's tensor maps, fetched while the head's state is read
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
+  }
   if (!early) {
     griddep_wait();
     griddep_launch_dependents();
@@ -133,14 +138,26 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   for (int i = tid; i < min(c.maxp, kPtCache); i += kThreads) s_pt[i] = c.page_table[li * c.maxp + i];
   const int cnt = c.count[li];
   const int t = FUSED ? c.pos[layer * c.B + bb] : 0;
-  const int4 pl = FUSED ? *plan_at(c, li, t) : make_int4(0, 0, 0, 0);
+  // both plan buffers in the same round trip as the position that picks one
+  const int4 pl0 = FUSED ? *plan_at(c, li, 0) : make_int4(0, 0, 0, 0);
+  const int4 pl1 = FUSED ? *plan_at(c, li, 1) : make_int4(0, 0, 0, 0);
+  const int4 pl = (t & 1) ? pl1 : pl0;
   const int masked_slot = (FUSED && (pl.y & 1)) ? pl.x : -1;
-  // ranks 0 .. cs-2 take `per` slots each, the owner the rest: a quarter share
-  // when it also computes the decision logit, half a share otherwise (it
-  // merges the partials and appends)
-  const int oq = (FUSED && fuse_decide) ? 1 : 2;
-  const int per = cs == 1 ? cnt : ((4 * cnt + 4 * (cs - 1) + oq - 1) / (4 * (cs - 1) + oq) + 15) / 16 * 16;
-  const int s_begin = min(cnt, rank * per), s_end = rank == owner ? cnt : min(cnt, s_begin + per);
+  // The decision logit of the new token: with cs >= 4, rank 0 computes it
+  // instead of attending (it sends the logit with an empty partial), so it
+  // is off the path of the streaming ranks; with a smaller cluster the owner
+  // computes it before streaming.
+  const bool rank0_decides = FUSED && fuse_decide && cs >= 4;
+  const bool owner_decides = FUSED && fuse_decide && cs < 4;
+  // the streaming ranks before the owner take `per` slots each, the owner
+  // the rest: half a share (it merges the partials and appends), a quarter
+  // share when it also computes the decision logit
+  const int r0 = rank0_decides ? 1 : 0;  // first streaming rank
+  const int oq = owner_decides ? 1 : 2;
+  const int nfull = cs - 1 - r0;
+  const int per = nfull == 0 ? 0 : ((4 * cnt + 4 * nfull + oq - 1) / (4 * nfull + oq) + 15) / 16 * 16;
+  const int s_begin = rank < r0 ? 0 : min(cnt, (rank - r0) * per);
+  const int s_end = rank < r0 ? 0 : rank == owner ? cnt : min(cnt, s_begin + per);
   __syncthreads();
   cluster_arrive_relaxed();  // this CTA's barriers are initialised (waited before the first remote store)
 
@@ -178,51 +195,58 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     griddep_launch_dependents();
   }
   const int next_page0 = FUSED ? c.ctrl[CTRL_NEXT_PAGE] : 0;
+  // this layer's adapter (hidden rows of the layer, its weights and offsets);
+  // decision logit of the new token (layer granularity: head 0's)
+  const int dsrc = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
+  DecideArgs dl = da;
+  if (FUSED && lrel > 0 && fuse_decide) {
+    dl.hidden = static_cast<const __nv_bfloat16*>(da.hidden) + static_cast<long>(lrel) * c.B * c.hidden;
+    dl.gamma = static_cast<const __nv_bfloat16*>(da.gamma) + lrel * da.gamma_lstride;
+    dl.W = static_cast<const __nv_bfloat16*>(da.W) + lrel * da.w_lstride;
+    if (da.bias) dl.bias = static_cast<const __nv_bfloat16*>(da.bias) + lrel * da.bias_lstride;
+    dl.offset = da.offset + lrel * da.offset_lstride;
+  }
+  // Everything read after the wait, in one round trip while the first tiles
+  // are in flight: the query rows, on the owner the new key/value row and the
+  // ring entry of t + 1 (held in registers until the merge), and on the CTA
+  // that computes the decision logit its operands.
+  constexpr int kDV = 4;  // 16-byte vectors per thread of the decision logit's rows
+  const bool decides = (rank0_decides && rank == 0) || (owner_decides && rank == owner);
+  const bool one_trip = c.hidden <= kThreads * kDV * 8;
+  DecideLoads<kDV> dq;
+  if (decides && one_trip) decide_issue<kDV>(c, dl, b, dsrc, dq);
   uint32_t qa[KS][4];
   const __nv_bfloat16* qb = q + (static_cast<long>(bb) * c.Hq + static_cast<long>(h) * g) * D;
   load_q_frags<D>(qb, g, qa);
+  uint4 kn = make_uint4(0, 0, 0, 0), vn = kn;
+  int ring_next = 0;
   if (FUSED && rank == owner) {
-    // everything the append needs, fetched while the first tiles are in flight:
-    // the new key/value row, the new token's scores, the ring entry of t + 1
     if (tid < D / 8) {
-      reinterpret_cast<uint4*>(s_knew)[tid] = reinterpret_cast<const uint4*>(k_new + static_cast<long>(vh) * D)[tid];
-      reinterpret_cast<uint4*>(s_vnew)[tid] = reinterpret_cast<const uint4*>(v_new + static_cast<long>(vh) * D)[tid];
+      kn = reinterpret_cast<const uint4*>(k_new + static_cast<long>(vh) * D)[tid];
+      vn = reinterpret_cast<const uint4*>(v_new + static_cast<long>(vh) * D)[tid];
     }
-    if (tid == 32) s_ring_next = (t + 1 >= c.w) ? c.ring[li * c.w + (t + 1) % c.w] : 0;
-    __syncthreads();
-    for (int r = warp; r < g; r += 4) {
-      float sdot = 0.f;
-      for (int d = lane; d < D; d += 32)
-        sdot = fmaf(__bfloat162float(qb[static_cast<long>(r) * D + d]), __bfloat162float(s_knew[d]), sdot);
-#pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, o2);
-      if (lane == 0) s_xscore[r] = sdot;
-    }
+    if (tid == 32 && t + 1 >= c.w) ring_next = c.ring[li * c.w + (t + 1) % c.w];
   }
-  float acc[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-  const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-  if (FUSED && rank == owner && fuse_decide) {
-    // decision logit of the new token (layer granularity: head 0's)
-    const int src = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
-    // this layer's adapter (hidden rows of the layer, its weights and offsets)
-    DecideArgs dl = da;
-    if (lrel > 0) {
-      dl.hidden = static_cast<const __nv_bfloat16*>(da.hidden) + static_cast<long>(lrel) * c.B * c.hidden;
-      dl.gamma = static_cast<const __nv_bfloat16*>(da.gamma) + lrel * da.gamma_lstride;
-      dl.W = static_cast<const __nv_bfloat16*>(da.W) + lrel * da.w_lstride;
-      if (da.bias) dl.bias = static_cast<const __nv_bfloat16*>(da.bias) + lrel * da.bias_lstride;
-      dl.offset = da.offset + lrel * da.offset_lstride;
-    }
-    const float a = decide_cta<4>(c, dl, b, src, s_fred);
+  if (decides) {
+    const float a = one_trip ? decide_reduce<kDV>(c, dq, s_fred) : decide_cta<4>(c, dl, b, dsrc, s_fred);
     if (tid == 0) {
       s_alpha = a;
       alpha[bb * c.Hkv + h] = a;
     }
   }
-
+  // TQ (g <= 8): keys as the mma M dimension (warp_tile_keys_t), else queries
+  constexpr int NA = TQ ? D / 16 : NT;
+  float acc[NA][4];
+#pragma unroll
+  for (int nt = 0; nt < NA; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+  uint32_t qt[KS][2];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    qt[ks][0] = qa[ks][0];
+    qt[ks][1] = qa[ks][2];
+  }
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
   if (FP8) __syncthreads();  // page scales staged
   {
     // this warp's sub-tiles n = warp, warp + 4, ...: local index j, stage
@@ -254,10 +278,17 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
       // hold whatever the stage held before, so only its 16 keys are read
       const unsigned char* vt = kt + (FP8 ? kCRows * D * 2 : S::TILE);
       const float kl2 = FP8 ? ks * sl2 : sl2;
-      if (m.rows > 16)
-        warp_tile_keys<D, kCRows, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
-      else
-        warp_tile_keys<D, 16, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
+      if constexpr (TQ) {
+        if (m.rows > 16)
+          warp_tile_keys_t<D, kCRows, kCRows>(kt, vt, m.rows, masked, kl2, vs, qt, acc, mrow, lrow);
+        else
+          warp_tile_keys_t<D, 16, kCRows>(kt, vt, m.rows, masked, kl2, vs, qt, acc, mrow, lrow);
+      } else {
+        if (m.rows > 16)
+          warp_tile_keys<D, kCRows, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
+        else
+          warp_tile_keys<D, 16, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
+      }
       __syncwarp();
       if (lane == 0 && n + 4 * S::MPER < nsub) {
         fence_proxy_async();  // this warp's reads of the stage before the copy that refills it
@@ -274,19 +305,60 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
 
   // merge the warps (and, for the owner of a fused step, the new token) into
   // this CTA's partial, written into slot `rank` of the owner's inbox
-  warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
-  int nsrc = 4;
+  if constexpr (TQ)
+    warp_state_t_to_smem<D>(merge, warp, g, acc, mrow, lrow);
+  else
+    warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
+  const int nsrc = (FUSED && rank == owner) ? 5 : 4;
   if (FUSED && rank == owner) {
-    // the new token as a fifth source: score q_r . k_new, weight 1, value v_new
-    for (int r = tid; r < g; r += kThreads) {
-      merge[(4 * g + r) * MLD + D] = s_xscore[r] * sl2;
-      merge[(4 * g + r) * MLD + D + 1] = 1.0f;
+    if (tid < D / 8) {
+      reinterpret_cast<uint4*>(s_knew)[tid] = kn;
+      reinterpret_cast<uint4*>(s_vnew)[tid] = vn;
     }
-    for (int idx = tid; idx < g * D; idx += kThreads) merge[(4 * g + idx / D) * MLD + idx % D] = __bfloat162float(s_vnew[idx % D]);
-    nsrc = 5;
+    if (tid == 32) s_ring_next = ring_next;
   }
   __syncthreads();
-  // per row: the sources' weights 2^(m_s - M) and the merged (M, L)
+  if (FUSED && rank == owner) {
+    // the new token as a fifth source: score q_r . k_new, weight 1, value v_new
+    for (int idx = tid; idx < g * D; idx += kThreads)
+      merge[(4 * g + idx / D) * MLD + idx % D] = __bfloat162float(s_vnew[idx % D]);
+    if (warp == 0) {
+      // q_r . k_new from the query fragments: lane holds columns
+      // 2 (lane % 4) + {0, 1, 8, 9} of every 16 of rows lane / 4 and lane / 4 + 8
+      const int ra = lane >> 2, rb = ra + 8;
+      float sa = 0.f, sb = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int col = ks * 16 + 2 * (lane & 3);
+        const float2 k0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_knew[col]));
+        const float2 k1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_knew[col + 8]));
+        const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][0]));
+        const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][1]));
+        const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][2]));
+        const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][3]));
+        sa = fmaf(a0.x, k0.x, fmaf(a0.y, k0.y, fmaf(a1.x, k1.x, fmaf(a1.y, k1.y, sa))));
+        sb = fmaf(b0.x, k0.x, fmaf(b0.y, k0.y, fmaf(b1.x, k1.x, fmaf(b1.y, k1.y, sb))));
+      }
+#pragma unroll
+      for (int o2 = 1; o2 < 4; o2 <<= 1) {
+        sa += __shfl_xor_sync(0xffffffffu, sa, o2);
+        sb += __shfl_xor_sync(0xffffffffu, sb, o2);
+      }
+      if ((lane & 3) == 0) {
+        if (ra < g) {
+          merge[(4 * g + ra) * MLD + D] = sa * sl2;
+          merge[(4 * g + ra) * MLD + D + 1] = 1.0f;
+        }
+        if (rb < g) {
+          merge[(4 * g + rb) * MLD + D] = sb * sl2;
+          merge[(4 * g + rb) * MLD + D + 1] = 1.0f;
+        }
+      }
+      __syncwarp();  // read back by lanes r < g of this warp
+    }
+  }
+  // per row: the sources' weights 2^(m_s - M) and the merged (M, L) (rows
+  // r < g <= 16: lanes of warp 0)
   if (tid < g) {
     float M = -INFINITY;
     for (int sv = 0; sv < nsrc; ++sv) M = fmaxf(M, merge[(sv * g + tid) * MLD + D]);
@@ -322,17 +394,27 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
       *reinterpret_cast<float4*>(inbox + (owner * g + r) * IMLD + d) = v;
   }
   if (tid < g) {
-    if (rank != owner)
-      st_async_v2(dst + 4u * static_cast<uint32_t>(tid * IMLD + D), sm_L[tid], sm_L[16 + tid], rbar);
-    else {
-      inbox[(owner * g + tid) * IMLD + D] = sm_L[tid];
-      inbox[(owner * g + tid) * IMLD + D + 1] = sm_L[16 + tid];
+    // (M, L); row 0 also carries the decision logit from rank 0
+    const float dlog = tid == 0 && rank0_decides && rank == 0 ? s_alpha : 0.f;
+    if (rank != owner) {
+      if (tid == 0)
+        st_async_v4(dst + 4u * static_cast<uint32_t>(D), make_float4(sm_L[0], sm_L[16], dlog, 0.f), rbar);
+      else
+        st_async_v2(dst + 4u * static_cast<uint32_t>(tid * IMLD + D), sm_L[tid], sm_L[16 + tid], rbar);
+    } else {
+      float* row = inbox + (owner * g + tid) * IMLD + D;
+      row[0] = sm_L[tid];
+      row[1] = sm_L[16 + tid];
+      if (tid == 0) {
+        row[2] = dlog;
+        row[3] = 0.f;
+      }
     }
   }
   if (rank != owner) {
     return;  // nothing reads this CTA's shared memory
   }
-  if (tid == 0) mbar_expect_tx(&inbox_bar, static_cast<uint32_t>((cs - 1) * g * (D + 2) * 4));
+  if (tid == 0) mbar_expect_tx(&inbox_bar, static_cast<uint32_t>((cs - 1) * (g * (D + 2) * 4 + 8)));
   bool landed = cs == 1 || mbar_wait_bounded(&inbox_bar, 0);
   landed = __syncthreads_and(landed);  // (one answer for the block); the owner's own partial is in place too
   if (!landed && tid == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
@@ -373,7 +455,9 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
           c.npages[li] = np_new;
         }
         const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
-        const float a = fuse_decide ? s_alpha : __ldcg(&alpha[bb * c.Hkv + hs]);
+        const float a = rank0_decides ? inbox[D + 2]  // rank 0's row 0
+                        : owner_decides ? s_alpha
+                                        : __ldcg(&alpha[bb * c.Hkv + hs]);
         const bool evict = shifted_mark(c, li, t, !c.disable && a > 0.0f);
         c.slot_pos[li * c.cap + slot] = t;
         c.ring[li * c.w + t % c.w] = slot | (evict ? static_cast<int>(RING_EVICT) : 0);
@@ -454,7 +538,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
 // Cluster size: the largest power of two <= 8 with cs * B * Hkv <= k * SMs,
 // k the CTAs per SM the kernel's shared memory allows (at most two), whose
 // shared memory fits and which the device can co-schedule.
-template <int D, bool FP8, bool FUSED>
+template <int D, bool FP8, bool FUSED, bool TQ>
 static int pick_cluster(int heads, int g, int num_sms) {
   static int max_cs[17] = {0}, per_sm[17] = {0};  // by g (<= 16)
   int& m = max_cs[g < 16 ? g : 16];
@@ -468,7 +552,7 @@ static int pick_cluster(int heads, int g, int num_sms) {
     for (int cs = kPickCluster; cs > 1; cs >>= 1) {
       const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs);
       if (smem + 4096 > static_cast<size_t>(optin)) continue;  // static shared memory on top
-      if (cudaFuncSetAttribute(k_decode_cluster<D, FP8, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(k_decode_cluster<D, FP8, FUSED, TQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem)) != cudaSuccess) {
         cudaGetLastError();
         continue;
@@ -485,10 +569,10 @@ static int pick_cluster(int heads, int g, int num_sms) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, k_decode_cluster<D, FP8, FUSED>, &cfg) == cudaSuccess && n > 0) {
+      if (cudaOccupancyMaxActiveClusters(&n, k_decode_cluster<D, FP8, FUSED, TQ>, &cfg) == cudaSuccess && n > 0) {
         m = cs;
         int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode_cluster<D, FP8, FUSED>, kThreads, smem) ==
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode_cluster<D, FP8, FUSED, TQ>, kThreads, smem) ==
                 cudaSuccess &&
             nb > 1)
           k = 2;
@@ -503,16 +587,16 @@ static int pick_cluster(int heads, int g, int num_sms) {
   return cs;
 }
 
-template <int D, bool FP8, bool FUSED>
+template <int D, bool FP8, bool FUSED, bool TQ>
 static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q, void* o, const void* k,
                                    const void* v, float* alpha, const DecideArgs* da, const CUtensorMap* kmap,
                                    const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early, int nl) {
   const int g = c.Hq / c.Hkv;
-  auto kern = k_decode_cluster<D, FP8, FUSED>;
+  auto kern = k_decode_cluster<D, FP8, FUSED, TQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
   const int heads = nl * c.B * c.Hkv;
-  const int cs = pick_cluster<D, FP8, FUSED>(heads, g, num_sms);
+  const int cs = pick_cluster<D, FP8, FUSED, TQ>(heads, g, num_sms);
   const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -536,26 +620,35 @@ static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q
                             static_cast<const __nv_bfloat16*>(v), alpha, da ? *da : none, da ? 1 : 0, *kmap, *vmap);
 }
 
+// One instantiation per (head dim, page type, fused step, key-major tiles).
+template <bool FP8, bool FUSED>
+static cudaError_t launch_cluster_dt(const CacheView& c, int layer, const void* q, void* o, const void* k,
+                                    const void* v, float* alpha, const DecideArgs* da, const CUtensorMap* kmap,
+                                    const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early, int nl) {
+  const bool tq = c.Hq / c.Hkv <= 8;
+  if (c.D == 64)
+    return tq ? launch_cluster_t<64, FP8, FUSED, true>(c, layer, q, o, k, v, alpha, da, kmap, vmap, num_sms, s, early,
+                                                       nl)
+              : launch_cluster_t<64, FP8, FUSED, false>(c, layer, q, o, k, v, alpha, da, kmap, vmap, num_sms, s,
+                                                        early, nl);
+  return tq ? launch_cluster_t<128, FP8, FUSED, true>(c, layer, q, o, k, v, alpha, da, kmap, vmap, num_sms, s, early,
+                                                      nl)
+            : launch_cluster_t<128, FP8, FUSED, false>(c, layer, q, o, k, v, alpha, da, kmap, vmap, num_sms, s, early,
+                                                       nl);
+}
+
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early, int nl) {
   if (!kmap || !vmap || c.kv_dtype == DMS_F32 || nl < 1) return cudaErrorInvalidValue;
   if (fused) {
     if (c.kv_dtype != DMS_BF16) return cudaErrorInvalidValue;
-    return c.D == 64 ? launch_cluster_t<64, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms,
-                                                         s, early, nl)
-                     : launch_cluster_t<128, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap,
-                                                          num_sms, s, early, nl);
+    return launch_cluster_dt<false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s, early,
+                                          nl);
   }
   if (c.kv_dtype == DMS_FP8_E4M3)
-    return c.D == 64 ? launch_cluster_t<64, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s,
-                                                         early, nl)
-                     : launch_cluster_t<128, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s,
-                                                          early, nl);
-  return c.D == 64 ? launch_cluster_t<64, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s,
-                                                        early, nl)
-                   : launch_cluster_t<128, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s,
-                                                         early, nl);
+    return launch_cluster_dt<true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early, nl);
+  return launch_cluster_dt<false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early, nl);
 }
 
 }  // namespace dms
