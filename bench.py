@@ -233,9 +233,9 @@ def kernel_launches_per_step(wl, n_dec, stacked=False):
 
 def decode_kernel_name(wl, choice, num_sms):
     """The decode kernel the library runs for this workload (its AUTO rule:
-    the cluster kernel while batch * Hkv * 8 <= 2 * SMs)."""
+    the cluster kernel)."""
     if choice == "auto":
-        choice = "cluster" if wl.batch * wl.kv_heads * 8 <= 2 * num_sms else "flat"
+        choice = "cluster"
     return "k_decode_" + choice
 
 

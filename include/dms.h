@@ -90,12 +90,12 @@ enum dms_alpha_source {
   DMS_ALPHA_SCORE_LINEAR = 3
 };
 
-/* Decode attention kernels.  CLUSTER: one thread-block cluster per (b, h),
- * partials combined on chip (lowest latency when B * Hkv is small).  FLAT: one
- * CTA per SM over a balanced list of every head's slots, partials combined by
- * the last CTA to finish a head (keeps HBM busy at any batch).  AUTO picks
- * CLUSTER when B * Hkv * 8 <= 2 * SMs (every head gets a full cluster of 8),
- * else FLAT; FLAT falls back to CLUSTER for shapes it does not stage. */
+/* Decode attention kernels.  CLUSTER: one thread-block cluster per (b, h)
+ * (cluster size from 8 down to 1 as B * Hkv grows), partials combined on chip.
+ * FLAT: one CTA per SM over a balanced list of every head's slots, partials
+ * combined by the last CTA to finish a head (for heads of very different
+ * lengths).  AUTO picks CLUSTER; FLAT falls back to CLUSTER for shapes it does
+ * not stage. */
 enum dms_decode_kernel { DMS_DECODE_AUTO = 0, DMS_DECODE_CLUSTER = 1, DMS_DECODE_FLAT = 2 };
 
 /* ---- cache descriptor ---------------------------------------------------------

@@ -199,7 +199,7 @@ struct dms_cache {
   std::vector<int> positions;  // host copy of tokens appended per layer
   std::vector<char> prefilled;
   CUtensorMap kmap, vmap;      // pool pages, 16-row boxes
-  CUtensorMap kmap64, vmap64;  // pool pages, 64-row boxes (flat decode kernel)
+  CUtensorMap kmap32, vmap32;  // pool pages, 32-row boxes (flat decode kernel)
   bool has_maps;
   CUtensorMap kept_kmap, kept_vmap;  // tcgen05 prefill: kept copies
   CUtensorMap win_kmap, win_vmap;    // tcgen05 prefill of a later chunk: window copies
@@ -322,7 +322,7 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
     int prev = cur;
     if (prev != c->device) cudaSetDevice(c->device);
     c->has_maps = make_pool_map(&c->kmap, v.k_pool, desc, 16) && make_pool_map(&c->vmap, v.v_pool, desc, 16) &&
-                  make_pool_map(&c->kmap64, v.k_pool, desc, 64) && make_pool_map(&c->vmap64, v.v_pool, desc, 64);
+                  make_pool_map(&c->kmap32, v.k_pool, desc, 32) && make_pool_map(&c->vmap32, v.v_pool, desc, 32);
     if (prev != c->device) cudaSetDevice(prev);
     if (!c->has_maps) {
       delete c;
@@ -674,11 +674,10 @@ int run_decode_kernel(dms_cache* c, int layer, const void* q, void* o, bool fuse
   const CacheView& cv = c->view;
   const bool early = track_launch(c, layer, s);
   int mode = c->desc.decode_kernel;
-  if (mode == DMS_DECODE_AUTO)
-    mode = static_cast<long>(cv.B) * cv.Hkv * 8 <= 2L * c->num_sms ? DMS_DECODE_CLUSTER : DMS_DECODE_FLAT;
+  if (mode == DMS_DECODE_AUTO) mode = DMS_DECODE_CLUSTER;
   if (mode == DMS_DECODE_FLAT) {
     bool taken = false;
-    if (launch_decode_flat(cv, layer, q, o, fused, k, v, alpha, da, &c->kmap64, &c->vmap64, s, early, &taken) !=
+    if (launch_decode_flat(cv, layer, q, o, fused, k, v, alpha, da, &c->kmap32, &c->vmap32, s, early, &taken) !=
         cudaSuccess)
       return DMS_ERR_CUDA;
     if (taken) return DMS_OK;

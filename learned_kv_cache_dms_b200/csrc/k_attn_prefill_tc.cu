@@ -531,10 +531,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (pen_tma) {
             const int st = t % ST;
             ok = ok && mbar_wait_bounded(&v_full[st], (t / ST) & 1);
-            const float* pr = &s_pen[st][0];
+            // (16-byte loads of the row every lane reads alike)
+            const float4* pr = reinterpret_cast<const float4*>(&s_pen[st][0]);
 #pragma unroll
-            for (int n = 0; n < kPfBN; ++n)
-              if (n >= c_lo && n <= c_hi) sv[n] = fmaf(pr[n], rs, sv[n]);
+            for (int n4 = 0; n4 < kPfBN / 4; ++n4) {
+              const float4 pv = pr[n4];
+              const float pe[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int n = 4 * n4 + e;
+                if (n >= c_lo && n <= c_hi) sv[n] = fmaf(pe[e], rs, sv[n]);
+              }
+            }
           } else {
             const float* pr = pen + static_cast<long>(it.bh) * T + jb;
 #pragma unroll

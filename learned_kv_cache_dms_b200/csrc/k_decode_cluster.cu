@@ -50,7 +50,7 @@ template <int D, bool FP8>
 struct ClusterSmem {
   static constexpr int TILE = FP8 ? kCRows * D : kCRows * D * 2;  // K (or V) of one sub-tile, as loaded
   static constexpr int STAGE = 2 * TILE;                           // K then V (a multiple of 1024 bytes)
-  static constexpr int MPER = D == 64 ? 4 : 2;                     // stages per warp
+  static constexpr int MPER = D == 64 ? 4 : 2;                     // stages per warp (at most)
   static constexpr int NST = 4 * MPER;
   static constexpr int CONV_WARP = FP8 ? 2 * kCRows * D * 2 : 0;   // widened bf16 K and V, per warp
   static constexpr int MLD = D + 2;
@@ -60,8 +60,8 @@ struct ClusterSmem {
   __host__ __device__ static int merge_floats(int g) { return (5 * g * MLD + 3) / 4 * 4; }
   // stages, conversion tile, merge buffer, the owner's inbox [cs][g][IMLD],
   // weights [max(cs, 5)][g], row maxima and sums [2][16]
-  static size_t bytes(int g, int cs) {
-    return 1024 + NST * STAGE + 4 * CONV_WARP + (merge_floats(g) + cs * g * IMLD) * sizeof(float) +
+  static size_t bytes(int g, int cs, int mper) {
+    return 1024 + 4 * mper * STAGE + 4 * CONV_WARP + (merge_floats(g) + cs * g * IMLD) * sizeof(float) +
            (kMaxCluster * 16 + 32) * sizeof(float);
   }
 };
@@ -75,6 +75,7 @@ struct SubMeta {
 template <int D, bool FP8, bool FUSED, bool TQ>
 __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int layer, int nl, int early,
                                                             const __nv_bfloat16* q, __nv_bfloat16* o, int cs,
+                                                            int mper,
                                                             const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
                                                             float* alpha, DecideArgs da, int fuse_decide,
                                                             const __grid_constant__ CUtensorMap kmap,
@@ -84,8 +85,8 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sbase =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* stage_buf = sbase;                              // [NST] stages; warp w owns w, w + 4, ...
-  unsigned char* conv_buf = sbase + S::NST * S::STAGE;           // FP8: [4 warps] widened K, V
+  unsigned char* stage_buf = sbase;                              // [4 mper] stages; warp w owns w, w + 4, ...
+  unsigned char* conv_buf = sbase + 4 * mper * S::STAGE;         // FP8: [4 warps] widened K, V
   const int g = c.Hq / c.Hkv;
   float* merge = reinterpret_cast<float*>(conv_buf + 4 * S::CONV_WARP);  // [5 sources][g][MLD]
   float* inbox = merge + S::merge_floats(g);  // [cs][g][IMLD] partials, on the owner (16-byte aligned)
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     griddep_launch_dependents();
   }
   if (tid == 0) {
-    for (int i = 0; i < S::NST; ++i) mbar_init(&full_bar[i], 1);
+    for (int i = 0; i < 4 * mper; ++i) mbar_init(&full_bar[i], 1);
     mbar_init(&inbox_bar, 1);
     fence_mbar_init();
   }
@@ -163,12 +164,12 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
 
   // sub-tile n of this CTA: slots [max(s_begin, (first + n) C), min(s_end, (first + n + 1) C)),
   // inside one page (C divides P); warp n % 4 takes it into stage
-  // n % 4 + 4 ((n / 4) mod MPER), issued by the warp's lane 0
+  // n % 4 + 4 ((n / 4) mod mper), issued by the warp's lane 0
   const int chunk = c.P % kCRows == 0 ? kCRows : 16;
   const int first = s_begin / chunk;
   const int nsub = s_end > s_begin ? (s_end - 1) / chunk - first + 1 : 0;
   auto issue = [&](int n) {
-    const int st = warp + 4 * ((n >> 2) % S::MPER);
+    const int st = warp + 4 * ((n >> 2) % mper);
     const int slot = max(s_begin, (first + n) * chunk);
     const int rows = min(s_end, (first + n + 1) * chunk) - slot;
     const int pi = slot / c.P;
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
                                &full_bar[st]);
   };
   if (lane == 0)
-    for (int n = warp; n < nsub && n < 4 * S::MPER; n += 4) issue(n);
+    for (int n = warp; n < nsub && n < 4 * mper; n += 4) issue(n);
   if (FP8) {
     // the scales of this CTA's pages, while the first tiles are in flight
     const int pf = s_begin / c.P, pl = nsub ? min((s_end - 1) / c.P, kPtCache - 1) : pf - 1;
@@ -250,15 +251,15 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   if (FP8) __syncthreads();  // page scales staged
   {
     // this warp's sub-tiles n = warp, warp + 4, ...: local index j, stage
-    // use j / MPER; the refill of a stage follows the warp's own reads of it
+    // use j / mper; the refill of a stage follows the warp's own reads of it
     unsigned char* conv = conv_buf + warp * S::CONV_WARP;
     const int nmine = nsub > warp ? (nsub - warp + 3) / 4 : 0;
     int j = 0;
     bool timed_out = false;
     for (; j < nmine; ++j) {
-      const int n = warp + 4 * j, st = warp + 4 * (j % S::MPER);
+      const int n = warp + 4 * j, st = warp + 4 * (j % mper);
       __syncwarp();
-      if (!mbar_wait_bounded(&full_bar[st], (j / S::MPER) & 1)) {
+      if (!mbar_wait_bounded(&full_bar[st], (j / mper) & 1)) {
         timed_out = true;
         break;
       }
@@ -290,15 +291,15 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
           warp_tile_keys<D, 16, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
       }
       __syncwarp();
-      if (lane == 0 && n + 4 * S::MPER < nsub) {
+      if (lane == 0 && n + 4 * mper < nsub) {
         fence_proxy_async();  // this warp's reads of the stage before the copy that refills it
-        issue(n + 4 * S::MPER);
+        issue(n + 4 * mper);
       }
     }
     if (timed_out) {
       // the copies of this warp still in flight land before the CTA exits
-      for (int jj = j; jj < min(nmine, j + S::MPER); ++jj)
-        mbar_wait_bounded(&full_bar[warp + 4 * (jj % S::MPER)], (jj / S::MPER) & 1);
+      for (int jj = j; jj < min(nmine, j + mper); ++jj)
+        mbar_wait_bounded(&full_bar[warp + 4 * (jj % mper)], (jj / mper) & 1);
       if (lane == 0) set_status(c.ctrl, DMS_ST_TIMEOUT);
     }
   }
@@ -535,56 +536,76 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   }
 }
 
-// Cluster size: the largest power of two <= 8 with cs * B * Hkv <= k * SMs,
-// k the CTAs per SM the kernel's shared memory allows (at most two), whose
-// shared memory fits and which the device can co-schedule.
+// Largest cluster (a power of two <= 8) the device co-schedules at `mper`
+// stages per warp, and the CTAs per SM (1 or 2) its shared memory allows.
 template <int D, bool FP8, bool FUSED, bool TQ>
-static int pick_cluster(int heads, int g, int num_sms) {
-  static int max_cs[17] = {0}, per_sm[17] = {0};  // by g (<= 16)
-  int& m = max_cs[g < 16 ? g : 16];
-  int& k = per_sm[g < 16 ? g : 16];
-  if (m == 0) {
-    m = 1;
-    k = 1;
-    int dev = 0, optin = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    for (int cs = kPickCluster; cs > 1; cs >>= 1) {
-      const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs);
-      if (smem + 4096 > static_cast<size_t>(optin)) continue;  // static shared memory on top
-      if (cudaFuncSetAttribute(k_decode_cluster<D, FP8, FUSED, TQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess) {
-        cudaGetLastError();
-        continue;
-      }
-      cudaLaunchConfig_t cfg = {};
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = cs;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.gridDim = dim3(cs, 1, 1);
-      cfg.blockDim = dim3(kThreads, 1, 1);
-      cfg.dynamicSmemBytes = smem;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, k_decode_cluster<D, FP8, FUSED, TQ>, &cfg) == cudaSuccess && n > 0) {
-        m = cs;
-        int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode_cluster<D, FP8, FUSED, TQ>, kThreads, smem) ==
-                cudaSuccess &&
-            nb > 1)
-          k = 2;
-        cudaGetLastError();
-        break;
-      }
+static void cluster_limits(int g, int mper, int* max_cs, int* per_sm) {
+  *max_cs = 1;
+  *per_sm = 1;
+  int dev = 0, optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  for (int cs = kPickCluster; cs > 1; cs >>= 1) {
+    const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs, mper);
+    if (smem + 4096 > static_cast<size_t>(optin)) continue;  // static shared memory on top
+    if (cudaFuncSetAttribute(k_decode_cluster<D, FP8, FUSED, TQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess) {
       cudaGetLastError();
+      continue;
     }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(cs, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_decode_cluster<D, FP8, FUSED, TQ>, &cfg) == cudaSuccess && n > 0) {
+      *max_cs = cs;
+      int nb = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode_cluster<D, FP8, FUSED, TQ>, kThreads, smem) ==
+              cudaSuccess &&
+          nb > 1)
+        *per_sm = 2;
+      cudaGetLastError();
+      return;
+    }
+    cudaGetLastError();
   }
-  int cs = 1;
-  while (cs * 2 <= m && static_cast<long>(cs) * 2 * heads <= static_cast<long>(k) * num_sms) cs *= 2;
-  return cs;
+}
+
+// Cluster size and stages per warp: the largest power of two cs with
+// cs * heads <= k * SMs (k the CTAs per SM the shared memory allows), at the
+// full stage count, or at half of it when that fits more CTAs per SM and so
+// gives a larger cluster, or when there are more heads than SMs (one CTA per
+// head; more CTAs share each SM).
+template <int D, bool FP8, bool FUSED, bool TQ>
+static void pick_cluster(int heads, int g, int num_sms, int* cs_out, int* mper_out) {
+  using S = ClusterSmem<D, FP8>;
+  static int lim[17][4] = {{0}};  // by g (<= 16): max cs and CTAs per SM at MPER, then at MPER / 2
+  int* l = lim[g < 16 ? g : 16];
+  if (l[0] == 0) {
+    cluster_limits<D, FP8, FUSED, TQ>(g, S::MPER, &l[0], &l[1]);
+    cluster_limits<D, FP8, FUSED, TQ>(g, (S::MPER + 1) / 2, &l[2], &l[3]);
+  }
+  auto size = [&](int m, int k) {
+    int cs = 1;
+    while (cs * 2 <= m && static_cast<long>(cs) * 2 * heads <= static_cast<long>(k) * num_sms) cs *= 2;
+    return cs;
+  };
+  const int full = size(l[0], l[1]), half = size(l[2], l[3]);
+  if (half > full || heads > num_sms) {
+    *cs_out = half;
+    *mper_out = (S::MPER + 1) / 2;
+  } else {
+    *cs_out = full;
+    *mper_out = S::MPER;
+  }
 }
 
 template <int D, bool FP8, bool FUSED, bool TQ>
@@ -596,8 +617,9 @@ static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
   const int heads = nl * c.B * c.Hkv;
-  const int cs = pick_cluster<D, FP8, FUSED, TQ>(heads, g, num_sms);
-  const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs);
+  int cs = 1, mper = 1;
+  pick_cluster<D, FP8, FUSED, TQ>(heads, g, num_sms, &cs, &mper);
+  const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs, mper);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -616,7 +638,7 @@ static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q
   cfg.numAttrs = 2;
   DecideArgs none{};
   return cudaLaunchKernelEx(&cfg, kern, c, layer, nl, early ? 1 : 0, static_cast<const __nv_bfloat16*>(q),
-                            static_cast<__nv_bfloat16*>(o), cs, static_cast<const __nv_bfloat16*>(k),
+                            static_cast<__nv_bfloat16*>(o), cs, mper, static_cast<const __nv_bfloat16*>(k),
                             static_cast<const __nv_bfloat16*>(v), alpha, da ? *da : none, da ? 1 : 0, *kmap, *vmap);
 }
 

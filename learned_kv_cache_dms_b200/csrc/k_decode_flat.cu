@@ -6,15 +6,16 @@
 // at most 62 units), laid end to end; CTA i of the G CTAs (one per SM) takes
 // units [i*U/G, (i+1)*U/G).  Its range covers the tail of one head, whole
 // heads, and the start of another ("segments").  A producer warp streams the
-// range through a ring of shared-memory stages with TMA, one 64-slot sub-tile
-// per stage (never crossing a page; one box per 128-byte column half of K and
-// of V, plus the head's query rows).  Sub-tile n is consumed by consumer warp
-// n mod 4 from one of that warp's own stages (stage w + 4 * (n/4 mod m), m
-// stages per warp, so every use of a stage is ordered by the one warp that
+// range through a ring of shared-memory stages with TMA, one 32-slot sub-tile
+// per stage (never crossing a page; one 32-row box per 128-byte column half of
+// K and of V, plus the head's query rows).  Sub-tile n is consumed by consumer
+// warp n mod 4 from one of that warp's own stages (stage w + 4 * (n/4 mod m),
+// m stages per warp, so every use of a stage is ordered by the one warp that
 // waits on it and no mbarrier is ever waited on two phases ahead), and the
-// warp runs the whole online-softmax update of its 64 keys with the
-// g query heads of the KV head as the M dimension of mma.sync tiles; the four
-// warps' states are merged at the end of each segment ([FastDMS], attention
+// warp runs the whole online-softmax update of its keys on mma.sync tiles
+// (keys as the M dimension and the g <= 8 query heads as N, else the
+// reverse); the four warps' states are merged at the end of each segment
+// ([FastDMS], attention
 // scoring: split-K grouped decode attention over variable-length per-head
 // spans; the balanced flat split keeps every SM streaming whatever the batch
 // and the retained lengths).
@@ -57,7 +58,7 @@ constexpr int kFlatSegMax = 64;                          // head segments per CT
 constexpr int kFlatPtMax = 512;                          // page ids staged per CTA
 constexpr int kFlatSubMax = 256;                         // sub-tile descriptors staged per CTA
 constexpr int kFlatMaxStages = 16;
-constexpr int kFlatRows = 64;                            // slots per sub-tile = rows per TMA box
+constexpr int kFlatRows = 32;                            // slots per sub-tile = rows per TMA box
 
 struct FlatSeg {
   int bh;           // head, b * Hkv + h
@@ -169,7 +170,7 @@ template <int D, bool FP8>
 struct FlatSmem {
   static constexpr int HALVES = D / 64;
   static constexpr int TILE = FP8 ? kFlatRows * D : HALVES * kFlatRows * 128;  // K (or V) of one sub-tile
-  static constexpr int CROWS = D == 64 ? 64 : 32;                              // FP8 rows widened at a time
+  static constexpr int CROWS = kFlatRows;                                      // FP8 rows widened at a time
   static constexpr int CONV_WARP = FP8 ? 2 * CROWS * D * 2 : 0;                // K + V widened, per warp
   static constexpr int MLD = D + 2;
   __host__ __device__ static size_t stage_stride(int g) {
@@ -181,7 +182,7 @@ struct FlatSmem {
   }
 };
 
-template <int D, bool FP8, bool FUSED>
+template <int D, bool FP8, bool FUSED, bool TQ>
 __global__ void __launch_bounds__(kFlatThreads, 1)
     k_decode_flat(CacheView c, int layer, int early, const __nv_bfloat16* q, __nv_bfloat16* o, int nst,
                   const __nv_bfloat16* k_new, const __nv_bfloat16* v_new, float* alpha, DecideArgs da, int fuse_decide,
@@ -403,7 +404,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     if (tid == 0) set_status(c.ctrl, DMS_ST_SPLIT_LIMIT);
     nseg = kFlatSegMax;
   }
-  const int chunk = c.P % kFlatRows == 0 ? kFlatRows : c.P % 32 == 0 ? 32 : 16;
+  const int chunk = c.P % kFlatRows == 0 ? kFlatRows : 16;
   // segments: warps 0 and 1, one lane per segment (kFlatSegMax = 64); their
   // sub-tile, page-id and ring-entry counts are scanned with shuffles
   FlatSeg sg{};
@@ -888,14 +889,16 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
     __syncwarp();
   } else {
     // ---- consumers ---------------------------------------------------------
-    uint32_t qa[KS][4];
-    float acc[NT][4];
+    // TQ (g <= 8): keys as the mma M dimension (warp_tile_keys_t), else queries
+    constexpr int NA = TQ ? D / 16 : NT;
+    uint32_t qa[KS][4], qt[KS][2];
+    float acc[NA][4];
     float mrow[2], lrow[2];
     bool timed_out = false;
     for (int k = 0; k < nseg; ++k) {
       const FlatSeg& sg = segs[k];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+      for (int nt = 0; nt < NA; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
       mrow[0] = mrow[1] = -INFINITY;
       lrow[0] = lrow[1] = 0.f;
       bool have_q = false;
@@ -911,26 +914,33 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
         const unsigned char* stage = sbase + st * stride;
         if (!have_q) {
           load_q_frags<D>(reinterpret_cast<const __nv_bfloat16*>(stage + 2 * F::TILE), g, qa);
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            qt[ks][0] = qa[ks][0];
+            qt[ks][1] = qa[ks][2];
+          }
           have_q = true;
         }
         if (ok && m.rows > 0) {
           const int masked = masked_slot >= 0 ? masked_slot - m.slot : -1;
+          // (a 32-row box is always loaded: rows past the sub-tile are pool
+          // rows, finite, and masked)
+          const unsigned char* kt = stage;
+          const unsigned char* vt = stage + F::TILE;
+          float kl2 = sl2, vs = 1.0f;
           if (FP8) {
             unsigned char* cv = conv_buf + warp * F::CONV_WARP;
-#pragma unroll
-            for (int cb = 0; cb < kFlatRows; cb += F::CROWS) {
-              if (cb >= m.rows) break;
-              widen_fp8_rows<D, F::CROWS, kFlatRows>(stage, cv, cb);
-              __syncwarp();
-              warp_tile_keys<D, F::CROWS, F::CROWS>(cv, cv + F::CROWS * D * 2, m.rows - cb,
-                                                    masked >= 0 ? masked - cb : -1, m.ks * sl2, m.vs, qa, acc, mrow,
-                                                    lrow);
-              __syncwarp();
-            }
-          } else {
-            warp_tile_keys<D, kFlatRows, kFlatRows>(stage, stage + F::TILE, m.rows, masked, sl2, 1.0f, qa, acc,
-                                                    mrow, lrow);
+            widen_fp8_rows<D, F::CROWS, kFlatRows>(stage, cv, 0);
+            __syncwarp();
+            kt = cv;
+            vt = cv + F::CROWS * D * 2;
+            kl2 = m.ks * sl2;
+            vs = m.vs;
           }
+          if constexpr (TQ)
+            warp_tile_keys_t<D, kFlatRows, kFlatRows>(kt, vt, m.rows, masked, kl2, vs, qt, acc, mrow, lrow);
+          else
+            warp_tile_keys<D, kFlatRows, kFlatRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[st]);
@@ -939,7 +949,10 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
       // ---- end of a segment: merge the four warps' states into cpart[k & 1]
       // (once the aux warp has released it) and hand it over -----------------
       const int j = k & 1;
-      warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
+      if constexpr (TQ)
+        warp_state_t_to_smem<D>(merge, warp, g, acc, mrow, lrow);
+      else
+        warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
       if (k >= 2 && !mbar_wait_bounded(&hq_empty[j], ((k >> 1) - 1) & 1)) timed_out = true;
       consumers_sync();
       float* cpj = cpart + j * g * MLD;
@@ -966,7 +979,7 @@ __global__ void __launch_bounds__(kFlatThreads, 1)
 
 // Launch geometry of the flat kernel, or false when the shape is outside what
 // it stages in shared memory (the caller then takes the cluster kernel).
-template <int D, bool FP8, bool FUSED>
+template <int D, bool FP8, bool FUSED, bool TQ>
 static bool flat_geometry(const CacheView& c, int* grid, int* nst, size_t* smem) {
   using F = FlatSmem<D, FP8>;
   static int budget = -1;  // dynamic shared memory a block may take beside its static arrays
@@ -975,7 +988,7 @@ static bool flat_geometry(const CacheView& c, int* grid, int* nst, size_t* smem)
     cudaFuncAttributes fa{};
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-        cudaFuncGetAttributes(&fa, k_decode_flat<D, FP8, FUSED>) != cudaSuccess) {
+        cudaFuncGetAttributes(&fa, k_decode_flat<D, FP8, FUSED, TQ>) != cudaSuccess) {
       cudaGetLastError();
       return false;
     }
@@ -1000,15 +1013,15 @@ static bool flat_geometry(const CacheView& c, int* grid, int* nst, size_t* smem)
   return true;
 }
 
-template <int D, bool FP8, bool FUSED>
+template <int D, bool FP8, bool FUSED, bool TQ>
 static cudaError_t launch_flat_t(const CacheView& c, int layer, const void* q, void* o, const void* k, const void* v,
                                  float* alpha, const DecideArgs* da, const CUtensorMap* kmap, const CUtensorMap* vmap,
                                  cudaStream_t s, bool early, bool* taken) {
   int grid = 0, nst = 0;
   size_t smem = 0;
-  *taken = (reinterpret_cast<uintptr_t>(q) & 15) == 0 && flat_geometry<D, FP8, FUSED>(c, &grid, &nst, &smem);
+  *taken = (reinterpret_cast<uintptr_t>(q) & 15) == 0 && flat_geometry<D, FP8, FUSED, TQ>(c, &grid, &nst, &smem);
   if (!*taken) return cudaSuccess;
-  auto kern = k_decode_flat<D, FP8, FUSED>;
+  auto kern = k_decode_flat<D, FP8, FUSED, TQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   DecideArgs none{};
@@ -1027,6 +1040,19 @@ static cudaError_t launch_flat_t(const CacheView& c, int layer, const void* q, v
                             static_cast<const __nv_bfloat16*>(v), alpha, da ? *da : none, da ? 1 : 0, *kmap, *vmap);
 }
 
+// One instantiation per (head dim, page type, fused step, key-major tiles).
+template <bool FP8, bool FUSED>
+static cudaError_t launch_flat_dt(const CacheView& c, int layer, const void* q, void* o, const void* k, const void* v,
+                                  float* alpha, const DecideArgs* da, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                  cudaStream_t s, bool early, bool* taken) {
+  const bool tq = c.Hq / c.Hkv <= 8;
+  if (c.D == 64)
+    return tq ? launch_flat_t<64, FP8, FUSED, true>(c, layer, q, o, k, v, alpha, da, kmap, vmap, s, early, taken)
+              : launch_flat_t<64, FP8, FUSED, false>(c, layer, q, o, k, v, alpha, da, kmap, vmap, s, early, taken);
+  return tq ? launch_flat_t<128, FP8, FUSED, true>(c, layer, q, o, k, v, alpha, da, kmap, vmap, s, early, taken)
+            : launch_flat_t<128, FP8, FUSED, false>(c, layer, q, o, k, v, alpha, da, kmap, vmap, s, early, taken);
+}
+
 cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
                                const CUtensorMap* vmap, cudaStream_t s, bool early, bool* taken) {
@@ -1034,14 +1060,11 @@ cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, voi
   if (!kmap || !vmap || c.kv_dtype == DMS_F32) return cudaErrorInvalidValue;
   if (fused) {
     if (c.kv_dtype != DMS_BF16) return cudaErrorInvalidValue;
-    return c.D == 64 ? launch_flat_t<64, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, s, early, taken)
-                     : launch_flat_t<128, false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, s, early, taken);
+    return launch_flat_dt<false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, s, early, taken);
   }
   if (c.kv_dtype == DMS_FP8_E4M3)
-    return c.D == 64 ? launch_flat_t<64, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken)
-                     : launch_flat_t<128, true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken);
-  return c.D == 64 ? launch_flat_t<64, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken)
-                   : launch_flat_t<128, false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken);
+    return launch_flat_dt<true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken);
+  return launch_flat_dt<false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, s, early, taken);
 }
 
 }  // namespace dms

@@ -11,8 +11,8 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 
-@pytest.mark.parametrize("name,kernel", [("qwen8b", "k_decode_cluster"), ("qwen8b_c8", "k_decode_flat"),
-                                         ("llama1b", "k_decode_cluster"), ("reason36", "k_decode_flat")])
+@pytest.mark.parametrize("name,kernel", [("qwen8b", "k_decode_cluster"), ("qwen8b_c8", "k_decode_cluster"),
+                                         ("llama1b", "k_decode_cluster"), ("reason36", "k_decode_cluster")])
 def test_decode_kernel_name_follows_auto_rule(name, kernel):
     wl = bench.I.WORKLOADS[name]
     assert bench.decode_kernel_name(wl, "auto", 148) == kernel
