@@ -247,7 +247,10 @@ typedef struct dms_prefill_args {
  * SMs and merged with a log-sum-exp combine ([FastDMS], attention scoring:
  * split-K grouped compact decode attention over variable-length per-head live
  * spans).  FP8 pages: when the new row's max |x| / 448 exceeds the page scale,
- * the page's rows are re-encoded at the larger scale before the row is written. */
+ * the page's rows are re-encoded at the larger scale before the row is written.
+ * bf16 and FP8 pages take one launch per step with DMS_DECODE_AUTO or
+ * DMS_DECODE_CLUSTER (FP8 with DMS_DECODE_FLAT: an append launch, then the
+ * attention), plus the neuron / rotary pass when it applies. */
 typedef struct dms_decode_args {
   void* q;                  /* device [B,Hq,D] act dtype (rotated in place)  */
   void* k;                  /* device [B,Hkv,D] act dtype (rotated in place) */
@@ -349,10 +352,9 @@ DMS_API int dms_decode_step(dms_cache* cache, int layer, const dms_decode_args* 
  * q/o [L',B,Hq,D], k/v [L',B,Hkv,D], alpha [L',B,Hkv]; with decision
  * parameters, hidden [L',B,hidden], norm_weight [L',hidden], proj_weight
  * [L',Hkv,hidden], proj_bias [L',Hkv] (or NULL) and offset [L',B,Hkv] (batch
- * stride Hkv) or [L',Hkv] (batch stride 0).  bf16 pages only
- * (DMS_ERR_INVALID otherwise: FP8 pages are re-encoded before they are
- * attended); every layer of the range must be prefilled and hold the same
- * number of tokens (else DMS_ERR_STATE). */
+ * stride Hkv) or [L',Hkv] (batch stride 0).  bf16 or FP8 pages
+ * (DMS_ERR_INVALID for fp32 pages); every layer of the range must be
+ * prefilled and hold the same number of tokens (else DMS_ERR_STATE). */
 DMS_API int dms_decode_step_layers(dms_cache* cache, int layer, int num_layers, const dms_decode_args* args,
                                    void* stream);
 

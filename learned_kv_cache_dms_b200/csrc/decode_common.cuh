@@ -827,6 +827,79 @@ __device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
   return old;
 }
 
+// FP8 append of one token's K and V rows, each into a page of P rows of D
+// codes with one scale per page ([DMS-Qwen3], FP8 KV pages): thread tid < D
+// holds the rows' values kx = k[tid], vx = v[tid] (the others 0), and
+// ks_old / vs_old are the pages' scales before the append.  When a row's
+// amax / 448 exceeds its page's scale, the page's first `rows` rows are first
+// re-encoded from their decoded values at the new scale (16 codes per thread
+// and vector, four vectors in flight), and the scale is raised; then the row
+// is encoded at row `r`.  Called by all kThreads threads of the block; `red`
+// holds 2 * kThreads / 32 floats.  Returns the pages' scales after the append
+// (in every thread).
+__device__ __forceinline__ float2 fp8_append_kv(float kx, float vx, uint8_t* kpage, uint8_t* vpage, float* kscale_p,
+                                               float* vscale_p, float ks_old, float vs_old, int r, int rows, int D,
+                                               float* red) {
+  constexpr int NW = kThreads / 32;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  float ka = fabsf(kx), va = fabsf(vx);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ka = fmaxf(ka, __shfl_xor_sync(0xffffffffu, ka, o));
+    va = fmaxf(va, __shfl_xor_sync(0xffffffffu, va, o));
+  }
+  if (lane == 0) {
+    red[wid] = ka;
+    red[NW + wid] = va;
+  }
+  __syncthreads();
+  ka = va = 0.f;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) {
+    ka = fmaxf(ka, red[i]);
+    va = fmaxf(va, red[NW + i]);
+  }
+  const float ks_new = __fdiv_rn(ka, 448.0f), vs_new = __fdiv_rn(va, 448.0f);
+  const bool kgrow = ks_new > ks_old, vgrow = vs_new > vs_old;
+  const int nvec = rows * D / 16;
+  for (int which = 0; which < 2; ++which) {
+    if (!(which ? vgrow : kgrow)) continue;
+    const float s_old = which ? vs_old : ks_old, s_new = which ? vs_new : ks_new;
+    uint4* pv = reinterpret_cast<uint4*>(which ? vpage : kpage);
+    for (int v0 = 0; v0 < nvec; v0 += 4 * kThreads) {
+      uint4 u[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int vi = v0 + e * kThreads + tid;
+        if (vi < nvec) u[e] = pv[vi];
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int vi = v0 + e * kThreads + tid;
+        if (vi >= nvec) continue;
+        uint8_t* cb = reinterpret_cast<uint8_t*>(&u[e]);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cb[j] = fp8_encode(__fdiv_rn(__fmul_rn(fp8_decode(cb[j]), s_old), s_new));
+        pv[vi] = u[e];
+      }
+    }
+  }
+  const float ks = kgrow ? ks_new : ks_old, vs = vgrow ? vs_new : vs_old;
+  if (kgrow || vgrow) {
+    __syncthreads();  // every code re-encoded before the rows and the scales
+    if (tid == 0) {
+      if (kgrow) *kscale_p = ks_new;
+      if (vgrow) *vscale_p = vs_new;
+    }
+  }
+  if (tid < D) {
+    kpage[static_cast<long>(r) * D + tid] = ks > 0.f ? fp8_encode(__fdiv_rn(kx, ks)) : 0;
+    vpage[static_cast<long>(r) * D + tid] = vs > 0.f ? fp8_encode(__fdiv_rn(vx, vs)) : 0;
+  }
+  __syncthreads();  // `red` reused by the caller
+  return make_float2(ks, vs);
+}
+
 // Distributed shared memory (thread-block clusters).
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -843,6 +916,15 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
+// arrive releasing this thread's prior memory operations to the cluster
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+// this thread's prior generic-proxy writes to global memory, ordered before
+// later async-proxy (TMA) accesses that synchronise with it
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;\n" ::: "memory");
+}
 // Stores into another CTA's shared memory of the cluster that complete their
 // bytes of the transaction count of an mbarrier there (16- and 8-byte aligned).
 __device__ __forceinline__ void st_async_v4(uint32_t addr, float4 v, uint32_t bar) {
@@ -867,6 +949,9 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
+}
+__device__ __forceinline__ void st_dsmem(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ float ld_dsmem(uint32_t addr) {
   float v;

@@ -713,9 +713,11 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
     if (e) return e;
     return dms_decode_attention(c, layer, a->q, a->o, stream);
   }
-  if (c->desc.kv_dtype == DMS_FP8_E4M3) {
-    // FP8 pages may be re-encoded by the append, so the attention follows it:
-    // the append kernel, then the cluster attention over the updated pages.
+  if (c->desc.kv_dtype == DMS_FP8_E4M3 && (c->desc.decode_kernel == DMS_DECODE_FLAT || !c->has_maps)) {
+    // FP8 pages may be re-encoded by the append, so the attention follows it;
+    // the flat kernel has no append-first step: the append kernel, then the
+    // attention over the updated pages.  (The cluster kernel appends first
+    // in the same launch.)
     int e = dms_decode_append(c, layer, a, stream);
     if (e) return e;
     return run_decode_kernel(c, layer, a->q, a->o, false, nullptr, nullptr, nullptr, nullptr,
@@ -743,8 +745,9 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   DecideArgs da{};
   const bool proj = a->decide && !neuron;
   if (proj) da = decide_args(c, a->decide);
-  // bf16 pages: one launch -- attention over the pre-append slots plus the new
-  // token, then the append, with the adapter's decision logits computed inside.
+  // One launch -- bf16 pages: attention over the pre-append slots plus the new
+  // token, then the append; FP8 pages: the append, then the attention over
+  // the updated pages; with the adapter's decision logits computed inside.
   if (int e = run_decode_kernel(c, layer, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, s)) return e;
   c->decoded[layer] = 1;
   c->positions[layer] += 1;
@@ -757,8 +760,8 @@ int dms_decode_step_layers(dms_cache* c, int layer0, int num_layers, const dms_d
   if (!a->q || !a->k || !a->v || !a->o || !a->alpha) return DMS_ERR_INVALID;
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o)) return DMS_ERR_INVALID;
   if ((a->rope_cos == nullptr) != (a->rope_sin == nullptr)) return DMS_ERR_INVALID;
-  // one fused launch: bf16 pages (FP8 pages append before they are attended)
-  if (c->desc.kv_dtype != DMS_BF16 || !c->has_maps) return DMS_ERR_INVALID;
+  // one fused launch of the cluster kernel over the layers (bf16 or FP8 pages)
+  if (c->desc.kv_dtype == DMS_F32 || !c->has_maps) return DMS_ERR_INVALID;
   if (a->decide) {
     int e = check_decide(c, a->decide);
     if (e) return e;

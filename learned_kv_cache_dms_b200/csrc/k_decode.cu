@@ -23,6 +23,7 @@ namespace dms {
 // (RMSNorm over the hidden row, one dot product) and writes it to `alpha`.
 // ---------------------------------------------------------------------------
 constexpr int kAppendThreads = 128;
+static_assert(kAppendThreads == kThreads, "fp8_append_row reduces over kThreads threads");
 
 template <typename TA, bool FP8>
 __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, int layer, const TA* k, const TA* v,
@@ -115,50 +116,10 @@ __global__ void __launch_bounds__(kAppendThreads) k_decode_append(CacheView c, i
       }
     } else {
       const int rows = min(P, cnt_new - (slot / P) * P);  // rows in use in that page after the append
-      for (int which = 0; which < 2; ++which) {
-        const TA* x = which ? vsrc : ksrc;
-        float* scale_p = (which ? c.v_scale : c.k_scale) + id;
-        uint8_t* page = static_cast<uint8_t*>(which ? c.v_pool : c.k_pool) + static_cast<long>(id) * P * D;
-        const float xv = tid < D ? to_f(x[tid]) : 0.f;
-        float amax = fabsf(xv);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        if (lane == 0) s_f[0][wid] = amax;
-        __syncthreads();
-        amax = 0.f;
-        for (int i = 0; i < kAppendThreads / 32; ++i) amax = fmaxf(amax, s_f[0][i]);
-        const float s_new = __fdiv_rn(amax, 448.0f);
-        const float s_old = *scale_p;
-        float scale = s_old;
-        if (s_new > s_old) {
-          // re-encode the page's rows at the larger scale from their decoded
-          // values, 16 codes per thread and vector, four vectors in flight
-          uint4* pv = reinterpret_cast<uint4*>(page);
-          const int nvec = rows * D / 16;
-          for (int v0 = 0; v0 < nvec; v0 += 4 * kAppendThreads) {
-            uint4 u[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int vi = v0 + e * kAppendThreads + tid;
-              if (vi < nvec) u[e] = pv[vi];
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int vi = v0 + e * kAppendThreads + tid;
-              if (vi >= nvec) continue;
-              uint8_t* cb = reinterpret_cast<uint8_t*>(&u[e]);
-#pragma unroll
-              for (int j = 0; j < 16; ++j) cb[j] = fp8_encode(__fdiv_rn(__fmul_rn(fp8_decode(cb[j]), s_old), s_new));
-              pv[vi] = u[e];
-            }
-          }
-          scale = s_new;
-          __syncthreads();  // every code re-encoded before the row and the scale
-          if (tid == 0) *scale_p = s_new;
-        }
-        if (tid < D) page[static_cast<long>(slot % P) * D + tid] = scale > 0.f ? fp8_encode(__fdiv_rn(xv, scale)) : 0;
-        __syncthreads();  // s_f reused
-      }
+      const long pb = static_cast<long>(id) * P * D;
+      fp8_append_kv(tid < D ? to_f(ksrc[tid]) : 0.f, tid < D ? to_f(vsrc[tid]) : 0.f,
+                    static_cast<uint8_t*>(c.k_pool) + pb, static_cast<uint8_t*>(c.v_pool) + pb, c.k_scale + id,
+                    c.v_scale + id, c.k_scale[id], c.v_scale[id], slot % P, rows, D, &s_f[0][0]);
     }
   }
   if (tid == 0) {

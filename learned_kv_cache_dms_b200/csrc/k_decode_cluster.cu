@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   __shared__ SubMeta meta[S::NST];
   __shared__ int s_ring_next;
   __shared__ float s_fred[8], s_alpha;
+  __shared__ int s_app_ok, s_app_id;  // append-first step: the owner's append succeeded, its page
+  __shared__ float s_app_sc[2];       // ... and the page's K and V scales after it
   __shared__ __align__(16) __nv_bfloat16 s_knew[D], s_vnew[D];
   constexpr int kPtCache = 256;  // page-table entries of the head kept in shared memory
   __shared__ int s_pt[kPtCache];
@@ -143,7 +145,18 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   const int4 pl0 = FUSED ? *plan_at(c, li, 0) : make_int4(0, 0, 0, 0);
   const int4 pl1 = FUSED ? *plan_at(c, li, 1) : make_int4(0, 0, 0, 0);
   const int4 pl = (t & 1) ? pl1 : pl0;
-  const int masked_slot = (FUSED && (pl.y & 1)) ? pl.x : -1;
+  // FP8 pages (fused step): the owner appends the token first (the page's
+  // rows are re-encoded when its scale grows) and the attention reads it from
+  // its page with the rest.  The visible slots are those after the append,
+  // assumed to succeed (only the owner's range depends on the outcome: a
+  // failed append can only drop the last slot), and page pa, which the append
+  // writes, is read only after the owner's cluster arrive.  bf16 pages: the
+  // attention covers the slots before the append, without the slot the
+  // token reuses, and takes the token from the input.
+  constexpr bool kAppendFirst = FUSED && FP8;
+  const int cnt_vis = (kAppendFirst && !(pl.y & 5)) ? cnt + 1 : cnt;
+  const int pa = (kAppendFirst && !(pl.y & 4)) ? pl.x / c.P : -1;
+  const int masked_slot = (FUSED && !kAppendFirst && (pl.y & 1)) ? pl.x : -1;
   // The decision logit of the new token: with cs >= 4, rank 0 computes it
   // instead of attending (it sends the logit with an empty partial), so it
   // is off the path of the streaming ranks; with a smaller cluster the owner
@@ -156,18 +169,20 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   const int r0 = rank0_decides ? 1 : 0;  // first streaming rank
   const int oq = owner_decides ? 1 : 2;
   const int nfull = cs - 1 - r0;
-  const int per = nfull == 0 ? 0 : ((4 * cnt + 4 * nfull + oq - 1) / (4 * nfull + oq) + 15) / 16 * 16;
-  const int s_begin = rank < r0 ? 0 : min(cnt, (rank - r0) * per);
-  const int s_end = rank < r0 ? 0 : rank == owner ? cnt : min(cnt, s_begin + per);
+  const int per = nfull == 0 ? 0 : ((4 * cnt_vis + 4 * nfull + oq - 1) / (4 * nfull + oq) + 15) / 16 * 16;
+  const int s_begin = rank < r0 ? 0 : min(cnt_vis, (rank - r0) * per);
+  int s_end = rank < r0 ? 0 : rank == owner ? cnt_vis : min(cnt_vis, s_begin + per);
   __syncthreads();
-  cluster_arrive_relaxed();  // this CTA's barriers are initialised (waited before the first remote store)
+  // this CTA's barriers are initialised (waited before the first remote
+  // store); the owner of an append-first step arrives after its append
+  if (!kAppendFirst || rank != owner) cluster_arrive_relaxed();
 
   // sub-tile n of this CTA: slots [max(s_begin, (first + n) C), min(s_end, (first + n + 1) C)),
   // inside one page (C divides P); warp n % 4 takes it into stage
   // n % 4 + 4 ((n / 4) mod mper), issued by the warp's lane 0
   const int chunk = c.P % kCRows == 0 ? kCRows : 16;
   const int first = s_begin / chunk;
-  const int nsub = s_end > s_begin ? (s_end - 1) / chunk - first + 1 : 0;
+  int nsub = s_end > s_begin ? (s_end - 1) / chunk - first + 1 : 0;
   auto issue = [&](int n) {
     const int st = warp + 4 * ((n >> 2) % mper);
     const int slot = max(s_begin, (first + n) * chunk);
@@ -180,17 +195,45 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     issue_rows<D, FP8, kCRows>(stage_buf + st * S::STAGE, &kmap, &vmap, page * c.P + slot % c.P, rows,
                                &full_bar[st]);
   };
+  // this warp's first stages (those before page pa of an append-first step)
+  int n_init = 0;
   if (lane == 0)
-    for (int n = warp; n < nsub && n < 4 * mper; n += 4) issue(n);
+    for (int n = warp; n < nsub && n < 4 * mper; n += 4) {
+      if (kAppendFirst && max(s_begin, (first + n) * chunk) / c.P == pa) break;
+      issue(n);
+      ++n_init;
+    }
+  n_init = __shfl_sync(0xffffffffu, n_init, 0);
   if (FP8) {
     // the scales of this CTA's pages, while the first tiles are in flight
-    const int pf = s_begin / c.P, pl = nsub ? min((s_end - 1) / c.P, kPtCache - 1) : pf - 1;
-    for (int pi = pf + tid; pi <= pl; pi += kThreads) {
+    // (the page an append-first step writes is read again after its append)
+    const int pf = s_begin / c.P, pe = nsub ? min((s_end - 1) / c.P, kPtCache - 1) : pf - 1;
+    for (int pi = pf + tid; pi <= pe; pi += kThreads) {
+      if (pi == pa) continue;
       s_ksc[pi] = c.k_scale[s_pt[pi]];
       s_vsc[pi] = c.v_scale[s_pt[pi]];
     }
   }
 
+  // append-first owner: what the append needs from this layer's state, before
+  // the wait: this head's rank among the heads needing a new page, or the
+  // page the token goes to and its scales (a new page's are 0)
+  int app_rank = 0, app_page = -1;
+  float app_ks = 0.f, app_vs = 0.f;
+  if (kAppendFirst && rank == owner && pa >= 0) {
+    if (pl.y & 2) {
+      if (warp == 0) {
+        int n_before = 0;
+        for (int i = lane; i < vh; i += 32)
+          n_before += (plan_at(c, static_cast<long>(layer) * BH + i, t)->y & 2) ? 1 : 0;
+        app_rank = __reduce_add_sync(0xffffffffu, n_before);
+      }
+    } else {
+      app_page = pa < kPtCache ? s_pt[pa] : c.page_table[li * c.maxp + pa];
+      app_ks = c.k_scale[app_page];
+      app_vs = c.v_scale[app_page];
+    }
+  }
   if (early) {
     griddep_wait();
     griddep_launch_dependents();
@@ -222,7 +265,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   uint4 kn = make_uint4(0, 0, 0, 0), vn = kn;
   int ring_next = 0;
   if (FUSED && rank == owner) {
-    if (tid < D / 8) {
+    if (!kAppendFirst && tid < D / 8) {
       kn = reinterpret_cast<const uint4*>(k_new + static_cast<long>(vh) * D)[tid];
       vn = reinterpret_cast<const uint4*>(v_new + static_cast<long>(vh) * D)[tid];
     }
@@ -234,6 +277,77 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
       s_alpha = a;
       alpha[bb * c.Hkv + h] = a;
     }
+  }
+  if constexpr (kAppendFirst) {
+    if (rank == owner) {
+      // the append: page id (a new page is numbered from the counter by this
+      // head's rank among the heads needing one), then the K and V codes
+      const int flags = pl.y, slot = pl.x;
+      bool ok = !(flags & 4);
+      int id = app_page;
+      if (ok && (flags & 2)) {
+        if (warp == 0 && lane == 0) s_app_id = next_page0 + app_rank;
+        __syncthreads();
+        id = s_app_id;
+        if (id >= c.pool_pages || pl.w >= c.maxp) ok = false;
+      }
+      float2 sc = make_float2(0.f, 0.f);
+      if (ok) {
+        const int rows = min(c.P, cnt_vis - pa * c.P);  // rows in use in the page after the append
+        const __nv_bfloat16* kr = k_new + static_cast<long>(vh) * D;
+        const __nv_bfloat16* vr = v_new + static_cast<long>(vh) * D;
+        const float kx = tid < D ? __bfloat162float(kr[tid]) : 0.f, vx = tid < D ? __bfloat162float(vr[tid]) : 0.f;
+        const long pbytes = static_cast<long>(c.P) * D;
+        sc = fp8_append_kv(kx, vx, static_cast<uint8_t*>(c.k_pool) + id * pbytes,
+                           static_cast<uint8_t*>(c.v_pool) + id * pbytes, c.k_scale + id, c.v_scale + id, app_ks,
+                           app_vs, slot % c.P, rows, D, s_fred);
+        if ((flags & 2) && tid == 0) c.page_table[li * c.maxp + pa] = id;  // read by ranks past kPtCache pages
+      } else if (!(flags & 1)) {
+        // the token has no slot: the owner's range ends before it
+        s_end = cnt;
+        nsub = s_end > s_begin ? (s_end - 1) / chunk - first + 1 : 0;
+      }
+      if (tid == 0) {
+        // the outcome, read by the other ranks after the barrier
+        s_app_ok = ok ? 1 : 0;
+        s_app_id = id;
+        s_app_sc[0] = sc.x;
+        s_app_sc[1] = sc.y;
+        if (pa >= 0 && pa < kPtCache) {
+          s_pt[pa] = ok ? id : -1;
+          s_ksc[pa] = sc.x;
+          s_vsc[pa] = sc.y;
+        }
+      }
+      fence_proxy_async_global();  // the codes, before the TMA loads that follow the barrier
+      __syncthreads();
+      cluster_arrive_release();
+    }
+    cluster_wait();
+    if (rank != owner) {
+      // the append's outcome from the owner's shared memory: the page's id
+      // and scales (pages past the cached table read them from global memory)
+      if (tid == 0) {
+        const int ok = __float_as_int(ld_dsmem(dsmem_addr(&s_app_ok, owner)));
+        const int id = __float_as_int(ld_dsmem(dsmem_addr(&s_app_id, owner)));
+        const float ks = ld_dsmem(dsmem_addr(&s_app_sc[0], owner)), vs = ld_dsmem(dsmem_addr(&s_app_sc[1], owner));
+        s_app_ok = ok;
+        if (pa >= 0 && pa < kPtCache) {
+          s_pt[pa] = ok ? id : -1;
+          s_ksc[pa] = ks;
+          s_vsc[pa] = vs;
+        }
+      }
+      __syncthreads();
+      if (!s_app_ok && !(pl.y & 1)) {
+        // the token has no slot
+        s_end = min(s_end, cnt);
+        nsub = s_end > s_begin ? (s_end - 1) / chunk - first + 1 : 0;
+      }
+    }
+    // the rest of this warp's first stages
+    if (lane == 0)
+      for (int n = warp + 4 * n_init; n < nsub && n < 4 * mper; n += 4) issue(n);
   }
   // TQ (g <= 8): keys as the mma M dimension (warp_tile_keys_t), else queries
   constexpr int NA = TQ ? D / 16 : NT;
@@ -310,16 +424,16 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     warp_state_t_to_smem<D>(merge, warp, g, acc, mrow, lrow);
   else
     warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
-  const int nsrc = (FUSED && rank == owner) ? 5 : 4;
+  const int nsrc = (FUSED && !kAppendFirst && rank == owner) ? 5 : 4;
   if (FUSED && rank == owner) {
-    if (tid < D / 8) {
+    if (!kAppendFirst && tid < D / 8) {
       reinterpret_cast<uint4*>(s_knew)[tid] = kn;
       reinterpret_cast<uint4*>(s_vnew)[tid] = vn;
     }
     if (tid == 32) s_ring_next = ring_next;
   }
   __syncthreads();
-  if (FUSED && rank == owner) {
+  if (FUSED && !kAppendFirst && rank == owner) {
     // the new token as a fifth source: score q_r . k_new, weight 1, value v_new
     for (int idx = tid; idx < g * D; idx += kThreads)
       merge[(4 * g + idx / D) * MLD + idx % D] = __bfloat162float(s_vnew[idx % D]);
@@ -374,7 +488,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     sm_L[16 + tid] = L;
   }
   __syncthreads();
-  cluster_wait();  // every CTA's barriers are initialised
+  if (!kAppendFirst) cluster_wait();  // every CTA's barriers are initialised
   // this CTA's partial row r: acc (4 values per thread and pass), then (M, L);
   // written into slot `rank` of the owner's inbox (st.async to another rank)
   const uint32_t dst = dsmem_addr(inbox + rank * g * IMLD, owner), rbar = dsmem_addr(&inbox_bar, owner);
@@ -427,7 +541,11 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     const int flags = pl.y, slot = pl.x;
     int id = -1;
     bool ok = !(flags & 4);
-    if (ok && (flags & 2)) {
+    if (kAppendFirst) {
+      // done before the attention
+      ok = s_app_ok != 0;
+      id = s_app_id;
+    } else if (ok && (flags & 2)) {
       // a new page: numbered by this head's rank among the heads that need one
       int n_before = 0;
       for (int i = lane; i < vh; i += 32)
@@ -442,7 +560,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     int cnt_new = cnt, np_new = pl.w;  // pages before the append (plan snapshot)
     if (ok) {
       const long row = static_cast<long>(id) * c.P + slot % c.P;
-      if (lane < D / 8) {
+      if (!kAppendFirst && lane < D / 8) {
         reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.k_pool) + row * D)[lane] =
             reinterpret_cast<const uint4*>(s_knew)[lane];
         reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c.v_pool) + row * D)[lane] =
@@ -663,11 +781,12 @@ cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, 
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early, int nl) {
   if (!kmap || !vmap || c.kv_dtype == DMS_F32 || nl < 1) return cudaErrorInvalidValue;
-  if (fused) {
-    if (c.kv_dtype != DMS_BF16) return cudaErrorInvalidValue;
-    return launch_cluster_dt<false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s, early,
-                                          nl);
-  }
+  if (fused)
+    return c.kv_dtype == DMS_FP8_E4M3
+               ? launch_cluster_dt<true, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s, early,
+                                               nl)
+               : launch_cluster_dt<false, true>(c, layer, q, o, k, v, alpha, fused_decide, kmap, vmap, num_sms, s,
+                                                early, nl);
   if (c.kv_dtype == DMS_FP8_E4M3)
     return launch_cluster_dt<true, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early, nl);
   return launch_cluster_dt<false, false>(c, layer, q, o, k, v, alpha, nullptr, kmap, vmap, num_sms, s, early, nl);

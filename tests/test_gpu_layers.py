@@ -1,6 +1,6 @@
 """dms_decode_step_layers: one decode step of several layers in one launch (a
 stack whose layers do not feed each other within a step, like the synthetic
-36-layer reasoning stack).  Against one oracle cache that replays the same
+36-layer reasoning stack), on bf16 and FP8 pages.  Against one oracle cache that replays the same
 calls in the same order (prefill of each layer, then every step appending to
 layer 0, 1, ...): state and page tables bit for bit, stored pages bit for bit,
 decision logits within 1e-3 (decisions exact), attention within 2e-2.
@@ -23,7 +23,7 @@ def _stack(ts):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("variant", ["proj", "input_shift_left", "proj_layer_d64"])
+@pytest.mark.parametrize("variant", ["proj", "input_shift_left", "proj_layer_d64", "fp8_proj", "fp8_input_d64"])
 def test_decode_step_layers_matches_the_oracle(variant):
     from learned_kv_cache_dms_b200 import binding as B_
     base = BASE
@@ -31,11 +31,18 @@ def test_decode_step_layers_matches_the_oracle(variant):
         base = dataclasses.replace(BASE, source="input", shift=-1, keep=0.3)
     elif variant == "proj_layer_d64":
         base = dataclasses.replace(BASE, D=64, per="layer", B=2, Hq=16)
+    elif variant == "fp8_proj":
+        # FP8 pages: each layer's owner CTA appends (re-encoding the page when
+        # its scale grows) before the attention reads the page
+        base = dataclasses.replace(BASE, kv="fp8")
+    elif variant == "fp8_input_d64":
+        base = dataclasses.replace(BASE, kv="fp8", source="input", D=64, B=2, Hq=16, keep=0.3)
     L, B, T, N = base.layers, base.B, base.T, base.N
     cases = [dataclasses.replace(base, layer=l, seed=80 + l) for l in range(L)]
     ins = [build(c) for c in cases]
     # the oracle: one cache, the GPU's call order
-    oc = O.Cache(L, B, base.Hkv, base.D, base.w, base.P, N, base.pool, base.prealloc, shift=base.shift)
+    oc = O.Cache(L, B, base.Hkv, base.D, base.w, base.P, N, base.pool, base.prealloc, fp8=base.kv == "fp8",
+                 shift=base.shift)
     for l, x in enumerate(ins):
         oc.prefill(l, np.ascontiguousarray(x["evict"][:, :, :T]), x["k_stored"][:, :T].astype(np.float32),
                    x["v"][:, :T].float().numpy())
