@@ -83,6 +83,31 @@ __device__ __forceinline__ void issue_rows(unsigned char* dst, const CUtensorMap
   }
 }
 
+// Issue the TMA loads of one TROWS-row sub-tile starting at pool row `row0`
+// into a stage: K then V, one TROWS-row box per 128-byte column half (bf16,
+// 128-byte swizzle) or one box of 128-byte lines of codes (FP8, 128-byte
+// swizzle; two rows per line for D = 64, row0 even); rows past the sub-tile's own
+// are read along (pool rows, finite; the pool's end reads as zeros) and
+// masked by the consumer.  Called by one thread; completes on `bar`.
+template <int D, bool FP8, int TROWS>
+__device__ __forceinline__ void issue_tile(unsigned char* dst, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                           int row0, uint64_t* bar) {
+  constexpr int HALVES = D / 64, TILE = FP8 ? TROWS * D : TROWS * D * 2;
+  mbar_expect_tx(bar, static_cast<uint32_t>(2 * TILE));
+  if (FP8) {
+    // (64-code rows: the maps' lines hold two rows; row0 is even)
+    const int line0 = D == 64 ? row0 >> 1 : row0;
+    tma_load_2d(dst, kmap, 0, line0, bar);
+    tma_load_2d(dst + TILE, vmap, 0, line0, bar);
+  } else {
+#pragma unroll
+    for (int hf = 0; hf < HALVES; ++hf) {
+      tma_load_2d(dst + hf * TROWS * 128, kmap, hf * 64, row0, bar);
+      tma_load_2d(dst + TILE + hf * TROWS * 128, vmap, hf * 64, row0, bar);
+    }
+  }
+}
+
 // Widen a staged FP8 sub-tile (K then V, unswizzled rows of D codes) to bf16
 // codes (exact) in the 128-byte swizzled layout of `conv` (K then V).
 template <int D>
@@ -467,6 +492,177 @@ __device__ __forceinline__ void warp_tile_keys_t(const unsigned char* kt, const 
       uint32_t a[4];
       ldmatrix_x4_trans(a[0], a[1], a[2], a[3], smem_u32(vt + (chunk / 8) * TROWS * 128 + sw128(key, chunk % 8)));
       mma_bf16_16816(acc[dt], a, pb);
+    }
+  }
+}
+
+// ---- FP8 pages on f16 tensor cores --------------------------------------
+// E4M3 codes convert exactly to f16, two per instruction.  FP8 tiles are
+// staged by TMA as 128-byte lines with the 128-byte swizzle (16-byte chunk c
+// of line l at c ^ (l & 7)): a line is one row of 128 codes, or, for D = 64,
+// two consecutive rows (so that every request TMA makes is 128 bytes), and
+// eight rows' same chunk fall in different banks.
+template <int D>
+__device__ __forceinline__ int fp8_sw_off(int row, int chunk) {
+  if (D == 128) return row * 128 + ((chunk ^ (row & 7)) << 4);
+  const int line = row >> 1;
+  return line * 128 + ((((row & 1) << 2 | chunk) ^ (line & 7)) << 4);
+}
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  const __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+// D = A * B + D, m16n8k16, f16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Widen ROWS rows of a staged, swizzled FP8 tile (D codes per row) to 16-bit
+// values (f16 when F16, else bf16; both exact) in the 128-byte swizzled layout
+// of a ROWS-row tile (column halves of 64 elements), by one warp.
+template <int D, int ROWS, bool F16>
+__device__ __forceinline__ void widen_fp8_tile(const unsigned char* raw, unsigned char* conv) {
+  constexpr int CH = D / 16;
+  const int lane = threadIdx.x & 31;
+  for (int idx = lane; idx < ROWS * CH; idx += 32) {
+    const int r = idx / CH, ch = idx % CH;  // 16 codes of row r
+    const uint4 u = *reinterpret_cast<const uint4*>(raw + fp8_sw_off<D>(r, ch));
+    const uint32_t wsrc[4] = {u.x, u.y, u.z, u.w};
+    uint32_t wds[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t lo = e4m3x2_to_f16x2(wsrc[e]), hi = e4m3x2_to_f16x2(wsrc[e] >> 16);
+      if (F16) {
+        wds[2 * e] = lo;
+        wds[2 * e + 1] = hi;
+      } else {
+        const float2 fl = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+        const float2 fh = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+        wds[2 * e] = pack_bf16(fl.x, fl.y);
+        wds[2 * e + 1] = pack_bf16(fh.x, fh.y);
+      }
+    }
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      const int chunk = 2 * ch + hc;
+      *reinterpret_cast<uint4*>(conv + (chunk / 8) * ROWS * 128 + sw128(r, chunk % 8)) =
+          make_uint4(wds[4 * hc], wds[4 * hc + 1], wds[4 * hc + 2], wds[4 * hc + 3]);
+    }
+  }
+}
+
+// Query rows as f16 B operands of warp_tile_keys_fp8: qh[ks] = Q[lane / 4]
+// [16 ks + 4 (lane % 4) + {0, 1}] and [... + {2, 3}] (rows >= g zero) -- the
+// k order of the K fragments that ldmatrix gives on raw FP8 rows.
+template <int D>
+__device__ __forceinline__ void load_q_frags_fp8(const __nv_bfloat16* qb, int g, uint32_t (&qh)[D / 16][2]) {
+  const int lane = threadIdx.x & 31, r = lane >> 2, j = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    if (r < g) {
+      const uint2 u = *reinterpret_cast<const uint2*>(qb + static_cast<long>(r) * D + 16 * ks + 4 * j);
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+      const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+      qh[ks][0] = pack_f16(a.x, a.y);
+      qh[ks][1] = pack_f16(b.x, b.y);
+    } else {
+      qh[ks][0] = qh[ks][1] = 0u;
+    }
+  }
+}
+
+// warp_tile_keys_t for FP8 pages: S^T = K Q^T with the K fragments taken by
+// ldmatrix straight from the swizzled FP8 rows and converted in registers
+// (lane's word of an 8x8 matrix is 4 codes, k slots 2j + e and 8 + 2j + e
+// holding codes 4j + e and 4j + 2 + e, j = lane % 4; qh follows the same
+// order), then O^T += V^T P^T from V widened to f16 (vt: a ROWS-row tile in
+// the 128-byte swizzled layout).  Scores in the log2 domain with the page's
+// K scale in kscale_l2; P carries the V scale.
+template <int D, int KEYS, int TROWS>
+__device__ __forceinline__ void warp_tile_keys_fp8(const unsigned char* kraw, const unsigned char* vt, int rows,
+                                                   int masked, float kscale_l2, float vscale,
+                                                   const uint32_t (&qh)[D / 16][2], float (&acc)[D / 16][4],
+                                                   float (&mrow)[2], float (&lrow)[2]) {
+  constexpr int MT = KEYS / 16, DT = D / 16;
+  const int lane = threadIdx.x & 31;
+  float s[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
+#pragma unroll
+  for (int kp = 0; kp < D / 32; ++kp) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int i = lane >> 3;
+      const int key = mt * 16 + (lane & 7) + (i & 1) * 8;
+      uint32_t r0, r1, r2, r3;
+      ldmatrix_x4(r0, r1, r2, r3, smem_u32(kraw + fp8_sw_off<D>(key, 2 * kp + (i >> 1))));
+      const uint32_t a0[4] = {e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r0 >> 16),
+                              e4m3x2_to_f16x2(r1 >> 16)};
+      const uint32_t a1[4] = {e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r2 >> 16),
+                              e4m3x2_to_f16x2(r3 >> 16)};
+      mma_f16_16816(s[mt], a0, qh[2 * kp]);
+      mma_f16_16816(s[mt], a1, qh[2 * kp + 1]);
+    }
+  }
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = mt * 16 + (lane >> 2) + (e >> 1) * 8;
+      const float x = (key < rows && key != masked) ? s[mt][e] * kscale_l2 : -INFINITY;
+      s[mt][e] = x;
+      mx[e & 1] = fmaxf(mx[e & 1], x);
+    }
+  float corr[2], mu[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 4));
+    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 8));
+    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 16));
+    const float mn = fmaxf(mrow[j], mx[j]);
+    mu[j] = mn == -INFINITY ? 0.f : mn;
+    corr[j] = exp2f(mrow[j] - mu[j]);
+    mrow[j] = mn;
+  }
+  float rs[2] = {0.f, 0.f};
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float p = exp2f(s[mt][e] - mu[e & 1]);
+      s[mt][e] = p;
+      rs[e & 1] += p;
+    }
+  lrow[0] = lrow[0] * corr[0] + rs[0];
+  lrow[1] = lrow[1] * corr[1] + rs[1];
+#pragma unroll
+  for (int dt = 0; dt < DT; ++dt) {
+    acc[dt][0] *= corr[0];
+    acc[dt][1] *= corr[1];
+    acc[dt][2] *= corr[0];
+    acc[dt][3] *= corr[1];
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    uint32_t pb[2];
+    pb[0] = movmatrix_trans(pack_f16(s[mt][0] * vscale, s[mt][1] * vscale));
+    pb[1] = movmatrix_trans(pack_f16(s[mt][2] * vscale, s[mt][3] * vscale));
+    const int key = mt * 16 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+    for (int dt = 0; dt < DT; ++dt) {
+      const int chunk = 2 * dt + ((lane >> 3) & 1);
+      uint32_t a[4];
+      ldmatrix_x4_trans(a[0], a[1], a[2], a[3], smem_u32(vt + (chunk / 8) * TROWS * 128 + sw128(key, chunk % 8)));
+      mma_f16_16816(acc[dt], a, pb);
     }
   }
 }

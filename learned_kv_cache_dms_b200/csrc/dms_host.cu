@@ -121,20 +121,26 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // Tensor map over a page pool viewed as a 2-D tensor [pool_pages * P rows, D].
 // Boxes are `rows` rows by up to 128 bytes; bf16 tiles use the 128-byte
-// swizzle, FP8 tiles none (they are widened to bf16 in shared memory).
-bool make_pool_map(CUtensorMap* map, void* base, const dms_cache_desc* d, int rows) {
+// swizzle; FP8 tiles none (widened in shared memory row by row), or with
+// `fp8_lines` the 128-byte swizzle over 128-byte lines -- for D = 64 the
+// pool viewed as [pool_pages * P / 2, 128] (two rows per line, boxes of
+// rows / 2 lines) -- for ldmatrix straight from the codes.
+bool make_pool_map(CUtensorMap* map, void* base, const dms_cache_desc* d, int rows, bool fp8_lines = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const int eb = elem_bytes(d->kv_dtype);
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d->head_dim),
-                        static_cast<cuuint64_t>(d->pool_pages) * static_cast<cuuint64_t>(d->block)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d->head_dim) * eb};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(std::min(d->head_dim, 128 / eb)), static_cast<cuuint32_t>(rows)};
+  const bool pair = fp8_lines && d->kv_dtype == DMS_FP8_E4M3 && d->head_dim == 64;
+  const int width = pair ? 128 : d->head_dim;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(width),
+                        static_cast<cuuint64_t>(d->pool_pages) * static_cast<cuuint64_t>(d->block) / (pair ? 2 : 1)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(width) * eb};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(std::min(width, 128 / eb)), static_cast<cuuint32_t>(pair ? rows / 2 : rows)};
   cuuint32_t estr[2] = {1u, 1u};
   CUtensorMapDataType dt = d->kv_dtype == DMS_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                            : d->kv_dtype == DMS_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                                     : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  CUtensorMapSwizzle sw = d->kv_dtype == DMS_FP8_E4M3 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (d->kv_dtype == DMS_FP8_E4M3) sw = fp8_lines ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
   CUresult r = enc(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -200,6 +206,7 @@ struct dms_cache {
   std::vector<char> prefilled;
   CUtensorMap kmap, vmap;      // pool pages, 16-row boxes
   CUtensorMap kmap32, vmap32;  // pool pages, 32-row boxes (flat decode kernel)
+  CUtensorMap kmapc, vmapc;    // pool pages, the cluster decode kernel's boxes (FP8 swizzled)
   bool has_maps;
   CUtensorMap kept_kmap, kept_vmap;  // tcgen05 prefill: kept copies
   CUtensorMap win_kmap, win_vmap;    // tcgen05 prefill of a later chunk: window copies
@@ -321,8 +328,11 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   if (desc->kv_dtype != DMS_F32) {
     int prev = cur;
     if (prev != c->device) cudaSetDevice(c->device);
+    const int crows = decode_cluster_box_rows(desc->head_dim, desc->kv_dtype == DMS_FP8_E4M3);
     c->has_maps = make_pool_map(&c->kmap, v.k_pool, desc, 16) && make_pool_map(&c->vmap, v.v_pool, desc, 16) &&
-                  make_pool_map(&c->kmap32, v.k_pool, desc, 32) && make_pool_map(&c->vmap32, v.v_pool, desc, 32);
+                  make_pool_map(&c->kmap32, v.k_pool, desc, 32) && make_pool_map(&c->vmap32, v.v_pool, desc, 32) &&
+                  make_pool_map(&c->kmapc, v.k_pool, desc, crows, true) &&
+                  make_pool_map(&c->vmapc, v.v_pool, desc, crows, true);
     if (prev != c->device) cudaSetDevice(prev);
     if (!c->has_maps) {
       delete c;
@@ -682,7 +692,7 @@ int run_decode_kernel(dms_cache* c, int layer, const void* q, void* o, bool fuse
       return DMS_ERR_CUDA;
     if (taken) return DMS_OK;
   }
-  return launch_decode_cluster(cv, layer, q, o, fused, k, v, alpha, da, &c->kmap, &c->vmap, c->num_sms, s, early) ==
+  return launch_decode_cluster(cv, layer, q, o, fused, k, v, alpha, da, &c->kmapc, &c->vmapc, c->num_sms, s, early) ==
                  cudaSuccess
              ? DMS_OK
              : DMS_ERR_CUDA;
@@ -798,8 +808,8 @@ int dms_decode_step_layers(dms_cache* c, int layer0, int num_layers, const dms_d
   }
   // every layer of the range in one launch (early reads only after the wait)
   track_launch(c, -1, s);
-  if (launch_decode_cluster(v, layer0, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, &c->kmap,
-                            &c->vmap, c->num_sms, s, false, num_layers) != cudaSuccess)
+  if (launch_decode_cluster(v, layer0, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, &c->kmapc,
+                            &c->vmapc, c->num_sms, s, false, num_layers) != cudaSuccess)
     return DMS_ERR_CUDA;
   for (int l = layer0; l < layer0 + num_layers; ++l) {
     c->decoded[l] = 1;

@@ -506,6 +506,8 @@ cudaError_t launch_decode_flat(const CacheView& c, int layer, const void* q, voi
 // One cluster per (layer, b, h) of layers [layer, layer + nl): with nl > 1
 // every input and output array holds the nl layers back to back (rows
 // layer-major), and the fused step appends to all of them in one launch.
+// Rows of the cluster decode kernel's TMA boxes for head dim D and page type.
+int decode_cluster_box_rows(int D, bool fp8);
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early, int nl = 1);

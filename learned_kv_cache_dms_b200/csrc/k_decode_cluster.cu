@@ -44,15 +44,19 @@ __device__ __forceinline__ float ex2_fast(float x) {
   return y;
 }
 
-constexpr int kCRows = 32;  // slots per warp sub-tile (two 16-row TMA boxes)
+// Slots per warp sub-tile: one TMA box of that many rows per K / V column
+// half (32 rows; 64-row FP8 boxes of 64-byte rows measured slower).
+__host__ __device__ constexpr int cluster_rows(int D, bool FP8) { return (void)D, (void)FP8, 32; }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool TQ>
 struct ClusterSmem {
-  static constexpr int TILE = FP8 ? kCRows * D : kCRows * D * 2;  // K (or V) of one sub-tile, as loaded
+  static constexpr int ROWS = cluster_rows(D, FP8);
+  static constexpr int TILE = FP8 ? ROWS * D : ROWS * D * 2;      // K (or V) of one sub-tile, as loaded
   static constexpr int STAGE = 2 * TILE;                           // K then V (a multiple of 1024 bytes)
   static constexpr int MPER = D == 64 ? 4 : 2;                     // stages per warp (at most)
   static constexpr int NST = 4 * MPER;
-  static constexpr int CONV_WARP = FP8 ? 2 * kCRows * D * 2 : 0;   // widened bf16 K and V, per warp
+  // widened FP8 codes per warp: V (to f16) with key-major tiles, else K and V (to bf16)
+  static constexpr int CONV_WARP = FP8 ? (TQ ? 1 : 2) * ROWS * D * 2 : 0;
   static constexpr int MLD = D + 2;
   static constexpr int IMLD = D + 4;  // inbox row: D values, max, sum, 2 pad (16-byte rows)
   // floats of the merge buffer [5 sources][g][MLD], rounded up so the inbox
@@ -80,7 +84,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
                                                             float* alpha, DecideArgs da, int fuse_decide,
                                                             const __grid_constant__ CUtensorMap kmap,
                                                             const __grid_constant__ CUtensorMap vmap) {
-  using S = ClusterSmem<D, FP8>;
+  using S = ClusterSmem<D, FP8, TQ>;
   constexpr int KS = D / 16, NT = D / 8, MLD = D + 2, IMLD = S::IMLD;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sbase =
@@ -180,7 +184,8 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   // sub-tile n of this CTA: slots [max(s_begin, (first + n) C), min(s_end, (first + n + 1) C)),
   // inside one page (C divides P); warp n % 4 takes it into stage
   // n % 4 + 4 ((n / 4) mod mper), issued by the warp's lane 0
-  const int chunk = c.P % kCRows == 0 ? kCRows : 16;
+  constexpr int kCRows = S::ROWS;
+  const int chunk = c.P % kCRows == 0 ? kCRows : c.P % 32 == 0 ? 32 : 16;
   const int first = s_begin / chunk;
   int nsub = s_end > s_begin ? (s_end - 1) / chunk - first + 1 : 0;
   auto issue = [&](int n) {
@@ -192,8 +197,8 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     meta[st].slot = slot;
     meta[st].rows = rows;
     meta[st].page = page;
-    issue_rows<D, FP8, kCRows>(stage_buf + st * S::STAGE, &kmap, &vmap, page * c.P + slot % c.P, rows,
-                               &full_bar[st]);
+    (void)rows;
+    issue_tile<D, FP8, kCRows>(stage_buf + st * S::STAGE, &kmap, &vmap, page * c.P + slot % c.P, &full_bar[st]);
   };
   // this warp's first stages (those before page pa of an append-first step)
   int n_init = 0;
@@ -204,15 +209,15 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
       ++n_init;
     }
   n_init = __shfl_sync(0xffffffffu, n_init, 0);
-  if (FP8) {
-    // the scales of this CTA's pages, while the first tiles are in flight
-    // (the page an append-first step writes is read again after its append)
-    const int pf = s_begin / c.P, pe = nsub ? min((s_end - 1) / c.P, kPtCache - 1) : pf - 1;
-    for (int pi = pf + tid; pi <= pe; pi += kThreads) {
-      if (pi == pa) continue;
-      s_ksc[pi] = c.k_scale[s_pt[pi]];
-      s_vsc[pi] = c.v_scale[s_pt[pi]];
-    }
+  // the scales of this CTA's pages (FP8), requested while the first tiles
+  // are in flight and stored before the streaming starts (the page an
+  // append-first step writes comes from the append)
+  const int sc_pf = s_begin / c.P, sc_pe = (FP8 && nsub) ? min((s_end - 1) / c.P, kPtCache - 1) : sc_pf - 1;
+  const int sc_pi = sc_pf + tid;
+  float sc_k = 0.f, sc_v = 0.f;
+  if (FP8 && sc_pi <= sc_pe && sc_pi != pa) {
+    sc_k = c.k_scale[s_pt[sc_pi]];
+    sc_v = c.v_scale[s_pt[sc_pi]];
   }
 
   // append-first owner: what the append needs from this layer's state, before
@@ -259,9 +264,14 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   const bool one_trip = c.hidden <= kThreads * kDV * 8;
   DecideLoads<kDV> dq;
   if (decides && one_trip) decide_issue<kDV>(c, dl, b, dsrc, dq);
-  uint32_t qa[KS][4];
+  // (FP8 pages with g <= 8: f16 fragments in the K fragments' k order)
+  constexpr bool kF16 = FP8 && TQ;
+  uint32_t qa[kF16 ? 1 : KS][4], qh[kF16 ? KS : 1][2];
   const __nv_bfloat16* qb = q + (static_cast<long>(bb) * c.Hq + static_cast<long>(h) * g) * D;
-  load_q_frags<D>(qb, g, qa);
+  if constexpr (kF16)
+    load_q_frags_fp8<D>(qb, g, qh);
+  else
+    load_q_frags<D>(qb, g, qa);
   uint4 kn = make_uint4(0, 0, 0, 0), vn = kn;
   int ring_next = 0;
   if (FUSED && rank == owner) {
@@ -349,16 +359,29 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     if (lane == 0)
       for (int n = warp + 4 * n_init; n < nsub && n < 4 * mper; n += 4) issue(n);
   }
+  if (FP8) {
+    if (sc_pi <= sc_pe && sc_pi != pa) {
+      s_ksc[sc_pi] = sc_k;
+      s_vsc[sc_pi] = sc_v;
+    }
+    for (int pi = sc_pf + kThreads + tid; pi <= sc_pe; pi += kThreads) {
+      if (pi == pa) continue;
+      s_ksc[pi] = c.k_scale[s_pt[pi]];
+      s_vsc[pi] = c.v_scale[s_pt[pi]];
+    }
+  }
   // TQ (g <= 8): keys as the mma M dimension (warp_tile_keys_t), else queries
   constexpr int NA = TQ ? D / 16 : NT;
   float acc[NA][4];
 #pragma unroll
   for (int nt = 0; nt < NA; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-  uint32_t qt[KS][2];
+  uint32_t qt[kF16 ? 1 : KS][2];
+  if constexpr (!kF16) {
 #pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
-    qt[ks][0] = qa[ks][0];
-    qt[ks][1] = qa[ks][2];
+    for (int ks = 0; ks < KS; ++ks) {
+      qt[ks][0] = qa[ks][0];
+      qt[ks][1] = qa[ks][2];
+    }
   }
   float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
@@ -385,24 +408,43 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
         const int pi = m.slot / c.P;
         ks = pi < kPtCache ? s_ksc[pi] : c.k_scale[m.page];
         vs = pi < kPtCache ? s_vsc[pi] : c.v_scale[m.page];
-        widen_fp8_rows<D, kCRows, kCRows>(kt, conv, 0);
-        __syncwarp();
-        kt = conv;
       }
-      // a sub-tile of at most 16 slots had one box loaded: the rows after it
-      // hold whatever the stage held before, so only its 16 keys are read
-      const unsigned char* vt = kt + (FP8 ? kCRows * D * 2 : S::TILE);
-      const float kl2 = FP8 ? ks * sl2 : sl2;
-      if constexpr (TQ) {
-        if (m.rows > 16)
-          warp_tile_keys_t<D, kCRows, kCRows>(kt, vt, m.rows, masked, kl2, vs, qt, acc, mrow, lrow);
+      // (a sub-tile of at most 16 slots: the tiles of 16 keys)
+      if constexpr (kF16) {
+        // K straight from the FP8 rows, V widened to f16
+        widen_fp8_tile<D, kCRows, true>(kt + S::TILE, conv);
+        __syncwarp();
+        if (kCRows > 32 && m.rows > 32)
+          warp_tile_keys_fp8<D, kCRows, kCRows>(kt, conv, m.rows, masked, ks * sl2, vs, qh, acc, mrow, lrow);
+        else if (m.rows > 16)
+          warp_tile_keys_fp8<D, 32, kCRows>(kt, conv, m.rows, masked, ks * sl2, vs, qh, acc, mrow, lrow);
         else
-          warp_tile_keys_t<D, 16, kCRows>(kt, vt, m.rows, masked, kl2, vs, qt, acc, mrow, lrow);
+          warp_tile_keys_fp8<D, 16, kCRows>(kt, conv, m.rows, masked, ks * sl2, vs, qh, acc, mrow, lrow);
       } else {
-        if (m.rows > 16)
-          warp_tile_keys<D, kCRows, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
-        else
-          warp_tile_keys<D, 16, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
+        if (FP8) {
+          // K and V widened to bf16
+          widen_fp8_tile<D, kCRows, false>(kt, conv);
+          widen_fp8_tile<D, kCRows, false>(kt + S::TILE, conv + kCRows * D * 2);
+          __syncwarp();
+          kt = conv;
+        }
+        const unsigned char* vt = kt + (FP8 ? kCRows * D * 2 : S::TILE);
+        const float kl2 = FP8 ? ks * sl2 : sl2;
+        if constexpr (TQ) {
+          if (kCRows > 32 && m.rows > 32)
+            warp_tile_keys_t<D, kCRows, kCRows>(kt, vt, m.rows, masked, kl2, vs, qt, acc, mrow, lrow);
+          else if (m.rows > 16)
+            warp_tile_keys_t<D, 32, kCRows>(kt, vt, m.rows, masked, kl2, vs, qt, acc, mrow, lrow);
+          else
+            warp_tile_keys_t<D, 16, kCRows>(kt, vt, m.rows, masked, kl2, vs, qt, acc, mrow, lrow);
+        } else {
+          if (kCRows > 32 && m.rows > 32)
+            warp_tile_keys<D, kCRows, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
+          else if (m.rows > 16)
+            warp_tile_keys<D, 32, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
+          else
+            warp_tile_keys<D, 16, kCRows>(kt, vt, m.rows, masked, kl2, vs, qa, acc, mrow, lrow);
+        }
       }
       __syncwarp();
       if (lane == 0 && n + 4 * mper < nsub) {
@@ -664,7 +706,7 @@ static void cluster_limits(int g, int mper, int* max_cs, int* per_sm) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   for (int cs = kPickCluster; cs > 1; cs >>= 1) {
-    const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs, mper);
+    const size_t smem = ClusterSmem<D, FP8, TQ>::bytes(g, cs, mper);
     if (smem + 4096 > static_cast<size_t>(optin)) continue;  // static shared memory on top
     if (cudaFuncSetAttribute(k_decode_cluster<D, FP8, FUSED, TQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess) {
@@ -704,7 +746,7 @@ static void cluster_limits(int g, int mper, int* max_cs, int* per_sm) {
 // head; more CTAs share each SM).
 template <int D, bool FP8, bool FUSED, bool TQ>
 static void pick_cluster(int heads, int g, int num_sms, int* cs_out, int* mper_out) {
-  using S = ClusterSmem<D, FP8>;
+  using S = ClusterSmem<D, FP8, TQ>;
   static int lim[17][4] = {{0}};  // by g (<= 16): max cs and CTAs per SM at MPER, then at MPER / 2
   int* l = lim[g < 16 ? g : 16];
   if (l[0] == 0) {
@@ -737,7 +779,7 @@ static cudaError_t launch_cluster_t(const CacheView& c, int layer, const void* q
   const int heads = nl * c.B * c.Hkv;
   int cs = 1, mper = 1;
   pick_cluster<D, FP8, FUSED, TQ>(heads, g, num_sms, &cs, &mper);
-  const size_t smem = ClusterSmem<D, FP8>::bytes(g, cs, mper);
+  const size_t smem = ClusterSmem<D, FP8, TQ>::bytes(g, cs, mper);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -776,6 +818,8 @@ static cudaError_t launch_cluster_dt(const CacheView& c, int layer, const void* 
             : launch_cluster_t<128, FP8, FUSED, false>(c, layer, q, o, k, v, alpha, da, kmap, vmap, num_sms, s, early,
                                                        nl);
 }
+
+int decode_cluster_box_rows(int D, bool fp8) { return cluster_rows(D, fp8); }
 
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,

@@ -35,6 +35,12 @@ CASES = {
                               source="query", keep=0.2, seed=7),
     "fp8_d128_input": Case(B=2, T=500, steps=20, Hq=4, Hkv=2, D=128, w=64, P=32, act="bf16", kv="fp8",
                            source="input", keep=0.4, seed=8),
+    # FP8 pages with 16 query heads per KV head (the query-major decode tiles,
+    # codes widened to bf16) and with 8 (key-major f16 tiles), D = 128 and 64
+    "fp8_g16_d128_input": Case(B=2, T=450, steps=16, Hq=32, Hkv=2, D=128, w=64, P=32, act="bf16", kv="fp8",
+                               source="input", keep=0.3, seed=41),
+    "fp8_g8_d64_input_p48": Case(B=2, T=420, steps=16, Hq=16, Hkv=2, D=64, w=64, P=48, act="bf16", kv="fp8",
+                                 source="input", keep=0.3, seed=42),
     "f32_rope_input": Case(B=1, T=200, steps=10, Hq=4, Hkv=1, D=128, w=40, P=16, act="f32", kv="f32",
                            source="input", keep=0.5, rope=True, seed=9),
     # degenerate decision patterns
