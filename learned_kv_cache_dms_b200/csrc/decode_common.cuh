@@ -83,6 +83,24 @@ __device__ __forceinline__ void issue_rows(unsigned char* dst, const CUtensorMap
   }
 }
 
+// 2-D TMA tile load (no multicast) with an L2 cache policy: the KV pages are
+// read once per step, so they are marked first to evict, which keeps the
+// small per-layer state (plans, page tables, ring) resident in L2 between
+// the steps of a deep layer stack.
+__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, int c0, int c1,
+                                                 uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+      "%3}], [%4], %5;\n" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
+
 // Issue the TMA loads of one TROWS-row sub-tile starting at pool row `row0`
 // into a stage: K then V, one TROWS-row box per 128-byte column half (bf16,
 // 128-byte swizzle) or one box of 128-byte lines of codes (FP8, 128-byte
@@ -91,19 +109,19 @@ __device__ __forceinline__ void issue_rows(unsigned char* dst, const CUtensorMap
 // masked by the consumer.  Called by one thread; completes on `bar`.
 template <int D, bool FP8, int TROWS>
 __device__ __forceinline__ void issue_tile(unsigned char* dst, const CUtensorMap* kmap, const CUtensorMap* vmap,
-                                           int row0, uint64_t* bar) {
+                                           int row0, uint64_t* bar, uint64_t policy) {
   constexpr int HALVES = D / 64, TILE = FP8 ? TROWS * D : TROWS * D * 2;
   mbar_expect_tx(bar, static_cast<uint32_t>(2 * TILE));
   if (FP8) {
     // (64-code rows: the maps' lines hold two rows; row0 is even)
     const int line0 = D == 64 ? row0 >> 1 : row0;
-    tma_load_2d(dst, kmap, 0, line0, bar);
-    tma_load_2d(dst + TILE, vmap, 0, line0, bar);
+    tma_load_2d_hint(dst, kmap, 0, line0, bar, policy);
+    tma_load_2d_hint(dst + TILE, vmap, 0, line0, bar, policy);
   } else {
 #pragma unroll
     for (int hf = 0; hf < HALVES; ++hf) {
-      tma_load_2d(dst + hf * TROWS * 128, kmap, hf * 64, row0, bar);
-      tma_load_2d(dst + TILE + hf * TROWS * 128, vmap, hf * 64, row0, bar);
+      tma_load_2d_hint(dst + hf * TROWS * 128, kmap, hf * 64, row0, bar, policy);
+      tma_load_2d_hint(dst + TILE + hf * TROWS * 128, vmap, hf * 64, row0, bar, policy);
     }
   }
 }

@@ -188,6 +188,9 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   const int chunk = c.P % kCRows == 0 ? kCRows : c.P % 32 == 0 ? 32 : 16;
   const int first = s_begin / chunk;
   int nsub = s_end > s_begin ? (s_end - 1) / chunk - first + 1 : 0;
+  // the pages are read once per step: first to leave L2, so that the small
+  // per-step tensors (state, query and new rows, adapter rows) stay there
+  const uint64_t kv_policy = l2_evict_first_policy();
   auto issue = [&](int n) {
     const int st = warp + 4 * ((n >> 2) % mper);
     const int slot = max(s_begin, (first + n) * chunk);
@@ -198,7 +201,8 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     meta[st].rows = rows;
     meta[st].page = page;
     (void)rows;
-    issue_tile<D, FP8, kCRows>(stage_buf + st * S::STAGE, &kmap, &vmap, page * c.P + slot % c.P, &full_bar[st]);
+    issue_tile<D, FP8, kCRows>(stage_buf + st * S::STAGE, &kmap, &vmap, page * c.P + slot % c.P, &full_bar[st],
+                               kv_policy);
   };
   // this warp's first stages (those before page pa of an append-first step)
   int n_init = 0;
@@ -639,40 +643,30 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     return;
   }
 
-  // the head's output rows: weights of the cs partials per row, then O / L
+  // the head's output rows: per row the weights of the cs partials (each
+  // thread for its own row, from the partials' maxima and sums), then O / L,
+  // four consecutive elements of one row per thread and pass; the merging
+  // threads are warps 0-2 in a fused step (warp 3 counts the step), else all
   if (landed) {
-    if (tid < g) {
-      float mk[kPickCluster], M = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < kPickCluster; ++k) {
-        mk[k] = k < cs ? inbox[(k * g + tid) * IMLD + D] : -INFINITY;
-        M = fmaxf(M, mk[k]);
-      }
-      const float Mu = M == -INFINITY ? 0.f : M;
-      float L = 0.f;
-#pragma unroll
-      for (int k = 0; k < kPickCluster; ++k) {
-        if (k < cs) {
-          const float wgt = ex2_fast(mk[k] - Mu);
-          sm_w[k * g + tid] = wgt;
-          L = fmaf(wgt, inbox[(k * g + tid) * IMLD + D + 1], L);
-        }
-      }
-      sm_L[tid] = L;
-    }
-    // the merging threads: warps 0-2 in a fused step (warp 3 counts the step), else all
     constexpr int kMergeThreads = FUSED ? kThreads - 32 : kThreads;
-    asm volatile("bar.sync 1, %0;\n" ::"n"(kMergeThreads) : "memory");
-    // four consecutive elements of one row per thread and pass
     __nv_bfloat16* ob = o + (static_cast<long>(bb) * c.Hq + static_cast<long>(h) * g) * D;
     const bool vec_out = (reinterpret_cast<uintptr_t>(ob) & 7) == 0;
     for (int e4 = tid; e4 < g * (D / 4); e4 += kMergeThreads) {
       const int r = e4 / (D / 4), d = 4 * (e4 % (D / 4));
+      float mk[kPickCluster], M = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kPickCluster; ++k) {
+        mk[k] = k < cs ? inbox[(k * g + r) * IMLD + D] : -INFINITY;
+        M = fmaxf(M, mk[k]);
+      }
+      const float Mu = M == -INFINITY ? 0.f : M;
+      float L = 0.f;
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int k = 0; k < kPickCluster; ++k) {
         if (k < cs) {
-          const float wgt = sm_w[k * g + r];
+          const float wgt = ex2_fast(mk[k] - Mu);
+          L = fmaf(wgt, inbox[(k * g + r) * IMLD + D + 1], L);
           const float4 v = *reinterpret_cast<const float4*>(inbox + (k * g + r) * IMLD + d);
           a.x = fmaf(wgt, v.x, a.x);
           a.y = fmaf(wgt, v.y, a.y);
@@ -680,7 +674,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
           a.w = fmaf(wgt, v.w, a.w);
         }
       }
-      const float L = sm_L[r], inv = L > 0.f ? 1.f / L : 0.f;
+      const float inv = L > 0.f ? 1.f / L : 0.f;
       const uint32_t lo = pack_bf16(a.x * inv, a.y * inv), hi = pack_bf16(a.z * inv, a.w * inv);
       if (vec_out) {
         *reinterpret_cast<uint2*>(ob + r * D + d) = make_uint2(lo, hi);

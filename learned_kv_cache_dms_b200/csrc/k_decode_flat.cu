@@ -102,23 +102,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
-// 2-D TMA tile load (no multicast) with an L2 cache policy: the KV pages are
-// read once per step, so they are marked first to evict, which keeps the
-// small per-layer state (plans, page tables, ring) resident in L2 between
-// the steps of a deep layer stack.
-__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, int c0, int c1,
-                                                 uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
-      "%3}], [%4], %5;\n" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
-  return p;
-}
 
 // Barrier of the four consumer warps only (the producer warp never joins).
 __device__ __forceinline__ void consumers_sync() { asm volatile("barrier.sync 1, 128;\n" ::: "memory"); }
