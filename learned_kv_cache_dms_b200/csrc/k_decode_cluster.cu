@@ -59,14 +59,12 @@ struct ClusterSmem {
   static constexpr int CONV_WARP = FP8 ? (TQ ? 1 : 2) * ROWS * D * 2 : 0;
   static constexpr int MLD = D + 2;
   static constexpr int IMLD = D + 4;  // inbox row: D values, max, sum, 2 pad (16-byte rows)
-  // floats of the merge buffer [5 sources][g][MLD], rounded up so the inbox
+  // floats of the merge buffer [4 warps][g][MLD], rounded up so the inbox
   // after it starts on 16 bytes
-  __host__ __device__ static int merge_floats(int g) { return (5 * g * MLD + 3) / 4 * 4; }
-  // stages, conversion tile, merge buffer, the owner's inbox [cs][g][IMLD],
-  // weights [max(cs, 5)][g], row maxima and sums [2][16]
+  __host__ __device__ static int merge_floats(int g) { return (4 * g * MLD + 3) / 4 * 4; }
+  // stages, conversion tiles, merge buffer, the owner's inbox [cs][g][IMLD]
   static size_t bytes(int g, int cs, int mper) {
-    return 1024 + 4 * mper * STAGE + 4 * CONV_WARP + (merge_floats(g) + cs * g * IMLD) * sizeof(float) +
-           (kMaxCluster * 16 + 32) * sizeof(float);
+    return 1024 + 4 * mper * STAGE + 4 * CONV_WARP + (merge_floats(g) + cs * g * IMLD) * sizeof(float);
   }
 };
 
@@ -77,7 +75,7 @@ struct SubMeta {
 };
 
 template <int D, bool FP8, bool FUSED, bool TQ>
-__global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int layer, int nl, int early,
+__global__ void __launch_bounds__(kThreads, 1) k_decode_cluster(CacheView c, int layer, int nl, int early,
                                                             const __nv_bfloat16* q, __nv_bfloat16* o, int cs,
                                                             int mper,
                                                             const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
@@ -92,10 +90,8 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   unsigned char* stage_buf = sbase;                              // [4 mper] stages; warp w owns w, w + 4, ...
   unsigned char* conv_buf = sbase + 4 * mper * S::STAGE;         // FP8: [4 warps] widened K, V
   const int g = c.Hq / c.Hkv;
-  float* merge = reinterpret_cast<float*>(conv_buf + 4 * S::CONV_WARP);  // [5 sources][g][MLD]
+  float* merge = reinterpret_cast<float*>(conv_buf + 4 * S::CONV_WARP);  // [4 warps][g][MLD]
   float* inbox = merge + S::merge_floats(g);  // [cs][g][IMLD] partials, on the owner (16-byte aligned)
-  float* sm_w = inbox + cs * g * IMLD;                          // [sources][g] weights
-  float* sm_L = sm_w + kMaxCluster * 16;                        // [g]
   __shared__ uint64_t full_bar[S::NST];
   __shared__ uint64_t inbox_bar;  // the owner: every rank's partial has landed
   __shared__ SubMeta meta[S::NST];
@@ -104,6 +100,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   __shared__ int s_app_ok, s_app_id;  // append-first step: the owner's append succeeded, its page
   __shared__ float s_app_sc[2];       // ... and the page's K and V scales after it
   __shared__ __align__(16) __nv_bfloat16 s_knew[D], s_vnew[D];
+  __shared__ float s_xs[16];  // the new token's scores (log2 domain), owner of a bf16 step
   constexpr int kPtCache = 256;  // page-table entries of the head kept in shared memory
   __shared__ int s_pt[kPtCache];
   __shared__ float s_ksc[FP8 ? kPtCache : 1], s_vsc[FP8 ? kPtCache : 1];  // FP8 page scales
@@ -389,6 +386,43 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
   }
   float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+  if (FUSED && !kAppendFirst && rank == owner) {
+    // the new token's rows and ring entry for the merge and the append, and
+    // (warp 0, once its query rows and the new key have landed) its scores
+    // q_r . k_new from the query fragments: lane holds columns
+    // 2 (lane % 4) + {0, 1, 8, 9} of every 16 of rows lane / 4 and lane / 4 + 8
+    if (tid < D / 8) {
+      reinterpret_cast<uint4*>(s_knew)[tid] = kn;
+      reinterpret_cast<uint4*>(s_vnew)[tid] = vn;
+    }
+    if (warp == 0) {
+      __syncwarp();
+      const int ra = lane >> 2, rb = ra + 8;
+      float sa = 0.f, sb = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int col = ks * 16 + 2 * (lane & 3);
+        const float2 k0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_knew[col]));
+        const float2 k1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_knew[col + 8]));
+        const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][0]));
+        const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][1]));
+        const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][2]));
+        const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][3]));
+        sa = fmaf(a0.x, k0.x, fmaf(a0.y, k0.y, fmaf(a1.x, k1.x, fmaf(a1.y, k1.y, sa))));
+        sb = fmaf(b0.x, k0.x, fmaf(b0.y, k0.y, fmaf(b1.x, k1.x, fmaf(b1.y, k1.y, sb))));
+      }
+#pragma unroll
+      for (int o2 = 1; o2 < 4; o2 <<= 1) {
+        sa += __shfl_xor_sync(0xffffffffu, sa, o2);
+        sb += __shfl_xor_sync(0xffffffffu, sb, o2);
+      }
+      if ((lane & 3) == 0) {
+        if (ra < g) s_xs[ra] = sa * sl2;
+        if (rb < g) s_xs[rb] = sb * sl2;
+      }
+    }
+  }
+  if (FUSED && rank == owner && tid == 32) s_ring_next = ring_next;  // read by the append after the merge
   if (FP8) __syncthreads();  // page scales staged
   {
     // this warp's sub-tiles n = warp, warp + 4, ...: local index j, stage
@@ -470,105 +504,66 @@ __global__ void __launch_bounds__(kThreads) k_decode_cluster(CacheView c, int la
     warp_state_t_to_smem<D>(merge, warp, g, acc, mrow, lrow);
   else
     warp_state_to_smem<D>(merge, warp, g, acc, mrow, lrow);
-  const int nsrc = (FUSED && !kAppendFirst && rank == owner) ? 5 : 4;
-  if (FUSED && rank == owner) {
-    if (!kAppendFirst && tid < D / 8) {
-      reinterpret_cast<uint4*>(s_knew)[tid] = kn;
-      reinterpret_cast<uint4*>(s_vnew)[tid] = vn;
-    }
-    if (tid == 32) s_ring_next = ring_next;
-  }
-  __syncthreads();
-  if (FUSED && !kAppendFirst && rank == owner) {
-    // the new token as a fifth source: score q_r . k_new, weight 1, value v_new
-    for (int idx = tid; idx < g * D; idx += kThreads)
-      merge[(4 * g + idx / D) * MLD + idx % D] = __bfloat162float(s_vnew[idx % D]);
-    if (warp == 0) {
-      // q_r . k_new from the query fragments: lane holds columns
-      // 2 (lane % 4) + {0, 1, 8, 9} of every 16 of rows lane / 4 and lane / 4 + 8
-      const int ra = lane >> 2, rb = ra + 8;
-      float sa = 0.f, sb = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        const int col = ks * 16 + 2 * (lane & 3);
-        const float2 k0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_knew[col]));
-        const float2 k1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_knew[col + 8]));
-        const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][0]));
-        const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][1]));
-        const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][2]));
-        const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[ks][3]));
-        sa = fmaf(a0.x, k0.x, fmaf(a0.y, k0.y, fmaf(a1.x, k1.x, fmaf(a1.y, k1.y, sa))));
-        sb = fmaf(b0.x, k0.x, fmaf(b0.y, k0.y, fmaf(b1.x, k1.x, fmaf(b1.y, k1.y, sb))));
-      }
-#pragma unroll
-      for (int o2 = 1; o2 < 4; o2 <<= 1) {
-        sa += __shfl_xor_sync(0xffffffffu, sa, o2);
-        sb += __shfl_xor_sync(0xffffffffu, sb, o2);
-      }
-      if ((lane & 3) == 0) {
-        if (ra < g) {
-          merge[(4 * g + ra) * MLD + D] = sa * sl2;
-          merge[(4 * g + ra) * MLD + D + 1] = 1.0f;
-        }
-        if (rb < g) {
-          merge[(4 * g + rb) * MLD + D] = sb * sl2;
-          merge[(4 * g + rb) * MLD + D + 1] = 1.0f;
-        }
-      }
-      __syncwarp();  // read back by lanes r < g of this warp
-    }
-  }
-  // per row: the sources' weights 2^(m_s - M) and the merged (M, L) (rows
-  // r < g <= 16: lanes of warp 0)
-  if (tid < g) {
-    float M = -INFINITY;
-    for (int sv = 0; sv < nsrc; ++sv) M = fmaxf(M, merge[(sv * g + tid) * MLD + D]);
-    const float Mu = M == -INFINITY ? 0.f : M;
-    float L = 0.f;
-    for (int sv = 0; sv < nsrc; ++sv) {
-      const float wgt = exp2f(merge[(sv * g + tid) * MLD + D] - Mu);
-      sm_w[sv * g + tid] = wgt;
-      L = fmaf(wgt, merge[(sv * g + tid) * MLD + D + 1], L);
-    }
-    sm_L[tid] = M;
-    sm_L[16 + tid] = L;
-  }
   __syncthreads();
   if (!kAppendFirst) cluster_wait();  // every CTA's barriers are initialised
-  // this CTA's partial row r: acc (4 values per thread and pass), then (M, L);
-  // written into slot `rank` of the owner's inbox (st.async to another rank)
+  // This CTA's partial, written into slot `rank` of the owner's inbox
+  // (st.async to another rank): per row the four warps' states and, for the
+  // owner of a bf16 step, the new token (score q_r . k_new, weight 1, value
+  // v_new) merged with weights 2^(m_s - M); each thread takes four values of
+  // one row and works out that row's weights, and the thread of the row's
+  // first four also sends (M, L) -- row 0 with rank 0's decision logit.
+  const bool xsrc = FUSED && !kAppendFirst && rank == owner;
   const uint32_t dst = dsmem_addr(inbox + rank * g * IMLD, owner), rbar = dsmem_addr(&inbox_bar, owner);
   for (int e4 = tid; e4 < g * (D / 4); e4 += kThreads) {
     const int r = e4 / (D / 4), d = 4 * (e4 % (D / 4));
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sv = 0; sv < nsrc; ++sv) {
-      const float wgt = sm_w[sv * g + r];
-      const float* src = merge + (sv * g + r) * MLD + d;
-      v.x = fmaf(wgt, src[0], v.x);
-      v.y = fmaf(wgt, src[1], v.y);
-      v.z = fmaf(wgt, src[2], v.z);
-      v.w = fmaf(wgt, src[3], v.w);
+    float ms[4], M = xsrc ? s_xs[r] : -INFINITY;
+#pragma unroll
+    for (int sv = 0; sv < 4; ++sv) {
+      ms[sv] = merge[(sv * g + r) * MLD + D];
+      M = fmaxf(M, ms[sv]);
     }
-    if (rank != owner)
-      st_async_v4(dst + 4u * static_cast<uint32_t>(r * IMLD + d), v, rbar);
-    else
-      *reinterpret_cast<float4*>(inbox + (owner * g + r) * IMLD + d) = v;
-  }
-  if (tid < g) {
-    // (M, L); row 0 also carries the decision logit from rank 0
-    const float dlog = tid == 0 && rank0_decides && rank == 0 ? s_alpha : 0.f;
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float L = 0.f;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int sv = 0; sv < 4; ++sv) {
+      const float wgt = exp2f(ms[sv] - Mu);
+      const float* src = merge + (sv * g + r) * MLD;
+      L = fmaf(wgt, src[D + 1], L);
+      v.x = fmaf(wgt, src[d], v.x);
+      v.y = fmaf(wgt, src[d + 1], v.y);
+      v.z = fmaf(wgt, src[d + 2], v.z);
+      v.w = fmaf(wgt, src[d + 3], v.w);
+    }
+    if (xsrc) {
+      const float wgt = exp2f(s_xs[r] - Mu);
+      L += wgt;
+      const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_vnew[d]));
+      const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_vnew[d + 2]));
+      v.x = fmaf(wgt, v01.x, v.x);
+      v.y = fmaf(wgt, v01.y, v.y);
+      v.z = fmaf(wgt, v23.x, v.z);
+      v.w = fmaf(wgt, v23.y, v.w);
+    }
+    const float dlog = r == 0 && rank0_decides && rank == 0 ? s_alpha : 0.f;
     if (rank != owner) {
-      if (tid == 0)
-        st_async_v4(dst + 4u * static_cast<uint32_t>(D), make_float4(sm_L[0], sm_L[16], dlog, 0.f), rbar);
-      else
-        st_async_v2(dst + 4u * static_cast<uint32_t>(tid * IMLD + D), sm_L[tid], sm_L[16 + tid], rbar);
+      st_async_v4(dst + 4u * static_cast<uint32_t>(r * IMLD + d), v, rbar);
+      if (d == 0) {
+        if (r == 0)
+          st_async_v4(dst + 4u * static_cast<uint32_t>(D), make_float4(M, L, dlog, 0.f), rbar);
+        else
+          st_async_v2(dst + 4u * static_cast<uint32_t>(r * IMLD + D), M, L, rbar);
+      }
     } else {
-      float* row = inbox + (owner * g + tid) * IMLD + D;
-      row[0] = sm_L[tid];
-      row[1] = sm_L[16 + tid];
-      if (tid == 0) {
-        row[2] = dlog;
-        row[3] = 0.f;
+      float* row = inbox + (owner * g + r) * IMLD;
+      *reinterpret_cast<float4*>(row + d) = v;
+      if (d == 0) {
+        row[D] = M;
+        row[D + 1] = L;
+        if (r == 0) {
+          row[D + 2] = dlog;
+          row[D + 3] = 0.f;
+        }
       }
     }
   }
