@@ -737,7 +737,7 @@ def run_ours(args, world, rank, local, primary=True):
         "bound": "hbm", "achieved": round(comp_bytes / (comp_only_ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"],
         "unit": "GB/s", "frac": round(comp_bytes / (comp_only_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
         "ms": round(comp_only_ms, 4), "algorithmic_bytes": int(comp_bytes),
-        "kernel": ("k_neuron_rope8 + " if neuron_pass else "") + "k_prefill_scan + k_prefill_scatter "
+        "kernel": ("k_neuron_rope8 + " if neuron_pass else "") + "k_prefill_scan_bits + k_prefill_scan_assign + k_prefill_scatter "
                   "(dms_prefill_compact minus dms_decide), L2-cold"}
 
     single_us = measure_single_step(B_, r)

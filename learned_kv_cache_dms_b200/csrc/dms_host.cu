@@ -23,7 +23,7 @@ constexpr int kMaxSmsForWork = 160;  // bound used to size the decode work list
 constexpr int kFuseDecideHeads = 64;  // decode decisions fused into the append up to B*Hkv heads
 
 struct Plan {
-  size_t ctrl, pos, count, carry, npages, page_table, slot_pos, ring, plan, kept, kept_count, kept_upto, kept_k, kept_v, win_k,
+  size_t ctrl, pos, count, carry, npages, page_table, slot_pos, ring, plan, kept, kept_count, kept_upto, scan, kept_k, kept_v, win_k,
       win_v, head_done, part_acc, part_ml, k_scale, v_scale, k_pool, v_pool, total;
   int maxp, cap, pre_pages, items_cap, first_free;
 };
@@ -89,6 +89,7 @@ Plan make_plan(const dms_cache_desc* d) {
   p.kept = take(B * H * d->max_positions * 4, 256);
   p.kept_count = take(B * H * 4, 256);
   p.kept_upto = take(B * H * (d->max_positions + 1) * 4, 256);
+  p.scan = take(B * H * static_cast<size_t>(prefill_scan_stride(d->max_positions, d->window)) * 4, 256);
   const size_t kept_rows_bytes = d->act_dtype == DMS_BF16 ? B * H * d->max_positions * d->head_dim * 2 : 0;
   p.kept_k = take(kept_rows_bytes, 1024);
   p.kept_v = take(kept_rows_bytes, 1024);
@@ -312,6 +313,8 @@ int dms_cache_alloc(const dms_cache_desc* desc, void* dev_mem, size_t bytes, voi
   v.kept = reinterpret_cast<int*>(b + p.kept);
   v.kept_count = reinterpret_cast<int*>(b + p.kept_count);
   v.kept_upto = reinterpret_cast<int*>(b + p.kept_upto);
+  v.scan = reinterpret_cast<int*>(b + p.scan);
+  v.scan_stride = prefill_scan_stride(desc->max_positions, desc->window);
   v.kept_k = desc->act_dtype == DMS_BF16 ? b + p.kept_k : nullptr;
   v.kept_v = desc->act_dtype == DMS_BF16 ? b + p.kept_v : nullptr;
   v.win_k = desc->act_dtype == DMS_BF16 ? b + p.win_k : nullptr;

@@ -40,6 +40,8 @@ struct CacheView {
   int* kept;        // [B,Hkv,max_pos]   prefill scratch: kept positions, ascending
   int* kept_count;  // [B,Hkv]
   int* kept_upto;   // [B,Hkv,max_pos+1] prefill scratch: kept tokens before position t
+  int* scan;        // [B,Hkv][scan_stride] prefill scratch of the two scan launches
+  int scan_stride;
   void* kept_k;     // [B*Hkv, max_pos, D] prefill scratch (bf16 activations): kept keys in list order
   void* kept_v;     //                      and values
   void* win_k;      // [B*Hkv, w, D] prefill scratch (bf16 activations): the keys of the last w positions
@@ -467,6 +469,8 @@ cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, vo
 // a chunked prefill; launch_prefill_context rebuilds the kept list, kept copy
 // and window copy of the layer first).
 size_t prefill_scan_smem(const CacheView& c, int T0, int T);
+// ints of scan scratch per (b, h)
+int prefill_scan_stride(int max_pos, int w);
 cudaError_t launch_prefill_context(const CacheView& c, int layer, int T0, int T, const float* alpha, cudaStream_t s);
 cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T0, int T, const float* alpha, cudaStream_t s);
 cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T0, int T, const void* k, const void* v,

@@ -16,144 +16,231 @@ namespace dms {
 
 __device__ __forceinline__ bool bit_at(const unsigned* bits, int t) { return (bits[t >> 5] >> (t & 31)) & 1u; }
 
-constexpr int kScanU = 16;    // decision-logit words a warp loads before its ballots
 constexpr int kScatterU = 4;  // 16-byte row chunks a thread loads before it stores any
 
-// One CTA per (b, h), over the T tokens of one prefill call at positions
-// T0 .. T0 + T - 1 (T0 > 0: a later chunk of a chunked prefill, continuing
-// from the layer's state).  Shared memory: five arrays of ceil(T/32) words,
-// then (T0 > 0) a snapshot of the ring: the slots and decisions of positions
-// T0 - w .. T0 - 1, read while this kernel rewrites the ring.  With T0 > 0:
+// The replay runs in two launches over (chunk of kScanChunk tokens, (b, h)),
+// so that a batch-1 prompt spreads over many SMs:
+//   k_prefill_scan_bits   each chunk's evict, open and kept-list bits, their
+//                         per-word prefixes within the chunk and the chunk's
+//                         totals, into the layer's scan scratch (the first
+//                         chunk also snapshots the ring and the counts);
+//   k_prefill_scan_assign the chunks' totals summed in order, then every
+//                         retained token of the chunk's slot (root walk over
+//                         the head's bits) and kept-list entry; the last CTA
+//                         grants pages in (b, h) order.
+// A call at positions T0 .. T0 + T - 1 with T0 > 0 (a later chunk of a
+// chunked prefill) continues from the layer's state:
 //   open(t)  also holds when t - w < T0 and token t - w was kept;
 //   root(t)  stops at the first r with r - w < T0: token r takes a fresh slot
 //            (r open), or the slot of the marked token r - w (its ring entry);
 //   fresh slots are numbered from the layer's count; kept-list entries from
 //   the context's kept count (k_prefill_context).
-__global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, int T0, int T, const float* alpha) {
-  extern __shared__ unsigned sm[];
-  const int nw = (T + 31) >> 5;
-  unsigned* ev = sm;                                       // evict bits
-  unsigned* op = sm + nw;                                  // open bits
-  unsigned* kb = sm + 2 * nw;                              // kept-list bits: kept and t < T0 + T - w
-  int* opre = reinterpret_cast<int*>(sm + 3 * nw);         // exclusive prefix of open bits per word
-  int* kpre = reinterpret_cast<int*>(sm + 4 * nw);         // exclusive prefix of kept-list bits per word
-  int* rs = reinterpret_cast<int*>(sm + 5 * nw);           // ring snapshot (T0 > 0)
-  __shared__ int tmp[32];
-  __shared__ int s_last, s_count0, s_kept0;
+constexpr int kScanChunk = 1024;  // tokens per CTA (32 words)
+constexpr int kScanThreads = 256;
 
+// Scan scratch of one (b, h): words of evict, open and kept-list bits and the
+// open / kept-list prefixes of each word within its chunk, then per chunk the
+// open and kept totals, the ring snapshot and the counts before the call.
+struct ScanScratch {
+  int nw, nc, w;
+  unsigned *ev, *op, *kb;
+  int *opre, *kpre, *ctot, *rs, *base;
+  __device__ ScanScratch(const CacheView& c, int bh) {
+    nw = (c.max_pos + 31) >> 5;
+    nc = (c.max_pos + kScanChunk - 1) / kScanChunk;
+    w = c.w;
+    int* p = c.scan + static_cast<long>(bh) * c.scan_stride;
+    ev = reinterpret_cast<unsigned*>(p);
+    op = ev + nw;
+    kb = op + nw;
+    opre = reinterpret_cast<int*>(kb + nw);
+    kpre = opre + nw;
+    ctot = kpre + nw;  // [nc][2]
+    rs = ctot + 2 * nc;
+    base = rs + w;     // count0, kept0
+  }
+};
+
+__global__ void __launch_bounds__(kScanThreads) k_prefill_scan_bits(CacheView c, int layer, int T0, int T,
+                                                                    const float* alpha) {
   const int BH = c.B * c.Hkv;
-  const int bh = blockIdx.x, b = bh / c.Hkv, h = bh % c.Hkv;
+  const int chunk = blockIdx.x, bh = blockIdx.y, b = bh / c.Hkv, h = bh % c.Hkv;
   const long lbh = static_cast<long>(layer) * BH + bh;
   const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
   const float* arow = alpha + (static_cast<long>(b) * c.Hkv + hs) * T;
-  const int tid = threadIdx.x, lane = tid & 31, bd = blockDim.x;
-  const int w = c.w;
-  const int end = T0 + T;  // positions held after this call
-  int* ring = c.ring + lbh * w;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int w = c.w, end = T0 + T;
+  const int t0 = chunk * kScanChunk, t1 = min(T, t0 + kScanChunk);
+  if (t0 >= T) return;
+  ScanScratch sc(c, bh);
+  const int* ring = c.ring + lbh * w;
   // decision shift +1: the mark of the call's first token is the previous
   // token's decision, carried from the previous call (0: the padding, keep)
   const bool carry_in = c.shift == 1 && T0 > 0 && c.carry[lbh] != 0;
-
-  if (T0 > 0) {
-    for (int i = tid; i < w; i += bd) rs[i] = ring[i];
+  if (chunk == 0) {
+    // what the assignment needs from before this call (it rewrites the ring)
+    if (T0 > 0)
+      for (int i = tid; i < w; i += kScanThreads) sc.rs[i] = ring[i];
     if (tid == 0) {
-      s_count0 = c.count[lbh];
-      s_kept0 = c.kept_count[bh];
-    }
-  } else if (tid == 0) {
-    s_count0 = 0;
-    s_kept0 = 0;
-  }
-  // decision of an earlier token e (0 <= e < T0): its ring entry
-  auto evict_before = [&](int e) { return (rs[e % w] & static_cast<int>(RING_EVICT)) != 0; };
-
-  // 1. evict bits (coalesced read, one ballot per 32 tokens).  Warp wid owns
-  //    words wid, wid + nwarp, ...; it issues the loads of kScanU words before
-  //    the first ballot so that they are in flight together.  Token t's mark
-  //    is the decision of token t - shift: +1 the previous token's (the
-  //    carried one for t = 0), -1 the next token's (none yet for the last).
-  const int wid = tid >> 5, nwarp = bd >> 5;
-  for (int w0 = wid; w0 < nw; w0 += nwarp * kScanU) {
-    bool e[kScanU];
-#pragma unroll
-    for (int u = 0; u < kScanU; ++u) {
-      const int t = (w0 + u * nwarp) * 32 + lane, src = t - c.shift;
-      e[u] = t < T && (src >= 0 && src < T ? arow[src] > 0.0f : (src < 0 && carry_in));
-    }
-#pragma unroll
-    for (int u = 0; u < kScanU; ++u) {
-      const unsigned m = __ballot_sync(0xffffffffu, e[u] && !c.disable);
-      if (lane == 0 && w0 + u * nwarp < nw) ev[w0 + u * nwarp] = m;
+      sc.base[0] = T0 > 0 ? c.count[lbh] : 0;
+      sc.base[1] = T0 > 0 ? c.kept_count[bh] : 0;
     }
   }
-  __syncthreads();
-  // 2. open bits and kept-list bits (t is the call's token index, T0 + t its position)
-  for (int t0 = (tid & ~31); t0 < nw * 32; t0 += bd) {
-    const int t = t0 + lane, e = T0 + t - w;
-    const bool o = t < T && (e < 0 || (e >= T0 ? !bit_at(ev, e - T0) : !evict_before(e)));
-    const bool k = T0 + t < end - w && t < T && !bit_at(ev, t);
+  // token t's eviction mark (0 <= t < T) is the decision of token t - shift:
+  // +1 the previous token's (the carried one for t = 0), -1 the next token's
+  // (none yet for the last)
+  auto mark = [&](int t) {
+    const int src = t - c.shift;
+    return !c.disable && (src >= 0 && src < T ? arow[src] > 0.0f : (src < 0 && carry_in));
+  };
+  // evict, open and kept-list bits of the chunk's words (t the call's token
+  // index, T0 + t its position); open(t) reads the mark of token t - w, in
+  // this call or, before it, in the ring
+  const int we = (t1 + 31) >> 5;
+  for (int wi = (t0 >> 5) + wid; wi < we; wi += kScanThreads / 32) {
+    const int t = wi * 32 + lane, e = T0 + t - w;
+    bool ev = false, o = false, k = false;
+    if (t < T) {
+      ev = mark(t);
+      const bool ev_e = e < 0 ? false : (e >= T0 ? mark(e - T0) : (ring[e % w] & static_cast<int>(RING_EVICT)) != 0);
+      o = !ev_e;
+      k = T0 + t < end - w && !ev;
+    }
+    const unsigned me = __ballot_sync(0xffffffffu, ev);
     const unsigned mo = __ballot_sync(0xffffffffu, o);
     const unsigned mk = __ballot_sync(0xffffffffu, k);
     if (lane == 0) {
-      op[t0 >> 5] = mo;
-      kb[t0 >> 5] = mk;
+      sc.ev[wi] = me;
+      sc.op[wi] = mo;
+      sc.kb[wi] = mk;
     }
   }
   __syncthreads();
-  // 3. exclusive scans over words: each thread owns a contiguous run
-  const int per = (nw + bd - 1) / bd;
-  const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
-  int so = 0, sk = 0;
-  for (int i = w0; i < w1; ++i) {
-    so += __popc(op[i]);
-    sk += __popc(kb[i]);
+  // prefixes within the chunk: warp 0, one word per lane (32 words per chunk)
+  if (wid == 0) {
+    const int wi = (t0 >> 5) + lane;
+    const bool in = wi < we;
+    const int po = in ? __popc(sc.op[wi]) : 0, pk = in ? __popc(sc.kb[wi]) : 0;
+    int xo = po, xk = pk;
+#pragma unroll
+    for (int o2 = 1; o2 < 32; o2 <<= 1) {
+      const int ao = __shfl_up_sync(0xffffffffu, xo, o2), ak = __shfl_up_sync(0xffffffffu, xk, o2);
+      if (lane >= o2) {
+        xo += ao;
+        xk += ak;
+      }
+    }
+    if (in) {
+      sc.opre[wi] = xo - po;
+      sc.kpre[wi] = xk - pk;
+    }
+    if (lane == 31) {
+      sc.ctot[2 * chunk] = xo;
+      sc.ctot[2 * chunk + 1] = xk;
+    }
   }
-  int tot_open, tot_keep;
-  int base_o = block_exclusive_scan(so, tmp, &tot_open);
-  int base_k = block_exclusive_scan(sk, tmp, &tot_keep);
-  for (int i = w0; i < w1; ++i) {
-    opre[i] = base_o;
-    kpre[i] = base_k;
-    base_o += __popc(op[i]);
-    base_k += __popc(kb[i]);
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_prefill_scan_assign(CacheView c, int layer, int T0, int T,
+                                                                      const float* alpha) {
+  extern __shared__ unsigned sm[];
+  __shared__ int tmp[32];
+  __shared__ int s_last;
+  const int BH = c.B * c.Hkv;
+  const int chunk = blockIdx.x, bh = blockIdx.y, b = bh / c.Hkv, h = bh % c.Hkv;
+  const long lbh = static_cast<long>(layer) * BH + bh;
+  const int hs = c.alpha_per == DMS_ALPHA_PER_LAYER ? 0 : h;
+  const float* arow = alpha + (static_cast<long>(b) * c.Hkv + hs) * T;
+  const int tid = threadIdx.x, bd = kScanThreads;
+  const int w = c.w, end = T0 + T;
+  const int t0 = chunk * kScanChunk, t1 = min(T, t0 + kScanChunk);
+  const int nch = (T + kScanChunk - 1) / kScanChunk;
+  ScanScratch sc(c, bh);
+  // shared memory: evict, open bits and open prefixes of the words up to the
+  // chunk's end (a root is at or before its token), the chunks' open and kept
+  // bases, the ring snapshot
+  const int nwu = (t1 + 31) >> 5;
+  unsigned* ev = sm;
+  unsigned* op = sm + nwu;
+  int* opre = reinterpret_cast<int*>(sm + 2 * nwu);
+  int* cbase = opre + nwu;  // [nch][2] exclusive bases, then the totals
+  int* rs = cbase + 2 * nch + 2;
+  if (t0 < T) {
+    for (int i = tid; i < nwu; i += bd) {
+      ev[i] = sc.ev[i];
+      op[i] = sc.op[i];
+      opre[i] = sc.opre[i];
+    }
+    if (T0 > 0)
+      for (int i = tid; i < w; i += bd) rs[i] = sc.rs[i];
+  }
+  // the chunks' bases: an exclusive scan of their totals (every CTA alike)
+  {
+    int carry_o = 0, carry_k = 0;
+    for (int i0 = 0; i0 < nch; i0 += bd) {
+      const int i = i0 + tid;
+      const int vo = i < nch ? sc.ctot[2 * i] : 0, vk = i < nch ? sc.ctot[2 * i + 1] : 0;
+      int to, tk;
+      const int xo = block_exclusive_scan(vo, tmp, &to);
+      const int xk = block_exclusive_scan(vk, tmp, &tk);
+      if (i < nch) {
+        cbase[2 * i] = carry_o + xo;
+        cbase[2 * i + 1] = carry_k + xk;
+      }
+      carry_o += to;
+      carry_k += tk;
+    }
+    if (tid == 0) {
+      cbase[2 * nch] = carry_o;
+      cbase[2 * nch + 1] = carry_k;
+    }
   }
   __syncthreads();
-  // 4. slots of the retained tokens; ring of the last w tokens; kept list
-  const int count0 = s_count0, kept0 = s_kept0;
-  int* slot_pos = c.slot_pos + lbh * c.cap;
-  int* kept = c.kept + static_cast<long>(bh) * c.max_pos;
-  int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
-  for (int t = tid; t < T; t += bd) {
-    const int pos = T0 + t;
-    const bool evt = bit_at(ev, t);
-    const unsigned below = (1u << (t & 31)) - 1u;
-    kept_upto[pos] = kept0 + kpre[t >> 5] + __popc(kb[t >> 5] & below);
-    const bool retained = (pos >= end - w) || !evt;
-    if (!retained) continue;
-    int r = t;
-    while (T0 + r - w >= T0 && bit_at(ev, r - w)) r -= w;
-    const int e = T0 + r - w;
-    int slot;
-    if (e >= 0 && e < T0 && evict_before(e))
-      slot = rs[e % w] & RING_SLOT_MASK;  // the marked token of the previous call leaves: its slot
-    else
-      slot = count0 + opre[r >> 5] + __popc(op[r >> 5] & ((1u << (r & 31)) - 1u));
-    slot_pos[slot] = pos;
-    if (pos >= end - w) ring[pos % w] = slot | (evt ? static_cast<int>(RING_EVICT) : 0);
-    if (pos < end - w) kept[kept0 + kpre[t >> 5] + __popc(kb[t >> 5] & below)] = pos;
+  const int count0 = sc.base[0], kept0 = sc.base[1];
+  if (t0 < T) {
+    // slots of the retained tokens; ring of the last w tokens; kept list
+    auto evict_before = [&](int e) { return (rs[e % w] & static_cast<int>(RING_EVICT)) != 0; };
+    int* slot_pos = c.slot_pos + lbh * c.cap;
+    int* kept = c.kept + static_cast<long>(bh) * c.max_pos;
+    int* kept_upto = c.kept_upto + static_cast<long>(bh) * (c.max_pos + 1);
+    int* ring = c.ring + lbh * w;
+    const int kbase = kept0 + cbase[2 * chunk + 1];
+    for (int t = t0 + tid; t < t1; t += bd) {
+      const int pos = T0 + t, wi = t >> 5;
+      const bool evt = bit_at(ev, t);
+      const unsigned below = (1u << (t & 31)) - 1u;
+      const unsigned kbw = sc.kb[wi];
+      const int kr = kbase + sc.kpre[wi] + __popc(kbw & below);
+      kept_upto[pos] = kr;
+      const bool retained = (pos >= end - w) || !evt;
+      if (!retained) continue;
+      int r = t;
+      while (T0 + r - w >= T0 && bit_at(ev, r - w)) r -= w;
+      const int e = T0 + r - w;
+      int slot;
+      if (e >= 0 && e < T0 && evict_before(e))
+        slot = rs[e % w] & RING_SLOT_MASK;  // the marked token of the previous call leaves: its slot
+      else
+        slot = count0 + cbase[2 * (r / kScanChunk)] + opre[r >> 5] + __popc(op[r >> 5] & ((1u << (r & 31)) - 1u));
+      slot_pos[slot] = pos;
+      if (pos >= end - w) ring[pos % w] = slot | (evt ? static_cast<int>(RING_EVICT) : 0);
+      if (pos < end - w) kept[kr] = pos;
+    }
+    if (chunk == nch - 1 && tid == 0) {
+      const int tot_open = cbase[2 * nch], tot_keep = cbase[2 * nch + 1];
+      kept_upto[end] = kept0 + tot_keep;
+      c.count[lbh] = count0 + tot_open;
+      c.kept_count[bh] = kept0 + tot_keep;
+      if (c.shift == 1) c.carry[lbh] = (!c.disable && arow[T - 1] > 0.0f) ? 1 : 0;
+      if (h == 0) c.pos[layer * c.B + b] = end;
+    }
   }
-  if (tid == 0) {
-    kept_upto[end] = kept0 + tot_keep;
-    c.count[lbh] = count0 + tot_open;
-    c.kept_count[bh] = kept0 + tot_keep;
-    if (c.shift == 1) c.carry[lbh] = (!c.disable && arow[T - 1] > 0.0f) ? 1 : 0;
-    if (h == 0) c.pos[layer * c.B + b] = end;
-  }
-  // 5. the last CTA to arrive grants the extra pages of every head, in (b, h)
-  //    row-major order, from the ascending page counter.
+  // the last CTA to arrive grants the extra pages of every head, in (b, h)
+  // row-major order, from the ascending page counter
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&c.ctrl[CTRL_DONE_SCAN], 1) == static_cast<int>(gridDim.x) - 1);
+  if (tid == 0)
+    s_last = (atomicAdd(&c.ctrl[CTRL_DONE_SCAN], 1) == static_cast<int>(gridDim.x * gridDim.y) - 1);
   __syncthreads();
   if (!s_last) return;
   __threadfence();
@@ -195,15 +282,24 @@ __global__ void __launch_bounds__(1024) k_prefill_scan(CacheView c, int layer, i
 }
 
 size_t prefill_scan_smem(const CacheView& c, int T0, int T) {
-  return (static_cast<size_t>((T + 31) / 32) * 5 + (T0 > 0 ? c.w : 0)) * 4;
+  const size_t nwu = (static_cast<size_t>(T) + 31) / 32, nch = (static_cast<size_t>(T) + kScanChunk - 1) / kScanChunk;
+  return (3 * nwu + 2 * nch + 2 + (T0 > 0 ? c.w : 0)) * 4;
+}
+
+int prefill_scan_stride(int max_pos, int w) {
+  const int nw = (max_pos + 31) / 32, nc = (max_pos + kScanChunk - 1) / kScanChunk;
+  return (5 * nw + 2 * nc + w + 2 + 7) / 8 * 8;
 }
 
 cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T0, int T, const float* alpha, cudaStream_t s) {
-  const size_t smem = prefill_scan_smem(c, T0, T);
-  cudaError_t e = cudaFuncSetAttribute(k_prefill_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  const dim3 grid((T + kScanChunk - 1) / kScanChunk, c.B * c.Hkv);
+  k_prefill_scan_bits<<<grid, kScanThreads, 0, s>>>(c, layer, T0, T, alpha);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_prefill_scan<<<c.B * c.Hkv, 1024, smem, s>>>(c, layer, T0, T, alpha);
+  const size_t smem = prefill_scan_smem(c, T0, T);
+  e = cudaFuncSetAttribute(k_prefill_scan_assign, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  k_prefill_scan_assign<<<grid, kScanThreads, smem, s>>>(c, layer, T0, T, alpha);
   return cudaGetLastError();
 }
 
