@@ -1027,13 +1027,6 @@ __device__ __forceinline__ float decide_cta(const CacheView& c, const DecideArgs
   return alpha;
 }
 
-// Programmatic dependent launch: let the next kernel of the stream start its
-// prologue, and wait until every kernel this one depends on has completed.
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-}
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
-
 // Atomic add with acquire-release semantics at GPU scope (returns the old value).
 __device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
   int old;

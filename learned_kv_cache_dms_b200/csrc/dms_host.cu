@@ -682,10 +682,13 @@ namespace {
 // Decode attention over a layer's pages (fused: the whole decode step) with
 // the kernel the descriptor selects; the flat kernel hands shapes it does not
 // stage to the cluster kernel.
+// after_wait: the previous kernel on the stream is a programmatic dependent
+// that waited for everything before it (the rotary pass), so the layer's
+// state may be read before this launch's own wait.
 int run_decode_kernel(dms_cache* c, int layer, const void* q, void* o, bool fused, const void* k, const void* v,
-                      float* alpha, const DecideArgs* da, cudaStream_t s) {
+                      float* alpha, const DecideArgs* da, cudaStream_t s, bool after_wait = false) {
   const CacheView& cv = c->view;
-  const bool early = track_launch(c, layer, s);
+  const bool early = track_launch(c, layer, s) || after_wait;
   int mode = c->desc.decode_kernel;
   if (mode == DMS_DECODE_AUTO) mode = DMS_DECODE_CLUSTER;
   if (mode == DMS_DECODE_FLAT) {
@@ -748,11 +751,15 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CacheView& v = c->view;
   const bool neuron = a->decide && !adapter_source(c->desc.alpha_source);
-  if (neuron || a->rope_cos) {
+  const bool rope = neuron || a->rope_cos;
+  if (rope) {
+    // the decision neuron / rotary pass, a programmatic dependent of the
+    // previous kernel: it waits for it, then lets the step's launch read the
+    // layer's state and request its first tiles while it runs
     track_launch(c, layer, s);
     if (launch_neuron_rope(v, 1, v.pos + static_cast<long>(layer) * v.B, a->q, a->k,
                            neuron ? a->decide->offset : nullptr, neuron ? a->decide->offset_batch_stride : 0, neuron,
-                           a->alpha, a->rope_cos, a->rope_sin, s) != cudaSuccess)
+                           a->alpha, a->rope_cos, a->rope_sin, s, true) != cudaSuccess)
       return DMS_ERR_CUDA;
   }
   DecideArgs da{};
@@ -761,7 +768,8 @@ int dms_decode_step(dms_cache* c, int layer, const dms_decode_args* a, void* str
   // One launch -- bf16 pages: attention over the pre-append slots plus the new
   // token, then the append; FP8 pages: the append, then the attention over
   // the updated pages; with the adapter's decision logits computed inside.
-  if (int e = run_decode_kernel(c, layer, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, s)) return e;
+  if (int e = run_decode_kernel(c, layer, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, s, rope))
+    return e;
   c->decoded[layer] = 1;
   c->positions[layer] += 1;
   c->worklist_layer = layer;
@@ -787,8 +795,10 @@ int dms_decode_step_layers(dms_cache* c, int layer0, int num_layers, const dms_d
   const int B = c->desc.batch, Hq = c->desc.num_q_heads, Hkv = c->desc.num_kv_heads, D = c->desc.head_dim;
   const bool neuron = a->decide && !adapter_source(c->desc.alpha_source);
   const long ostride_layer = a->decide ? static_cast<long>(a->decide->offset_batch_stride ? B * Hkv : Hkv) : 0;
-  if (neuron || a->rope_cos) {
-    // the decision neuron / rotary pass of each layer (its rows of q and k)
+  const bool rope = neuron || a->rope_cos;
+  if (rope) {
+    // the decision neuron / rotary pass of each layer (its rows of q and k),
+    // each a programmatic dependent of the kernel before it
     track_launch(c, -1, s);
     for (int l = 0; l < num_layers; ++l) {
       char* ql = static_cast<char*>(a->q) + static_cast<long>(l) * B * Hq * D * 2;
@@ -796,7 +806,7 @@ int dms_decode_step_layers(dms_cache* c, int layer0, int num_layers, const dms_d
       if (launch_neuron_rope(v, 1, v.pos + static_cast<long>(layer0 + l) * B, ql, kl,
                              neuron ? a->decide->offset + l * ostride_layer : nullptr,
                              neuron ? a->decide->offset_batch_stride : 0, neuron, a->alpha + static_cast<long>(l) * B * Hkv,
-                             a->rope_cos, a->rope_sin, s) != cudaSuccess)
+                             a->rope_cos, a->rope_sin, s, true) != cudaSuccess)
         return DMS_ERR_CUDA;
     }
   }
@@ -809,10 +819,11 @@ int dms_decode_step_layers(dms_cache* c, int layer0, int num_layers, const dms_d
     da.bias_lstride = Hkv;
     da.offset_lstride = ostride_layer;
   }
-  // every layer of the range in one launch (early reads only after the wait)
+  // every layer of the range in one launch (the layers' state read before the
+  // wait only after the rotary passes, which waited for everything before)
   track_launch(c, -1, s);
   if (launch_decode_cluster(v, layer0, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, &c->kmapc,
-                            &c->vmapc, c->num_sms, s, false, num_layers) != cudaSuccess)
+                            &c->vmapc, c->num_sms, s, rope, num_layers) != cudaSuccess)
     return DMS_ERR_CUDA;
   for (int l = layer0; l < layer0 + num_layers; ++l) {
     c->decoded[l] = 1;

@@ -462,9 +462,12 @@ cudaError_t launch_init(const CacheView& c, bool full, cudaStream_t s);
 // box 64 x 64), or null (CUDA-core kernel).
 cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, float* alpha, const CUtensorMap* hmap,
                                cudaStream_t s);
+// pdl: launched as a programmatic dependent of the previous kernel on the
+// stream (the kernels wait for it before reading, then let the next kernel
+// start its prologue).
 cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
                                int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
-                               const float* sin_t, cudaStream_t s);
+                               const float* sin_t, cudaStream_t s, bool pdl = false);
 // Prefill of T tokens at positions T0 .. T0 + T - 1 (T0 > 0: a later chunk of
 // a chunked prefill; launch_prefill_context rebuilds the kept list, kept copy
 // and window copy of the layer first).
@@ -515,5 +518,12 @@ int decode_cluster_box_rows(int D, bool fp8);
 cudaError_t launch_decode_cluster(const CacheView& c, int layer, const void* q, void* o, bool fused, const void* k,
                                   const void* v, float* alpha, const DecideArgs* fused_decide, const CUtensorMap* kmap,
                                   const CUtensorMap* vmap, int num_sms, cudaStream_t s, bool early, int nl = 1);
+
+// Programmatic dependent launch: let the next kernel of the stream start its
+// prologue, and wait until every kernel this one depends on has completed.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
 }  // namespace dms

@@ -502,6 +502,8 @@ cudaError_t launch_decide_proj(const CacheView& c, int T, const DecideArgs& a, f
 template <typename TA>
 __global__ void k_neuron_rope(CacheView c, int T, const int* pos_dev, TA* q, TA* k, const float* offset, int ostride,
                               int do_alpha, float* alpha, const float* cos_t, const float* sin_t) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int D = c.D, half = D / 2, g = c.Hq / c.Hkv;
   const bool key = c.alpha_source == DMS_ALPHA_KEY_NEURON;
   // with rotary tables every (token, row, i < D/2) pair, else only the
@@ -595,6 +597,8 @@ __device__ __forceinline__ float narrow_f64<__nv_bfloat16>(double x) { return f6
 template <typename TA>
 __global__ void k_neuron_rope4(CacheView c, int T, const int* pos_dev, TA* q, TA* k, const float* offset, int ostride,
                                int do_alpha, float* alpha, const float* cos_t, const float* sin_t) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int D = c.D, half = D / 2, nq = half / 4, g = c.Hq / c.Hkv;
   const bool key = c.alpha_source == DMS_ALPHA_KEY_NEURON;
   const int nrow = c.Hq + c.Hkv;
@@ -654,6 +658,8 @@ __global__ void __launch_bounds__(256, 3) k_neuron_rope8(CacheView c, int T, con
                                                       __nv_bfloat16* k, const float* offset, int ostride,
                                                       int do_alpha, float* alpha, const float* cos_t,
                                                       const float* sin_t) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int D = c.D, half = D / 2, nq = half / 8, g = c.Hq / c.Hkv;
   const bool key = c.alpha_source == DMS_ALPHA_KEY_NEURON;
   const int nrow = c.Hq + c.Hkv;
@@ -722,42 +728,54 @@ __global__ void __launch_bounds__(256, 3) k_neuron_rope8(CacheView c, int T, con
   }
 }
 
+// A launch of kern<<<grid, 256, 0, s>>>, as a programmatic dependent of the
+// previous kernel on the stream when pdl is set.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_rope_kernel(void (*kern)(KArgs...), int grid, cudaStream_t s, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
                                int offset_bstride, bool do_alpha, float* alpha, const float* cos_t,
-                               const float* sin_t, cudaStream_t s) {
+                               const float* sin_t, cudaStream_t s, bool pdl) {
   const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                        reinterpret_cast<uintptr_t>(cos_t) | reinterpret_cast<uintptr_t>(sin_t);
+  const int da = do_alpha ? 1 : 0;
   // large bf16 launches: one thread per (token, 8 pairs), rows walked in groups
   const long total8 = static_cast<long>(c.B) * T * (c.D / 16);
   if (cos_t && (al & 15) == 0 && (c.D / 2) % 8 == 0 && c.act_dtype == DMS_BF16 &&
       total8 >= static_cast<long>(c.num_sms) * 256 && total8 < (1L << 30)) {
     const int grid8 = static_cast<int>(min((total8 + 255) / 256, static_cast<long>(c.num_sms) * 3));
-    k_neuron_rope8<<<grid8, 256, 0, s>>>(c, T, pos_dev, static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
-                                         offset, offset_bstride, do_alpha ? 1 : 0, alpha, cos_t, sin_t);
-    return cudaGetLastError();
+    return launch_rope_kernel(k_neuron_rope8, grid8, s, pdl, c, T, pos_dev, static_cast<__nv_bfloat16*>(q),
+                              static_cast<__nv_bfloat16*>(k), offset, offset_bstride, da, alpha, cos_t, sin_t);
   }
   if (cos_t && (al & 15) == 0 && (c.D / 2) % 4 == 0) {
     const long total4 = static_cast<long>(c.B) * T * (c.Hq + c.Hkv) * (c.D / 8);
     const int grid4 = static_cast<int>(max(1L, min((total4 + 255) / 256, static_cast<long>(c.num_sms) * 16)));
     if (c.act_dtype == DMS_BF16)
-      k_neuron_rope4<__nv_bfloat16><<<grid4, 256, 0, s>>>(c, T, pos_dev, static_cast<__nv_bfloat16*>(q),
-                                                           static_cast<__nv_bfloat16*>(k), offset, offset_bstride,
-                                                           do_alpha ? 1 : 0, alpha, cos_t, sin_t);
-    else
-      k_neuron_rope4<float><<<grid4, 256, 0, s>>>(c, T, pos_dev, static_cast<float*>(q), static_cast<float*>(k),
-                                                  offset, offset_bstride, do_alpha ? 1 : 0, alpha, cos_t, sin_t);
-    return cudaGetLastError();
+      return launch_rope_kernel(k_neuron_rope4<__nv_bfloat16>, grid4, s, pdl, c, T, pos_dev,
+                                static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), offset, offset_bstride,
+                                da, alpha, cos_t, sin_t);
+    return launch_rope_kernel(k_neuron_rope4<float>, grid4, s, pdl, c, T, pos_dev, static_cast<float*>(q),
+                              static_cast<float*>(k), offset, offset_bstride, da, alpha, cos_t, sin_t);
   }
   const long total = static_cast<long>(c.B) * T * (cos_t ? (c.Hq + c.Hkv) * (c.D / 2) : c.Hkv);
   const int grid = static_cast<int>(max(1L, min((total + 255) / 256, static_cast<long>(c.num_sms) * 16)));
   if (c.act_dtype == DMS_BF16)
-    k_neuron_rope<__nv_bfloat16><<<grid, 256, 0, s>>>(c, T, pos_dev, static_cast<__nv_bfloat16*>(q),
-                                                       static_cast<__nv_bfloat16*>(k), offset, offset_bstride,
-                                                       do_alpha ? 1 : 0, alpha, cos_t, sin_t);
-  else
-    k_neuron_rope<float><<<grid, 256, 0, s>>>(c, T, pos_dev, static_cast<float*>(q), static_cast<float*>(k), offset,
-                                              offset_bstride, do_alpha ? 1 : 0, alpha, cos_t, sin_t);
-  return cudaGetLastError();
+    return launch_rope_kernel(k_neuron_rope<__nv_bfloat16>, grid, s, pdl, c, T, pos_dev,
+                              static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), offset, offset_bstride,
+                              da, alpha, cos_t, sin_t);
+  return launch_rope_kernel(k_neuron_rope<float>, grid, s, pdl, c, T, pos_dev, static_cast<float*>(q),
+                            static_cast<float*>(k), offset, offset_bstride, da, alpha, cos_t, sin_t);
 }
 
 }  // namespace dms
