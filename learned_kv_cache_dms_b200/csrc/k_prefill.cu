@@ -63,6 +63,8 @@ struct ScanScratch {
 
 __global__ void __launch_bounds__(kScanThreads) k_prefill_scan_bits(CacheView c, int layer, int T0, int T,
                                                                     const float* alpha) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int BH = c.B * c.Hkv;
   const int chunk = blockIdx.x, bh = blockIdx.y, b = bh / c.Hkv, h = bh % c.Hkv;
   const long lbh = static_cast<long>(layer) * BH + bh;
@@ -146,6 +148,8 @@ __global__ void __launch_bounds__(kScanThreads) k_prefill_scan_assign(CacheView 
   extern __shared__ unsigned sm[];
   __shared__ int tmp[32];
   __shared__ int s_last;
+  griddep_wait();
+  griddep_launch_dependents();
   const int BH = c.B * c.Hkv;
   const int chunk = blockIdx.x, bh = blockIdx.y, b = bh / c.Hkv, h = bh % c.Hkv;
   const long lbh = static_cast<long>(layer) * BH + bh;
@@ -293,14 +297,13 @@ int prefill_scan_stride(int max_pos, int w) {
 
 cudaError_t launch_prefill_scan(const CacheView& c, int layer, int T0, int T, const float* alpha, cudaStream_t s) {
   const dim3 grid((T + kScanChunk - 1) / kScanChunk, c.B * c.Hkv);
-  k_prefill_scan_bits<<<grid, kScanThreads, 0, s>>>(c, layer, T0, T, alpha);
-  cudaError_t e = cudaGetLastError();
+  // each launch a programmatic dependent of the one before it
+  cudaError_t e = launch_dependent(k_prefill_scan_bits, grid, dim3(kScanThreads), 0, s, c, layer, T0, T, alpha);
   if (e != cudaSuccess) return e;
   const size_t smem = prefill_scan_smem(c, T0, T);
   e = cudaFuncSetAttribute(k_prefill_scan_assign, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  k_prefill_scan_assign<<<grid, kScanThreads, smem, s>>>(c, layer, T0, T, alpha);
-  return cudaGetLastError();
+  return launch_dependent(k_prefill_scan_assign, grid, dim3(kScanThreads), smem, s, c, layer, T0, T, alpha);
 }
 
 // ---------------------------------------------------------------------------
@@ -435,6 +438,8 @@ cudaError_t launch_prefill_context(const CacheView& c, int layer, int T0, int T,
 template <typename TA>
 __global__ void __launch_bounds__(256) k_prefill_scatter(CacheView c, int layer, int T0, int T, int rg, const TA* k,
                                                          const TA* v) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int gpp = (c.P + rg - 1) / rg;
   const int p = blockIdx.x / gpp, r0 = (blockIdx.x % gpp) * rg, bh = blockIdx.y;
   const int b = bh / c.Hkv, h = bh % c.Hkv;
@@ -534,6 +539,8 @@ __device__ __forceinline__ float amax8(const uint4 x, float m) {
 __global__ void __launch_bounds__(256) k_prefill_scatter_fp8(CacheView c, int layer, int T0, int T,
                                                             const __nv_bfloat16* k, const __nv_bfloat16* v) {
   __shared__ float red[32];
+  griddep_wait();
+  griddep_launch_dependents();
   const int p = blockIdx.x, bh = blockIdx.y;
   const int b = bh / c.Hkv, h = bh % c.Hkv;
   const long lbh = static_cast<long>(layer) * c.B * c.Hkv + bh;
@@ -636,22 +643,18 @@ cudaError_t launch_prefill_scatter(const CacheView& c, int layer, int T0, int T,
   // count (slots reused in place may sit in any earlier page)
   const int pages = min(c.maxp, (T0 + T + c.P - 1) / c.P);
   if (c.kv_dtype == DMS_FP8_E4M3) {
-    k_prefill_scatter_fp8<<<dim3(pages, c.B * c.Hkv), 256, 0, s>>>(c, layer, T0, T,
-                                                                   static_cast<const __nv_bfloat16*>(k),
-                                                                   static_cast<const __nv_bfloat16*>(v));
-    return cudaGetLastError();
+    return launch_dependent(k_prefill_scatter_fp8, dim3(pages, c.B * c.Hkv), dim3(256), 0, s, c, layer, T0, T,
+                            static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v));
   }
   // rows per CTA: one batch of kScatterU chunks per thread
   const int cpr = c.D * (c.kv_dtype == DMS_BF16 ? 2 : 4) / 16;
   const int rg = max(1, min(c.P, kScatterU * 256 / cpr));
   dim3 grid(pages * ((c.P + rg - 1) / rg), c.B * c.Hkv);
   if (c.kv_dtype == DMS_BF16)
-    k_prefill_scatter<__nv_bfloat16><<<grid, 256, 0, s>>>(c, layer, T0, T, rg, static_cast<const __nv_bfloat16*>(k),
-                                                          static_cast<const __nv_bfloat16*>(v));
-  else
-    k_prefill_scatter<float><<<grid, 256, 0, s>>>(c, layer, T0, T, rg, static_cast<const float*>(k),
-                                                  static_cast<const float*>(v));
-  return cudaGetLastError();
+    return launch_dependent(k_prefill_scatter<__nv_bfloat16>, grid, dim3(256), 0, s, c, layer, T0, T, rg,
+                            static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v));
+  return launch_dependent(k_prefill_scatter<float>, grid, dim3(256), 0, s, c, layer, T0, T, rg,
+                          static_cast<const float*>(k), static_cast<const float*>(v));
 }
 
 }  // namespace dms

@@ -63,6 +63,10 @@ CASES = {
     # fused decode over many heads (batch 8: decision logits inside the kernel)
     "bf16_b8_proj": Case(B=8, T=300, steps=40, Hq=16, Hkv=8, D=128, hidden=256, w=64, P=32, act="bf16", kv="bf16",
                          source="proj", keep=(1 / 16, 1 / 4), prealloc=96, seed=17),
+    # 32 heads of D = 64 with 8 query heads each: the decode kernel's 16-row
+    # sub-tiles (pages of 48 slots, three sub-tiles each), key-major tiles
+    "bf16_d64_b8_g8_p48": Case(B=8, T=280, steps=24, Hq=32, Hkv=4, D=64, w=64, P=48, act="bf16", kv="bf16",
+                               source="input", keep=(1 / 16, 1 / 4), prealloc=96, seed=18),
     # a prompt large enough for the row-walking rotary kernel (batch x tokens x
     # 8-pair chunks above 148 x 256), 256-slot pages scattered by several CTAs
     # each, the last page ragged
