@@ -159,20 +159,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_cluster(CacheView c, int
   const int pa = (kAppendFirst && !(pl.y & 4)) ? pl.x / c.P : -1;
   const int masked_slot = (FUSED && !kAppendFirst && (pl.y & 1)) ? pl.x : -1;
   // The decision logit of the new token: with cs >= 4, rank 0 computes it
-  // instead of attending (it sends the logit with an empty partial), so it
-  // is off the path of the streaming ranks; with a smaller cluster the owner
-  // computes it before streaming.
+  // before attending a reduced share (it sends the logit with its partial),
+  // so it is off the path of the other ranks; with a smaller cluster the
+  // owner computes it before streaming.
   const bool rank0_decides = FUSED && fuse_decide && cs >= 4;
   const bool owner_decides = FUSED && fuse_decide && cs < 4;
   // the streaming ranks before the owner take `per` slots each, the owner
   // the rest: half a share (it merges the partials and appends), a quarter
-  // share when it also computes the decision logit
-  const int r0 = rank0_decides ? 1 : 0;  // first streaming rank
+  // share when it also computes the decision logit; rank 0 computing the
+  // logit takes no slots of a short head and half a share of a long one
+  // (at least 512 slots per rank), which outlasts the logit
+  const int r0 = rank0_decides ? 1 : 0;  // first rank with a full share
   const int oq = owner_decides ? 1 : 2;
+  const int q0 = rank0_decides && cnt_vis >= 512 * (cs - 1) ? 2 : 0;  // rank 0's share, in quarters
   const int nfull = cs - 1 - r0;
-  const int per = nfull == 0 ? 0 : ((4 * cnt_vis + 4 * nfull + oq - 1) / (4 * nfull + oq) + 15) / 16 * 16;
-  const int s_begin = rank < r0 ? 0 : min(cnt_vis, (rank - r0) * per);
-  int s_end = rank < r0 ? 0 : rank == owner ? cnt_vis : min(cnt_vis, s_begin + per);
+  const int per_q = 4 * nfull + q0 + oq;
+  const int per = nfull == 0 ? 0 : ((4 * cnt_vis + per_q - 1) / per_q + (q0 ? 31 : 15)) / (q0 ? 32 : 16) * (q0 ? 32 : 16);
+  const int r0end = q0 ? min(cnt_vis, per / 2) : 0;  // rank 0's slots [0, r0end)
+  const int s_begin = rank < r0 ? 0 : min(cnt_vis, r0end + (rank - r0) * per);
+  int s_end = rank < r0 ? r0end : rank == owner ? cnt_vis : min(cnt_vis, s_begin + per);
   __syncthreads();
   // this CTA's barriers are initialised (waited before the first remote
   // store); the owner of an append-first step arrives after its append

@@ -63,8 +63,12 @@ CASES = {
     # fused decode over many heads (batch 8: decision logits inside the kernel)
     "bf16_b8_proj": Case(B=8, T=300, steps=40, Hq=16, Hkv=8, D=128, hidden=256, w=64, P=32, act="bf16", kv="bf16",
                          source="proj", keep=(1 / 16, 1 / 4), prealloc=96, seed=17),
-    # 32 heads of D = 64 with 8 query heads each: the decode kernel's 16-row
-    # sub-tiles (pages of 48 slots, three sub-tiles each), key-major tiles
+    # heads long enough (>= 512 slots per rank of an 8-CTA cluster) that the
+    # rank computing the decision logit also attends half a share
+    "bf16_proj_long_heads": Case(B=1, T=4100, steps=12, Hq=8, Hkv=2, D=128, hidden=256, w=64, P=32, act="bf16",
+                                 kv="bf16", source="proj", keep=0.95, attn_rows=64, seed=19),
+    # 32 heads of D = 64 with 8 query heads each (two CTAs per SM), pages of 48
+    # slots cut into 16-slot sub-tiles, key-major tiles
     "bf16_d64_b8_g8_p48": Case(B=8, T=280, steps=24, Hq=32, Hkv=4, D=64, w=64, P=48, act="bf16", kv="bf16",
                                source="input", keep=(1 / 16, 1 / 4), prealloc=96, seed=18),
     # a prompt large enough for the row-walking rotary kernel (batch x tokens x
