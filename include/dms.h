@@ -33,6 +33,14 @@
  *    unspecified until dms_cache_reset.
  *  - All calls on one cache must be issued on one stream (or ordered by the
  *    caller); calls on different caches are independent.
+ *  - Launch overlap: the decode step kernels, the rotary / decision-neuron
+ *    pass and the compaction kernels are programmatic dependents of the
+ *    kernel before them on the stream: they may start while it runs and read
+ *    none of the caller's inputs before it has completed.  A decode step
+ *    kernel may read its cache's own state (counts, plans, page tables) and
+ *    request its first pages earlier, when the launch before it is this
+ *    library's for another cache or layer, or the same step's rotary pass;
+ *    so the cache's buffer must be written by nothing but this library.
  *  - q, k, v and o (prefill and decode) are read and written as 16-byte
  *    vectors: their base pointers must be 16-byte aligned (DMS_ERR_INVALID
  *    otherwise).
