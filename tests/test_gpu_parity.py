@@ -67,6 +67,8 @@ CASES = {
     # rank computing the decision logit also attends half a share
     "bf16_proj_long_heads": Case(B=1, T=4100, steps=12, Hq=8, Hkv=2, D=128, hidden=256, w=64, P=32, act="bf16",
                                  kv="bf16", source="proj", keep=0.95, attn_rows=64, seed=19),
+    "fp8_proj_long_heads": Case(B=1, T=4100, steps=12, Hq=8, Hkv=2, D=128, hidden=256, w=64, P=32, act="bf16",
+                                kv="fp8", source="proj", keep=0.95, attn_rows=64, seed=20),
     # 32 heads of D = 64 with 8 query heads each (two CTAs per SM), pages of 48
     # slots cut into 16-slot sub-tiles, key-major tiles
     "bf16_d64_b8_g8_p48": Case(B=8, T=280, steps=24, Hq=32, Hkv=4, D=64, w=64, P=48, act="bf16", kv="bf16",
