@@ -216,19 +216,29 @@ def make_desc(B_, wl, kernel="auto"):
 
 
 def decode_launches_per_step(wl):
-    """Kernels one dms_decode_step launches per layer."""
-    pre = 1 if (wl.alpha_source not in ("proj", "score") or wl.rope) else 0  # decision neuron / rotary pass
-    if wl.kv_dtype == "fp8":
-        return pre + 2  # append (re-encodes pages), then the cluster attention
-    return pre + 1      # one fused kernel: decision, attention, combine, append
+    """Kernels one dms_decode_step launches per layer: the decision neuron /
+    rotary pass where needed, then one fused kernel (decision logit,
+    attention, combine, append; FP8 pages appended first inside it)."""
+    pre = 1 if (wl.alpha_source not in ("proj", "score") or wl.rope) else 0
+    return pre + 1
+
+
+def prefill_launches_per_layer(wl):
+    """Kernels one dms_prefill launches: the adapter / score logits or the
+    decision neuron and rotary pass, the two scan kernels, the scatter and the
+    masked attention."""
+    decide = 1 if wl.alpha_source in ("proj", "score") else 0
+    rope = 1 if (wl.alpha_source not in ("proj", "score") or wl.rope) else 0
+    return decide + rope + 2 + 1 + 1
 
 
 def kernel_launches_per_step(wl, n_dec, stacked=False):
-    # reset (1) + per layer: compaction (decide or neuron/rotary pass, scan,
-    # scatter) + prefill attention (1) + the decode steps (one launch for the
-    # whole stack with dms_decode_step_layers)
-    per_step = 1 if stacked else wl.layers * decode_launches_per_step(wl)
-    return 1 + wl.layers * (3 + 1) + n_dec * per_step
+    # reset (1) + per layer the prefill + the decode steps (with
+    # dms_decode_step_layers: each layer's rotary pass where needed, then one
+    # launch for the whole stack)
+    pre = decode_launches_per_step(wl) - 1
+    per_step = wl.layers * pre + 1 if stacked else wl.layers * decode_launches_per_step(wl)
+    return 1 + wl.layers * prefill_launches_per_layer(wl) + n_dec * per_step
 
 
 def decode_kernel_name(wl, choice, num_sms):

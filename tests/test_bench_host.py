@@ -1,6 +1,7 @@
 """Host logic of bench.py (no GPU): which decode kernel a workload's line
-names, and the recorded DRAM traffic, which is reported only while the
-kernel's sources are the ones the capture was taken on."""
+names, the recorded DRAM traffic, which is reported only while the kernel's
+sources are the ones the capture was taken on, and the kernel launches the
+line claims."""
 import os
 import sys
 
@@ -57,3 +58,18 @@ def test_executed_tiles_cover_the_visible_pairs():
         i1 = min(wl.prompt, i0 + span)
         tiles += (i1 - 1 - max(0, i0 - wl.window + 1) + 64) // 64
     assert bench.executed_tile_flops(allev, wl) == 8 * tiles * 2 * 4 * 128 * 64 * wl.head_dim
+
+
+def test_kernel_launch_counts():
+    """The launches the bench claims per bench step and replica follow the
+    library's launch structure: reset; per layer the logits (adapter / score)
+    or the decision neuron and rotary pass, two scan kernels, the scatter and
+    the attention; per decode step the rotary pass where needed and one fused
+    kernel (one for the whole stack with the layer-range call)."""
+    wl = bench.I.WORKLOADS
+    assert bench.kernel_launches_per_step(wl["qwen8b"], 128) == 1 + 5 + 128
+    assert bench.kernel_launches_per_step(wl["qwen8b_c8"], 128) == 1 + 5 + 128
+    assert bench.kernel_launches_per_step(wl["kvzap8b"], 128) == 1 + 5 + 128
+    assert bench.kernel_launches_per_step(wl["llama1b"], 256) == 1 + 5 + 256 * 2
+    assert bench.kernel_launches_per_step(wl["llama1b_layer"], 256) == 1 + 5 + 256 * 2
+    assert bench.kernel_launches_per_step(wl["reason36"], 512, stacked=True) == 1 + 36 * 5 + 512
