@@ -241,6 +241,25 @@ def kernel_launches_per_step(wl, n_dec, stacked=False):
     return 1 + wl.layers * prefill_launches_per_layer(wl) + n_dec * per_step
 
 
+def decode_label(wl, kern, stacked, layers):
+    """What the decode roofline's time covers, for the JSON line."""
+    parts = ["split-K attention",
+             "on-chip combine" if kern == "k_decode_cluster" else "partials merged by the last CTA of a head"]
+    fp8_inside = wl.kv_dtype == "fp8" and kern == "k_decode_cluster"
+    if wl.kv_dtype == "bf16" or fp8_inside:
+        parts.append("append" + (" first (page re-encode), then the attention" if fp8_inside else ""))
+    if wl.alpha_source in ("proj", "score"):
+        parts.append("decision logit")
+    label = "decode step: %s<%d,%s> (%s)%s%s" % (
+        kern, wl.head_dim, wl.kv_dtype, ", ".join(parts),
+        " after k_decode_append" if wl.kv_dtype == "fp8" and not fp8_inside else "",
+        "; the step's time includes the decision-neuron / rotary pass before it"
+        if decode_launches_per_step(wl) > 1 else "")
+    if stacked:
+        label += ", all %d layers in one launch (dms_decode_step_layers)" % layers
+    return label
+
+
 def decode_kernel_name(wl, choice, num_sms):
     """The decode kernel the library runs for this workload (its AUTO rule:
     the cluster kernel)."""
@@ -757,13 +776,7 @@ def run_ours(args, world, rank, local, primary=True):
         cpu = cpu_baseline(wl, args.cpu_seconds)
     kern = ("k_decode_cluster" if r.stacked else
             decode_kernel_name(wl, args.decode_kernel, torch.cuda.get_device_properties(0).multi_processor_count))
-    kname = ("decode step: %s<%d,%s> (split-K attention, %s%s)%s"
-             % (kern, wl.head_dim, wl.kv_dtype,
-                "on-chip combine" if kern == "k_decode_cluster" else "partials merged by the last CTA of a head",
-                ", append, decision logit" if wl.kv_dtype == "bf16" else "",
-                " after k_decode_append" if wl.kv_dtype == "fp8" else ""))
-    if r.stacked:
-        kname += ", all %d layers in one launch (dms_decode_step_layers)" % L
+    kname = decode_label(wl, kern, r.stacked, L)
     traffic = recorded_traffic(kern, workload_label(wl, S)) if args.replicas is None else None
     roof = {"bound": "hbm", "achieved": round(decode_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(decode_gbs / pk["hbm_gbs"], 4), "traffic": traffic, "kernel": kname,

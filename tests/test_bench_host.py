@@ -73,3 +73,14 @@ def test_kernel_launch_counts():
     assert bench.kernel_launches_per_step(wl["llama1b"], 256) == 1 + 5 + 256 * 2
     assert bench.kernel_launches_per_step(wl["llama1b_layer"], 256) == 1 + 5 + 256 * 2
     assert bench.kernel_launches_per_step(wl["reason36"], 512, stacked=True) == 1 + 36 * 5 + 512
+
+
+def test_decode_label_says_what_the_time_covers():
+    wl = bench.I.WORKLOADS
+    b1 = bench.decode_label(wl["qwen8b"], "k_decode_cluster", False, 1)
+    assert "append" in b1 and "decision logit" in b1 and "rotary" not in b1
+    fp8 = bench.decode_label(wl["llama1b"], "k_decode_cluster", False, 1)
+    assert "append first" in fp8 and "k_decode_append" not in fp8 and "decision logit" not in fp8
+    assert "rotary pass" in fp8
+    assert "after k_decode_append" in bench.decode_label(wl["llama1b"], "k_decode_flat", False, 1)
+    assert "all 36 layers in one launch" in bench.decode_label(wl["reason36"], "k_decode_cluster", True, 36)
