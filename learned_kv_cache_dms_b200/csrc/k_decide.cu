@@ -732,16 +732,9 @@ __global__ void __launch_bounds__(256, 3) k_neuron_rope8(CacheView c, int T, con
 // previous kernel on the stream when pdl is set.
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_rope_kernel(void (*kern)(KArgs...), int grid, cudaStream_t s, bool pdl, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(256, 1, 1);
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (pdl) return launch_dependent(kern, dim3(grid), dim3(256), 0, s, args...);
+  kern<<<grid, 256, 0, s>>>(static_cast<KArgs>(args)...);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_neuron_rope(const CacheView& c, int T, const int* pos_dev, void* q, void* k, const float* offset,
