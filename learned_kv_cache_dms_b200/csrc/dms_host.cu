@@ -819,11 +819,10 @@ int dms_decode_step_layers(dms_cache* c, int layer0, int num_layers, const dms_d
     da.bias_lstride = Hkv;
     da.offset_lstride = ostride_layer;
   }
-  // every layer of the range in one launch (the layers' state read before the
-  // wait only after the rotary passes, which waited for everything before)
+  // every layer of the range in one launch (early reads only after the wait)
   track_launch(c, -1, s);
   if (launch_decode_cluster(v, layer0, a->q, a->o, true, a->k, a->v, a->alpha, proj ? &da : nullptr, &c->kmapc,
-                            &c->vmapc, c->num_sms, s, rope, num_layers) != cudaSuccess)
+                            &c->vmapc, c->num_sms, s, false, num_layers) != cudaSuccess)
     return DMS_ERR_CUDA;
   for (int l = layer0; l < layer0 + num_layers; ++l) {
     c->decoded[l] = 1;
